@@ -1,0 +1,347 @@
+"""Benchmark of the edge message-passing step (energy + forces) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: the seeded N=4096 diamond (8x8x8 conventional cells, sigma 0.02 A,
+seed 2), cutoff 6 A (E = 647168 directed edges), C = 128, lmax = 3, three gated
+residual layers, 8192-edge receiver-sorted cohorts.  One step = the whole hot
+path on one frame: neighbour list build + forward (radial, rotate, SO(2)
+mixing, rotate back, receiver sums, gates, readout) + recomputing backward +
+forces.  Metric: edges/s = E / step time (whole job: summed over replicas).
+
+N > 1 (launched with torch.distributed.run, one rank per GPU): every rank runs
+its own replica of the frame (replicas only: weak scaling), timed between
+barriers, max over ranks.
+
+--impl reference times the float64 oracle (test infrastructure, CPU) on a
+bounded sample of the same workload: the edges of the first receivers.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+WORKLOAD = "n4096_diamond"
+METRIC = "edges/s fwd+force at N=4096 diamond (E~647k)"
+L2_BYTES = 126 * 2 ** 20
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TF32_OVER_BF16 = 1.1 / 2.25     # nominal dense TF32 / BF16 tensor throughput on B200
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+# ------------------------------------------------------------------ distributed helpers
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def reduce_max(value: float, backend_device=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=backend_device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None:
+            dist.barrier(device_ids=[device])
+        else:
+            dist.barrier()
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples (200 ms) during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ the oracle arm
+def oracle_sample(n_recv: int):
+    """The oracle's energy + forces on the edges of the first n_recv receivers."""
+    from oracle import model as omodel
+    from oracle import nl as onl
+    w = synth.workload(WORKLOAD)
+    st = w.structure
+    g = onl.brute_force(st.pos, st.box, w.spec.cutoff)
+    e1 = int(g.recv_off[n_recv])
+    sel = slice(0, e1)
+
+    def run():
+        return omodel.energy_forces(w.spec, w.weights, st.species, g.recv[sel], g.send[sel], g.r[sel],
+                                    st.pos.shape[0])
+    return run, e1, g.n_edges
+
+
+def threads_used() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(n_recv: int = 48):
+    run, e, _ = oracle_sample(n_recv)
+    run()                       # warm caches / thread pools
+    t0 = time.perf_counter()
+    run()
+    dt = time.perf_counter() - t0
+    return {"value": e / dt, "unit": "edges/s", "cores": threads_used(), "kind": "oracle",
+            "sample": f"float64 oracle energy+forces over the {e} edges of the first {n_recv} receivers "
+                      f"of the {WORKLOAD} frame (3 layers fwd + reverse mode), one run after one warm-up, "
+                      f"{dt:.1f} s"}
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    n_recv = 32
+    run, e, E = oracle_sample(n_recv)
+    for _ in range(args.warmup):
+        run()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        run()
+        times.append(time.perf_counter() - t0)
+    dt = sum(times) / len(times)
+    v = e / dt
+    cores = threads_used()
+    sample = (f"float64 oracle energy+forces over the {e} edges of the first {n_recv} receivers of the "
+              f"{WORKLOAD} frame per step")
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "edges/s", "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "n_atoms": 4096, "n_edges": E, "sample_edges": e, "C": 128,
+                       "lmax": 3, "layers": 3, "cohort_edges": 8192},
+            "cpu_baseline": {"value": v, "unit": "edges/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "edges/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import edge_message_passing_b200 as emp
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.cuda.current_device()
+    w = synth.workload(WORKLOAD)
+    st, spec = w.structure, w.spec
+    N = st.pos.shape[0]
+    model = emp.Model(spec, w.weights)
+    pos_h = torch.from_numpy(st.pos).pin_memory()
+    sp_h = torch.from_numpy(st.species).pin_memory()
+    pos = pos_h.cuda()
+    sp = sp_h.cuda()
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(p):
+        g = emp.nl_build(p, st.box, spec.cutoff, capacity=cap)
+        e, f, _, _ = emp.mp_energy_forces(model, g, sp)
+        return g, e, f
+
+    g0 = emp.nl_build(pos, st.box, spec.cutoff)
+    cap = g0.n_edges
+    E = g0.n_edges
+    for _ in range(max(args.warmup, 3)):
+        step(pos)
+    torch.cuda.synchronize()
+
+    # ---- device-resident timing: K steps, L2 flushed between steps (outside the events)
+    barrier(dev if ws > 1 else None)
+    torch.cuda.synchronize()
+    launches0 = emp.launch_count()
+    emp.profile_enable(True)
+    times = []
+    with ClockSampler(dev) as clk:
+        for _ in range(args.steps):
+            flush.fill_(1.0)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            step(pos)
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+    torch.cuda.synchronize()
+    barrier(dev if ws > 1 else None)
+    launches = emp.launch_count() - launches0
+    fam = {n: emp.profile_read(n) for n in emp.profile_names()}
+    emp.profile_enable(False)
+    ms_local = sum(times) / len(times)
+    ms = reduce_max(ms_local, torch.device("cuda", dev))
+    value = E * ws / (ms * 1e-3)
+
+    # ---- end to end through the public API with host buffers (H2D positions + species, D2H energy + forces)
+    e_h = torch.empty(1, dtype=torch.float64).pin_memory()
+    f_h = torch.empty((N, 3), dtype=torch.float32).pin_memory()
+    e2e_times = []
+    for k in range(args.steps + 1):
+        flush.fill_(1.0)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        pd = pos_h.to("cuda", non_blocking=True)
+        sp.copy_(sp_h, non_blocking=True)
+        g, e, f = step(pd)
+        e_h.copy_(e, non_blocking=True)
+        f_h.copy_(f, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        if k:
+            e2e_times.append(a.elapsed_time(b))
+    e2e_ms = reduce_max(sum(e2e_times) / len(e2e_times), torch.device("cuda", dev))
+
+    # ---- roofline of the dominant kernel family
+    pk, pk_kind = peaks()
+    dom = max(fam.items(), key=lambda kv: kv[1][0])[0] if fam else None
+    C = spec.C
+    fl_per_edge = 2 * 72 * C * C                      # useful flops of one SO(2) mixing of one edge
+    so2_launches = fam.get("so2_tc", (0, 0))[1]
+    roof = None
+    if dom == "so2_tc" and so2_launches:
+        so2_ms = fam["so2_tc"][0] / so2_launches
+        # launches per step: 3 per layer per cohort (forward, backward recompute, transpose)
+        ncoh = -(-E // spec.cohort_edges)
+        rows = E * 3 * spec.n_layers / (ncoh * 3 * spec.n_layers)   # mean rows per launch
+        achieved = rows * fl_per_edge / (so2_ms * 1e-3) / 1e12
+        peak_tf32 = pk["bf16_tflops_sustained"] * TF32_OVER_BF16
+        peak = peak_tf32 / 3.0
+        roof = {"bound": "tensor", "kernel": "so2_tc (3xTF32 tcgen05 SO(2) mixing)", "achieved": achieved,
+                "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                "peak_note": f"useful FP32-equivalent flops vs (sustained bf16 {pk_kind} x {TF32_OVER_BF16:.3f}) / 3 "
+                             f"for 3xTF32"}
+    elif dom is not None:
+        roof = {"bound": "hbm", "kernel": dom, "achieved": None, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": None, "traffic": None}
+    kernel_ms = {k: round(v[0] / len(times), 3) for k, v in sorted(fam.items(), key=lambda kv: -kv[1][0])}
+
+    result = None
+    if rank == 0:
+        cpu = cpu_baseline() if (ws == 1 and not args.no_cpu_baseline) else None
+        result = {"metric": METRIC, "value": value, "unit": "edges/s", "n_gpus": ws, "steps": args.steps,
+                  "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                  "vs_baseline": None, "dtype": "f32 (3xTF32 tensor-core mixing)", "data": "synthetic",
+                  "config": {"workload": WORKLOAD, "n_atoms": N, "n_edges": E, "C": C, "lmax": 3,
+                             "layers": spec.n_layers, "cohort_edges": spec.cohort_edges,
+                             "parallelism": "replicas" if ws > 1 else "single",
+                             "l2": "flushed between timed steps (256 MB write outside the timed events)"},
+                  "clocks": clk.summary(), "gpu_launches": launches,
+                  "e2e": {"value": E * ws / (e2e_ms * 1e-3), "unit": "edges/s",
+                          "h2d_bytes_per_step": int(pos_h.numel() * 8 + sp_h.numel() * 4),
+                          "d2h_bytes_per_step": int(8 + N * 3 * 4)},
+                  "roofline": roof, "cpu_baseline": cpu, "kernel_ms_per_step": kernel_ms,
+                  "ns_per_atom": ms * 1e6 / N}
+        print(json.dumps(result))
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

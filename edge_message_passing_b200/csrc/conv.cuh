@@ -1,0 +1,774 @@
+// Per-edge kernels of the SO(2) message-passing layer and its recomputing
+// backward (page "first-order SO(2) input-gradient path": the reverse mixing
+// chain is finished one receiver-sorted 8192-edge cohort at a time; page
+// "deepmd-kit PR #6108": radial basis -> radial network; the model's steps are
+// the convolution of the spec workloads: Bessel basis with polynomial
+// envelope, radial MLP giving per-(l, channel) scales, Wigner-D rotation of the
+// sender's irreps into the edge frame, per-m SO(2) mixing, rotation back and a
+// normalised sum onto the receiver).
+//
+// Thread mapping of the edge kernels: blockDim = (C, EPB); thread x owns channel
+// c = x and its 16 components; row y owns one edge at a time.  Every edge's 84
+// Wigner-D values are staged in shared memory.  All sums over edges have a fixed
+// order (edges ascending within a receiver or sender segment, cohorts in order),
+// so results are bitwise reproducible.
+#pragma once
+#include "emp_common.cuh"
+#include "model.cuh"
+
+namespace emp {
+
+constexpr float PI_F = 3.14159265358979323846f;
+
+// ------------------------------------------------------------------ rotations
+// u = D x (transpose = false) or u = D^T x, per degree block; D in shared memory
+template <bool TRANSPOSE>
+__device__ __forceinline__ void rotate16(const float* __restrict__ D, const float (&x)[16], float (&u)[16]) {
+  u[0] = x[0];
+#pragma unroll
+  for (int l = 1; l <= 3; ++l) {
+    const int w = 2 * l + 1, o = l * l;
+    const float* B = D + dblk_off(l);
+#pragma unroll
+    for (int m = 0; m < w; ++m) {
+      float acc = 0.f;
+#pragma unroll
+      for (int n = 0; n < w; ++n) acc = fmaf(TRANSPOSE ? B[n * w + m] : B[m * w + n], x[o + n], acc);
+      u[o + m] = acc;
+    }
+  }
+}
+
+__device__ __forceinline__ int deg_of(int k) { return k == 0 ? 0 : k < 4 ? 1 : k < 9 ? 2 : 3; }
+
+// ------------------------------------------------------------------ geometry
+// D(R_e) (84 floats) and d = |r_e| from the float32 edge vector.
+__global__ void k_geometry(long long E, const float* __restrict__ vec, float* __restrict__ D, float* __restrict__ dist) {
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= E) return;
+  const float vx = vec[3 * e], vy = vec[3 * e + 1], vz = vec[3 * e + 2];
+  const float d = sqrtf(vx * vx + vy * vy + vz * vz);
+  const float inv = 1.0f / d;
+  float R[3][3];
+  edge_frame<float>(vx * inv, vy * inv, vz * inv, R);
+  float Dl[NDBLK];
+  wigner_blocks<float>(R, Dl);
+  float* out = D + (size_t)e * NDBLK;
+#pragma unroll
+  for (int k = 0; k < NDBLK; ++k) out[k] = Dl[k];
+  dist[e] = d;
+}
+
+// ------------------------------------------------------------------ radial part
+// e_n(d) = u(d/rc) sin(n pi d / rc) / d, u(x) = 1 - 28 x^6 + 48 x^7 - 21 x^8 for x < 1.
+__device__ __forceinline__ void bessel8(float d, float rc, float (&e)[8], float (&de)[8]) {
+  const float x = d / rc;
+  const float x2 = x * x, x5 = x2 * x2 * x, x6 = x5 * x;
+  float u = 1.f + x6 * (-28.f + x * (48.f - 21.f * x));
+  float du = x5 * (-168.f + x * (336.f - 168.f * x)) / rc;
+  if (x >= 1.f) { u = 0.f; du = 0.f; }
+  const float inv = 1.f / d;
+#pragma unroll
+  for (int n = 0; n < 8; ++n) {
+    const float k = PI_F * (float)(n + 1) / rc;
+    float s, c;
+    sincosf(k * d, &s, &c);
+    e[n] = u * s * inv;
+    de[n] = du * s * inv + u * (k * c * inv - s * inv * inv);
+  }
+}
+
+__device__ __forceinline__ int pair_of(int a, int b, int S) {
+  const int lo = a < b ? a : b, hi = a < b ? b : a;
+  return lo * S - lo * (lo - 1) / 2 + (hi - lo);
+}
+
+struct RadialArgs {
+  const float* rad;        // model radial weights (per layer, per pair)
+  size_t layer_off;        // float offset of layer t's first pair
+  size_t pair_stride;      // floats per pair
+  int C, n_species, pair_radial;
+  float rc;
+};
+
+constexpr int RT = 64;      // edges per radial tile
+constexpr int RAD_THREADS = 256;
+
+// shared-memory tile of the radial network
+struct RadialSmem {
+  float e[RT][8];
+  float de[RT][8];
+  float z1[RT][64];
+  float h1[RT][65];
+  float z2[RT][64];
+  float h2[RT][65];
+  float w[64][132];     // a 64 x 128 chunk of W3^T (forward) or W3 (backward, [o][k] read)
+  float g[RT][132];     // backward: a 64 x 128 chunk of dE/dR
+  int pair[RT];
+  unsigned mask;
+};
+
+// basis, hidden layers (for edges of pair p) -- all 256 threads participate
+__device__ void radial_hidden(RadialSmem& s, const float* __restrict__ W1, const float* __restrict__ W2) {
+  const int t = threadIdx.x;
+  // layer 1: z1[e][j] = sum_n W1[j][n] e[n]
+  for (int idx = t; idx < RT * 64; idx += RAD_THREADS) {
+    const int e = idx >> 6, j = idx & 63;
+    float acc = 0.f;
+#pragma unroll
+    for (int n = 0; n < 8; ++n) acc = fmaf(__ldg(&W1[j * 8 + n]), s.e[e][n], acc);
+    s.z1[e][j] = acc;
+    s.h1[e][j] = silu_f(acc);
+  }
+  __syncthreads();
+  // layer 2: thread owns output j and 16 edges
+  {
+    const int j = t & 63, eg = (t >> 6) * 16;
+    float acc[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) acc[q] = 0.f;
+    for (int k = 0; k < 64; ++k) {
+      const float w = __ldg(&W2[j * 64 + k]);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) acc[q] = fmaf(w, s.h1[eg + q][k], acc[q]);
+    }
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      s.z2[eg + q][j] = acc[q];
+      s.h2[eg + q][j] = silu_f(acc[q]);
+    }
+  }
+  __syncthreads();
+}
+
+__device__ void radial_tile_setup(RadialSmem& s, long long e0, long long E, const float* __restrict__ dist,
+                                  const int* __restrict__ recv, const int* __restrict__ send,
+                                  const int* __restrict__ species, const RadialArgs& a) {
+  const int t = threadIdx.x;
+  if (t == 0) s.mask = 0u;
+  __syncthreads();
+  if (t < RT) {
+    const long long e = e0 + t;
+    int p = 0;
+    float d = 1.f;
+    if (e < E) {
+      d = dist[e];
+      if (a.pair_radial) p = pair_of(species[recv[e]], species[send[e]], a.n_species);
+      atomicOr(&s.mask, 1u << p);
+    }
+    s.pair[t] = e < E ? p : -1;
+    float ev[8], dv[8];
+    bessel8(d, a.rc, ev, dv);
+#pragma unroll
+    for (int n = 0; n < 8; ++n) { s.e[t][n] = ev[n]; s.de[t][n] = dv[n]; }
+  }
+  __syncthreads();
+}
+
+// R [E][4C] for layer t
+__global__ void __launch_bounds__(RAD_THREADS) k_radial_fwd(long long E, const float* __restrict__ dist,
+                                                           const int* __restrict__ recv, const int* __restrict__ send,
+                                                           const int* __restrict__ species, RadialArgs a,
+                                                           float* __restrict__ R) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  RadialSmem& s = *reinterpret_cast<RadialSmem*>(smem_raw);
+  const long long e0 = (long long)blockIdx.x * RT;
+  radial_tile_setup(s, e0, E, dist, recv, send, species, a);
+  const int t = threadIdx.x, ty = t >> 4, tx = t & 15;
+  const int CO = 4 * a.C;
+  unsigned mask = s.mask;
+  while (mask) {
+    const int p = __ffs(mask) - 1;
+    mask &= mask - 1;
+    const float* W1 = a.rad + a.layer_off + (size_t)p * a.pair_stride;
+    const float* W2 = W1 + 64 * 8;
+    const float* W3 = W2 + 64 * 64;
+    radial_hidden(s, W1, W2);
+    for (int oc = 0; oc < CO; oc += 128) {
+      // W3 rows oc..oc+127 -> w[k][o]
+      for (int idx = t; idx < 128 * 64; idx += RAD_THREADS) {
+        const int o = idx >> 6, k = idx & 63;
+        s.w[k][o] = __ldg(&W3[(size_t)(oc + o) * 64 + k]);
+      }
+      __syncthreads();
+      float acc[4][8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+      for (int k = 0; k < 64; ++k) {
+        float av[4], bv[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) av[i] = s.h2[ty * 4 + i][k];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) bv[j] = s.w[k][tx + 16 * j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int el = ty * 4 + i;
+        if (s.pair[el] == p) {
+          float* out = R + (size_t)(e0 + el) * CO + oc;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) out[tx + 16 * j] = acc[i][j];
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// dE/dd from dE/dR (gR [E][4C]); adds (dE/dd) rhat to g_r
+__global__ void __launch_bounds__(RAD_THREADS) k_radial_bwd(long long E, const float* __restrict__ dist,
+                                                           const float* __restrict__ vec,
+                                                           const int* __restrict__ recv, const int* __restrict__ send,
+                                                           const int* __restrict__ species, RadialArgs a,
+                                                           const float* __restrict__ gR, float* __restrict__ g_r) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  RadialSmem& s = *reinterpret_cast<RadialSmem*>(smem_raw);
+  const long long e0 = (long long)blockIdx.x * RT;
+  radial_tile_setup(s, e0, E, dist, recv, send, species, a);
+  const int t = threadIdx.x;
+  const int CO = 4 * a.C;
+  unsigned mask = s.mask;
+  while (mask) {
+    const int p = __ffs(mask) - 1;
+    mask &= mask - 1;
+    const float* W1 = a.rad + a.layer_off + (size_t)p * a.pair_stride;
+    const float* W2 = W1 + 64 * 8;
+    const float* W3 = W2 + 64 * 64;
+    radial_hidden(s, W1, W2);
+    // g_h2[e][k] = sum_o gR[e][o] W3[o][k]; thread owns k = t & 63 and 16 edges
+    const int k = t & 63, eg = (t >> 6) * 16;
+    float acc[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) acc[q] = 0.f;
+    for (int oc = 0; oc < CO; oc += 128) {
+      for (int idx = t; idx < 128 * 64; idx += RAD_THREADS) {
+        const int o = idx >> 6, kk = idx & 63;
+        s.w[kk][o] = __ldg(&W3[(size_t)(oc + o) * 64 + kk]);
+      }
+      for (int idx = t; idx < RT * 128; idx += RAD_THREADS) {
+        const int el = idx >> 7, o = idx & 127;
+        const long long e = e0 + el;
+        s.g[el][o] = (e < E) ? gR[(size_t)e * CO + oc + o] : 0.f;
+      }
+      __syncthreads();
+      for (int o = 0; o < 128; ++o) {
+        const float w = s.w[k][o];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) acc[q] = fmaf(s.g[eg + q][o], w, acc[q]);
+      }
+      __syncthreads();
+    }
+    // g_z2 -> reuse h2 as storage
+#pragma unroll
+    for (int q = 0; q < 16; ++q) s.h2[eg + q][k] = acc[q] * dsilu_f(s.z2[eg + q][k]);
+    __syncthreads();
+    // g_h1[e][j] = sum_k g_z2[e][k] W2[k][j]; g_z1 = g_h1 dsilu(z1) -> reuse h1
+    {
+      const int j = t & 63;
+      float a2[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) a2[q] = 0.f;
+      for (int kk = 0; kk < 64; ++kk) {
+        const float w = __ldg(&W2[kk * 64 + j]);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) a2[q] = fmaf(s.h2[eg + q][kk], w, a2[q]);
+      }
+      __syncthreads();
+#pragma unroll
+      for (int q = 0; q < 16; ++q) s.h1[eg + q][j] = a2[q] * dsilu_f(s.z1[eg + q][j]);
+    }
+    __syncthreads();
+    // dE/dd = sum_n (sum_j g_z1[j] W1[j][n]) de_n/dd
+    if (t < RT) {
+      const int el = t;
+      const long long e = e0 + el;
+      if (e < E && s.pair[el] == p) {
+        float dEdd = 0.f;
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+          float ge = 0.f;
+          for (int j = 0; j < 64; ++j) ge = fmaf(s.h1[el][j], __ldg(&W1[j * 8 + n]), ge);
+          dEdd = fmaf(ge, s.de[el][n], dEdd);
+        }
+        const float d = dist[e];
+        const float inv = 1.f / d;
+        g_r[3 * e + 0] += dEdd * vec[3 * e + 0] * inv;
+        g_r[3 * e + 1] += dEdd * vec[3 * e + 1] * inv;
+        g_r[3 * e + 2] += dEdd * vec[3 * e + 2] * inv;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------ rotate in
+// XT[e - e0][col(k) C + c] = R_e[l(k)][c] * (D_e x_send)[k][c]  (edge frame, m-major)
+__global__ void k_rotate_in(long long e0, long long e1, int C, const int* __restrict__ send,
+                            const float* __restrict__ D, const float* __restrict__ R,
+                            const float* __restrict__ x, float* __restrict__ XT, float* __restrict__ XTlo) {
+  extern __shared__ __align__(16) float sD[];           // [EPB][84]
+  const int c = threadIdx.x, row = threadIdx.y, EPB = blockDim.y;
+  const long long n = e1 - e0;
+  for (long long base = (long long)blockIdx.x * EPB; base < n; base += (long long)gridDim.x * EPB) {
+    const long long el = base + row;
+    const bool ok = el < n;
+    const long long e = e0 + el;
+    __syncthreads();
+    if (ok)
+      for (int k = c; k < NDBLK; k += C) sD[row * NDBLK + k] = D[(size_t)e * NDBLK + k];
+    __syncthreads();
+    if (!ok) continue;
+    const int j = send[e];
+    float xv[16], u[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) xv[k] = x[((size_t)j * 16 + k) * C + c];
+    rotate16<false>(sD + row * NDBLK, xv, u);
+    float Rv[4];
+#pragma unroll
+    for (int l = 0; l < 4; ++l) Rv[l] = R[(size_t)e * 4 * C + l * C + c];
+    float* out = XT + (size_t)el * 16 * C;
+    float* olo = XTlo + (size_t)el * 16 * C;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const float v = Rv[deg_of(k)] * u[k], h = tf32_rna(v);
+      out[col_of_k(k) * C + c] = h;
+      olo[col_of_k(k) * C + c] = tf32_rna(v - h);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ rotate back + receiver sums
+// S[i] (+)= sum over the cohort's edges of receiver i of D_e^T y_e, in edge order.
+// A receiver whose edges started in an earlier cohort continues its running sum.
+__global__ void k_rotate_back_scatter(long long e0, long long e1, int C, const int* __restrict__ recv,
+                                      const int* __restrict__ recv_off, const float* __restrict__ D,
+                                      const float* __restrict__ Y, float* __restrict__ S) {
+  __shared__ __align__(16) float sD[NDBLK];
+  const int lane = threadIdx.x;                           // 32 channels per block
+  const int c = blockIdx.y * 32 + lane;
+  const int first = recv[e0], last = recv[e1 - 1];
+  for (int i = first + blockIdx.x; i <= last; i += gridDim.x) {
+    const long long b = max((long long)recv_off[i], e0), e_end = min((long long)recv_off[i + 1], e1);
+    float acc[16];
+    const bool carry = recv_off[i] < e0;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) acc[k] = carry ? S[((size_t)i * 16 + k) * C + c] : 0.f;
+    for (long long e = b; e < e_end; ++e) {
+      __syncwarp();
+      for (int k = lane; k < NDBLK; k += 32) sD[k] = D[(size_t)e * NDBLK + k];
+      __syncwarp();
+      const float* y = Y + (size_t)(e - e0) * 16 * C;
+      float yv[16], m[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) yv[k] = y[col_of_k(k) * C + c];
+      rotate16<true>(sD, yv, m);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) acc[k] += m[k];
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) S[((size_t)i * 16 + k) * C + c] = acc[k];
+  }
+}
+
+// ------------------------------------------------------------------ node update, readout
+// a = S / avg; gated: x_next = x + G(a) with G(a)[0] = SiLU(a0), G(a)[l>0] = a SiLU(a0); else x_next = a
+__global__ void k_update(int N, int C, float inv_avg, int gated, float* __restrict__ S_to_a,
+                         const float* __restrict__ x, float* __restrict__ x_next) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= N * C) return;
+  const int i = idx / C, c = idx % C;
+  float a[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    a[k] = S_to_a[((size_t)i * 16 + k) * C + c] * inv_avg;
+    S_to_a[((size_t)i * 16 + k) * C + c] = a[k];
+  }
+  if (gated) {
+    const float s = silu_f(a[0]);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const float gk = k == 0 ? s : a[k] * s;
+      x_next[((size_t)i * 16 + k) * C + c] = x[((size_t)i * 16 + k) * C + c] + gk;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) x_next[((size_t)i * 16 + k) * C + c] = a[k];
+  }
+}
+
+// e_i = w_o . SiLU(W_ro h_i[0]); g_h = dE/dh (degree 0 only; other components zero)
+__global__ void k_readout(int N, int C, int Hro, const float* __restrict__ h, const float* __restrict__ ro_W,
+                          const float* __restrict__ ro_w, float* __restrict__ e_atom, float* __restrict__ g_h) {
+  __shared__ float sh[256];
+  __shared__ float gz[256];
+  __shared__ float part[256];
+  const int i = blockIdx.x, t = threadIdx.x;
+  if (t < C) sh[t] = h[(size_t)i * 16 * C + t];
+  __syncthreads();
+  float ep = 0.f;
+  if (t < Hro) {
+    float z = 0.f;
+    for (int c = 0; c < C; ++c) z = fmaf(ro_W[(size_t)t * C + c], sh[c], z);
+    ep = ro_w[t] * silu_f(z);
+    gz[t] = ro_w[t] * dsilu_f(z);
+  }
+  part[t] = ep;
+  __syncthreads();
+  for (int s = 128; s > 0; s >>= 1) {
+    if (t < s) part[t] += part[t + s];
+    __syncthreads();
+  }
+  if (t == 0) e_atom[i] = part[0];
+  if (g_h) {
+    for (int c = t; c < C; c += blockDim.x) {
+      float g = 0.f;
+      for (int k = 0; k < Hro; ++k) g = fmaf(ro_W[(size_t)k * C + c], gz[k], g);
+      g_h[(size_t)i * 16 * C + c] = g;
+      for (int k = 1; k < 16; ++k) g_h[((size_t)i * 16 + k) * C + c] = 0.f;
+    }
+  }
+}
+
+// energy = sum_i e_i in double, fixed order (one block)
+__global__ void k_energy_sum(int N, const float* __restrict__ e_atom, double* __restrict__ energy) {
+  __shared__ double part[1024];
+  const int t = threadIdx.x;
+  double s = 0.0;
+  for (int i = t; i < N; i += blockDim.x) s += (double)e_atom[i];
+  part[t] = s;
+  __syncthreads();
+  for (int w = blockDim.x >> 1; w > 0; w >>= 1) {
+    if (t < w) part[t] += part[t + w];
+    __syncthreads();
+  }
+  if (t == 0) energy[0] = part[0];
+}
+
+// ------------------------------------------------------------------ backward
+// gS = dE/dS (S = raw receiver sums) from g = dE/dx_next; gx = residual part of dE/dx
+__global__ void k_gate_bwd(int N, int C, float inv_avg, int gated, const float* __restrict__ a,
+                           const float* __restrict__ g, float* __restrict__ gS, float* __restrict__ gx) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= N * C) return;
+  const int i = idx / C, c = idx % C;
+  float gv[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) gv[k] = g[((size_t)i * 16 + k) * C + c];
+  if (gated) {
+    const float a0 = a[(size_t)i * 16 * C + c];
+    const float s = silu_f(a0), ds = dsilu_f(a0);
+    float acc = gv[0];
+#pragma unroll
+    for (int k = 1; k < 16; ++k) acc = fmaf(gv[k], a[((size_t)i * 16 + k) * C + c], acc);
+    gS[(size_t)i * 16 * C + c] = acc * ds * inv_avg;
+#pragma unroll
+    for (int k = 1; k < 16; ++k) gS[((size_t)i * 16 + k) * C + c] = gv[k] * s * inv_avg;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) gx[((size_t)i * 16 + k) * C + c] = gv[k];
+  } else {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      gS[((size_t)i * 16 + k) * C + c] = gv[k] * inv_avg;
+      gx[((size_t)i * 16 + k) * C + c] = 0.f;
+    }
+  }
+}
+
+// per edge: XT = R (.) D x_send (recomputed) and GY = D gS[recv] (edge-frame output gradient)
+__global__ void k_bwd_prep(long long e0, long long e1, int C, const int* __restrict__ recv,
+                           const int* __restrict__ send, const float* __restrict__ D, const float* __restrict__ R,
+                           const float* __restrict__ x, const float* __restrict__ gS, float* __restrict__ XT,
+                           float* __restrict__ XTlo, float* __restrict__ GY, float* __restrict__ GYhi,
+                           float* __restrict__ GYlo) {
+  extern __shared__ __align__(16) float sD[];
+  const int c = threadIdx.x, row = threadIdx.y, EPB = blockDim.y;
+  const long long n = e1 - e0;
+  for (long long base = (long long)blockIdx.x * EPB; base < n; base += (long long)gridDim.x * EPB) {
+    const long long el = base + row;
+    const bool ok = el < n;
+    const long long e = e0 + el;
+    __syncthreads();
+    if (ok)
+      for (int k = c; k < NDBLK; k += C) sD[row * NDBLK + k] = D[(size_t)e * NDBLK + k];
+    __syncthreads();
+    if (!ok) continue;
+    const float* Dr = sD + row * NDBLK;
+    const int j = send[e], i = recv[e];
+    float v[16], u[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[k] = x[((size_t)j * 16 + k) * C + c];
+    rotate16<false>(Dr, v, u);
+    float Rv[4];
+#pragma unroll
+    for (int l = 0; l < 4; ++l) Rv[l] = R[(size_t)e * 4 * C + l * C + c];
+    const size_t ro = (size_t)el * 16 * C;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const float t = Rv[deg_of(k)] * u[k], h = tf32_rna(t);
+      XT[ro + col_of_k(k) * C + c] = h;
+      XTlo[ro + col_of_k(k) * C + c] = tf32_rna(t - h);
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[k] = gS[((size_t)i * 16 + k) * C + c];
+    rotate16<false>(Dr, v, u);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const float h = tf32_rna(u[k]);
+      GY[ro + col_of_k(k) * C + c] = u[k];
+      GYhi[ro + col_of_k(k) * C + c] = h;
+      GYlo[ro + col_of_k(k) * C + c] = tf32_rna(u[k] - h);
+    }
+  }
+}
+
+// per edge, from y (recomputed), g_y and g_x~ = W^T g_y:
+//   gR[e][l][c] = sum_m g_x~ u;  g_u = R (.) g_x~;  g_xs = D^T g_u (-> GXS, [16][C] rows)
+//   b_j = sum_c (y^T J_j g_y + g_u^T J_j u), j = x, y (edge frame); a = -R_e^T (b_x, b_y, 0);
+//   g_r[e] += (a x r) / |r|^2  (direction part of dE/dr; the radial part is added by k_radial_bwd)
+__global__ void k_bwd_edge(long long e0, long long e1, int C, int need_gx, const int* __restrict__ send,
+                           const float* __restrict__ vec, const float* __restrict__ D, const float* __restrict__ R,
+                           const float* __restrict__ x, const float* __restrict__ Y, const float* __restrict__ GY,
+                           const float* __restrict__ GXT, float* __restrict__ GXS, float* __restrict__ gR,
+                           float* __restrict__ g_r) {
+  extern __shared__ __align__(16) float smem[];
+  const int c = threadIdx.x, row = threadIdx.y, EPB = blockDim.y;
+  float* sD = smem;                                 // [EPB][84]
+  float* red = smem + EPB * NDBLK;                  // [EPB][2][C/32]
+  const int nw = C / 32, warp = c >> 5, lane = c & 31;
+  const long long n = e1 - e0;
+  for (long long base = (long long)blockIdx.x * EPB; base < n; base += (long long)gridDim.x * EPB) {
+    const long long el = base + row;
+    const bool ok = el < n;
+    const long long e = e0 + el;
+    __syncthreads();
+    if (ok)
+      for (int k = c; k < NDBLK; k += C) sD[row * NDBLK + k] = D[(size_t)e * NDBLK + k];
+    __syncthreads();
+    float bx = 0.f, by = 0.f;
+    if (ok) {
+      const float* Dr = sD + row * NDBLK;
+      const int j = send[e];
+      float v[16], u[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) v[k] = x[((size_t)j * 16 + k) * C + c];
+      rotate16<false>(Dr, v, u);
+      float Rv[4];
+#pragma unroll
+      for (int l = 0; l < 4; ++l) Rv[l] = R[(size_t)e * 4 * C + l * C + c];
+      const size_t rowoff = (size_t)el * 16 * C;
+      float gxt[16], gu[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) gxt[k] = GXT[rowoff + col_of_k(k) * C + c];
+      float gr[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        gr[deg_of(k)] = fmaf(gxt[k], u[k], gr[deg_of(k)]);
+        gu[k] = Rv[deg_of(k)] * gxt[k];
+      }
+#pragma unroll
+      for (int l = 0; l < 4; ++l) gR[(size_t)e * 4 * C + l * C + c] = gr[l];
+      float yv[16], gy[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        yv[k] = Y[rowoff + col_of_k(k) * C + c];
+        gy[k] = GY[rowoff + col_of_k(k) * C + c];
+      }
+#pragma unroll
+      for (int p = 0; p < NJPAIR; ++p) {
+        const int A = jpair_a(p), B = jpair_b(p);
+        const float q = (yv[A] * gy[B] - yv[B] * gy[A]) + (gu[A] * u[B] - gu[B] * u[A]);
+        bx = fmaf(c_jx[p], q, bx);
+        by = fmaf(c_jy[p], q, by);
+      }
+      if (need_gx) {
+        float gxs[16];
+        rotate16<true>(Dr, gu, gxs);
+        float* out = GXS + rowoff;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) out[k * C + c] = gxs[k];
+      }
+    }
+    // deterministic reduction of (bx, by) over the row's channels
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      bx += __shfl_xor_sync(0xffffffffu, bx, o);
+      by += __shfl_xor_sync(0xffffffffu, by, o);
+    }
+    if (lane == 0) {
+      red[(row * 2 + 0) * nw + warp] = bx;
+      red[(row * 2 + 1) * nw + warp] = by;
+    }
+    __syncthreads();
+    if (ok && c == 0) {
+      float sx = 0.f, sy = 0.f;
+      for (int w = 0; w < nw; ++w) {
+        sx += red[(row * 2 + 0) * nw + w];
+        sy += red[(row * 2 + 1) * nw + w];
+      }
+      const float vx = vec[3 * e], vy = vec[3 * e + 1], vz = vec[3 * e + 2];
+      const float d2 = vx * vx + vy * vy + vz * vz;
+      const float inv = rsqrtf(d2);
+      float Rf[3][3];
+      edge_frame<float>(vx * inv, vy * inv, vz * inv, Rf);
+      const float ax = -(Rf[0][0] * sx + Rf[1][0] * sy);
+      const float ay = -(Rf[0][1] * sx + Rf[1][1] * sy);
+      const float az = -(Rf[0][2] * sx + Rf[1][2] * sy);
+      const float id2 = 1.f / d2;
+      g_r[3 * e + 0] += (ay * vz - az * vy) * id2;
+      g_r[3 * e + 1] += (az * vx - ax * vz) * id2;
+      g_r[3 * e + 2] += (ax * vy - ay * vx) * id2;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ cohort sender order
+// For each cohort: its edges sorted by (sender, edge), the start of each sender
+// segment, and the number of segments.  One block per cohort.
+__global__ void k_cohort_sort(long long E, int cohort, const int* __restrict__ send, int* __restrict__ perm,
+                              int* __restrict__ seg, int* __restrict__ nseg) {
+  extern __shared__ unsigned long long keys[];     // [P]
+  __shared__ int wsum[32];
+  const long long e0 = (long long)blockIdx.x * cohort;
+  const int n = (int)min((long long)cohort, E - e0);
+  int P = 1;
+  while (P < n) P <<= 1;
+  for (int k = threadIdx.x; k < P; k += blockDim.x)
+    keys[k] = k < n ? (((unsigned long long)(unsigned)send[e0 + k]) << 21) | (unsigned long long)k : ~0ull;
+  __syncthreads();
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = threadIdx.x; t < P; t += blockDim.x) {
+        const int partner = t ^ stride;
+        if (partner > t) {
+          const bool up = (t & size) == 0;
+          const unsigned long long a = keys[t], b = keys[partner];
+          if ((a > b) == up) { keys[t] = b; keys[partner] = a; }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // segment starts: serial over chunks, each thread a contiguous chunk
+  const int T = blockDim.x;
+  const int per = (n + T - 1) / T;
+  const int b = threadIdx.x * per, en = min(n, b + per);
+  int cnt = 0;
+  for (int k = b; k < en; ++k)
+    if (k == 0 || (keys[k] >> 21) != (keys[k - 1] >> 21)) ++cnt;
+  // block exclusive scan of cnt (T <= 1024)
+  int v = cnt;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += y;
+  }
+  if (lane == 31) wsum[w] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int q = 0; q < (T + 31) / 32; ++q) { const int y = wsum[q]; wsum[q] = acc; acc += y; }
+    nseg[blockIdx.x] = acc;
+  }
+  __syncthreads();
+  int pos = wsum[w] + v - cnt;
+  for (int k = b; k < en; ++k) {
+    if (k == 0 || (keys[k] >> 21) != (keys[k - 1] >> 21)) seg[e0 + pos++] = k;
+    perm[e0 + k] = (int)(keys[k] & ((1ull << 21) - 1));
+  }
+}
+
+// g_x[j] += sum over the cohort's edges with sender j (ascending edge) of GXS rows
+__global__ void k_sender_scatter(long long e0, long long e1, int C, int cohort_idx, const int* __restrict__ send,
+                                 const int* __restrict__ perm, const int* __restrict__ seg,
+                                 const int* __restrict__ nseg, const float* __restrict__ GXS,
+                                 float* __restrict__ gx) {
+  const int lane = threadIdx.x;
+  const int c = blockIdx.y * 32 + lane;
+  const int ns = nseg[cohort_idx];
+  const int n = (int)(e1 - e0);
+  for (int s = blockIdx.x; s < ns; s += gridDim.x) {
+    const int b = seg[e0 + s], en = (s + 1 < ns) ? seg[e0 + s + 1] : n;
+    const int j = send[e0 + perm[e0 + b]];
+    float acc[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+    for (int q = b; q < en; ++q) {
+      const float* g = GXS + (size_t)perm[e0 + q] * 16 * C;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) acc[k] += g[k * C + c];
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) gx[((size_t)j * 16 + k) * C + c] += acc[k];
+  }
+}
+
+// ------------------------------------------------------------------ forces and virial
+// F_i = sum over receiver i's edges of (g_e - g_mirror(e)), edge order
+__global__ void k_forces(int N, const int* __restrict__ recv_off, const int* __restrict__ mirror,
+                         const float* __restrict__ g_r, float* __restrict__ F) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= N) return;
+  float fx = 0.f, fy = 0.f, fz = 0.f;
+  for (int e = recv_off[i]; e < recv_off[i + 1]; ++e) {
+    const int m = mirror[e];
+    fx += g_r[3 * e + 0] - g_r[3 * m + 0];
+    fy += g_r[3 * e + 1] - g_r[3 * m + 1];
+    fz += g_r[3 * e + 2] - g_r[3 * m + 2];
+  }
+  F[3 * i + 0] = fx;
+  F[3 * i + 1] = fy;
+  F[3 * i + 2] = fz;
+}
+
+constexpr int VIR_BLOCKS = 256;
+// virial partials: block b sums edges b, b + VIR_BLOCKS*T, ... in double
+__global__ void k_virial_partial(long long E, const float* __restrict__ vec, const float* __restrict__ g_r,
+                                 double* __restrict__ part) {
+  __shared__ double s[9][256];
+  const int t = threadIdx.x;
+  double acc[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
+  for (long long e = (long long)blockIdx.x * blockDim.x + t; e < E; e += (long long)gridDim.x * blockDim.x)
+    for (int a = 0; a < 3; ++a)
+      for (int b = 0; b < 3; ++b) acc[a * 3 + b] -= (double)vec[3 * e + a] * (double)g_r[3 * e + b];
+  for (int q = 0; q < 9; ++q) s[q][t] = acc[q];
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (t < w)
+      for (int q = 0; q < 9; ++q) s[q][t] += s[q][t + w];
+    __syncthreads();
+  }
+  if (t == 0)
+    for (int q = 0; q < 9; ++q) part[blockIdx.x * 9 + q] = s[q][0];
+}
+
+__global__ void k_virial_final(int nb, const double* __restrict__ part, float* __restrict__ vir) {
+  const int q = threadIdx.x;
+  if (q >= 9) return;
+  double s = 0.0;
+  for (int b = 0; b < nb; ++b) s += part[b * 9 + q];
+  vir[q] = (float)s;
+}
+
+// x_0: degree 0 = emb[species], higher degrees zero
+__global__ void k_embed(int N, int C, const int* __restrict__ species, int n_species, const float* __restrict__ emb,
+                        float* __restrict__ x) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= N * 16 * C) return;
+  const int i = idx / (16 * C), r = idx % (16 * C), k = r / C, c = r % C;
+  int s = species ? species[i] : 0;
+  if (s < 0 || s >= n_species) { set_device_error(DEV_ERR_INDEX); s = 0; }
+  x[idx] = k == 0 ? emb[(size_t)s * C + c] : 0.f;
+}
+
+__global__ void k_scale(size_t n, float a, float* __restrict__ v) {
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) v[i] *= a;
+}
+
+}  // namespace emp

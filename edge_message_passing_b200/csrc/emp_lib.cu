@@ -1,0 +1,650 @@
+// C-ABI entry points of the equivariant edge message-passing library.
+// One translation unit: the kernel headers are included here.
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <vector>
+#include <algorithm>
+
+#include "emp_common.cuh"
+
+#include "nl.cuh"
+#include "model.cuh"
+#include "conv.cuh"
+#include "so2_tc.cuh"
+#include "chain.cuh"
+
+using namespace emp;
+
+#include <map>
+#include <string>
+#include <mutex>
+
+namespace {
+
+// ------------------------------------------------------------------ launch counting and event timing
+// Every kernel launch is counted.  When profiling is on, a pair of CUDA events
+// is recorded on the launching stream around each launch of a named kernel
+// family, so a benchmark can read the device time of each family.
+struct Prof {
+  std::mutex mu;
+  bool on = false;
+  long long launches = 0;
+  std::map<std::string, std::vector<std::pair<cudaEvent_t, cudaEvent_t>>> ev;
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t get() {
+    if (!pool.empty()) { cudaEvent_t e = pool.back(); pool.pop_back(); return e; }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+  void clear() {
+    for (auto& kv : ev)
+      for (auto& pr : kv.second) { pool.push_back(pr.first); pool.push_back(pr.second); }
+    ev.clear();
+  }
+} g_prof;
+
+struct Scope {
+  const char* name;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr;
+  Scope(const char* n, cudaStream_t st, int count = 1) : name(n), s(st) {
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    g_prof.launches += count;
+    if (g_prof.on) {
+      a = g_prof.get();
+      cudaEventRecord(a, s);
+    }
+  }
+  ~Scope() {
+    if (!a) return;
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    cudaEvent_t b = g_prof.get();
+    cudaEventRecord(b, s);
+    g_prof.ev[name].push_back({a, b});
+  }
+};
+
+inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
+
+// ------------------------------------------------------------------ workspace layout
+struct WsLayout {
+  size_t D, dist, R, gR, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GY, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir;
+  size_t total;
+};
+
+WsLayout ws_layout(const Model& m, long long E, int N) {
+  WsLayout L{};
+  const size_t C = m.spec.C, T = m.spec.n_layers;
+  const size_t coh = std::min<long long>(m.spec.cohort_edges, std::max<long long>(E, 1));
+  const size_t ncoh = E > 0 ? (E + m.spec.cohort_edges - 1) / m.spec.cohort_edges : 0;
+  const size_t feat = (size_t)N * 16 * C * 4;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t r = o; o = align_up(o + bytes); return r; };
+  L.D = take((size_t)E * NDBLK * 4);
+  L.dist = take((size_t)E * 4);
+  L.R = take(T * (size_t)E * 4 * C * 4);
+  L.gR = take((size_t)E * 4 * C * 4);
+  L.g_r = take((size_t)E * 3 * 4);
+  L.xs = take((T + 1) * feat);
+  L.aggs = take(T * feat);
+  L.gx0 = take(feat);
+  L.gx1 = take(feat);
+  L.gS = take(feat);
+  L.e_atom = take((size_t)N * 4);
+  const size_t cb = coh * 16 * C * 4;
+  L.XT = take(cb);
+  L.Y = take(cb);
+  L.GY = take(cb);
+  L.GXT = take(cb);
+  L.XTlo = take(cb);
+  L.GYhi = take(cb);
+  L.GYlo = take(cb);
+  L.perm = take((size_t)E * 4);
+  L.seg = take((size_t)E * 4);
+  L.nseg = take(ncoh * 4 + 4);
+  L.vir = take(VIR_BLOCKS * 9 * 8);
+  L.total = o;
+  return L;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
+
+bool graph_ok(const emp_graph* g) {
+  return g && g->recv && g->send && g->mirror && g->recv_off && g->vec && g->n_edges >= 0 &&
+         g->n_edges < (1ll << 31);
+}
+
+RadialArgs radial_args(const Model& m, int t) {
+  RadialArgs a;
+  a.rad = m.rad;
+  a.pair_stride = m.rad_stride();
+  a.layer_off = (size_t)t * m.n_pairs * a.pair_stride;
+  a.C = m.spec.C;
+  a.n_species = m.spec.n_species;
+  a.pair_radial = m.spec.pair_radial;
+  a.rc = m.spec.cutoff;
+  return a;
+}
+
+dim3 edge_block(int C) { return dim3(C, std::max(1, 256 / C)); }
+
+int grid_for(long long n, int per, int cap = 148 * 32) {
+  long long g = (n + per - 1) / per;
+  return (int)std::max<long long>(1, std::min<long long>(g, cap));
+}
+
+// one SO(2) block product of a cohort: tensor cores (3xTF32) with operands pre-split
+struct So2Operands {
+  const float* A_hi;
+  const float* A_lo;
+  const float* B_hi;
+  const float* B_lo;
+  const float* A;      // fp32 (simt path)
+  const float* B;
+};
+
+int so2_product(const Model& m, long long M, const So2Operands& op, float* Y, cudaStream_t s) {
+  Scope sc_("so2_tc", s);
+  return so2_tc(M, m.spec.C, op.A_hi, op.A_lo, op.B_hi, op.B_lo, Y, s);
+}
+
+void split(const float* a, float* hi, float* lo, size_t n, cudaStream_t s) {
+  { Scope sc_("split", s); k_split_tf32<<<grid_for((long long)n, 256, 148 * 16), 256, 0, s>>>(a, hi, lo, n); }
+}
+
+// forward of layer t over all cohorts: S (raw receiver sums) from x
+int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, const float* D, const float* R,
+                  float* S, void* ws, const WsLayout& L, cudaStream_t s) {
+  const int C = m.spec.C;
+  const long long E = g->n_edges, coh = m.spec.cohort_edges;
+  const dim3 eb = edge_block(C);
+  const size_t esmem = (size_t)eb.y * NDBLK * 4;
+  float* XT = at<float>(ws, L.XT);
+  float* XTlo = at<float>(ws, L.XTlo);
+  float* Y = at<float>(ws, L.Y);
+  const size_t so2off = (size_t)t * m.so2_stride();
+  for (long long e0 = 0; e0 < E; e0 += coh) {
+    const long long e1 = std::min(E, e0 + coh);
+    { Scope sc_("rotate_in", s); k_rotate_in<<<grid_for(e1 - e0, eb.y), eb, esmem, s>>>(e0, e1, C, g->send, D, R, x, XT, XTlo); }
+    So2Operands op{XT, XTlo, m.so2_fwd_hi + so2off, m.so2_fwd_lo + so2off, nullptr, nullptr};
+    int st = so2_product(m, e1 - e0, op, Y, s);
+    if (st != EMP_OK) return st;
+    dim3 grid(std::min<long long>(coh, 1024), C / 32);
+    { Scope sc_("rotate_back_scatter", s); k_rotate_back_scatter<<<grid, 32, 0, s>>>(e0, e1, C, g->recv, g->recv_off, D, Y, S); }
+  }
+  return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
+}
+
+void radial_forward(const Model& m, const emp_graph* g, int t, const int* species, const float* dist, float* R,
+                    cudaStream_t s) {
+  const long long E = g->n_edges;
+  { Scope sc_("radial_fwd", s); k_radial_fwd<<<(unsigned)((E + RT - 1) / RT), RAD_THREADS, sizeof(RadialSmem), s>>>(
+      E, dist, g->recv, g->send, species, radial_args(m, t), R); }
+}
+
+bool g_attrs_set = false;
+int ensure_attrs() {
+  if (g_attrs_set) return EMP_OK;
+  EMP_CUDA_TRY(cudaFuncSetAttribute(k_radial_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(RadialSmem)));
+  EMP_CUDA_TRY(cudaFuncSetAttribute(k_radial_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(RadialSmem)));
+  EMP_CUDA_TRY(cudaFuncSetAttribute(k_cohort_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, 8 << 14));
+  EMP_CUDA_TRY(cudaFuncSetAttribute(k_chain_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ChainFwdSmem)));
+  EMP_CUDA_TRY(cudaFuncSetAttribute(k_chain_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ChainBwdSmem)));
+  int st = so2_tc_init();
+  if (st != EMP_OK) return st;
+  g_attrs_set = true;
+  return EMP_OK;
+}
+
+int check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return EMP_ERR_UNSUPPORTED;
+  cudaDeviceProp p;
+  if (cudaGetDeviceProperties(&p, dev) != cudaSuccess) return EMP_ERR_UNSUPPORTED;
+  return p.major == 10 ? EMP_OK : EMP_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+const char* emp_status_string(int status) {
+  switch (status) {
+    case EMP_OK: return "ok";
+    case EMP_ERR_ARG: return "invalid argument";
+    case EMP_ERR_CAPACITY: return "graph capacity smaller than the edge count";
+    case EMP_ERR_CUDA: return "CUDA runtime error";
+    case EMP_ERR_TIMEOUT: return "bounded device wait timed out";
+    case EMP_ERR_NONFINITE: return "non-finite positions";
+    case EMP_ERR_WORKSPACE: return "workspace too small";
+    case EMP_ERR_DEVICE: return "device-side check failed";
+    case EMP_ERR_UNSUPPORTED: return "unsupported device or size";
+    default: return "unknown status";
+  }
+}
+
+int emp_profile_enable(int enable) {
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  g_prof.clear();
+  g_prof.on = enable != 0;
+  return EMP_OK;
+}
+
+int emp_profile_read(const char* name, double* total_ms, int64_t* launches) {
+  if (!name || !total_ms || !launches) return EMP_ERR_ARG;
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  double ms = 0.0;
+  int64_t n = 0;
+  for (auto& kv : g_prof.ev) {
+    if (std::strcmp(name, "*") != 0 && kv.first != name) continue;
+    for (auto& pr : kv.second) {
+      if (cudaEventSynchronize(pr.second) != cudaSuccess) return EMP_ERR_CUDA;
+      float t = 0.f;
+      if (cudaEventElapsedTime(&t, pr.first, pr.second) != cudaSuccess) return EMP_ERR_CUDA;
+      ms += t;
+      ++n;
+    }
+  }
+  *total_ms = ms;
+  *launches = n;
+  return EMP_OK;
+}
+
+int emp_profile_names(char* buf, size_t n) {
+  if (!buf || n == 0) return EMP_ERR_ARG;
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  std::string all;
+  for (auto& kv : g_prof.ev) { all += kv.first; all += ','; }
+  std::strncpy(buf, all.c_str(), n - 1);
+  buf[n - 1] = 0;
+  return EMP_OK;
+}
+
+int64_t emp_launch_count(void) {
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  return g_prof.launches;
+}
+
+int emp_last_device_error(void) {
+  int h = 0, z = 0;
+  if (cudaMemcpyFromSymbol(&h, g_device_error, sizeof(int)) != cudaSuccess) return EMP_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_device_error, &z, sizeof(int)) != cudaSuccess) return EMP_ERR_CUDA;
+  if (h == 0) return EMP_OK;
+  return h == DEV_ERR_TIMEOUT ? EMP_ERR_TIMEOUT : EMP_ERR_DEVICE;
+}
+
+// ------------------------------------------------------------------ neighbour list
+size_t nl_workspace_bytes(int32_t n_atoms) {
+  const size_t n = std::max(n_atoms, 1);
+  return align_up(n * 4) * 7 + align_up(n * 12) + align_up(16) + align_up(8) + 4096;
+}
+
+int nl_build(const emp_nl_params* p, const double* pos, emp_graph* g, int64_t* n_edges, void* ws,
+             size_t ws_bytes, cudaStream_t stream) {
+  if (!p || !pos || !g || !n_edges || !ws) return EMP_ERR_ARG;
+  const int N = p->n_atoms;
+  if (N < 1 || !(p->cutoff > 0) || !g->recv_off) return EMP_ERR_ARG;
+  for (int d = 0; d < 3; ++d)
+    if (!(p->box[d] > 0) || !std::isfinite(p->box[d])) return EMP_ERR_ARG;
+  if (ws_bytes < nl_workspace_bytes(N)) return EMP_ERR_WORKSPACE;
+  if (p->capacity > 0 && !graph_ok(g)) return EMP_ERR_ARG;
+  int st = check_device();
+  if (st != EMP_OK) return st;
+  // cell grid: cells no smaller than rc (1 + 1e-9), at most N cells
+  nl::Grid G;
+  const double rcp = p->cutoff * (1.0 + 1e-9);
+  long long ncell = 1;
+  for (int d = 0; d < 3; ++d) {
+    G.L[d] = p->box[d];
+    G.nc[d] = std::max(1, (int)std::floor(p->box[d] / rcp));
+  }
+  while ((ncell = (long long)G.nc[0] * G.nc[1] * G.nc[2]) > N) {
+    int d = 0;
+    for (int q = 1; q < 3; ++q)
+      if (G.nc[q] > G.nc[d]) d = q;
+    G.nc[d] = std::max(1, G.nc[d] / 2);
+  }
+  for (int d = 0; d < 3; ++d) G.s[d] = (int)std::ceil(rcp / (p->box[d] / G.nc[d]));
+  G.rc2 = p->cutoff * p->cutoff;
+  G.n_cells = (int)ncell;
+  // workspace carve
+  char* w = static_cast<char*>(ws);
+  size_t o = 0;
+  auto take = [&](size_t b) { char* r = w + o; o += align_up(b); return r; };
+  nl::Ws W;
+  W.cell_of = (int*)take(N * 4);
+  W.wrap = (int*)take((size_t)N * 12);
+  W.cell_count = (int*)take(N * 4);
+  W.cell_start = (int*)take((size_t)(N + 1) * 4);
+  W.cell_cursor = (int*)take(N * 4);
+  W.cell_atoms = (int*)take(N * 4);
+  W.deg = (int*)take(N * 4);
+  W.flags = (int*)take(16);
+  W.total = (long long*)take(8);
+  EMP_CUDA_TRY(cudaMemsetAsync(W.cell_count, 0, (size_t)G.n_cells * 4, stream));
+  EMP_CUDA_TRY(cudaMemsetAsync(W.cell_cursor, 0, (size_t)G.n_cells * 4, stream));
+  EMP_CUDA_TRY(cudaMemsetAsync(W.flags, 0, 16, stream));
+  { Scope sc_("nl", stream); nl::k_bin<<<(N + 255) / 256, 256, 0, stream>>>(pos, N, G, W); }
+  { Scope sc_("nl", stream); nl::k_scan<<<1, 1024, 0, stream>>>(W.cell_count, W.cell_start, G.n_cells, nullptr); }
+  { Scope sc_("nl", stream); nl::k_fill_cells<<<(N + 255) / 256, 256, 0, stream>>>(N, W); }
+  { Scope sc_("nl", stream); nl::k_count<<<(N * 32 + 255) / 256, 256, 0, stream>>>(pos, N, G, W); }
+  { Scope sc_("nl", stream); nl::k_scan<<<1, 1024, 0, stream>>>(W.deg, g->recv_off, N, W.total); }
+  long long total = 0;
+  int flags[4] = {0, 0, 0, 0};
+  EMP_CUDA_TRY(cudaMemcpyAsync(&total, W.total, 8, cudaMemcpyDeviceToHost, stream));
+  EMP_CUDA_TRY(cudaMemcpyAsync(flags, W.flags, 16, cudaMemcpyDeviceToHost, stream));
+  EMP_CUDA_TRY(cudaStreamSynchronize(stream));
+  if (flags[0]) return EMP_ERR_NONFINITE;
+  *n_edges = total;
+  g->n_edges = total;
+  g->n_atoms = N;
+  if (total > p->capacity) return EMP_ERR_CAPACITY;
+  if (total >= (1ll << 31)) return EMP_ERR_CAPACITY;
+  { Scope sc_("nl", stream); nl::k_emit<<<N, nl::EMIT_THREADS, 0, stream>>>(pos, N, G, W, g->recv_off, *g); }
+  if (total > 0) { Scope sc_("nl", stream); nl::k_mirror<<<(unsigned)((total + 255) / 256), 256, 0, stream>>>(total, N, *g); }
+  return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ model
+size_t mp_weight_count(const emp_model_spec* spec) { return spec ? weight_count(*spec) : 0; }
+
+int mp_model_create(const emp_model_spec* spec, const float* weights, size_t n_floats, void** model) {
+  if (!spec || !weights || !model) return EMP_ERR_ARG;
+  if (!spec_ok(*spec)) return EMP_ERR_ARG;
+  if (n_floats != weight_count(*spec)) return EMP_ERR_ARG;
+  int st = check_device();
+  if (st != EMP_OK) return st;
+  st = ensure_attrs();
+  if (st != EMP_OK) return st;
+  Model* m = new Model();
+  m->spec = *spec;
+  m->H = spec->radial_hidden;
+  m->Hro = spec->readout_hidden > 0 ? spec->readout_hidden : spec->C;
+  m->n_pairs = spec->pair_radial ? spec->n_species * (spec->n_species + 1) / 2 : 1;
+  cudaGetDevice(&m->device);
+  const size_t C = spec->C, T = spec->n_layers, S = spec->n_species;
+  const size_t n_emb = S * C, n_rad = T * m->n_pairs * m->rad_stride(), n_so2 = T * m->so2_stride();
+  const size_t n_ro = (size_t)m->Hro * C + m->Hro;
+  const size_t total = n_emb + n_rad + 6 * n_so2 + n_ro + n_floats;   // + raw staging
+  float* base = nullptr;
+  if (cudaMalloc(&base, total * 4) != cudaSuccess) { delete m; return EMP_ERR_CUDA; }
+  m->base = base;
+  m->emb = base;
+  m->rad = m->emb + n_emb;
+  m->so2_fwd = m->rad + n_rad;
+  m->so2_bwd = m->so2_fwd + n_so2;
+  m->so2_fwd_hi = m->so2_bwd + n_so2;
+  m->so2_fwd_lo = m->so2_fwd_hi + n_so2;
+  m->so2_bwd_hi = m->so2_fwd_lo + n_so2;
+  m->so2_bwd_lo = m->so2_bwd_hi + n_so2;
+  m->ro_W = m->so2_bwd_lo + n_so2;
+  m->ro_w = m->ro_W + (size_t)m->Hro * C;
+  float* raw = m->ro_w + m->Hro;
+  auto fail = [&](int code) { cudaFree(base); delete m; return code; };
+  if (cudaMemcpy(raw, weights, n_floats * 4, cudaMemcpyHostToDevice) != cudaSuccess) return fail(EMP_ERR_CUDA);
+  // walk the blob in declaration order
+  size_t o = 0;
+  if (cudaMemcpy(m->emb, raw + o, n_emb * 4, cudaMemcpyDeviceToDevice) != cudaSuccess) return fail(EMP_ERR_CUDA);
+  o += n_emb;
+  const size_t H = m->H;
+  for (size_t t = 0; t < T; ++t) {
+    const size_t rad_t = m->n_pairs * m->rad_stride();
+    if (cudaMemcpy(m->rad + t * rad_t, raw + o, rad_t * 4, cudaMemcpyDeviceToDevice) != cudaSuccess)
+      return fail(EMP_ERR_CUDA);
+    o += rad_t;
+    const float* W0 = raw + o;
+    o += 16 * C * C;
+    const float* Wr[3];
+    const float* Wi[3];
+    for (int mm = 1; mm <= 3; ++mm) {
+      const size_t h = (4 - mm) * C;
+      Wr[mm - 1] = raw + o;
+      o += h * h;
+      Wi[mm - 1] = raw + o;
+      o += h * h;
+    }
+    k_stack_so2<<<256, 256>>>(W0, Wr[0], Wi[0], Wr[1], Wi[1], Wr[2], Wi[2], (int)C, m->so2_fwd + t * m->so2_stride(),
+                              m->so2_bwd + t * m->so2_stride());
+  }
+  (void)H;
+  if (cudaMemcpy(m->ro_W, raw + o, n_ro * 4, cudaMemcpyDeviceToDevice) != cudaSuccess) return fail(EMP_ERR_CUDA);
+  o += n_ro;
+  if (o != n_floats) return fail(EMP_ERR_ARG);
+  k_split_tf32<<<256, 256>>>(m->so2_fwd, m->so2_fwd_hi, m->so2_fwd_lo, n_so2);
+  k_split_tf32<<<256, 256>>>(m->so2_bwd, m->so2_bwd_hi, m->so2_bwd_lo, n_so2);
+  // rotation generators on the structural pairs; every other entry must vanish
+  double J[3][NDBLK];
+  generator_blocks(J);
+  float jx[NJPAIR], jy[NJPAIR];
+  double outside = 0.0;
+  for (int a = 0; a < 16; ++a)
+    for (int b = 0; b < 16; ++b) {
+      bool listed = false;
+      for (int q = 0; q < NJPAIR; ++q)
+        if ((jpair_a(q) == a && jpair_b(q) == b) || (jpair_a(q) == b && jpair_b(q) == a)) listed = true;
+      if (!listed) outside += std::fabs(gen_at(J[0], a, b)) + std::fabs(gen_at(J[1], a, b));
+    }
+  if (outside > 1e-12) return fail(EMP_ERR_DEVICE);
+  for (int q = 0; q < NJPAIR; ++q) {
+    jx[q] = (float)gen_at(J[0], jpair_a(q), jpair_b(q));
+    jy[q] = (float)gen_at(J[1], jpair_a(q), jpair_b(q));
+  }
+  if (cudaMemcpyToSymbol(c_jx, jx, sizeof(jx)) != cudaSuccess) return fail(EMP_ERR_CUDA);
+  if (cudaMemcpyToSymbol(c_jy, jy, sizeof(jy)) != cudaSuccess) return fail(EMP_ERR_CUDA);
+  if (cudaDeviceSynchronize() != cudaSuccess) return fail(EMP_ERR_CUDA);
+  *model = m;
+  return EMP_OK;
+}
+
+void mp_model_destroy(void* model) {
+  if (!model) return;
+  Model* m = static_cast<Model*>(model);
+  cudaFree(m->base);
+  delete m;
+}
+
+size_t mp_workspace_bytes(const void* model, int64_t n_edges, int32_t n_atoms) {
+  if (!model || n_edges < 0 || n_atoms < 1) return 0;
+  return ws_layout(*static_cast<const Model*>(model), n_edges, n_atoms).total;
+}
+
+
+int mp_forward(const void* model, const emp_graph* g, int32_t layer, const int32_t* species, const float* x_in,
+               float* agg_out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!model || !graph_ok(g) || !x_in || !agg_out || !ws || g->n_atoms < 1) return EMP_ERR_ARG;
+  const Model& m = *static_cast<const Model*>(model);
+  if (layer < 0 || layer >= m.spec.n_layers) return EMP_ERR_ARG;
+  if (m.spec.pair_radial && !species) return EMP_ERR_ARG;
+  const long long E = g->n_edges;
+  const int N = g->n_atoms, C = m.spec.C;
+  const WsLayout L = ws_layout(m, E, N);
+  if (ws_bytes < L.total) return EMP_ERR_WORKSPACE;
+  int st = check_device();
+  if (st != EMP_OK) return st;
+  EMP_CUDA_TRY(cudaMemsetAsync(agg_out, 0, (size_t)N * 16 * C * 4, stream));
+  if (E == 0) return EMP_OK;
+  float* D = at<float>(ws, L.D);
+  float* dist = at<float>(ws, L.dist);
+  float* R = at<float>(ws, L.R);
+  { Scope sc_("geometry", stream); k_geometry<<<(unsigned)((E + 127) / 128), 128, 0, stream>>>(E, g->vec, D, dist); }
+  radial_forward(m, g, layer, species, dist, R, stream);
+  st = layer_forward(m, g, layer, x_in, D, R, agg_out, ws, L, stream);
+  if (st != EMP_OK) return st;
+  const size_t n = (size_t)N * 16 * C;
+  { Scope sc_("scale", stream); k_scale<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(n, 1.0f / m.spec.avg_degree, agg_out); }
+  return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
+}
+
+int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* species, double* energy, float* forces,
+                     float* virial, float* atom_energy, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!model || !graph_ok(g) || !energy || !forces || !ws || g->n_atoms < 1) return EMP_ERR_ARG;
+  const Model& m = *static_cast<const Model*>(model);
+  if ((m.spec.pair_radial || m.spec.n_species > 1) && !species) return EMP_ERR_ARG;
+  const long long E = g->n_edges, coh = m.spec.cohort_edges;
+  const int N = g->n_atoms, C = m.spec.C, T = m.spec.n_layers;
+  const WsLayout L = ws_layout(m, E, N);
+  if (ws_bytes < L.total) return EMP_ERR_WORKSPACE;
+  int st = check_device();
+  if (st != EMP_OK) return st;
+  const size_t feat = (size_t)N * 16 * C;
+  float* D = at<float>(ws, L.D);
+  float* dist = at<float>(ws, L.dist);
+  float* Rall = at<float>(ws, L.R);
+  float* gR = at<float>(ws, L.gR);
+  float* g_r = at<float>(ws, L.g_r);
+  float* xs = at<float>(ws, L.xs);
+  float* aggs = at<float>(ws, L.aggs);
+  float* gxa = at<float>(ws, L.gx0);
+  float* gxb = at<float>(ws, L.gx1);
+  float* gS = at<float>(ws, L.gS);
+  float* e_atom = atom_energy ? atom_energy : at<float>(ws, L.e_atom);
+  float* XT = at<float>(ws, L.XT);
+  float* XTlo = at<float>(ws, L.XTlo);
+  float* Y = at<float>(ws, L.Y);
+  float* GY = at<float>(ws, L.GY);
+  float* GYhi = at<float>(ws, L.GYhi);
+  float* GYlo = at<float>(ws, L.GYlo);
+  float* GXT = at<float>(ws, L.GXT);
+  int* perm = at<int>(ws, L.perm);
+  int* seg = at<int>(ws, L.seg);
+  int* nseg = at<int>(ws, L.nseg);
+  const float inv_avg = 1.0f / m.spec.avg_degree;
+  const dim3 eb = edge_block(C);
+
+  EMP_CUDA_TRY(cudaMemsetAsync(g_r, 0, (size_t)E * 12 + 4, stream));
+  EMP_CUDA_TRY(cudaMemsetAsync(aggs, 0, (size_t)T * feat * 4, stream));
+  { Scope sc_("embed", stream); k_embed<<<(unsigned)((feat + 255) / 256), 256, 0, stream>>>(N, C, species, m.spec.n_species, m.emb, xs); }
+  if (E > 0) {
+    { Scope sc_("geometry", stream); k_geometry<<<(unsigned)((E + 127) / 128), 128, 0, stream>>>(E, g->vec, D, dist); }
+    const int ncoh = (int)((E + coh - 1) / coh);
+    int P = 1;
+    while (P < coh) P <<= 1;
+    { Scope sc_("cohort_sort", stream); k_cohort_sort<<<ncoh, 1024, (size_t)P * 8, stream>>>(E, (int)coh, g->send, perm, seg, nseg); }
+  }
+  // ---------------- forward
+  for (int t = 0; t < T; ++t) {
+    float* R = Rall + (size_t)t * E * 4 * C;
+    if (E > 0) {
+      radial_forward(m, g, t, species, dist, R, stream);
+      st = layer_forward(m, g, t, xs + (size_t)t * feat, D, R, aggs + (size_t)t * feat, ws, L, stream);
+      if (st != EMP_OK) return st;
+    }
+    { Scope sc_("update", stream); k_update<<<(unsigned)((N * C + 255) / 256), 256, 0, stream>>>(N, C, inv_avg, m.spec.gated, aggs + (size_t)t * feat,
+                                                                   xs + (size_t)t * feat, xs + (size_t)(t + 1) * feat); }
+  }
+  { Scope sc_("readout", stream); k_readout<<<N, 256, 0, stream>>>(N, C, m.Hro, xs + (size_t)T * feat, m.ro_W, m.ro_w, e_atom, gxa); }
+  { Scope sc_("energy_sum", stream); k_energy_sum<<<1, 1024, 0, stream>>>(N, e_atom, energy); }
+  // ---------------- backward, one layer at a time in reverse, one cohort at a time
+  for (int t = T - 1; t >= 0; --t) {
+    const float* R = Rall + (size_t)t * E * 4 * C;
+    const float* xt = xs + (size_t)t * feat;
+    { Scope sc_("gate_bwd", stream); k_gate_bwd<<<(unsigned)((N * C + 255) / 256), 256, 0, stream>>>(N, C, inv_avg, m.spec.gated,
+                                                                     aggs + (size_t)t * feat, gxa, gS, gxb); }
+    const size_t so2off = (size_t)t * m.so2_stride();
+    int ci = 0;
+    for (long long e0 = 0; e0 < E; e0 += coh, ++ci) {
+      const long long e1 = std::min(E, e0 + coh), n = e1 - e0;
+      const int grid = grid_for(n, eb.y);
+      { Scope sc_("bwd_prep", stream); k_bwd_prep<<<grid, eb, (size_t)eb.y * NDBLK * 4, stream>>>(e0, e1, C, g->recv, g->send, D, R, xt, gS, XT, XTlo,
+                                                                  GY, GYhi, GYlo); }
+      So2Operands fwd{XT, XTlo, m.so2_fwd_hi + so2off, m.so2_fwd_lo + so2off, nullptr, nullptr};
+      st = so2_product(m, n, fwd, Y, stream);
+      if (st != EMP_OK) return st;
+      So2Operands bwd{GYhi, GYlo, m.so2_bwd_hi + so2off, m.so2_bwd_lo + so2off, nullptr, nullptr};
+      st = so2_product(m, n, bwd, GXT, stream);
+      if (st != EMP_OK) return st;
+      const size_t smem = (size_t)eb.y * NDBLK * 4 + (size_t)eb.y * 2 * (C / 32) * 4;
+      { Scope sc_("bwd_edge", stream); k_bwd_edge<<<grid, eb, smem, stream>>>(e0, e1, C, t > 0, g->send, g->vec, D, R, xt, Y, GY, GXT, XT, gR, g_r); }
+      if (t > 0) {
+        dim3 sg(std::min<long long>(n, 2048), C / 32);
+        { Scope sc_("sender_scatter", stream); k_sender_scatter<<<sg, 32, 0, stream>>>(e0, e1, C, ci, g->send, perm, seg, nseg, XT, gxb); }
+      }
+    }
+    if (E > 0)
+      { Scope sc_("radial_bwd", stream); k_radial_bwd<<<(unsigned)((E + RT - 1) / RT), RAD_THREADS, sizeof(RadialSmem), stream>>>(
+          E, dist, g->vec, g->recv, g->send, species, radial_args(m, t), gR, g_r); }
+    std::swap(gxa, gxb);
+  }
+  { Scope sc_("forces", stream); k_forces<<<(N + 127) / 128, 128, 0, stream>>>(N, g->recv_off, g->mirror, g_r, forces); }
+  if (virial) {
+    double* part = at<double>(ws, L.vir);
+    { Scope sc_("virial", stream); k_virial_partial<<<VIR_BLOCKS, 256, 0, stream>>>(E, g->vec, g_r, part); }
+    { Scope sc_("virial", stream); k_virial_final<<<1, 32, 0, stream>>>(VIR_BLOCKS, part, virial); }
+  }
+  return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
+}
+
+// One SO(2) mixing of a batch of edge-frame rows (the per-m block products
+// alone): Y = X B_b^T per block (transpose = 0) or Y = X B_b (transpose = 1),
+// X and Y [M][16C] in the m-major column layout.  Workspace: 2 M 16C floats.
+int mp_so2_mix(const void* model, int32_t layer, int32_t transpose, int64_t M, const float* X, float* Y, void* ws,
+               size_t ws_bytes, cudaStream_t stream) {
+  if (!model || !X || !Y || M < 0 || (M > 0 && !ws)) return EMP_ERR_ARG;
+  const Model& m = *static_cast<const Model*>(model);
+  if (layer < 0 || layer >= m.spec.n_layers) return EMP_ERR_ARG;
+  const size_t n = (size_t)M * 16 * m.spec.C;
+  if (ws_bytes < 2 * n * 4) return EMP_ERR_WORKSPACE;
+  if (M == 0) return EMP_OK;
+  int st = check_device();
+  if (st != EMP_OK) return st;
+  float* hi = static_cast<float*>(ws);
+  float* lo = hi + n;
+  split(X, hi, lo, n, stream);
+  const size_t off = (size_t)layer * m.so2_stride();
+  So2Operands op{hi, lo, (transpose ? m.so2_bwd_hi : m.so2_fwd_hi) + off, (transpose ? m.so2_bwd_lo : m.so2_fwd_lo) + off,
+                 nullptr, nullptr};
+  return so2_product(m, M, op, Y, stream);
+}
+
+// ------------------------------------------------------------------ radial chain
+int mp_chain_create(const float* U, const float* M, void** chain) {
+  if (!U || !M || !chain) return EMP_ERR_ARG;
+  int st = check_device();
+  if (st != EMP_OK) return st;
+  st = ensure_attrs();
+  if (st != EMP_OK) return st;
+  Chain* c = new Chain();
+  float* base = nullptr;
+  const size_t n = 128 * 25 + 32 * 64 + 4 * 32 * 64 + 256 * 25;
+  if (cudaMalloc(&base, n * 4) != cudaSuccess) { delete c; return EMP_ERR_CUDA; }
+  c->base = base;
+  c->Weff = base;
+  c->U0 = base + 128 * 25;
+  float* dU = c->U0 + 32 * 64;
+  float* dM = dU + 4 * 32 * 64;
+  if (cudaMemcpy(dU, U, 4 * 32 * 64 * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(dM, M, 256 * 25 * 4, cudaMemcpyHostToDevice) != cudaSuccess) {
+    cudaFree(base);
+    delete c;
+    return EMP_ERR_CUDA;
+  }
+  k_chain_fold<<<(128 * 25 + 255) / 256, 256>>>(dU, dM, c->Weff, c->U0);
+  if (cudaDeviceSynchronize() != cudaSuccess) { cudaFree(base); delete c; return EMP_ERR_CUDA; }
+  *chain = c;
+  return EMP_OK;
+}
+
+void mp_chain_destroy(void* chain) {
+  if (!chain) return;
+  Chain* c = static_cast<Chain*>(chain);
+  cudaFree(c->base);
+  delete c;
+}
+
+int mp_radial_chain(const void* chain, int64_t E, const float* x, float* kc, float* y0, const float* g_kc,
+                    const float* g_y0, float* g_x, cudaStream_t stream) {
+  if (!chain || E < 0 || (E > 0 && (!x || !kc || !y0))) return EMP_ERR_ARG;
+  if (g_x && E > 0 && (!g_kc || !g_y0)) return EMP_ERR_ARG;
+  if (E == 0) return EMP_OK;
+  const Chain& c = *static_cast<const Chain*>(chain);
+  const unsigned grid = (unsigned)((E + CH_ROWS - 1) / CH_ROWS);
+  { Scope sc_("chain_fwd", stream); k_chain_fwd<<<grid, 256, sizeof(ChainFwdSmem), stream>>>(E, x, c.Weff, c.U0, kc, y0); }
+  if (g_x) { Scope sc_("chain_bwd", stream); k_chain_bwd<<<grid, 256, sizeof(ChainBwdSmem), stream>>>(E, g_kc, g_y0, c.Weff, c.U0, g_x); }
+  return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,188 @@
+/*
+ * emp.h -- C ABI of the B200 equivariant edge message-passing library.
+ *
+ * The library computes the per-edge equivariant SO(2) message-passing
+ * convolution of a machine-learned interatomic potential (lmax = 3) and its
+ * input-gradient (force) backward, as described on the page "deepmd-kit PR:
+ * first-order SO(2) input-gradient path" (sections "Implementation and scope"
+ * and "Multi-model and N4096 update": 8192-edge receiver-sorted cohorts, strict
+ * FP32), with the radial projection chain of the page "deepmd-kit PR #6108:
+ * radial head fold" (section "What").
+ *
+ * Conventions shared by every entry point
+ *   - Pointers are DEVICE pointers unless the comment says (host).
+ *   - The caller owns every input, output and workspace buffer.  The library
+ *     owns only the model / chain objects it creates.  Inputs are never
+ *     written; outputs must not alias inputs.  (Ownership rule of the page
+ *     "first-order SO(2) input-gradient path", section "Implementation and
+ *     scope": never overwrite caller inputs.)
+ *   - Every call enqueues work on `stream` and returns; the only host
+ *     synchronisation is nl_build's read-back of the edge count.
+ *   - Results are bitwise identical from run to run (no floating-point
+ *     atomics; every sum has a fixed order).
+ *   - Errors are returned as emp_status codes; no exception crosses the ABI.
+ *     Errors detected on the device (index out of range, a bounded wait that
+ *     ran out) set a device error word reported by emp_last_device_error().
+ *
+ * Layouts
+ *   positions     double [N][3]
+ *   node features float  [N][16][C], component index lm = l*l + l + m
+ *                 (m = -l..l), channel-contiguous; real orthonormal spherical
+ *                 harmonics with z as polar axis, no Condon-Shortley phase
+ *                 (degree 1 is ordered y, z, x)
+ *   edges         sorted by receiver, then sender, then image shift
+ */
+#ifndef EMP_H
+#define EMP_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  EMP_OK = 0,
+  EMP_ERR_ARG = -1,        /* null pointer, bad size or alignment, inconsistent spec */
+  EMP_ERR_CAPACITY = -2,   /* graph buffers smaller than the edge count (see nl_build) */
+  EMP_ERR_CUDA = -3,       /* a CUDA runtime call failed */
+  EMP_ERR_TIMEOUT = -4,    /* a bounded device wait gave up */
+  EMP_ERR_NONFINITE = -5,  /* non-finite positions */
+  EMP_ERR_WORKSPACE = -6,  /* workspace smaller than the *_workspace_bytes value */
+  EMP_ERR_DEVICE = -7,     /* device-side check failed (index out of range, degree limit) */
+  EMP_ERR_UNSUPPORTED = -8 /* no sm_100 device, or a size the kernels do not support */
+} emp_status;
+
+/* ------------------------------------------------------------ neighbour list
+ * Defined on the page "first-order SO(2) input-gradient path" only as "the
+ * neighbour list" of the N64 / N4096 diamond workloads; this library builds
+ * the bit-exact cell-list form: an edge (i, j, S) exists iff, with
+ * r = (x_j - x_i) + S * L per Cartesian component in IEEE double (separate
+ * roundings, no fused multiply-add) and d2 = (rx*rx + ry*ry) + rz*rz,
+ * d2 < cutoff*cutoff; (i, i, 0) is excluded.  i is the receiver, j the sender.
+ */
+typedef struct {
+  int32_t n_atoms;
+  double box[3];       /* orthorhombic periodic box edges L (angstrom) */
+  double cutoff;       /* rc (angstrom) */
+  int64_t capacity;    /* edge capacity of the graph buffers */
+} emp_nl_params;
+
+typedef struct {
+  int32_t* recv;       /* [capacity] receiver i */
+  int32_t* send;       /* [capacity] sender j */
+  int32_t* mirror;     /* [capacity] index of the edge (j, i, -S) */
+  int32_t* recv_off;   /* [N+1] CSR offsets over receivers */
+  int32_t* shift;      /* [capacity][3] image shift S */
+  float* vec;          /* [capacity][3] r rounded to float32 */
+  int64_t n_edges;     /* number of valid edges (set by nl_build) */
+  int32_t n_atoms;     /* number of atoms N (set by nl_build) */
+} emp_graph;
+
+/* Workspace bytes nl_build needs for n_atoms atoms. */
+size_t nl_workspace_bytes(int32_t n_atoms);
+
+/* Build the neighbour list of `pos` into `g`.
+ * n_edges (host, out): the edge count, set also when EMP_ERR_CAPACITY is
+ * returned (two-phase use: call once with capacity 0 to size the buffers).
+ * Errors: EMP_ERR_ARG (null pointers, n_atoms < 1, non-positive box or
+ * cutoff), EMP_ERR_NONFINITE, EMP_ERR_CAPACITY, EMP_ERR_WORKSPACE,
+ * EMP_ERR_DEVICE (more than 4096 candidate neighbours for one receiver). */
+int nl_build(const emp_nl_params* p, const double* pos, emp_graph* g, int64_t* n_edges,
+             void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------ the model
+ * Hyper-parameters of the interatomic potential (configs of the seeded
+ * workloads; model of the page "first-order SO(2) input-gradient path":
+ * lmax = 3, three layers, strict FP32).  lmax is fixed at 3. */
+typedef struct {
+  int32_t C;              /* channels per component; multiple of 32, 32..256 */
+  int32_t n_layers;       /* interaction layers (>= 1) */
+  int32_t n_species;      /* >= 1 */
+  int32_t n_basis;        /* Bessel functions; must be 8 */
+  int32_t radial_hidden;  /* radial MLP width; must be 64 */
+  int32_t readout_hidden; /* readout MLP width (<= 256) */
+  int32_t gated;          /* 1: x <- x + G(agg) after each layer; 0: h = agg */
+  int32_t pair_radial;    /* 1: one radial MLP per unordered species pair */
+  int32_t cohort_edges;   /* receiver-sorted edge cohort size (multiple of 128, <= 16384) */
+  float cutoff;           /* rc */
+  int32_t env_p;          /* envelope exponent; must be 6 */
+  float avg_degree;       /* aggregation normaliser (158) */
+} emp_model_spec;
+
+/* Number of floats of the weight blob for `spec` (declaration order: emb
+ * [S][C]; per layer: per radial network W1 [H][8], W2 [H][H], W3 [4C][H];
+ * W0 [4C][4C]; for m = 1, 2, 3: Wr_m, Wi_m [(4-m)C][(4-m)C]; then readout
+ * W_ro [H_ro][C], w_o [H_ro]).  All linear maps bias-free, stored (out, in). */
+size_t mp_weight_count(const emp_model_spec* spec);
+
+/* Copy (host blob -> device), stack the SO(2) blocks, split them for
+ * 3xTF32 and build the rotation generators.  model (host, out). */
+int mp_model_create(const emp_model_spec* spec, const float* weights /*(host)*/, size_t n_floats,
+                    void** model);
+void mp_model_destroy(void* model);
+
+/* Workspace bytes mp_forward / mp_energy_forces need. */
+size_t mp_workspace_bytes(const void* model, int64_t n_edges, int32_t n_atoms);
+
+/* One interaction layer (forward only): agg_out[i] = (1/avg_degree) * sum over
+ * edges e with recv(e) = i of D(R_e)^T SO2_layer(R_e(d) (.) D(R_e) x_in[send(e)]).
+ * species [N] int32 selects the radial network when pair_radial is set. */
+int mp_forward(const void* model, const emp_graph* g, int32_t layer, const int32_t* species,
+               const float* x_in, float* agg_out, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Energy and forces: energy (double[1]) = sum_i e_i, forces [N][3] = -dE/dx,
+ * virial [9] = -sum_e r_e (x) dE/dr_e (row-major) or NULL, atom_energy [N] or NULL. */
+int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* species,
+                     double* energy, float* forces, float* virial, float* atom_energy,
+                     void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* The per-m SO(2) channel mixing of a batch of edge-frame rows on its own
+ * (page "first-order SO(2) input-gradient path": the mixing GEMMs, strict
+ * FP32 -- here 3xTF32 on the tensor cores).  X, Y [M][16C] in the m-major
+ * column layout [m=0 (l=0..3) | +1 (l=1..3) | -1 | +2 | -2 | +3 | -3], each
+ * entry C channels.  transpose = 0: Y_b = X_b B_b^T (forward, y+ = Wr x+ - Wi x-,
+ * y- = Wi x+ + Wr x-, y0 = W0 x0); transpose = 1: the adjoint map.
+ * Workspace >= 2 * M * 16 * C floats (the TF32 split of X). */
+int mp_so2_mix(const void* model, int32_t layer, int32_t transpose, int64_t M, const float* X, float* Y,
+               void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------ radial chain
+ * Page "deepmd-kit PR #6108: radial head fold", section "What": basis x
+ * (E,4,32) -> per-degree up-projection U_l (32 -> 64) -> (E,256) @ M (256,25).
+ * The chain object folds W_eff = vstack_l(U_l M_l) (128 x 25) once. */
+int mp_chain_create(const float* U /*(host) [4][32][64] (in,out)*/,
+                    const float* M /*(host) [256][25] (in,out)*/, void** chain /*(host) out*/);
+void mp_chain_destroy(void* chain);
+
+/* kc [E][25] = x_flat @ W_eff; y0 [E][64] = x[:,0,:] @ U_0.  If g_x is not
+ * NULL also g_x [E][4][32] = g_kc @ W_eff^T (+ g_y0 @ U_0^T into degree 0).
+ * x, g_kc, g_y0 row-major; E >= 0. */
+int mp_radial_chain(const void* chain, int64_t E, const float* x, float* kc, float* y0,
+                    const float* g_kc, const float* g_y0, float* g_x, cudaStream_t stream);
+
+/* ------------------------------------------------------------ timing
+ * Every kernel launch of the library is counted.  With profiling enabled, a
+ * pair of CUDA events is recorded on the launching stream around each launch,
+ * grouped by kernel family ("so2_tc", "rotate_in", "rotate_back_scatter",
+ * "bwd_prep", "bwd_edge", "sender_scatter", "radial_fwd", "radial_bwd",
+ * "geometry", "nl", ...).  Host-side bookkeeping only; kernels are unchanged. */
+int emp_profile_enable(int enable);                    /* also clears recorded events */
+/* Device milliseconds and launch count of one family ("*" = all) recorded since
+ * the last emp_profile_enable; synchronises on the recorded events. */
+int emp_profile_read(const char* name, double* total_ms, int64_t* launches);
+/* Comma-separated names of the families recorded so far, into buf[n]. */
+int emp_profile_names(char* buf, size_t n);
+int64_t emp_launch_count(void);                        /* kernels launched since the library was loaded */
+
+/* ------------------------------------------------------------ status */
+const char* emp_status_string(int status);
+/* Reads and clears the device error word of the current device (synchronises). */
+int emp_last_device_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* EMP_H */
