@@ -290,18 +290,18 @@ def run_ours(args):
     fl_per_edge = 2 * 72 * C * C                      # useful flops of one SO(2) mixing of one edge
     so2_launches = fam.get("so2_tc", (0, 0))[1]
     roof = None
-    if dom == "so2_tc" and so2_launches:
+    if so2_launches:
         so2_ms = fam["so2_tc"][0] / so2_launches
-        # launches per step: 3 per layer per cohort (forward, backward recompute, transpose)
         ncoh = -(-E // spec.cohort_edges)
-        rows = E * 3 * spec.n_layers / (ncoh * 3 * spec.n_layers)   # mean rows per launch
+        rows = E / ncoh                                   # mean rows (edges) per launch: one cohort
         achieved = rows * fl_per_edge / (so2_ms * 1e-3) / 1e12
         peak_tf32 = pk["bf16_tflops_sustained"] * TF32_OVER_BF16
         peak = peak_tf32 / 3.0
         roof = {"bound": "tensor", "kernel": "so2_tc (3xTF32 tcgen05 SO(2) mixing)", "achieved": achieved,
                 "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
-                "peak_note": f"useful FP32-equivalent flops vs (sustained bf16 {pk_kind} x {TF32_OVER_BF16:.3f}) / 3 "
-                             f"for 3xTF32"}
+                "launch_ms": so2_ms, "dominant": dom == "so2_tc",
+                "peak_note": f"useful FP32 flops (2*72*C^2 per edge) per launch / event time, vs sustained bf16 "
+                             f"({pk_kind}) x {TF32_OVER_BF16:.3f} (TF32/BF16 nominal) / 3 (3xTF32)"}
     elif dom is not None:
         roof = {"bound": "hbm", "kernel": dom, "achieved": None, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": None, "traffic": None}
