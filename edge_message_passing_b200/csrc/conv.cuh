@@ -344,35 +344,61 @@ __global__ void k_rotate_in(long long e0, long long e1, int C, const int* __rest
 }
 
 // ------------------------------------------------------------------ rotate back + receiver sums
-// S[i] (+)= sum over the cohort's edges of receiver i of D_e^T y_e, in edge order.
-// A receiver whose edges started in an earlier cohort continues its running sum.
-__global__ void k_rotate_back_scatter(long long e0, long long e1, int C, const int* __restrict__ recv,
-                                      const int* __restrict__ recv_off, const float* __restrict__ D,
-                                      const float* __restrict__ Y, float* __restrict__ S) {
-  __shared__ __align__(16) float sD[NDBLK];
-  const int lane = threadIdx.x;                           // 32 channels per block
-  const int c = blockIdx.y * 32 + lane;
+// S[i] (+)= sum over the cohort's edges of receiver i of D_e^T y_e.
+// One block per (receiver, 64-channel group): RB_ROWS rows take the receiver's
+// edges round-robin (row r: edges b + r, b + r + RB_ROWS, ...), each row sums
+// its edges in order, then the rows are added in row order onto the running
+// sum carried from earlier cohorts.  The order is fixed, so results are
+// reproducible; a receiver whose edges started in an earlier cohort continues
+// its running sum.
+constexpr int RB_ROWS = 8;
+constexpr int RB_CG = 64;
+
+__global__ void __launch_bounds__(RB_CG * RB_ROWS) k_rotate_back_scatter(long long e0, long long e1, int C,
+                                                                         const int* __restrict__ recv,
+                                                                         const int* __restrict__ recv_off,
+                                                                         const float* __restrict__ D,
+                                                                         const float* __restrict__ Y,
+                                                                         float* __restrict__ S) {
+  __shared__ __align__(16) float sD[RB_ROWS][NDBLK];
+  __shared__ float part[RB_ROWS][16][RB_CG];
+  const int cg = min(C, RB_CG);
+  const int tx = threadIdx.x, row = threadIdx.y;
+  const int c = blockIdx.y * cg + tx;
   const int first = recv[e0], last = recv[e1 - 1];
   for (int i = first + blockIdx.x; i <= last; i += gridDim.x) {
-    const long long b = max((long long)recv_off[i], e0), e_end = min((long long)recv_off[i + 1], e1);
-    float acc[16];
+    const long long b = max((long long)recv_off[i], e0), en = min((long long)recv_off[i + 1], e1);
     const bool carry = recv_off[i] < e0;
+    float acc[16];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) acc[k] = carry ? S[((size_t)i * 16 + k) * C + c] : 0.f;
-    for (long long e = b; e < e_end; ++e) {
-      __syncwarp();
-      for (int k = lane; k < NDBLK; k += 32) sD[k] = D[(size_t)e * NDBLK + k];
-      __syncwarp();
-      const float* y = Y + (size_t)(e - e0) * 16 * C;
-      float yv[16], m[16];
+    for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+    for (long long base = b; base < en; base += RB_ROWS) {
+      const long long e = base + row;
+      const bool ok = e < en;
+      __syncthreads();
+      if (ok)
+        for (int k = tx; k < NDBLK; k += cg) sD[row][k] = D[(size_t)e * NDBLK + k];
+      __syncthreads();
+      if (ok) {
+        const float* y = Y + (size_t)(e - e0) * 16 * C;
+        float yv[16], m[16];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) yv[k] = y[col_of_k(k) * C + c];
-      rotate16<true>(sD, yv, m);
+        for (int k = 0; k < 16; ++k) yv[k] = y[col_of_k(k) * C + c];
+        rotate16<true>(sD[row], yv, m);
 #pragma unroll
-      for (int k = 0; k < 16; ++k) acc[k] += m[k];
+        for (int k = 0; k < 16; ++k) acc[k] += m[k];
+      }
     }
 #pragma unroll
-    for (int k = 0; k < 16; ++k) S[((size_t)i * 16 + k) * C + c] = acc[k];
+    for (int k = 0; k < 16; ++k) part[row][k][tx] = acc[k];
+    __syncthreads();
+    for (int k = row; k < 16; k += RB_ROWS) {
+      float s = carry ? S[((size_t)i * 16 + k) * C + c] : 0.f;
+#pragma unroll
+      for (int r = 0; r < RB_ROWS; ++r) s += part[r][k][tx];
+      S[((size_t)i * 16 + k) * C + c] = s;
+    }
+    __syncthreads();
   }
 }
 
@@ -531,11 +557,75 @@ __global__ void k_bwd_prep(long long e0, long long e1, int C, const int* __restr
 //   gR[e][l][c] = sum_m g_x~ u;  g_u = R (.) g_x~;  g_xs = D^T g_u (-> GXS, [16][C] rows)
 //   b_j = sum_c (y^T J_j g_y + g_u^T J_j u), j = x, y (edge frame); a = -R_e^T (b_x, b_y, 0);
 //   g_r[e] += (a x r) / |r|^2  (direction part of dE/dr; the radial part is added by k_radial_bwd)
-__global__ void k_bwd_edge(long long e0, long long e1, int C, int need_gx, const int* __restrict__ send,
-                           const float* __restrict__ vec, const float* __restrict__ D, const float* __restrict__ R,
-                           const float* __restrict__ x, const float* __restrict__ Y, const float* __restrict__ GY,
-                           const float* __restrict__ GXT, float* __restrict__ GXS, float* __restrict__ gR,
-                           float* __restrict__ g_r) {
+// J_x, J_y are antisymmetric and couple components of one degree whose |m| differ by
+// one, so v^T J w = sum over the structural pairs (a < b) of J_ab (v_a w_b - v_b w_a).
+template <int L>
+__device__ __forceinline__ void torque_pairs_l(const float* v, const float* w, float& bx, float& by) {
+  // v, w: the 2L+1 components of degree L (local index m + L)
+  constexpr int p0 = L == 1 ? 0 : L == 2 ? 2 : 8;
+  constexpr int p1 = L == 1 ? 2 : L == 2 ? 8 : NJPAIR;
+#pragma unroll
+  for (int p = p0; p < p1; ++p) {
+    const int A = jpair_a(p) - L * L, B = jpair_b(p) - L * L;
+    const float q = v[A] * w[B] - v[B] * w[A];
+    bx = fmaf(c_jx[p], q, bx);
+    by = fmaf(c_jy[p], q, by);
+  }
+}
+
+// degree-L part of the per-edge backward for one channel
+template <int L>
+__device__ __forceinline__ void bwd_edge_degree(const float* __restrict__ Dr, const float* __restrict__ xs,
+                                                const float* __restrict__ yrow, const float* __restrict__ gyrow,
+                                                const float* __restrict__ gxtrow, float Rl, int C, int c,
+                                                bool need_gx, float* __restrict__ gxsrow, float& grl,
+                                                float& bx, float& by) {
+  constexpr int W = 2 * L + 1, O = L * L;
+  const float* B = Dr + dblk_off(L);
+  float v[W], u[W], gu[W];
+#pragma unroll
+  for (int n = 0; n < W; ++n) v[n] = xs[(O + n) * C];
+#pragma unroll
+  for (int m = 0; m < W; ++m) {
+    float a = 0.f;
+#pragma unroll
+    for (int n = 0; n < W; ++n) a = fmaf(B[m * W + n], v[n], a);
+    u[m] = a;
+  }
+  grl = 0.f;
+#pragma unroll
+  for (int m = 0; m < W; ++m) {
+    const float g = gxtrow[col_of_k(O + m) * C];
+    grl = fmaf(g, u[m], grl);
+    gu[m] = Rl * g;
+  }
+  if (L > 0) {
+    torque_pairs_l<L>(gu, u, bx, by);
+#pragma unroll
+    for (int m = 0; m < W; ++m) {
+      v[m] = yrow[col_of_k(O + m) * C];
+      u[m] = gyrow[col_of_k(O + m) * C];
+    }
+    torque_pairs_l<L>(v, u, bx, by);
+  }
+  if (need_gx) {
+#pragma unroll
+    for (int m = 0; m < W; ++m) {
+      float a = 0.f;
+#pragma unroll
+      for (int n = 0; n < W; ++n) a = fmaf(B[n * W + m], gu[n], a);
+      gxsrow[(O + m) * C] = a;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256, 2) k_bwd_edge(long long e0, long long e1, int C, int need_gx,
+                                                     const int* __restrict__ send, const float* __restrict__ vec,
+                                                     const float* __restrict__ D, const float* __restrict__ R,
+                                                     const float* __restrict__ x, const float* __restrict__ Y,
+                                                     const float* __restrict__ GY, const float* __restrict__ GXT,
+                                                     float* __restrict__ GXS, float* __restrict__ gR,
+                                                     float* __restrict__ g_r) {
   extern __shared__ __align__(16) float smem[];
   const int c = threadIdx.x, row = threadIdx.y, EPB = blockDim.y;
   float* sD = smem;                                 // [EPB][84]
@@ -553,46 +643,23 @@ __global__ void k_bwd_edge(long long e0, long long e1, int C, int need_gx, const
     float bx = 0.f, by = 0.f;
     if (ok) {
       const float* Dr = sD + row * NDBLK;
-      const int j = send[e];
-      float v[16], u[16];
-#pragma unroll
-      for (int k = 0; k < 16; ++k) v[k] = x[((size_t)j * 16 + k) * C + c];
-      rotate16<false>(Dr, v, u);
-      float Rv[4];
-#pragma unroll
-      for (int l = 0; l < 4; ++l) Rv[l] = R[(size_t)e * 4 * C + l * C + c];
       const size_t rowoff = (size_t)el * 16 * C;
-      float gxt[16], gu[16];
-#pragma unroll
-      for (int k = 0; k < 16; ++k) gxt[k] = GXT[rowoff + col_of_k(k) * C + c];
-      float gr[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        gr[deg_of(k)] = fmaf(gxt[k], u[k], gr[deg_of(k)]);
-        gu[k] = Rv[deg_of(k)] * gxt[k];
-      }
-#pragma unroll
-      for (int l = 0; l < 4; ++l) gR[(size_t)e * 4 * C + l * C + c] = gr[l];
-      float yv[16], gy[16];
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        yv[k] = Y[rowoff + col_of_k(k) * C + c];
-        gy[k] = GY[rowoff + col_of_k(k) * C + c];
-      }
-#pragma unroll
-      for (int p = 0; p < NJPAIR; ++p) {
-        const int A = jpair_a(p), B = jpair_b(p);
-        const float q = (yv[A] * gy[B] - yv[B] * gy[A]) + (gu[A] * u[B] - gu[B] * u[A]);
-        bx = fmaf(c_jx[p], q, bx);
-        by = fmaf(c_jy[p], q, by);
-      }
-      if (need_gx) {
-        float gxs[16];
-        rotate16<true>(Dr, gu, gxs);
-        float* out = GXS + rowoff;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) out[k * C + c] = gxs[k];
-      }
+      const float* xs = x + (size_t)send[e] * 16 * C + c;
+      const float* Rr = R + (size_t)e * 4 * C + c;
+      float* gRr = gR + (size_t)e * 4 * C + c;
+      const float* yr = Y + rowoff + c;
+      const float* gyr = GY + rowoff + c;
+      const float* gxr = GXT + rowoff + c;
+      float* gsr = GXS + rowoff + c;
+      float gr;
+      bwd_edge_degree<0>(Dr, xs, yr, gyr, gxr, Rr[0], C, c, need_gx, gsr, gr, bx, by);
+      gRr[0] = gr;
+      bwd_edge_degree<1>(Dr, xs, yr, gyr, gxr, Rr[C], C, c, need_gx, gsr, gr, bx, by);
+      gRr[C] = gr;
+      bwd_edge_degree<2>(Dr, xs, yr, gyr, gxr, Rr[2 * C], C, c, need_gx, gsr, gr, bx, by);
+      gRr[2 * C] = gr;
+      bwd_edge_degree<3>(Dr, xs, yr, gyr, gxr, Rr[3 * C], C, c, need_gx, gsr, gr, bx, by);
+      gRr[3 * C] = gr;
     }
     // deterministic reduction of (bx, by) over the row's channels
 #pragma unroll

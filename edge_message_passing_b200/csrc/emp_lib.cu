@@ -172,8 +172,9 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
     So2Operands op{XT, XTlo, m.so2_fwd_hi + so2off, m.so2_fwd_lo + so2off, nullptr, nullptr};
     int st = so2_product(m, e1 - e0, op, Y, s);
     if (st != EMP_OK) return st;
-    dim3 grid(std::min<long long>(coh, 1024), C / 32);
-    { Scope sc_("rotate_back_scatter", s); k_rotate_back_scatter<<<grid, 32, 0, s>>>(e0, e1, C, g->recv, g->recv_off, D, Y, S); }
+    const int cg = std::min(C, RB_CG);
+    dim3 grid((unsigned)std::min<long long>(coh, 512), C / cg);
+    { Scope sc_("rotate_back_scatter", s); k_rotate_back_scatter<<<grid, dim3(cg, RB_ROWS), 0, s>>>(e0, e1, C, g->recv, g->recv_off, D, Y, S); }
   }
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
