@@ -288,7 +288,7 @@ def mp_so2_mix(model: Model, layer: int, X, transpose: bool = False):
     torch = _torch()
     X = X.contiguous()
     Y = torch.empty_like(X)
-    ws = _workspace(2 * X.numel() * 4)
+    ws = _workspace(2 * X.numel() * 4 + 256)
     _check(lib().mp_so2_mix(model.handle, layer, int(transpose), X.shape[0], _ptr(X), _ptr(Y), _ptr(ws),
                             ws.numel(), _stream()), "mp_so2_mix")
     return Y

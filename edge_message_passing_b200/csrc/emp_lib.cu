@@ -70,7 +70,7 @@ inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 
 // ------------------------------------------------------------------ workspace layout
 struct WsLayout {
-  size_t D, dist, R, gR, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GY, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir;
+  size_t D, dist, R, gR, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GY, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
   size_t total;
 };
 
@@ -105,6 +105,7 @@ WsLayout ws_layout(const Model& m, long long E, int N) {
   L.seg = take((size_t)E * 4);
   L.nseg = take(ncoh * 4 + 4);
   L.vir = take(VIR_BLOCKS * 9 * 8);
+  L.counter = take(64);
   L.total = o;
   return L;
 }
@@ -136,20 +137,29 @@ int grid_for(long long n, int per, int cap = 148 * 32) {
   return (int)std::max<long long>(1, std::min<long long>(g, cap));
 }
 
-// one SO(2) block product of a cohort: tensor cores (3xTF32) with operands pre-split
-struct So2Operands {
-  const float* A_hi;
-  const float* A_lo;
-  const float* B_hi;
-  const float* B_lo;
-  const float* A;      // fp32 (simt path)
-  const float* B;
-};
-
-int so2_product(const Model& m, long long M, const So2Operands& op, float* Y, cudaStream_t s) {
+// SO(2) block products of a cohort on the tensor cores (3xTF32, operands pre-split):
+// one operand set (forward) or two sharing the rows (backward: recompute + transpose)
+int so2_product(const Model& m, long long M, const So2Part* parts, int nparts, int* counter, cudaStream_t s) {
   Scope sc_("so2_tc", s);
-  return so2_tc(M, m.spec.C, op.A_hi, op.A_lo, op.B_hi, op.B_lo, Y, s);
+  return so2_tc(M, m.spec.C, parts, nparts, counter, s);
 }
+
+// tensor maps of a cohort buffer pair for the full cohort size and for the last (short) cohort
+struct CohortMaps {
+  So2AMaps full, tail;
+  long long coh = 0, tail_rows = 0;
+  int build(int C, long long E, long long cohort, const float* hi, const float* lo) {
+    coh = std::min(E, cohort);
+    tail_rows = E % cohort;
+    if (coh > 0) {
+      int st = so2_make_amaps(&full, C, coh, hi, lo);
+      if (st != EMP_OK) return st;
+    }
+    if (tail_rows > 0 && tail_rows != coh) return so2_make_amaps(&tail, C, tail_rows, hi, lo);
+    return EMP_OK;
+  }
+  const So2AMaps* get(long long rows) const { return rows == coh ? &full : &tail; }
+};
 
 void split(const float* a, float* hi, float* lo, size_t n, cudaStream_t s) {
   { Scope sc_("split", s); k_split_tf32<<<grid_for((long long)n, 256, 148 * 16), 256, 0, s>>>(a, hi, lo, n); }
@@ -165,12 +175,15 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
   float* XT = at<float>(ws, L.XT);
   float* XTlo = at<float>(ws, L.XTlo);
   float* Y = at<float>(ws, L.Y);
-  const size_t so2off = (size_t)t * m.so2_stride();
+  CohortMaps am;
+  int st0 = am.build(C, E, coh, XT, XTlo);
+  if (st0 != EMP_OK) return st0;
+  int* counter = at<int>(ws, L.counter);
   for (long long e0 = 0; e0 < E; e0 += coh) {
     const long long e1 = std::min(E, e0 + coh);
     { Scope sc_("rotate_in", s); k_rotate_in<<<grid_for(e1 - e0, eb.y), eb, esmem, s>>>(e0, e1, C, g->send, D, R, x, XT, XTlo); }
-    So2Operands op{XT, XTlo, m.so2_fwd_hi + so2off, m.so2_fwd_lo + so2off, nullptr, nullptr};
-    int st = so2_product(m, e1 - e0, op, Y, s);
+    So2Part part{am.get(e1 - e0), &m.bmaps_fwd[t], Y};
+    int st = so2_product(m, e1 - e0, &part, 1, counter, s);
     if (st != EMP_OK) return st;
     const int cg = std::min(C, RB_CG);
     dim3 grid((unsigned)std::min<long long>(coh, 512), C / cg);
@@ -417,6 +430,14 @@ int mp_model_create(const emp_model_spec* spec, const float* weights, size_t n_f
   if (o != n_floats) return fail(EMP_ERR_ARG);
   k_split_tf32<<<256, 256>>>(m->so2_fwd, m->so2_fwd_hi, m->so2_fwd_lo, n_so2);
   k_split_tf32<<<256, 256>>>(m->so2_bwd, m->so2_bwd_hi, m->so2_bwd_lo, n_so2);
+  m->bmaps_fwd.resize(T);
+  m->bmaps_bwd.resize(T);
+  for (size_t t = 0; t < T; ++t) {
+    const size_t off = t * m->so2_stride();
+    if (so2_make_bmaps(&m->bmaps_fwd[t], (int)C, m->so2_fwd_hi + off, m->so2_fwd_lo + off) != EMP_OK ||
+        so2_make_bmaps(&m->bmaps_bwd[t], (int)C, m->so2_bwd_hi + off, m->so2_bwd_lo + off) != EMP_OK)
+      return fail(EMP_ERR_CUDA);
+  }
   // rotation generators on the structural pairs; every other entry must vanish
   double J[3][NDBLK];
   generator_blocks(J);
@@ -515,6 +536,12 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
   int* nseg = at<int>(ws, L.nseg);
   const float inv_avg = 1.0f / m.spec.avg_degree;
   const dim3 eb = edge_block(C);
+  int* counter = at<int>(ws, L.counter);
+  CohortMaps am_xt, am_gy;
+  st = am_xt.build(C, E, coh, XT, XTlo);
+  if (st != EMP_OK) return st;
+  st = am_gy.build(C, E, coh, GYhi, GYlo);
+  if (st != EMP_OK) return st;
 
   EMP_CUDA_TRY(cudaMemsetAsync(g_r, 0, (size_t)E * 12 + 4, stream));
   EMP_CUDA_TRY(cudaMemsetAsync(aggs, 0, (size_t)T * feat * 4, stream));
@@ -545,18 +572,14 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
     const float* xt = xs + (size_t)t * feat;
     { Scope sc_("gate_bwd", stream); k_gate_bwd<<<(unsigned)((N * C + 255) / 256), 256, 0, stream>>>(N, C, inv_avg, m.spec.gated,
                                                                      aggs + (size_t)t * feat, gxa, gS, gxb); }
-    const size_t so2off = (size_t)t * m.so2_stride();
     int ci = 0;
     for (long long e0 = 0; e0 < E; e0 += coh, ++ci) {
       const long long e1 = std::min(E, e0 + coh), n = e1 - e0;
       const int grid = grid_for(n, eb.y);
       { Scope sc_("bwd_prep", stream); k_bwd_prep<<<grid, eb, (size_t)eb.y * NDBLK * 4, stream>>>(e0, e1, C, g->recv, g->send, D, R, xt, gS, XT, XTlo,
                                                                   GY, GYhi, GYlo); }
-      So2Operands fwd{XT, XTlo, m.so2_fwd_hi + so2off, m.so2_fwd_lo + so2off, nullptr, nullptr};
-      st = so2_product(m, n, fwd, Y, stream);
-      if (st != EMP_OK) return st;
-      So2Operands bwd{GYhi, GYlo, m.so2_bwd_hi + so2off, m.so2_bwd_lo + so2off, nullptr, nullptr};
-      st = so2_product(m, n, bwd, GXT, stream);
+      So2Part parts[2] = {{am_xt.get(n), &m.bmaps_fwd[t], Y}, {am_gy.get(n), &m.bmaps_bwd[t], GXT}};
+      st = so2_product(m, n, parts, 2, counter, stream);
       if (st != EMP_OK) return st;
       const size_t smem = (size_t)eb.y * NDBLK * 4 + (size_t)eb.y * 2 * (C / 32) * 4;
       { Scope sc_("bwd_edge", stream); k_bwd_edge<<<grid, eb, smem, stream>>>(e0, e1, C, t > 0, g->send, g->vec, D, R, xt, Y, GY, GXT, XT, gR, g_r); }
@@ -588,17 +611,19 @@ int mp_so2_mix(const void* model, int32_t layer, int32_t transpose, int64_t M, c
   const Model& m = *static_cast<const Model*>(model);
   if (layer < 0 || layer >= m.spec.n_layers) return EMP_ERR_ARG;
   const size_t n = (size_t)M * 16 * m.spec.C;
-  if (ws_bytes < 2 * n * 4) return EMP_ERR_WORKSPACE;
+  if (ws_bytes < 2 * n * 4 + 256) return EMP_ERR_WORKSPACE;
   if (M == 0) return EMP_OK;
   int st = check_device();
   if (st != EMP_OK) return st;
   float* hi = static_cast<float*>(ws);
   float* lo = hi + n;
+  int* counter = reinterpret_cast<int*>(lo + n);
   split(X, hi, lo, n, stream);
-  const size_t off = (size_t)layer * m.so2_stride();
-  So2Operands op{hi, lo, (transpose ? m.so2_bwd_hi : m.so2_fwd_hi) + off, (transpose ? m.so2_bwd_lo : m.so2_fwd_lo) + off,
-                 nullptr, nullptr};
-  return so2_product(m, M, op, Y, stream);
+  So2AMaps am;
+  st = so2_make_amaps(&am, m.spec.C, M, hi, lo);
+  if (st != EMP_OK) return st;
+  So2Part part{&am, transpose ? &m.bmaps_bwd[layer] : &m.bmaps_fwd[layer], Y};
+  return so2_product(m, M, &part, 1, counter, stream);
 }
 
 // ------------------------------------------------------------------ radial chain

@@ -5,6 +5,7 @@
 #include <vector>
 #include <cstring>
 #include "emp_common.cuh"
+#include "so2_tc.cuh"
 
 namespace emp {
 
@@ -28,6 +29,7 @@ struct Model {
   float* ro_w;                  // [Hro]
   void* base;
   int device;
+  std::vector<So2BMaps> bmaps_fwd, bmaps_bwd;   // tensor maps of each layer's stacked blocks
 
   size_t rad_stride() const { return (size_t)H * 8 + (size_t)H * H + (size_t)4 * spec.C * H; }
   const float* W1(int t, int p) const { return rad + ((size_t)t * n_pairs + p) * rad_stride(); }

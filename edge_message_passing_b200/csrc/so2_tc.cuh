@@ -3,17 +3,21 @@
 // in strict FP32 with TF32 off ("first-order SO(2) input-gradient path",
 // "Primary capacity": strict level2 mixing FP32, TF32/AMP off), so each operand
 // is split a = hi + lo with hi = RN_tf32(a), lo = RN_tf32(a - hi), and
-//   Y = A_hi B_hi^T + A_hi B_lo^T + A_lo B_hi^T   (FP32 accumulation in TMEM).
+//   Y = A_lo B_hi^T + A_hi B_lo^T + A_hi B_hi^T   (FP32 accumulation in TMEM).
 //
-// For block b (= |m|) of a cohort:  Y[:, cols_b] = X[:, cols_b] @ B_b^T with
-// B_b the (K_b x K_b) stacked weight stored [n][k] (K-major), K_b = blk_width(b) C.
+// A launch is a group of sub-problems that share the row count M (one cohort):
+//   out_s[:, col_s : col_s + K_s] = A_{a(s)}[:, col_s : col_s + K_s] @ B_s^T,
+// B_s a (K_s x K_s) matrix stored [n][k] (K-major).  The forward of a layer is
+// the 4 m-blocks of the cohort; the backward groups the 4 recomputed forward
+// blocks with the 4 transposed blocks (8 sub-problems, two A operands).
 //
-// One CTA computes a 128 x BN output tile of one block.  Warp 0 issues TMA
-// loads (128B-swizzled, 32 fp32 of K per row) into an ST-stage ring guarded by
-// mbarriers; warp 1 allocates TMEM and issues tcgen05.mma (one thread);
-// warps 2..5 read the accumulator back with tcgen05.ld and store FP32 rows.
-// Every mbarrier wait is bounded: on timeout the CTA records a device error,
-// drains what it issued and frees its TMEM.
+// Persistent kernel: one CTA per SM takes 128 x 256 output tiles from a shared
+// atomic counter (tiles ordered by decreasing K).  Warp 0 issues TMA loads (64-byte swizzle, 16 fp32 of K per row) into
+// a 4-stage ring; warp 1 issues tcgen05.mma (one thread) into one of two TMEM
+// accumulators (2 x 256 columns); warps 2..5 drain the other accumulator with
+// tcgen05.ld and store FP32 rows, so the epilogue of a tile overlaps the next
+// tile's MMAs.  Every mbarrier wait is bounded: on timeout the CTA records a
+// device error, stops, waits (bounded) for its own copies and MMAs and frees TMEM.
 #pragma once
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -23,20 +27,35 @@ namespace emp {
 namespace tc {
 
 constexpr int BM = 128;
-constexpr int BK = 32;                 // fp32 elements per 128-byte swizzled row
-constexpr int BN = 128;
-constexpr int ST = 3;
+constexpr int BN = 256;
+constexpr int BK = 16;                 // fp32 elements per 64-byte swizzled row
+constexpr int ST = 4;
 constexpr int THREADS = 192;
+constexpr int MAXSUB = 8;
+constexpr int TMEM_COLS = 512;         // two 128 x 256 fp32 accumulators
 constexpr long long TIMEOUT_CYCLES = 4000000000ll;   // ~2 s at 1.9 GHz
 
-constexpr int A_BYTES = BM * BK * 4;   // 16 KB
+constexpr int A_BYTES = BM * BK * 4;   // 8 KB
 constexpr int B_BYTES = BN * BK * 4;   // 16 KB
-constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;
-constexpr int SMEM_BYTES = ST * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;   // 48 KB
+constexpr int SMEM_BYTES = ST * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers, tile ring*/;
+
+struct Group {
+  int M, nsub, mtiles;
+  int a_idx[MAXSUB];    // which A operand pair (0 or 1)
+  int b_idx[MAXSUB];    // which B map pair
+  int col[MAXSUB];      // first column (A and output) of the sub-problem
+  int K[MAXSUB];        // K = N of the sub-problem
+  int ntiles[MAXSUB];   // n-tiles per m-tile
+  int first[MAXSUB + 1];// first tile index of each sub-problem (sub-problems ordered by decreasing K)
+  int ld;               // row pitch (elements) of A and of the outputs
+  float* out[MAXSUB];
+  int* counter;         // dynamic tile counter (zeroed by the host before the launch)
+};
 
 struct Maps {
-  CUtensorMap a_hi, a_lo;       // [M rows][16C cols]
-  CUtensorMap b_hi[4], b_lo[4]; // block b: [K_b rows][K_b cols]
+  CUtensorMap a_hi[2], a_lo[2];             // [M rows][ld cols]
+  CUtensorMap b_hi[MAXSUB], b_lo[MAXSUB];   // [K rows][K cols]
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -46,6 +65,9 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 }
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
@@ -77,10 +99,10 @@ __device__ __forceinline__ void tma_load(void* dst, const CUtensorMap* map, uint
       : "memory");
 }
 
-// shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart
+// shared-memory matrix descriptor: K-major, 64-byte swizzle, 8-row groups 512 B apart
 __device__ __forceinline__ uint64_t sdesc(uint32_t addr) {
-  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(512 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)4 << 61);
 }
 
 // instruction descriptor: D f32, A/B tf32, both K-major, M = 128, N = BN
@@ -116,123 +138,186 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// n-tile index -> (block b, first output column of the tile within the block)
-__device__ __forceinline__ void tile_of(int C, int y, int& b, int& n0) {
-  for (b = 0; b < 4; ++b) {
-    const int nt = (blk_width(b) * C + BN - 1) / BN;
-    if (y < nt) { n0 = y * BN; return; }
-    y -= nt;
-  }
-  b = -1;
-  n0 = 0;
+struct TileInfo {
+  int m0, sub, n0;
+};
+
+// tile t: sub-problem by prefix, then m-major within it (the n-tiles of one m-tile
+// are consecutive, so they share the A tile in L2)
+__device__ __forceinline__ TileInfo tile_info(const Group& g, int t) {
+  TileInfo ti;
+  int s = 0;
+  while (s < g.nsub - 1 && t >= g.first[s + 1]) ++s;
+  const int r = t - g.first[s];
+  ti.sub = s;
+  ti.m0 = (r / g.ntiles[s]) * BM;
+  ti.n0 = (r % g.ntiles[s]) * BN;
+  return ti;
 }
 
-__global__ void __launch_bounds__(THREADS, 1) k_so2_tc(int M, int C, const __grid_constant__ Maps maps,
-                                                       float* __restrict__ Y) {
+constexpr int TQ = 4;    // depth of the tile-index ring from the scheduler to the MMA and epilogue warps
+
+__global__ void __launch_bounds__(THREADS, 1) k_so2_tc(const __grid_constant__ Group g, const __grid_constant__ Maps maps,
+                                                       int total_tiles) {
+  // Tiles are handed out dynamically (an atomic counter over tiles ordered by
+  // decreasing K): the TMA warp takes the next tile and passes its index to the
+  // MMA and epilogue warps through a TQ-deep ring; an index >= total ends a role.
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * STAGE_BYTES);
   uint64_t* empty = full + ST;
-  uint64_t* acc_bar = empty + ST;
-  uint64_t* drain_bar = acc_bar + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  uint64_t* acc_full = empty + ST;       // [2]
+  uint64_t* acc_empty = acc_full + 2;    // [2]
+  uint64_t* drain = acc_empty + 2;
+  uint64_t* tq_full = drain + 1;         // [TQ]
+  uint64_t* tq_empty = tq_full + TQ;     // [TQ]
+  int* tq = reinterpret_cast<int*>(tq_empty + TQ);   // [TQ] tile indices
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tq + TQ);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int* issued = abort_flag + 1;          // k-chunks whose loads were issued
+  int* consumed = issued + 1;            // k-chunks whose full barrier completed
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int b, n0;
-  tile_of(C, blockIdx.y, b, n0);
-  if (b < 0) return;
-  const int K = blk_width(b) * C, N = K;
-  const int m0 = blockIdx.x * BM;
-  const int col0 = blk_off(b) * C;      // column offset of the block in the 16C-wide rows
-  const int nk = K / BK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_bar, 1);
-    mbar_init(drain_bar, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    mbar_init(drain, 1);
+    for (int j = 0; j < TQ; ++j) {
+      mbar_init(&tq_full[j], 1);
+      mbar_init(&tq_empty[j], 5);        // the MMA thread and one thread per epilogue warp
+    }
     *abort_flag = 0;
+    *issued = 0;
+    *consumed = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"((uint32_t)BN));
+                 "r"((uint32_t)TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   fence_before();
   __syncthreads();
   fence_after();
   const uint32_t tmem = *tmem_slot;
+  volatile int* vabort = abort_flag;
 
   if (warp == 0 && lane == 0) {
-    // ---------------------------------------------------------------- producer
-    for (int kc = 0; kc < nk; ++kc) {
-      const int s = kc % ST;
-      if (kc >= ST && !mbar_wait(&empty[s], ((kc / ST) - 1) & 1)) { atomicExch(abort_flag, 1); break; }
-      if (*(volatile int*)abort_flag) break;
-      unsigned char* st = smem + s * STAGE_BYTES;
-      mbar_expect_tx(&full[s], STAGE_BYTES);
-      tma_load(st, &maps.a_hi, &full[s], col0 + kc * BK, m0);
-      tma_load(st + A_BYTES, &maps.a_lo, &full[s], col0 + kc * BK, m0);
-      tma_load(st + 2 * A_BYTES, &maps.b_hi[b], &full[s], kc * BK, n0);
-      tma_load(st + 2 * A_BYTES + B_BYTES, &maps.b_lo[b], &full[s], kc * BK, n0);
+    // ---------------------------------------------------------------- scheduler + TMA producer
+    int it = 0;
+    for (int j = 0;; ++j) {
+      const int slot = j % TQ;
+      if (j >= TQ && !mbar_wait(&tq_empty[slot], ((j / TQ) - 1) & 1)) { *vabort = 1; break; }
+      const int t = *vabort ? total_tiles : atomicAdd(g.counter, 1);
+      tq[slot] = t;
+      mbar_arrive(&tq_full[slot]);
+      if (t >= total_tiles) break;
+      const TileInfo ti = tile_info(g, t);
+      const int a = g.a_idx[ti.sub], b = g.b_idx[ti.sub];
+      const int nk = g.K[ti.sub] / BK;
+      for (int kc = 0; kc < nk; ++kc, ++it) {
+        const int s = it % ST;
+        if (it >= ST && !mbar_wait(&empty[s], ((it / ST) - 1) & 1)) { *vabort = 1; break; }
+        if (*vabort) break;
+        unsigned char* st = smem + s * STAGE_BYTES;
+        mbar_expect_tx(&full[s], STAGE_BYTES);
+        tma_load(st, &maps.a_hi[a], &full[s], g.col[ti.sub] + kc * BK, ti.m0);
+        tma_load(st + A_BYTES, &maps.a_lo[a], &full[s], g.col[ti.sub] + kc * BK, ti.m0);
+        tma_load(st + 2 * A_BYTES, &maps.b_hi[b], &full[s], kc * BK, ti.n0);
+        tma_load(st + 2 * A_BYTES + B_BYTES, &maps.b_lo[b], &full[s], kc * BK, ti.n0);
+        *issued = it + 1;
+      }
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------------- MMA issuer
+    int it = 0;
     bool ok = true;
-    for (int kc = 0; kc < nk; ++kc) {
-      const int s = kc % ST;
-      if (!mbar_wait(&full[s], (kc / ST) & 1)) { ok = false; atomicExch(abort_flag, 1); break; }
+    for (int i = 0;; ++i) {
+      const int slot = i % TQ;
+      if (!mbar_wait(&tq_full[slot], (i / TQ) & 1)) { ok = false; break; }
+      const int t = tq[slot];
+      mbar_arrive(&tq_empty[slot]);
+      if (t >= total_tiles) break;
+      const TileInfo ti = tile_info(g, t);
+      const int nk = g.K[ti.sub] / BK;
+      const int buf = i & 1;
+      if (i >= 2 && !mbar_wait(&acc_empty[buf], ((i >> 1) - 1) & 1)) { ok = false; break; }
       fence_after();
-      const uint32_t a_hi = smem_u32(smem + s * STAGE_BYTES);
-      const uint32_t a_lo = a_hi + A_BYTES;
-      const uint32_t b_hi = a_hi + 2 * A_BYTES;
-      const uint32_t b_lo = b_hi + B_BYTES;
+      const uint32_t d = tmem + (uint32_t)(buf * BN);
+      for (int kc = 0; kc < nk; ++kc, ++it) {
+        const int s = it % ST;
+        if (!mbar_wait(&full[s], (it / ST) & 1)) { ok = false; break; }
+        *consumed = it + 1;
+        fence_after();
+        const uint32_t a_hi = smem_u32(smem + s * STAGE_BYTES);
+        const uint32_t a_lo = a_hi + A_BYTES;
+        const uint32_t b_hi = a_hi + 2 * A_BYTES;
+        const uint32_t b_lo = b_hi + B_BYTES;
 #pragma unroll
-      for (int kk = 0; kk < BK / 8; ++kk) {
-        const uint32_t off = kk * 32;   // 8 fp32 of K = 32 bytes inside the swizzled row
-        const uint32_t acc = (kc | kk) ? 1u : 0u;
-        mma_tf32(tmem, sdesc(a_lo + off), sdesc(b_hi + off), acc);
-        mma_tf32(tmem, sdesc(a_hi + off), sdesc(b_lo + off), 1u);
-        mma_tf32(tmem, sdesc(a_hi + off), sdesc(b_hi + off), 1u);
+        for (int kk = 0; kk < BK / 8; ++kk) {
+          const uint32_t off = kk * 32;   // 8 fp32 of K = 32 bytes inside the swizzled row
+          mma_tf32(d, sdesc(a_lo + off), sdesc(b_hi + off), (kc | kk) ? 1u : 0u);
+          mma_tf32(d, sdesc(a_hi + off), sdesc(b_lo + off), 1u);
+          mma_tf32(d, sdesc(a_hi + off), sdesc(b_hi + off), 1u);
+        }
+        mma_commit(&empty[s]);
       }
-      mma_commit(&empty[s]);
+      if (!ok) break;
+      mma_commit(&acc_full[buf]);
     }
-    mma_commit(ok ? acc_bar : drain_bar);
-    if (!ok) mbar_wait(drain_bar, 0);     // let issued MMAs finish before TMEM is freed
+    if (!ok) *vabort = 1;
+    mma_commit(drain);                  // completes once every MMA this thread issued is done
+    mbar_wait(drain, 0);
   } else if (warp >= 2) {
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;               // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;
-    const bool ok = mbar_wait(acc_bar, 0);
-    fence_after();
-    if (ok) {
-      const int m = m0 + row;
-      float* yrow = Y + (size_t)m * 16 * C + col0 + n0;
+    for (int i = 0;; ++i) {
+      const int slot = i % TQ;
+      if (!mbar_wait(&tq_full[slot], (i / TQ) & 1)) { *vabort = 1; break; }
+      const int t = tq[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tq_empty[slot]);
+      if (t >= total_tiles) break;
+      const TileInfo ti = tile_info(g, t);
+      const int buf = i & 1;
+      if (!mbar_wait(&acc_full[buf], (i >> 1) & 1)) { *vabort = 1; break; }
+      fence_after();
+      const int m = ti.m0 + row;
+      const int N = g.K[ti.sub];
+      float* orow = g.out[ti.sub] + (size_t)m * g.ld + g.col[ti.sub] + ti.n0;
 #pragma unroll 1
       for (int cc = 0; cc < BN; cc += 32) {
         float v[32];
-        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)cc, v);
-        if (m < M && n0 + cc < N) {
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + cc), v);
+        if (m < g.M && ti.n0 + cc < N) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(yrow + cc + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(orow + cc + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
         }
       }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
   }
   fence_before();
   __syncthreads();
-  if (threadIdx.x == 0 && *abort_flag) {
-    // wait (bounded) for loads that may still be landing in shared memory
-    for (int s = 0; s < ST; ++s) mbar_try_wait(&full[s], 0);
+  if (threadIdx.x == 0 && *vabort) {
+    // let loads still in flight land before the shared memory is released
+    for (int it = *consumed; it < *issued; ++it) mbar_wait(&full[it % ST], (it / ST) & 1);
   }
+  __syncthreads();
   if (warp == 1) {
     fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)BN));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)TMEM_COLS));
   }
 }
 
@@ -258,8 +343,19 @@ inline bool make_map(CUtensorMap* m, const float* base, uint64_t cols, uint64_t 
   cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
 }
 
 }  // namespace tc
@@ -271,27 +367,78 @@ inline int so2_tc_init() {
   return EMP_OK;
 }
 
-inline int so2_tc_tiles(int C) {
-  int n = 0;
-  for (int b = 0; b < 4; ++b) n += (blk_width(b) * C + tc::BN - 1) / tc::BN;
-  return n;
-}
+// Tensor maps of one operand set of the SO(2) mixing: A (hi, lo) rows [M][16C] and a
+// layer's stacked 4-block weights (hi, lo).  Built once (weights: at model
+// creation; activations: once per call and cohort size) and reused by every launch.
+struct So2BMaps {
+  CUtensorMap hi[4], lo[4];
+};
+struct So2AMaps {
+  CUtensorMap hi, lo;
+};
 
-// Y (M x 16C) = per-block products of A (M x 16C) with the layer's stacked weights (split hi/lo)
-inline int so2_tc(long long M, int C, const float* A_hi, const float* A_lo, const float* B_hi, const float* B_lo,
-                  float* Y, cudaStream_t s) {
-  if (M <= 0) return EMP_OK;
-  tc::Maps maps;
-  if (!tc::make_map(&maps.a_hi, A_hi, 16 * C, M, 16 * C, tc::BM)) return EMP_ERR_CUDA;
-  if (!tc::make_map(&maps.a_lo, A_lo, 16 * C, M, 16 * C, tc::BM)) return EMP_ERR_CUDA;
+inline int so2_make_bmaps(So2BMaps* m, int C, const float* b_hi, const float* b_lo) {
   for (int b = 0; b < 4; ++b) {
     const uint64_t K = (uint64_t)blk_width(b) * C;
     const size_t off = (size_t)wblk_off(b) * C * C;
-    if (!tc::make_map(&maps.b_hi[b], B_hi + off, K, K, K, tc::BN)) return EMP_ERR_CUDA;
-    if (!tc::make_map(&maps.b_lo[b], B_lo + off, K, K, K, tc::BN)) return EMP_ERR_CUDA;
+    if (!tc::make_map(&m->hi[b], b_hi + off, K, K, K, tc::BN)) return EMP_ERR_CUDA;
+    if (!tc::make_map(&m->lo[b], b_lo + off, K, K, K, tc::BN)) return EMP_ERR_CUDA;
   }
-  dim3 grid((unsigned)((M + tc::BM - 1) / tc::BM), so2_tc_tiles(C));
-  tc::k_so2_tc<<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>((int)M, C, maps, Y);
+  return EMP_OK;
+}
+
+inline int so2_make_amaps(So2AMaps* m, int C, long long M, const float* a_hi, const float* a_lo) {
+  if (!tc::make_map(&m->hi, a_hi, 16 * C, M, 16 * C, tc::BM)) return EMP_ERR_CUDA;
+  if (!tc::make_map(&m->lo, a_lo, 16 * C, M, 16 * C, tc::BM)) return EMP_ERR_CUDA;
+  return EMP_OK;
+}
+
+struct So2Part {
+  const So2AMaps* a;
+  const So2BMaps* b;
+  float* out;
+};
+
+// Grouped launch over one or two operand sets sharing M (forward: 1; backward: 2).
+// counter: one device int of scratch, zeroed here before the launch.
+inline int so2_tc(long long M, int C, const So2Part* parts, int nparts, int* counter, cudaStream_t s) {
+  if (M <= 0) return EMP_OK;
+  if (nparts < 1 || nparts > 2) return EMP_ERR_ARG;
+  tc::Group g{};
+  tc::Maps maps;
+  g.M = (int)M;
+  g.ld = 16 * C;
+  g.nsub = 4 * nparts;
+  g.mtiles = (int)((M + tc::BM - 1) / tc::BM);
+  g.counter = counter;
+  // sub-problems ordered by decreasing K (block 1, then 0, 2, then 3) so the longest tiles go first
+  const int order[4] = {1, 0, 2, 3};
+  int sidx = 0, first = 0;
+  for (int q = 0; q < 4; ++q) {
+    const int b = order[q];
+    for (int p = 0; p < nparts; ++p, ++sidx) {
+      const int K = blk_width(b) * C;
+      maps.b_hi[sidx] = parts[p].b->hi[b];
+      maps.b_lo[sidx] = parts[p].b->lo[b];
+      g.a_idx[sidx] = p;
+      g.b_idx[sidx] = sidx;
+      g.col[sidx] = blk_off(b) * C;
+      g.K[sidx] = K;
+      g.ntiles[sidx] = (K + tc::BN - 1) / tc::BN;
+      g.out[sidx] = parts[p].out;
+      g.first[sidx] = first;
+      first += g.ntiles[sidx] * g.mtiles;
+    }
+  }
+  g.first[g.nsub] = first;
+  for (int p = 0; p < nparts; ++p) {
+    maps.a_hi[p] = parts[p].a->hi;
+    maps.a_lo[p] = parts[p].a->lo;
+  }
+  const int total = first;
+  if (cudaMemsetAsync(counter, 0, sizeof(int), s) != cudaSuccess) return EMP_ERR_CUDA;
+  const int grid = std::min(total, tc::num_sms());
+  tc::k_so2_tc<<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(g, maps, total);
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
 

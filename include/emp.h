@@ -145,7 +145,7 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
  * column layout [m=0 (l=0..3) | +1 (l=1..3) | -1 | +2 | -2 | +3 | -3], each
  * entry C channels.  transpose = 0: Y_b = X_b B_b^T (forward, y+ = Wr x+ - Wi x-,
  * y- = Wi x+ + Wr x-, y0 = W0 x0); transpose = 1: the adjoint map.
- * Workspace >= 2 * M * 16 * C floats (the TF32 split of X). */
+ * Workspace >= 2 * M * 16 * C floats (the TF32 split of X) + 256 bytes. */
 int mp_so2_mix(const void* model, int32_t layer, int32_t transpose, int64_t M, const float* X, float* Y,
                void* ws, size_t ws_bytes, cudaStream_t stream);
 
