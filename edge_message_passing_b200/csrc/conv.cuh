@@ -84,17 +84,17 @@ __device__ __forceinline__ int pair_of(int a, int b, int S) {
 }
 
 struct RadialArgs {
-  const float* rad;        // model radial weights (per layer, per pair)
+  const float* rad;        // model radial weights (per layer, per pair): W1 [64][8], W2 [64][64], W3 [4C][64]
   size_t layer_off;        // float offset of layer t's first pair
   size_t pair_stride;      // floats per pair
   int C, n_species, pair_radial;
   float rc;
 };
 
-constexpr int RT = 64;      // edges per radial tile
+constexpr int RT = 64;      // rows per radial tile
 constexpr int RAD_THREADS = 256;
 
-// shared-memory tile of the radial network
+// shared-memory tile of the radial network's hidden layers
 struct RadialSmem {
   float e[RT][8];
   float de[RT][8];
@@ -102,13 +102,13 @@ struct RadialSmem {
   float h1[RT][65];
   float z2[RT][64];
   float h2[RT][65];
-  float w[64][132];     // a 64 x 128 chunk of W3^T (forward) or W3 (backward, [o][k] read)
-  float g[RT][132];     // backward: a 64 x 128 chunk of dE/dR
+  float g[RT][65];      // backward: dE/dh2 rows
   int pair[RT];
+  int edge[RT];
   unsigned mask;
 };
 
-// basis, hidden layers (for edges of pair p) -- all 256 threads participate
+// hidden layers (for the tile's rows, with pair p's weights) -- all 256 threads participate
 __device__ void radial_hidden(RadialSmem& s, const float* __restrict__ W1, const float* __restrict__ W2) {
   const int t = threadIdx.x;
   // layer 1: z1[e][j] = sum_n W1[j][n] e[n]
@@ -121,7 +121,7 @@ __device__ void radial_hidden(RadialSmem& s, const float* __restrict__ W1, const
     s.h1[e][j] = silu_f(acc);
   }
   __syncthreads();
-  // layer 2: thread owns output j and 16 edges
+  // layer 2: thread owns output j and 16 rows
   {
     const int j = t & 63, eg = (t >> 6) * 16;
     float acc[16];
@@ -141,22 +141,25 @@ __device__ void radial_hidden(RadialSmem& s, const float* __restrict__ W1, const
   __syncthreads();
 }
 
-__device__ void radial_tile_setup(RadialSmem& s, long long e0, long long E, const float* __restrict__ dist,
-                                  const int* __restrict__ recv, const int* __restrict__ send,
-                                  const int* __restrict__ species, const RadialArgs& a) {
+// rows r0 .. r0+63 of the (pair-sorted, or edge-ordered when perm is null) row list
+__device__ void radial_tile_setup(RadialSmem& s, long long r0, long long E, const int* __restrict__ perm,
+                                  const float* __restrict__ dist, const int* __restrict__ recv,
+                                  const int* __restrict__ send, const int* __restrict__ species, const RadialArgs& a) {
   const int t = threadIdx.x;
   if (t == 0) s.mask = 0u;
   __syncthreads();
   if (t < RT) {
-    const long long e = e0 + t;
-    int p = 0;
+    const long long r = r0 + t;
+    int p = 0, e = -1;
     float d = 1.f;
-    if (e < E) {
+    if (r < E) {
+      e = perm ? perm[r] : (int)r;
       d = dist[e];
       if (a.pair_radial) p = pair_of(species[recv[e]], species[send[e]], a.n_species);
       atomicOr(&s.mask, 1u << p);
     }
-    s.pair[t] = e < E ? p : -1;
+    s.pair[t] = r < E ? p : -1;
+    s.edge[t] = e;
     float ev[8], dv[8];
     bessel8(d, a.rc, ev, dv);
 #pragma unroll
@@ -165,112 +168,68 @@ __device__ void radial_tile_setup(RadialSmem& s, long long e0, long long E, cons
   __syncthreads();
 }
 
-// R [E][4C] for layer t
-__global__ void __launch_bounds__(RAD_THREADS) k_radial_fwd(long long E, const float* __restrict__ dist,
-                                                           const int* __restrict__ recv, const int* __restrict__ send,
-                                                           const int* __restrict__ species, RadialArgs a,
-                                                           float* __restrict__ R) {
+// h2 rows (3xTF32 split) of the radial network for every row: the input of the
+// tensor-core head R = h2 W3^T
+__global__ void __launch_bounds__(RAD_THREADS) k_radial_h2(long long E, const int* __restrict__ perm,
+                                                          const float* __restrict__ dist, const int* __restrict__ recv,
+                                                          const int* __restrict__ send, const int* __restrict__ species,
+                                                          RadialArgs a, float* __restrict__ h2_hi,
+                                                          float* __restrict__ h2_lo) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   RadialSmem& s = *reinterpret_cast<RadialSmem*>(smem_raw);
-  const long long e0 = (long long)blockIdx.x * RT;
-  radial_tile_setup(s, e0, E, dist, recv, send, species, a);
-  const int t = threadIdx.x, ty = t >> 4, tx = t & 15;
-  const int CO = 4 * a.C;
+  const long long r0 = (long long)blockIdx.x * RT;
+  radial_tile_setup(s, r0, E, perm, dist, recv, send, species, a);
+  const int t = threadIdx.x;
   unsigned mask = s.mask;
   while (mask) {
     const int p = __ffs(mask) - 1;
     mask &= mask - 1;
     const float* W1 = a.rad + a.layer_off + (size_t)p * a.pair_stride;
-    const float* W2 = W1 + 64 * 8;
-    const float* W3 = W2 + 64 * 64;
-    radial_hidden(s, W1, W2);
-    for (int oc = 0; oc < CO; oc += 128) {
-      // W3 rows oc..oc+127 -> w[k][o]
-      for (int idx = t; idx < 128 * 64; idx += RAD_THREADS) {
-        const int o = idx >> 6, k = idx & 63;
-        s.w[k][o] = __ldg(&W3[(size_t)(oc + o) * 64 + k]);
+    radial_hidden(s, W1, W1 + 64 * 8);
+    for (int idx = t; idx < RT * 64; idx += RAD_THREADS) {
+      const int el = idx >> 6, j = idx & 63;
+      if (s.pair[el] == p) {
+        const float v = s.h2[el][j], h = tf32_rna(v);
+        h2_hi[(size_t)(r0 + el) * 64 + j] = h;
+        h2_lo[(size_t)(r0 + el) * 64 + j] = tf32_rna(v - h);
       }
-      __syncthreads();
-      float acc[4][8];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-      for (int k = 0; k < 64; ++k) {
-        float av[4], bv[8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) av[i] = s.h2[ty * 4 + i][k];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) bv[j] = s.w[k][tx + 16 * j];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int el = ty * 4 + i;
-        if (s.pair[el] == p) {
-          float* out = R + (size_t)(e0 + el) * CO + oc;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) out[tx + 16 * j] = acc[i][j];
-        }
-      }
-      __syncthreads();
     }
+    __syncthreads();
   }
 }
 
-// dE/dd from dE/dR (gR [E][4C]); adds (dE/dd) rhat to g_r
-__global__ void __launch_bounds__(RAD_THREADS) k_radial_bwd(long long E, const float* __restrict__ dist,
-                                                           const float* __restrict__ vec,
-                                                           const int* __restrict__ recv, const int* __restrict__ send,
-                                                           const int* __restrict__ species, RadialArgs a,
-                                                           const float* __restrict__ gR, float* __restrict__ g_r) {
+// dE/dd from dE/dh2 (rows gh2 [E][64], the tensor-core product dE/dR W3); adds (dE/dd) rhat to g_r
+__global__ void __launch_bounds__(RAD_THREADS) k_radial_bwd(long long E, const int* __restrict__ perm,
+                                                           const float* __restrict__ dist,
+                                                           const float* __restrict__ vec, const int* __restrict__ recv,
+                                                           const int* __restrict__ send, const int* __restrict__ species,
+                                                           RadialArgs a, const float* __restrict__ gh2,
+                                                           float* __restrict__ g_r) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   RadialSmem& s = *reinterpret_cast<RadialSmem*>(smem_raw);
-  const long long e0 = (long long)blockIdx.x * RT;
-  radial_tile_setup(s, e0, E, dist, recv, send, species, a);
+  const long long r0 = (long long)blockIdx.x * RT;
+  radial_tile_setup(s, r0, E, perm, dist, recv, send, species, a);
   const int t = threadIdx.x;
-  const int CO = 4 * a.C;
+  for (int idx = t; idx < RT * 64; idx += RAD_THREADS) {
+    const int el = idx >> 6, j = idx & 63;
+    s.g[el][j] = (r0 + el < E) ? gh2[(size_t)(r0 + el) * 64 + j] : 0.f;
+  }
   unsigned mask = s.mask;
   while (mask) {
     const int p = __ffs(mask) - 1;
     mask &= mask - 1;
     const float* W1 = a.rad + a.layer_off + (size_t)p * a.pair_stride;
     const float* W2 = W1 + 64 * 8;
-    const float* W3 = W2 + 64 * 64;
     radial_hidden(s, W1, W2);
-    // g_h2[e][k] = sum_o gR[e][o] W3[o][k]; thread owns k = t & 63 and 16 edges
-    const int k = t & 63, eg = (t >> 6) * 16;
-    float acc[16];
-#pragma unroll
-    for (int q = 0; q < 16; ++q) acc[q] = 0.f;
-    for (int oc = 0; oc < CO; oc += 128) {
-      for (int idx = t; idx < 128 * 64; idx += RAD_THREADS) {
-        const int o = idx >> 6, kk = idx & 63;
-        s.w[kk][o] = __ldg(&W3[(size_t)(oc + o) * 64 + kk]);
-      }
-      for (int idx = t; idx < RT * 128; idx += RAD_THREADS) {
-        const int el = idx >> 7, o = idx & 127;
-        const long long e = e0 + el;
-        s.g[el][o] = (e < E) ? gR[(size_t)e * CO + oc + o] : 0.f;
-      }
-      __syncthreads();
-      for (int o = 0; o < 128; ++o) {
-        const float w = s.w[k][o];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) acc[q] = fmaf(s.g[eg + q][o], w, acc[q]);
-      }
-      __syncthreads();
+    // g_z2 = g_h2 dsilu(z2) -> h2
+    for (int idx = t; idx < RT * 64; idx += RAD_THREADS) {
+      const int el = idx >> 6, j = idx & 63;
+      s.h2[el][j] = s.g[el][j] * dsilu_f(s.z2[el][j]);
     }
-    // g_z2 -> reuse h2 as storage
-#pragma unroll
-    for (int q = 0; q < 16; ++q) s.h2[eg + q][k] = acc[q] * dsilu_f(s.z2[eg + q][k]);
     __syncthreads();
-    // g_h1[e][j] = sum_k g_z2[e][k] W2[k][j]; g_z1 = g_h1 dsilu(z1) -> reuse h1
+    // g_h1[e][j] = sum_k g_z2[e][k] W2[k][j]; g_z1 = g_h1 dsilu(z1) -> h1
     {
-      const int j = t & 63;
+      const int j = t & 63, eg = (t >> 6) * 16;
       float a2[16];
 #pragma unroll
       for (int q = 0; q < 16; ++q) a2[q] = 0.f;
@@ -285,32 +244,78 @@ __global__ void __launch_bounds__(RAD_THREADS) k_radial_bwd(long long E, const f
     }
     __syncthreads();
     // dE/dd = sum_n (sum_j g_z1[j] W1[j][n]) de_n/dd
-    if (t < RT) {
-      const int el = t;
-      const long long e = e0 + el;
-      if (e < E && s.pair[el] == p) {
-        float dEdd = 0.f;
+    if (t < RT && s.pair[t] == p) {
+      const int e = s.edge[t];
+      float dEdd = 0.f;
 #pragma unroll
-        for (int n = 0; n < 8; ++n) {
-          float ge = 0.f;
-          for (int j = 0; j < 64; ++j) ge = fmaf(s.h1[el][j], __ldg(&W1[j * 8 + n]), ge);
-          dEdd = fmaf(ge, s.de[el][n], dEdd);
-        }
-        const float d = dist[e];
-        const float inv = 1.f / d;
-        g_r[3 * e + 0] += dEdd * vec[3 * e + 0] * inv;
-        g_r[3 * e + 1] += dEdd * vec[3 * e + 1] * inv;
-        g_r[3 * e + 2] += dEdd * vec[3 * e + 2] * inv;
+      for (int n = 0; n < 8; ++n) {
+        float ge = 0.f;
+        for (int j = 0; j < 64; ++j) ge = fmaf(s.h1[t][j], __ldg(&W1[j * 8 + n]), ge);
+        dEdd = fmaf(ge, s.de[t][n], dEdd);
       }
+      const float inv = 1.f / dist[e];
+      g_r[3 * e + 0] += dEdd * vec[3 * e + 0] * inv;
+      g_r[3 * e + 1] += dEdd * vec[3 * e + 1] * inv;
+      g_r[3 * e + 2] += dEdd * vec[3 * e + 2] * inv;
     }
     __syncthreads();
+  }
+}
+
+// Stable, deterministic counting sort of the edges by species pair (one block of
+// 1024 threads; thread t owns a contiguous run of edges).  perm[k] = edge at row k,
+// inv[e] = row of edge e, off[p] = first row of pair p (off[n_pairs] = E).
+constexpr int PS_THREADS = 1024;
+__global__ void __launch_bounds__(PS_THREADS) k_pair_sort(long long E, int n_species, int n_pairs,
+                                                         const int* __restrict__ recv, const int* __restrict__ send,
+                                                         const int* __restrict__ species, int* __restrict__ perm,
+                                                         int* __restrict__ inv, int* __restrict__ off) {
+  extern __shared__ int cnt[];          // [n_pairs][PS_THREADS]
+  __shared__ int wsum[32];
+  __shared__ int ptot[33];
+  const int t = threadIdx.x;
+  const long long per = (E + PS_THREADS - 1) / PS_THREADS;
+  const long long b = t * per, en = min(E, b + per);
+  for (int p = 0; p < n_pairs; ++p) cnt[p * PS_THREADS + t] = 0;
+  for (long long e = b; e < en; ++e) ++cnt[pair_of(species[recv[e]], species[send[e]], n_species) * PS_THREADS + t];
+  __syncthreads();
+  const int lane = t & 31, w = t >> 5;
+  for (int p = 0; p < n_pairs; ++p) {
+    const int c = cnt[p * PS_THREADS + t];
+    int v = c;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    if (lane == 31) wsum[w] = v;
+    __syncthreads();
+    if (t == 0) {
+      int acc = 0;
+      for (int q = 0; q < 32; ++q) { const int y = wsum[q]; wsum[q] = acc; acc += y; }
+      ptot[p] = acc;
+    }
+    __syncthreads();
+    cnt[p * PS_THREADS + t] = wsum[w] + v - c;     // exclusive prefix within pair p
+    __syncthreads();
+  }
+  if (t == 0) {
+    int acc = 0;
+    for (int p = 0; p < n_pairs; ++p) { const int y = ptot[p]; ptot[p] = acc; off[p] = acc; acc += y; }
+    off[n_pairs] = acc;
+  }
+  __syncthreads();
+  for (long long e = b; e < en; ++e) {
+    const int p = pair_of(species[recv[e]], species[send[e]], n_species);
+    const int pos = ptot[p] + cnt[p * PS_THREADS + t]++;
+    perm[pos] = (int)e;
+    inv[e] = pos;
   }
 }
 
 // ------------------------------------------------------------------ rotate in
 // XT[e - e0][col(k) C + c] = R_e[l(k)][c] * (D_e x_send)[k][c]  (edge frame, m-major)
 __global__ void k_rotate_in(long long e0, long long e1, int C, const int* __restrict__ send,
-                            const float* __restrict__ D, const float* __restrict__ R,
+                            const int* __restrict__ rrow, const float* __restrict__ D, const float* __restrict__ R,
                             const float* __restrict__ x, float* __restrict__ XT, float* __restrict__ XTlo) {
   extern __shared__ __align__(16) float sD[];           // [EPB][84]
   const int c = threadIdx.x, row = threadIdx.y, EPB = blockDim.y;
@@ -330,8 +335,9 @@ __global__ void k_rotate_in(long long e0, long long e1, int C, const int* __rest
     for (int k = 0; k < 16; ++k) xv[k] = x[((size_t)j * 16 + k) * C + c];
     rotate16<false>(sD + row * NDBLK, xv, u);
     float Rv[4];
+    const size_t rr = rrow ? (size_t)rrow[e] : (size_t)e;
 #pragma unroll
-    for (int l = 0; l < 4; ++l) Rv[l] = R[(size_t)e * 4 * C + l * C + c];
+    for (int l = 0; l < 4; ++l) Rv[l] = R[rr * 4 * C + l * C + c];
     float* out = XT + (size_t)el * 16 * C;
     float* olo = XTlo + (size_t)el * 16 * C;
 #pragma unroll
@@ -345,14 +351,19 @@ __global__ void k_rotate_in(long long e0, long long e1, int C, const int* __rest
 
 // ------------------------------------------------------------------ rotate back + receiver sums
 // S[i] (+)= sum over the cohort's edges of receiver i of D_e^T y_e.
-// One block per (receiver, 64-channel group): RB_ROWS rows take the receiver's
+// One block per (receiver, 32-channel group): RB_ROWS rows take the receiver's
 // edges round-robin (row r: edges b + r, b + r + RB_ROWS, ...), each row sums
 // its edges in order, then the rows are added in row order onto the running
 // sum carried from earlier cohorts.  The order is fixed, so results are
 // reproducible; a receiver whose edges started in an earlier cohort continues
 // its running sum.
-constexpr int RB_ROWS = 8;
-constexpr int RB_CG = 64;
+constexpr int RB_ROWS = 16;
+constexpr int RB_CG = 32;
+constexpr int RB_CHUNK = 128;     // edges whose Wigner-D blocks are staged at once
+struct RbSmem {
+  float sD[RB_CHUNK * NDBLK];
+  float part[RB_ROWS][16][RB_CG];
+};
 
 __global__ void __launch_bounds__(RB_CG * RB_ROWS) k_rotate_back_scatter(long long e0, long long e1, int C,
                                                                          const int* __restrict__ recv,
@@ -360,10 +371,12 @@ __global__ void __launch_bounds__(RB_CG * RB_ROWS) k_rotate_back_scatter(long lo
                                                                          const float* __restrict__ D,
                                                                          const float* __restrict__ Y,
                                                                          float* __restrict__ S) {
-  __shared__ __align__(16) float sD[RB_ROWS][NDBLK];
-  __shared__ float part[RB_ROWS][16][RB_CG];
+  extern __shared__ __align__(16) unsigned char rb_smem[];
+  RbSmem& sm = *reinterpret_cast<RbSmem*>(rb_smem);
+  float* sD = sm.sD;
+  auto& part = sm.part;
   const int cg = min(C, RB_CG);
-  const int tx = threadIdx.x, row = threadIdx.y;
+  const int tx = threadIdx.x, row = threadIdx.y, tid = row * cg + tx, nthr = cg * RB_ROWS;
   const int c = blockIdx.y * cg + tx;
   const int first = recv[e0], last = recv[e1 - 1];
   for (int i = first + blockIdx.x; i <= last; i += gridDim.x) {
@@ -372,27 +385,31 @@ __global__ void __launch_bounds__(RB_CG * RB_ROWS) k_rotate_back_scatter(long lo
     float acc[16];
 #pragma unroll
     for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-    for (long long base = b; base < en; base += RB_ROWS) {
-      const long long e = base + row;
-      const bool ok = e < en;
+    for (long long cb = b; cb < en; cb += RB_CHUNK) {
+      const int nch = (int)min((long long)RB_CHUNK, en - cb);
       __syncthreads();
-      if (ok)
-        for (int k = tx; k < NDBLK; k += cg) sD[row][k] = D[(size_t)e * NDBLK + k];
+      {
+        const float4* src = reinterpret_cast<const float4*>(D + (size_t)cb * NDBLK);
+        float4* dst = reinterpret_cast<float4*>(sD);
+        for (int q = tid; q < nch * (NDBLK / 4); q += nthr) dst[q] = src[q];
+      }
       __syncthreads();
-      if (ok) {
-        const float* y = Y + (size_t)(e - e0) * 16 * C;
+#pragma unroll 2
+      for (int k = row; k < nch; k += RB_ROWS) {
+        const float* y = Y + (size_t)(cb + k - e0) * 16 * C;
         float yv[16], m[16];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) yv[k] = y[col_of_k(k) * C + c];
-        rotate16<true>(sD[row], yv, m);
+        for (int q = 0; q < 16; ++q) yv[q] = y[col_of_k(q) * C + c];
+        rotate16<true>(sD + k * NDBLK, yv, m);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) acc[k] += m[k];
+        for (int q = 0; q < 16; ++q) acc[q] += m[q];
       }
     }
 #pragma unroll
     for (int k = 0; k < 16; ++k) part[row][k][tx] = acc[k];
     __syncthreads();
-    for (int k = row; k < 16; k += RB_ROWS) {
+    if (row < 16) {
+      const int k = row;
       float s = carry ? S[((size_t)i * 16 + k) * C + c] : 0.f;
 #pragma unroll
       for (int r = 0; r < RB_ROWS; ++r) s += part[r][k][tx];
@@ -508,7 +525,8 @@ __global__ void k_gate_bwd(int N, int C, float inv_avg, int gated, const float* 
 
 // per edge: XT = R (.) D x_send (recomputed) and GY = D gS[recv] (edge-frame output gradient)
 __global__ void k_bwd_prep(long long e0, long long e1, int C, const int* __restrict__ recv,
-                           const int* __restrict__ send, const float* __restrict__ D, const float* __restrict__ R,
+                           const int* __restrict__ send, const int* __restrict__ rrow, const float* __restrict__ D,
+                           const float* __restrict__ R,
                            const float* __restrict__ x, const float* __restrict__ gS, float* __restrict__ XT,
                            float* __restrict__ XTlo, float* __restrict__ GY, float* __restrict__ GYhi,
                            float* __restrict__ GYlo) {
@@ -531,8 +549,9 @@ __global__ void k_bwd_prep(long long e0, long long e1, int C, const int* __restr
     for (int k = 0; k < 16; ++k) v[k] = x[((size_t)j * 16 + k) * C + c];
     rotate16<false>(Dr, v, u);
     float Rv[4];
+    const size_t rr = rrow ? (size_t)rrow[e] : (size_t)e;
 #pragma unroll
-    for (int l = 0; l < 4; ++l) Rv[l] = R[(size_t)e * 4 * C + l * C + c];
+    for (int l = 0; l < 4; ++l) Rv[l] = R[rr * 4 * C + l * C + c];
     const size_t ro = (size_t)el * 16 * C;
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
@@ -620,12 +639,13 @@ __device__ __forceinline__ void bwd_edge_degree(const float* __restrict__ Dr, co
 }
 
 __global__ void __launch_bounds__(256, 2) k_bwd_edge(long long e0, long long e1, int C, int need_gx,
-                                                     const int* __restrict__ send, const float* __restrict__ vec,
+                                                     const int* __restrict__ send, const int* __restrict__ rrow,
+                                                     const float* __restrict__ vec,
                                                      const float* __restrict__ D, const float* __restrict__ R,
                                                      const float* __restrict__ x, const float* __restrict__ Y,
                                                      const float* __restrict__ GY, const float* __restrict__ GXT,
-                                                     float* __restrict__ GXS, float* __restrict__ gR,
-                                                     float* __restrict__ g_r) {
+                                                     float* __restrict__ GXS, float* __restrict__ gR_hi,
+                                                     float* __restrict__ gR_lo, float* __restrict__ g_r) {
   extern __shared__ __align__(16) float smem[];
   const int c = threadIdx.x, row = threadIdx.y, EPB = blockDim.y;
   float* sD = smem;                                 // [EPB][84]
@@ -645,21 +665,27 @@ __global__ void __launch_bounds__(256, 2) k_bwd_edge(long long e0, long long e1,
       const float* Dr = sD + row * NDBLK;
       const size_t rowoff = (size_t)el * 16 * C;
       const float* xs = x + (size_t)send[e] * 16 * C + c;
-      const float* Rr = R + (size_t)e * 4 * C + c;
-      float* gRr = gR + (size_t)e * 4 * C + c;
+      const size_t rr = rrow ? (size_t)rrow[e] : (size_t)e;
+      const float* Rr = R + rr * 4 * C + c;
+      float* gHi = gR_hi + rr * 4 * C + c;
+      float* gLo = gR_lo + rr * 4 * C + c;
       const float* yr = Y + rowoff + c;
       const float* gyr = GY + rowoff + c;
       const float* gxr = GXT + rowoff + c;
       float* gsr = GXS + rowoff + c;
       float gr;
       bwd_edge_degree<0>(Dr, xs, yr, gyr, gxr, Rr[0], C, c, need_gx, gsr, gr, bx, by);
-      gRr[0] = gr;
+      gHi[0] = tf32_rna(gr);
+      gLo[0] = tf32_rna(gr - tf32_rna(gr));
       bwd_edge_degree<1>(Dr, xs, yr, gyr, gxr, Rr[C], C, c, need_gx, gsr, gr, bx, by);
-      gRr[C] = gr;
+      gHi[C] = tf32_rna(gr);
+      gLo[C] = tf32_rna(gr - tf32_rna(gr));
       bwd_edge_degree<2>(Dr, xs, yr, gyr, gxr, Rr[2 * C], C, c, need_gx, gsr, gr, bx, by);
-      gRr[2 * C] = gr;
+      gHi[2 * C] = tf32_rna(gr);
+      gLo[2 * C] = tf32_rna(gr - tf32_rna(gr));
       bwd_edge_degree<3>(Dr, xs, yr, gyr, gxr, Rr[3 * C], C, c, need_gx, gsr, gr, bx, by);
-      gRr[3 * C] = gr;
+      gHi[3 * C] = tf32_rna(gr);
+      gLo[3 * C] = tf32_rna(gr - tf32_rna(gr));
     }
     // deterministic reduction of (bx, by) over the row's channels
 #pragma unroll

@@ -70,7 +70,7 @@ inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 
 // ------------------------------------------------------------------ workspace layout
 struct WsLayout {
-  size_t D, dist, R, gR, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GY, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
+  size_t D, dist, R, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GY, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
   size_t total;
 };
 
@@ -85,7 +85,14 @@ WsLayout ws_layout(const Model& m, long long E, int N) {
   L.D = take((size_t)E * NDBLK * 4);
   L.dist = take((size_t)E * 4);
   L.R = take(T * (size_t)E * 4 * C * 4);
-  L.gR = take((size_t)E * 4 * C * 4);
+  L.gRhi = take((size_t)E * 4 * C * 4);
+  L.gRlo = take((size_t)E * 4 * C * 4);
+  L.h2hi = take((size_t)E * 64 * 4);
+  L.h2lo = take((size_t)E * 64 * 4);
+  L.gh2 = take((size_t)E * 64 * 4);
+  L.pperm = take((size_t)E * 4);
+  L.pinv = take((size_t)E * 4);
+  L.poff = take(64 * 4);
   L.g_r = take((size_t)E * 3 * 4);
   L.xs = take((T + 1) * feat);
   L.aggs = take(T * feat);
@@ -166,7 +173,7 @@ void split(const float* a, float* hi, float* lo, size_t n, cudaStream_t s) {
 }
 
 // forward of layer t over all cohorts: S (raw receiver sums) from x
-int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, const float* D, const float* R,
+int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, const float* D, const float* R, const int* rrow,
                   float* S, void* ws, const WsLayout& L, cudaStream_t s) {
   const int C = m.spec.C;
   const long long E = g->n_edges, coh = m.spec.cohort_edges;
@@ -181,30 +188,103 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
   int* counter = at<int>(ws, L.counter);
   for (long long e0 = 0; e0 < E; e0 += coh) {
     const long long e1 = std::min(E, e0 + coh);
-    { Scope sc_("rotate_in", s); k_rotate_in<<<grid_for(e1 - e0, eb.y), eb, esmem, s>>>(e0, e1, C, g->send, D, R, x, XT, XTlo); }
+    { Scope sc_("rotate_in", s); k_rotate_in<<<grid_for(e1 - e0, eb.y), eb, esmem, s>>>(e0, e1, C, g->send, rrow, D, R, x, XT, XTlo); }
     So2Part part{am.get(e1 - e0), &m.bmaps_fwd[t], Y};
     int st = so2_product(m, e1 - e0, &part, 1, counter, s);
     if (st != EMP_OK) return st;
     const int cg = std::min(C, RB_CG);
-    dim3 grid((unsigned)std::min<long long>(coh, 512), C / cg);
-    { Scope sc_("rotate_back_scatter", s); k_rotate_back_scatter<<<grid, dim3(cg, RB_ROWS), 0, s>>>(e0, e1, C, g->recv, g->recv_off, D, Y, S); }
+    dim3 grid((unsigned)std::min<long long>(coh, 128), C / cg);
+    { Scope sc_("rotate_back_scatter", s); k_rotate_back_scatter<<<grid, dim3(cg, RB_ROWS), sizeof(RbSmem), s>>>(e0, e1, C, g->recv, g->recv_off, D, Y, S); }
   }
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
 
-void radial_forward(const Model& m, const emp_graph* g, int t, const int* species, const float* dist, float* R,
-                    cudaStream_t s) {
+// Rows of the radial network: edge order for one radial network, pair-sorted for
+// per-pair networks (stable counting sort; the host reads the pair offsets once).
+struct RadialRows {
+  const int* perm = nullptr;   // row -> edge (null: identity)
+  const int* inv = nullptr;    // edge -> row
+  std::vector<int> off;        // [n_pairs + 1] first row of each pair
+};
+
+int radial_rows(const Model& m, const emp_graph* g, const int* species, void* ws, const WsLayout& L,
+                RadialRows& rr, cudaStream_t s) {
   const long long E = g->n_edges;
-  { Scope sc_("radial_fwd", s); k_radial_fwd<<<(unsigned)((E + RT - 1) / RT), RAD_THREADS, sizeof(RadialSmem), s>>>(
-      E, dist, g->recv, g->send, species, radial_args(m, t), R); }
+  rr.off.assign(m.n_pairs + 1, 0);
+  if (!m.spec.pair_radial) {
+    rr.off[1] = (int)E;
+    return EMP_OK;
+  }
+  int* perm = at<int>(ws, L.pperm);
+  int* inv = at<int>(ws, L.pinv);
+  int* off = at<int>(ws, L.poff);
+  { Scope sc_("pair_sort", s); k_pair_sort<<<1, PS_THREADS, (size_t)m.n_pairs * PS_THREADS * 4, s>>>(
+        E, m.spec.n_species, m.n_pairs, g->recv, g->send, species, perm, inv, off); }
+  EMP_CUDA_TRY(cudaMemcpyAsync(rr.off.data(), off, (m.n_pairs + 1) * sizeof(int), cudaMemcpyDeviceToHost, s));
+  EMP_CUDA_TRY(cudaStreamSynchronize(s));
+  rr.perm = perm;
+  rr.inv = inv;
+  return EMP_OK;
+}
+
+// R rows [E][4C] of layer t: hidden layers on SIMT, head R = h2 W3^T on the tensor cores
+int radial_forward(const Model& m, const emp_graph* g, int t, const int* species, const float* dist, float* R,
+                   const RadialRows& rr, void* ws, const WsLayout& L, cudaStream_t s) {
+  const long long E = g->n_edges;
+  const int C = m.spec.C;
+  float* h2hi = at<float>(ws, L.h2hi);
+  float* h2lo = at<float>(ws, L.h2lo);
+  { Scope sc_("radial_h2", s); k_radial_h2<<<(unsigned)((E + RT - 1) / RT), RAD_THREADS, sizeof(RadialSmem), s>>>(
+        E, rr.perm, dist, g->recv, g->send, species, radial_args(m, t), h2hi, h2lo); }
+  for (int p = 0; p < m.n_pairs; ++p) {
+    const long long r0 = rr.off[p], n = rr.off[p + 1] - r0;
+    if (n <= 0) continue;
+    MapPair a;
+    int st = make_pair(&a, h2hi + r0 * 64, h2lo + r0 * 64, n, 64, 64, tc::BM);
+    if (st != EMP_OK) return st;
+    const MapPair& b = m.w3_maps[(size_t)t * m.n_pairs + p];
+    GemmSub sub{&a.hi, &a.lo, &b.hi, &b.lo, 0, 64, 4 * C, 0, R + r0 * 4 * C};
+    Scope sc_("radial_head", s);
+    st = tc_group(n, 4 * C, &sub, 1, at<int>(ws, L.counter), s);
+    if (st != EMP_OK) return st;
+  }
+  return EMP_OK;
+}
+
+// dE/dd of layer t from dE/dR (rows split hi/lo): dE/dh2 = dE/dR W3 on the tensor cores, then the
+// hidden layers' backward on SIMT; adds (dE/dd) rhat to g_r
+int radial_backward(const Model& m, const emp_graph* g, int t, const int* species, const float* dist,
+                    const RadialRows& rr, float* g_r, void* ws, const WsLayout& L, cudaStream_t s) {
+  const long long E = g->n_edges;
+  const int C = m.spec.C;
+  float* gRhi = at<float>(ws, L.gRhi);
+  float* gRlo = at<float>(ws, L.gRlo);
+  float* gh2 = at<float>(ws, L.gh2);
+  for (int p = 0; p < m.n_pairs; ++p) {
+    const long long r0 = rr.off[p], n = rr.off[p + 1] - r0;
+    if (n <= 0) continue;
+    MapPair a;
+    int st = make_pair(&a, gRhi + r0 * 4 * C, gRlo + r0 * 4 * C, n, 4 * C, 4 * C, tc::BM);
+    if (st != EMP_OK) return st;
+    const MapPair& b = m.w3t_maps[(size_t)t * m.n_pairs + p];
+    GemmSub sub{&a.hi, &a.lo, &b.hi, &b.lo, 0, 4 * C, 64, 0, gh2 + r0 * 64};
+    Scope sc_("radial_head_bwd", s);
+    st = tc_group(n, 64, &sub, 1, at<int>(ws, L.counter), s);
+    if (st != EMP_OK) return st;
+  }
+  { Scope sc_("radial_bwd", s); k_radial_bwd<<<(unsigned)((E + RT - 1) / RT), RAD_THREADS, sizeof(RadialSmem), s>>>(
+        E, rr.perm, dist, g->vec, g->recv, g->send, species, radial_args(m, t), gh2, g_r); }
+  return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
 
 bool g_attrs_set = false;
 int ensure_attrs() {
   if (g_attrs_set) return EMP_OK;
-  EMP_CUDA_TRY(cudaFuncSetAttribute(k_radial_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(RadialSmem)));
+  EMP_CUDA_TRY(cudaFuncSetAttribute(k_radial_h2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(RadialSmem)));
+  EMP_CUDA_TRY(cudaFuncSetAttribute(k_pair_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * PS_THREADS * 4));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_radial_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(RadialSmem)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_cohort_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, 8 << 14));
+  EMP_CUDA_TRY(cudaFuncSetAttribute(k_rotate_back_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(RbSmem)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_chain_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ChainFwdSmem)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_chain_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ChainBwdSmem)));
   int st = so2_tc_init();
@@ -383,7 +463,8 @@ int mp_model_create(const emp_model_spec* spec, const float* weights, size_t n_f
   const size_t C = spec->C, T = spec->n_layers, S = spec->n_species;
   const size_t n_emb = S * C, n_rad = T * m->n_pairs * m->rad_stride(), n_so2 = T * m->so2_stride();
   const size_t n_ro = (size_t)m->Hro * C + m->Hro;
-  const size_t total = n_emb + n_rad + 6 * n_so2 + n_ro + n_floats;   // + raw staging
+  const size_t n_w3 = T * m->n_pairs * (size_t)4 * C * 64;
+  const size_t total = n_emb + n_rad + 6 * n_so2 + 4 * n_w3 + n_ro + n_floats;   // + raw staging
   float* base = nullptr;
   if (cudaMalloc(&base, total * 4) != cudaSuccess) { delete m; return EMP_ERR_CUDA; }
   m->base = base;
@@ -395,7 +476,11 @@ int mp_model_create(const emp_model_spec* spec, const float* weights, size_t n_f
   m->so2_fwd_lo = m->so2_fwd_hi + n_so2;
   m->so2_bwd_hi = m->so2_fwd_lo + n_so2;
   m->so2_bwd_lo = m->so2_bwd_hi + n_so2;
-  m->ro_W = m->so2_bwd_lo + n_so2;
+  m->w3_hi = m->so2_bwd_lo + n_so2;
+  m->w3_lo = m->w3_hi + n_w3;
+  m->w3t_hi = m->w3_lo + n_w3;
+  m->w3t_lo = m->w3t_hi + n_w3;
+  m->ro_W = m->w3t_lo + n_w3;
   m->ro_w = m->ro_W + (size_t)m->Hro * C;
   float* raw = m->ro_w + m->Hro;
   auto fail = [&](int code) { cudaFree(base); delete m; return code; };
@@ -430,6 +515,25 @@ int mp_model_create(const emp_model_spec* spec, const float* weights, size_t n_f
   if (o != n_floats) return fail(EMP_ERR_ARG);
   k_split_tf32<<<256, 256>>>(m->so2_fwd, m->so2_fwd_hi, m->so2_fwd_lo, n_so2);
   k_split_tf32<<<256, 256>>>(m->so2_bwd, m->so2_bwd_hi, m->so2_bwd_lo, n_so2);
+  // radial heads: W3 split, and W3^T split (input gradient dE/dh2 = dE/dR W3)
+  for (size_t t = 0; t < T; ++t)
+    for (int p = 0; p < m->n_pairs; ++p) {
+      const size_t wo = (t * m->n_pairs + p) * m->w3_stride();
+      const float* W3 = m->W3((int)t, p);
+      float* tmpT = m->w3t_hi + wo;   // transpose lands in the hi slot, then is split in place
+      k_transpose<<<(int)((m->w3_stride() + 255) / 256), 256>>>(W3, tmpT, 4 * (int)C, 64);
+      k_split_tf32<<<64, 256>>>(W3, m->w3_hi + wo, m->w3_lo + wo, m->w3_stride());
+      k_split_tf32<<<64, 256>>>(tmpT, m->w3t_hi + wo, m->w3t_lo + wo, m->w3_stride());
+    }
+  m->w3_maps.resize(T * m->n_pairs);
+  m->w3t_maps.resize(T * m->n_pairs);
+  for (size_t q = 0; q < T * m->n_pairs; ++q) {
+    const size_t wo = q * m->w3_stride();
+    if (make_pair(&m->w3_maps[q], m->w3_hi + wo, m->w3_lo + wo, 4 * C, 64, 64, (int)std::min<size_t>(4 * C, 256)) !=
+            EMP_OK ||
+        make_pair(&m->w3t_maps[q], m->w3t_hi + wo, m->w3t_lo + wo, 64, 4 * (int)C, 4 * (int)C, 64) != EMP_OK)
+      return fail(EMP_ERR_CUDA);
+  }
   m->bmaps_fwd.resize(T);
   m->bmaps_bwd.resize(T);
   for (size_t t = 0; t < T; ++t) {
@@ -493,8 +597,12 @@ int mp_forward(const void* model, const emp_graph* g, int32_t layer, const int32
   float* dist = at<float>(ws, L.dist);
   float* R = at<float>(ws, L.R);
   { Scope sc_("geometry", stream); k_geometry<<<(unsigned)((E + 127) / 128), 128, 0, stream>>>(E, g->vec, D, dist); }
-  radial_forward(m, g, layer, species, dist, R, stream);
-  st = layer_forward(m, g, layer, x_in, D, R, agg_out, ws, L, stream);
+  RadialRows rr;
+  st = radial_rows(m, g, species, ws, L, rr, stream);
+  if (st != EMP_OK) return st;
+  st = radial_forward(m, g, layer, species, dist, R, rr, ws, L, stream);
+  if (st != EMP_OK) return st;
+  st = layer_forward(m, g, layer, x_in, D, R, rr.inv, agg_out, ws, L, stream);
   if (st != EMP_OK) return st;
   const size_t n = (size_t)N * 16 * C;
   { Scope sc_("scale", stream); k_scale<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(n, 1.0f / m.spec.avg_degree, agg_out); }
@@ -516,7 +624,8 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
   float* D = at<float>(ws, L.D);
   float* dist = at<float>(ws, L.dist);
   float* Rall = at<float>(ws, L.R);
-  float* gR = at<float>(ws, L.gR);
+  float* gRhi = at<float>(ws, L.gRhi);
+  float* gRlo = at<float>(ws, L.gRlo);
   float* g_r = at<float>(ws, L.g_r);
   float* xs = at<float>(ws, L.xs);
   float* aggs = at<float>(ws, L.aggs);
@@ -553,12 +662,18 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
     while (P < coh) P <<= 1;
     { Scope sc_("cohort_sort", stream); k_cohort_sort<<<ncoh, 1024, (size_t)P * 8, stream>>>(E, (int)coh, g->send, perm, seg, nseg); }
   }
+  RadialRows rr;
+  if (E > 0) {
+    st = radial_rows(m, g, species, ws, L, rr, stream);
+    if (st != EMP_OK) return st;
+  }
   // ---------------- forward
   for (int t = 0; t < T; ++t) {
     float* R = Rall + (size_t)t * E * 4 * C;
     if (E > 0) {
-      radial_forward(m, g, t, species, dist, R, stream);
-      st = layer_forward(m, g, t, xs + (size_t)t * feat, D, R, aggs + (size_t)t * feat, ws, L, stream);
+      st = radial_forward(m, g, t, species, dist, R, rr, ws, L, stream);
+      if (st != EMP_OK) return st;
+      st = layer_forward(m, g, t, xs + (size_t)t * feat, D, R, rr.inv, aggs + (size_t)t * feat, ws, L, stream);
       if (st != EMP_OK) return st;
     }
     { Scope sc_("update", stream); k_update<<<(unsigned)((N * C + 255) / 256), 256, 0, stream>>>(N, C, inv_avg, m.spec.gated, aggs + (size_t)t * feat,
@@ -576,21 +691,22 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
     for (long long e0 = 0; e0 < E; e0 += coh, ++ci) {
       const long long e1 = std::min(E, e0 + coh), n = e1 - e0;
       const int grid = grid_for(n, eb.y);
-      { Scope sc_("bwd_prep", stream); k_bwd_prep<<<grid, eb, (size_t)eb.y * NDBLK * 4, stream>>>(e0, e1, C, g->recv, g->send, D, R, xt, gS, XT, XTlo,
+      { Scope sc_("bwd_prep", stream); k_bwd_prep<<<grid, eb, (size_t)eb.y * NDBLK * 4, stream>>>(e0, e1, C, g->recv, g->send, rr.inv, D, R, xt, gS, XT, XTlo,
                                                                   GY, GYhi, GYlo); }
       So2Part parts[2] = {{am_xt.get(n), &m.bmaps_fwd[t], Y}, {am_gy.get(n), &m.bmaps_bwd[t], GXT}};
       st = so2_product(m, n, parts, 2, counter, stream);
       if (st != EMP_OK) return st;
       const size_t smem = (size_t)eb.y * NDBLK * 4 + (size_t)eb.y * 2 * (C / 32) * 4;
-      { Scope sc_("bwd_edge", stream); k_bwd_edge<<<grid, eb, smem, stream>>>(e0, e1, C, t > 0, g->send, g->vec, D, R, xt, Y, GY, GXT, XT, gR, g_r); }
+      { Scope sc_("bwd_edge", stream); k_bwd_edge<<<grid, eb, smem, stream>>>(e0, e1, C, t > 0, g->send, rr.inv, g->vec, D, R, xt, Y, GY, GXT, XT, gRhi, gRlo, g_r); }
       if (t > 0) {
         dim3 sg(std::min<long long>(n, 2048), C / 32);
         { Scope sc_("sender_scatter", stream); k_sender_scatter<<<sg, 32, 0, stream>>>(e0, e1, C, ci, g->send, perm, seg, nseg, XT, gxb); }
       }
     }
-    if (E > 0)
-      { Scope sc_("radial_bwd", stream); k_radial_bwd<<<(unsigned)((E + RT - 1) / RT), RAD_THREADS, sizeof(RadialSmem), stream>>>(
-          E, dist, g->vec, g->recv, g->send, species, radial_args(m, t), gR, g_r); }
+    if (E > 0) {
+      st = radial_backward(m, g, t, species, dist, rr, g_r, ws, L, stream);
+      if (st != EMP_OK) return st;
+    }
     std::swap(gxa, gxb);
   }
   { Scope sc_("forces", stream); k_forces<<<(N + 127) / 128, 128, 0, stream>>>(N, g->recv_off, g->mirror, g_r, forces); }

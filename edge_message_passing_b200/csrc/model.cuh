@@ -30,6 +30,10 @@ struct Model {
   void* base;
   int device;
   std::vector<So2BMaps> bmaps_fwd, bmaps_bwd;   // tensor maps of each layer's stacked blocks
+  // radial head W3 [4C][64] of each (layer, pair) split for 3xTF32, and its transpose [64][4C]
+  float *w3_hi, *w3_lo, *w3t_hi, *w3t_lo;
+  std::vector<MapPair> w3_maps, w3t_maps;      // index t * n_pairs + p
+  size_t w3_stride() const { return (size_t)4 * spec.C * 64; }
 
   size_t rad_stride() const { return (size_t)H * 8 + (size_t)H * H + (size_t)4 * spec.C * H; }
   const float* W1(int t, int p) const { return rad + ((size_t)t * n_pairs + p) * rad_stride(); }
@@ -125,6 +129,14 @@ __global__ void k_stack_so2(const float* __restrict__ W0, const float* __restric
     fwd[idx] = v;
     bwd[(size_t)wblk_off(b) * C * C + (size_t)k * K + n] = v;
   }
+}
+
+// dst [cols][rows] = src [rows][cols]^T
+__global__ void k_transpose(const float* __restrict__ src, float* __restrict__ dst, int rows, int cols) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= rows * cols) return;
+  const int r = idx / cols, c = idx % cols;
+  dst[(size_t)c * rows + r] = src[idx];
 }
 
 // 3xTF32 split: hi = round-to-nearest TF32 of a, lo = TF32(a - hi)

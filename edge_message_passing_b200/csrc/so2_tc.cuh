@@ -21,6 +21,7 @@
 #pragma once
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <algorithm>
 #include "emp_common.cuh"
 
 namespace emp {
@@ -44,11 +45,14 @@ struct Group {
   int M, nsub, mtiles;
   int a_idx[MAXSUB];    // which A operand pair (0 or 1)
   int b_idx[MAXSUB];    // which B map pair
-  int col[MAXSUB];      // first column (A and output) of the sub-problem
-  int K[MAXSUB];        // K = N of the sub-problem
+  int acol[MAXSUB];     // first A column of the sub-problem
+  int K[MAXSUB];
+  int N[MAXSUB];        // output columns
+  int bn[MAXSUB];       // tile width (MMA N): min(N, 256), a multiple of 16
+  int ccol[MAXSUB];     // first output column
   int ntiles[MAXSUB];   // n-tiles per m-tile
   int first[MAXSUB + 1];// first tile index of each sub-problem (sub-problems ordered by decreasing K)
-  int ld;               // row pitch (elements) of A and of the outputs
+  int ldc;              // row pitch (elements) of the outputs
   float* out[MAXSUB];
   int* counter;         // dynamic tile counter (zeroed by the host before the launch)
 };
@@ -105,15 +109,17 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr) {
          ((uint64_t)1 << 46) | ((uint64_t)4 << 61);
 }
 
-// instruction descriptor: D f32, A/B tf32, both K-major, M = 128, N = BN
-constexpr uint32_t IDESC = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+// instruction descriptor: D f32, A/B tf32, both K-major, M = 128, N = n
+__host__ __device__ constexpr uint32_t idesc_for(int n) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
 
-__device__ __forceinline__ void mma_tf32(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accum) {
+__device__ __forceinline__ void mma_tf32(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accum) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n"
-      ::"r"(tmem_d), "l"(a), "l"(b), "r"(IDESC), "r"(accum));
+      ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(accum));
 }
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -151,7 +157,7 @@ __device__ __forceinline__ TileInfo tile_info(const Group& g, int t) {
   const int r = t - g.first[s];
   ti.sub = s;
   ti.m0 = (r / g.ntiles[s]) * BM;
-  ti.n0 = (r % g.ntiles[s]) * BN;
+  ti.n0 = (r % g.ntiles[s]) * g.bn[s];
   return ti;
 }
 
@@ -227,9 +233,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_so2_tc(const __grid_constant__ G
         if (it >= ST && !mbar_wait(&empty[s], ((it / ST) - 1) & 1)) { *vabort = 1; break; }
         if (*vabort) break;
         unsigned char* st = smem + s * STAGE_BYTES;
-        mbar_expect_tx(&full[s], STAGE_BYTES);
-        tma_load(st, &maps.a_hi[a], &full[s], g.col[ti.sub] + kc * BK, ti.m0);
-        tma_load(st + A_BYTES, &maps.a_lo[a], &full[s], g.col[ti.sub] + kc * BK, ti.m0);
+        mbar_expect_tx(&full[s], 2 * A_BYTES + 2 * g.bn[ti.sub] * BK * 4);
+        tma_load(st, &maps.a_hi[a], &full[s], g.acol[ti.sub] + kc * BK, ti.m0);
+        tma_load(st + A_BYTES, &maps.a_lo[a], &full[s], g.acol[ti.sub] + kc * BK, ti.m0);
         tma_load(st + 2 * A_BYTES, &maps.b_hi[b], &full[s], kc * BK, ti.n0);
         tma_load(st + 2 * A_BYTES + B_BYTES, &maps.b_lo[b], &full[s], kc * BK, ti.n0);
         *issued = it + 1;
@@ -251,6 +257,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_so2_tc(const __grid_constant__ G
       if (i >= 2 && !mbar_wait(&acc_empty[buf], ((i >> 1) - 1) & 1)) { ok = false; break; }
       fence_after();
       const uint32_t d = tmem + (uint32_t)(buf * BN);
+      const uint32_t idesc = idesc_for(g.bn[ti.sub]);
       for (int kc = 0; kc < nk; ++kc, ++it) {
         const int s = it % ST;
         if (!mbar_wait(&full[s], (it / ST) & 1)) { ok = false; break; }
@@ -263,9 +270,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_so2_tc(const __grid_constant__ G
 #pragma unroll
         for (int kk = 0; kk < BK / 8; ++kk) {
           const uint32_t off = kk * 32;   // 8 fp32 of K = 32 bytes inside the swizzled row
-          mma_tf32(d, sdesc(a_lo + off), sdesc(b_hi + off), (kc | kk) ? 1u : 0u);
-          mma_tf32(d, sdesc(a_hi + off), sdesc(b_lo + off), 1u);
-          mma_tf32(d, sdesc(a_hi + off), sdesc(b_hi + off), 1u);
+          mma_tf32(d, sdesc(a_lo + off), sdesc(b_hi + off), idesc, (kc | kk) ? 1u : 0u);
+          mma_tf32(d, sdesc(a_hi + off), sdesc(b_lo + off), idesc, 1u);
+          mma_tf32(d, sdesc(a_hi + off), sdesc(b_hi + off), idesc, 1u);
         }
         mma_commit(&empty[s]);
       }
@@ -291,10 +298,10 @@ __global__ void __launch_bounds__(THREADS, 1) k_so2_tc(const __grid_constant__ G
       if (!mbar_wait(&acc_full[buf], (i >> 1) & 1)) { *vabort = 1; break; }
       fence_after();
       const int m = ti.m0 + row;
-      const int N = g.K[ti.sub];
-      float* orow = g.out[ti.sub] + (size_t)m * g.ld + g.col[ti.sub] + ti.n0;
+      const int N = g.N[ti.sub], bn = g.bn[ti.sub];
+      float* orow = g.out[ti.sub] + (size_t)m * g.ldc + g.ccol[ti.sub] + ti.n0;
 #pragma unroll 1
-      for (int cc = 0; cc < BN; cc += 32) {
+      for (int cc = 0; cc < bn; cc += 32) {
         float v[32];
         tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + cc), v);
         if (m < g.M && ti.n0 + cc < N) {
@@ -367,30 +374,99 @@ inline int so2_tc_init() {
   return EMP_OK;
 }
 
+// One plain product on the tensor cores (3xTF32): out[:, ccol + n] = sum_k A[:, acol + k] B[n][k].
+struct GemmSub {
+  const CUtensorMap* a_hi;
+  const CUtensorMap* a_lo;
+  const CUtensorMap* b_hi;
+  const CUtensorMap* b_lo;
+  int acol, K, N, ccol;
+  float* out;
+};
+
+// Launch a group of products sharing the row count M (at most two distinct A operands).
+// Sub-problems are reordered by decreasing K; counter: one device int, zeroed here.
+inline int tc_group(long long M, int ldc, const GemmSub* subs, int nsub, int* counter, cudaStream_t s) {
+  if (M <= 0) return EMP_OK;
+  if (nsub < 1 || nsub > tc::MAXSUB || M >= (1ll << 31)) return EMP_ERR_ARG;
+  tc::Group g{};
+  tc::Maps maps;
+  g.M = (int)M;
+  g.ldc = ldc;
+  g.nsub = nsub;
+  g.mtiles = (int)((M + tc::BM - 1) / tc::BM);
+  g.counter = counter;
+  int ord[tc::MAXSUB];
+  for (int i = 0; i < nsub; ++i) ord[i] = i;
+  std::stable_sort(ord, ord + nsub, [&](int a, int b) { return subs[a].K > subs[b].K; });
+  const CUtensorMap* a_seen[2] = {nullptr, nullptr};
+  int na = 0;
+  long long first = 0;
+  for (int q = 0; q < nsub; ++q) {
+    const GemmSub& u = subs[ord[q]];
+    if (u.K % tc::BK != 0 || u.N < 16 || u.N % 16 != 0) return EMP_ERR_ARG;
+    int a = 0;
+    while (a < na && a_seen[a] != u.a_hi) ++a;
+    if (a == na) {
+      if (na == 2) return EMP_ERR_ARG;
+      a_seen[na] = u.a_hi;
+      maps.a_hi[na] = *u.a_hi;
+      maps.a_lo[na] = *u.a_lo;
+      ++na;
+    }
+    maps.b_hi[q] = *u.b_hi;
+    maps.b_lo[q] = *u.b_lo;
+    g.a_idx[q] = a;
+    g.b_idx[q] = q;
+    g.acol[q] = u.acol;
+    g.K[q] = u.K;
+    g.N[q] = u.N;
+    g.bn[q] = std::min(u.N, tc::BN);
+    g.ccol[q] = u.ccol;
+    g.ntiles[q] = (u.N + g.bn[q] - 1) / g.bn[q];
+    g.out[q] = u.out;
+    g.first[q] = (int)first;
+    first += (long long)g.ntiles[q] * g.mtiles;
+  }
+  if (first >= (1ll << 31)) return EMP_ERR_UNSUPPORTED;
+  g.first[nsub] = (int)first;
+  if (cudaMemsetAsync(counter, 0, sizeof(int), s) != cudaSuccess) return EMP_ERR_CUDA;
+  const int grid = (int)std::min<long long>(first, tc::num_sms());
+  tc::k_so2_tc<<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(g, maps, (int)first);
+  return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
+}
+
+// Tensor maps (hi, lo) of a row-major fp32 matrix [rows][cols] with row pitch ld,
+// tiles of box_rows rows (BM for A operands, min(N, 256) for B operands).
+struct MapPair {
+  CUtensorMap hi, lo;
+};
+inline int make_pair(MapPair* m, const float* hi, const float* lo, long long rows, int cols, int ld, int box_rows) {
+  if (!tc::make_map(&m->hi, hi, cols, rows, ld, box_rows)) return EMP_ERR_CUDA;
+  if (!tc::make_map(&m->lo, lo, cols, rows, ld, box_rows)) return EMP_ERR_CUDA;
+  return EMP_OK;
+}
+
 // Tensor maps of one operand set of the SO(2) mixing: A (hi, lo) rows [M][16C] and a
 // layer's stacked 4-block weights (hi, lo).  Built once (weights: at model
 // creation; activations: once per call and cohort size) and reused by every launch.
 struct So2BMaps {
-  CUtensorMap hi[4], lo[4];
+  MapPair blk[4];
 };
-struct So2AMaps {
-  CUtensorMap hi, lo;
-};
+typedef MapPair So2AMaps;
 
 inline int so2_make_bmaps(So2BMaps* m, int C, const float* b_hi, const float* b_lo) {
   for (int b = 0; b < 4; ++b) {
-    const uint64_t K = (uint64_t)blk_width(b) * C;
+    const int K = blk_width(b) * C;
     const size_t off = (size_t)wblk_off(b) * C * C;
-    if (!tc::make_map(&m->hi[b], b_hi + off, K, K, K, tc::BN)) return EMP_ERR_CUDA;
-    if (!tc::make_map(&m->lo[b], b_lo + off, K, K, K, tc::BN)) return EMP_ERR_CUDA;
+    int st = make_pair(&m->blk[b], b_hi + off, b_lo + off, K, K, K, std::min(K, tc::BN));
+    if (st != EMP_OK) return st;
   }
   return EMP_OK;
 }
 
 inline int so2_make_amaps(So2AMaps* m, int C, long long M, const float* a_hi, const float* a_lo) {
-  if (!tc::make_map(&m->hi, a_hi, 16 * C, M, 16 * C, tc::BM)) return EMP_ERR_CUDA;
-  if (!tc::make_map(&m->lo, a_lo, 16 * C, M, 16 * C, tc::BM)) return EMP_ERR_CUDA;
-  return EMP_OK;
+  return make_pair(m, a_hi, a_lo, M, 16 * C, 16 * C, tc::BM);
 }
 
 struct So2Part {
@@ -399,47 +475,18 @@ struct So2Part {
   float* out;
 };
 
-// Grouped launch over one or two operand sets sharing M (forward: 1; backward: 2).
-// counter: one device int of scratch, zeroed here before the launch.
+// SO(2) mixing of a cohort: one operand set (forward) or two sharing the rows (backward).
 inline int so2_tc(long long M, int C, const So2Part* parts, int nparts, int* counter, cudaStream_t s) {
-  if (M <= 0) return EMP_OK;
   if (nparts < 1 || nparts > 2) return EMP_ERR_ARG;
-  tc::Group g{};
-  tc::Maps maps;
-  g.M = (int)M;
-  g.ld = 16 * C;
-  g.nsub = 4 * nparts;
-  g.mtiles = (int)((M + tc::BM - 1) / tc::BM);
-  g.counter = counter;
-  // sub-problems ordered by decreasing K (block 1, then 0, 2, then 3) so the longest tiles go first
-  const int order[4] = {1, 0, 2, 3};
-  int sidx = 0, first = 0;
-  for (int q = 0; q < 4; ++q) {
-    const int b = order[q];
-    for (int p = 0; p < nparts; ++p, ++sidx) {
+  GemmSub subs[tc::MAXSUB];
+  int n = 0;
+  for (int p = 0; p < nparts; ++p)
+    for (int b = 0; b < 4; ++b, ++n) {
       const int K = blk_width(b) * C;
-      maps.b_hi[sidx] = parts[p].b->hi[b];
-      maps.b_lo[sidx] = parts[p].b->lo[b];
-      g.a_idx[sidx] = p;
-      g.b_idx[sidx] = sidx;
-      g.col[sidx] = blk_off(b) * C;
-      g.K[sidx] = K;
-      g.ntiles[sidx] = (K + tc::BN - 1) / tc::BN;
-      g.out[sidx] = parts[p].out;
-      g.first[sidx] = first;
-      first += g.ntiles[sidx] * g.mtiles;
+      subs[n] = GemmSub{&parts[p].a->hi, &parts[p].a->lo, &parts[p].b->blk[b].hi, &parts[p].b->blk[b].lo,
+                        blk_off(b) * C, K, K, blk_off(b) * C, parts[p].out};
     }
-  }
-  g.first[g.nsub] = first;
-  for (int p = 0; p < nparts; ++p) {
-    maps.a_hi[p] = parts[p].a->hi;
-    maps.a_lo[p] = parts[p].a->lo;
-  }
-  const int total = first;
-  if (cudaMemsetAsync(counter, 0, sizeof(int), s) != cudaSuccess) return EMP_ERR_CUDA;
-  const int grid = std::min(total, tc::num_sms());
-  tc::k_so2_tc<<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(g, maps, total);
-  return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
+  return tc_group(M, 16 * C, subs, n, counter, s);
 }
 
 }  // namespace emp
