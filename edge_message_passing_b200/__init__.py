@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libemp.so")
 
 # exported symbols (kept in step with include/emp.h)
 SYMBOLS = (
-    "nl_workspace_bytes", "nl_build", "mp_weight_count", "mp_model_create", "mp_model_destroy",
+    "nl_workspace_bytes", "nl_build", "nl_build_noalloc", "mp_weight_count", "mp_model_create", "mp_model_destroy",
     "mp_workspace_bytes", "mp_forward", "mp_energy_forces", "mp_so2_mix", "mp_chain_create",
     "mp_chain_destroy", "mp_radial_chain", "emp_status_string", "emp_last_device_error",
     "emp_profile_enable", "emp_profile_read", "emp_profile_names", "emp_launch_count",
@@ -64,6 +64,8 @@ def lib() -> ctypes.CDLL:
         L.nl_workspace_bytes.argtypes = [i32]
         L.nl_build.restype = ctypes.c_int
         L.nl_build.argtypes = [ctypes.POINTER(NlParams), vp, ctypes.POINTER(GraphC), ctypes.POINTER(i64), vp, sz, vp]
+        L.nl_build_noalloc.restype = ctypes.c_int
+        L.nl_build_noalloc.argtypes = [ctypes.POINTER(NlParams), vp, ctypes.POINTER(GraphC), ctypes.POINTER(i64), vp]
         L.mp_weight_count.restype = sz
         L.mp_weight_count.argtypes = [ctypes.POINTER(SpecC)]
         L.mp_model_create.restype = ctypes.c_int

@@ -303,6 +303,35 @@ int check_device() {
 
 }  // namespace
 
+// ------------------------------------------------------------------ fixed scratch of nl_build_noalloc
+// Held by every device that loads the library, until the process exits.  Every
+// nl_build_noalloc call on a device shares it: calls whose work overlaps on the
+// GPU (different streams, no ordering between them) race on it.  nl_build clears
+// everything that must start at zero (cell counters, cursors, flags) at the start
+// of each call, and writes every other entry before reading it.
+static __device__ __align__(256) unsigned char g_nl_noalloc_scratch[EMP_NL_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64] = {};
+
+// Device address of the scratch array for the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up with
+// cudaGetSymbolAddress (once per device, with that device current).
+int nl_noalloc_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EMP_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_nl_noalloc_scratch) != cudaSuccess || !ptr) return EMP_ERR_CUDA;
+    g_noalloc_addr[dev] = ptr;
+  }
+  *out = g_noalloc_addr[dev];
+  return EMP_OK;
+}
+}  // namespace
+
 // ====================================================================== C ABI
 extern "C" {
 
@@ -377,8 +406,8 @@ size_t nl_workspace_bytes(int32_t n_atoms) {
   return align_up(n * 4) * 7 + align_up(n * 12) + align_up(16) + align_up(8) + 4096;
 }
 
-int nl_build(const emp_nl_params* p, const double* pos, emp_graph* g, int64_t* n_edges, void* ws,
-             size_t ws_bytes, cudaStream_t stream) {
+static int nl_build_impl(const emp_nl_params* p, const double* pos, emp_graph* g, int64_t* n_edges, void* ws,
+                         size_t ws_bytes, cudaStream_t stream) {
   if (!p || !pos || !g || !n_edges || !ws) return EMP_ERR_ARG;
   const int N = p->n_atoms;
   if (N < 1 || !(p->cutoff > 0) || !g->recv_off) return EMP_ERR_ARG;
@@ -441,6 +470,29 @@ int nl_build(const emp_nl_params* p, const double* pos, emp_graph* g, int64_t* n
   { Scope sc_("nl", stream); nl::k_emit<<<N, nl::EMIT_THREADS, 0, stream>>>(pos, N, G, W, g->recv_off, *g); }
   if (total > 0) { Scope sc_("nl", stream); nl::k_mirror<<<(unsigned)((total + 255) / 256), 256, 0, stream>>>(total, N, *g); }
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
+}
+
+int nl_build(const emp_nl_params* p, const double* pos, emp_graph* g, int64_t* n_edges, void* ws,
+             size_t ws_bytes, cudaStream_t stream) {
+  return nl_build_impl(p, pos, g, n_edges, ws, ws_bytes, stream);
+}
+
+// Neighbour list with the library's own fixed scratch (no allocation anywhere).
+// For callers that cannot allocate device memory themselves -- for example a
+// plug-in inside a host program whose device memory all comes from that
+// program's own pool, or a code path that must not trigger the device-wide
+// synchronisation cudaMalloc/cudaFree can cause.  The scratch is the file-scope
+// array g_nl_noalloc_scratch below; its device address is looked up once per
+// device, on the first call made with that device current.
+int nl_build_noalloc(const emp_nl_params* p, const double* pos, emp_graph* g, int64_t* n_edges,
+                     cudaStream_t stream) {
+  if (!p || !pos || !g || !n_edges) return EMP_ERR_ARG;
+  if (p->n_atoms > EMP_NL_NOALLOC_MAX_ATOMS) return EMP_ERR_WORKSPACE;
+  if (nl_workspace_bytes(std::max(p->n_atoms, 1)) > sizeof(g_nl_noalloc_scratch)) return EMP_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const int st = nl_noalloc_scratch_address(&scratch);
+  if (st != EMP_OK) return st;
+  return nl_build_impl(p, pos, g, n_edges, scratch, sizeof(g_nl_noalloc_scratch), stream);
 }
 
 // ------------------------------------------------------------------ model

@@ -93,6 +93,25 @@ size_t nl_workspace_bytes(int32_t n_atoms);
 int nl_build(const emp_nl_params* p, const double* pos, emp_graph* g, int64_t* n_edges,
              void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* Same neighbour list as nl_build, for callers that cannot allocate device
+ * memory (for example a plug-in inside a host program that owns all device
+ * memory through its own pool, or a code path that must not trigger the
+ * device-wide synchronisation that cudaMalloc / cudaFree can cause).  The
+ * caller still provides positions and the graph buffers; the cell-list scratch
+ * is a fixed array inside the library (EMP_NL_NOALLOC_SCRATCH_BYTES, held by
+ * every device that loads the library until the process exits).  Nothing is
+ * allocated.  The subject pages have no counterpart of this entry point.
+ *   - n_atoms above EMP_NL_NOALLOC_MAX_ATOMS: EMP_ERR_WORKSPACE.
+ *   - The first call on a device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls on a device share the scratch; calls whose GPU work overlaps
+ *     (unordered streams) race on it.  Each call clears what must start at zero.
+ * Other arguments, results and errors as nl_build. */
+#define EMP_NL_NOALLOC_MAX_ATOMS 65536
+#define EMP_NL_NOALLOC_SCRATCH_BYTES (3u << 20)
+int nl_build_noalloc(const emp_nl_params* p, const double* pos, emp_graph* g, int64_t* n_edges,
+                     cudaStream_t stream);
+
 /* ------------------------------------------------------------ the model
  * Hyper-parameters of the interatomic potential (configs of the seeded
  * workloads; model of the page "first-order SO(2) input-gradient path":
