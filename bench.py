@@ -299,16 +299,20 @@ def run_ours(args):
     if so2_launches:
         so2_ms = fam["so2_tc"][0] / so2_launches
         # per step: every layer mixes every edge three times (forward, backward recompute,
-        # backward transpose), in 2 launches per cohort (forward; grouped backward)
-        flops_step = 3 * spec.n_layers * E * fl_per_edge
+        # backward transpose), in 2 launches per cohort (forward; grouped backward).  The first
+        # layer's input is the species embedding (degree 0 only): its three products reduce to
+        # the m = 0 block with C inputs (forward, recompute) or C outputs (transpose): 4C^2 each.
+        flops_step = E * 2 * C * C * (3 * 72 * (spec.n_layers - 1) + 3 * 4)
         achieved = flops_step * len(ptimes) / (fam["so2_tc"][0] * 1e-3) / 1e12
         peak_tf32 = pk["bf16_tflops"] * TF32_OVER_BF16
         peak = peak_tf32 / 3.0
         roof = {"bound": "tensor", "kernel": "so2_tc (3xTF32 tcgen05 SO(2) mixing)", "achieved": achieved,
+                "flops_per_step": flops_step,
                 "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
                 "launch_ms": so2_ms, "launches_per_step": so2_launches / len(ptimes), "dominant": dom == "so2_tc",
                 "frac_vs_sustained": achieved / (pk["bf16_tflops_sustained"] * TF32_OVER_BF16 / 3.0),
-                "peak_note": f"useful FP32 flops (2*72*C^2 per edge per mixing, 3 mixings per layer) over the "
+                "peak_note": f"useful FP32 flops of the mixings actually required (2*72*C^2 per edge per "
+                             f"mixing, 3 mixings per layer; 2*4*C^2 in the degree-0-input first layer) over the "
                              f"summed launch event time, vs burst bf16 ({pk_kind}) x {TF32_OVER_BF16:.3f} "
                              f"(TF32/BF16 nominal) / 3 (3xTF32); SM clock stays at max during the step"}
     elif dom is not None:
@@ -328,6 +332,7 @@ def run_ours(args):
                              "l2": "flushed between timed steps (256 MB write outside the timed events)"},
                   "clocks": clk.summary(), "gpu_launches": launches,
                   "ms_per_step_profiled": sum(ptimes) / len(ptimes),
+                  "step_ms": [round(t, 3) for t in times], "step_ms_profiled": [round(t, 3) for t in ptimes],
                   "e2e": {"value": E * ws / (e2e_ms * 1e-3), "unit": "edges/s",
                           "h2d_bytes_per_step": int(pos_h.numel() * 8 + sp_h.numel() * 4),
                           "d2h_bytes_per_step": int(8 + N * 3 * 4)},

@@ -314,7 +314,9 @@ __global__ void __launch_bounds__(PS_THREADS) k_pair_sort(long long E, int n_spe
 
 // ------------------------------------------------------------------ rotate in
 // XT[e - e0][col(k) C + c] = R_e[l(k)][c] * (D_e x_send)[k][c]  (edge frame, m-major)
-__global__ void k_rotate_in(long long e0, long long e1, int C, const int* __restrict__ send,
+// scalar_in: the input has only degree-0 components (the first layer, whose input is the
+// species embedding), so only the (l=0, m=0) column of x~ is non-zero and only it is written.
+__global__ void k_rotate_in(long long e0, long long e1, int C, int scalar_in, const int* __restrict__ send,
                             const int* __restrict__ rrow, const float* __restrict__ D, const float* __restrict__ R,
                             const float* __restrict__ x, float* __restrict__ XT, float* __restrict__ XTlo) {
   extern __shared__ __align__(16) float sD[];           // [EPB][84]
@@ -330,6 +332,13 @@ __global__ void k_rotate_in(long long e0, long long e1, int C, const int* __rest
     __syncthreads();
     if (!ok) continue;
     const int j = send[e];
+    if (scalar_in) {
+      const size_t rr = rrow ? (size_t)rrow[e] : (size_t)e;
+      const float v = R[rr * 4 * C + c] * x[(size_t)j * 16 * C + c], h = tf32_rna(v);
+      XT[(size_t)el * 16 * C + c] = h;
+      XTlo[(size_t)el * 16 * C + c] = tf32_rna(v - h);
+      continue;
+    }
     float xv[16], u[16];
 #pragma unroll
     for (int k = 0; k < 16; ++k) xv[k] = x[((size_t)j * 16 + k) * C + c];
@@ -366,6 +375,7 @@ struct RbSmem {
 };
 
 __global__ void __launch_bounds__(RB_CG * RB_ROWS) k_rotate_back_scatter(long long e0, long long e1, int C,
+                                                                         int scalar_in,
                                                                          const int* __restrict__ recv,
                                                                          const int* __restrict__ recv_off,
                                                                          const float* __restrict__ D,
@@ -397,10 +407,22 @@ __global__ void __launch_bounds__(RB_CG * RB_ROWS) k_rotate_back_scatter(long lo
 #pragma unroll 2
       for (int k = row; k < nch; k += RB_ROWS) {
         const float* y = Y + (size_t)(cb + k - e0) * 16 * C;
+        const float* Dk = sD + k * NDBLK;
+        if (scalar_in) {
+          // y is non-zero only at m = 0: message[l][n] = D^l[0][n] y[l][0]
+#pragma unroll
+          for (int l = 0; l < 4; ++l) {
+            const float yl = y[col_of(l, 0) * C + c];
+            const float* row0 = Dk + dblk_off(l) + l * (2 * l + 1);
+#pragma unroll
+            for (int n = 0; n < 2 * l + 1; ++n) acc[l * l + n] = fmaf(row0[n], yl, acc[l * l + n]);
+          }
+          continue;
+        }
         float yv[16], m[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q) yv[q] = y[col_of_k(q) * C + c];
-        rotate16<true>(sD + k * NDBLK, yv, m);
+        rotate16<true>(Dk, yv, m);
 #pragma unroll
         for (int q = 0; q < 16; ++q) acc[q] += m[q];
       }
@@ -524,7 +546,7 @@ __global__ void k_gate_bwd(int N, int C, float inv_avg, int gated, const float* 
 }
 
 // per edge: XT = R (.) D x_send (recomputed) and GY = D gS[recv] (edge-frame output gradient)
-__global__ void k_bwd_prep(long long e0, long long e1, int C, const int* __restrict__ recv,
+__global__ void k_bwd_prep(long long e0, long long e1, int C, int scalar_in, const int* __restrict__ recv,
                            const int* __restrict__ send, const int* __restrict__ rrow, const float* __restrict__ D,
                            const float* __restrict__ R,
                            const float* __restrict__ x, const float* __restrict__ gS, float* __restrict__ XT,
@@ -544,30 +566,39 @@ __global__ void k_bwd_prep(long long e0, long long e1, int C, const int* __restr
     if (!ok) continue;
     const float* Dr = sD + row * NDBLK;
     const int j = send[e], i = recv[e];
-    float v[16], u[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) v[k] = x[((size_t)j * 16 + k) * C + c];
-    rotate16<false>(Dr, v, u);
-    float Rv[4];
-    const size_t rr = rrow ? (size_t)rrow[e] : (size_t)e;
-#pragma unroll
-    for (int l = 0; l < 4; ++l) Rv[l] = R[rr * 4 * C + l * C + c];
     const size_t ro = (size_t)el * 16 * C;
+    float v[16], u[16];
+    const size_t rr = rrow ? (size_t)rrow[e] : (size_t)e;
+    if (scalar_in) {
+      const float t = R[rr * 4 * C + c] * x[(size_t)j * 16 * C + c], h = tf32_rna(t);
+      XT[ro + c] = h;
+      XTlo[ro + c] = tf32_rna(t - h);
+    } else {
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const float t = Rv[deg_of(k)] * u[k], h = tf32_rna(t);
-      XT[ro + col_of_k(k) * C + c] = h;
-      XTlo[ro + col_of_k(k) * C + c] = tf32_rna(t - h);
+      for (int k = 0; k < 16; ++k) v[k] = x[((size_t)j * 16 + k) * C + c];
+      rotate16<false>(Dr, v, u);
+      float Rv[4];
+#pragma unroll
+      for (int l = 0; l < 4; ++l) Rv[l] = R[rr * 4 * C + l * C + c];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const float t = Rv[deg_of(k)] * u[k], h = tf32_rna(t);
+        XT[ro + col_of_k(k) * C + c] = h;
+        XTlo[ro + col_of_k(k) * C + c] = tf32_rna(t - h);
+      }
     }
 #pragma unroll
     for (int k = 0; k < 16; ++k) v[k] = gS[((size_t)i * 16 + k) * C + c];
     rotate16<false>(Dr, v, u);
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
-      const float h = tf32_rna(u[k]);
       GY[ro + col_of_k(k) * C + c] = u[k];
-      GYhi[ro + col_of_k(k) * C + c] = h;
-      GYlo[ro + col_of_k(k) * C + c] = tf32_rna(u[k] - h);
+      // with a scalar-only input only the m = 0 block of g_y enters a product
+      if (!scalar_in || col_of_k(k) < 4) {
+        const float h = tf32_rna(u[k]);
+        GYhi[ro + col_of_k(k) * C + c] = h;
+        GYlo[ro + col_of_k(k) * C + c] = tf32_rna(u[k] - h);
+      }
     }
   }
 }
@@ -598,10 +629,22 @@ __device__ __forceinline__ void bwd_edge_degree(const float* __restrict__ Dr, co
                                                 const float* __restrict__ yrow, const float* __restrict__ gyrow,
                                                 const float* __restrict__ gxtrow, float Rl, int C, int c,
                                                 bool need_gx, float* __restrict__ gxsrow, float& grl,
-                                                float& bx, float& by) {
+                                                float& bx, float& by, bool scalar_in) {
   constexpr int W = 2 * L + 1, O = L * L;
   const float* B = Dr + dblk_off(L);
   float v[W], u[W], gu[W];
+  if (scalar_in && L > 0) {
+    // input of degree 0 only: u, g_x~ and g_R vanish for L > 0 and y is non-zero only at m = 0,
+    // so only the y^T J g_y part of the torque remains
+    grl = 0.f;
+#pragma unroll
+    for (int m = 0; m < W; ++m) {
+      v[m] = (m == L) ? yrow[col_of_k(O + m) * C] : 0.f;
+      u[m] = gyrow[col_of_k(O + m) * C];
+    }
+    torque_pairs_l<L>(v, u, bx, by);
+    return;
+  }
 #pragma unroll
   for (int n = 0; n < W; ++n) v[n] = xs[(O + n) * C];
 #pragma unroll
@@ -638,7 +681,7 @@ __device__ __forceinline__ void bwd_edge_degree(const float* __restrict__ Dr, co
   }
 }
 
-__global__ void __launch_bounds__(256, 2) k_bwd_edge(long long e0, long long e1, int C, int need_gx,
+__global__ void __launch_bounds__(256, 2) k_bwd_edge(long long e0, long long e1, int C, int need_gx, int scalar_in,
                                                      const int* __restrict__ send, const int* __restrict__ rrow,
                                                      const float* __restrict__ vec,
                                                      const float* __restrict__ D, const float* __restrict__ R,
@@ -674,16 +717,16 @@ __global__ void __launch_bounds__(256, 2) k_bwd_edge(long long e0, long long e1,
       const float* gxr = GXT + rowoff + c;
       float* gsr = GXS + rowoff + c;
       float gr;
-      bwd_edge_degree<0>(Dr, xs, yr, gyr, gxr, Rr[0], C, c, need_gx, gsr, gr, bx, by);
+      bwd_edge_degree<0>(Dr, xs, yr, gyr, gxr, Rr[0], C, c, need_gx, gsr, gr, bx, by, scalar_in != 0);
       gHi[0] = tf32_rna(gr);
       gLo[0] = tf32_rna(gr - tf32_rna(gr));
-      bwd_edge_degree<1>(Dr, xs, yr, gyr, gxr, Rr[C], C, c, need_gx, gsr, gr, bx, by);
+      bwd_edge_degree<1>(Dr, xs, yr, gyr, gxr, Rr[C], C, c, need_gx, gsr, gr, bx, by, scalar_in != 0);
       gHi[C] = tf32_rna(gr);
       gLo[C] = tf32_rna(gr - tf32_rna(gr));
-      bwd_edge_degree<2>(Dr, xs, yr, gyr, gxr, Rr[2 * C], C, c, need_gx, gsr, gr, bx, by);
+      bwd_edge_degree<2>(Dr, xs, yr, gyr, gxr, Rr[2 * C], C, c, need_gx, gsr, gr, bx, by, scalar_in != 0);
       gHi[2 * C] = tf32_rna(gr);
       gLo[2 * C] = tf32_rna(gr - tf32_rna(gr));
-      bwd_edge_degree<3>(Dr, xs, yr, gyr, gxr, Rr[3 * C], C, c, need_gx, gsr, gr, bx, by);
+      bwd_edge_degree<3>(Dr, xs, yr, gyr, gxr, Rr[3 * C], C, c, need_gx, gsr, gr, bx, by, scalar_in != 0);
       gHi[3 * C] = tf32_rna(gr);
       gLo[3 * C] = tf32_rna(gr - tf32_rna(gr));
     }

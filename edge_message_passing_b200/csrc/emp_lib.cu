@@ -173,8 +173,10 @@ void split(const float* a, float* hi, float* lo, size_t n, cudaStream_t s) {
 }
 
 // forward of layer t over all cohorts: S (raw receiver sums) from x
+// scalar_in: x has only degree-0 components (the first layer's species embedding); then only the
+// m = 0 block with its first C input columns contributes, and y is non-zero only in that block.
 int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, const float* D, const float* R, const int* rrow,
-                  float* S, void* ws, const WsLayout& L, cudaStream_t s) {
+                  int scalar_in, float* S, void* ws, const WsLayout& L, cudaStream_t s) {
   const int C = m.spec.C;
   const long long E = g->n_edges, coh = m.spec.cohort_edges;
   const dim3 eb = edge_block(C);
@@ -188,13 +190,22 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
   int* counter = at<int>(ws, L.counter);
   for (long long e0 = 0; e0 < E; e0 += coh) {
     const long long e1 = std::min(E, e0 + coh);
-    { Scope sc_("rotate_in", s); k_rotate_in<<<grid_for(e1 - e0, eb.y), eb, esmem, s>>>(e0, e1, C, g->send, rrow, D, R, x, XT, XTlo); }
-    So2Part part{am.get(e1 - e0), &m.bmaps_fwd[t], Y};
-    int st = so2_product(m, e1 - e0, &part, 1, counter, s);
+    { Scope sc_("rotate_in", s); k_rotate_in<<<grid_for(e1 - e0, eb.y), eb, esmem, s>>>(e0, e1, C, scalar_in, g->send, rrow, D, R, x, XT, XTlo); }
+    int st;
+    if (scalar_in) {
+      const So2AMaps* a = am.get(e1 - e0);
+      const MapPair& b0 = m.bmaps_fwd[t].blk[0];
+      GemmSub sub{&a->hi, &a->lo, &b0.hi, &b0.lo, 0, C, 4 * C, 0, Y};
+      Scope sc_("so2_tc", s);
+      st = tc_group(e1 - e0, 16 * C, &sub, 1, counter, s);
+    } else {
+      So2Part part{am.get(e1 - e0), &m.bmaps_fwd[t], Y};
+      st = so2_product(m, e1 - e0, &part, 1, counter, s);
+    }
     if (st != EMP_OK) return st;
     const int cg = std::min(C, RB_CG);
     dim3 grid((unsigned)std::min<long long>(coh, 128), C / cg);
-    { Scope sc_("rotate_back_scatter", s); k_rotate_back_scatter<<<grid, dim3(cg, RB_ROWS), sizeof(RbSmem), s>>>(e0, e1, C, g->recv, g->recv_off, D, Y, S); }
+    { Scope sc_("rotate_back_scatter", s); k_rotate_back_scatter<<<grid, dim3(cg, RB_ROWS), sizeof(RbSmem), s>>>(e0, e1, C, scalar_in, g->recv, g->recv_off, D, Y, S); }
   }
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
@@ -588,6 +599,13 @@ int mp_model_create(const emp_model_spec* spec, const float* weights, size_t n_f
   }
   m->bmaps_fwd.resize(T);
   m->bmaps_bwd.resize(T);
+  m->b0_bwd_narrow.resize(T);
+  for (size_t t = 0; t < T; ++t) {
+    const size_t off = t * m->so2_stride();
+    if (make_pair(&m->b0_bwd_narrow[t], m->so2_bwd_hi + off, m->so2_bwd_lo + off, 4 * C, 4 * (int)C, 4 * (int)C,
+                  (int)std::min<size_t>(C, 256)) != EMP_OK)
+      return fail(EMP_ERR_CUDA);
+  }
   for (size_t t = 0; t < T; ++t) {
     const size_t off = t * m->so2_stride();
     if (so2_make_bmaps(&m->bmaps_fwd[t], (int)C, m->so2_fwd_hi + off, m->so2_fwd_lo + off) != EMP_OK ||
@@ -654,7 +672,7 @@ int mp_forward(const void* model, const emp_graph* g, int32_t layer, const int32
   if (st != EMP_OK) return st;
   st = radial_forward(m, g, layer, species, dist, R, rr, ws, L, stream);
   if (st != EMP_OK) return st;
-  st = layer_forward(m, g, layer, x_in, D, R, rr.inv, agg_out, ws, L, stream);
+  st = layer_forward(m, g, layer, x_in, D, R, rr.inv, 0, agg_out, ws, L, stream);
   if (st != EMP_OK) return st;
   const size_t n = (size_t)N * 16 * C;
   { Scope sc_("scale", stream); k_scale<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(n, 1.0f / m.spec.avg_degree, agg_out); }
@@ -725,7 +743,8 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
     if (E > 0) {
       st = radial_forward(m, g, t, species, dist, R, rr, ws, L, stream);
       if (st != EMP_OK) return st;
-      st = layer_forward(m, g, t, xs + (size_t)t * feat, D, R, rr.inv, aggs + (size_t)t * feat, ws, L, stream);
+      // the first layer's input is the species embedding: degree 0 only
+      st = layer_forward(m, g, t, xs + (size_t)t * feat, D, R, rr.inv, t == 0, aggs + (size_t)t * feat, ws, L, stream);
       if (st != EMP_OK) return st;
     }
     { Scope sc_("update", stream); k_update<<<(unsigned)((N * C + 255) / 256), 256, 0, stream>>>(N, C, inv_avg, m.spec.gated, aggs + (size_t)t * feat,
@@ -743,13 +762,26 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
     for (long long e0 = 0; e0 < E; e0 += coh, ++ci) {
       const long long e1 = std::min(E, e0 + coh), n = e1 - e0;
       const int grid = grid_for(n, eb.y);
-      { Scope sc_("bwd_prep", stream); k_bwd_prep<<<grid, eb, (size_t)eb.y * NDBLK * 4, stream>>>(e0, e1, C, g->recv, g->send, rr.inv, D, R, xt, gS, XT, XTlo,
+      { Scope sc_("bwd_prep", stream); k_bwd_prep<<<grid, eb, (size_t)eb.y * NDBLK * 4, stream>>>(e0, e1, C, t == 0, g->recv, g->send, rr.inv, D, R, xt, gS, XT, XTlo,
                                                                   GY, GYhi, GYlo); }
-      So2Part parts[2] = {{am_xt.get(n), &m.bmaps_fwd[t], Y}, {am_gy.get(n), &m.bmaps_bwd[t], GXT}};
-      st = so2_product(m, n, parts, 2, counter, stream);
+      if (t == 0) {
+        // degree-0 input: y needs only the m = 0 block's first C input columns, and only the
+        // degree-0 part of dE/dx~ is used (the radial scale of l = 0)
+        const So2AMaps* ax = am_xt.get(n);
+        const So2AMaps* ag = am_gy.get(n);
+        const MapPair& f0 = m.bmaps_fwd[t].blk[0];
+        const MapPair& b0 = m.b0_bwd_narrow[t];
+        GemmSub subs[2] = {{&ax->hi, &ax->lo, &f0.hi, &f0.lo, 0, C, 4 * C, 0, Y},
+                           {&ag->hi, &ag->lo, &b0.hi, &b0.lo, 0, 4 * C, C, 0, GXT}};
+        Scope sc_("so2_tc", stream);
+        st = tc_group(n, 16 * C, subs, 2, counter, stream);
+      } else {
+        So2Part parts[2] = {{am_xt.get(n), &m.bmaps_fwd[t], Y}, {am_gy.get(n), &m.bmaps_bwd[t], GXT}};
+        st = so2_product(m, n, parts, 2, counter, stream);
+      }
       if (st != EMP_OK) return st;
       const size_t smem = (size_t)eb.y * NDBLK * 4 + (size_t)eb.y * 2 * (C / 32) * 4;
-      { Scope sc_("bwd_edge", stream); k_bwd_edge<<<grid, eb, smem, stream>>>(e0, e1, C, t > 0, g->send, rr.inv, g->vec, D, R, xt, Y, GY, GXT, XT, gRhi, gRlo, g_r); }
+      { Scope sc_("bwd_edge", stream); k_bwd_edge<<<grid, eb, smem, stream>>>(e0, e1, C, t > 0, t == 0, g->send, rr.inv, g->vec, D, R, xt, Y, GY, GXT, XT, gRhi, gRlo, g_r); }
       if (t > 0) {
         dim3 sg(std::min<long long>(n, 2048), C / 32);
         { Scope sc_("sender_scatter", stream); k_sender_scatter<<<sg, 32, 0, stream>>>(e0, e1, C, ci, g->send, perm, seg, nseg, XT, gxb); }
