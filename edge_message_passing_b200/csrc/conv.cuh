@@ -546,12 +546,43 @@ __global__ void k_gate_bwd(int N, int C, float inv_avg, int gated, const float* 
 }
 
 // per edge: XT = R (.) D x_send (recomputed) and GY = D gS[recv] (edge-frame output gradient)
-__global__ void k_bwd_prep(long long e0, long long e1, int C, int scalar_in, const int* __restrict__ recv,
-                           const int* __restrict__ send, const int* __restrict__ rrow, const float* __restrict__ D,
-                           const float* __restrict__ R,
-                           const float* __restrict__ x, const float* __restrict__ gS, float* __restrict__ XT,
-                           float* __restrict__ XTlo, float* __restrict__ GY, float* __restrict__ GYhi,
-                           float* __restrict__ GYlo) {
+// degree-L block of one edge and channel: rotate v (global frame, stride C) by D^L into the
+// edge frame; optionally scale by Rl; write fp32 and/or the 3xTF32 split into m-major columns
+template <int L>
+__device__ __forceinline__ void rotate_write_degree(const float* __restrict__ Dr, const float* __restrict__ v, int C,
+                                                    float Rl, float* __restrict__ f32, float* __restrict__ hi,
+                                                    float* __restrict__ lo) {
+  constexpr int W = 2 * L + 1, O = L * L;
+  const float* B = Dr + dblk_off(L);
+  float a[W];
+#pragma unroll
+  for (int n = 0; n < W; ++n) a[n] = v[(O + n) * C];
+#pragma unroll
+  for (int m = 0; m < W; ++m) {
+    float u = 0.f;
+#pragma unroll
+    for (int n = 0; n < W; ++n) u = fmaf(B[m * W + n], a[n], u);
+    u *= Rl;
+    const int col = col_of_k(O + m) * C;
+    if (f32) f32[col] = u;
+    if (hi) {
+      const float h = tf32_rna(u);
+      hi[col] = h;
+      lo[col] = tf32_rna(u - h);
+    }
+  }
+}
+
+// per edge: XT = R (.) D x_send (recomputed, split) and GY = D gS[recv] (edge-frame output gradient,
+// fp32 and split).  scalar_in: x has degree 0 only, so only the (0,0) column of XT is non-zero and
+// only the m = 0 block of GY enters a product.
+__global__ void __launch_bounds__(256, 4) k_bwd_prep(long long e0, long long e1, int C, int scalar_in,
+                                                     const int* __restrict__ recv, const int* __restrict__ send,
+                                                     const int* __restrict__ rrow, const float* __restrict__ D,
+                                                     const float* __restrict__ R, const float* __restrict__ x,
+                                                     const float* __restrict__ gS, float* __restrict__ XT,
+                                                     float* __restrict__ XTlo, float* __restrict__ GY,
+                                                     float* __restrict__ GYhi, float* __restrict__ GYlo) {
   extern __shared__ __align__(16) float sD[];
   const int c = threadIdx.x, row = threadIdx.y, EPB = blockDim.y;
   const long long n = e1 - e0;
@@ -565,39 +596,34 @@ __global__ void k_bwd_prep(long long e0, long long e1, int C, int scalar_in, con
     __syncthreads();
     if (!ok) continue;
     const float* Dr = sD + row * NDBLK;
-    const int j = send[e], i = recv[e];
-    const size_t ro = (size_t)el * 16 * C;
-    float v[16], u[16];
+    const size_t ro = (size_t)el * 16 * C + c;
     const size_t rr = rrow ? (size_t)rrow[e] : (size_t)e;
-    if (scalar_in) {
-      const float t = R[rr * 4 * C + c] * x[(size_t)j * 16 * C + c], h = tf32_rna(t);
-      XT[ro + c] = h;
-      XTlo[ro + c] = tf32_rna(t - h);
-    } else {
-#pragma unroll
-      for (int k = 0; k < 16; ++k) v[k] = x[((size_t)j * 16 + k) * C + c];
-      rotate16<false>(Dr, v, u);
-      float Rv[4];
-#pragma unroll
-      for (int l = 0; l < 4; ++l) Rv[l] = R[rr * 4 * C + l * C + c];
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const float t = Rv[deg_of(k)] * u[k], h = tf32_rna(t);
-        XT[ro + col_of_k(k) * C + c] = h;
-        XTlo[ro + col_of_k(k) * C + c] = tf32_rna(t - h);
-      }
+    const float* Rr = R + rr * 4 * C + c;
+    const float* xs = x + (size_t)send[e] * 16 * C + c;
+    const float* gs = gS + (size_t)recv[e] * 16 * C + c;
+    rotate_write_degree<0>(Dr, xs, C, Rr[0], nullptr, XT + ro, XTlo + ro);
+    if (!scalar_in) {
+      rotate_write_degree<1>(Dr, xs, C, Rr[C], nullptr, XT + ro, XTlo + ro);
+      rotate_write_degree<2>(Dr, xs, C, Rr[2 * C], nullptr, XT + ro, XTlo + ro);
+      rotate_write_degree<3>(Dr, xs, C, Rr[3 * C], nullptr, XT + ro, XTlo + ro);
     }
+    // with a degree-0 input only the m = 0 block of g_y (its first 4C columns) is split
+    rotate_write_degree<0>(Dr, gs, C, 1.f, GY + ro, GYhi + ro, GYlo + ro);
+    if (!scalar_in) {
+      rotate_write_degree<1>(Dr, gs, C, 1.f, GY + ro, GYhi + ro, GYlo + ro);
+      rotate_write_degree<2>(Dr, gs, C, 1.f, GY + ro, GYhi + ro, GYlo + ro);
+      rotate_write_degree<3>(Dr, gs, C, 1.f, GY + ro, GYhi + ro, GYlo + ro);
+    } else {
+      rotate_write_degree<1>(Dr, gs, C, 1.f, GY + ro, nullptr, nullptr);
+      rotate_write_degree<2>(Dr, gs, C, 1.f, GY + ro, nullptr, nullptr);
+      rotate_write_degree<3>(Dr, gs, C, 1.f, GY + ro, nullptr, nullptr);
+      // the m = 0 entries of degrees 1..3 are in the first block: split them too
 #pragma unroll
-    for (int k = 0; k < 16; ++k) v[k] = gS[((size_t)i * 16 + k) * C + c];
-    rotate16<false>(Dr, v, u);
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      GY[ro + col_of_k(k) * C + c] = u[k];
-      // with a scalar-only input only the m = 0 block of g_y enters a product
-      if (!scalar_in || col_of_k(k) < 4) {
-        const float h = tf32_rna(u[k]);
-        GYhi[ro + col_of_k(k) * C + c] = h;
-        GYlo[ro + col_of_k(k) * C + c] = tf32_rna(u[k] - h);
+      for (int l = 1; l < 4; ++l) {
+        const int col = col_of(l, 0) * C;
+        const float u = GY[ro + col], h = tf32_rna(u);
+        GYhi[ro + col] = h;
+        GYlo[ro + col] = tf32_rna(u - h);
       }
     }
   }
@@ -681,7 +707,7 @@ __device__ __forceinline__ void bwd_edge_degree(const float* __restrict__ Dr, co
   }
 }
 
-__global__ void __launch_bounds__(256, 2) k_bwd_edge(long long e0, long long e1, int C, int need_gx, int scalar_in,
+__global__ void __launch_bounds__(256, 3) k_bwd_edge(long long e0, long long e1, int C, int need_gx, int scalar_in,
                                                      const int* __restrict__ send, const int* __restrict__ rrow,
                                                      const float* __restrict__ vec,
                                                      const float* __restrict__ D, const float* __restrict__ R,
@@ -720,12 +746,15 @@ __global__ void __launch_bounds__(256, 2) k_bwd_edge(long long e0, long long e1,
       bwd_edge_degree<0>(Dr, xs, yr, gyr, gxr, Rr[0], C, c, need_gx, gsr, gr, bx, by, scalar_in != 0);
       gHi[0] = tf32_rna(gr);
       gLo[0] = tf32_rna(gr - tf32_rna(gr));
+      asm volatile("" ::: "memory");   // keep the degree blocks' loads apart (register pressure)
       bwd_edge_degree<1>(Dr, xs, yr, gyr, gxr, Rr[C], C, c, need_gx, gsr, gr, bx, by, scalar_in != 0);
       gHi[C] = tf32_rna(gr);
       gLo[C] = tf32_rna(gr - tf32_rna(gr));
+      asm volatile("" ::: "memory");   // keep the degree blocks' loads apart (register pressure)
       bwd_edge_degree<2>(Dr, xs, yr, gyr, gxr, Rr[2 * C], C, c, need_gx, gsr, gr, bx, by, scalar_in != 0);
       gHi[2 * C] = tf32_rna(gr);
       gLo[2 * C] = tf32_rna(gr - tf32_rna(gr));
+      asm volatile("" ::: "memory");   // keep the degree blocks' loads apart (register pressure)
       bwd_edge_degree<3>(Dr, xs, yr, gyr, gxr, Rr[3 * C], C, c, need_gx, gsr, gr, bx, by, scalar_in != 0);
       gHi[3 * C] = tf32_rna(gr);
       gLo[3 * C] = tf32_rna(gr - tf32_rna(gr));

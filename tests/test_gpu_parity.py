@@ -212,3 +212,50 @@ def test_radial_chain_ragged_and_empty():
     e = torch.empty((0, 4, 32), device="cuda")
     kc, y0, _ = emp.mp_radial_chain(ch, e)
     assert kc.shape == (0, 25)
+
+
+# ------------------------------------------------------------------ full-size workloads
+def _stored_oracle(name):
+    path = os.path.join(GOLD, f"{name}_oracle.npz")
+    if not os.path.exists(path):
+        pytest.skip(f"{path} not generated (tests/golden/make_oracle_refs.py)")
+    return np.load(path)
+
+
+@pytest.mark.parametrize("name", ["n512_diamond", "n4096_diamond", "ternary_n2000"])
+def test_energy_forces_full_size_against_stored_oracle(name):
+    """The benchmark workloads at full size, in the launch configuration bench.py times."""
+    ref = _stored_oracle(name)
+    w = synth.workload(name)
+    st = w.structure
+    g = _graph(st, w.spec.cutoff)
+    assert g.n_edges == int(ref["n_edges"])
+    model = emp.Model(w.spec, w.weights)
+    e, f, v, ea = emp.mp_energy_forces(model, g, _cuda(st.species), virial=True, atom_energy=True)
+    E = float(e.cpu().numpy()[0])
+    F = f.cpu().numpy()
+    rE, rF = float(ref["energy"]), ref["forces"]
+    assert abs(E - rE) <= 1e-5 * abs(rE), (E, rE)
+    assert np.abs(F - rF).max() <= 1e-4 * np.abs(rF).max()
+    assert np.abs(ea.cpu().numpy() - ref["atom_energy"]).max() <= 1e-5 * np.abs(ref["atom_energy"]).max()
+    assert np.abs(v.cpu().numpy() - ref["virial"]).max() <= 1e-4 * np.abs(ref["virial"]).max()
+    assert emp.last_device_error() == 0
+
+
+def test_single_layer_n4096_sampled_receivers():
+    """Full-size single layer with random full features (all degrees): the oracle computes the
+    aggregates of a sample of receivers from their own edges."""
+    w = synth.workload("n4096_diamond")
+    st = w.structure
+    g = _graph(st)
+    ref_g = onl.brute_force(st.pos, st.box, 6.0)
+    x = synth.random_features(st.pos.shape[0], w.spec.C, seed=8)
+    model = emp.Model(w.spec, w.weights)
+    agg = emp.mp_forward(model, g, 1, _cuda(st.species), _cuda(x)).cpu().numpy()
+    rng = np.random.default_rng(3)
+    sample = np.sort(rng.choice(st.pos.shape[0], 24, replace=False))
+    for i in sample:
+        sl = slice(int(ref_g.recv_off[i]), int(ref_g.recv_off[i + 1]))
+        ref = omodel.single_layer(w.spec, w.weights, 1, x, ref_g.recv[sl], ref_g.send[sl], ref_g.r[sl], st.species,
+                                  st.pos.shape[0])[i]
+        assert np.abs(agg[i] - ref).max() <= 2e-5 * np.abs(ref).max()
