@@ -261,6 +261,12 @@ def run_ours(args):
 
     launches0 = emp.launch_count()
     with ClockSampler(dev) as clk:
+        # let the sampler start polling before the timed steps (its start-up stalls the driver)
+        for _ in range(2):
+            step(pos)
+        torch.cuda.synchronize()
+        time.sleep(1.0)
+        launches0 = emp.launch_count()
         times, _ = timed_steps(False)
         launches = emp.launch_count() - launches0
         # the same steps again with CUDA events recorded around every library launch

@@ -592,9 +592,9 @@ int mp_model_create(const emp_model_spec* spec, const float* weights, size_t n_f
   m->w3t_maps.resize(T * m->n_pairs);
   for (size_t q = 0; q < T * m->n_pairs; ++q) {
     const size_t wo = q * m->w3_stride();
-    if (make_pair(&m->w3_maps[q], m->w3_hi + wo, m->w3_lo + wo, 4 * C, 64, 64, (int)std::min<size_t>(4 * C, 256)) !=
-            EMP_OK ||
-        make_pair(&m->w3t_maps[q], m->w3t_hi + wo, m->w3t_lo + wo, 64, 4 * (int)C, 4 * (int)C, 64) != EMP_OK)
+    if (make_pair(&m->w3_maps[q], m->w3_hi + wo, m->w3_lo + wo, 4 * C, 64, 64, tc::b_box_rows(4 * (int)C)) != EMP_OK ||
+        make_pair(&m->w3t_maps[q], m->w3t_hi + wo, m->w3t_lo + wo, 64, 4 * (int)C, 4 * (int)C, tc::b_box_rows(64)) !=
+            EMP_OK)
       return fail(EMP_ERR_CUDA);
   }
   m->bmaps_fwd.resize(T);
@@ -603,7 +603,7 @@ int mp_model_create(const emp_model_spec* spec, const float* weights, size_t n_f
   for (size_t t = 0; t < T; ++t) {
     const size_t off = t * m->so2_stride();
     if (make_pair(&m->b0_bwd_narrow[t], m->so2_bwd_hi + off, m->so2_bwd_lo + off, 4 * C, 4 * (int)C, 4 * (int)C,
-                  (int)std::min<size_t>(C, 256)) != EMP_OK)
+                  tc::b_box_rows((int)C)) != EMP_OK)
       return fail(EMP_ERR_CUDA);
   }
   for (size_t t = 0; t < T; ++t) {

@@ -11,13 +11,16 @@
 // the 4 m-blocks of the cohort; the backward groups the 4 recomputed forward
 // blocks with the 4 transposed blocks (8 sub-problems, two A operands).
 //
-// Persistent kernel: one CTA per SM takes 128 x 256 output tiles from a shared
-// atomic counter (tiles ordered by decreasing K).  Warp 0 issues TMA loads (64-byte swizzle, 16 fp32 of K per row) into
-// a 4-stage ring; warp 1 issues tcgen05.mma (one thread) into one of two TMEM
-// accumulators (2 x 256 columns); warps 2..5 drain the other accumulator with
-// tcgen05.ld and store FP32 rows, so the epilogue of a tile overlaps the next
-// tile's MMAs.  Every mbarrier wait is bounded: on timeout the CTA records a
-// device error, stops, waits (bounded) for its own copies and MMAs and frees TMEM.
+// Persistent kernel on CTA pairs (clusters of 2, cta_group::2): each pair computes
+// 256 x 256 output tiles taken from a shared atomic counter (tiles ordered by
+// decreasing K).  In each CTA warp 0 issues TMA loads (64-byte swizzle, 16 fp32 of
+// K per row) of its 128 A rows and its half of the B rows into a 6-stage ring; the
+// even CTA's warp 1 issues tcgen05.mma (one thread) into one of two TMEM
+// accumulators (2 x 256 columns) in both CTAs; warps 2..5 of each CTA drain its
+// other accumulator with tcgen05.ld and store FP32 rows, so the epilogue of a tile
+// overlaps the next tile's MMAs.  Every mbarrier wait is bounded: on timeout the
+// CTA records a device error, stops, waits (bounded) for its own copies and MMAs
+// and frees TMEM.
 #pragma once
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -30,16 +33,12 @@ namespace tc {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 16;                 // fp32 elements per 64-byte swizzled row
-constexpr int ST = 4;
 constexpr int THREADS = 192;
 constexpr int MAXSUB = 8;
 constexpr int TMEM_COLS = 512;         // two 128 x 256 fp32 accumulators
 constexpr long long TIMEOUT_CYCLES = 4000000000ll;   // ~2 s at 1.9 GHz
 
 constexpr int A_BYTES = BM * BK * 4;   // 8 KB
-constexpr int B_BYTES = BN * BK * 4;   // 16 KB
-constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;   // 48 KB
-constexpr int SMEM_BYTES = ST * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers, tile ring*/;
 
 struct Group {
   int M, nsub, mtiles;
@@ -109,22 +108,6 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr) {
          ((uint64_t)1 << 46) | ((uint64_t)4 << 61);
 }
 
-// instruction descriptor: D f32, A/B tf32, both K-major, M = 128, N = n
-__host__ __device__ constexpr uint32_t idesc_for(int n) {
-  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-}
-
-__device__ __forceinline__ void mma_tf32(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accum) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n"
-      ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(accum));
-}
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
 __device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -148,56 +131,138 @@ struct TileInfo {
   int m0, sub, n0;
 };
 
-// tile t: sub-problem by prefix, then m-major within it (the n-tiles of one m-tile
-// are consecutive, so they share the A tile in L2)
-__device__ __forceinline__ TileInfo tile_info(const Group& g, int t) {
+constexpr int TQ = 4;    // depth of the tile-index ring from the scheduler to the MMA and epilogue warps
+
+// The products run on CTA pairs (cta_group::2); B tensor maps hold half-height tiles.
+__host__ __device__ constexpr int b_box_rows(int n) { return (n < BN ? n : BN) / 2; }
+
+// ------------------------------------------------------------------ 2-SM form (cta_group::2)
+// A pair of CTAs (a cluster of 2 on neighbouring SMs) computes a 256 x bn tile with
+// one tcgen05.mma.cta_group::2 stream issued by the even CTA (the leader): each CTA
+// stages its own 128 rows of A and its own half (bn/2 rows) of B, so each SM reads
+// half the B bytes per flop that the 1-SM form does.  Both CTAs' TMA loads complete
+// on the leader's full barrier; the MMA completion is multicast to both CTAs' stage
+// and accumulator barriers; the leader takes tiles from the counter and publishes
+// each index to both CTAs (distributed shared memory + remote mbarrier arrive).
+constexpr int ST2 = 6;
+constexpr int B2_BYTES = (BN / 2) * BK * 4;            // 8 KB: half of a 256-row B tile
+constexpr int STAGE2 = 2 * A_BYTES + 2 * B2_BYTES;     // 32 KB per CTA
+constexpr int SMEM2 = ST2 * STAGE2 + 1024 + 512;
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t local_addr, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(local_addr), "r"(rank));
+  return a;
+}
+__device__ __forceinline__ void remote_arrive(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void remote_store(uint32_t cluster_addr, int v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ int remote_load(uint32_t cluster_addr) {
+  int v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait_cluster(bar, parity)) {
+    if (clock64() - t0 > TIMEOUT_CYCLES) {
+      set_device_error(DEV_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tma_load_pair(void* dst, const CUtensorMap* map, uint32_t leader_bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void mma_tf32_pair(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n"
+      ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(accum));
+}
+// arrive (once) on the barrier at this address in both CTAs of the pair when the issued MMAs are done
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+      ::"r"(smem_u32(bar)), "h"((uint16_t)3)
+      : "memory");
+}
+__host__ __device__ constexpr uint32_t idesc_pair(int n) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+}
+
+__device__ __forceinline__ TileInfo tile_info2(const Group& g, int t) {
   TileInfo ti;
   int s = 0;
   while (s < g.nsub - 1 && t >= g.first[s + 1]) ++s;
   const int r = t - g.first[s];
   ti.sub = s;
-  ti.m0 = (r / g.ntiles[s]) * BM;
+  ti.m0 = (r / g.ntiles[s]) * (2 * BM);
   ti.n0 = (r % g.ntiles[s]) * g.bn[s];
   return ti;
 }
 
-constexpr int TQ = 4;    // depth of the tile-index ring from the scheduler to the MMA and epilogue warps
-
-__global__ void __launch_bounds__(THREADS, 1) k_so2_tc(const __grid_constant__ Group g, const __grid_constant__ Maps maps,
-                                                       int total_tiles) {
-  // Tiles are handed out dynamically (an atomic counter over tiles ordered by
-  // decreasing K): the TMA warp takes the next tile and passes its index to the
-  // MMA and epilogue warps through a TQ-deep ring; an index >= total ends a role.
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    k_so2_tc2(const __grid_constant__ Group g, const __grid_constant__ Maps maps, int total_tiles) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * STAGE_BYTES);
-  uint64_t* empty = full + ST;
-  uint64_t* acc_full = empty + ST;       // [2]
-  uint64_t* acc_empty = acc_full + 2;    // [2]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST2 * STAGE2);   // [ST2] (the leader's are used)
+  uint64_t* empty = full + ST2;                                        // [ST2]
+  uint64_t* acc_full = empty + ST2;                                    // [2]
+  uint64_t* acc_empty = acc_full + 2;                                  // [2] (the leader's are used)
   uint64_t* drain = acc_empty + 2;
-  uint64_t* tq_full = drain + 1;         // [TQ]
-  uint64_t* tq_empty = tq_full + TQ;     // [TQ]
-  int* tq = reinterpret_cast<int*>(tq_empty + TQ);   // [TQ] tile indices
+  uint64_t* tq_full = drain + 1;                                       // [TQ]
+  uint64_t* tq_empty = tq_full + TQ;                                   // [TQ] (the leader's are used)
+  int* tq = reinterpret_cast<int*>(tq_empty + TQ);                     // [TQ]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tq + TQ);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-  int* issued = abort_flag + 1;          // k-chunks whose loads were issued
-  int* consumed = issued + 1;            // k-chunks whose full barrier completed
+  int* issued = abort_flag + 1;
+  int* consumed = issued + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < ST; ++s) {
+    for (int s = 0; s < ST2; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+      mbar_init(&acc_empty[b], 8);        // 4 epilogue warps in each CTA
     }
     mbar_init(drain, 1);
     for (int j = 0; j < TQ; ++j) {
       mbar_init(&tq_full[j], 1);
-      mbar_init(&tq_empty[j], 5);        // the MMA thread and one thread per epilogue warp
+      mbar_init(&tq_empty[j], 10);        // leader MMA + 4 leader epilogue warps + peer producer + 4 peer warps
     }
     *abort_flag = 0;
     *issued = 0;
@@ -205,44 +270,60 @@ __global__ void __launch_bounds__(THREADS, 1) k_so2_tc(const __grid_constant__ G
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"((uint32_t)TMEM_COLS));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
   }
   fence_before();
   __syncthreads();
+  cluster_sync();
   fence_after();
   const uint32_t tmem = *tmem_slot;
   volatile int* vabort = abort_flag;
+  // addresses in the leader CTA (barriers the peer arrives on)
+  const uint32_t full_l = map_to_rank(smem_u32(full), 0);
+  const uint32_t acc_empty_l = map_to_rank(smem_u32(acc_empty), 0);
+  const uint32_t tq_empty_l = map_to_rank(smem_u32(tq_empty), 0);
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- scheduler + TMA producer
     int it = 0;
     for (int j = 0;; ++j) {
       const int slot = j % TQ;
-      if (j >= TQ && !mbar_wait(&tq_empty[slot], ((j / TQ) - 1) & 1)) { *vabort = 1; break; }
-      const int t = *vabort ? total_tiles : atomicAdd(g.counter, 1);
-      tq[slot] = t;
-      mbar_arrive(&tq_full[slot]);
+      int t;
+      if (leader) {
+        if (j >= TQ && !mbar_wait_cluster(&tq_empty[slot], ((j / TQ) - 1) & 1)) { *vabort = 1; t = total_tiles; }
+        else t = *vabort ? total_tiles : atomicAdd(g.counter, 1);
+        tq[slot] = t;
+        remote_store(map_to_rank(smem_u32(&tq[slot]), 1), t);
+        mbar_arrive(&tq_full[slot]);
+        remote_arrive(map_to_rank(smem_u32(&tq_full[slot]), 1));
+      } else {
+        if (!mbar_wait_cluster(&tq_full[slot], (j / TQ) & 1)) { *vabort = 1; break; }
+        t = tq[slot];
+        remote_arrive(tq_empty_l + (uint32_t)(slot * 8));
+      }
       if (t >= total_tiles) break;
-      const TileInfo ti = tile_info(g, t);
+      const TileInfo ti = tile_info2(g, t);
       const int a = g.a_idx[ti.sub], b = g.b_idx[ti.sub];
       const int nk = g.K[ti.sub] / BK;
+      const int bh = g.bn[ti.sub] / 2;                       // this CTA's B rows
       for (int kc = 0; kc < nk; ++kc, ++it) {
-        const int s = it % ST;
-        if (it >= ST && !mbar_wait(&empty[s], ((it / ST) - 1) & 1)) { *vabort = 1; break; }
+        const int s = it % ST2;
+        if (it >= ST2 && !mbar_wait(&empty[s], ((it / ST2) - 1) & 1)) { *vabort = 1; break; }
         if (*vabort) break;
-        unsigned char* st = smem + s * STAGE_BYTES;
-        mbar_expect_tx(&full[s], 2 * A_BYTES + 2 * g.bn[ti.sub] * BK * 4);
-        tma_load(st, &maps.a_hi[a], &full[s], g.acol[ti.sub] + kc * BK, ti.m0);
-        tma_load(st + A_BYTES, &maps.a_lo[a], &full[s], g.acol[ti.sub] + kc * BK, ti.m0);
-        tma_load(st + 2 * A_BYTES, &maps.b_hi[b], &full[s], kc * BK, ti.n0);
-        tma_load(st + 2 * A_BYTES + B_BYTES, &maps.b_lo[b], &full[s], kc * BK, ti.n0);
+        unsigned char* st = smem + s * STAGE2;
+        if (leader) mbar_expect_tx(&full[s], 2 * (2 * A_BYTES + 2 * bh * BK * 4));
+        const uint32_t fb = full_l + (uint32_t)(s * 8);
+        tma_load_pair(st, &maps.a_hi[a], fb, g.acol[ti.sub] + kc * BK, ti.m0 + (int)rank * BM);
+        tma_load_pair(st + A_BYTES, &maps.a_lo[a], fb, g.acol[ti.sub] + kc * BK, ti.m0 + (int)rank * BM);
+        tma_load_pair(st + 2 * A_BYTES, &maps.b_hi[b], fb, kc * BK, ti.n0 + (int)rank * bh);
+        tma_load_pair(st + 2 * A_BYTES + B2_BYTES, &maps.b_lo[b], fb, kc * BK, ti.n0 + (int)rank * bh);
         *issued = it + 1;
       }
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------------------------------------------------------- MMA issuer
+  } else if (warp == 1 && lane == 0 && leader) {
+    // ---------------------------------------------------------------- MMA issuer (leader only)
     int it = 0;
     bool ok = true;
     for (int i = 0;; ++i) {
@@ -251,53 +332,56 @@ __global__ void __launch_bounds__(THREADS, 1) k_so2_tc(const __grid_constant__ G
       const int t = tq[slot];
       mbar_arrive(&tq_empty[slot]);
       if (t >= total_tiles) break;
-      const TileInfo ti = tile_info(g, t);
+      const TileInfo ti = tile_info2(g, t);
       const int nk = g.K[ti.sub] / BK;
       const int buf = i & 1;
-      if (i >= 2 && !mbar_wait(&acc_empty[buf], ((i >> 1) - 1) & 1)) { ok = false; break; }
+      if (i >= 2 && !mbar_wait_cluster(&acc_empty[buf], ((i >> 1) - 1) & 1)) { ok = false; break; }
       fence_after();
       const uint32_t d = tmem + (uint32_t)(buf * BN);
-      const uint32_t idesc = idesc_for(g.bn[ti.sub]);
+      const uint32_t idesc = idesc_pair(g.bn[ti.sub]);
       for (int kc = 0; kc < nk; ++kc, ++it) {
-        const int s = it % ST;
-        if (!mbar_wait(&full[s], (it / ST) & 1)) { ok = false; break; }
+        const int s = it % ST2;
+        if (!mbar_wait(&full[s], (it / ST2) & 1)) { ok = false; break; }
         *consumed = it + 1;
         fence_after();
-        const uint32_t a_hi = smem_u32(smem + s * STAGE_BYTES);
+        const uint32_t a_hi = smem_u32(smem + s * STAGE2);
         const uint32_t a_lo = a_hi + A_BYTES;
         const uint32_t b_hi = a_hi + 2 * A_BYTES;
-        const uint32_t b_lo = b_hi + B_BYTES;
+        const uint32_t b_lo = b_hi + B2_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BK / 8; ++kk) {
-          const uint32_t off = kk * 32;   // 8 fp32 of K = 32 bytes inside the swizzled row
-          mma_tf32(d, sdesc(a_lo + off), sdesc(b_hi + off), idesc, (kc | kk) ? 1u : 0u);
-          mma_tf32(d, sdesc(a_hi + off), sdesc(b_lo + off), idesc, 1u);
-          mma_tf32(d, sdesc(a_hi + off), sdesc(b_hi + off), idesc, 1u);
+          const uint32_t off = kk * 32;
+          mma_tf32_pair(d, sdesc(a_lo + off), sdesc(b_hi + off), idesc, (kc | kk) ? 1u : 0u);
+          mma_tf32_pair(d, sdesc(a_hi + off), sdesc(b_lo + off), idesc, 1u);
+          mma_tf32_pair(d, sdesc(a_hi + off), sdesc(b_hi + off), idesc, 1u);
         }
-        mma_commit(&empty[s]);
+        mma_commit_pair(&empty[s]);
       }
       if (!ok) break;
-      mma_commit(&acc_full[buf]);
+      mma_commit_pair(&acc_full[buf]);
     }
     if (!ok) *vabort = 1;
-    mma_commit(drain);                  // completes once every MMA this thread issued is done
+    mma_commit_pair(drain);
     mbar_wait(drain, 0);
   } else if (warp >= 2) {
-    // ---------------------------------------------------------------- epilogue
-    const int q = warp & 3;               // TMEM lane quarter this warp may access
+    // ---------------------------------------------------------------- epilogue (both CTAs: own 128 rows)
+    const int q = warp & 3;
     const int row = q * 32 + lane;
     for (int i = 0;; ++i) {
       const int slot = i % TQ;
-      if (!mbar_wait(&tq_full[slot], (i / TQ) & 1)) { *vabort = 1; break; }
+      if (!mbar_wait_cluster(&tq_full[slot], (i / TQ) & 1)) { *vabort = 1; break; }
       const int t = tq[slot];
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tq_empty[slot]);
+      if (lane == 0) {
+        if (leader) mbar_arrive(&tq_empty[slot]);
+        else remote_arrive(tq_empty_l + (uint32_t)(slot * 8));
+      }
       if (t >= total_tiles) break;
-      const TileInfo ti = tile_info(g, t);
+      const TileInfo ti = tile_info2(g, t);
       const int buf = i & 1;
       if (!mbar_wait(&acc_full[buf], (i >> 1) & 1)) { *vabort = 1; break; }
       fence_after();
-      const int m = ti.m0 + row;
+      const int m = ti.m0 + (int)rank * BM + row;
       const int N = g.N[ti.sub], bn = g.bn[ti.sub];
       float* orow = g.out[ti.sub] + (size_t)m * g.ldc + g.ccol[ti.sub] + ti.n0;
 #pragma unroll 1
@@ -312,19 +396,26 @@ __global__ void __launch_bounds__(THREADS, 1) k_so2_tc(const __grid_constant__ G
       }
       fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      if (lane == 0) {
+        if (leader) mbar_arrive(&acc_empty[buf]);
+        else remote_arrive(acc_empty_l + (uint32_t)(buf * 8));
+      }
     }
   }
   fence_before();
   __syncthreads();
-  if (threadIdx.x == 0 && *vabort) {
-    // let loads still in flight land before the shared memory is released
-    for (int it = *consumed; it < *issued; ++it) mbar_wait(&full[it % ST], (it / ST) & 1);
+  cluster_sync();
+  if (threadIdx.x == 0 && leader && *vabort) {
+    // let loads of either CTA still in flight land (they complete on the leader's barriers)
+    const int peer_issued = remote_load(map_to_rank(smem_u32(issued), 1));
+    const int last = max(*issued, peer_issued);
+    for (int it = *consumed; it < last; ++it) mbar_wait(&full[it % ST2], (it / ST2) & 1);
   }
   __syncthreads();
+  cluster_sync();
   if (warp == 1) {
     fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)TMEM_COLS));
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)TMEM_COLS));
   }
 }
 
@@ -369,7 +460,7 @@ inline int num_sms() {
 
 inline int so2_tc_init() {
   if (!tc::encode_fn()) return EMP_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(tc::k_so2_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES) != cudaSuccess)
+  if (cudaFuncSetAttribute(tc::k_so2_tc2, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM2) != cudaSuccess)
     return EMP_ERR_CUDA;
   return EMP_OK;
 }
@@ -394,7 +485,7 @@ inline int tc_group(long long M, int ldc, const GemmSub* subs, int nsub, int* co
   g.M = (int)M;
   g.ldc = ldc;
   g.nsub = nsub;
-  g.mtiles = (int)((M + tc::BM - 1) / tc::BM);
+  g.mtiles = (int)((M + 2 * tc::BM - 1) / (2 * tc::BM));
   g.counter = counter;
   int ord[tc::MAXSUB];
   for (int i = 0; i < nsub; ++i) ord[i] = i;
@@ -404,7 +495,7 @@ inline int tc_group(long long M, int ldc, const GemmSub* subs, int nsub, int* co
   long long first = 0;
   for (int q = 0; q < nsub; ++q) {
     const GemmSub& u = subs[ord[q]];
-    if (u.K % tc::BK != 0 || u.N < 16 || u.N % 16 != 0) return EMP_ERR_ARG;
+    if (u.K % tc::BK != 0 || u.N < 32 || u.N % 32 != 0) return EMP_ERR_ARG;
     int a = 0;
     while (a < na && a_seen[a] != u.a_hi) ++a;
     if (a == na) {
@@ -431,8 +522,8 @@ inline int tc_group(long long M, int ldc, const GemmSub* subs, int nsub, int* co
   if (first >= (1ll << 31)) return EMP_ERR_UNSUPPORTED;
   g.first[nsub] = (int)first;
   if (cudaMemsetAsync(counter, 0, sizeof(int), s) != cudaSuccess) return EMP_ERR_CUDA;
-  const int grid = (int)std::min<long long>(first, tc::num_sms());
-  tc::k_so2_tc<<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(g, maps, (int)first);
+  const int pairs = (int)std::min<long long>(first, tc::num_sms() / 2);
+  tc::k_so2_tc2<<<2 * pairs, tc::THREADS, tc::SMEM2, s>>>(g, maps, (int)first);
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
 
@@ -459,7 +550,7 @@ inline int so2_make_bmaps(So2BMaps* m, int C, const float* b_hi, const float* b_
   for (int b = 0; b < 4; ++b) {
     const int K = blk_width(b) * C;
     const size_t off = (size_t)wblk_off(b) * C * C;
-    int st = make_pair(&m->blk[b], b_hi + off, b_lo + off, K, K, K, std::min(K, tc::BN));
+    int st = make_pair(&m->blk[b], b_hi + off, b_lo + off, K, K, K, tc::b_box_rows(K));
     if (st != EMP_OK) return st;
   }
   return EMP_OK;
