@@ -182,8 +182,12 @@ class Graph:
                       _ptr(self.shift), _ptr(self.vec), self.n_edges, self.n_atoms)
 
 
-def nl_build(pos, box: Sequence[float], cutoff: float, capacity: Optional[int] = None) -> Graph:
-    """Neighbour list of device positions pos [N,3] float64 (see include/emp.h)."""
+def nl_build(pos, box: Sequence[float], cutoff: float, capacity: Optional[int] = None,
+             reuse: Optional["Graph"] = None) -> Graph:
+    """Neighbour list of device positions pos [N,3] float64 (see include/emp.h).
+
+    reuse: a Graph from an earlier call whose buffers are written again when they
+    are large enough (same atom count), instead of allocating new ones."""
     torch = _torch()
     if pos.dtype != torch.float64 or pos.dim() != 2 or pos.shape[1] != 3 or not pos.is_cuda:
         raise EmpError("pos must be a CUDA float64 tensor [N,3]")
@@ -192,11 +196,17 @@ def nl_build(pos, box: Sequence[float], cutoff: float, capacity: Optional[int] =
     L = lib()
     ws = _workspace(L.nl_workspace_bytes(N))
     cap = capacity if capacity is not None else max(256, 200 * N)
+    bufs = None
+    if reuse is not None and reuse.n_atoms == N and getattr(reuse, "_full", None) is not None:
+        bufs = reuse._full
+        cap = bufs[0].shape[0]
     for _ in range(2):
-        g = Graph(*(torch.empty(cap, dtype=torch.int32, device="cuda") for _ in range(3)),
-                  torch.empty(N + 1, dtype=torch.int32, device="cuda"),
-                  torch.empty((cap, 3), dtype=torch.int32, device="cuda"),
-                  torch.empty((cap, 3), dtype=torch.float32, device="cuda"), 0, N)
+        if bufs is None or bufs[0].shape[0] < cap:
+            bufs = (*(torch.empty(cap, dtype=torch.int32, device="cuda") for _ in range(3)),
+                    torch.empty(N + 1, dtype=torch.int32, device="cuda"),
+                    torch.empty((cap, 3), dtype=torch.int32, device="cuda"),
+                    torch.empty((cap, 3), dtype=torch.float32, device="cuda"))
+        g = Graph(*bufs, 0, N)
         p = NlParams(N, (ctypes.c_double * 3)(*[float(b) for b in box]), float(cutoff), cap)
         gc = g.c()
         ne = ctypes.c_int64(0)
@@ -204,10 +214,13 @@ def nl_build(pos, box: Sequence[float], cutoff: float, capacity: Optional[int] =
                         _stream())
         if st == -2 and ne.value > cap:           # capacity: grow once to the reported size
             cap = int(ne.value)
+            bufs = None
             continue
         _check(st, "nl_build")
         E = int(ne.value)
-        return Graph(g.recv[:E], g.send[:E], g.mirror[:E], g.recv_off, g.shift[:E], g.vec[:E], E, N)
+        out = Graph(bufs[0][:E], bufs[1][:E], bufs[2][:E], bufs[3], bufs[4][:E], bufs[5][:E], E, N)
+        out._full = bufs
+        return out
     raise EmpError("nl_build: capacity retry failed")
 
 

@@ -312,6 +312,35 @@ __global__ void __launch_bounds__(PS_THREADS) k_pair_sort(long long E, int n_spe
   }
 }
 
+// degree-L block of one edge and channel: rotate v (global frame, stride C) by D^L into the
+// edge frame; optionally scale by Rl; write fp32 and/or the 3xTF32 split into m-major columns
+template <int L>
+__device__ __forceinline__ void rotate_write_degree(const float* __restrict__ Dr, const float* __restrict__ v, int C,
+                                                    float Rl, float* __restrict__ f32, float* __restrict__ hi,
+                                                    float* __restrict__ lo) {
+  constexpr int W = 2 * L + 1, O = L * L;
+  const float* B = Dr + dblk_off(L);
+  float a[W];
+#pragma unroll
+  for (int n = 0; n < W; ++n) a[n] = v[(O + n) * C];
+#pragma unroll
+  for (int m = 0; m < W; ++m) {
+    float u = 0.f;
+#pragma unroll
+    for (int n = 0; n < W; ++n) u = fmaf(B[m * W + n], a[n], u);
+    u *= Rl;
+    const int col = col_of_k(O + m) * C;
+    if (f32) f32[col] = u;
+    if (hi) {
+      const float h = tf32_rna(u);
+      hi[col] = h;
+      lo[col] = tf32_rna(u - h);
+    }
+  }
+}
+
+constexpr int BE_CHUNK = 16;   // edges whose Wigner-D blocks are staged per barrier pair
+
 // ------------------------------------------------------------------ rotate in
 // XT[e - e0][col(k) C + c] = R_e[l(k)][c] * (D_e x_send)[k][c]  (edge frame, m-major)
 // scalar_in: the input has only degree-0 components (the first layer, whose input is the
@@ -319,41 +348,38 @@ __global__ void __launch_bounds__(PS_THREADS) k_pair_sort(long long E, int n_spe
 __global__ void k_rotate_in(long long e0, long long e1, int C, int scalar_in, const int* __restrict__ send,
                             const int* __restrict__ rrow, const float* __restrict__ D, const float* __restrict__ R,
                             const float* __restrict__ x, float* __restrict__ XT, float* __restrict__ XTlo) {
-  extern __shared__ __align__(16) float sD[];           // [EPB][84]
+  extern __shared__ __align__(16) float sD[];           // [BE_CHUNK][84]
   const int c = threadIdx.x, row = threadIdx.y, EPB = blockDim.y;
+  const int tid = row * C + c, nthr = C * EPB;
   const long long n = e1 - e0;
-  for (long long base = (long long)blockIdx.x * EPB; base < n; base += (long long)gridDim.x * EPB) {
-    const long long el = base + row;
-    const bool ok = el < n;
-    const long long e = e0 + el;
+  for (long long base = (long long)blockIdx.x * BE_CHUNK; base < n; base += (long long)gridDim.x * BE_CHUNK) {
+    const int nch = (int)min((long long)BE_CHUNK, n - base);
     __syncthreads();
-    if (ok)
-      for (int k = c; k < NDBLK; k += C) sD[row * NDBLK + k] = D[(size_t)e * NDBLK + k];
-    __syncthreads();
-    if (!ok) continue;
-    const int j = send[e];
-    if (scalar_in) {
-      const size_t rr = rrow ? (size_t)rrow[e] : (size_t)e;
-      const float v = R[rr * 4 * C + c] * x[(size_t)j * 16 * C + c], h = tf32_rna(v);
-      XT[(size_t)el * 16 * C + c] = h;
-      XTlo[(size_t)el * 16 * C + c] = tf32_rna(v - h);
-      continue;
+    {
+      const float4* src = reinterpret_cast<const float4*>(D + (size_t)(e0 + base) * NDBLK);
+      float4* dst = reinterpret_cast<float4*>(sD);
+      for (int q = tid; q < nch * (NDBLK / 4); q += nthr) dst[q] = src[q];
     }
-    float xv[16], u[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) xv[k] = x[((size_t)j * 16 + k) * C + c];
-    rotate16<false>(sD + row * NDBLK, xv, u);
-    float Rv[4];
-    const size_t rr = rrow ? (size_t)rrow[e] : (size_t)e;
-#pragma unroll
-    for (int l = 0; l < 4; ++l) Rv[l] = R[rr * 4 * C + l * C + c];
-    float* out = XT + (size_t)el * 16 * C;
-    float* olo = XTlo + (size_t)el * 16 * C;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const float v = Rv[deg_of(k)] * u[k], h = tf32_rna(v);
-      out[col_of_k(k) * C + c] = h;
-      olo[col_of_k(k) * C + c] = tf32_rna(v - h);
+    __syncthreads();
+    for (int k = row; k < nch; k += EPB) {
+      const long long el = base + k;
+      const long long e = e0 + el;
+      const int j = send[e];
+      const size_t rr = rrow ? (size_t)rrow[e] : (size_t)e;
+      if (scalar_in) {
+        const float v = R[rr * 4 * C + c] * x[(size_t)j * 16 * C + c], h = tf32_rna(v);
+        XT[(size_t)el * 16 * C + c] = h;
+        XTlo[(size_t)el * 16 * C + c] = tf32_rna(v - h);
+        continue;
+      }
+      const float* Dr = sD + k * NDBLK;
+      const size_t ro = (size_t)el * 16 * C + c;
+      const float* Rr = R + rr * 4 * C + c;
+      const float* xs = x + (size_t)j * 16 * C + c;
+      rotate_write_degree<0>(Dr, xs, C, Rr[0], nullptr, XT + ro, XTlo + ro);
+      rotate_write_degree<1>(Dr, xs, C, Rr[C], nullptr, XT + ro, XTlo + ro);
+      rotate_write_degree<2>(Dr, xs, C, Rr[2 * C], nullptr, XT + ro, XTlo + ro);
+      rotate_write_degree<3>(Dr, xs, C, Rr[3 * C], nullptr, XT + ro, XTlo + ro);
     }
   }
 }
@@ -546,33 +572,6 @@ __global__ void k_gate_bwd(int N, int C, float inv_avg, int gated, const float* 
 }
 
 // per edge: XT = R (.) D x_send (recomputed) and GY = D gS[recv] (edge-frame output gradient)
-// degree-L block of one edge and channel: rotate v (global frame, stride C) by D^L into the
-// edge frame; optionally scale by Rl; write fp32 and/or the 3xTF32 split into m-major columns
-template <int L>
-__device__ __forceinline__ void rotate_write_degree(const float* __restrict__ Dr, const float* __restrict__ v, int C,
-                                                    float Rl, float* __restrict__ f32, float* __restrict__ hi,
-                                                    float* __restrict__ lo) {
-  constexpr int W = 2 * L + 1, O = L * L;
-  const float* B = Dr + dblk_off(L);
-  float a[W];
-#pragma unroll
-  for (int n = 0; n < W; ++n) a[n] = v[(O + n) * C];
-#pragma unroll
-  for (int m = 0; m < W; ++m) {
-    float u = 0.f;
-#pragma unroll
-    for (int n = 0; n < W; ++n) u = fmaf(B[m * W + n], a[n], u);
-    u *= Rl;
-    const int col = col_of_k(O + m) * C;
-    if (f32) f32[col] = u;
-    if (hi) {
-      const float h = tf32_rna(u);
-      hi[col] = h;
-      lo[col] = tf32_rna(u - h);
-    }
-  }
-}
-
 // per edge: XT = R (.) D x_send (recomputed, split) and GY = D gS[recv] (edge-frame output gradient,
 // fp32 and split).  scalar_in: x has degree 0 only, so only the (0,0) column of XT is non-zero and
 // only the m = 0 block of GY enters a product.
@@ -707,7 +706,11 @@ __device__ __forceinline__ void bwd_edge_degree(const float* __restrict__ Dr, co
   }
 }
 
-__global__ void __launch_bounds__(256, 3) k_bwd_edge(long long e0, long long e1, int C, int need_gx, int scalar_in,
+// Edges are taken in chunks of BE_CHUNK: their Wigner-D blocks are staged with one
+// barrier pair, each row then walks its share of the chunk back to back, and the
+// per-edge torque sums are finished once per chunk.
+
+__global__ void __launch_bounds__(256, 2) k_bwd_edge(long long e0, long long e1, int C, int need_gx, int scalar_in,
                                                      const int* __restrict__ send, const int* __restrict__ rrow,
                                                      const float* __restrict__ vec,
                                                      const float* __restrict__ D, const float* __restrict__ R,
@@ -717,21 +720,26 @@ __global__ void __launch_bounds__(256, 3) k_bwd_edge(long long e0, long long e1,
                                                      float* __restrict__ gR_lo, float* __restrict__ g_r) {
   extern __shared__ __align__(16) float smem[];
   const int c = threadIdx.x, row = threadIdx.y, EPB = blockDim.y;
-  float* sD = smem;                                 // [EPB][84]
-  float* red = smem + EPB * NDBLK;                  // [EPB][2][C/32]
+  const int tid = row * C + c, nthr = C * EPB;
+  float* sD = smem;                                 // [BE_CHUNK][84]
+  float* red = smem + BE_CHUNK * NDBLK;             // [BE_CHUNK][2][C/32]
   const int nw = C / 32, warp = c >> 5, lane = c & 31;
   const long long n = e1 - e0;
-  for (long long base = (long long)blockIdx.x * EPB; base < n; base += (long long)gridDim.x * EPB) {
-    const long long el = base + row;
-    const bool ok = el < n;
-    const long long e = e0 + el;
+  for (long long base = (long long)blockIdx.x * BE_CHUNK; base < n; base += (long long)gridDim.x * BE_CHUNK) {
+    const int nch = (int)min((long long)BE_CHUNK, n - base);
     __syncthreads();
-    if (ok)
-      for (int k = c; k < NDBLK; k += C) sD[row * NDBLK + k] = D[(size_t)e * NDBLK + k];
+    {
+      const float4* src = reinterpret_cast<const float4*>(D + (size_t)(e0 + base) * NDBLK);
+      float4* dst = reinterpret_cast<float4*>(sD);
+      for (int q = tid; q < nch * (NDBLK / 4); q += nthr) dst[q] = src[q];
+    }
     __syncthreads();
-    float bx = 0.f, by = 0.f;
-    if (ok) {
-      const float* Dr = sD + row * NDBLK;
+#pragma unroll 1
+    for (int k = row; k < nch; k += EPB) {
+      const long long el = base + k;
+      const long long e = e0 + el;
+      float bx = 0.f, by = 0.f;
+      const float* Dr = sD + k * NDBLK;
       const size_t rowoff = (size_t)el * 16 * C;
       const float* xs = x + (size_t)send[e] * 16 * C + c;
       const size_t rr = rrow ? (size_t)rrow[e] : (size_t)e;
@@ -746,35 +754,34 @@ __global__ void __launch_bounds__(256, 3) k_bwd_edge(long long e0, long long e1,
       bwd_edge_degree<0>(Dr, xs, yr, gyr, gxr, Rr[0], C, c, need_gx, gsr, gr, bx, by, scalar_in != 0);
       gHi[0] = tf32_rna(gr);
       gLo[0] = tf32_rna(gr - tf32_rna(gr));
-      asm volatile("" ::: "memory");   // keep the degree blocks' loads apart (register pressure)
       bwd_edge_degree<1>(Dr, xs, yr, gyr, gxr, Rr[C], C, c, need_gx, gsr, gr, bx, by, scalar_in != 0);
       gHi[C] = tf32_rna(gr);
       gLo[C] = tf32_rna(gr - tf32_rna(gr));
-      asm volatile("" ::: "memory");   // keep the degree blocks' loads apart (register pressure)
       bwd_edge_degree<2>(Dr, xs, yr, gyr, gxr, Rr[2 * C], C, c, need_gx, gsr, gr, bx, by, scalar_in != 0);
       gHi[2 * C] = tf32_rna(gr);
       gLo[2 * C] = tf32_rna(gr - tf32_rna(gr));
-      asm volatile("" ::: "memory");   // keep the degree blocks' loads apart (register pressure)
       bwd_edge_degree<3>(Dr, xs, yr, gyr, gxr, Rr[3 * C], C, c, need_gx, gsr, gr, bx, by, scalar_in != 0);
       gHi[3 * C] = tf32_rna(gr);
       gLo[3 * C] = tf32_rna(gr - tf32_rna(gr));
-    }
-    // deterministic reduction of (bx, by) over the row's channels
+      // fixed-order reduction of (bx, by) over the warp, then per warp into shared memory
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      bx += __shfl_xor_sync(0xffffffffu, bx, o);
-      by += __shfl_xor_sync(0xffffffffu, by, o);
-    }
-    if (lane == 0) {
-      red[(row * 2 + 0) * nw + warp] = bx;
-      red[(row * 2 + 1) * nw + warp] = by;
+      for (int o = 16; o > 0; o >>= 1) {
+        bx += __shfl_xor_sync(0xffffffffu, bx, o);
+        by += __shfl_xor_sync(0xffffffffu, by, o);
+      }
+      if (lane == 0) {
+        red[(k * 2 + 0) * nw + warp] = bx;
+        red[(k * 2 + 1) * nw + warp] = by;
+      }
     }
     __syncthreads();
-    if (ok && c == 0) {
+    if (tid < nch) {
+      const int k = tid;
+      const long long e = e0 + base + k;
       float sx = 0.f, sy = 0.f;
       for (int w = 0; w < nw; ++w) {
-        sx += red[(row * 2 + 0) * nw + w];
-        sy += red[(row * 2 + 1) * nw + w];
+        sx += red[(k * 2 + 0) * nw + w];
+        sy += red[(k * 2 + 1) * nw + w];
       }
       const float vx = vec[3 * e], vy = vec[3 * e + 1], vz = vec[3 * e + 2];
       const float d2 = vx * vx + vy * vy + vz * vz;
@@ -848,7 +855,8 @@ __global__ void k_cohort_sort(long long E, int cohort, const int* __restrict__ s
   }
 }
 
-// g_x[j] += sum over the cohort's edges with sender j (ascending edge) of GXS rows
+// g_x[j] += sum over the cohort's edges with sender j (ascending edge) of GXS rows.
+// Rows are fetched four at a time and added in edge order.
 __global__ void k_sender_scatter(long long e0, long long e1, int C, int cohort_idx, const int* __restrict__ send,
                                  const int* __restrict__ perm, const int* __restrict__ seg,
                                  const int* __restrict__ nseg, const float* __restrict__ GXS,
@@ -863,10 +871,22 @@ __global__ void k_sender_scatter(long long e0, long long e1, int C, int cohort_i
     float acc[16];
 #pragma unroll
     for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-    for (int q = b; q < en; ++q) {
-      const float* g = GXS + (size_t)perm[e0 + q] * 16 * C;
+    for (int q = b; q < en; q += 4) {
+      const int cnt = min(4, en - q);
+      float v[4][16];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) acc[k] += g[k * C + c];
+      for (int u = 0; u < 4; ++u) {
+        if (u < cnt) {
+          const float* g = GXS + (size_t)perm[e0 + q + u] * 16 * C + c;
+#pragma unroll
+          for (int k = 0; k < 16; ++k) v[u][k] = g[k * C];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (u < cnt)
+#pragma unroll
+          for (int k = 0; k < 16; ++k) acc[k] += v[u][k];
     }
 #pragma unroll
     for (int k = 0; k < 16; ++k) gx[((size_t)j * 16 + k) * C + c] += acc[k];

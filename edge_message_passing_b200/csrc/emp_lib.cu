@@ -190,7 +190,7 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
   int* counter = at<int>(ws, L.counter);
   for (long long e0 = 0; e0 < E; e0 += coh) {
     const long long e1 = std::min(E, e0 + coh);
-    { Scope sc_("rotate_in", s); k_rotate_in<<<grid_for(e1 - e0, eb.y), eb, esmem, s>>>(e0, e1, C, scalar_in, g->send, rrow, D, R, x, XT, XTlo); }
+    { Scope sc_("rotate_in", s); k_rotate_in<<<grid_for(e1 - e0, BE_CHUNK), eb, (size_t)BE_CHUNK * NDBLK * 4, s>>>(e0, e1, C, scalar_in, g->send, rrow, D, R, x, XT, XTlo); }
     int st;
     if (scalar_in) {
       const So2AMaps* a = am.get(e1 - e0);
@@ -780,8 +780,8 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
         st = so2_product(m, n, parts, 2, counter, stream);
       }
       if (st != EMP_OK) return st;
-      const size_t smem = (size_t)eb.y * NDBLK * 4 + (size_t)eb.y * 2 * (C / 32) * 4;
-      { Scope sc_("bwd_edge", stream); k_bwd_edge<<<grid, eb, smem, stream>>>(e0, e1, C, t > 0, t == 0, g->send, rr.inv, g->vec, D, R, xt, Y, GY, GXT, XT, gRhi, gRlo, g_r); }
+      const size_t smem = (size_t)BE_CHUNK * NDBLK * 4 + (size_t)BE_CHUNK * 2 * (C / 32) * 4;
+      { Scope sc_("bwd_edge", stream); k_bwd_edge<<<grid_for(n, BE_CHUNK), eb, smem, stream>>>(e0, e1, C, t > 0, t == 0, g->send, rr.inv, g->vec, D, R, xt, Y, GY, GXT, XT, gRhi, gRlo, g_r); }
       if (t > 0) {
         dim3 sg(std::min<long long>(n, 2048), C / 32);
         { Scope sc_("sender_scatter", stream); k_sender_scatter<<<sg, 32, 0, stream>>>(e0, e1, C, ci, g->send, perm, seg, nseg, XT, gxb); }
