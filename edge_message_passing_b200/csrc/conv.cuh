@@ -60,22 +60,20 @@ __global__ void k_geometry(long long E, const float* __restrict__ vec, float* __
 }
 
 // ------------------------------------------------------------------ radial part
-// e_n(d) = u(d/rc) sin(n pi d / rc) / d, u(x) = 1 - 28 x^6 + 48 x^7 - 21 x^8 for x < 1.
-__device__ __forceinline__ void bessel8(float d, float rc, float (&e)[8], float (&de)[8]) {
+// e_n(d) = u(d/rc) sin(n pi d / rc) / d, u(x) = 1 - 28 x^6 + 48 x^7 - 21 x^8 for x < 1,
+// and its derivative in d (one basis function: every (row, n) pair is its own work item).
+__device__ __forceinline__ void bessel_n(float d, float rc, int n, float& e, float& de) {
   const float x = d / rc;
   const float x2 = x * x, x5 = x2 * x2 * x, x6 = x5 * x;
   float u = 1.f + x6 * (-28.f + x * (48.f - 21.f * x));
   float du = x5 * (-168.f + x * (336.f - 168.f * x)) / rc;
   if (x >= 1.f) { u = 0.f; du = 0.f; }
   const float inv = 1.f / d;
-#pragma unroll
-  for (int n = 0; n < 8; ++n) {
-    const float k = PI_F * (float)(n + 1) / rc;
-    float s, c;
-    sincosf(k * d, &s, &c);
-    e[n] = u * s * inv;
-    de[n] = du * s * inv + u * (k * c * inv - s * inv * inv);
-  }
+  const float k = PI_F * (float)(n + 1) / rc;
+  float s, c;
+  sincosf(k * d, &s, &c);
+  e = u * s * inv;
+  de = du * s * inv + u * (k * c * inv - s * inv * inv);
 }
 
 __device__ __forceinline__ int pair_of(int a, int b, int S) {
@@ -93,58 +91,31 @@ struct RadialArgs {
 
 constexpr int RT = 64;      // rows per radial tile
 constexpr int RAD_THREADS = 256;
+constexpr int RP = 68;      // padded pitch of the transposed [64][RT] tiles (16-byte rows)
 
-// shared-memory tile of the radial network's hidden layers
+// Shared memory of a radial tile.  Thread t owns the 4 x 4 register tile of rows
+// 4 (t >> 4) .. +3 and hidden units 4 (t & 15) .. +3 in every layer, so layer 1's
+// outputs, layer 2's outputs and the backward's dE/dh1 of a thread share positions.
 struct RadialSmem {
   float e[RT][8];
   float de[RT][8];
-  float z1[RT][64];
-  float h1[RT][65];
-  float z2[RT][64];
-  float h2[RT][65];
-  float g[RT][65];      // backward: dE/dh2 rows
+  float W1[64 * 8];        // [j][n]
+  float W2T[64][RP];       // [i][o] = W2[o][i]
+  float W2[64][RP];        // backward: [o][i]
+  float h1T[64][RP];       // [i][r]
+  float gT[64][RP];        // backward: dE/dz2 as [o][r]
   int pair[RT];
   int edge[RT];
+  float dist[RT];
   unsigned mask;
 };
 
-// hidden layers (for the tile's rows, with pair p's weights) -- all 256 threads participate
-__device__ void radial_hidden(RadialSmem& s, const float* __restrict__ W1, const float* __restrict__ W2) {
-  const int t = threadIdx.x;
-  // layer 1: z1[e][j] = sum_n W1[j][n] e[n]
-  for (int idx = t; idx < RT * 64; idx += RAD_THREADS) {
-    const int e = idx >> 6, j = idx & 63;
-    float acc = 0.f;
-#pragma unroll
-    for (int n = 0; n < 8; ++n) acc = fmaf(__ldg(&W1[j * 8 + n]), s.e[e][n], acc);
-    s.z1[e][j] = acc;
-    s.h1[e][j] = silu_f(acc);
-  }
-  __syncthreads();
-  // layer 2: thread owns output j and 16 rows
-  {
-    const int j = t & 63, eg = (t >> 6) * 16;
-    float acc[16];
-#pragma unroll
-    for (int q = 0; q < 16; ++q) acc[q] = 0.f;
-    for (int k = 0; k < 64; ++k) {
-      const float w = __ldg(&W2[j * 64 + k]);
-#pragma unroll
-      for (int q = 0; q < 16; ++q) acc[q] = fmaf(w, s.h1[eg + q][k], acc[q]);
-    }
-#pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      s.z2[eg + q][j] = acc[q];
-      s.h2[eg + q][j] = silu_f(acc[q]);
-    }
-  }
-  __syncthreads();
-}
-
-// rows r0 .. r0+63 of the (pair-sorted, or edge-ordered when perm is null) row list
+// rows r0 .. r0+63 of the (pair-sorted, or edge-ordered when perm is null) row list:
+// edge, pair, distance and the basis (with its derivative when want_de)
 __device__ void radial_tile_setup(RadialSmem& s, long long r0, long long E, const int* __restrict__ perm,
                                   const float* __restrict__ dist, const int* __restrict__ recv,
-                                  const int* __restrict__ send, const int* __restrict__ species, const RadialArgs& a) {
+                                  const int* __restrict__ send, const int* __restrict__ species, const RadialArgs& a,
+                                  bool want_de) {
   const int t = threadIdx.x;
   if (t == 0) s.mask = 0u;
   __syncthreads();
@@ -160,12 +131,64 @@ __device__ void radial_tile_setup(RadialSmem& s, long long r0, long long E, cons
     }
     s.pair[t] = r < E ? p : -1;
     s.edge[t] = e;
-    float ev[8], dv[8];
-    bessel8(d, a.rc, ev, dv);
-#pragma unroll
-    for (int n = 0; n < 8; ++n) { s.e[t][n] = ev[n]; s.de[t][n] = dv[n]; }
+    s.dist[t] = d;
   }
   __syncthreads();
+  for (int idx = t; idx < RT * 8; idx += RAD_THREADS) {
+    const int r = idx >> 3, n = idx & 7;
+    float ev, dv;
+    bessel_n(s.dist[r], a.rc, n, ev, dv);
+    s.e[r][n] = ev;
+    if (want_de) s.de[r][n] = dv;
+  }
+}
+
+// pair p's weights into shared memory (W2 also untransposed for the backward)
+__device__ void radial_stage_weights(RadialSmem& s, const float* __restrict__ W1, const float* __restrict__ W2,
+                                     bool want_w2) {
+  const int t = threadIdx.x;
+  for (int idx = t; idx < 64 * 8; idx += RAD_THREADS) s.W1[idx] = __ldg(&W1[idx]);
+  for (int idx = t; idx < 64 * 64; idx += RAD_THREADS) {
+    const int o = idx >> 6, i = idx & 63;
+    const float w = __ldg(&W2[idx]);
+    s.W2T[i][o] = w;
+    if (want_w2) s.W2[o][i] = w;
+  }
+}
+
+// layer 1 of the thread's tile: z1[r][j] = sum_n W1[j][n] e[r][n]; h1 = SiLU(z1) stored as h1T
+__device__ __forceinline__ void radial_layer1(RadialSmem& s, int r0, int j0, float (&z1)[4][4]) {
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      float acc = 0.f;
+#pragma unroll
+      for (int n = 0; n < 8; ++n) acc = fmaf(s.W1[(j0 + b) * 8 + n], s.e[r0 + a][n], acc);
+      z1[a][b] = acc;
+    }
+#pragma unroll
+  for (int b = 0; b < 4; ++b)
+    *reinterpret_cast<float4*>(&s.h1T[j0 + b][r0]) =
+        make_float4(silu_f(z1[0][b]), silu_f(z1[1][b]), silu_f(z1[2][b]), silu_f(z1[3][b]));
+}
+
+// layer 2 of the thread's tile: z2[r][o] = sum_i W2[o][i] h1[r][i]
+__device__ __forceinline__ void radial_layer2(const RadialSmem& s, int r0, int j0, float (&z2)[4][4]) {
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) z2[a][b] = 0.f;
+#pragma unroll 8
+  for (int i = 0; i < 64; ++i) {
+    const float4 h = *reinterpret_cast<const float4*>(&s.h1T[i][r0]);
+    const float4 w = *reinterpret_cast<const float4*>(&s.W2T[i][j0]);
+    const float hv[4] = {h.x, h.y, h.z, h.w}, wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) z2[a][b] = fmaf(hv[a], wv[b], z2[a][b]);
+  }
 }
 
 // h2 rows (3xTF32 split) of the radial network for every row: the input of the
@@ -177,22 +200,34 @@ __global__ void __launch_bounds__(RAD_THREADS) k_radial_h2(long long E, const in
                                                           float* __restrict__ h2_lo) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   RadialSmem& s = *reinterpret_cast<RadialSmem*>(smem_raw);
-  const long long r0 = (long long)blockIdx.x * RT;
-  radial_tile_setup(s, r0, E, perm, dist, recv, send, species, a);
+  const long long r0g = (long long)blockIdx.x * RT;
+  radial_tile_setup(s, r0g, E, perm, dist, recv, send, species, a, false);
   const int t = threadIdx.x;
+  const int r0 = (t >> 4) * 4, j0 = (t & 15) * 4;
   unsigned mask = s.mask;
   while (mask) {
     const int p = __ffs(mask) - 1;
     mask &= mask - 1;
     const float* W1 = a.rad + a.layer_off + (size_t)p * a.pair_stride;
-    radial_hidden(s, W1, W1 + 64 * 8);
-    for (int idx = t; idx < RT * 64; idx += RAD_THREADS) {
-      const int el = idx >> 6, j = idx & 63;
-      if (s.pair[el] == p) {
-        const float v = s.h2[el][j], h = tf32_rna(v);
-        h2_hi[(size_t)(r0 + el) * 64 + j] = h;
-        h2_lo[(size_t)(r0 + el) * 64 + j] = tf32_rna(v - h);
+    radial_stage_weights(s, W1, W1 + 64 * 8, false);
+    __syncthreads();
+    float z[4][4];
+    radial_layer1(s, r0, j0, z);
+    __syncthreads();
+    radial_layer2(s, r0, j0, z);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const long long r = r0g + r0 + q;
+      if (s.pair[r0 + q] != p) continue;
+      float hi[4], lo[4];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const float v = silu_f(z[q][b]);
+        hi[b] = tf32_rna(v);
+        lo[b] = tf32_rna(v - hi[b]);
       }
+      *reinterpret_cast<float4*>(h2_hi + (size_t)r * 64 + j0) = make_float4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<float4*>(h2_lo + (size_t)r * 64 + j0) = make_float4(lo[0], lo[1], lo[2], lo[3]);
     }
     __syncthreads();
   }
@@ -207,56 +242,80 @@ __global__ void __launch_bounds__(RAD_THREADS) k_radial_bwd(long long E, const i
                                                            float* __restrict__ g_r) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   RadialSmem& s = *reinterpret_cast<RadialSmem*>(smem_raw);
-  const long long r0 = (long long)blockIdx.x * RT;
-  radial_tile_setup(s, r0, E, perm, dist, recv, send, species, a);
+  const long long r0g = (long long)blockIdx.x * RT;
+  radial_tile_setup(s, r0g, E, perm, dist, recv, send, species, a, true);
   const int t = threadIdx.x;
-  for (int idx = t; idx < RT * 64; idx += RAD_THREADS) {
-    const int el = idx >> 6, j = idx & 63;
-    s.g[el][j] = (r0 + el < E) ? gh2[(size_t)(r0 + el) * 64 + j] : 0.f;
+  const int r0 = (t >> 4) * 4, j0 = (t & 15) * 4;
+  float g[4][4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const long long r = r0g + r0 + q;
+    const float4 v = r < E ? *reinterpret_cast<const float4*>(gh2 + (size_t)r * 64 + j0) : make_float4(0.f, 0.f, 0.f, 0.f);
+    g[q][0] = v.x; g[q][1] = v.y; g[q][2] = v.z; g[q][3] = v.w;
   }
   unsigned mask = s.mask;
   while (mask) {
     const int p = __ffs(mask) - 1;
     mask &= mask - 1;
     const float* W1 = a.rad + a.layer_off + (size_t)p * a.pair_stride;
-    const float* W2 = W1 + 64 * 8;
-    radial_hidden(s, W1, W2);
-    // g_z2 = g_h2 dsilu(z2) -> h2
-    for (int idx = t; idx < RT * 64; idx += RAD_THREADS) {
-      const int el = idx >> 6, j = idx & 63;
-      s.h2[el][j] = s.g[el][j] * dsilu_f(s.z2[el][j]);
-    }
+    radial_stage_weights(s, W1, W1 + 64 * 8, true);
     __syncthreads();
-    // g_h1[e][j] = sum_k g_z2[e][k] W2[k][j]; g_z1 = g_h1 dsilu(z1) -> h1
-    {
-      const int j = t & 63, eg = (t >> 6) * 16;
-      float a2[16];
-#pragma unroll
-      for (int q = 0; q < 16; ++q) a2[q] = 0.f;
-      for (int kk = 0; kk < 64; ++kk) {
-        const float w = __ldg(&W2[kk * 64 + j]);
-#pragma unroll
-        for (int q = 0; q < 16; ++q) a2[q] = fmaf(s.h2[eg + q][kk], w, a2[q]);
-      }
-      __syncthreads();
-#pragma unroll
-      for (int q = 0; q < 16; ++q) s.h1[eg + q][j] = a2[q] * dsilu_f(s.z1[eg + q][j]);
-    }
+    float z1[4][4], z2[4][4];
+    radial_layer1(s, r0, j0, z1);
     __syncthreads();
-    // dE/dd = sum_n (sum_j g_z1[j] W1[j][n]) de_n/dd
-    if (t < RT && s.pair[t] == p) {
-      const int e = s.edge[t];
-      float dEdd = 0.f;
+    radial_layer2(s, r0, j0, z2);
+    // dE/dz2 = dE/dh2 SiLU'(z2), stored transposed
 #pragma unroll
-      for (int n = 0; n < 8; ++n) {
-        float ge = 0.f;
-        for (int j = 0; j < 64; ++j) ge = fmaf(s.h1[t][j], __ldg(&W1[j * 8 + n]), ge);
-        dEdd = fmaf(ge, s.de[t][n], dEdd);
+    for (int b = 0; b < 4; ++b)
+      *reinterpret_cast<float4*>(&s.gT[j0 + b][r0]) =
+          make_float4(g[0][b] * dsilu_f(z2[0][b]), g[1][b] * dsilu_f(z2[1][b]), g[2][b] * dsilu_f(z2[2][b]),
+                      g[3][b] * dsilu_f(z2[3][b]));
+    __syncthreads();
+    // dE/dh1[r][i] = sum_o dE/dz2[r][o] W2[o][i]; dE/dz1 = dE/dh1 SiLU'(z1)
+    float gh[4][4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) gh[q][b] = 0.f;
+#pragma unroll 8
+    for (int o = 0; o < 64; ++o) {
+      const float4 gz = *reinterpret_cast<const float4*>(&s.gT[o][r0]);
+      const float4 w = *reinterpret_cast<const float4*>(&s.W2[o][j0]);
+      const float gv[4] = {gz.x, gz.y, gz.z, gz.w}, wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) gh[q][b] = fmaf(gv[q], wv[b], gh[q][b]);
+    }
+    // dE/dd[r] = sum_j dE/dz1[r][j] sum_n W1[j][n] de_n[r]: this thread's 4 units, then
+    // summed over the 16 threads of the half-warp that share the rows
+    float part[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float acc = 0.f;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        float w = 0.f;
+#pragma unroll
+        for (int n = 0; n < 8; ++n) w = fmaf(s.W1[(j0 + b) * 8 + n], s.de[r0 + q][n], w);
+        acc = fmaf(gh[q][b] * dsilu_f(z1[q][b]), w, acc);
       }
-      const float inv = 1.f / dist[e];
-      g_r[3 * e + 0] += dEdd * vec[3 * e + 0] * inv;
-      g_r[3 * e + 1] += dEdd * vec[3 * e + 1] * inv;
-      g_r[3 * e + 2] += dEdd * vec[3 * e + 2] * inv;
+      part[q] = acc;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int off = 8; off >= 1; off >>= 1) part[q] += __shfl_xor_sync(0xffffffffu, part[q], off);
+    if ((t & 15) == 0) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (s.pair[r0 + q] != p) continue;
+        const int e = s.edge[r0 + q];
+        const float inv = 1.f / s.dist[r0 + q];
+        g_r[3 * e + 0] += part[q] * vec[3 * e + 0] * inv;
+        g_r[3 * e + 1] += part[q] * vec[3 * e + 1] * inv;
+        g_r[3 * e + 2] += part[q] * vec[3 * e + 2] * inv;
+      }
     }
     __syncthreads();
   }

@@ -147,7 +147,9 @@ __host__ __device__ constexpr int b_box_rows(int n) { return (n < BN ? n : BN) /
 constexpr int ST2 = 6;
 constexpr int B2_BYTES = (BN / 2) * BK * 4;            // 8 KB: half of a 256-row B tile
 constexpr int STAGE2 = 2 * A_BYTES + 2 * B2_BYTES;     // 32 KB per CTA
-constexpr int SMEM2 = ST2 * STAGE2 + 1024 + 512;
+constexpr int EPI_PITCH = 36;                          // floats per staged row (16-byte aligned, conflict-free)
+constexpr int EPI_BYTES = 4 * 32 * EPI_PITCH * 4;      // one 32 x 32 staging tile per epilogue warp
+constexpr int SMEM2 = ST2 * STAGE2 + 1024 + 512 + EPI_BYTES;
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -245,6 +247,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* issued = abort_flag + 1;
   int* consumed = issued + 1;
+  float* epi = reinterpret_cast<float*>(smem + ST2 * STAGE2 + 512);   // epilogue staging tiles
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
@@ -381,17 +384,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const int buf = i & 1;
       if (!mbar_wait(&acc_full[buf], (i >> 1) & 1)) { *vabort = 1; break; }
       fence_after();
-      const int m = ti.m0 + (int)rank * BM + row;
+      // 32 x 32 chunks: TMEM -> registers (a row per thread) -> this warp's staging tile ->
+      // rows stored 8 threads x 16 bytes at a time, so every store writes whole 128-byte segments
+      const int mw = ti.m0 + (int)rank * BM + q * 32;
       const int N = g.N[ti.sub], bn = g.bn[ti.sub];
-      float* orow = g.out[ti.sub] + (size_t)m * g.ldc + g.ccol[ti.sub] + ti.n0;
+      float* obase = g.out[ti.sub] + (size_t)g.ccol[ti.sub] + ti.n0;
+      float* stg = epi + q * 32 * EPI_PITCH;
+      (void)row;
 #pragma unroll 1
       for (int cc = 0; cc < bn; cc += 32) {
         float v[32];
         tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + cc), v);
-        if (m < g.M && ti.n0 + cc < N) {
+        if (ti.n0 + cc < N) {
 #pragma unroll
           for (int j = 0; j < 32; j += 4)
-            *reinterpret_cast<float4*>(orow + cc + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+            *reinterpret_cast<float4*>(stg + lane * EPI_PITCH + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int rr = k * 4 + (lane >> 3), c4 = (lane & 7) * 4;
+            const int m = mw + rr;
+            const float4 w = *reinterpret_cast<const float4*>(stg + rr * EPI_PITCH + c4);
+            if (m < g.M) *reinterpret_cast<float4*>(obase + (size_t)m * g.ldc + cc + c4) = w;
+          }
+          __syncwarp();
         }
       }
       fence_before();
