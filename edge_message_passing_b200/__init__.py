@@ -298,6 +298,50 @@ def mp_energy_forces(model: Model, graph: Graph, species, virial: bool = False, 
     return energy, forces, vir, ea
 
 
+class EnergyForcesGraph:
+    """mp_energy_forces of one neighbour graph and species array, captured once as a
+    CUDA graph and replayed.  The replay runs the library's own kernels with the
+    pointers captured here: the outputs (energy, forces, virial, atom_energy) are
+    this object's tensors, overwritten by every replay, and graph, species and the
+    workspace are kept alive by the object.  The positions must not change between
+    replays without a new capture (the graph's edge vectors are inputs)."""
+
+    def __init__(self, model: Model, graph: Graph, species, virial: bool = False, atom_energy: bool = False):
+        torch = _torch()
+        if getattr(model.spec, "pair_radial", False):
+            # per-pair radial networks read the pair offsets back to the host once per call
+            raise EmpError("EnergyForcesGraph: models with per-pair radial networks cannot be captured")
+        N = graph.n_atoms
+        self.model, self.graph, self.species = model, graph, species
+        self.energy = torch.empty(1, dtype=torch.float64, device="cuda")
+        self.forces = torch.empty((N, 3), dtype=torch.float32, device="cuda")
+        self.virial = torch.empty((3, 3), dtype=torch.float32, device="cuda") if virial else None
+        self.atom_energy = torch.empty(N, dtype=torch.float32, device="cuda") if atom_energy else None
+        self.ws = torch.empty(max(model.workspace_bytes(graph.n_edges, N), 256), dtype=torch.uint8, device="cuda")
+        self._gc = graph.c()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self._call()                      # first call outside the capture (one-time set-up)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        self.cuda_graph = torch.cuda.CUDAGraph()
+        n0 = launch_count()
+        with torch.cuda.graph(self.cuda_graph):
+            self._call()
+        self.launches = launch_count() - n0   # library kernels per replay
+
+    def _call(self):
+        _check(lib().mp_energy_forces(self.model.handle, ctypes.byref(self._gc), _ptr(self.species),
+                                      _ptr(self.energy), _ptr(self.forces), _ptr(self.virial),
+                                      _ptr(self.atom_energy), _ptr(self.ws), self.ws.numel(), _stream()),
+               "mp_energy_forces")
+
+    def replay(self):
+        self.cuda_graph.replay()
+        return self.energy, self.forces, self.virial, self.atom_energy
+
+
 def mp_so2_mix(model: Model, layer: int, X, transpose: bool = False):
     """The per-m SO(2) block products of X [M,16C] (m-major column layout)."""
     torch = _torch()

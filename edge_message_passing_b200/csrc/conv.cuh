@@ -445,84 +445,130 @@ __global__ void k_rotate_in(long long e0, long long e1, int C, int scalar_in, co
 
 // ------------------------------------------------------------------ rotate back + receiver sums
 // S[i] (+)= sum over the cohort's edges of receiver i of D_e^T y_e.
-// One block per (receiver, 32-channel group): RB_ROWS rows take the receiver's
-// edges round-robin (row r: edges b + r, b + r + RB_ROWS, ...), each row sums
-// its edges in order, then the rows are added in row order onto the running
-// sum carried from earlier cohorts.  The order is fixed, so results are
-// reproducible; a receiver whose edges started in an earlier cohort continues
-// its running sum.
-constexpr int RB_ROWS = 16;
-constexpr int RB_CG = 32;
-constexpr int RB_CHUNK = 128;     // edges whose Wigner-D blocks are staged at once
-struct RbSmem {
-  float sD[RB_CHUNK * NDBLK];
-  float part[RB_ROWS][16][RB_CG];
-};
+// The cohort's rows (receiver-sorted) are cut into chunks of RB_CHUNK consecutive
+// edges, one block of C threads (one per channel) per chunk.  A thread sums its
+// chunk's messages in edge order, one running sum per receiver run.  A receiver
+// whose edges (within the cohort) all lie in the chunk is finished at once: its
+// sum is written to S, added to the running sum that S carries when the receiver's
+// edges began in an earlier cohort.  A receiver that crosses a chunk boundary
+// leaves its chunk sum in a partial slot (slot 0: the chunk's first receiver, slot
+// 1: its last), and k_rb_combine adds the partials in chunk order.  The order of
+// every sum is fixed, so results are reproducible.
+constexpr int RB_CHUNK = 8;
+constexpr int RB_BATCH = 2;      // edges whose rows are loaded before any is used
 
-__global__ void __launch_bounds__(RB_CG * RB_ROWS) k_rotate_back_scatter(long long e0, long long e1, int C,
-                                                                         int scalar_in,
-                                                                         const int* __restrict__ recv,
-                                                                         const int* __restrict__ recv_off,
-                                                                         const float* __restrict__ D,
-                                                                         const float* __restrict__ Y,
-                                                                         float* __restrict__ S) {
-  extern __shared__ __align__(16) unsigned char rb_smem[];
-  RbSmem& sm = *reinterpret_cast<RbSmem*>(rb_smem);
-  float* sD = sm.sD;
-  auto& part = sm.part;
-  const int cg = min(C, RB_CG);
-  const int tx = threadIdx.x, row = threadIdx.y, tid = row * cg + tx, nthr = cg * RB_ROWS;
-  const int c = blockIdx.y * cg + tx;
-  const int first = recv[e0], last = recv[e1 - 1];
-  for (int i = first + blockIdx.x; i <= last; i += gridDim.x) {
-    const long long b = max((long long)recv_off[i], e0), en = min((long long)recv_off[i + 1], e1);
+__device__ __forceinline__ void rb_flush(int i, int c0, int c1, long long e0, long long e1, int chunk, int first_recv,
+                                         const int* __restrict__ recv_off, int C, int c, const float (&acc)[16],
+                                         float* __restrict__ S, float* __restrict__ P) {
+  const long long lo = max((long long)recv_off[i], e0) - e0, hi = min((long long)recv_off[i + 1], e1) - e0;
+  if (lo >= c0 && hi <= c1) {
+    float* Si = S + (size_t)i * 16 * C + c;
     const bool carry = recv_off[i] < e0;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) Si[k * C] = carry ? Si[k * C] + acc[k] : acc[k];
+  } else {
+    float* Pc = P + ((size_t)chunk * 2 + (i == first_recv ? 0 : 1)) * 16 * C + c;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) Pc[k * C] = acc[k];
+  }
+}
+
+__global__ void __launch_bounds__(256, 3) k_rb_chunks(long long e0, long long e1, int C, int scalar_in,
+                                                   const int* __restrict__ recv, const int* __restrict__ recv_off,
+                                                   const float* __restrict__ D, const float* __restrict__ Y,
+                                                   float* __restrict__ S, float* __restrict__ P) {
+  __shared__ __align__(16) float sD[RB_CHUNK * NDBLK];
+  __shared__ int srv[RB_CHUNK];
+  const int c = threadIdx.x;
+  const int n = (int)(e1 - e0);
+  const int nchunks = (n + RB_CHUNK - 1) / RB_CHUNK;
+  for (int chunk = blockIdx.x; chunk < nchunks; chunk += gridDim.x) {
+    const int c0 = chunk * RB_CHUNK, nch = min(RB_CHUNK, n - c0), c1 = c0 + nch;
+    __syncthreads();
+    for (int q = c; q < nch * (NDBLK / 4); q += C)
+      reinterpret_cast<float4*>(sD)[q] = reinterpret_cast<const float4*>(D + (size_t)(e0 + c0) * NDBLK)[q];
+    if (c < nch) srv[c] = recv[e0 + c0 + c];
+    __syncthreads();
+    const int first = srv[0];
+    int cur = first;
     float acc[16];
 #pragma unroll
     for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-    for (long long cb = b; cb < en; cb += RB_CHUNK) {
-      const int nch = (int)min((long long)RB_CHUNK, en - cb);
-      __syncthreads();
-      {
-        const float4* src = reinterpret_cast<const float4*>(D + (size_t)cb * NDBLK);
-        float4* dst = reinterpret_cast<float4*>(sD);
-        for (int q = tid; q < nch * (NDBLK / 4); q += nthr) dst[q] = src[q];
+    for (int k0 = 0; k0 < nch; k0 += RB_BATCH) {
+      float yv[RB_BATCH][16];
+#pragma unroll
+      for (int u = 0; u < RB_BATCH; ++u) {
+        if (k0 + u < nch) {
+          const float* y = Y + (size_t)(c0 + k0 + u) * 16 * C + c;
+          if (scalar_in) {
+#pragma unroll
+            for (int l = 0; l < 4; ++l) yv[u][l] = y[col_of(l, 0) * C];
+          } else {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) yv[u][q] = y[col_of_k(q) * C];
+          }
+        }
       }
-      __syncthreads();
-#pragma unroll 2
-      for (int k = row; k < nch; k += RB_ROWS) {
-        const float* y = Y + (size_t)(cb + k - e0) * 16 * C;
+#pragma unroll
+      for (int u = 0; u < RB_BATCH; ++u) {
+        const int k = k0 + u;
+        if (k >= nch) break;
+        if (srv[k] != cur) {
+          rb_flush(cur, c0, c1, e0, e1, chunk, first, recv_off, C, c, acc, S, P);
+#pragma unroll
+          for (int q = 0; q < 16; ++q) acc[q] = 0.f;
+          cur = srv[k];
+        }
         const float* Dk = sD + k * NDBLK;
         if (scalar_in) {
           // y is non-zero only at m = 0: message[l][n] = D^l[0][n] y[l][0]
 #pragma unroll
           for (int l = 0; l < 4; ++l) {
-            const float yl = y[col_of(l, 0) * C + c];
             const float* row0 = Dk + dblk_off(l) + l * (2 * l + 1);
 #pragma unroll
-            for (int n = 0; n < 2 * l + 1; ++n) acc[l * l + n] = fmaf(row0[n], yl, acc[l * l + n]);
+            for (int q = 0; q < 2 * l + 1; ++q) acc[l * l + q] = fmaf(row0[q], yv[u][l], acc[l * l + q]);
           }
-          continue;
+        } else {
+          float m[16];
+          rotate16<true>(Dk, yv[u], m);
+#pragma unroll
+          for (int q = 0; q < 16; ++q) acc[q] += m[q];
         }
-        float yv[16], m[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) yv[q] = y[col_of_k(q) * C + c];
-        rotate16<true>(Dk, yv, m);
-#pragma unroll
-        for (int q = 0; q < 16; ++q) acc[q] += m[q];
       }
     }
+    rb_flush(cur, c0, c1, e0, e1, chunk, first, recv_off, C, c, acc, S, P);
+  }
+}
+
+// receivers of the cohort that cross a chunk boundary: S[i] = carried sum + chunk partials in
+// order.  Block (x, k): receivers first + x, first + x + gridDim.x, ..., component k; the
+// partials are fetched eight chunks at a time and added in chunk order.
+__global__ void k_rb_combine(long long e0, long long e1, int C, const int* __restrict__ recv,
+                             const int* __restrict__ recv_off, const float* __restrict__ P, float* __restrict__ S) {
+  const int c = threadIdx.x, k = blockIdx.y;
+  const int first = recv[e0], last = recv[e1 - 1];
+  for (int i = first + blockIdx.x; i <= last; i += gridDim.x) {
+    const long long lo = max((long long)recv_off[i], e0) - e0, hi = min((long long)recv_off[i + 1], e1) - e0;
+    if (hi <= lo) continue;
+    const int cf = (int)(lo / RB_CHUNK), cl = (int)((hi - 1) / RB_CHUNK);
+    if (cf == cl) continue;
+    float* Si = S + ((size_t)i * 16 + k) * C + c;
+    float acc = recv_off[i] < e0 ? *Si : 0.f;
+    for (int ch0 = cf; ch0 <= cl; ch0 += 8) {
+      float v[8];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) part[row][k][tx] = acc[k];
-    __syncthreads();
-    if (row < 16) {
-      const int k = row;
-      float s = carry ? S[((size_t)i * 16 + k) * C + c] : 0.f;
+      for (int u = 0; u < 8; ++u) {
+        const int ch = ch0 + u;
+        if (ch <= cl) {
+          const int slot = recv[e0 + (long long)ch * RB_CHUNK] == i ? 0 : 1;
+          v[u] = P[(((size_t)ch * 2 + slot) * 16 + k) * C + c];
+        }
+      }
 #pragma unroll
-      for (int r = 0; r < RB_ROWS; ++r) s += part[r][k][tx];
-      S[((size_t)i * 16 + k) * C + c] = s;
+      for (int u = 0; u < 8; ++u)
+        if (ch0 + u <= cl) acc += v[u];
     }
-    __syncthreads();
+    *Si = acc;
   }
 }
 
@@ -712,7 +758,7 @@ template <int L>
 __device__ __forceinline__ void bwd_edge_degree(const float* __restrict__ Dr, const float* __restrict__ xs,
                                                 const float* __restrict__ yrow, const float* __restrict__ gyrow,
                                                 const float* __restrict__ gxtrow, float Rl, int C, int c,
-                                                bool need_gx, float* __restrict__ gxsrow, float& grl,
+                                                bool need_gx, float (&gxs)[16], float& grl,
                                                 float& bx, float& by, bool scalar_in) {
   constexpr int W = 2 * L + 1, O = L * L;
   const float* B = Dr + dblk_off(L);
@@ -760,101 +806,197 @@ __device__ __forceinline__ void bwd_edge_degree(const float* __restrict__ Dr, co
       float a = 0.f;
 #pragma unroll
       for (int n = 0; n < W; ++n) a = fmaf(B[n * W + m], gu[n], a);
-      gxsrow[(O + m) * C] = a;
+      gxs[O + m] += a;
     }
   }
 }
 
-// Edges are taken in chunks of BE_CHUNK: their Wigner-D blocks are staged with one
-// barrier pair, each row then walks its share of the chunk back to back, and the
-// per-edge torque sums are finished once per chunk.
+// Per-edge backward over the cohort, one block of C threads (one per channel) per
+// contiguous range of `per` positions.  With need_gx the positions follow the
+// cohort's sender sort (perm), so each sender's edges are consecutive: the block
+// sums g_xs over each sender run in registers and stores the sum of each run piece
+// (a run, or the part of one that lies in the range) as row Pg[first position of the
+// piece]; k_gx_combine then adds every run's pieces to g_x[sender] in order.  Without
+// need_gx the positions are the cohort's edges in order.
+// The rows an edge reads (y, g_y, g_x~, x_send, R and its Wigner-D blocks, all
+// contiguous) are brought into a BE_STAGES-deep shared-memory ring by bulk copies
+// (cp.async.bulk, completing on one mbarrier per stage) issued by thread 0 ahead of
+// use, so the loads of later edges overlap the arithmetic of the current one.  The
+// per-edge torque sums are kept per position and finished for the whole range at
+// the end, by one thread per edge.
+constexpr int BE_STAGES = 3;
+constexpr int BE_MAXP = 64;           // positions per block at most
 
-__global__ void __launch_bounds__(256, 2) k_bwd_edge(long long e0, long long e1, int C, int need_gx, int scalar_in,
-                                                     const int* __restrict__ send, const int* __restrict__ rrow,
-                                                     const float* __restrict__ vec,
-                                                     const float* __restrict__ D, const float* __restrict__ R,
-                                                     const float* __restrict__ x, const float* __restrict__ Y,
-                                                     const float* __restrict__ GY, const float* __restrict__ GXT,
-                                                     float* __restrict__ GXS, float* __restrict__ gR_hi,
-                                                     float* __restrict__ gR_lo, float* __restrict__ g_r) {
-  extern __shared__ __align__(16) float smem[];
-  const int c = threadIdx.x, row = threadIdx.y, EPB = blockDim.y;
-  const int tid = row * C + c, nthr = C * EPB;
-  float* sD = smem;                                 // [BE_CHUNK][84]
-  float* red = smem + BE_CHUNK * NDBLK;             // [BE_CHUNK][2][C/32]
+struct BeMeta {
+  int el, rr, j, pad;                 // cohort-local row, radial row, sender
+};
+
+// stage layout (floats): Y [16C] | GY [16C] | GXT [16C] | X [16C] | R [4C] | D [84]
+__host__ __device__ inline size_t be_stage_floats(int C) { return (size_t)68 * C + NDBLK; }
+__host__ __device__ inline size_t be_smem_bytes(int C) {
+  return BE_STAGES * be_stage_floats(C) * 4 + BE_STAGES * 8 + (size_t)BE_MAXP * 2 * (C / 32) * 4 +
+         BE_MAXP * sizeof(BeMeta) + BE_MAXP * 4 * 4;
+}
+// positions per block for a cohort of n edges on `sms` SMs (two blocks per SM)
+inline int be_per(long long n, int sms) {
+  const long long want = (n + 2 * sms - 1) / (2 * sms);
+  return (int)std::max<long long>(1, std::min<long long>(BE_MAXP, want));
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(tc::smem_u32(dst)), "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
+               : "memory");
+}
+
+__global__ void __launch_bounds__(256, 2)
+    k_bwd_edge(long long e0, long long e1, int C, int need_gx, int scalar_in, int per,
+               const int* __restrict__ send, const int* __restrict__ rrow, const float* __restrict__ vec,
+               const float* __restrict__ D, const float* __restrict__ R, const float* __restrict__ x,
+               const float* __restrict__ Y, const float* __restrict__ GY, const float* __restrict__ GXT,
+               const int* __restrict__ perm, float* __restrict__ gR_hi, float* __restrict__ gR_lo,
+               float* __restrict__ g_r, float* __restrict__ Pg) {
+  extern __shared__ __align__(128) unsigned char be_smem[];
+  const size_t SF = be_stage_floats(C);
+  float* stage0 = reinterpret_cast<float*>(be_smem);
+  uint64_t* full = reinterpret_cast<uint64_t*>(be_smem + BE_STAGES * SF * 4);
+  float* red = reinterpret_cast<float*>(full + BE_STAGES);               // [BE_MAXP][2][C/32]
+  BeMeta* meta = reinterpret_cast<BeMeta*>(red + BE_MAXP * 2 * (C / 32));
+  float* svec = reinterpret_cast<float*>(meta + BE_MAXP);                // [BE_MAXP][4]
+  const int c = threadIdx.x;
   const int nw = C / 32, warp = c >> 5, lane = c & 31;
-  const long long n = e1 - e0;
-  for (long long base = (long long)blockIdx.x * BE_CHUNK; base < n; base += (long long)gridDim.x * BE_CHUNK) {
-    const int nch = (int)min((long long)BE_CHUNK, n - base);
-    __syncthreads();
-    {
-      const float4* src = reinterpret_cast<const float4*>(D + (size_t)(e0 + base) * NDBLK);
-      float4* dst = reinterpret_cast<float4*>(sD);
-      for (int q = tid; q < nch * (NDBLK / 4); q += nthr) dst[q] = src[q];
-    }
-    __syncthreads();
-#pragma unroll 1
-    for (int k = row; k < nch; k += EPB) {
-      const long long el = base + k;
-      const long long e = e0 + el;
-      float bx = 0.f, by = 0.f;
-      const float* Dr = sD + k * NDBLK;
-      const size_t rowoff = (size_t)el * 16 * C;
-      const float* xs = x + (size_t)send[e] * 16 * C + c;
-      const size_t rr = rrow ? (size_t)rrow[e] : (size_t)e;
-      const float* Rr = R + rr * 4 * C + c;
-      float* gHi = gR_hi + rr * 4 * C + c;
-      float* gLo = gR_lo + rr * 4 * C + c;
-      const float* yr = Y + rowoff + c;
-      const float* gyr = GY + rowoff + c;
-      const float* gxr = GXT + rowoff + c;
-      float* gsr = GXS + rowoff + c;
-      float gr;
-      bwd_edge_degree<0>(Dr, xs, yr, gyr, gxr, Rr[0], C, c, need_gx, gsr, gr, bx, by, scalar_in != 0);
-      gHi[0] = tf32_rna(gr);
-      gLo[0] = tf32_rna(gr - tf32_rna(gr));
-      bwd_edge_degree<1>(Dr, xs, yr, gyr, gxr, Rr[C], C, c, need_gx, gsr, gr, bx, by, scalar_in != 0);
-      gHi[C] = tf32_rna(gr);
-      gLo[C] = tf32_rna(gr - tf32_rna(gr));
-      bwd_edge_degree<2>(Dr, xs, yr, gyr, gxr, Rr[2 * C], C, c, need_gx, gsr, gr, bx, by, scalar_in != 0);
-      gHi[2 * C] = tf32_rna(gr);
-      gLo[2 * C] = tf32_rna(gr - tf32_rna(gr));
-      bwd_edge_degree<3>(Dr, xs, yr, gyr, gxr, Rr[3 * C], C, c, need_gx, gsr, gr, bx, by, scalar_in != 0);
-      gHi[3 * C] = tf32_rna(gr);
-      gLo[3 * C] = tf32_rna(gr - tf32_rna(gr));
-      // fixed-order reduction of (bx, by) over the warp, then per warp into shared memory
+  const int n = (int)(e1 - e0);
+  const int p0 = blockIdx.x * per, p1 = min(n, p0 + per);
+  if (p0 >= p1) return;
+  const int np = p1 - p0;
+  if (c == 0) {
+    for (int s = 0; s < BE_STAGES; ++s) tc::mbar_init(&full[s], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  for (int q = c; q < np; q += C) {
+    const int el = need_gx ? perm[e0 + p0 + q] : p0 + q;
+    const long long e = e0 + el;
+    meta[q] = BeMeta{el, rrow ? rrow[e] : (int)e, send[e], 0};
+    svec[4 * q + 0] = vec[3 * e];
+    svec[4 * q + 1] = vec[3 * e + 1];
+    svec[4 * q + 2] = vec[3 * e + 2];
+  }
+  __syncthreads();
+  // bytes of each section that the edge's arithmetic reads
+  const uint32_t bY = scalar_in ? 16u * C : 64u * C, bG = 64u * C, bX = scalar_in ? 4u * C : 64u * C;
+  const uint32_t bR = scalar_in ? 4u * C : 16u * C;
+  auto issue = [&](int q) {
+    const int s = q % BE_STAGES;
+    float* st = stage0 + s * SF;
+    const BeMeta m = meta[q];
+    tc::mbar_expect_tx(&full[s], bY + bG + bX + bX + bR + NDBLK * 4);
+    bulk_g2s(st, Y + (size_t)m.el * 16 * C, bY, &full[s]);
+    bulk_g2s(st + 16 * C, GY + (size_t)m.el * 16 * C, bG, &full[s]);
+    bulk_g2s(st + 32 * C, GXT + (size_t)m.el * 16 * C, bX, &full[s]);
+    bulk_g2s(st + 48 * C, x + (size_t)m.j * 16 * C, bX, &full[s]);
+    bulk_g2s(st + 64 * C, R + (size_t)m.rr * 4 * C, bR, &full[s]);
+    bulk_g2s(st + 68 * C, D + (size_t)(e0 + m.el) * NDBLK, NDBLK * 4, &full[s]);
+  };
+  if (c == 0)
+    for (int q = 0; q < min(BE_STAGES, np); ++q) issue(q);
+  float gxs[16];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        bx += __shfl_xor_sync(0xffffffffu, bx, o);
-        by += __shfl_xor_sync(0xffffffffu, by, o);
-      }
-      if (lane == 0) {
-        red[(k * 2 + 0) * nw + warp] = bx;
-        red[(k * 2 + 1) * nw + warp] = by;
-      }
+  for (int k = 0; k < 16; ++k) gxs[k] = 0.f;
+  int qs = 0;                          // first position of the current sender run piece
+#pragma unroll 1
+  for (int q = 0; q < np; ++q) {
+    const int s = q % BE_STAGES;
+    tc::mbar_wait(&full[s], (uint32_t)((q / BE_STAGES) & 1));   // bounded; a timeout sets the device error
+    const float* st = stage0 + s * SF;
+    const BeMeta m = meta[q];
+    const float* sY = st + c;
+    const float* sGY = st + 16 * C + c;
+    const float* sGX = st + 32 * C + c;
+    const float* sX = st + 48 * C + c;
+    const float* sR = st + 64 * C + c;
+    const float* Dr = st + 68 * C;
+    float* gHi = gR_hi + (size_t)m.rr * 4 * C + c;
+    float* gLo = gR_lo + (size_t)m.rr * 4 * C + c;
+    float bx = 0.f, by = 0.f, gr;
+    bwd_edge_degree<0>(Dr, sX, sY, sGY, sGX, sR[0], C, c, need_gx, gxs, gr, bx, by, scalar_in != 0);
+    gHi[0] = tf32_rna(gr);
+    gLo[0] = tf32_rna(gr - tf32_rna(gr));
+    bwd_edge_degree<1>(Dr, sX, sY, sGY, sGX, scalar_in ? 0.f : sR[C], C, c, need_gx, gxs, gr, bx, by, scalar_in != 0);
+    gHi[C] = tf32_rna(gr);
+    gLo[C] = tf32_rna(gr - tf32_rna(gr));
+    bwd_edge_degree<2>(Dr, sX, sY, sGY, sGX, scalar_in ? 0.f : sR[2 * C], C, c, need_gx, gxs, gr, bx, by, scalar_in != 0);
+    gHi[2 * C] = tf32_rna(gr);
+    gLo[2 * C] = tf32_rna(gr - tf32_rna(gr));
+    bwd_edge_degree<3>(Dr, sX, sY, sGY, sGX, scalar_in ? 0.f : sR[3 * C], C, c, need_gx, gxs, gr, bx, by, scalar_in != 0);
+    gHi[3 * C] = tf32_rna(gr);
+    gLo[3 * C] = tf32_rna(gr - tf32_rna(gr));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      bx += __shfl_xor_sync(0xffffffffu, bx, o);
+      by += __shfl_xor_sync(0xffffffffu, by, o);
     }
-    __syncthreads();
-    if (tid < nch) {
-      const int k = tid;
-      const long long e = e0 + base + k;
-      float sx = 0.f, sy = 0.f;
-      for (int w = 0; w < nw; ++w) {
-        sx += red[(k * 2 + 0) * nw + w];
-        sy += red[(k * 2 + 1) * nw + w];
-      }
-      const float vx = vec[3 * e], vy = vec[3 * e + 1], vz = vec[3 * e + 2];
-      const float d2 = vx * vx + vy * vy + vz * vz;
-      const float inv = rsqrtf(d2);
-      float Rf[3][3];
-      edge_frame<float>(vx * inv, vy * inv, vz * inv, Rf);
-      const float ax = -(Rf[0][0] * sx + Rf[1][0] * sy);
-      const float ay = -(Rf[0][1] * sx + Rf[1][1] * sy);
-      const float az = -(Rf[0][2] * sx + Rf[1][2] * sy);
-      const float id2 = 1.f / d2;
-      g_r[3 * e + 0] += (ay * vz - az * vy) * id2;
-      g_r[3 * e + 1] += (az * vx - ax * vz) * id2;
-      g_r[3 * e + 2] += (ax * vy - ay * vx) * id2;
+    if (lane == 0) {
+      red[(q * 2 + 0) * nw + warp] = bx;
+      red[(q * 2 + 1) * nw + warp] = by;
     }
+    if (need_gx && (q == np - 1 || meta[q + 1].j != m.j)) {
+      // end of a sender run piece: its sum becomes row Pg[first position of the piece]
+      float* dst = Pg + (size_t)(p0 + qs) * 16 * C + c;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        dst[k * C] = gxs[k];
+        gxs[k] = 0.f;
+      }
+      qs = q + 1;
+    }
+    __syncthreads();                   // stage s read by every thread: free for reuse
+    if (c == 0 && q + BE_STAGES < np) issue(q + BE_STAGES);
+  }
+  // torque of every edge of the range: a = -R_e^T (b_x, b_y, 0), g_r += (a x r) / |r|^2
+  for (int q = c; q < np; q += C) {
+    const long long e = e0 + meta[q].el;
+    float sx = 0.f, sy = 0.f;
+    for (int w = 0; w < nw; ++w) {
+      sx += red[(q * 2 + 0) * nw + w];
+      sy += red[(q * 2 + 1) * nw + w];
+    }
+    const float vx = svec[4 * q], vy = svec[4 * q + 1], vz = svec[4 * q + 2];
+    const float d2 = vx * vx + vy * vy + vz * vz;
+    const float inv = rsqrtf(d2);
+    float Rf[3][3];
+    edge_frame<float>(vx * inv, vy * inv, vz * inv, Rf);
+    const float ax = -(Rf[0][0] * sx + Rf[1][0] * sy);
+    const float ay = -(Rf[0][1] * sx + Rf[1][1] * sy);
+    const float az = -(Rf[0][2] * sx + Rf[1][2] * sy);
+    const float id2 = 1.f / d2;
+    g_r[3 * e + 0] += (ay * vz - az * vy) * id2;
+    g_r[3 * e + 1] += (az * vx - ax * vz) * id2;
+    g_r[3 * e + 2] += (ax * vy - ay * vx) * id2;
+  }
+  // every copy was waited for above; after a timed-out wait, wait (bounded) once more for the
+  // last copy into each stage so that none is still landing when the block exits
+  if (c == 0)
+    for (int s = 0; s < BE_STAGES && s < np; ++s) {
+      const int ql = s + ((np - 1 - s) / BE_STAGES) * BE_STAGES;
+      tc::mbar_wait(&full[s], (uint32_t)((ql / BE_STAGES) & 1));
+    }
+}
+
+// g_x[sender] += the cohort's sender runs, each the sum of its pieces in position order: a run
+// [b, en) has pieces starting at b and at every multiple of `per` inside it (rows of Pg).
+// Block (x, k): runs x, x + gridDim.x, ..., component k.
+__global__ void k_gx_combine(long long e0, long long e1, int C, int cohort_idx, int per, const int* __restrict__ send,
+                             const int* __restrict__ perm, const int* __restrict__ seg, const int* __restrict__ nseg,
+                             const float* __restrict__ Pg, float* __restrict__ gx) {
+  const int c = threadIdx.x, k = blockIdx.y;
+  const int ns = nseg[cohort_idx];
+  const int n = (int)(e1 - e0);
+  for (int r = blockIdx.x; r < ns; r += gridDim.x) {
+    const int b = seg[e0 + r], en = r + 1 < ns ? seg[e0 + r + 1] : n;
+    float acc = Pg[((size_t)b * 16 + k) * C + c];
+    for (int p = (b / per + 1) * per; p < en; p += per) acc += Pg[((size_t)p * 16 + k) * C + c];
+    float* g = gx + ((size_t)send[e0 + perm[e0 + b]] * 16 + k) * C + c;
+    *g += acc;
   }
 }
 
@@ -911,44 +1053,6 @@ __global__ void k_cohort_sort(long long E, int cohort, const int* __restrict__ s
   for (int k = b; k < en; ++k) {
     if (k == 0 || (keys[k] >> 21) != (keys[k - 1] >> 21)) seg[e0 + pos++] = k;
     perm[e0 + k] = (int)(keys[k] & ((1ull << 21) - 1));
-  }
-}
-
-// g_x[j] += sum over the cohort's edges with sender j (ascending edge) of GXS rows.
-// Rows are fetched four at a time and added in edge order.
-__global__ void k_sender_scatter(long long e0, long long e1, int C, int cohort_idx, const int* __restrict__ send,
-                                 const int* __restrict__ perm, const int* __restrict__ seg,
-                                 const int* __restrict__ nseg, const float* __restrict__ GXS,
-                                 float* __restrict__ gx) {
-  const int lane = threadIdx.x;
-  const int c = blockIdx.y * 32 + lane;
-  const int ns = nseg[cohort_idx];
-  const int n = (int)(e1 - e0);
-  for (int s = blockIdx.x; s < ns; s += gridDim.x) {
-    const int b = seg[e0 + s], en = (s + 1 < ns) ? seg[e0 + s + 1] : n;
-    const int j = send[e0 + perm[e0 + b]];
-    float acc[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-    for (int q = b; q < en; q += 4) {
-      const int cnt = min(4, en - q);
-      float v[4][16];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (u < cnt) {
-          const float* g = GXS + (size_t)perm[e0 + q + u] * 16 * C + c;
-#pragma unroll
-          for (int k = 0; k < 16; ++k) v[u][k] = g[k * C];
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (u < cnt)
-#pragma unroll
-          for (int k = 0; k < 16; ++k) acc[k] += v[u][k];
-    }
-#pragma unroll
-    for (int k = 0; k < 16; ++k) gx[((size_t)j * 16 + k) * C + c] += acc[k];
   }
 }
 

@@ -70,7 +70,7 @@ inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 
 // ------------------------------------------------------------------ workspace layout
 struct WsLayout {
-  size_t D, dist, R, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GY, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
+  size_t D, dist, R, rbP, gxP, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GY, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
   size_t total;
 };
 
@@ -85,6 +85,7 @@ WsLayout ws_layout(const Model& m, long long E, int N) {
   L.D = take((size_t)E * NDBLK * 4);
   L.dist = take((size_t)E * 4);
   L.R = take(T * (size_t)E * 4 * C * 4);
+  L.rbP = take(((coh + RB_CHUNK - 1) / RB_CHUNK) * 2 * 16 * C * 4);
   L.gRhi = take((size_t)E * 4 * C * 4);
   L.gRlo = take((size_t)E * 4 * C * 4);
   L.h2hi = take((size_t)E * 64 * 4);
@@ -101,6 +102,7 @@ WsLayout ws_layout(const Model& m, long long E, int N) {
   L.gS = take(feat);
   L.e_atom = take((size_t)N * 4);
   const size_t cb = coh * 16 * C * 4;
+  L.gxP = take(cb);
   L.XT = take(cb);
   L.Y = take(cb);
   L.GY = take(cb);
@@ -180,10 +182,10 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
   const int C = m.spec.C;
   const long long E = g->n_edges, coh = m.spec.cohort_edges;
   const dim3 eb = edge_block(C);
-  const size_t esmem = (size_t)eb.y * NDBLK * 4;
   float* XT = at<float>(ws, L.XT);
   float* XTlo = at<float>(ws, L.XTlo);
   float* Y = at<float>(ws, L.Y);
+  float* P = at<float>(ws, L.rbP);
   CohortMaps am;
   int st0 = am.build(C, E, coh, XT, XTlo);
   if (st0 != EMP_OK) return st0;
@@ -203,9 +205,9 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
       st = so2_product(m, e1 - e0, &part, 1, counter, s);
     }
     if (st != EMP_OK) return st;
-    const int cg = std::min(C, RB_CG);
-    dim3 grid((unsigned)std::min<long long>(coh, 128), C / cg);
-    { Scope sc_("rotate_back_scatter", s); k_rotate_back_scatter<<<grid, dim3(cg, RB_ROWS), sizeof(RbSmem), s>>>(e0, e1, C, scalar_in, g->recv, g->recv_off, D, Y, S); }
+    const int nchunks = (int)((e1 - e0 + RB_CHUNK - 1) / RB_CHUNK);
+    { Scope sc_("rotate_back_scatter", s); k_rb_chunks<<<nchunks, C, 0, s>>>(e0, e1, C, scalar_in, g->recv, g->recv_off, D, Y, S, P); }
+    { Scope sc_("rb_combine", s); k_rb_combine<<<dim3((unsigned)std::min<long long>(e1 - e0, 128), 16), C, 0, s>>>(e0, e1, C, g->recv, g->recv_off, P, S); }
   }
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
@@ -295,7 +297,7 @@ int ensure_attrs() {
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_pair_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * PS_THREADS * 4));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_radial_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(RadialSmem)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_cohort_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, 8 << 14));
-  EMP_CUDA_TRY(cudaFuncSetAttribute(k_rotate_back_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(RbSmem)));
+  EMP_CUDA_TRY(cudaFuncSetAttribute(k_bwd_edge, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)be_smem_bytes(256)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_chain_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ChainFwdSmem)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_chain_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ChainBwdSmem)));
   int st = so2_tc_init();
@@ -780,11 +782,17 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
         st = so2_product(m, n, parts, 2, counter, stream);
       }
       if (st != EMP_OK) return st;
-      const size_t smem = (size_t)BE_CHUNK * NDBLK * 4 + (size_t)BE_CHUNK * 2 * (C / 32) * 4;
-      { Scope sc_("bwd_edge", stream); k_bwd_edge<<<grid_for(n, BE_CHUNK), eb, smem, stream>>>(e0, e1, C, t > 0, t == 0, g->send, rr.inv, g->vec, D, R, xt, Y, GY, GXT, XT, gRhi, gRlo, g_r); }
+      // per-edge backward; for t > 0 also the sender sums of dE/dx_send into gxb
+      const int per = be_per(n, tc::num_sms());
+      const int nb = (int)((n + per - 1) / per);
+      float* Pg = at<float>(ws, L.gxP);
+      { Scope sc_("bwd_edge", stream); k_bwd_edge<<<nb, C, be_smem_bytes(C), stream>>>(
+            e0, e1, C, t > 0, t == 0, per, g->send, rr.inv, g->vec, D, R, xt, Y, GY, GXT, perm, gRhi, gRlo,
+            g_r, Pg); }
       if (t > 0) {
-        dim3 sg(std::min<long long>(n, 2048), C / 32);
-        { Scope sc_("sender_scatter", stream); k_sender_scatter<<<sg, 32, 0, stream>>>(e0, e1, C, ci, g->send, perm, seg, nseg, XT, gxb); }
+        Scope sc_("gx_combine", stream);
+        k_gx_combine<<<dim3((unsigned)std::min<long long>(n, 128), 16), C, 0, stream>>>(e0, e1, C, ci, per, g->send,
+                                                                                       perm, seg, nseg, Pg, gxb);
       }
     }
     if (E > 0) {
