@@ -398,50 +398,6 @@ __device__ __forceinline__ void rotate_write_degree(const float* __restrict__ Dr
   }
 }
 
-constexpr int BE_CHUNK = 16;   // edges whose Wigner-D blocks are staged per barrier pair
-
-// ------------------------------------------------------------------ rotate in
-// XT[e - e0][col(k) C + c] = R_e[l(k)][c] * (D_e x_send)[k][c]  (edge frame, m-major)
-// scalar_in: the input has only degree-0 components (the first layer, whose input is the
-// species embedding), so only the (l=0, m=0) column of x~ is non-zero and only it is written.
-__global__ void k_rotate_in(long long e0, long long e1, int C, int scalar_in, const int* __restrict__ send,
-                            const int* __restrict__ rrow, const float* __restrict__ D, const float* __restrict__ R,
-                            const float* __restrict__ x, float* __restrict__ XT, float* __restrict__ XTlo) {
-  extern __shared__ __align__(16) float sD[];           // [BE_CHUNK][84]
-  const int c = threadIdx.x, row = threadIdx.y, EPB = blockDim.y;
-  const int tid = row * C + c, nthr = C * EPB;
-  const long long n = e1 - e0;
-  for (long long base = (long long)blockIdx.x * BE_CHUNK; base < n; base += (long long)gridDim.x * BE_CHUNK) {
-    const int nch = (int)min((long long)BE_CHUNK, n - base);
-    __syncthreads();
-    {
-      const float4* src = reinterpret_cast<const float4*>(D + (size_t)(e0 + base) * NDBLK);
-      float4* dst = reinterpret_cast<float4*>(sD);
-      for (int q = tid; q < nch * (NDBLK / 4); q += nthr) dst[q] = src[q];
-    }
-    __syncthreads();
-    for (int k = row; k < nch; k += EPB) {
-      const long long el = base + k;
-      const long long e = e0 + el;
-      const int j = send[e];
-      const size_t rr = rrow ? (size_t)rrow[e] : (size_t)e;
-      if (scalar_in) {
-        const float v = R[rr * 4 * C + c] * x[(size_t)j * 16 * C + c], h = tf32_rna(v);
-        XT[(size_t)el * 16 * C + c] = h;
-        XTlo[(size_t)el * 16 * C + c] = tf32_rna(v - h);
-        continue;
-      }
-      const float* Dr = sD + k * NDBLK;
-      const size_t ro = (size_t)el * 16 * C + c;
-      const float* Rr = R + rr * 4 * C + c;
-      const float* xs = x + (size_t)j * 16 * C + c;
-      rotate_write_degree<0>(Dr, xs, C, Rr[0], nullptr, XT + ro, XTlo + ro);
-      rotate_write_degree<1>(Dr, xs, C, Rr[C], nullptr, XT + ro, XTlo + ro);
-      rotate_write_degree<2>(Dr, xs, C, Rr[2 * C], nullptr, XT + ro, XTlo + ro);
-      rotate_write_degree<3>(Dr, xs, C, Rr[3 * C], nullptr, XT + ro, XTlo + ro);
-    }
-  }
-}
 
 // ------------------------------------------------------------------ rotate back + receiver sums
 // S[i] (+)= sum over the cohort's edges of receiver i of D_e^T y_e.
@@ -541,10 +497,13 @@ __global__ void __launch_bounds__(256, 3) k_rb_chunks(long long e0, long long e1
 }
 
 // receivers of the cohort that cross a chunk boundary: S[i] = carried sum + chunk partials in
-// order.  Block (x, k): receivers first + x, first + x + gridDim.x, ..., component k; the
-// partials are fetched eight chunks at a time and added in chunk order.
+// order.  Block (x, k): receivers first + x, first + x + gridDim.x, ..., component k.  A
+// chunk's partial of receiver i is in slot 0 when i is the chunk's first receiver, which
+// holds for every chunk after the first one the receiver touches, and for that first one
+// when the receiver's edges start at the chunk's start.
 __global__ void k_rb_combine(long long e0, long long e1, int C, const int* __restrict__ recv,
                              const int* __restrict__ recv_off, const float* __restrict__ P, float* __restrict__ S) {
+  constexpr int B = 16;
   const int c = threadIdx.x, k = blockIdx.y;
   const int first = recv[e0], last = recv[e1 - 1];
   for (int i = first + blockIdx.x; i <= last; i += gridDim.x) {
@@ -554,18 +513,16 @@ __global__ void k_rb_combine(long long e0, long long e1, int C, const int* __res
     if (cf == cl) continue;
     float* Si = S + ((size_t)i * 16 + k) * C + c;
     float acc = recv_off[i] < e0 ? *Si : 0.f;
-    for (int ch0 = cf; ch0 <= cl; ch0 += 8) {
-      float v[8];
+    for (int ch0 = cf; ch0 <= cl; ch0 += B) {
+      float v[B];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < B; ++u) {
         const int ch = ch0 + u;
-        if (ch <= cl) {
-          const int slot = recv[e0 + (long long)ch * RB_CHUNK] == i ? 0 : 1;
-          v[u] = P[(((size_t)ch * 2 + slot) * 16 + k) * C + c];
-        }
+        const int slot = (ch > cf || lo == (long long)ch * RB_CHUNK) ? 0 : 1;
+        v[u] = ch <= cl ? P[(((size_t)ch * 2 + slot) * 16 + k) * C + c] : 0.f;
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
+      for (int u = 0; u < B; ++u)
         if (ch0 + u <= cl) acc += v[u];
     }
     *Si = acc;
@@ -676,63 +633,6 @@ __global__ void k_gate_bwd(int N, int C, float inv_avg, int gated, const float* 
   }
 }
 
-// per edge: XT = R (.) D x_send (recomputed) and GY = D gS[recv] (edge-frame output gradient)
-// per edge: XT = R (.) D x_send (recomputed, split) and GY = D gS[recv] (edge-frame output gradient,
-// fp32 and split).  scalar_in: x has degree 0 only, so only the (0,0) column of XT is non-zero and
-// only the m = 0 block of GY enters a product.
-__global__ void __launch_bounds__(256, 4) k_bwd_prep(long long e0, long long e1, int C, int scalar_in,
-                                                     const int* __restrict__ recv, const int* __restrict__ send,
-                                                     const int* __restrict__ rrow, const float* __restrict__ D,
-                                                     const float* __restrict__ R, const float* __restrict__ x,
-                                                     const float* __restrict__ gS, float* __restrict__ XT,
-                                                     float* __restrict__ XTlo, float* __restrict__ GY,
-                                                     float* __restrict__ GYhi, float* __restrict__ GYlo) {
-  extern __shared__ __align__(16) float sD[];
-  const int c = threadIdx.x, row = threadIdx.y, EPB = blockDim.y;
-  const long long n = e1 - e0;
-  for (long long base = (long long)blockIdx.x * EPB; base < n; base += (long long)gridDim.x * EPB) {
-    const long long el = base + row;
-    const bool ok = el < n;
-    const long long e = e0 + el;
-    __syncthreads();
-    if (ok)
-      for (int k = c; k < NDBLK; k += C) sD[row * NDBLK + k] = D[(size_t)e * NDBLK + k];
-    __syncthreads();
-    if (!ok) continue;
-    const float* Dr = sD + row * NDBLK;
-    const size_t ro = (size_t)el * 16 * C + c;
-    const size_t rr = rrow ? (size_t)rrow[e] : (size_t)e;
-    const float* Rr = R + rr * 4 * C + c;
-    const float* xs = x + (size_t)send[e] * 16 * C + c;
-    const float* gs = gS + (size_t)recv[e] * 16 * C + c;
-    rotate_write_degree<0>(Dr, xs, C, Rr[0], nullptr, XT + ro, XTlo + ro);
-    if (!scalar_in) {
-      rotate_write_degree<1>(Dr, xs, C, Rr[C], nullptr, XT + ro, XTlo + ro);
-      rotate_write_degree<2>(Dr, xs, C, Rr[2 * C], nullptr, XT + ro, XTlo + ro);
-      rotate_write_degree<3>(Dr, xs, C, Rr[3 * C], nullptr, XT + ro, XTlo + ro);
-    }
-    // with a degree-0 input only the m = 0 block of g_y (its first 4C columns) is split
-    rotate_write_degree<0>(Dr, gs, C, 1.f, GY + ro, GYhi + ro, GYlo + ro);
-    if (!scalar_in) {
-      rotate_write_degree<1>(Dr, gs, C, 1.f, GY + ro, GYhi + ro, GYlo + ro);
-      rotate_write_degree<2>(Dr, gs, C, 1.f, GY + ro, GYhi + ro, GYlo + ro);
-      rotate_write_degree<3>(Dr, gs, C, 1.f, GY + ro, GYhi + ro, GYlo + ro);
-    } else {
-      rotate_write_degree<1>(Dr, gs, C, 1.f, GY + ro, nullptr, nullptr);
-      rotate_write_degree<2>(Dr, gs, C, 1.f, GY + ro, nullptr, nullptr);
-      rotate_write_degree<3>(Dr, gs, C, 1.f, GY + ro, nullptr, nullptr);
-      // the m = 0 entries of degrees 1..3 are in the first block: split them too
-#pragma unroll
-      for (int l = 1; l < 4; ++l) {
-        const int col = col_of(l, 0) * C;
-        const float u = GY[ro + col], h = tf32_rna(u);
-        GYhi[ro + col] = h;
-        GYlo[ro + col] = tf32_rna(u - h);
-      }
-    }
-  }
-}
-
 // per edge, from y (recomputed), g_y and g_x~ = W^T g_y:
 //   gR[e][l][c] = sum_m g_x~ u;  g_u = R (.) g_x~;  g_xs = D^T g_u (-> GXS, [16][C] rows)
 //   b_j = sum_c (y^T J_j g_y + g_u^T J_j u), j = x, y (edge frame); a = -R_e^T (b_x, b_y, 0);
@@ -756,7 +656,7 @@ __device__ __forceinline__ void torque_pairs_l(const float* v, const float* w, f
 // degree-L part of the per-edge backward for one channel
 template <int L>
 __device__ __forceinline__ void bwd_edge_degree(const float* __restrict__ Dr, const float* __restrict__ xs,
-                                                const float* __restrict__ yrow, const float* __restrict__ gyrow,
+                                                const float* __restrict__ yrow, const float* __restrict__ gsrow,
                                                 const float* __restrict__ gxtrow, float Rl, int C, int c,
                                                 bool need_gx, float (&gxs)[16], float& grl,
                                                 float& bx, float& by, bool scalar_in) {
@@ -765,12 +665,17 @@ __device__ __forceinline__ void bwd_edge_degree(const float* __restrict__ Dr, co
   float v[W], u[W], gu[W];
   if (scalar_in && L > 0) {
     // input of degree 0 only: u, g_x~ and g_R vanish for L > 0 and y is non-zero only at m = 0,
-    // so only the y^T J g_y part of the torque remains
+    // so only the y^T J g_y part of the torque remains (g_y = D gS[recv], edge frame)
     grl = 0.f;
 #pragma unroll
+    for (int n = 0; n < W; ++n) gu[n] = gsrow[(O + n) * C];
+#pragma unroll
     for (int m = 0; m < W; ++m) {
+      float a = 0.f;
+#pragma unroll
+      for (int n = 0; n < W; ++n) a = fmaf(B[m * W + n], gu[n], a);
+      u[m] = a;
       v[m] = (m == L) ? yrow[col_of_k(O + m) * C] : 0.f;
-      u[m] = gyrow[col_of_k(O + m) * C];
     }
     torque_pairs_l<L>(v, u, bx, by);
     return;
@@ -793,11 +698,18 @@ __device__ __forceinline__ void bwd_edge_degree(const float* __restrict__ Dr, co
   }
   if (L > 0) {
     torque_pairs_l<L>(gu, u, bx, by);
+    // g_y = D gS[recv] (edge frame), recomputed from the receiver's row
+#pragma unroll
+    for (int n = 0; n < W; ++n) v[n] = gsrow[(O + n) * C];
 #pragma unroll
     for (int m = 0; m < W; ++m) {
-      v[m] = yrow[col_of_k(O + m) * C];
-      u[m] = gyrow[col_of_k(O + m) * C];
+      float a = 0.f;
+#pragma unroll
+      for (int n = 0; n < W; ++n) a = fmaf(B[m * W + n], v[n], a);
+      u[m] = a;
     }
+#pragma unroll
+    for (int m = 0; m < W; ++m) v[m] = yrow[col_of_k(O + m) * C];
     torque_pairs_l<L>(v, u, bx, by);
   }
   if (need_gx) {
@@ -818,8 +730,8 @@ __device__ __forceinline__ void bwd_edge_degree(const float* __restrict__ Dr, co
 // (a run, or the part of one that lies in the range) as row Pg[first position of the
 // piece]; k_gx_combine then adds every run's pieces to g_x[sender] in order.  Without
 // need_gx the positions are the cohort's edges in order.
-// The rows an edge reads (y, g_y, g_x~, x_send, R and its Wigner-D blocks, all
-// contiguous) are brought into a BE_STAGES-deep shared-memory ring by bulk copies
+// The rows an edge reads (y, g_x~, gS of the receiver, x of the sender, R and its
+// Wigner-D blocks, all contiguous) are brought into a BE_STAGES-deep shared-memory ring by bulk copies
 // (cp.async.bulk, completing on one mbarrier per stage) issued by thread 0 ahead of
 // use, so the loads of later edges overlap the arithmetic of the current one.  The
 // per-edge torque sums are kept per position and finished for the whole range at
@@ -828,10 +740,10 @@ constexpr int BE_STAGES = 3;
 constexpr int BE_MAXP = 64;           // positions per block at most
 
 struct BeMeta {
-  int el, rr, j, pad;                 // cohort-local row, radial row, sender
+  int el, rr, j, i;                   // cohort-local row, radial row, sender, receiver
 };
 
-// stage layout (floats): Y [16C] | GY [16C] | GXT [16C] | X [16C] | R [4C] | D [84]
+// stage layout (floats): Y [16C] | gS[recv] [16C] | GXT [16C] | X [16C] | R [4C] | D [84]
 __host__ __device__ inline size_t be_stage_floats(int C) { return (size_t)68 * C + NDBLK; }
 __host__ __device__ inline size_t be_smem_bytes(int C) {
   return BE_STAGES * be_stage_floats(C) * 4 + BE_STAGES * 8 + (size_t)BE_MAXP * 2 * (C / 32) * 4 +
@@ -853,9 +765,9 @@ __global__ void __launch_bounds__(256, 2)
     k_bwd_edge(long long e0, long long e1, int C, int need_gx, int scalar_in, int per,
                const int* __restrict__ send, const int* __restrict__ rrow, const float* __restrict__ vec,
                const float* __restrict__ D, const float* __restrict__ R, const float* __restrict__ x,
-               const float* __restrict__ Y, const float* __restrict__ GY, const float* __restrict__ GXT,
-               const int* __restrict__ perm, float* __restrict__ gR_hi, float* __restrict__ gR_lo,
-               float* __restrict__ g_r, float* __restrict__ Pg) {
+               const float* __restrict__ Y, const float* __restrict__ gS, const float* __restrict__ GXT,
+               const int* __restrict__ recv, const int* __restrict__ perm, float* __restrict__ gR_hi,
+               float* __restrict__ gR_lo, float* __restrict__ g_r, float* __restrict__ Pg) {
   extern __shared__ __align__(128) unsigned char be_smem[];
   const size_t SF = be_stage_floats(C);
   float* stage0 = reinterpret_cast<float*>(be_smem);
@@ -876,7 +788,7 @@ __global__ void __launch_bounds__(256, 2)
   for (int q = c; q < np; q += C) {
     const int el = need_gx ? perm[e0 + p0 + q] : p0 + q;
     const long long e = e0 + el;
-    meta[q] = BeMeta{el, rrow ? rrow[e] : (int)e, send[e], 0};
+    meta[q] = BeMeta{el, rrow ? rrow[e] : (int)e, send[e], recv[e]};
     svec[4 * q + 0] = vec[3 * e];
     svec[4 * q + 1] = vec[3 * e + 1];
     svec[4 * q + 2] = vec[3 * e + 2];
@@ -891,7 +803,7 @@ __global__ void __launch_bounds__(256, 2)
     const BeMeta m = meta[q];
     tc::mbar_expect_tx(&full[s], bY + bG + bX + bX + bR + NDBLK * 4);
     bulk_g2s(st, Y + (size_t)m.el * 16 * C, bY, &full[s]);
-    bulk_g2s(st + 16 * C, GY + (size_t)m.el * 16 * C, bG, &full[s]);
+    bulk_g2s(st + 16 * C, gS + (size_t)m.i * 16 * C, bG, &full[s]);
     bulk_g2s(st + 32 * C, GXT + (size_t)m.el * 16 * C, bX, &full[s]);
     bulk_g2s(st + 48 * C, x + (size_t)m.j * 16 * C, bX, &full[s]);
     bulk_g2s(st + 64 * C, R + (size_t)m.rr * 4 * C, bR, &full[s]);
@@ -910,7 +822,7 @@ __global__ void __launch_bounds__(256, 2)
     const float* st = stage0 + s * SF;
     const BeMeta m = meta[q];
     const float* sY = st + c;
-    const float* sGY = st + 16 * C + c;
+    const float* sGS = st + 16 * C + c;
     const float* sGX = st + 32 * C + c;
     const float* sX = st + 48 * C + c;
     const float* sR = st + 64 * C + c;
@@ -918,16 +830,16 @@ __global__ void __launch_bounds__(256, 2)
     float* gHi = gR_hi + (size_t)m.rr * 4 * C + c;
     float* gLo = gR_lo + (size_t)m.rr * 4 * C + c;
     float bx = 0.f, by = 0.f, gr;
-    bwd_edge_degree<0>(Dr, sX, sY, sGY, sGX, sR[0], C, c, need_gx, gxs, gr, bx, by, scalar_in != 0);
+    bwd_edge_degree<0>(Dr, sX, sY, sGS, sGX, sR[0], C, c, need_gx, gxs, gr, bx, by, scalar_in != 0);
     gHi[0] = tf32_rna(gr);
     gLo[0] = tf32_rna(gr - tf32_rna(gr));
-    bwd_edge_degree<1>(Dr, sX, sY, sGY, sGX, scalar_in ? 0.f : sR[C], C, c, need_gx, gxs, gr, bx, by, scalar_in != 0);
+    bwd_edge_degree<1>(Dr, sX, sY, sGS, sGX, scalar_in ? 0.f : sR[C], C, c, need_gx, gxs, gr, bx, by, scalar_in != 0);
     gHi[C] = tf32_rna(gr);
     gLo[C] = tf32_rna(gr - tf32_rna(gr));
-    bwd_edge_degree<2>(Dr, sX, sY, sGY, sGX, scalar_in ? 0.f : sR[2 * C], C, c, need_gx, gxs, gr, bx, by, scalar_in != 0);
+    bwd_edge_degree<2>(Dr, sX, sY, sGS, sGX, scalar_in ? 0.f : sR[2 * C], C, c, need_gx, gxs, gr, bx, by, scalar_in != 0);
     gHi[2 * C] = tf32_rna(gr);
     gLo[2 * C] = tf32_rna(gr - tf32_rna(gr));
-    bwd_edge_degree<3>(Dr, sX, sY, sGY, sGX, scalar_in ? 0.f : sR[3 * C], C, c, need_gx, gxs, gr, bx, by, scalar_in != 0);
+    bwd_edge_degree<3>(Dr, sX, sY, sGS, sGX, scalar_in ? 0.f : sR[3 * C], C, c, need_gx, gxs, gr, bx, by, scalar_in != 0);
     gHi[3 * C] = tf32_rna(gr);
     gLo[3 * C] = tf32_rna(gr - tf32_rna(gr));
 #pragma unroll
@@ -984,20 +896,143 @@ __global__ void __launch_bounds__(256, 2)
 
 // g_x[sender] += the cohort's sender runs, each the sum of its pieces in position order: a run
 // [b, en) has pieces starting at b and at every multiple of `per` inside it (rows of Pg).
-// Block (x, k): runs x, x + gridDim.x, ..., component k.
+// One block of C threads per run (runs x, x + gridDim.x, ...), all 16 components at once.
 __global__ void k_gx_combine(long long e0, long long e1, int C, int cohort_idx, int per, const int* __restrict__ send,
                              const int* __restrict__ perm, const int* __restrict__ seg, const int* __restrict__ nseg,
                              const float* __restrict__ Pg, float* __restrict__ gx) {
-  const int c = threadIdx.x, k = blockIdx.y;
+  const int c = threadIdx.x;
   const int ns = nseg[cohort_idx];
   const int n = (int)(e1 - e0);
   for (int r = blockIdx.x; r < ns; r += gridDim.x) {
     const int b = seg[e0 + r], en = r + 1 < ns ? seg[e0 + r + 1] : n;
-    float acc = Pg[((size_t)b * 16 + k) * C + c];
-    for (int p = (b / per + 1) * per; p < en; p += per) acc += Pg[((size_t)p * 16 + k) * C + c];
-    float* g = gx + ((size_t)send[e0 + perm[e0 + b]] * 16 + k) * C + c;
-    *g += acc;
+    float* g = gx + (size_t)send[e0 + perm[e0 + b]] * 16 * C + c;
+    float acc[16], old[16];
+    const float* P0 = Pg + (size_t)b * 16 * C + c;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      acc[k] = P0[k * C];
+      old[k] = g[k * C];
+    }
+    for (int p = (b / per + 1) * per; p < en; p += per) {
+      const float* Pp = Pg + (size_t)p * 16 * C + c;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) acc[k] += Pp[k * C];
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) g[k * C] = old[k] + acc[k];
   }
+}
+
+// ------------------------------------------------------------------ staged rotate-in / backward prep
+// Rotate-in (BWD = false): XT[e - e0][col(k) C + c] = R_e[l(k)][c] (D_e x_send)[k][c] in
+// the edge frame, m-major columns, split hi/lo for the products.  Backward prep (BWD =
+// true): also GY = D_e gS[recv] (edge-frame output gradient), split.  scalar_in: x has
+// degree 0 only (the first layer's input is the species embedding), so only the (0,0)
+// column of XT is non-zero, and only the m = 0 block of GY (the m = 0 entry of each
+// degree) enters a product.  One block of C threads per contiguous range of `per`
+// edges of the cohort.  The rows an edge reads (x of the
+// sender, gS of the receiver, R and its Wigner-D blocks) are brought into an
+// RS_STAGES-deep shared-memory ring by bulk copies issued by thread 0 ahead of use;
+// the split rows are written with coalesced stores.
+constexpr int RS_STAGES = 3;         // at most 4: the barriers take 32 bytes before the metadata
+
+__host__ __device__ inline size_t rs_stage_floats(int C, bool bwd) { return (size_t)(bwd ? 36 : 20) * C + NDBLK; }
+__host__ __device__ inline size_t rs_smem_bytes(int C, bool bwd) {
+  return RS_STAGES * rs_stage_floats(C, bwd) * 4 + 32 + (size_t)BE_MAXP * 4 * 4;
+}
+inline int rs_per(long long n, int sms, int blocks_per_sm) {
+  const long long want = (n + (long long)blocks_per_sm * sms - 1) / ((long long)blocks_per_sm * sms);
+  return (int)std::max<long long>(1, std::min<long long>(BE_MAXP, want));
+}
+
+template <bool BWD>
+__global__ void __launch_bounds__(256, 2)
+    k_rotate_staged(long long e0, long long e1, int C, int scalar_in, int per, const int* __restrict__ recv,
+                    const int* __restrict__ send, const int* __restrict__ rrow, const float* __restrict__ D,
+                    const float* __restrict__ R, const float* __restrict__ x, const float* __restrict__ gS,
+                    float* __restrict__ XT, float* __restrict__ XTlo, float* __restrict__ GYhi,
+                    float* __restrict__ GYlo) {
+  extern __shared__ __align__(128) unsigned char rs_smem[];
+  const size_t SF = rs_stage_floats(C, BWD);
+  float* stage0 = reinterpret_cast<float*>(rs_smem);
+  uint64_t* full = reinterpret_cast<uint64_t*>(rs_smem + RS_STAGES * SF * 4);
+  int4* meta = reinterpret_cast<int4*>(full + 4);                         // [BE_MAXP] (j, i, rr, -), 16-byte aligned
+  const int c = threadIdx.x;
+  const int n = (int)(e1 - e0);
+  const int p0 = blockIdx.x * per, p1 = min(n, p0 + per);
+  if (p0 >= p1) return;
+  const int np = p1 - p0;
+  if (c == 0) {
+    for (int s = 0; s < RS_STAGES; ++s) tc::mbar_init(&full[s], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  for (int q = c; q < np; q += C) {
+    const long long e = e0 + p0 + q;
+    meta[q] = make_int4(send[e], BWD ? recv[e] : 0, rrow ? rrow[e] : (int)e, 0);
+  }
+  __syncthreads();
+  const uint32_t bX = scalar_in ? 4u * C : 64u * C, bG = BWD ? 64u * C : 0u, bR = scalar_in ? 4u * C : 16u * C;
+  const int offG = 16 * C, offR = (BWD ? 32 : 16) * C, offD = offR + 4 * C;
+  auto issue = [&](int q) {
+    const int s = q % RS_STAGES;
+    float* st = stage0 + s * SF;
+    const int4 m = meta[q];
+    tc::mbar_expect_tx(&full[s], bX + bG + bR + NDBLK * 4);
+    bulk_g2s(st, x + (size_t)m.x * 16 * C, bX, &full[s]);
+    if (BWD) bulk_g2s(st + offG, gS + (size_t)m.y * 16 * C, bG, &full[s]);
+    bulk_g2s(st + offR, R + (size_t)m.z * 4 * C, bR, &full[s]);
+    bulk_g2s(st + offD, D + (size_t)(e0 + p0 + q) * NDBLK, NDBLK * 4, &full[s]);
+  };
+  if (c == 0)
+    for (int q = 0; q < min(RS_STAGES, np); ++q) issue(q);
+#pragma unroll 1
+  for (int q = 0; q < np; ++q) {
+    const int s = q % RS_STAGES;
+    tc::mbar_wait(&full[s], (uint32_t)((q / RS_STAGES) & 1));   // bounded; a timeout sets the device error
+    const float* st = stage0 + s * SF;
+    const float* sX = st + c;
+    const float* sR = st + offR + c;
+    const float* Dr = st + offD;
+    const size_t ro = (size_t)(p0 + q) * 16 * C + c;
+    if (scalar_in) {
+      const float v = sR[0] * sX[0], h = tf32_rna(v);
+      XT[ro] = h;
+      XTlo[ro] = tf32_rna(v - h);
+    } else {
+      rotate_write_degree<0>(Dr, sX, C, sR[0], nullptr, XT + ro, XTlo + ro);
+      rotate_write_degree<1>(Dr, sX, C, sR[C], nullptr, XT + ro, XTlo + ro);
+      rotate_write_degree<2>(Dr, sX, C, sR[2 * C], nullptr, XT + ro, XTlo + ro);
+      rotate_write_degree<3>(Dr, sX, C, sR[3 * C], nullptr, XT + ro, XTlo + ro);
+    }
+    if (BWD) {
+      const float* sG = st + offG + c;
+      if (!scalar_in) {
+        rotate_write_degree<0>(Dr, sG, C, 1.f, nullptr, GYhi + ro, GYlo + ro);
+        rotate_write_degree<1>(Dr, sG, C, 1.f, nullptr, GYhi + ro, GYlo + ro);
+        rotate_write_degree<2>(Dr, sG, C, 1.f, nullptr, GYhi + ro, GYlo + ro);
+        rotate_write_degree<3>(Dr, sG, C, 1.f, nullptr, GYhi + ro, GYlo + ro);
+      } else {
+        // the m = 0 entry of each degree: g_y[l][0] = sum_n D^l[0][n] gS[l][n]
+#pragma unroll
+        for (int l = 0; l < 4; ++l) {
+          const float* row0 = Dr + dblk_off(l) + l * (2 * l + 1);
+          float u = 0.f;
+          for (int k = 0; k < 2 * l + 1; ++k) u = fmaf(row0[k], sG[(l * l + k) * C], u);
+          const int col = col_of(l, 0) * C;
+          const float h = tf32_rna(u);
+          GYhi[ro + col] = h;
+          GYlo[ro + col] = tf32_rna(u - h);
+        }
+      }
+    }
+    __syncthreads();                   // stage s read by every thread: free for reuse
+    if (c == 0 && q + RS_STAGES < np) issue(q + RS_STAGES);
+  }
+  if (c == 0)
+    for (int s = 0; s < RS_STAGES && s < np; ++s) {
+      const int ql = s + ((np - 1 - s) / RS_STAGES) * RS_STAGES;
+      tc::mbar_wait(&full[s], (uint32_t)((ql / RS_STAGES) & 1));
+    }
 }
 
 // ------------------------------------------------------------------ cohort sender order

@@ -70,7 +70,7 @@ inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 
 // ------------------------------------------------------------------ workspace layout
 struct WsLayout {
-  size_t D, dist, R, rbP, gxP, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GY, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
+  size_t D, dist, R, rbP, gxP, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
   size_t total;
 };
 
@@ -105,7 +105,6 @@ WsLayout ws_layout(const Model& m, long long E, int N) {
   L.gxP = take(cb);
   L.XT = take(cb);
   L.Y = take(cb);
-  L.GY = take(cb);
   L.GXT = take(cb);
   L.XTlo = take(cb);
   L.GYhi = take(cb);
@@ -174,6 +173,65 @@ void split(const float* a, float* hi, float* lo, size_t n, cudaStream_t s) {
   { Scope sc_("split", s); k_split_tf32<<<grid_for((long long)n, 256, 148 * 16), 256, 0, s>>>(a, hi, lo, n); }
 }
 
+// A second stream per device and host thread for the short, latency-bound combine
+// kernels: each runs beside the next cohort's leading kernels and is joined back
+// before the first kernel that reads what it writes (or rewrites what it reads).  The
+// stream and its two events are created on the first call of the thread that is not
+// being captured; until then (and if creation fails) the combines run on the caller's
+// stream.  They are per thread so that calls from different host threads never share
+// an event; calls of one thread on different streams share the second stream, which
+// orders their combines but adds no other dependency.
+struct Side {
+  cudaStream_t aux = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  bool pending = false;       // a combine was issued on aux and not yet joined
+  cudaStream_t s = nullptr;
+  // run the launch f on aux after everything issued on s so far
+  template <typename F>
+  void run(F f) {
+    if (!aux) { f(s); return; }
+    cudaEventRecord(fork, s);
+    cudaStreamWaitEvent(aux, fork, 0);
+    f(aux);
+    cudaEventRecord(join, aux);
+    pending = true;
+  }
+  // make s wait for the last combine
+  void wait() {
+    if (aux && pending) cudaStreamWaitEvent(s, join, 0);
+    pending = false;
+  }
+};
+thread_local Side g_side[64];
+
+Side side_for(cudaStream_t s) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  Side out;
+  out.s = s;
+  if (dev < 0 || dev >= 64) return out;
+  Side& d = g_side[dev];
+  if (!d.aux) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return out;
+    cudaStream_t a = nullptr;
+    cudaEvent_t f = nullptr, j = nullptr;
+    if (cudaStreamCreateWithFlags(&a, cudaStreamNonBlocking) != cudaSuccess) { cudaGetLastError(); return out; }
+    if (cudaEventCreateWithFlags(&f, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&j, cudaEventDisableTiming) != cudaSuccess) {
+      cudaGetLastError();
+      return out;
+    }
+    d.aux = a;
+    d.fork = f;
+    d.join = j;
+  }
+  out.aux = d.aux;
+  out.fork = d.fork;
+  out.join = d.join;
+  return out;
+}
+
 // forward of layer t over all cohorts: S (raw receiver sums) from x
 // scalar_in: x has only degree-0 components (the first layer's species embedding); then only the
 // m = 0 block with its first C input columns contributes, and y is non-zero only in that block.
@@ -186,13 +244,19 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
   float* XTlo = at<float>(ws, L.XTlo);
   float* Y = at<float>(ws, L.Y);
   float* P = at<float>(ws, L.rbP);
+  Side side = side_for(s);
   CohortMaps am;
   int st0 = am.build(C, E, coh, XT, XTlo);
   if (st0 != EMP_OK) return st0;
   int* counter = at<int>(ws, L.counter);
   for (long long e0 = 0; e0 < E; e0 += coh) {
     const long long e1 = std::min(E, e0 + coh);
-    { Scope sc_("rotate_in", s); k_rotate_in<<<grid_for(e1 - e0, BE_CHUNK), eb, (size_t)BE_CHUNK * NDBLK * 4, s>>>(e0, e1, C, scalar_in, g->send, rrow, D, R, x, XT, XTlo); }
+    {
+      const int per = rs_per(e1 - e0, tc::num_sms(), 6);
+      Scope sc_("rotate_in", s);
+      k_rotate_staged<false><<<(unsigned)((e1 - e0 + per - 1) / per), C, rs_smem_bytes(C, false), s>>>(
+          e0, e1, C, scalar_in, per, g->recv, g->send, rrow, D, R, x, nullptr, XT, XTlo, nullptr, nullptr);
+    }
     int st;
     if (scalar_in) {
       const So2AMaps* a = am.get(e1 - e0);
@@ -206,9 +270,14 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
     }
     if (st != EMP_OK) return st;
     const int nchunks = (int)((e1 - e0 + RB_CHUNK - 1) / RB_CHUNK);
+    side.wait();        // the previous cohort's combine: S of its last receiver, and P
     { Scope sc_("rotate_back_scatter", s); k_rb_chunks<<<nchunks, C, 0, s>>>(e0, e1, C, scalar_in, g->recv, g->recv_off, D, Y, S, P); }
-    { Scope sc_("rb_combine", s); k_rb_combine<<<dim3((unsigned)std::min<long long>(e1 - e0, 128), 16), C, 0, s>>>(e0, e1, C, g->recv, g->recv_off, P, S); }
+    side.run([&](cudaStream_t q) {
+      Scope sc_("rb_combine", q);
+      k_rb_combine<<<dim3((unsigned)std::min<long long>(e1 - e0, 128), 16), C, 0, q>>>(e0, e1, C, g->recv, g->recv_off, P, S);
+    });
   }
+  side.wait();
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
 
@@ -298,6 +367,10 @@ int ensure_attrs() {
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_radial_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(RadialSmem)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_cohort_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, 8 << 14));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_bwd_edge, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)be_smem_bytes(256)));
+  EMP_CUDA_TRY(cudaFuncSetAttribute(k_rotate_staged<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)rs_smem_bytes(256, false)));
+  EMP_CUDA_TRY(cudaFuncSetAttribute(k_rotate_staged<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)rs_smem_bytes(256, true)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_chain_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ChainFwdSmem)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_chain_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ChainBwdSmem)));
   int st = so2_tc_init();
@@ -307,11 +380,10 @@ int ensure_attrs() {
 }
 
 int check_device() {
-  int dev = 0;
+  int dev = 0, major = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return EMP_ERR_UNSUPPORTED;
-  cudaDeviceProp p;
-  if (cudaGetDeviceProperties(&p, dev) != cudaSuccess) return EMP_ERR_UNSUPPORTED;
-  return p.major == 10 ? EMP_OK : EMP_ERR_UNSUPPORTED;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return EMP_ERR_UNSUPPORTED;
+  return major == 10 ? EMP_OK : EMP_ERR_UNSUPPORTED;
 }
 
 }  // namespace
@@ -708,7 +780,6 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
   float* XT = at<float>(ws, L.XT);
   float* XTlo = at<float>(ws, L.XTlo);
   float* Y = at<float>(ws, L.Y);
-  float* GY = at<float>(ws, L.GY);
   float* GYhi = at<float>(ws, L.GYhi);
   float* GYlo = at<float>(ws, L.GYlo);
   float* GXT = at<float>(ws, L.GXT);
@@ -718,6 +789,7 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
   const float inv_avg = 1.0f / m.spec.avg_degree;
   const dim3 eb = edge_block(C);
   int* counter = at<int>(ws, L.counter);
+  Side side = side_for(stream);
   CohortMaps am_xt, am_gy;
   st = am_xt.build(C, E, coh, XT, XTlo);
   if (st != EMP_OK) return st;
@@ -764,8 +836,12 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
     for (long long e0 = 0; e0 < E; e0 += coh, ++ci) {
       const long long e1 = std::min(E, e0 + coh), n = e1 - e0;
       const int grid = grid_for(n, eb.y);
-      { Scope sc_("bwd_prep", stream); k_bwd_prep<<<grid, eb, (size_t)eb.y * NDBLK * 4, stream>>>(e0, e1, C, t == 0, g->recv, g->send, rr.inv, D, R, xt, gS, XT, XTlo,
-                                                                  GY, GYhi, GYlo); }
+      {
+        const int per = rs_per(n, tc::num_sms(), 3);
+        Scope sc_("bwd_prep", stream);
+        k_rotate_staged<true><<<(unsigned)((n + per - 1) / per), C, rs_smem_bytes(C, true), stream>>>(
+            e0, e1, C, t == 0, per, g->recv, g->send, rr.inv, D, R, xt, gS, XT, XTlo, GYhi, GYlo);
+      }
       if (t == 0) {
         // degree-0 input: y needs only the m = 0 block's first C input columns, and only the
         // degree-0 part of dE/dx~ is used (the radial scale of l = 0)
@@ -786,15 +862,18 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
       const int per = be_per(n, tc::num_sms());
       const int nb = (int)((n + per - 1) / per);
       float* Pg = at<float>(ws, L.gxP);
+      side.wait();      // the previous cohort's combine has read Pg
       { Scope sc_("bwd_edge", stream); k_bwd_edge<<<nb, C, be_smem_bytes(C), stream>>>(
-            e0, e1, C, t > 0, t == 0, per, g->send, rr.inv, g->vec, D, R, xt, Y, GY, GXT, perm, gRhi, gRlo,
-            g_r, Pg); }
-      if (t > 0) {
-        Scope sc_("gx_combine", stream);
-        k_gx_combine<<<dim3((unsigned)std::min<long long>(n, 128), 16), C, 0, stream>>>(e0, e1, C, ci, per, g->send,
-                                                                                       perm, seg, nseg, Pg, gxb);
-      }
+            e0, e1, C, t > 0, t == 0, per, g->send, rr.inv, g->vec, D, R, xt, Y, gS, GXT, g->recv, perm, gRhi,
+            gRlo, g_r, Pg); }
+      if (t > 0)
+        side.run([&](cudaStream_t q) {
+          Scope sc_("gx_combine", q);
+          k_gx_combine<<<(unsigned)std::min<long long>(n, 2048), C, 0, q>>>(e0, e1, C, ci, per, g->send, perm, seg,
+                                                                          nseg, Pg, gxb);
+        });
     }
+    side.wait();        // g_x of this layer complete
     if (E > 0) {
       st = radial_backward(m, g, t, species, dist, rr, g_r, ws, L, stream);
       if (st != EMP_OK) return st;
