@@ -202,6 +202,62 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------------------ per-kernel HBM figures
+# Algorithmic HBM bytes per edge of each SIMT kernel family (layers after the first; the
+# first layer's input is degree 0 only, so it moves the m = 0 columns alone).  Node rows
+# gathered per edge (x of the sender, gS of the receiver; 33.5 MB arrays that stay in L2)
+# are not counted: their minimal HBM traffic is one read per layer.
+def alg_bytes(name: str, C: int, first: bool) -> float:
+    row = 16 * C * 4                      # one [16][C] fp32 row
+    d = 84 * 4                            # Wigner-D blocks
+    if name == "rotate_in":               # R row in; x~ hi/lo out
+        return (C * 4 + 2 * C * 4 + d) if first else (4 * C * 4 + 2 * row + d)
+    if name == "bwd_prep":                # R row in; x~ hi/lo and g_y hi/lo out
+        return (C * 4 + 2 * C * 4 + 2 * 4 * C * 4 + d) if first else (4 * C * 4 + 4 * row + d)
+    if name == "bwd_edge":                # y, g_x~, R, D in; dE/dR hi/lo out
+        return (4 * C * 4 + C * 4 + C * 4 + d + 2 * 4 * C * 4) if first else (2 * row + 4 * C * 4 + d + 2 * 4 * C * 4)
+    if name == "rotate_back_scatter":     # y, D in
+        return (4 * C * 4 + d) if first else (row + d)
+    if name == "radial_h2":               # d in; h2 hi/lo out
+        return 4 + 2 * 64 * 4
+    if name == "radial_head":             # h2 hi/lo in; R out (tensor-core product)
+        return 2 * 64 * 4 + 4 * C * 4
+    if name == "radial_head_bwd":         # dE/dR hi/lo in; dE/dh2 out
+        return 2 * 4 * C * 4 + 64 * 4
+    if name == "radial_bwd":              # d, dE/dh2 in; g_r read-modify-write
+        return 4 + 64 * 4 + 2 * 12
+    raise KeyError(name)
+
+
+def hbm_fractions(fam, steps: int, E: int, C: int, T: int, hbm_gbs: float):
+    out = {}
+    for name in ("rotate_in", "bwd_prep", "bwd_edge", "rotate_back_scatter", "radial_h2", "radial_head",
+                 "radial_head_bwd", "radial_bwd"):
+        if name not in fam or fam[name][0] <= 0:
+            continue
+        per_layer = [alg_bytes(name, C, t == 0) for t in range(T)]
+        bytes_step = E * sum(per_layer)
+        ms = fam[name][0] / steps
+        gbs = bytes_step / (ms * 1e-3) / 1e9
+        out[name] = {"ms": round(ms, 3), "alg_bytes_per_step": int(bytes_step), "achieved_gbs": round(gbs, 1),
+                     "frac_of_hbm": round(gbs / hbm_gbs, 3)}
+    return out
+
+
+# DRAM bytes per launch of the SO(2) mixing kernel, from one ncu capture (see profiles/),
+# valid only for the kernel source it was taken on (else the roofline's traffic is null).
+SO2_TRAFFIC = {"source_sha1": "11299b462d5f1927c735be9f437909bd68bd6a29", "bytes_per_launch": 197.7e6}
+
+
+def so2_traffic_per_launch():
+    import hashlib
+    src = os.path.join(ROOT, "edge_message_passing_b200", "csrc", "so2_tc.cuh")
+    if not SO2_TRAFFIC["source_sha1"] or not os.path.exists(src):
+        return None
+    h = hashlib.sha1(open(src, "rb").read()).hexdigest()
+    return SO2_TRAFFIC["bytes_per_launch"] if h == SO2_TRAFFIC["source_sha1"] else None
+
+
 # ------------------------------------------------------------------ our arm
 def run_ours(args):
     import torch
@@ -323,6 +379,7 @@ def run_ours(args):
     pk, pk_kind = peaks()
     dom = max(fam.items(), key=lambda kv: kv[1][0])[0] if fam else None
     C = spec.C
+    T = spec.n_layers
     fl_per_edge = 2 * 72 * C * C                      # useful flops of one SO(2) mixing of one edge
     so2_launches = fam.get("so2_tc", (0, 0))[1]
     roof = None
@@ -332,22 +389,29 @@ def run_ours(args):
         # backward transpose), in 2 launches per cohort (forward; grouped backward).  The first
         # layer's input is the species embedding (degree 0 only): its three products reduce to
         # the m = 0 block with C inputs (forward, recompute) or C outputs (transpose): 4C^2 each.
-        flops_step = E * 2 * C * C * (3 * 72 * (spec.n_layers - 1) + 3 * 4)
+        flops_step = E * 2 * C * C * (3 * 72 * (T - 1) + 3 * 4)
         achieved = flops_step * len(ptimes) / (fam["so2_tc"][0] * 1e-3) / 1e12
-        peak_tf32 = pk["bf16_tflops"] * TF32_OVER_BF16
-        peak = peak_tf32 / 3.0
+        # the mixing is timed inside the long step: the sustained BF16 figure is the reference
+        peak = pk["bf16_tflops_sustained"] * TF32_OVER_BF16 / 3.0
+        peak_burst = pk["bf16_tflops"] * TF32_OVER_BF16 / 3.0
+        traffic = so2_traffic_per_launch()
         roof = {"bound": "tensor", "kernel": "so2_tc (3xTF32 tcgen05 SO(2) mixing)", "achieved": achieved,
                 "flops_per_step": flops_step,
-                "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                "traffic_unit": "bytes per launch (DRAM read + write, ncu, mean of a forward and a grouped "
+                                "backward cohort launch)" if traffic else None,
                 "launch_ms": so2_ms, "launches_per_step": so2_launches / len(ptimes), "dominant": dom == "so2_tc",
-                "frac_vs_sustained": achieved / (pk["bf16_tflops_sustained"] * TF32_OVER_BF16 / 3.0),
+                "frac_vs_burst": achieved / peak_burst,
                 "peak_note": f"useful FP32 flops of the mixings actually required (2*72*C^2 per edge per "
                              f"mixing, 3 mixings per layer; 2*4*C^2 in the degree-0-input first layer) over the "
-                             f"summed launch event time, vs burst bf16 ({pk_kind}) x {TF32_OVER_BF16:.3f} "
-                             f"(TF32/BF16 nominal) / 3 (3xTF32); SM clock stays at max during the step"}
+                             f"summed launch event time (CUDA events on the launching stream), vs sustained "
+                             f"bf16 ({pk_kind}, the kernel runs inside a long step) x {TF32_OVER_BF16:.3f} "
+                             f"(TF32/BF16 nominal) / 3 (3xTF32); median SM clock during the step "
+                             f"{clk.summary().get('sm_mhz')} MHz"}
     elif dom is not None:
         roof = {"bound": "hbm", "kernel": dom, "achieved": None, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": None, "traffic": None}
+    hbm = hbm_fractions(fam, len(ptimes), E, C, T, pk["hbm_gbs"])
     kernel_ms = {k: round(v[0] / len(ptimes), 3) for k, v in sorted(fam.items(), key=lambda kv: -kv[1][0])}
 
     result = None
@@ -369,7 +433,7 @@ def run_ours(args):
                   "e2e": {"value": E * ws / (e2e_ms * 1e-3), "unit": "edges/s",
                           "h2d_bytes_per_step": int(pos_h.numel() * 8 + sp_h.numel() * 4),
                           "d2h_bytes_per_step": int(8 + N * 3 * 4)},
-                  "roofline": roof, "cpu_baseline": cpu, "kernel_ms_per_step": kernel_ms,
+                  "roofline": roof, "hbm_kernels": hbm, "cpu_baseline": cpu, "kernel_ms_per_step": kernel_ms,
                   "ns_per_atom": ms * 1e6 / N}
         print(json.dumps(result))
     if ws > 1:

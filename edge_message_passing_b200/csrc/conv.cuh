@@ -633,92 +633,136 @@ __global__ void k_gate_bwd(int N, int C, float inv_avg, int gated, const float* 
   }
 }
 
+// V adjacent channels per thread: float, float2 or float4 arithmetic, loads and stores
+template <int V> struct VecT;
+template <> struct VecT<1> { typedef float type; };
+template <> struct VecT<2> { typedef float2 type; };
+template <> struct VecT<4> { typedef float4 type; };
+
+__device__ __forceinline__ float vfma(float a, float b, float c) { return fmaf(a, b, c); }
+__device__ __forceinline__ float2 vfma(float a, float2 b, float2 c) { return make_float2(fmaf(a, b.x, c.x), fmaf(a, b.y, c.y)); }
+__device__ __forceinline__ float4 vfma(float a, float4 b, float4 c) {
+  return make_float4(fmaf(a, b.x, c.x), fmaf(a, b.y, c.y), fmaf(a, b.z, c.z), fmaf(a, b.w, c.w));
+}
+__device__ __forceinline__ float vmul(float a, float b) { return a * b; }
+__device__ __forceinline__ float2 vmul(float2 a, float2 b) { return make_float2(a.x * b.x, a.y * b.y); }
+__device__ __forceinline__ float4 vmul(float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); }
+template <typename T> __device__ __forceinline__ T vset(float v);
+template <> __device__ __forceinline__ float vset<float>(float v) { return v; }
+template <> __device__ __forceinline__ float2 vset<float2>(float v) { return make_float2(v, v); }
+template <> __device__ __forceinline__ float4 vset<float4>(float v) { return make_float4(v, v, v, v); }
+__device__ __forceinline__ void vsplit(float v, float& h, float& l) {
+  h = tf32_rna(v);
+  l = tf32_rna(v - h);
+}
+__device__ __forceinline__ void vsplit(float2 v, float2& h, float2& l) {
+  vsplit(v.x, h.x, l.x);
+  vsplit(v.y, h.y, l.y);
+}
+__device__ __forceinline__ void vsplit(float4 v, float4& h, float4& l) {
+  vsplit(v.x, h.x, l.x);
+  vsplit(v.y, h.y, l.y);
+  vsplit(v.z, h.z, l.z);
+  vsplit(v.w, h.w, l.w);
+}
+
+__device__ __forceinline__ float vsub(float a, float b) { return a - b; }
+__device__ __forceinline__ float2 vsub(float2 a, float2 b) { return make_float2(a.x - b.x, a.y - b.y); }
+__device__ __forceinline__ float vadd(float a, float b) { return a + b; }
+__device__ __forceinline__ float2 vadd(float2 a, float2 b) { return make_float2(a.x + b.x, a.y + b.y); }
+__device__ __forceinline__ float vscale(float a, float b) { return a * b; }
+__device__ __forceinline__ float2 vscale(float a, float2 b) { return make_float2(a * b.x, a * b.y); }
+__device__ __forceinline__ float hsum(float a) { return a; }
+__device__ __forceinline__ float hsum(float2 a) { return a.x + a.y; }
+__device__ __forceinline__ float vdot(float a, float b, float c) { return fmaf(a, b, c); }
+__device__ __forceinline__ float2 vdot(float2 a, float2 b, float2 c) { return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y)); }
+
 // per edge, from y (recomputed), g_y and g_x~ = W^T g_y:
 //   gR[e][l][c] = sum_m g_x~ u;  g_u = R (.) g_x~;  g_xs = D^T g_u (-> GXS, [16][C] rows)
 //   b_j = sum_c (y^T J_j g_y + g_u^T J_j u), j = x, y (edge frame); a = -R_e^T (b_x, b_y, 0);
 //   g_r[e] += (a x r) / |r|^2  (direction part of dE/dr; the radial part is added by k_radial_bwd)
 // J_x, J_y are antisymmetric and couple components of one degree whose |m| differ by
 // one, so v^T J w = sum over the structural pairs (a < b) of J_ab (v_a w_b - v_b w_a).
-template <int L>
-__device__ __forceinline__ void torque_pairs_l(const float* v, const float* w, float& bx, float& by) {
+template <int L, typename T>
+__device__ __forceinline__ void torque_pairs_l(const T* v, const T* w, T& bx, T& by) {
   // v, w: the 2L+1 components of degree L (local index m + L)
   constexpr int p0 = L == 1 ? 0 : L == 2 ? 2 : 8;
   constexpr int p1 = L == 1 ? 2 : L == 2 ? 8 : NJPAIR;
 #pragma unroll
   for (int p = p0; p < p1; ++p) {
     const int A = jpair_a(p) - L * L, B = jpair_b(p) - L * L;
-    const float q = v[A] * w[B] - v[B] * w[A];
-    bx = fmaf(c_jx[p], q, bx);
-    by = fmaf(c_jy[p], q, by);
+    const T q = vsub(vmul(v[A], w[B]), vmul(v[B], w[A]));
+    bx = vfma(c_jx[p], q, bx);
+    by = vfma(c_jy[p], q, by);
   }
 }
 
-// degree-L part of the per-edge backward for one channel
-template <int L>
-__device__ __forceinline__ void bwd_edge_degree(const float* __restrict__ Dr, const float* __restrict__ xs,
-                                                const float* __restrict__ yrow, const float* __restrict__ gsrow,
-                                                const float* __restrict__ gxtrow, float Rl, int C, int c,
-                                                bool need_gx, float (&gxs)[16], float& grl,
-                                                float& bx, float& by, bool scalar_in) {
+// degree-L part of the per-edge backward for V = sizeof(T) / 4 adjacent channels; the row
+// pointers are offset to the thread's first channel and have a stride of CV vectors
+template <int L, typename T>
+__device__ __forceinline__ void bwd_edge_degree(const float* __restrict__ Dr, const T* __restrict__ xs,
+                                                const T* __restrict__ yrow, const T* __restrict__ gsrow,
+                                                const T* __restrict__ gxtrow, T Rl, int CV, bool need_gx,
+                                                T (&gxs)[16], T& grl, T& bx, T& by, bool scalar_in) {
   constexpr int W = 2 * L + 1, O = L * L;
   const float* B = Dr + dblk_off(L);
-  float v[W], u[W], gu[W];
+  T v[W], u[W], gu[W];
   if (scalar_in && L > 0) {
     // input of degree 0 only: u, g_x~ and g_R vanish for L > 0 and y is non-zero only at m = 0,
     // so only the y^T J g_y part of the torque remains (g_y = D gS[recv], edge frame)
-    grl = 0.f;
+    grl = vset<T>(0.f);
 #pragma unroll
-    for (int n = 0; n < W; ++n) gu[n] = gsrow[(O + n) * C];
+    for (int n = 0; n < W; ++n) gu[n] = gsrow[(O + n) * CV];
 #pragma unroll
     for (int m = 0; m < W; ++m) {
-      float a = 0.f;
+      T a = vset<T>(0.f);
 #pragma unroll
-      for (int n = 0; n < W; ++n) a = fmaf(B[m * W + n], gu[n], a);
+      for (int n = 0; n < W; ++n) a = vfma(B[m * W + n], gu[n], a);
       u[m] = a;
-      v[m] = (m == L) ? yrow[col_of_k(O + m) * C] : 0.f;
+      v[m] = (m == L) ? yrow[col_of_k(O + m) * CV] : vset<T>(0.f);
     }
     torque_pairs_l<L>(v, u, bx, by);
     return;
   }
 #pragma unroll
-  for (int n = 0; n < W; ++n) v[n] = xs[(O + n) * C];
+  for (int n = 0; n < W; ++n) v[n] = xs[(O + n) * CV];
 #pragma unroll
   for (int m = 0; m < W; ++m) {
-    float a = 0.f;
+    T a = vset<T>(0.f);
 #pragma unroll
-    for (int n = 0; n < W; ++n) a = fmaf(B[m * W + n], v[n], a);
+    for (int n = 0; n < W; ++n) a = vfma(B[m * W + n], v[n], a);
     u[m] = a;
   }
-  grl = 0.f;
+  grl = vset<T>(0.f);
 #pragma unroll
   for (int m = 0; m < W; ++m) {
-    const float g = gxtrow[col_of_k(O + m) * C];
-    grl = fmaf(g, u[m], grl);
-    gu[m] = Rl * g;
+    const T g = gxtrow[col_of_k(O + m) * CV];
+    grl = vdot(g, u[m], grl);
+    gu[m] = vmul(Rl, g);
   }
   if (L > 0) {
     torque_pairs_l<L>(gu, u, bx, by);
     // g_y = D gS[recv] (edge frame), recomputed from the receiver's row
 #pragma unroll
-    for (int n = 0; n < W; ++n) v[n] = gsrow[(O + n) * C];
+    for (int n = 0; n < W; ++n) v[n] = gsrow[(O + n) * CV];
 #pragma unroll
     for (int m = 0; m < W; ++m) {
-      float a = 0.f;
+      T a = vset<T>(0.f);
 #pragma unroll
-      for (int n = 0; n < W; ++n) a = fmaf(B[m * W + n], v[n], a);
+      for (int n = 0; n < W; ++n) a = vfma(B[m * W + n], v[n], a);
       u[m] = a;
     }
 #pragma unroll
-    for (int m = 0; m < W; ++m) v[m] = yrow[col_of_k(O + m) * C];
+    for (int m = 0; m < W; ++m) v[m] = yrow[col_of_k(O + m) * CV];
     torque_pairs_l<L>(v, u, bx, by);
   }
   if (need_gx) {
 #pragma unroll
     for (int m = 0; m < W; ++m) {
-      float a = 0.f;
+      T a = vset<T>(0.f);
 #pragma unroll
-      for (int n = 0; n < W; ++n) a = fmaf(B[n * W + m], gu[n], a);
-      gxs[O + m] += a;
+      for (int n = 0; n < W; ++n) a = vfma(B[n * W + m], gu[n], a);
+      gxs[O + m] = vadd(gxs[O + m], a);
     }
   }
 }
@@ -736,7 +780,7 @@ __device__ __forceinline__ void bwd_edge_degree(const float* __restrict__ Dr, co
 // use, so the loads of later edges overlap the arithmetic of the current one.  The
 // per-edge torque sums are kept per position and finished for the whole range at
 // the end, by one thread per edge.
-constexpr int BE_STAGES = 3;
+constexpr int BE_STAGES = 2;
 constexpr int BE_MAXP = 64;           // positions per block at most
 
 struct BeMeta {
@@ -746,12 +790,12 @@ struct BeMeta {
 // stage layout (floats): Y [16C] | gS[recv] [16C] | GXT [16C] | X [16C] | R [4C] | D [84]
 __host__ __device__ inline size_t be_stage_floats(int C) { return (size_t)68 * C + NDBLK; }
 __host__ __device__ inline size_t be_smem_bytes(int C) {
-  return BE_STAGES * be_stage_floats(C) * 4 + BE_STAGES * 8 + (size_t)BE_MAXP * 2 * (C / 32) * 4 +
+  return BE_STAGES * be_stage_floats(C) * 4 + BE_STAGES * 8 + (size_t)BE_MAXP * 2 * ((C + 31) / 32) * 4 +
          BE_MAXP * sizeof(BeMeta) + BE_MAXP * 4 * 4;
 }
-// positions per block for a cohort of n edges on `sms` SMs (two blocks per SM)
+// positions per block for a cohort of n edges on `sms` SMs (three blocks per SM)
 inline int be_per(long long n, int sms) {
-  const long long want = (n + 2 * sms - 1) / (2 * sms);
+  const long long want = (n + 3 * sms - 1) / (3 * sms);
   return (int)std::max<long long>(1, std::min<long long>(BE_MAXP, want));
 }
 
@@ -761,6 +805,7 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
                : "memory");
 }
 
+template <int V>
 __global__ void __launch_bounds__(256, 2)
     k_bwd_edge(long long e0, long long e1, int C, int need_gx, int scalar_in, int per,
                const int* __restrict__ send, const int* __restrict__ rrow, const float* __restrict__ vec,
@@ -768,24 +813,27 @@ __global__ void __launch_bounds__(256, 2)
                const float* __restrict__ Y, const float* __restrict__ gS, const float* __restrict__ GXT,
                const int* __restrict__ recv, const int* __restrict__ perm, float* __restrict__ gR_hi,
                float* __restrict__ gR_lo, float* __restrict__ g_r, float* __restrict__ Pg) {
+  typedef typename VecT<V>::type T;
   extern __shared__ __align__(128) unsigned char be_smem[];
   const size_t SF = be_stage_floats(C);
   float* stage0 = reinterpret_cast<float*>(be_smem);
   uint64_t* full = reinterpret_cast<uint64_t*>(be_smem + BE_STAGES * SF * 4);
-  float* red = reinterpret_cast<float*>(full + BE_STAGES);               // [BE_MAXP][2][C/32]
-  BeMeta* meta = reinterpret_cast<BeMeta*>(red + BE_MAXP * 2 * (C / 32));
+  const int CV = C / V;
+  const int nw = (CV + 31) / 32;
+  float* red = reinterpret_cast<float*>(full + BE_STAGES);               // [BE_MAXP][2][nw]
+  BeMeta* meta = reinterpret_cast<BeMeta*>(red + BE_MAXP * 2 * nw);
   float* svec = reinterpret_cast<float*>(meta + BE_MAXP);                // [BE_MAXP][4]
-  const int c = threadIdx.x;
-  const int nw = C / 32, warp = c >> 5, lane = c & 31;
+  const int t = threadIdx.x;
+  const int warp = t >> 5, lane = t & 31;
   const int n = (int)(e1 - e0);
   const int p0 = blockIdx.x * per, p1 = min(n, p0 + per);
   if (p0 >= p1) return;
   const int np = p1 - p0;
-  if (c == 0) {
+  if (t == 0) {
     for (int s = 0; s < BE_STAGES; ++s) tc::mbar_init(&full[s], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  for (int q = c; q < np; q += C) {
+  for (int q = t; q < np; q += CV) {
     const int el = need_gx ? perm[e0 + p0 + q] : p0 + q;
     const long long e = e0 + el;
     meta[q] = BeMeta{el, rrow ? rrow[e] : (int)e, send[e], recv[e]};
@@ -809,63 +857,72 @@ __global__ void __launch_bounds__(256, 2)
     bulk_g2s(st + 64 * C, R + (size_t)m.rr * 4 * C, bR, &full[s]);
     bulk_g2s(st + 68 * C, D + (size_t)(e0 + m.el) * NDBLK, NDBLK * 4, &full[s]);
   };
-  if (c == 0)
+  if (t == 0)
     for (int q = 0; q < min(BE_STAGES, np); ++q) issue(q);
-  float gxs[16];
+  T gxs[16];
 #pragma unroll
-  for (int k = 0; k < 16; ++k) gxs[k] = 0.f;
+  for (int k = 0; k < 16; ++k) gxs[k] = vset<T>(0.f);
   int qs = 0;                          // first position of the current sender run piece
+  T* gHv = reinterpret_cast<T*>(gR_hi);
+  T* gLv = reinterpret_cast<T*>(gR_lo);
+  T* Pgv = reinterpret_cast<T*>(Pg);
 #pragma unroll 1
   for (int q = 0; q < np; ++q) {
     const int s = q % BE_STAGES;
     tc::mbar_wait(&full[s], (uint32_t)((q / BE_STAGES) & 1));   // bounded; a timeout sets the device error
     const float* st = stage0 + s * SF;
     const BeMeta m = meta[q];
-    const float* sY = st + c;
-    const float* sGS = st + 16 * C + c;
-    const float* sGX = st + 32 * C + c;
-    const float* sX = st + 48 * C + c;
-    const float* sR = st + 64 * C + c;
+    const T* sY = reinterpret_cast<const T*>(st) + t;
+    const T* sGS = reinterpret_cast<const T*>(st + 16 * C) + t;
+    const T* sGX = reinterpret_cast<const T*>(st + 32 * C) + t;
+    const T* sX = reinterpret_cast<const T*>(st + 48 * C) + t;
+    const T* sR = reinterpret_cast<const T*>(st + 64 * C) + t;
     const float* Dr = st + 68 * C;
-    float* gHi = gR_hi + (size_t)m.rr * 4 * C + c;
-    float* gLo = gR_lo + (size_t)m.rr * 4 * C + c;
-    float bx = 0.f, by = 0.f, gr;
-    bwd_edge_degree<0>(Dr, sX, sY, sGS, sGX, sR[0], C, c, need_gx, gxs, gr, bx, by, scalar_in != 0);
-    gHi[0] = tf32_rna(gr);
-    gLo[0] = tf32_rna(gr - tf32_rna(gr));
-    bwd_edge_degree<1>(Dr, sX, sY, sGS, sGX, scalar_in ? 0.f : sR[C], C, c, need_gx, gxs, gr, bx, by, scalar_in != 0);
-    gHi[C] = tf32_rna(gr);
-    gLo[C] = tf32_rna(gr - tf32_rna(gr));
-    bwd_edge_degree<2>(Dr, sX, sY, sGS, sGX, scalar_in ? 0.f : sR[2 * C], C, c, need_gx, gxs, gr, bx, by, scalar_in != 0);
-    gHi[2 * C] = tf32_rna(gr);
-    gLo[2 * C] = tf32_rna(gr - tf32_rna(gr));
-    bwd_edge_degree<3>(Dr, sX, sY, sGS, sGX, scalar_in ? 0.f : sR[3 * C], C, c, need_gx, gxs, gr, bx, by, scalar_in != 0);
-    gHi[3 * C] = tf32_rna(gr);
-    gLo[3 * C] = tf32_rna(gr - tf32_rna(gr));
+    const size_t go = (size_t)m.rr * 4 * CV + t;
+    T bx = vset<T>(0.f), by = vset<T>(0.f), gr, h, l;
+    const T zero = vset<T>(0.f);
+    bwd_edge_degree<0>(Dr, sX, sY, sGS, sGX, sR[0], CV, need_gx, gxs, gr, bx, by, scalar_in != 0);
+    vsplit(gr, h, l);
+    gHv[go] = h;
+    gLv[go] = l;
+    bwd_edge_degree<1>(Dr, sX, sY, sGS, sGX, scalar_in ? zero : sR[CV], CV, need_gx, gxs, gr, bx, by, scalar_in != 0);
+    vsplit(gr, h, l);
+    gHv[go + CV] = h;
+    gLv[go + CV] = l;
+    bwd_edge_degree<2>(Dr, sX, sY, sGS, sGX, scalar_in ? zero : sR[2 * CV], CV, need_gx, gxs, gr, bx, by, scalar_in != 0);
+    vsplit(gr, h, l);
+    gHv[go + 2 * CV] = h;
+    gLv[go + 2 * CV] = l;
+    bwd_edge_degree<3>(Dr, sX, sY, sGS, sGX, scalar_in ? zero : sR[3 * CV], CV, need_gx, gxs, gr, bx, by, scalar_in != 0);
+    vsplit(gr, h, l);
+    gHv[go + 3 * CV] = h;
+    gLv[go + 3 * CV] = l;
+    // fixed-order sums of (b_x, b_y) over this thread's channels, the warp, then (at the end) the warps
+    float sx = hsum(bx), sy = hsum(by);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      bx += __shfl_xor_sync(0xffffffffu, bx, o);
-      by += __shfl_xor_sync(0xffffffffu, by, o);
+      sx += __shfl_xor_sync(0xffffffffu, sx, o);
+      sy += __shfl_xor_sync(0xffffffffu, sy, o);
     }
     if (lane == 0) {
-      red[(q * 2 + 0) * nw + warp] = bx;
-      red[(q * 2 + 1) * nw + warp] = by;
+      red[(q * 2 + 0) * nw + warp] = sx;
+      red[(q * 2 + 1) * nw + warp] = sy;
     }
     if (need_gx && (q == np - 1 || meta[q + 1].j != m.j)) {
       // end of a sender run piece: its sum becomes row Pg[first position of the piece]
-      float* dst = Pg + (size_t)(p0 + qs) * 16 * C + c;
+      T* dst = Pgv + (size_t)(p0 + qs) * 16 * CV + t;
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
-        dst[k * C] = gxs[k];
-        gxs[k] = 0.f;
+        dst[k * CV] = gxs[k];
+        gxs[k] = zero;
       }
       qs = q + 1;
     }
     __syncthreads();                   // stage s read by every thread: free for reuse
-    if (c == 0 && q + BE_STAGES < np) issue(q + BE_STAGES);
+    if (t == 0 && q + BE_STAGES < np) issue(q + BE_STAGES);
   }
   // torque of every edge of the range: a = -R_e^T (b_x, b_y, 0), g_r += (a x r) / |r|^2
-  for (int q = c; q < np; q += C) {
+  for (int q = t; q < np; q += CV) {
     const long long e = e0 + meta[q].el;
     float sx = 0.f, sy = 0.f;
     for (int w = 0; w < nw; ++w) {
@@ -887,12 +944,15 @@ __global__ void __launch_bounds__(256, 2)
   }
   // every copy was waited for above; after a timed-out wait, wait (bounded) once more for the
   // last copy into each stage so that none is still landing when the block exits
-  if (c == 0)
+  if (t == 0)
     for (int s = 0; s < BE_STAGES && s < np; ++s) {
       const int ql = s + ((np - 1 - s) / BE_STAGES) * BE_STAGES;
       tc::mbar_wait(&full[s], (uint32_t)((ql / BE_STAGES) & 1));
     }
 }
+
+// channels per thread of the backward edge kernel
+constexpr int BE_V = 2;
 
 // g_x[sender] += the cohort's sender runs, each the sum of its pieces in position order: a run
 // [b, en) has pieces starting at b and at every multiple of `per` inside it (rows of Pg).
@@ -929,11 +989,11 @@ __global__ void k_gx_combine(long long e0, long long e1, int C, int cohort_idx, 
 // true): also GY = D_e gS[recv] (edge-frame output gradient), split.  scalar_in: x has
 // degree 0 only (the first layer's input is the species embedding), so only the (0,0)
 // column of XT is non-zero, and only the m = 0 block of GY (the m = 0 entry of each
-// degree) enters a product.  One block of C threads per contiguous range of `per`
-// edges of the cohort.  The rows an edge reads (x of the
-// sender, gS of the receiver, R and its Wigner-D blocks) are brought into an
-// RS_STAGES-deep shared-memory ring by bulk copies issued by thread 0 ahead of use;
-// the split rows are written with coalesced stores.
+// degree) enters a product.  One block of C/4 threads (four adjacent channels each,
+// float4 loads and stores) per contiguous range of `per` edges of the cohort.  The rows
+// an edge reads (x of the sender, gS of the receiver, R and its Wigner-D blocks) are
+// brought into an RS_STAGES-deep shared-memory ring by bulk copies issued by thread 0
+// ahead of use.
 constexpr int RS_STAGES = 3;         // at most 4: the barriers take 32 bytes before the metadata
 
 __host__ __device__ inline size_t rs_stage_floats(int C, bool bwd) { return (size_t)(bwd ? 36 : 20) * C + NDBLK; }
@@ -945,28 +1005,53 @@ inline int rs_per(long long n, int sms, int blocks_per_sm) {
   return (int)std::max<long long>(1, std::min<long long>(BE_MAXP, want));
 }
 
-template <bool BWD>
-__global__ void __launch_bounds__(256, 2)
+// degree-L block for V channels: rotate v (node layout, stride CV vectors) by D^L into the
+// edge frame, scale by Rl and store the 3xTF32 split into m-major columns
+template <int L, typename T>
+__device__ __forceinline__ void rotate_write_degree_v(const float* __restrict__ Dr, const T* __restrict__ v, int CV,
+                                                      T Rl, T* __restrict__ hi, T* __restrict__ lo) {
+  constexpr int W = 2 * L + 1, O = L * L;
+  const float* B = Dr + dblk_off(L);
+  T a[W];
+#pragma unroll
+  for (int n = 0; n < W; ++n) a[n] = v[(O + n) * CV];
+#pragma unroll
+  for (int m = 0; m < W; ++m) {
+    T u = vset<T>(0.f);
+#pragma unroll
+    for (int n = 0; n < W; ++n) u = vfma(B[m * W + n], a[n], u);
+    u = vmul(u, Rl);
+    T h, l;
+    vsplit(u, h, l);
+    const int col = col_of_k(O + m) * CV;
+    hi[col] = h;
+    lo[col] = l;
+  }
+}
+
+template <bool BWD, int V>
+__global__ void __launch_bounds__(256)
     k_rotate_staged(long long e0, long long e1, int C, int scalar_in, int per, const int* __restrict__ recv,
                     const int* __restrict__ send, const int* __restrict__ rrow, const float* __restrict__ D,
                     const float* __restrict__ R, const float* __restrict__ x, const float* __restrict__ gS,
                     float* __restrict__ XT, float* __restrict__ XTlo, float* __restrict__ GYhi,
                     float* __restrict__ GYlo) {
+  typedef typename VecT<V>::type T;
   extern __shared__ __align__(128) unsigned char rs_smem[];
   const size_t SF = rs_stage_floats(C, BWD);
   float* stage0 = reinterpret_cast<float*>(rs_smem);
   uint64_t* full = reinterpret_cast<uint64_t*>(rs_smem + RS_STAGES * SF * 4);
   int4* meta = reinterpret_cast<int4*>(full + 4);                         // [BE_MAXP] (j, i, rr, -), 16-byte aligned
-  const int c = threadIdx.x;
+  const int t = threadIdx.x, CV = C / V;
   const int n = (int)(e1 - e0);
   const int p0 = blockIdx.x * per, p1 = min(n, p0 + per);
   if (p0 >= p1) return;
   const int np = p1 - p0;
-  if (c == 0) {
+  if (t == 0) {
     for (int s = 0; s < RS_STAGES; ++s) tc::mbar_init(&full[s], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  for (int q = c; q < np; q += C) {
+  for (int q = t; q < np; q += CV) {
     const long long e = e0 + p0 + q;
     meta[q] = make_int4(send[e], BWD ? recv[e] : 0, rrow ? rrow[e] : (int)e, 0);
   }
@@ -983,57 +1068,68 @@ __global__ void __launch_bounds__(256, 2)
     bulk_g2s(st + offR, R + (size_t)m.z * 4 * C, bR, &full[s]);
     bulk_g2s(st + offD, D + (size_t)(e0 + p0 + q) * NDBLK, NDBLK * 4, &full[s]);
   };
-  if (c == 0)
+  if (t == 0)
     for (int q = 0; q < min(RS_STAGES, np); ++q) issue(q);
+  T* XTv = reinterpret_cast<T*>(XT);
+  T* XLv = reinterpret_cast<T*>(XTlo);
+  T* GHv = reinterpret_cast<T*>(GYhi);
+  T* GLv = reinterpret_cast<T*>(GYlo);
 #pragma unroll 1
   for (int q = 0; q < np; ++q) {
     const int s = q % RS_STAGES;
     tc::mbar_wait(&full[s], (uint32_t)((q / RS_STAGES) & 1));   // bounded; a timeout sets the device error
     const float* st = stage0 + s * SF;
-    const float* sX = st + c;
-    const float* sR = st + offR + c;
+    const T* sX = reinterpret_cast<const T*>(st) + t;
+    const T* sR = reinterpret_cast<const T*>(st + offR) + t;
     const float* Dr = st + offD;
-    const size_t ro = (size_t)(p0 + q) * 16 * C + c;
+    const size_t ro = (size_t)(p0 + q) * 16 * CV + t;
     if (scalar_in) {
-      const float v = sR[0] * sX[0], h = tf32_rna(v);
-      XT[ro] = h;
-      XTlo[ro] = tf32_rna(v - h);
+      T h, l;
+      vsplit(vmul(sR[0], sX[0]), h, l);
+      XTv[ro] = h;
+      XLv[ro] = l;
     } else {
-      rotate_write_degree<0>(Dr, sX, C, sR[0], nullptr, XT + ro, XTlo + ro);
-      rotate_write_degree<1>(Dr, sX, C, sR[C], nullptr, XT + ro, XTlo + ro);
-      rotate_write_degree<2>(Dr, sX, C, sR[2 * C], nullptr, XT + ro, XTlo + ro);
-      rotate_write_degree<3>(Dr, sX, C, sR[3 * C], nullptr, XT + ro, XTlo + ro);
+      rotate_write_degree_v<0>(Dr, sX, CV, sR[0], XTv + ro, XLv + ro);
+      rotate_write_degree_v<1>(Dr, sX, CV, sR[CV], XTv + ro, XLv + ro);
+      rotate_write_degree_v<2>(Dr, sX, CV, sR[2 * CV], XTv + ro, XLv + ro);
+      rotate_write_degree_v<3>(Dr, sX, CV, sR[3 * CV], XTv + ro, XLv + ro);
     }
     if (BWD) {
-      const float* sG = st + offG + c;
+      const T* sG = reinterpret_cast<const T*>(st + offG) + t;
+      const T one = vset<T>(1.f);
       if (!scalar_in) {
-        rotate_write_degree<0>(Dr, sG, C, 1.f, nullptr, GYhi + ro, GYlo + ro);
-        rotate_write_degree<1>(Dr, sG, C, 1.f, nullptr, GYhi + ro, GYlo + ro);
-        rotate_write_degree<2>(Dr, sG, C, 1.f, nullptr, GYhi + ro, GYlo + ro);
-        rotate_write_degree<3>(Dr, sG, C, 1.f, nullptr, GYhi + ro, GYlo + ro);
+        rotate_write_degree_v<0>(Dr, sG, CV, one, GHv + ro, GLv + ro);
+        rotate_write_degree_v<1>(Dr, sG, CV, one, GHv + ro, GLv + ro);
+        rotate_write_degree_v<2>(Dr, sG, CV, one, GHv + ro, GLv + ro);
+        rotate_write_degree_v<3>(Dr, sG, CV, one, GHv + ro, GLv + ro);
       } else {
         // the m = 0 entry of each degree: g_y[l][0] = sum_n D^l[0][n] gS[l][n]
 #pragma unroll
         for (int l = 0; l < 4; ++l) {
           const float* row0 = Dr + dblk_off(l) + l * (2 * l + 1);
-          float u = 0.f;
-          for (int k = 0; k < 2 * l + 1; ++k) u = fmaf(row0[k], sG[(l * l + k) * C], u);
-          const int col = col_of(l, 0) * C;
-          const float h = tf32_rna(u);
-          GYhi[ro + col] = h;
-          GYlo[ro + col] = tf32_rna(u - h);
+          T u = vset<T>(0.f);
+          for (int k = 0; k < 2 * l + 1; ++k) u = vfma(row0[k], sG[(l * l + k) * CV], u);
+          T h, lo;
+          vsplit(u, h, lo);
+          const int col = col_of(l, 0) * CV;
+          GHv[ro + col] = h;
+          GLv[ro + col] = lo;
         }
       }
     }
     __syncthreads();                   // stage s read by every thread: free for reuse
-    if (c == 0 && q + RS_STAGES < np) issue(q + RS_STAGES);
+    if (t == 0 && q + RS_STAGES < np) issue(q + RS_STAGES);
   }
-  if (c == 0)
+  if (t == 0)
     for (int s = 0; s < RS_STAGES && s < np; ++s) {
       const int ql = s + ((np - 1 - s) / RS_STAGES) * RS_STAGES;
       tc::mbar_wait(&full[s], (uint32_t)((ql / RS_STAGES) & 1));
     }
 }
+
+// vector widths (channels per thread) of the staged rotate kernels
+constexpr int RS_V_FWD = 4;
+constexpr int RS_V_BWD = 1;
 
 // ------------------------------------------------------------------ cohort sender order
 // For each cohort: its edges sorted by (sender, edge), the start of each sender

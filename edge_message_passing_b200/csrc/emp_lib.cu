@@ -254,7 +254,7 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
     {
       const int per = rs_per(e1 - e0, tc::num_sms(), 6);
       Scope sc_("rotate_in", s);
-      k_rotate_staged<false><<<(unsigned)((e1 - e0 + per - 1) / per), C, rs_smem_bytes(C, false), s>>>(
+      k_rotate_staged<false, RS_V_FWD><<<(unsigned)((e1 - e0 + per - 1) / per), C / RS_V_FWD, rs_smem_bytes(C, false), s>>>(
           e0, e1, C, scalar_in, per, g->recv, g->send, rrow, D, R, x, nullptr, XT, XTlo, nullptr, nullptr);
     }
     int st;
@@ -366,10 +366,10 @@ int ensure_attrs() {
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_pair_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * PS_THREADS * 4));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_radial_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(RadialSmem)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_cohort_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, 8 << 14));
-  EMP_CUDA_TRY(cudaFuncSetAttribute(k_bwd_edge, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)be_smem_bytes(256)));
-  EMP_CUDA_TRY(cudaFuncSetAttribute(k_rotate_staged<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  EMP_CUDA_TRY(cudaFuncSetAttribute(k_bwd_edge<BE_V>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)be_smem_bytes(256)));
+  EMP_CUDA_TRY(cudaFuncSetAttribute(k_rotate_staged<false, RS_V_FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)rs_smem_bytes(256, false)));
-  EMP_CUDA_TRY(cudaFuncSetAttribute(k_rotate_staged<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  EMP_CUDA_TRY(cudaFuncSetAttribute(k_rotate_staged<true, RS_V_BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)rs_smem_bytes(256, true)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_chain_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ChainFwdSmem)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_chain_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ChainBwdSmem)));
@@ -839,7 +839,7 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
       {
         const int per = rs_per(n, tc::num_sms(), 3);
         Scope sc_("bwd_prep", stream);
-        k_rotate_staged<true><<<(unsigned)((n + per - 1) / per), C, rs_smem_bytes(C, true), stream>>>(
+        k_rotate_staged<true, RS_V_BWD><<<(unsigned)((n + per - 1) / per), C / RS_V_BWD, rs_smem_bytes(C, true), stream>>>(
             e0, e1, C, t == 0, per, g->recv, g->send, rr.inv, D, R, xt, gS, XT, XTlo, GYhi, GYlo);
       }
       if (t == 0) {
@@ -863,7 +863,7 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
       const int nb = (int)((n + per - 1) / per);
       float* Pg = at<float>(ws, L.gxP);
       side.wait();      // the previous cohort's combine has read Pg
-      { Scope sc_("bwd_edge", stream); k_bwd_edge<<<nb, C, be_smem_bytes(C), stream>>>(
+      { Scope sc_("bwd_edge", stream); k_bwd_edge<BE_V><<<nb, C / BE_V, be_smem_bytes(C), stream>>>(
             e0, e1, C, t > 0, t == 0, per, g->send, rr.inv, g->vec, D, R, xt, Y, gS, GXT, g->recv, perm, gRhi,
             gRlo, g_r, Pg); }
       if (t > 0)
