@@ -246,7 +246,7 @@ def hbm_fractions(fam, steps: int, E: int, C: int, T: int, hbm_gbs: float):
 
 # DRAM bytes per launch of the SO(2) mixing kernel, from one ncu capture (see profiles/),
 # valid only for the kernel source it was taken on (else the roofline's traffic is null).
-SO2_TRAFFIC = {"source_sha1": "11299b462d5f1927c735be9f437909bd68bd6a29", "bytes_per_launch": 197.7e6}
+SO2_TRAFFIC = {"source_sha1": "aeb165151cca2f602305e04e9d1d07bfc712ea1e", "bytes_per_launch": 197e6}
 
 
 def so2_traffic_per_launch():

@@ -47,7 +47,7 @@ struct Group {
   int acol[MAXSUB];     // first A column of the sub-problem
   int K[MAXSUB];
   int N[MAXSUB];        // output columns
-  int bn[MAXSUB];       // tile width (MMA N): min(N, 256), a multiple of 16
+  int bn[MAXSUB];       // tile width (MMA N): tile_n(N), a multiple of 16 up to 256
   int ccol[MAXSUB];     // first output column
   int ntiles[MAXSUB];   // n-tiles per m-tile
   int first[MAXSUB + 1];// first tile index of each sub-problem (sub-problems ordered by decreasing K)
@@ -133,8 +133,13 @@ struct TileInfo {
 
 constexpr int TQ = 4;    // depth of the tile-index ring from the scheduler to the MMA and epilogue warps
 
+// Tile width (MMA N) of a product with N output columns: N itself up to 256; beyond that
+// the widest of 256, 192, 128 that divides N (no padded columns), else 256.
+__host__ __device__ constexpr int tile_n(int n) {
+  return n <= BN ? n : n % BN == 0 ? BN : n % 192 == 0 ? 192 : n % 128 == 0 ? 128 : BN;
+}
 // The products run on CTA pairs (cta_group::2); B tensor maps hold half-height tiles.
-__host__ __device__ constexpr int b_box_rows(int n) { return (n < BN ? n : BN) / 2; }
+__host__ __device__ constexpr int b_box_rows(int n) { return tile_n(n) / 2; }
 
 // ------------------------------------------------------------------ 2-SM form (cta_group::2)
 // A pair of CTAs (a cluster of 2 on neighbouring SMs) computes a 256 x bn tile with
@@ -528,7 +533,7 @@ inline int tc_group(long long M, int ldc, const GemmSub* subs, int nsub, int* co
     g.acol[q] = u.acol;
     g.K[q] = u.K;
     g.N[q] = u.N;
-    g.bn[q] = std::min(u.N, tc::BN);
+    g.bn[q] = tc::tile_n(u.N);
     g.ccol[q] = u.ccol;
     g.ntiles[q] = (u.N + g.bn[q] - 1) / g.bn[q];
     g.out[q] = u.out;
