@@ -170,7 +170,7 @@ __device__ __forceinline__ void radial_layer1(RadialSmem& s, int r0, int j0, flo
 #pragma unroll
   for (int b = 0; b < 4; ++b)
     *reinterpret_cast<float4*>(&s.h1T[j0 + b][r0]) =
-        make_float4(silu_f(z1[0][b]), silu_f(z1[1][b]), silu_f(z1[2][b]), silu_f(z1[3][b]));
+        make_float4(silu_fast(z1[0][b]), silu_fast(z1[1][b]), silu_fast(z1[2][b]), silu_fast(z1[3][b]));
 }
 
 // layer 2 of the thread's tile: z2[r][o] = sum_i W2[o][i] h1[r][i]
@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(RAD_THREADS) k_radial_h2(long long E, const in
       float hi[4], lo[4];
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
-        const float v = silu_f(z[q][b]);
+        const float v = silu_fast(z[q][b]);
         hi[b] = tf32_rna(v);
         lo[b] = tf32_rna(v - hi[b]);
       }
@@ -268,8 +268,8 @@ __global__ void __launch_bounds__(RAD_THREADS) k_radial_bwd(long long E, const i
 #pragma unroll
     for (int b = 0; b < 4; ++b)
       *reinterpret_cast<float4*>(&s.gT[j0 + b][r0]) =
-          make_float4(g[0][b] * dsilu_f(z2[0][b]), g[1][b] * dsilu_f(z2[1][b]), g[2][b] * dsilu_f(z2[2][b]),
-                      g[3][b] * dsilu_f(z2[3][b]));
+          make_float4(g[0][b] * dsilu_fast(z2[0][b]), g[1][b] * dsilu_fast(z2[1][b]), g[2][b] * dsilu_fast(z2[2][b]),
+                      g[3][b] * dsilu_fast(z2[3][b]));
     __syncthreads();
     // dE/dh1[r][i] = sum_o dE/dz2[r][o] W2[o][i]; dE/dz1 = dE/dh1 SiLU'(z1)
     float gh[4][4];
@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(RAD_THREADS) k_radial_bwd(long long E, const i
         float w = 0.f;
 #pragma unroll
         for (int n = 0; n < 8; ++n) w = fmaf(s.W1[(j0 + b) * 8 + n], s.de[r0 + q][n], w);
-        acc = fmaf(gh[q][b] * dsilu_f(z1[q][b]), w, acc);
+        acc = fmaf(gh[q][b] * dsilu_fast(z1[q][b]), w, acc);
       }
       part[q] = acc;
     }

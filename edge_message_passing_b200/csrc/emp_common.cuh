@@ -169,6 +169,14 @@ __host__ __device__ constexpr int jpair_b(int p) {
 }
 
 // ------------------------------------------------------------- misc math
+// SiLU and its derivative with the fast exponential and division intrinsics (a few ulp):
+// the radial network evaluates them 128-192 times per edge and layer
+__device__ __forceinline__ float sigmoid_fast(float z) { return __fdividef(1.0f, 1.0f + __expf(-z)); }
+__device__ __forceinline__ float silu_fast(float z) { return z * sigmoid_fast(z); }
+__device__ __forceinline__ float dsilu_fast(float z) {
+  const float s = sigmoid_fast(z);
+  return s * (1.0f + z * (1.0f - s));
+}
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
 __device__ __forceinline__ float dsilu_f(float z) {
   const float s = 1.0f / (1.0f + expf(-z));

@@ -70,7 +70,7 @@ inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 
 // ------------------------------------------------------------------ workspace layout
 struct WsLayout {
-  size_t D, dist, R, rbP, gxP, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
+  size_t D, dist, R, rbP, gxP, XT2, XTlo2, Y2, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
   size_t total;
 };
 
@@ -103,6 +103,9 @@ WsLayout ws_layout(const Model& m, long long E, int N) {
   L.e_atom = take((size_t)N * 4);
   const size_t cb = coh * 16 * C * 4;
   L.gxP = take(cb);
+  L.XT2 = take(cb);
+  L.XTlo2 = take(cb);
+  L.Y2 = take(cb);
   L.XT = take(cb);
   L.Y = take(cb);
   L.GXT = take(cb);
@@ -239,43 +242,58 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
                   int scalar_in, float* S, void* ws, const WsLayout& L, cudaStream_t s) {
   const int C = m.spec.C;
   const long long E = g->n_edges, coh = m.spec.cohort_edges;
-  const dim3 eb = edge_block(C);
-  float* XT = at<float>(ws, L.XT);
-  float* XTlo = at<float>(ws, L.XTlo);
-  float* Y = at<float>(ws, L.Y);
+  float* XT[2] = {at<float>(ws, L.XT), at<float>(ws, L.XT2)};
+  float* XTlo[2] = {at<float>(ws, L.XTlo), at<float>(ws, L.XTlo2)};
+  float* Y[2] = {at<float>(ws, L.Y), at<float>(ws, L.Y2)};
   float* P = at<float>(ws, L.rbP);
   Side side = side_for(s);
-  CohortMaps am;
-  int st0 = am.build(C, E, coh, XT, XTlo);
-  if (st0 != EMP_OK) return st0;
+  CohortMaps am[2];
+  for (int b = 0; b < 2; ++b) {
+    const int st0 = am[b].build(C, E, coh, XT[b], XTlo[b]);
+    if (st0 != EMP_OK) return st0;
+  }
   int* counter = at<int>(ws, L.counter);
-  for (long long e0 = 0; e0 < E; e0 += coh) {
+  // Cohorts are taken two at a time (a shorter last cohort alone): both are rotated in, then
+  // one grouped launch computes both cohorts' products (twice the tiles, so the CTA pairs
+  // stay evenly loaded), then the receiver sums run cohort by cohort, in order.
+  for (long long e0 = 0; e0 < E;) {
     const long long e1 = std::min(E, e0 + coh);
-    {
-      const int per = rs_per(e1 - e0, tc::num_sms(), 6);
+    const bool two = e1 < E && std::min(E, e1 + coh) - e1 == e1 - e0;
+    const long long ee[3] = {e0, e1, two ? e1 + (e1 - e0) : e1};
+    const int nc = two ? 2 : 1;
+    const long long M = e1 - e0;
+    for (int b = 0; b < nc; ++b) {
+      const int per = rs_per(M, tc::num_sms(), 6);
       Scope sc_("rotate_in", s);
-      k_rotate_staged<false, RS_V_FWD><<<(unsigned)((e1 - e0 + per - 1) / per), C / RS_V_FWD, rs_smem_bytes(C, false), s>>>(
-          e0, e1, C, scalar_in, per, g->recv, g->send, rrow, D, R, x, nullptr, XT, XTlo, nullptr, nullptr);
+      k_rotate_staged<false, RS_V_FWD><<<(unsigned)((M + per - 1) / per), C / RS_V_FWD, rs_smem_bytes(C, false), s>>>(
+          ee[b], ee[b + 1], C, scalar_in, per, g->recv, g->send, rrow, D, R, x, nullptr, XT[b], XTlo[b], nullptr, nullptr);
     }
     int st;
     if (scalar_in) {
-      const So2AMaps* a = am.get(e1 - e0);
       const MapPair& b0 = m.bmaps_fwd[t].blk[0];
-      GemmSub sub{&a->hi, &a->lo, &b0.hi, &b0.lo, 0, C, 4 * C, 0, Y};
+      GemmSub subs[2];
+      for (int b = 0; b < nc; ++b) {
+        const So2AMaps* a = am[b].get(M);
+        subs[b] = GemmSub{&a->hi, &a->lo, &b0.hi, &b0.lo, 0, C, 4 * C, 0, Y[b]};
+      }
       Scope sc_("so2_tc", s);
-      st = tc_group(e1 - e0, 16 * C, &sub, 1, counter, s);
+      st = tc_group(M, 16 * C, subs, nc, counter, s);
     } else {
-      So2Part part{am.get(e1 - e0), &m.bmaps_fwd[t], Y};
-      st = so2_product(m, e1 - e0, &part, 1, counter, s);
+      So2Part parts[2] = {{am[0].get(M), &m.bmaps_fwd[t], Y[0]}, {am[1].get(M), &m.bmaps_fwd[t], Y[1]}};
+      st = so2_product(m, M, parts, nc, counter, s);
     }
     if (st != EMP_OK) return st;
-    const int nchunks = (int)((e1 - e0 + RB_CHUNK - 1) / RB_CHUNK);
-    side.wait();        // the previous cohort's combine: S of its last receiver, and P
-    { Scope sc_("rotate_back_scatter", s); k_rb_chunks<<<nchunks, C, 0, s>>>(e0, e1, C, scalar_in, g->recv, g->recv_off, D, Y, S, P); }
-    side.run([&](cudaStream_t q) {
-      Scope sc_("rb_combine", q);
-      k_rb_combine<<<dim3((unsigned)std::min<long long>(e1 - e0, 128), 16), C, 0, q>>>(e0, e1, C, g->recv, g->recv_off, P, S);
-    });
+    for (int b = 0; b < nc; ++b) {
+      const long long c0 = ee[b], c1 = ee[b + 1];
+      const int nchunks = (int)((c1 - c0 + RB_CHUNK - 1) / RB_CHUNK);
+      side.wait();        // the previous cohort's combine: S of its last receiver, and P
+      { Scope sc_("rotate_back_scatter", s); k_rb_chunks<<<nchunks, C, 0, s>>>(c0, c1, C, scalar_in, g->recv, g->recv_off, D, Y[b], S, P); }
+      side.run([&](cudaStream_t q) {
+        Scope sc_("rb_combine", q);
+        k_rb_combine<<<dim3((unsigned)std::min<long long>(c1 - c0, 128), 16), C, 0, q>>>(c0, c1, C, g->recv, g->recv_off, P, S);
+      });
+    }
+    e0 = ee[2];
   }
   side.wait();
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
