@@ -951,8 +951,9 @@ __global__ void __launch_bounds__(256, 2)
     }
 }
 
-// channels per thread of the backward edge kernel
-constexpr int BE_V = 2;
+// channels per thread of the backward edge kernel: two when the C / 2 threads fill whole
+// warps (the torque sums reduce over full warps), else one
+inline int be_v(int C) { return C % 64 == 0 ? 2 : 1; }
 
 // g_x[sender] += the cohort's sender runs, each the sum of its pieces in position order: a run
 // [b, en) has pieces starting at b and at every multiple of `per` inside it (rows of Pg).

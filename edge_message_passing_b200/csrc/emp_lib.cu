@@ -384,7 +384,8 @@ int ensure_attrs() {
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_pair_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * PS_THREADS * 4));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_radial_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(RadialSmem)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_cohort_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, 8 << 14));
-  EMP_CUDA_TRY(cudaFuncSetAttribute(k_bwd_edge<BE_V>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)be_smem_bytes(256)));
+  EMP_CUDA_TRY(cudaFuncSetAttribute(k_bwd_edge<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)be_smem_bytes(256)));
+  EMP_CUDA_TRY(cudaFuncSetAttribute(k_bwd_edge<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)be_smem_bytes(256)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_rotate_staged<false, RS_V_FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)rs_smem_bytes(256, false)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_rotate_staged<true, RS_V_BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -881,9 +882,12 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
       const int nb = (int)((n + per - 1) / per);
       float* Pg = at<float>(ws, L.gxP);
       side.wait();      // the previous cohort's combine has read Pg
-      { Scope sc_("bwd_edge", stream); k_bwd_edge<BE_V><<<nb, C / BE_V, be_smem_bytes(C), stream>>>(
-            e0, e1, C, t > 0, t == 0, per, g->send, rr.inv, g->vec, D, R, xt, Y, gS, GXT, g->recv, perm, gRhi,
-            gRlo, g_r, Pg); }
+      {
+        Scope sc_("bwd_edge", stream);
+        auto kern = be_v(C) == 2 ? k_bwd_edge<2> : k_bwd_edge<1>;
+        kern<<<nb, C / be_v(C), be_smem_bytes(C), stream>>>(e0, e1, C, t > 0, t == 0, per, g->send, rr.inv, g->vec, D, R,
+                                                           xt, Y, gS, GXT, g->recv, perm, gRhi, gRlo, g_r, Pg);
+      }
       if (t > 0)
         side.run([&](cudaStream_t q) {
           Scope sc_("gx_combine", q);

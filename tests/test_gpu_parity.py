@@ -95,7 +95,7 @@ def _to_cols(x, C):
     return out
 
 
-@pytest.mark.parametrize("C,M", [(32, 300), (64, 128), (128, 1000)])
+@pytest.mark.parametrize("C,M", [(32, 300), (64, 128), (96, 257), (128, 1000), (256, 300)])
 @pytest.mark.parametrize("transpose", [False, True])
 def test_so2_mix_matches_oracle(C, M, transpose):
     spec = synth.ModelSpec(C=C, n_layers=1)
@@ -158,6 +158,13 @@ def _check_ef(w, cohort=None, virial=True):
 @pytest.mark.parametrize("cohort", [8192, 128])
 def test_energy_forces_small_gated(cohort):
     _check_ef(synth.small_workload(ncell=1, C=32, n_layers=2, gated=True, sigma=0.1), cohort=cohort)
+
+
+@pytest.mark.parametrize("C", [96, 256])
+def test_energy_forces_other_widths(C):
+    """Channel counts off the bench's: 96 (one channel per thread in the backward edge
+    kernel, 192-wide product tiles) and 256 (the largest the library accepts)."""
+    _check_ef(synth.small_workload(ncell=1, C=C, n_layers=2, gated=True, sigma=0.1), cohort=512)
 
 
 def test_energy_forces_small_pair_radial():
