@@ -258,6 +258,63 @@ def so2_traffic_per_launch():
     return SO2_TRAFFIC["bytes_per_launch"] if h == SO2_TRAFFIC["source_sha1"] else None
 
 
+# ------------------------------------------------------------------ the other seeded configs
+def other_configs(emp, torch, stream, flush, hbm_gbs: float, steps: int = 10):
+    """Edges/s and ns/atom of the energy + force call on the other seeded workloads (the
+    same timing: CUDA events, L2 flushed between steps, neighbour graph resident), and
+    the radial fold chain (forward + input gradient) against the HBM roofline."""
+    out = {}
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(steps):
+            flush.fill_(1.0)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return sum(ts) / len(ts)
+
+    for name in ("n64_diamond", "n512_diamond", "ternary_n2000"):
+        w = synth.workload(name)
+        st, spec = w.structure, w.spec
+        model = emp.Model(spec, w.weights)
+        pos = torch.from_numpy(st.pos).cuda()
+        sp = torch.from_numpy(st.species).cuda()
+        g = emp.nl_build(pos, st.box, spec.cutoff)
+        if spec.pair_radial:
+            fn = lambda: emp.mp_energy_forces(model, g, sp)           # eager: one pair-offset read-back per call
+            how = "eager call"
+        else:
+            efg = emp.EnergyForcesGraph(model, g, sp)
+            fn = efg.replay
+            how = "CUDA-graph replay"
+        ms = timed(fn)
+        N = st.pos.shape[0]
+        out[name] = {"n_atoms": N, "n_edges": g.n_edges, "C": spec.C, "layers": spec.n_layers,
+                     "ms_per_step": round(ms, 4), "edges_per_s": g.n_edges / (ms * 1e-3),
+                     "ns_per_atom": ms * 1e6 / N, "timed": how}
+        del model, g
+    ci = synth.chain_inputs()
+    ch = emp.Chain(ci.U, ci.M)
+    x, gk, gy = (torch.from_numpy(t).cuda() for t in (ci.x, ci.g_kc, ci.g_y0))
+    E = x.shape[0]
+    bufs = (torch.empty((E, 25), device="cuda"), torch.empty((E, 64), device="cuda"), torch.empty_like(x))
+    ms = timed(lambda: emp.mp_radial_chain(ch, x, gk, gy, out=bufs))
+    alg = E * (4 * 32 * 4 + 25 * 4 + 64 * 4) + E * (25 * 4 + 64 * 4 + 4 * 32 * 4)   # forward + input gradient
+    gbs = alg / (ms * 1e-3) / 1e9
+    out["radial_chain"] = {"rows": E, "ms": round(ms, 4), "alg_bytes": alg, "achieved_gbs": round(gbs, 1),
+                           "frac_of_hbm": round(gbs / hbm_gbs, 3),
+                           "note": "forward (x -> kc, y0) + input gradient (g_kc, g_y0 -> g_x) per call"}
+    return out
+
+
 # ------------------------------------------------------------------ our arm
 def run_ours(args):
     import torch
@@ -412,6 +469,7 @@ def run_ours(args):
         roof = {"bound": "hbm", "kernel": dom, "achieved": None, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": None, "traffic": None}
     hbm = hbm_fractions(fam, len(ptimes), E, C, T, pk["hbm_gbs"])
+    configs = other_configs(emp, torch, stream, flush, pk["hbm_gbs"]) if (ws == 1 and not args.no_configs) else None
     kernel_ms = {k: round(v[0] / len(ptimes), 3) for k, v in sorted(fam.items(), key=lambda kv: -kv[1][0])}
 
     result = None
@@ -434,6 +492,7 @@ def run_ours(args):
                           "h2d_bytes_per_step": int(pos_h.numel() * 8 + sp_h.numel() * 4),
                           "d2h_bytes_per_step": int(8 + N * 3 * 4)},
                   "roofline": roof, "hbm_kernels": hbm, "cpu_baseline": cpu, "kernel_ms_per_step": kernel_ms,
+                  "configs": configs,
                   "ns_per_atom": ms * 1e6 / N}
         print(json.dumps(result))
     if ws > 1:
@@ -449,6 +508,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other seeded workloads")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

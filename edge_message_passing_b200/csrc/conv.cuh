@@ -787,16 +787,22 @@ struct BeMeta {
   int el, rr, j, i;                   // cohort-local row, radial row, sender, receiver
 };
 
-// stage layout (floats): Y [16C] | gS[recv] [16C] | GXT [16C] | X [16C] | R [4C] | D [84]
-__host__ __device__ inline size_t be_stage_floats(int C) { return (size_t)68 * C + NDBLK; }
+// Whether the sender's node row goes through the ring too (else it is read from global
+// memory: the node array stays in L2, and consecutive positions of a sender run share it).
+// Staged measured faster, although the smaller ring would allow four blocks per SM.
+constexpr bool BE_STAGE_X = true;
+// stage layout (floats): Y [16C] | gS[recv] [16C] | GXT [16C] | (X [16C]) | R [4C] | D [84]
+__host__ __device__ inline size_t be_stage_floats(int C) { return (size_t)(BE_STAGE_X ? 68 : 52) * C + NDBLK; }
+constexpr int BE_MAXP_EDGE = 32;      // positions per block at most (backward edge kernel)
+constexpr int BE_BLOCKS_PER_SM = 3;   // resident blocks the ring's shared memory allows
 __host__ __device__ inline size_t be_smem_bytes(int C) {
-  return BE_STAGES * be_stage_floats(C) * 4 + BE_STAGES * 8 + (size_t)BE_MAXP * 2 * ((C + 31) / 32) * 4 +
-         BE_MAXP * sizeof(BeMeta) + BE_MAXP * 4 * 4;
+  return BE_STAGES * be_stage_floats(C) * 4 + BE_STAGES * 8 + (size_t)BE_MAXP_EDGE * 2 * ((C + 31) / 32) * 4 +
+         BE_MAXP_EDGE * sizeof(BeMeta) + BE_MAXP_EDGE * 4 * 4;
 }
-// positions per block for a cohort of n edges on `sms` SMs (three blocks per SM)
+// positions per block for a cohort of n edges on `sms` SMs
 inline int be_per(long long n, int sms) {
-  const long long want = (n + 3 * sms - 1) / (3 * sms);
-  return (int)std::max<long long>(1, std::min<long long>(BE_MAXP, want));
+  const long long want = (n + BE_BLOCKS_PER_SM * sms - 1) / (BE_BLOCKS_PER_SM * sms);
+  return (int)std::max<long long>(1, std::min<long long>(BE_MAXP_EDGE, want));
 }
 
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -820,9 +826,9 @@ __global__ void __launch_bounds__(256, 2)
   uint64_t* full = reinterpret_cast<uint64_t*>(be_smem + BE_STAGES * SF * 4);
   const int CV = C / V;
   const int nw = (CV + 31) / 32;
-  float* red = reinterpret_cast<float*>(full + BE_STAGES);               // [BE_MAXP][2][nw]
-  BeMeta* meta = reinterpret_cast<BeMeta*>(red + BE_MAXP * 2 * nw);
-  float* svec = reinterpret_cast<float*>(meta + BE_MAXP);                // [BE_MAXP][4]
+  float* red = reinterpret_cast<float*>(full + BE_STAGES);               // [BE_MAXP_EDGE][2][nw]
+  BeMeta* meta = reinterpret_cast<BeMeta*>(red + BE_MAXP_EDGE * 2 * nw);
+  float* svec = reinterpret_cast<float*>(meta + BE_MAXP_EDGE);           // [BE_MAXP_EDGE][4]
   const int t = threadIdx.x;
   const int warp = t >> 5, lane = t & 31;
   const int n = (int)(e1 - e0);
@@ -849,13 +855,14 @@ __global__ void __launch_bounds__(256, 2)
     const int s = q % BE_STAGES;
     float* st = stage0 + s * SF;
     const BeMeta m = meta[q];
-    tc::mbar_expect_tx(&full[s], bY + bG + bX + bX + bR + NDBLK * 4);
+    const int oR = BE_STAGE_X ? 64 * C : 48 * C;
+    tc::mbar_expect_tx(&full[s], bY + bG + bX + (BE_STAGE_X ? bX : 0u) + bR + NDBLK * 4);
     bulk_g2s(st, Y + (size_t)m.el * 16 * C, bY, &full[s]);
     bulk_g2s(st + 16 * C, gS + (size_t)m.i * 16 * C, bG, &full[s]);
     bulk_g2s(st + 32 * C, GXT + (size_t)m.el * 16 * C, bX, &full[s]);
-    bulk_g2s(st + 48 * C, x + (size_t)m.j * 16 * C, bX, &full[s]);
-    bulk_g2s(st + 64 * C, R + (size_t)m.rr * 4 * C, bR, &full[s]);
-    bulk_g2s(st + 68 * C, D + (size_t)(e0 + m.el) * NDBLK, NDBLK * 4, &full[s]);
+    if (BE_STAGE_X) bulk_g2s(st + 48 * C, x + (size_t)m.j * 16 * C, bX, &full[s]);
+    bulk_g2s(st + oR, R + (size_t)m.rr * 4 * C, bR, &full[s]);
+    bulk_g2s(st + oR + 4 * C, D + (size_t)(e0 + m.el) * NDBLK, NDBLK * 4, &full[s]);
   };
   if (t == 0)
     for (int q = 0; q < min(BE_STAGES, np); ++q) issue(q);
@@ -875,9 +882,11 @@ __global__ void __launch_bounds__(256, 2)
     const T* sY = reinterpret_cast<const T*>(st) + t;
     const T* sGS = reinterpret_cast<const T*>(st + 16 * C) + t;
     const T* sGX = reinterpret_cast<const T*>(st + 32 * C) + t;
-    const T* sX = reinterpret_cast<const T*>(st + 48 * C) + t;
-    const T* sR = reinterpret_cast<const T*>(st + 64 * C) + t;
-    const float* Dr = st + 68 * C;
+    const T* sX = BE_STAGE_X ? reinterpret_cast<const T*>(st + 48 * C) + t
+                             : reinterpret_cast<const T*>(x + (size_t)m.j * 16 * C) + t;
+    const int oR = BE_STAGE_X ? 64 * C : 48 * C;
+    const T* sR = reinterpret_cast<const T*>(st + oR) + t;
+    const float* Dr = st + oR + 4 * C;
     const size_t go = (size_t)m.rr * 4 * CV + t;
     T bx = vset<T>(0.f), by = vset<T>(0.f), gr, h, l;
     const T zero = vset<T>(0.f);
@@ -951,9 +960,11 @@ __global__ void __launch_bounds__(256, 2)
     }
 }
 
-// channels per thread of the backward edge kernel: two when the C / 2 threads fill whole
-// warps (the torque sums reduce over full warps), else one
-inline int be_v(int C) { return C % 64 == 0 ? 2 : 1; }
+// channels per thread of the backward edge kernel.  One: with the ring's shared memory
+// allowing three blocks per SM, C threads per block keep the most warps resident (the
+// kernel is bound by resident warps; two channels per thread measured 10 % slower), and
+// C threads always fill whole warps, which the torque sums reduce over.
+constexpr int BE_V = 1;
 
 // g_x[sender] += the cohort's sender runs, each the sum of its pieces in position order: a run
 // [b, en) has pieces starting at b and at every multiple of `per` inside it (rows of Pg).

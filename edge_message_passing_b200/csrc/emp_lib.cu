@@ -384,8 +384,7 @@ int ensure_attrs() {
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_pair_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * PS_THREADS * 4));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_radial_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(RadialSmem)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_cohort_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, 8 << 14));
-  EMP_CUDA_TRY(cudaFuncSetAttribute(k_bwd_edge<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)be_smem_bytes(256)));
-  EMP_CUDA_TRY(cudaFuncSetAttribute(k_bwd_edge<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)be_smem_bytes(256)));
+  EMP_CUDA_TRY(cudaFuncSetAttribute(k_bwd_edge<BE_V>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)be_smem_bytes(256)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_rotate_staged<false, RS_V_FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)rs_smem_bytes(256, false)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_rotate_staged<true, RS_V_BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -884,8 +883,7 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
       side.wait();      // the previous cohort's combine has read Pg
       {
         Scope sc_("bwd_edge", stream);
-        auto kern = be_v(C) == 2 ? k_bwd_edge<2> : k_bwd_edge<1>;
-        kern<<<nb, C / be_v(C), be_smem_bytes(C), stream>>>(e0, e1, C, t > 0, t == 0, per, g->send, rr.inv, g->vec, D, R,
+        k_bwd_edge<BE_V><<<nb, C / BE_V, be_smem_bytes(C), stream>>>(e0, e1, C, t > 0, t == 0, per, g->send, rr.inv, g->vec, D, R,
                                                            xt, Y, gS, GXT, g->recv, perm, gRhi, gRlo, g_r, Pg);
       }
       if (t > 0)
@@ -974,11 +972,16 @@ int mp_radial_chain(const void* chain, int64_t E, const float* x, float* kc, flo
                     const float* g_y0, float* g_x, cudaStream_t stream) {
   if (!chain || E < 0 || (E > 0 && (!x || !kc || !y0))) return EMP_ERR_ARG;
   if (g_x && E > 0 && (!g_kc || !g_y0)) return EMP_ERR_ARG;
+  auto a16 = [](const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; };
+  if (!a16(x) || !a16(y0) || (g_x && (!a16(g_x) || !a16(g_y0) || !a16(g_kc)))) return EMP_ERR_ARG;
   if (E == 0) return EMP_OK;
   const Chain& c = *static_cast<const Chain*>(chain);
-  const unsigned grid = (unsigned)((E + CH_ROWS - 1) / CH_ROWS);
-  { Scope sc_("chain_fwd", stream); k_chain_fwd<<<grid, 256, sizeof(ChainFwdSmem), stream>>>(E, x, c.Weff, c.U0, kc, y0); }
-  if (g_x) { Scope sc_("chain_bwd", stream); k_chain_bwd<<<grid, 256, sizeof(ChainBwdSmem), stream>>>(E, g_kc, g_y0, c.Weff, c.U0, g_x); }
+  // persistent grids: as many blocks as stay resident (shared memory: 2 / 3 per SM)
+  const long long ntiles = (E + CH_ROWS - 1) / CH_ROWS;
+  const unsigned gf = (unsigned)std::min<long long>(ntiles, 2 * tc::num_sms());
+  const unsigned gb = (unsigned)std::min<long long>(ntiles, 3 * tc::num_sms());
+  { Scope sc_("chain_fwd", stream); k_chain_fwd<<<gf, CH_FWD_THREADS, sizeof(ChainFwdSmem), stream>>>(E, x, c.Weff, c.U0, kc, y0); }
+  if (g_x) { Scope sc_("chain_bwd", stream); k_chain_bwd<<<gb, 256, sizeof(ChainBwdSmem), stream>>>(E, g_kc, g_y0, c.Weff, c.U0, g_x); }
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
 
