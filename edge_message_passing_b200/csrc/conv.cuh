@@ -41,6 +41,50 @@ __device__ __forceinline__ void rotate16(const float* __restrict__ D, const floa
 
 __device__ __forceinline__ int deg_of(int k) { return k == 0 ? 0 : k < 4 ? 1 : k < 9 ? 2 : 3; }
 
+// V adjacent channels per thread: float, float2 or float4 arithmetic, loads and stores
+template <int V> struct VecT;
+template <> struct VecT<1> { typedef float type; };
+template <> struct VecT<2> { typedef float2 type; };
+template <> struct VecT<4> { typedef float4 type; };
+
+__device__ __forceinline__ float vfma(float a, float b, float c) { return fmaf(a, b, c); }
+__device__ __forceinline__ float2 vfma(float a, float2 b, float2 c) { return make_float2(fmaf(a, b.x, c.x), fmaf(a, b.y, c.y)); }
+__device__ __forceinline__ float4 vfma(float a, float4 b, float4 c) {
+  return make_float4(fmaf(a, b.x, c.x), fmaf(a, b.y, c.y), fmaf(a, b.z, c.z), fmaf(a, b.w, c.w));
+}
+__device__ __forceinline__ float vmul(float a, float b) { return a * b; }
+__device__ __forceinline__ float2 vmul(float2 a, float2 b) { return make_float2(a.x * b.x, a.y * b.y); }
+__device__ __forceinline__ float4 vmul(float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); }
+template <typename T> __device__ __forceinline__ T vset(float v);
+template <> __device__ __forceinline__ float vset<float>(float v) { return v; }
+template <> __device__ __forceinline__ float2 vset<float2>(float v) { return make_float2(v, v); }
+template <> __device__ __forceinline__ float4 vset<float4>(float v) { return make_float4(v, v, v, v); }
+__device__ __forceinline__ void vsplit(float v, float& h, float& l) {
+  h = tf32_rna(v);
+  l = tf32_rna(v - h);
+}
+__device__ __forceinline__ void vsplit(float2 v, float2& h, float2& l) {
+  vsplit(v.x, h.x, l.x);
+  vsplit(v.y, h.y, l.y);
+}
+__device__ __forceinline__ void vsplit(float4 v, float4& h, float4& l) {
+  vsplit(v.x, h.x, l.x);
+  vsplit(v.y, h.y, l.y);
+  vsplit(v.z, h.z, l.z);
+  vsplit(v.w, h.w, l.w);
+}
+
+__device__ __forceinline__ float vsub(float a, float b) { return a - b; }
+__device__ __forceinline__ float2 vsub(float2 a, float2 b) { return make_float2(a.x - b.x, a.y - b.y); }
+__device__ __forceinline__ float vadd(float a, float b) { return a + b; }
+__device__ __forceinline__ float2 vadd(float2 a, float2 b) { return make_float2(a.x + b.x, a.y + b.y); }
+__device__ __forceinline__ float vscale(float a, float b) { return a * b; }
+__device__ __forceinline__ float2 vscale(float a, float2 b) { return make_float2(a * b.x, a * b.y); }
+__device__ __forceinline__ float hsum(float a) { return a; }
+__device__ __forceinline__ float hsum(float2 a) { return a.x + a.y; }
+__device__ __forceinline__ float vdot(float a, float b, float c) { return fmaf(a, b, c); }
+__device__ __forceinline__ float2 vdot(float2 a, float2 b, float2 c) { return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y)); }
+
 // ------------------------------------------------------------------ geometry
 // D(R_e) (84 floats) and d = |r_e| from the float32 edge vector.
 __global__ void k_geometry(long long E, const float* __restrict__ vec, float* __restrict__ D, float* __restrict__ dist) {
@@ -411,88 +455,104 @@ __device__ __forceinline__ void rotate_write_degree(const float* __restrict__ Dr
 // 1: its last), and k_rb_combine adds the partials in chunk order.  The order of
 // every sum is fixed, so results are reproducible.
 constexpr int RB_CHUNK = 8;
-constexpr int RB_BATCH = 2;      // edges whose rows are loaded before any is used
 
+template <typename T>
 __device__ __forceinline__ void rb_flush(int i, int c0, int c1, long long e0, long long e1, int chunk, int first_recv,
-                                         const int* __restrict__ recv_off, int C, int c, const float (&acc)[16],
-                                         float* __restrict__ S, float* __restrict__ P) {
+                                         const int* __restrict__ recv_off, int CV, int t, const T (&acc)[16],
+                                         T* __restrict__ S, T* __restrict__ P) {
   const long long lo = max((long long)recv_off[i], e0) - e0, hi = min((long long)recv_off[i + 1], e1) - e0;
   if (lo >= c0 && hi <= c1) {
-    float* Si = S + (size_t)i * 16 * C + c;
+    T* Si = S + (size_t)i * 16 * CV + t;
     const bool carry = recv_off[i] < e0;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) Si[k * C] = carry ? Si[k * C] + acc[k] : acc[k];
+    for (int k = 0; k < 16; ++k) Si[k * CV] = carry ? vadd(Si[k * CV], acc[k]) : acc[k];
   } else {
-    float* Pc = P + ((size_t)chunk * 2 + (i == first_recv ? 0 : 1)) * 16 * C + c;
+    T* Pc = P + ((size_t)chunk * 2 + (i == first_recv ? 0 : 1)) * 16 * CV + t;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) Pc[k * C] = acc[k];
+    for (int k = 0; k < 16; ++k) Pc[k * CV] = acc[k];
   }
 }
 
-__global__ void __launch_bounds__(256, 3) k_rb_chunks(long long e0, long long e1, int C, int scalar_in,
-                                                   const int* __restrict__ recv, const int* __restrict__ recv_off,
-                                                   const float* __restrict__ D, const float* __restrict__ Y,
-                                                   float* __restrict__ S, float* __restrict__ P) {
+// u = D^T x per degree block for V channels (D in shared memory)
+template <typename T>
+__device__ __forceinline__ void rotate16t_v(const float* __restrict__ D, const T (&x)[16], T (&u)[16]) {
+  u[0] = x[0];
+#pragma unroll
+  for (int l = 1; l <= 3; ++l) {
+    const int w = 2 * l + 1, o = l * l;
+    const float* B = D + dblk_off(l);
+#pragma unroll
+    for (int m = 0; m < w; ++m) {
+      T acc = vset<T>(0.f);
+#pragma unroll
+      for (int n = 0; n < w; ++n) acc = vfma(B[n * w + m], x[o + n], acc);
+      u[o + m] = acc;
+    }
+  }
+}
+
+// One block of C / RB_V threads (RB_V adjacent channels each) per 8-edge chunk.
+constexpr int RB_V = 2;
+template <int V>
+__global__ void __launch_bounds__(128) k_rb_chunks(long long e0, long long e1, int C, int scalar_in,
+                                                 const int* __restrict__ recv, const int* __restrict__ recv_off,
+                                                 const float* __restrict__ D, const float* __restrict__ Y,
+                                                 float* __restrict__ S, float* __restrict__ P) {
+  typedef typename VecT<V>::type T;
   __shared__ __align__(16) float sD[RB_CHUNK * NDBLK];
   __shared__ int srv[RB_CHUNK];
-  const int c = threadIdx.x;
+  const int t = threadIdx.x, CV = C / V;
   const int n = (int)(e1 - e0);
+  const T* Yv = reinterpret_cast<const T*>(Y);
+  T* Sv = reinterpret_cast<T*>(S);
+  T* Pv = reinterpret_cast<T*>(P);
   const int nchunks = (n + RB_CHUNK - 1) / RB_CHUNK;
   for (int chunk = blockIdx.x; chunk < nchunks; chunk += gridDim.x) {
     const int c0 = chunk * RB_CHUNK, nch = min(RB_CHUNK, n - c0), c1 = c0 + nch;
     __syncthreads();
-    for (int q = c; q < nch * (NDBLK / 4); q += C)
+    for (int q = t; q < nch * (NDBLK / 4); q += CV)
       reinterpret_cast<float4*>(sD)[q] = reinterpret_cast<const float4*>(D + (size_t)(e0 + c0) * NDBLK)[q];
-    if (c < nch) srv[c] = recv[e0 + c0 + c];
+    if (t < nch) srv[t] = recv[e0 + c0 + t];
     __syncthreads();
     const int first = srv[0];
     int cur = first;
-    float acc[16];
+    T acc[16];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-    for (int k0 = 0; k0 < nch; k0 += RB_BATCH) {
-      float yv[RB_BATCH][16];
+    for (int k = 0; k < 16; ++k) acc[k] = vset<T>(0.f);
+#pragma unroll 1
+    for (int k = 0; k < nch; ++k) {
+      const T* y = Yv + (size_t)(c0 + k) * 16 * CV + t;
+      T yv[16];
+      if (scalar_in) {
 #pragma unroll
-      for (int u = 0; u < RB_BATCH; ++u) {
-        if (k0 + u < nch) {
-          const float* y = Y + (size_t)(c0 + k0 + u) * 16 * C + c;
-          if (scalar_in) {
+        for (int l = 0; l < 4; ++l) yv[l] = y[col_of(l, 0) * CV];
+      } else {
 #pragma unroll
-            for (int l = 0; l < 4; ++l) yv[u][l] = y[col_of(l, 0) * C];
-          } else {
-#pragma unroll
-            for (int q = 0; q < 16; ++q) yv[u][q] = y[col_of_k(q) * C];
-          }
-        }
+        for (int q = 0; q < 16; ++q) yv[q] = y[col_of_k(q) * CV];
       }
+      if (srv[k] != cur) {
+        rb_flush(cur, c0, c1, e0, e1, chunk, first, recv_off, CV, t, acc, Sv, Pv);
 #pragma unroll
-      for (int u = 0; u < RB_BATCH; ++u) {
-        const int k = k0 + u;
-        if (k >= nch) break;
-        if (srv[k] != cur) {
-          rb_flush(cur, c0, c1, e0, e1, chunk, first, recv_off, C, c, acc, S, P);
+        for (int q = 0; q < 16; ++q) acc[q] = vset<T>(0.f);
+        cur = srv[k];
+      }
+      const float* Dk = sD + k * NDBLK;
+      if (scalar_in) {
+        // y is non-zero only at m = 0: message[l][n] = D^l[0][n] y[l][0]
 #pragma unroll
-          for (int q = 0; q < 16; ++q) acc[q] = 0.f;
-          cur = srv[k];
+        for (int l = 0; l < 4; ++l) {
+          const float* row0 = Dk + dblk_off(l) + l * (2 * l + 1);
+#pragma unroll
+          for (int q = 0; q < 2 * l + 1; ++q) acc[l * l + q] = vfma(row0[q], yv[l], acc[l * l + q]);
         }
-        const float* Dk = sD + k * NDBLK;
-        if (scalar_in) {
-          // y is non-zero only at m = 0: message[l][n] = D^l[0][n] y[l][0]
+      } else {
+        T m[16];
+        rotate16t_v(Dk, yv, m);
 #pragma unroll
-          for (int l = 0; l < 4; ++l) {
-            const float* row0 = Dk + dblk_off(l) + l * (2 * l + 1);
-#pragma unroll
-            for (int q = 0; q < 2 * l + 1; ++q) acc[l * l + q] = fmaf(row0[q], yv[u][l], acc[l * l + q]);
-          }
-        } else {
-          float m[16];
-          rotate16<true>(Dk, yv[u], m);
-#pragma unroll
-          for (int q = 0; q < 16; ++q) acc[q] += m[q];
-        }
+        for (int q = 0; q < 16; ++q) acc[q] = vadd(acc[q], m[q]);
       }
     }
-    rb_flush(cur, c0, c1, e0, e1, chunk, first, recv_off, C, c, acc, S, P);
+    rb_flush(cur, c0, c1, e0, e1, chunk, first, recv_off, CV, t, acc, Sv, Pv);
   }
 }
 
@@ -632,50 +692,6 @@ __global__ void k_gate_bwd(int N, int C, float inv_avg, int gated, const float* 
     }
   }
 }
-
-// V adjacent channels per thread: float, float2 or float4 arithmetic, loads and stores
-template <int V> struct VecT;
-template <> struct VecT<1> { typedef float type; };
-template <> struct VecT<2> { typedef float2 type; };
-template <> struct VecT<4> { typedef float4 type; };
-
-__device__ __forceinline__ float vfma(float a, float b, float c) { return fmaf(a, b, c); }
-__device__ __forceinline__ float2 vfma(float a, float2 b, float2 c) { return make_float2(fmaf(a, b.x, c.x), fmaf(a, b.y, c.y)); }
-__device__ __forceinline__ float4 vfma(float a, float4 b, float4 c) {
-  return make_float4(fmaf(a, b.x, c.x), fmaf(a, b.y, c.y), fmaf(a, b.z, c.z), fmaf(a, b.w, c.w));
-}
-__device__ __forceinline__ float vmul(float a, float b) { return a * b; }
-__device__ __forceinline__ float2 vmul(float2 a, float2 b) { return make_float2(a.x * b.x, a.y * b.y); }
-__device__ __forceinline__ float4 vmul(float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); }
-template <typename T> __device__ __forceinline__ T vset(float v);
-template <> __device__ __forceinline__ float vset<float>(float v) { return v; }
-template <> __device__ __forceinline__ float2 vset<float2>(float v) { return make_float2(v, v); }
-template <> __device__ __forceinline__ float4 vset<float4>(float v) { return make_float4(v, v, v, v); }
-__device__ __forceinline__ void vsplit(float v, float& h, float& l) {
-  h = tf32_rna(v);
-  l = tf32_rna(v - h);
-}
-__device__ __forceinline__ void vsplit(float2 v, float2& h, float2& l) {
-  vsplit(v.x, h.x, l.x);
-  vsplit(v.y, h.y, l.y);
-}
-__device__ __forceinline__ void vsplit(float4 v, float4& h, float4& l) {
-  vsplit(v.x, h.x, l.x);
-  vsplit(v.y, h.y, l.y);
-  vsplit(v.z, h.z, l.z);
-  vsplit(v.w, h.w, l.w);
-}
-
-__device__ __forceinline__ float vsub(float a, float b) { return a - b; }
-__device__ __forceinline__ float2 vsub(float2 a, float2 b) { return make_float2(a.x - b.x, a.y - b.y); }
-__device__ __forceinline__ float vadd(float a, float b) { return a + b; }
-__device__ __forceinline__ float2 vadd(float2 a, float2 b) { return make_float2(a.x + b.x, a.y + b.y); }
-__device__ __forceinline__ float vscale(float a, float b) { return a * b; }
-__device__ __forceinline__ float2 vscale(float a, float2 b) { return make_float2(a * b.x, a * b.y); }
-__device__ __forceinline__ float hsum(float a) { return a; }
-__device__ __forceinline__ float hsum(float2 a) { return a.x + a.y; }
-__device__ __forceinline__ float vdot(float a, float b, float c) { return fmaf(a, b, c); }
-__device__ __forceinline__ float2 vdot(float2 a, float2 b, float2 c) { return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y)); }
 
 // per edge, from y (recomputed), g_y and g_x~ = W^T g_y:
 //   gR[e][l][c] = sum_m g_x~ u;  g_u = R (.) g_x~;  g_xs = D^T g_u (-> GXS, [16][C] rows)

@@ -287,7 +287,7 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
       const long long c0 = ee[b], c1 = ee[b + 1];
       const int nchunks = (int)((c1 - c0 + RB_CHUNK - 1) / RB_CHUNK);
       side.wait();        // the previous cohort's combine: S of its last receiver, and P
-      { Scope sc_("rotate_back_scatter", s); k_rb_chunks<<<nchunks, C, 0, s>>>(c0, c1, C, scalar_in, g->recv, g->recv_off, D, Y[b], S, P); }
+      { Scope sc_("rotate_back_scatter", s); k_rb_chunks<RB_V><<<nchunks, C / RB_V, 0, s>>>(c0, c1, C, scalar_in, g->recv, g->recv_off, D, Y[b], S, P); }
       side.run([&](cudaStream_t q) {
         Scope sc_("rb_combine", q);
         k_rb_combine<<<dim3((unsigned)std::min<long long>(c1 - c0, 128), 16), C, 0, q>>>(c0, c1, C, g->recv, g->recv_off, P, S);
