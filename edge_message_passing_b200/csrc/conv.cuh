@@ -491,13 +491,14 @@ __device__ __forceinline__ void rotate16t_v(const float* __restrict__ D, const T
   }
 }
 
-// One block of C / RB_V threads (RB_V adjacent channels each) per 8-edge chunk.
+// One block of C / RB_V threads (RB_V adjacent channels each) per 8-edge chunk.  y rows are
+// y_pitch floats apart (16C; 4C for a degree-0 input, whose y is non-zero only there).
 constexpr int RB_V = 2;
 template <int V>
 __global__ void __launch_bounds__(128) k_rb_chunks(long long e0, long long e1, int C, int scalar_in,
                                                  const int* __restrict__ recv, const int* __restrict__ recv_off,
                                                  const float* __restrict__ D, const float* __restrict__ Y,
-                                                 float* __restrict__ S, float* __restrict__ P) {
+                                                 int y_pitch, float* __restrict__ S, float* __restrict__ P) {
   typedef typename VecT<V>::type T;
   __shared__ __align__(16) float sD[RB_CHUNK * NDBLK];
   __shared__ int srv[RB_CHUNK];
@@ -521,7 +522,7 @@ __global__ void __launch_bounds__(128) k_rb_chunks(long long e0, long long e1, i
     for (int k = 0; k < 16; ++k) acc[k] = vset<T>(0.f);
 #pragma unroll 1
     for (int k = 0; k < nch; ++k) {
-      const T* y = Yv + (size_t)(c0 + k) * 16 * CV + t;
+      const T* y = Yv + (size_t)(c0 + k) * (y_pitch / V) + t;
       T yv[16];
       if (scalar_in) {
 #pragma unroll
@@ -833,7 +834,8 @@ __global__ void __launch_bounds__(256, 2)
                const int* __restrict__ send, const int* __restrict__ rrow, const float* __restrict__ vec,
                const float* __restrict__ D, const float* __restrict__ R, const float* __restrict__ x,
                const float* __restrict__ Y, const float* __restrict__ gS, const float* __restrict__ GXT,
-               const int* __restrict__ recv, const int* __restrict__ perm, float* __restrict__ gR_hi,
+               int y_pitch, int gxt_pitch, const int* __restrict__ recv, const int* __restrict__ perm,
+               float* __restrict__ gR_hi,
                float* __restrict__ gR_lo, float* __restrict__ g_r, float* __restrict__ Pg) {
   typedef typename VecT<V>::type T;
   extern __shared__ __align__(128) unsigned char be_smem[];
@@ -873,9 +875,9 @@ __global__ void __launch_bounds__(256, 2)
     const BeMeta m = meta[q];
     const int oR = BE_STAGE_X ? 64 * C : 48 * C;
     tc::mbar_expect_tx(&full[s], bY + bG + bX + (BE_STAGE_X ? bX : 0u) + bR + NDBLK * 4);
-    bulk_g2s(st, Y + (size_t)m.el * 16 * C, bY, &full[s]);
+    bulk_g2s(st, Y + (size_t)m.el * y_pitch, bY, &full[s]);
     bulk_g2s(st + 16 * C, gS + (size_t)m.i * 16 * C, bG, &full[s]);
-    bulk_g2s(st + 32 * C, GXT + (size_t)m.el * 16 * C, bX, &full[s]);
+    bulk_g2s(st + 32 * C, GXT + (size_t)m.el * gxt_pitch, bX, &full[s]);
     if (BE_STAGE_X) bulk_g2s(st + 48 * C, x + (size_t)m.j * 16 * C, bX, &full[s]);
     bulk_g2s(st + oR, R + (size_t)m.rr * 4 * C, bR, &full[s]);
     bulk_g2s(st + oR + 4 * C, D + (size_t)(e0 + m.el) * NDBLK, NDBLK * 4, &full[s]);
@@ -1017,8 +1019,9 @@ __global__ void k_gx_combine(long long e0, long long e1, int C, int cohort_idx, 
 // true): also GY = D_e gS[recv] (edge-frame output gradient), split.  scalar_in: x has
 // degree 0 only (the first layer's input is the species embedding), so only the (0,0)
 // column of XT is non-zero, and only the m = 0 block of GY (the m = 0 entry of each
-// degree) enters a product.  One block of C/4 threads (four adjacent channels each,
-// float4 loads and stores) per contiguous range of `per` edges of the cohort.  The rows
+// degree) enters a product.  x~ and g_y rows are xt_pitch / gy_pitch floats apart (16C; for a
+// degree-0 input C and 4C, the only columns that can be non-zero).  One block of C / V threads
+// (V adjacent channels each, vector loads and stores) per contiguous range of `per` edges.  The rows
 // an edge reads (x of the sender, gS of the receiver, R and its Wigner-D blocks) are
 // brought into an RS_STAGES-deep shared-memory ring by bulk copies issued by thread 0
 // ahead of use.
@@ -1062,8 +1065,8 @@ __global__ void __launch_bounds__(256)
     k_rotate_staged(long long e0, long long e1, int C, int scalar_in, int per, const int* __restrict__ recv,
                     const int* __restrict__ send, const int* __restrict__ rrow, const float* __restrict__ D,
                     const float* __restrict__ R, const float* __restrict__ x, const float* __restrict__ gS,
-                    float* __restrict__ XT, float* __restrict__ XTlo, float* __restrict__ GYhi,
-                    float* __restrict__ GYlo) {
+                    float* __restrict__ XT, float* __restrict__ XTlo, int xt_pitch, float* __restrict__ GYhi,
+                    float* __restrict__ GYlo, int gy_pitch) {
   typedef typename VecT<V>::type T;
   extern __shared__ __align__(128) unsigned char rs_smem[];
   const size_t SF = rs_stage_floats(C, BWD);
@@ -1110,7 +1113,8 @@ __global__ void __launch_bounds__(256)
     const T* sX = reinterpret_cast<const T*>(st) + t;
     const T* sR = reinterpret_cast<const T*>(st + offR) + t;
     const float* Dr = st + offD;
-    const size_t ro = (size_t)(p0 + q) * 16 * CV + t;
+    const size_t ro = (size_t)(p0 + q) * (xt_pitch / V) + t;
+    const size_t go = (size_t)(p0 + q) * (gy_pitch / V) + t;
     if (scalar_in) {
       T h, l;
       vsplit(vmul(sR[0], sX[0]), h, l);
@@ -1126,10 +1130,10 @@ __global__ void __launch_bounds__(256)
       const T* sG = reinterpret_cast<const T*>(st + offG) + t;
       const T one = vset<T>(1.f);
       if (!scalar_in) {
-        rotate_write_degree_v<0>(Dr, sG, CV, one, GHv + ro, GLv + ro);
-        rotate_write_degree_v<1>(Dr, sG, CV, one, GHv + ro, GLv + ro);
-        rotate_write_degree_v<2>(Dr, sG, CV, one, GHv + ro, GLv + ro);
-        rotate_write_degree_v<3>(Dr, sG, CV, one, GHv + ro, GLv + ro);
+        rotate_write_degree_v<0>(Dr, sG, CV, one, GHv + go, GLv + go);
+        rotate_write_degree_v<1>(Dr, sG, CV, one, GHv + go, GLv + go);
+        rotate_write_degree_v<2>(Dr, sG, CV, one, GHv + go, GLv + go);
+        rotate_write_degree_v<3>(Dr, sG, CV, one, GHv + go, GLv + go);
       } else {
         // the m = 0 entry of each degree: g_y[l][0] = sum_n D^l[0][n] gS[l][n]
 #pragma unroll
@@ -1140,8 +1144,8 @@ __global__ void __launch_bounds__(256)
           T h, lo;
           vsplit(u, h, lo);
           const int col = col_of(l, 0) * CV;
-          GHv[ro + col] = h;
-          GLv[ro + col] = lo;
+          GHv[go + col] = h;
+          GLv[go + col] = lo;
         }
       }
     }

@@ -68,6 +68,9 @@ struct Scope {
 
 inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 
+// cohorts the first layer (degree-0 input) takes at once: its rows are a quarter as wide
+constexpr int LAYER0_COHORTS = 4;
+
 // ------------------------------------------------------------------ workspace layout
 struct WsLayout {
   size_t D, dist, R, rbP, gxP, XT2, XTlo2, Y2, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
@@ -85,7 +88,7 @@ WsLayout ws_layout(const Model& m, long long E, int N) {
   L.D = take((size_t)E * NDBLK * 4);
   L.dist = take((size_t)E * 4);
   L.R = take(T * (size_t)E * 4 * C * 4);
-  L.rbP = take(((coh + RB_CHUNK - 1) / RB_CHUNK) * 2 * 16 * C * 4);
+  L.rbP = take(((LAYER0_COHORTS * coh + RB_CHUNK - 1) / RB_CHUNK) * 2 * 16 * C * 4);
   L.gRhi = take((size_t)E * 4 * C * 4);
   L.gRlo = take((size_t)E * 4 * C * 4);
   L.h2hi = take((size_t)E * 64 * 4);
@@ -159,14 +162,17 @@ int so2_product(const Model& m, long long M, const So2Part* parts, int nparts, i
 struct CohortMaps {
   So2AMaps full, tail;
   long long coh = 0, tail_rows = 0;
-  int build(int C, long long E, long long cohort, const float* hi, const float* lo) {
+  // rows of `cols` columns, `ld` floats apart (default: the full 16C-column rows)
+  int build(int C, long long E, long long cohort, const float* hi, const float* lo, int cols = 0, int ld = 0) {
+    if (!cols) cols = 16 * C;
+    if (!ld) ld = 16 * C;
     coh = std::min(E, cohort);
     tail_rows = E % cohort;
     if (coh > 0) {
-      int st = so2_make_amaps(&full, C, coh, hi, lo);
+      int st = make_pair(&full, hi, lo, coh, cols, ld, tc::BM);
       if (st != EMP_OK) return st;
     }
-    if (tail_rows > 0 && tail_rows != coh) return so2_make_amaps(&tail, C, tail_rows, hi, lo);
+    if (tail_rows > 0 && tail_rows != coh) return make_pair(&tail, hi, lo, tail_rows, cols, ld, tc::BM);
     return EMP_OK;
   }
   const So2AMaps* get(long long rows) const { return rows == coh ? &full : &tail; }
@@ -247,18 +253,22 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
   float* Y[2] = {at<float>(ws, L.Y), at<float>(ws, L.Y2)};
   float* P = at<float>(ws, L.rbP);
   Side side = side_for(s);
+  // A degree-0 input touches only the first C columns of x~ and the first 4C of y: their rows
+  // are stored that narrow, so that a cohort buffer holds LAYER0_COHORTS cohorts, taken at once.
+  const long long span = scalar_in ? LAYER0_COHORTS * coh : coh;
+  const int xp = scalar_in ? C : 16 * C, yp = scalar_in ? 4 * C : 16 * C;
   CohortMaps am[2];
   for (int b = 0; b < 2; ++b) {
-    const int st0 = am[b].build(C, E, coh, XT[b], XTlo[b]);
+    const int st0 = am[b].build(C, E, span, XT[b], XTlo[b], scalar_in ? C : 0, xp);
     if (st0 != EMP_OK) return st0;
   }
   int* counter = at<int>(ws, L.counter);
-  // Cohorts are taken two at a time (a shorter last cohort alone): both are rotated in, then
-  // one grouped launch computes both cohorts' products (twice the tiles, so the CTA pairs
-  // stay evenly loaded), then the receiver sums run cohort by cohort, in order.
+  // Full-width cohorts are taken two at a time (a shorter last cohort alone): both are rotated
+  // in, then one grouped launch computes both cohorts' products (twice the tiles, so the CTA
+  // pairs stay evenly loaded), then the receiver sums run cohort by cohort, in order.
   for (long long e0 = 0; e0 < E;) {
-    const long long e1 = std::min(E, e0 + coh);
-    const bool two = e1 < E && std::min(E, e1 + coh) - e1 == e1 - e0;
+    const long long e1 = std::min(E, e0 + span);
+    const bool two = !scalar_in && e1 < E && std::min(E, e1 + span) - e1 == e1 - e0;
     const long long ee[3] = {e0, e1, two ? e1 + (e1 - e0) : e1};
     const int nc = two ? 2 : 1;
     const long long M = e1 - e0;
@@ -266,18 +276,16 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
       const int per = rs_per(M, tc::num_sms(), 6);
       Scope sc_("rotate_in", s);
       k_rotate_staged<false, RS_V_FWD><<<(unsigned)((M + per - 1) / per), C / RS_V_FWD, rs_smem_bytes(C, false), s>>>(
-          ee[b], ee[b + 1], C, scalar_in, per, g->recv, g->send, rrow, D, R, x, nullptr, XT[b], XTlo[b], nullptr, nullptr);
+          ee[b], ee[b + 1], C, scalar_in, per, g->recv, g->send, rrow, D, R, x, nullptr, XT[b], XTlo[b], xp,
+          nullptr, nullptr, 16 * C);
     }
     int st;
     if (scalar_in) {
       const MapPair& b0 = m.bmaps_fwd[t].blk[0];
-      GemmSub subs[2];
-      for (int b = 0; b < nc; ++b) {
-        const So2AMaps* a = am[b].get(M);
-        subs[b] = GemmSub{&a->hi, &a->lo, &b0.hi, &b0.lo, 0, C, 4 * C, 0, Y[b]};
-      }
+      const So2AMaps* a = am[0].get(M);
+      GemmSub sub{&a->hi, &a->lo, &b0.hi, &b0.lo, 0, C, 4 * C, 0, Y[0]};
       Scope sc_("so2_tc", s);
-      st = tc_group(M, 16 * C, subs, nc, counter, s);
+      st = tc_group(M, yp, &sub, 1, counter, s);
     } else {
       So2Part parts[2] = {{am[0].get(M), &m.bmaps_fwd[t], Y[0]}, {am[1].get(M), &m.bmaps_fwd[t], Y[1]}};
       st = so2_product(m, M, parts, nc, counter, s);
@@ -287,7 +295,7 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
       const long long c0 = ee[b], c1 = ee[b + 1];
       const int nchunks = (int)((c1 - c0 + RB_CHUNK - 1) / RB_CHUNK);
       side.wait();        // the previous cohort's combine: S of its last receiver, and P
-      { Scope sc_("rotate_back_scatter", s); k_rb_chunks<RB_V><<<nchunks, C / RB_V, 0, s>>>(c0, c1, C, scalar_in, g->recv, g->recv_off, D, Y[b], S, P); }
+      { Scope sc_("rotate_back_scatter", s); k_rb_chunks<RB_V><<<nchunks, C / RB_V, 0, s>>>(c0, c1, C, scalar_in, g->recv, g->recv_off, D, Y[b], yp, S, P); }
       side.run([&](cudaStream_t q) {
         Scope sc_("rb_combine", q);
         k_rb_combine<<<dim3((unsigned)std::min<long long>(c1 - c0, 128), 16), C, 0, q>>>(c0, c1, C, g->recv, g->recv_off, P, S);
@@ -850,15 +858,22 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
     const float* xt = xs + (size_t)t * feat;
     { Scope sc_("gate_bwd", stream); k_gate_bwd<<<(unsigned)((N * C + 255) / 256), 256, 0, stream>>>(N, C, inv_avg, m.spec.gated,
                                                                      aggs + (size_t)t * feat, gxa, gS, gxb); }
+    // the first layer (degree-0 input) takes LAYER0_COHORTS cohorts at once, in narrow rows
+    const long long span = t == 0 ? LAYER0_COHORTS * coh : coh;
+    const int xp = t == 0 ? C : 16 * C, gp = t == 0 ? 4 * C : 16 * C;
+    if (t == 0) {
+      st = am_xt.build(C, E, span, XT, XTlo, C, xp);
+      if (st == EMP_OK) st = am_gy.build(C, E, span, GYhi, GYlo, 4 * C, gp);
+      if (st != EMP_OK) return st;
+    }
     int ci = 0;
-    for (long long e0 = 0; e0 < E; e0 += coh, ++ci) {
-      const long long e1 = std::min(E, e0 + coh), n = e1 - e0;
-      const int grid = grid_for(n, eb.y);
+    for (long long e0 = 0; e0 < E; e0 += span, ++ci) {
+      const long long e1 = std::min(E, e0 + span), n = e1 - e0;
       {
         const int per = rs_per(n, tc::num_sms(), 3);
         Scope sc_("bwd_prep", stream);
         k_rotate_staged<true, RS_V_BWD><<<(unsigned)((n + per - 1) / per), C / RS_V_BWD, rs_smem_bytes(C, true), stream>>>(
-            e0, e1, C, t == 0, per, g->recv, g->send, rr.inv, D, R, xt, gS, XT, XTlo, GYhi, GYlo);
+            e0, e1, C, t == 0, per, g->recv, g->send, rr.inv, D, R, xt, gS, XT, XTlo, xp, GYhi, GYlo, gp);
       }
       if (t == 0) {
         // degree-0 input: y needs only the m = 0 block's first C input columns, and only the
@@ -870,7 +885,7 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
         GemmSub subs[2] = {{&ax->hi, &ax->lo, &f0.hi, &f0.lo, 0, C, 4 * C, 0, Y},
                            {&ag->hi, &ag->lo, &b0.hi, &b0.lo, 0, 4 * C, C, 0, GXT}};
         Scope sc_("so2_tc", stream);
-        st = tc_group(n, 16 * C, subs, 2, counter, stream);
+        st = tc_group(n, gp, subs, 2, counter, stream);
       } else {
         So2Part parts[2] = {{am_xt.get(n), &m.bmaps_fwd[t], Y}, {am_gy.get(n), &m.bmaps_bwd[t], GXT}};
         st = so2_product(m, n, parts, 2, counter, stream);
@@ -884,7 +899,7 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
       {
         Scope sc_("bwd_edge", stream);
         k_bwd_edge<BE_V><<<nb, C / BE_V, be_smem_bytes(C), stream>>>(e0, e1, C, t > 0, t == 0, per, g->send, rr.inv, g->vec, D, R,
-                                                           xt, Y, gS, GXT, g->recv, perm, gRhi, gRlo, g_r, Pg);
+                                                           xt, Y, gS, GXT, gp, gp, g->recv, perm, gRhi, gRlo, g_r, Pg);
       }
       if (t > 0)
         side.run([&](cudaStream_t q) {
