@@ -244,16 +244,20 @@ __global__ void __launch_bounds__(RAD_THREADS) k_radial_h2(long long E, const in
                                                           float* __restrict__ h2_lo) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   RadialSmem& s = *reinterpret_cast<RadialSmem*>(smem_raw);
-  const long long r0g = (long long)blockIdx.x * RT;
-  radial_tile_setup(s, r0g, E, perm, dist, recv, send, species, a, false);
   const int t = threadIdx.x;
   const int r0 = (t >> 4) * 4, j0 = (t & 15) * 4;
+  int staged = -1;                     // pair whose weights are in shared memory
+  for (long long r0g = (long long)blockIdx.x * RT; r0g < E; r0g += (long long)gridDim.x * RT) {
+  radial_tile_setup(s, r0g, E, perm, dist, recv, send, species, a, false);
   unsigned mask = s.mask;
   while (mask) {
     const int p = __ffs(mask) - 1;
     mask &= mask - 1;
-    const float* W1 = a.rad + a.layer_off + (size_t)p * a.pair_stride;
-    radial_stage_weights(s, W1, W1 + 64 * 8, false);
+    if (p != staged) {
+      const float* W1 = a.rad + a.layer_off + (size_t)p * a.pair_stride;
+      radial_stage_weights(s, W1, W1 + 64 * 8, false);
+      staged = p;
+    }
     __syncthreads();
     float z[4][4];
     radial_layer1(s, r0, j0, z);
@@ -275,6 +279,7 @@ __global__ void __launch_bounds__(RAD_THREADS) k_radial_h2(long long E, const in
     }
     __syncthreads();
   }
+  }
 }
 
 // dE/dd from dE/dh2 (rows gh2 [E][64], the tensor-core product dE/dR W3); adds (dE/dd) rhat to g_r
@@ -286,10 +291,11 @@ __global__ void __launch_bounds__(RAD_THREADS) k_radial_bwd(long long E, const i
                                                            float* __restrict__ g_r) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   RadialSmem& s = *reinterpret_cast<RadialSmem*>(smem_raw);
-  const long long r0g = (long long)blockIdx.x * RT;
-  radial_tile_setup(s, r0g, E, perm, dist, recv, send, species, a, true);
   const int t = threadIdx.x;
   const int r0 = (t >> 4) * 4, j0 = (t & 15) * 4;
+  int staged = -1;                     // pair whose weights are in shared memory
+  for (long long r0g = (long long)blockIdx.x * RT; r0g < E; r0g += (long long)gridDim.x * RT) {
+  radial_tile_setup(s, r0g, E, perm, dist, recv, send, species, a, true);
   float g[4][4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
@@ -302,7 +308,10 @@ __global__ void __launch_bounds__(RAD_THREADS) k_radial_bwd(long long E, const i
     const int p = __ffs(mask) - 1;
     mask &= mask - 1;
     const float* W1 = a.rad + a.layer_off + (size_t)p * a.pair_stride;
-    radial_stage_weights(s, W1, W1 + 64 * 8, true);
+    if (p != staged) {
+      radial_stage_weights(s, W1, W1 + 64 * 8, true);
+      staged = p;
+    }
     __syncthreads();
     float z1[4][4], z2[4][4];
     radial_layer1(s, r0, j0, z1);
@@ -362,6 +371,7 @@ __global__ void __launch_bounds__(RAD_THREADS) k_radial_bwd(long long E, const i
       }
     }
     __syncthreads();
+  }
   }
 }
 

@@ -342,7 +342,7 @@ int radial_forward(const Model& m, const emp_graph* g, int t, const int* species
   const int C = m.spec.C;
   float* h2hi = at<float>(ws, L.h2hi);
   float* h2lo = at<float>(ws, L.h2lo);
-  { Scope sc_("radial_h2", s); k_radial_h2<<<(unsigned)((E + RT - 1) / RT), RAD_THREADS, sizeof(RadialSmem), s>>>(
+  { Scope sc_("radial_h2", s); k_radial_h2<<<(unsigned)std::min<long long>((E + RT - 1) / RT, 3 * tc::num_sms()), RAD_THREADS, sizeof(RadialSmem), s>>>(
         E, rr.perm, dist, g->recv, g->send, species, radial_args(m, t), h2hi, h2lo); }
   for (int p = 0; p < m.n_pairs; ++p) {
     const long long r0 = rr.off[p], n = rr.off[p + 1] - r0;
@@ -380,7 +380,7 @@ int radial_backward(const Model& m, const emp_graph* g, int t, const int* specie
     st = tc_group(n, 64, &sub, 1, at<int>(ws, L.counter), s);
     if (st != EMP_OK) return st;
   }
-  { Scope sc_("radial_bwd", s); k_radial_bwd<<<(unsigned)((E + RT - 1) / RT), RAD_THREADS, sizeof(RadialSmem), s>>>(
+  { Scope sc_("radial_bwd", s); k_radial_bwd<<<(unsigned)std::min<long long>((E + RT - 1) / RT, 2 * tc::num_sms()), RAD_THREADS, sizeof(RadialSmem), s>>>(
         E, rr.perm, dist, g->vec, g->recv, g->send, species, radial_args(m, t), gh2, g_r); }
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
