@@ -244,18 +244,24 @@ def hbm_fractions(fam, steps: int, E: int, C: int, T: int, hbm_gbs: float):
     return out
 
 
-# DRAM bytes per launch of the SO(2) mixing kernel, from one ncu capture (see profiles/),
-# valid only for the kernel source it was taken on (else the roofline's traffic is null).
-SO2_TRAFFIC = {"source_sha1": "aeb165151cca2f602305e04e9d1d07bfc712ea1e", "bytes_per_launch": 197e6}
+# DRAM bytes per launch of the SO(2) mixing kernel (mean over one N=4096 step's launches), from
+# one ncu capture (see profiles/), valid only for the kernel source and launch structure it was
+# taken on (else the roofline's traffic is null).
+SO2_TRAFFIC = {"source_sha1": None, "bytes_per_launch": None}
 
 
 def so2_traffic_per_launch():
+    # the kernel and the launch structure (which cohorts each launch covers) must both be
+    # those the counters were taken on
     import hashlib
-    src = os.path.join(ROOT, "edge_message_passing_b200", "csrc", "so2_tc.cuh")
-    if not SO2_TRAFFIC["source_sha1"] or not os.path.exists(src):
-        return None
-    h = hashlib.sha1(open(src, "rb").read()).hexdigest()
-    return SO2_TRAFFIC["bytes_per_launch"] if h == SO2_TRAFFIC["source_sha1"] else None
+    h = hashlib.sha1()
+    for f in ("so2_tc.cuh", "emp_lib.cu"):
+        src = os.path.join(ROOT, "edge_message_passing_b200", "csrc", f)
+        if not os.path.exists(src):
+            return None
+        h.update(open(src, "rb").read())
+    ok = SO2_TRAFFIC["source_sha1"] and h.hexdigest() == SO2_TRAFFIC["source_sha1"]
+    return SO2_TRAFFIC["bytes_per_launch"] if ok else None
 
 
 # ------------------------------------------------------------------ the other seeded configs

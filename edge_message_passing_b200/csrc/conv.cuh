@@ -21,23 +21,6 @@ namespace emp {
 constexpr float PI_F = 3.14159265358979323846f;
 
 // ------------------------------------------------------------------ rotations
-// u = D x (transpose = false) or u = D^T x, per degree block; D in shared memory
-template <bool TRANSPOSE>
-__device__ __forceinline__ void rotate16(const float* __restrict__ D, const float (&x)[16], float (&u)[16]) {
-  u[0] = x[0];
-#pragma unroll
-  for (int l = 1; l <= 3; ++l) {
-    const int w = 2 * l + 1, o = l * l;
-    const float* B = D + dblk_off(l);
-#pragma unroll
-    for (int m = 0; m < w; ++m) {
-      float acc = 0.f;
-#pragma unroll
-      for (int n = 0; n < w; ++n) acc = fmaf(TRANSPOSE ? B[n * w + m] : B[m * w + n], x[o + n], acc);
-      u[o + m] = acc;
-    }
-  }
-}
 
 __device__ __forceinline__ int deg_of(int k) { return k == 0 ? 0 : k < 4 ? 1 : k < 9 ? 2 : 3; }
 

@@ -144,7 +144,6 @@ RadialArgs radial_args(const Model& m, int t) {
   return a;
 }
 
-dim3 edge_block(int C) { return dim3(C, std::max(1, 256 / C)); }
 
 int grid_for(long long n, int per, int cap = 148 * 32) {
   long long g = (n + per - 1) / per;
@@ -813,7 +812,6 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
   int* seg = at<int>(ws, L.seg);
   int* nseg = at<int>(ws, L.nseg);
   const float inv_avg = 1.0f / m.spec.avg_degree;
-  const dim3 eb = edge_block(C);
   int* counter = at<int>(ws, L.counter);
   Side side = side_for(stream);
   CohortMaps am_xt, am_gy;
