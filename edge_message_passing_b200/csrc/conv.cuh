@@ -1020,7 +1020,14 @@ __global__ void k_gx_combine(long long e0, long long e1, int C, int cohort_idx, 
 // ahead of use.
 constexpr int RS_STAGES = 3;         // at most 4: the barriers take 32 bytes before the metadata
 
-__host__ __device__ inline size_t rs_stage_floats(int C, bool bwd) { return (size_t)(bwd ? 36 : 20) * C + NDBLK; }
+// Whether the backward prep stages the receiver's gS row per edge (else it reads it from global
+// memory: in edge order consecutive edges share the receiver, so L1 serves the repeats).  Both
+// measured the same: with twice the resident warps the kernel is no faster, its 32 KB of
+// writes per edge bound it.
+constexpr bool RS_STAGE_G = true;
+__host__ __device__ inline size_t rs_stage_floats(int C, bool bwd) {
+  return (size_t)(bwd && RS_STAGE_G ? 36 : 20) * C + NDBLK;
+}
 __host__ __device__ inline size_t rs_smem_bytes(int C, bool bwd) {
   return RS_STAGES * rs_stage_floats(C, bwd) * 4 + 32 + (size_t)BE_MAXP * 4 * 4;
 }
@@ -1080,15 +1087,16 @@ __global__ void __launch_bounds__(256)
     meta[q] = make_int4(send[e], BWD ? recv[e] : 0, rrow ? rrow[e] : (int)e, 0);
   }
   __syncthreads();
-  const uint32_t bX = scalar_in ? 4u * C : 64u * C, bG = BWD ? 64u * C : 0u, bR = scalar_in ? 4u * C : 16u * C;
-  const int offG = 16 * C, offR = (BWD ? 32 : 16) * C, offD = offR + 4 * C;
+  constexpr bool SG = BWD && RS_STAGE_G;
+  const uint32_t bX = scalar_in ? 4u * C : 64u * C, bG = SG ? 64u * C : 0u, bR = scalar_in ? 4u * C : 16u * C;
+  const int offG = 16 * C, offR = (SG ? 32 : 16) * C, offD = offR + 4 * C;
   auto issue = [&](int q) {
     const int s = q % RS_STAGES;
     float* st = stage0 + s * SF;
     const int4 m = meta[q];
     tc::mbar_expect_tx(&full[s], bX + bG + bR + NDBLK * 4);
     bulk_g2s(st, x + (size_t)m.x * 16 * C, bX, &full[s]);
-    if (BWD) bulk_g2s(st + offG, gS + (size_t)m.y * 16 * C, bG, &full[s]);
+    if (SG) bulk_g2s(st + offG, gS + (size_t)m.y * 16 * C, bG, &full[s]);
     bulk_g2s(st + offR, R + (size_t)m.z * 4 * C, bR, &full[s]);
     bulk_g2s(st + offD, D + (size_t)(e0 + p0 + q) * NDBLK, NDBLK * 4, &full[s]);
   };
@@ -1120,7 +1128,8 @@ __global__ void __launch_bounds__(256)
       rotate_write_degree_v<3>(Dr, sX, CV, sR[3 * CV], XTv + ro, XLv + ro);
     }
     if (BWD) {
-      const T* sG = reinterpret_cast<const T*>(st + offG) + t;
+      const T* sG = SG ? reinterpret_cast<const T*>(st + offG) + t
+                       : reinterpret_cast<const T*>(gS + (size_t)meta[q].y * 16 * C) + t;
       const T one = vset<T>(1.f);
       if (!scalar_in) {
         rotate_write_degree_v<0>(Dr, sG, CV, one, GHv + go, GLv + go);
