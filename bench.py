@@ -247,7 +247,7 @@ def hbm_fractions(fam, steps: int, E: int, C: int, T: int, hbm_gbs: float):
 # DRAM bytes per launch of the SO(2) mixing kernel (mean over one N=4096 step's launches), from
 # one ncu capture (see profiles/), valid only for the kernel source and launch structure it was
 # taken on (else the roofline's traffic is null).
-SO2_TRAFFIC = {"source_sha1": "40ebd77b5abaaf052289f7fd4140695f541d8930", "bytes_per_launch": 346.1e6}
+SO2_TRAFFIC = {"source_sha1": "b3686220c4cde0b668d6edaaeb10b0657b37113a", "bytes_per_launch": 346.1e6}
 
 
 def so2_traffic_per_launch():

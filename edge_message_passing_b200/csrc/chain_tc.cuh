@@ -1,0 +1,424 @@
+// Radial fold chain on the tensor cores (page "deepmd-kit PR #6108: radial head fold",
+// section "What"): the forward kc = x_flat W_eff (128 -> 25) and y0 = x[:,0,:] U_0
+// (32 -> 64), and the input gradient g_x = g_kc W_eff^T (+ g_y0 U_0^T on degree 0), as
+// products in 3xTF32 (a = hi + lo, hi = RN_tf32(a), lo = RN_tf32(a - hi); hi.hi + hi.lo
+// + lo.hi accumulated in FP32 in tensor memory), so that the chain keeps FP32 accuracy
+// and is bound by its HBM bytes rather than by FP32 SIMT arithmetic.
+//
+// Persistent kernel, one CTA per SM (cta_group::1, M = 128 rows per tile, tiles taken
+// round-robin).  Roles:
+//  - one producer thread fills a ring of fp32 k-blocks (128 rows x 16 fp32, 10 stages
+//    forward, 8 backward) with TMA loads of x (forward) or g_y0 (backward), and copies
+//    each tile's g_kc rows (100 bytes, a pitch no tensor map can describe) with one bulk
+//    copy into a double buffer;
+//  - four groups of two split warps, group g owning stage g of a second, 4-stage ring,
+//    each read a whole k-block into registers, free its fp32 stage at once, and write hi
+//    and lo in the 64-byte-swizzled K-major layout the MMA descriptors read.  The two
+//    rings keep the DRAM latency out of the loop between the split and the tensor cores,
+//    and the four groups overlap the proxy fence that closes each k-block;
+//  - one thread issues the MMAs into one of two TMEM accumulators of 256 columns;
+//  - four warps sum the accumulator's partial columns and store the rows.
+// The weights are split once, when the chain is created, into an operand image whose
+// hi and lo rows are stacked along N: one MMA of A_hi against [B_hi; B_lo] yields both
+// hi.hi and hi.lo (in separate columns), so A is read twice per k-step, not three times.
+// Every mbarrier wait is bounded; the producer waits out its own copies before exit.
+#pragma once
+#include "so2_tc.cuh"
+
+namespace emp {
+namespace ctc {
+
+constexpr int BM = 128;                          // rows per tile
+constexpr int HSTAGES = 4;                       // hi/lo k-blocks of A in the MMA ring
+constexpr int SPLIT_WARPS = 2 * HSTAGES;          // two per hi/lo stage
+constexpr int EPI_WARPS = 4;
+constexpr int THREADS = 32 * (2 + EPI_WARPS + SPLIT_WARPS);
+constexpr int A_BYTES = BM * 64;                 // one k-block of hi (or lo): 128 rows x 64 bytes
+constexpr int STAGE_BYTES = 2 * A_BYTES;
+constexpr int ACC_COLS = 256;                    // one accumulator
+constexpr int EPI_PITCH = 36;
+constexpr int FWD_KB = 8;                        // k-blocks of x (K = 128)
+constexpr int BWD_KB = 6;                        // k-blocks of [g_kc | 0 | g_y0] (K = 32 + 64)
+constexpr int KC_FLOATS = BM * 25;               // one tile of g_kc rows
+constexpr int B_FLOATS = 12288;                  // operand image of either direction
+constexpr int BAR_BYTES = 512;                   // mbarriers and the TMEM address
+__host__ __device__ constexpr int fstages(bool fwd) { return fwd ? 10 : 8; }   // fp32 landing ring
+static_assert((2 * fstages(true) + 2 * HSTAGES + 9) * 8 + 4 <= BAR_BYTES, "barrier area");
+
+// Operand image: k-blocks of [N_kb rows][16 fp32] (K-major), stacked.
+//  forward,  kb < 2:  [W_eff^T hi (32, rows >= 25 zero); U_0^T hi (64); W_eff^T lo (32); U_0^T lo (64)]
+//            kb >= 2: [W_eff^T hi (32); W_eff^T lo (32)]
+//  backward, kb < 2:  [W_eff hi (128 rows, K = g_kc column, >= 25 zero); W_eff lo (128)]
+//            kb >= 2: [U_0 hi (32 rows, K = g_y0 column); U_0 lo (32)]
+// Accumulator columns (per buffer):
+//  forward:  0-31 kc hh+lh (kb < 2), 32-95 y0 hh+lh, 96-127 kc hl, 128-191 y0 hl,
+//            192-223 kc hh+lh (kb >= 2), 224-255 kc hl (kb >= 2)
+//  backward: 0-127 g_x hh+lh, 128-255 g_x hl
+__host__ __device__ constexpr int b_off(bool fwd, int kb) {
+  return fwd ? (kb < 2 ? kb * 192 * 64 : 2 * 192 * 64 + (kb - 2) * 64 * 64)
+             : (kb < 2 ? kb * 256 * 64 : 2 * 256 * 64 + (kb - 2) * 64 * 64);
+}
+static_assert(b_off(true, FWD_KB) == B_FLOATS * 4 && b_off(false, BWD_KB) == B_FLOATS * 4, "operand image size");
+
+__host__ __device__ constexpr int smem_bytes(bool fwd) {
+  return 1024 + fstages(fwd) * A_BYTES + HSTAGES * STAGE_BYTES + B_FLOATS * 4 + EPI_WARPS * 32 * EPI_PITCH * 4 + (fwd ? 0 : 2 * KC_FLOATS * 4) +
+         BAR_BYTES;
+}
+
+// byte offset of element (row r, k) (k < 16) of a k-block of 64-byte rows, 64-byte swizzle
+// (the 16-byte chunk index of a row is XORed with bits 1-2 of the row index)
+__device__ __forceinline__ uint32_t swz(int r, int k) {
+  return (uint32_t)(r * 64 + ((((k >> 2) ^ (r >> 1)) & 3) << 4) + (k & 3) * 4);
+}
+
+__device__ __forceinline__ void mma1(uint32_t d, uint32_t a, uint32_t b, int n, bool acc) {
+  const uint32_t id = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
+      "l"(tc::sdesc(a)), "l"(tc::sdesc(b)), "r"(id), "r"((uint32_t)acc));
+}
+__device__ __forceinline__ void commit1(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(tc::smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(tc::smem_u32(dst)), "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void add32(float (&v)[32], const float (&w)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] += w[j];
+}
+
+// one warp: 32 rows (r0 ..) x 32 columns of v (one row per lane) -> out[row * pitch + col0 ..], via stg
+__device__ __forceinline__ void store_rows32(const float (&v)[32], float* stg, int lane, long long E, long long r0,
+                                             float* out, int pitch, int col0) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 4)
+    *reinterpret_cast<float4*>(stg + lane * EPI_PITCH + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int rr = k * 4 + (lane >> 3), c4 = (lane & 7) * 4;
+    const float4 w = *reinterpret_cast<const float4*>(stg + rr * EPI_PITCH + c4);
+    if (r0 + rr < E) *reinterpret_cast<float4*>(out + (size_t)(r0 + rr) * pitch + col0 + c4) = w;
+  }
+  __syncwarp();
+}
+
+// FWD: amap = x as [E][128]; out0 = kc [E][25], out1 = y0 [E][64].
+// !FWD: amap = g_y0 as [E][64], g_kc [E][25]; out0 = g_x [E][128].
+template <bool FWD>
+__global__ void __launch_bounds__(THREADS, 1)
+    k_chain_tc(long long E, const __grid_constant__ CUtensorMap amap, const float* __restrict__ g_kc,
+               const float* __restrict__ Bimg, float* __restrict__ out0, float* __restrict__ out1) {
+  extern __shared__ __align__(1024) unsigned char ctc_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(ctc_raw) + 1023) & ~(uintptr_t)1023);
+  constexpr int KBN = FWD ? FWD_KB : BWD_KB;
+  constexpr int FS = fstages(FWD);
+  unsigned char* fring = sm;                                            // [FS] fp32 k-blocks (TMA)
+  unsigned char* hring = fring + FS * A_BYTES;                          // [HSTAGES] hi, lo k-blocks
+  unsigned char* bimg = hring + HSTAGES * STAGE_BYTES;
+  float* epi = reinterpret_cast<float*>(bimg + B_FLOATS * 4);
+  float* kcbuf = epi + EPI_WARPS * 32 * EPI_PITCH;                      // [2][KC_FLOATS] (backward)
+  uint64_t* ffull = reinterpret_cast<uint64_t*>(kcbuf + (FWD ? 0 : 2 * KC_FLOATS));   // [FS] landed
+  uint64_t* fempty = ffull + FS;                                        // [FS] read by the split warps
+  uint64_t* sfull = fempty + FS;                                        // [HSTAGES] hi and lo written
+  uint64_t* sempty = sfull + HSTAGES;                                   // [HSTAGES] MMAs done with them
+  uint64_t* acc_full = sempty + HSTAGES;                                // [2]
+  uint64_t* acc_empty = acc_full + 2;                                   // [2]
+  uint64_t* kc_full = acc_empty + 2;                                    // [2] g_kc rows of a tile landed
+  uint64_t* kc_empty = kc_full + 2;                                     // [2] g_kc rows of a tile read
+  uint64_t* drain = kc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long ntiles = (E + BM - 1) / BM;
+  const long long nmine = (long long)blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  if (nmine == 0) return;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < FS; ++s) {
+      tc::mbar_init(&ffull[s], 1);
+      tc::mbar_init(&fempty[s], 2);
+    }
+    for (int s = 0; s < HSTAGES; ++s) {
+      tc::mbar_init(&sfull[s], 2);
+      tc::mbar_init(&sempty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&acc_full[b], 1);
+      tc::mbar_init(&acc_empty[b], EPI_WARPS);
+      tc::mbar_init(&kc_full[b], 1);
+      tc::mbar_init(&kc_empty[b], 4);
+    }
+    tc::mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tc::smem_u32(tmem_slot)),
+                 "r"((uint32_t)(2 * ACC_COLS)));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  // the operand image, 16-byte chunks swizzled (image offsets of k-blocks are multiples of 512)
+  for (int i = threadIdx.x; i < B_FLOATS / 4; i += THREADS) {
+    const uint32_t off = (uint32_t)i * 16;
+    *reinterpret_cast<float4*>(bimg + (off ^ ((off >> 3) & 0x30))) = reinterpret_cast<const float4*>(Bimg)[i];
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------------- producer
+    long long fi = 0, kc_issued = 0;
+    bool ok = true;
+    for (long long i = 0; i < nmine && ok; ++i) {
+      const long long row0 = (blockIdx.x + i * gridDim.x) * BM;
+      for (int kb = 0; kb < KBN; ++kb) {
+        if (FWD || kb >= 2) {
+          const int f = (int)(fi % FS);
+          if (fi >= FS && !tc::mbar_wait(&fempty[f], (uint32_t)(((fi / FS) - 1) & 1))) { ok = false; break; }
+          tc::mbar_expect_tx(&ffull[f], A_BYTES);
+          tc::tma_load(fring + f * A_BYTES, &amap, &ffull[f], (FWD ? kb : kb - 2) * 16, (int)row0);
+          ++fi;
+        } else if (kb == 0) {
+          const int b = (int)(i & 1);
+          if (i >= 2 && !tc::mbar_wait(&kc_empty[b], (uint32_t)(((i >> 1) - 1) & 1))) { ok = false; break; }
+          const long long rows = E - row0 < BM ? E - row0 : BM;
+          const uint32_t nb = (uint32_t)(rows * 100) & ~15u;        // the tail (< 16 bytes) is read directly
+          tc::mbar_expect_tx(&kc_full[b], nb);
+          if (nb) bulk_load(kcbuf + b * KC_FLOATS, g_kc + row0 * 25, nb, &kc_full[b]);
+          ++kc_issued;
+        }
+      }
+    }
+    // copies still in flight can only be among the last FS stages and the last two g_kc tiles
+    for (long long j = fi > FS ? fi - FS : 0; j < fi; ++j) tc::mbar_wait(&ffull[j % FS], (uint32_t)((j / FS) & 1));
+    for (long long t = kc_issued > 2 ? kc_issued - 2 : 0; t < kc_issued; ++t) tc::mbar_wait(&kc_full[t & 1], (uint32_t)((t >> 1) & 1));
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------------- MMA issuer
+    long long it = 0;
+    bool ok = true;
+    const uint32_t bbase = tc::smem_u32(bimg);
+    for (long long i = 0; i < nmine && ok; ++i) {
+      const int buf = (int)(i & 1);
+      if (i >= 2 && !tc::mbar_wait(&acc_empty[buf], (uint32_t)(((i >> 1) - 1) & 1))) break;
+      tc::fence_after();
+      const uint32_t d = tmem + (uint32_t)(buf * ACC_COLS);
+      for (int kb = 0; kb < KBN; ++kb, ++it) {
+        const int s = (int)(it % HSTAGES);
+        if (!tc::mbar_wait(&sfull[s], (uint32_t)((it / HSTAGES) & 1))) { ok = false; break; }
+        tc::fence_after();
+        const uint32_t ahi = tc::smem_u32(hring + s * STAGE_BYTES), alo = ahi + A_BYTES;
+        const uint32_t bb = bbase + (uint32_t)b_off(FWD, kb);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const uint32_t o = kk * 32;                              // 8 fp32 of K
+          if (FWD) {
+            if (kb < 2) {
+              mma1(d, ahi + o, bb + o, 192, kb | kk);
+              mma1(d, alo + o, bb + o, 96, true);
+            } else {
+              mma1(d + 192, ahi + o, bb + o, 64, kb > 2 || kk);
+              mma1(d + 192, alo + o, bb + o, 32, true);
+            }
+          } else {
+            if (kb < 2) {
+              mma1(d, ahi + o, bb + o, 256, kb | kk);
+              mma1(d, alo + o, bb + o, 128, true);
+            } else {
+              mma1(d, ahi + o, bb + o, 32, true);
+              mma1(d + 128, ahi + o, bb + 32 * 64 + o, 32, true);
+              mma1(d, alo + o, bb + o, 32, true);
+            }
+          }
+        }
+        commit1(&sempty[s]);
+      }
+      if (!ok) break;
+      commit1(&acc_full[buf]);
+    }
+    commit1(drain);
+    tc::mbar_wait(drain, 0);
+  } else if (warp >= 2 && warp < 2 + EPI_WARPS) {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;                    // TMEM lanes q*32 .. q*32 + 31
+    float* stg = epi + (warp - 2) * 32 * EPI_PITCH;
+    for (long long i = 0; i < nmine; ++i) {
+      const int buf = (int)(i & 1);
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&acc_full[buf], (uint32_t)((i >> 1) & 1)))) break;
+      tc::fence_after();
+      const long long r0 = (blockIdx.x + i * gridDim.x) * BM + q * 32;   // this warp's first row
+      const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * ACC_COLS);
+      float v[32], w[32];
+      if (FWD) {
+        // kc: the four partial column groups; the warp's 32 rows of 25 are 800 contiguous floats
+        tc::tmem_ld32(base, v);
+        tc::tmem_ld32(base + 96, w);
+        add32(v, w);
+        tc::tmem_ld32(base + 192, w);
+        add32(v, w);
+        tc::tmem_ld32(base + 224, w);
+        add32(v, w);
+#pragma unroll
+        for (int j = 0; j < 24; j += 4)
+          *reinterpret_cast<float4*>(stg + lane * EPI_PITCH + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        stg[lane * EPI_PITCH + 24] = v[24];
+        __syncwarp();
+        const long long nrow = E - r0 < 32 ? E - r0 : 32;
+        float* dst = out0 + (size_t)r0 * 25;
+#pragma unroll 5
+        for (int idx = lane; idx < 800; idx += 32)
+          if (idx < nrow * 25) dst[idx] = stg[(idx / 25) * EPI_PITCH + idx % 25];
+        __syncwarp();
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          tc::tmem_ld32(base + 32 + 32 * h, v);
+          tc::tmem_ld32(base + 128 + 32 * h, w);
+          add32(v, w);
+          store_rows32(v, stg, lane, E, r0, out1, 64, 32 * h);
+        }
+      } else {
+#pragma unroll 1
+        for (int h = 0; h < 4; ++h) {
+          tc::tmem_ld32(base + 32 * h, v);
+          tc::tmem_ld32(base + 128 + 32 * h, w);
+          add32(v, w);
+          store_rows32(v, stg, lane, E, r0, out0, 128, 32 * h);
+        }
+      }
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&acc_empty[buf]);
+    }
+  } else if (warp >= 2 + EPI_WARPS) {
+    // ---------------------------------------------------------------- split warps
+    // four groups of two warps; group g owns hi/lo stage g and takes k-blocks g, g + 4, ...
+    // (one proxy fence per k-block and group, the four groups' fences overlapping).
+    // Thread t of a group: rows t and t + 64, all 16 columns.
+    const int sw = warp - (2 + EPI_WARPS);
+    const int g = sw >> 1;
+    const int t = (sw & 1) * 32 + lane;
+    const long long total = nmine * KBN;
+    unsigned char* hi = hring + g * STAGE_BYTES;
+    unsigned char* lo = hi + A_BYTES;
+    for (long long m = 0;; ++m) {
+      const long long it = g + m * HSTAGES;
+      if (it >= total) break;
+      const long long i = it / KBN;
+      const int kb = (int)(it % KBN);
+      float v[2][16];
+      if (FWD || kb >= 2) {
+        const long long fi = FWD ? it : i * 4 + (kb - 2);
+        const int f = (int)(fi % FS);
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(&ffull[f], (uint32_t)((fi / FS) & 1)))) break;
+        const unsigned char* src = fring + f * A_BYTES;
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const float4 a = *reinterpret_cast<const float4*>(src + swz(t + 64 * q, 4 * c));
+            v[q][4 * c] = a.x; v[q][4 * c + 1] = a.y; v[q][4 * c + 2] = a.z; v[q][4 * c + 3] = a.w;
+          }
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&fempty[f]);
+      } else {
+        const int b = (int)(i & 1);
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(&kc_full[b], (uint32_t)((i >> 1) & 1)))) break;
+        const long long row0 = (blockIdx.x + i * gridDim.x) * BM;
+        const long long rows = E - row0 < BM ? E - row0 : BM;
+        const int nbf = (int)(((rows * 100) & ~15LL) >> 2);
+        const float* ks = kcbuf + b * KC_FLOATS;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int r = t + 64 * q;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int k = kb * 16 + j, f = r * 25 + k;
+            v[q][j] = (k < 25 && r < rows) ? (f < nbf ? ks[f] : g_kc[row0 * 25 + f]) : 0.f;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&kc_empty[b]);           // two groups of two warps per tile
+      }
+      if (m >= 1 && !__all_sync(0xffffffffu, tc::mbar_wait(&sempty[g], (uint32_t)((m - 1) & 1)))) break;
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float* x = &v[q][4 * c];
+          float4 hv, lv;
+          hv.x = tf32_rna(x[0]); lv.x = tf32_rna(x[0] - hv.x);
+          hv.y = tf32_rna(x[1]); lv.y = tf32_rna(x[1] - hv.y);
+          hv.z = tf32_rna(x[2]); lv.z = tf32_rna(x[2] - hv.z);
+          hv.w = tf32_rna(x[3]); lv.w = tf32_rna(x[3] - hv.w);
+          *reinterpret_cast<float4*>(hi + swz(t + 64 * q, 4 * c)) = hv;
+          *reinterpret_cast<float4*>(lo + swz(t + 64 * q, 4 * c)) = lv;
+        }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sfull[g]);
+    }
+  }
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)(2 * ACC_COLS)));
+  }
+}
+
+// The operand images of both directions (layout above) from W_eff [128][25] and U_0 [32][64].
+__global__ void k_chain_bmats(const float* __restrict__ Weff, const float* __restrict__ U0, float* __restrict__ bfwd,
+                              float* __restrict__ bbwd) {
+  const int f = blockIdx.x * blockDim.x + threadIdx.x;
+  if (f >= B_FLOATS) return;
+  const int off = f * 4, k = f & 15;
+  {
+    // forward: B[n][K] = weight[K][n]
+    int kb, n;
+    if (off < 2 * 192 * 64) { kb = off / (192 * 64); n = (off % (192 * 64)) / 64; }
+    else { kb = 2 + (off - 2 * 192 * 64) / (64 * 64); n = ((off - 2 * 192 * 64) % (64 * 64)) / 64; }
+    const int K = kb * 16 + k;
+    float v;
+    bool lo;
+    if (kb < 2) {
+      lo = n >= 96;
+      const int nn = n % 96;
+      v = nn < 32 ? (nn < 25 ? Weff[K * 25 + nn] : 0.f) : U0[K * 64 + (nn - 32)];
+    } else {
+      lo = n >= 32;
+      const int nn = n % 32;
+      v = nn < 25 ? Weff[K * 25 + nn] : 0.f;
+    }
+    const float h = tf32_rna(v);
+    bfwd[f] = lo ? tf32_rna(v - h) : h;
+  }
+  {
+    // backward: B[n][K] = weight[n][K]
+    int kb, n;
+    if (off < 2 * 256 * 64) { kb = off / (256 * 64); n = (off % (256 * 64)) / 64; }
+    else { kb = 2 + (off - 2 * 256 * 64) / (64 * 64); n = ((off - 2 * 256 * 64) % (64 * 64)) / 64; }
+    float v;
+    bool lo;
+    if (kb < 2) {
+      lo = n >= 128;
+      const int nn = n % 128, K = kb * 16 + k;
+      v = K < 25 ? Weff[nn * 25 + K] : 0.f;
+    } else {
+      lo = n >= 32;
+      const int nn = n % 32, K = (kb - 2) * 16 + k;
+      v = U0[nn * 64 + K];
+    }
+    const float h = tf32_rna(v);
+    bbwd[f] = lo ? tf32_rna(v - h) : h;
+  }
+}
+
+}  // namespace ctc
+}  // namespace emp

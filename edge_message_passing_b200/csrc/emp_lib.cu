@@ -13,6 +13,7 @@
 #include "conv.cuh"
 #include "so2_tc.cuh"
 #include "chain.cuh"
+#include "chain_tc.cuh"
 
 using namespace emp;
 
@@ -396,8 +397,8 @@ int ensure_attrs() {
                                     (int)rs_smem_bytes(256, false)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(k_rotate_staged<true, RS_V_BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)rs_smem_bytes(256, true)));
-  EMP_CUDA_TRY(cudaFuncSetAttribute(k_chain_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ChainFwdSmem)));
-  EMP_CUDA_TRY(cudaFuncSetAttribute(k_chain_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ChainBwdSmem)));
+  EMP_CUDA_TRY(cudaFuncSetAttribute(ctc::k_chain_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, ctc::smem_bytes(true)));
+  EMP_CUDA_TRY(cudaFuncSetAttribute(ctc::k_chain_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, ctc::smem_bytes(false)));
   int st = so2_tc_init();
   if (st != EMP_OK) return st;
   g_attrs_set = true;
@@ -955,12 +956,14 @@ int mp_chain_create(const float* U, const float* M, void** chain) {
   if (st != EMP_OK) return st;
   Chain* c = new Chain();
   float* base = nullptr;
-  const size_t n = 128 * 25 + 32 * 64 + 4 * 32 * 64 + 256 * 25;
+  const size_t n = 128 * 25 + 32 * 64 + 2 * ctc::B_FLOATS + 4 * 32 * 64 + 256 * 25;
   if (cudaMalloc(&base, n * 4) != cudaSuccess) { delete c; return EMP_ERR_CUDA; }
   c->base = base;
   c->Weff = base;
   c->U0 = base + 128 * 25;
-  float* dU = c->U0 + 32 * 64;
+  c->bfwd = c->U0 + 32 * 64;
+  c->bbwd = c->bfwd + ctc::B_FLOATS;
+  float* dU = c->bbwd + ctc::B_FLOATS;
   float* dM = dU + 4 * 32 * 64;
   if (cudaMemcpy(dU, U, 4 * 32 * 64 * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
       cudaMemcpy(dM, M, 256 * 25 * 4, cudaMemcpyHostToDevice) != cudaSuccess) {
@@ -969,6 +972,7 @@ int mp_chain_create(const float* U, const float* M, void** chain) {
     return EMP_ERR_CUDA;
   }
   k_chain_fold<<<(128 * 25 + 255) / 256, 256>>>(dU, dM, c->Weff, c->U0);
+  ctc::k_chain_bmats<<<(ctc::B_FLOATS + 255) / 256, 256>>>(c->Weff, c->U0, c->bfwd, c->bbwd);
   if (cudaDeviceSynchronize() != cudaSuccess) { cudaFree(base); delete c; return EMP_ERR_CUDA; }
   *chain = c;
   return EMP_OK;
@@ -989,12 +993,19 @@ int mp_radial_chain(const void* chain, int64_t E, const float* x, float* kc, flo
   if (!a16(x) || !a16(y0) || (g_x && (!a16(g_x) || !a16(g_y0) || !a16(g_kc)))) return EMP_ERR_ARG;
   if (E == 0) return EMP_OK;
   const Chain& c = *static_cast<const Chain*>(chain);
-  // persistent grids: as many blocks as stay resident (shared memory: 2 / 3 per SM)
-  const long long ntiles = (E + CH_ROWS - 1) / CH_ROWS;
-  const unsigned gf = (unsigned)std::min<long long>(ntiles, 2 * tc::num_sms());
-  const unsigned gb = (unsigned)std::min<long long>(ntiles, 3 * tc::num_sms());
-  { Scope sc_("chain_fwd", stream); k_chain_fwd<<<gf, CH_FWD_THREADS, sizeof(ChainFwdSmem), stream>>>(E, x, c.Weff, c.U0, kc, y0); }
-  if (g_x) { Scope sc_("chain_bwd", stream); k_chain_bwd<<<gb, 256, sizeof(ChainBwdSmem), stream>>>(E, g_kc, g_y0, c.Weff, c.U0, g_x); }
+  if (E > INT32_MAX - ctc::BM) return EMP_ERR_ARG;             // tensor-map row coordinates are 32-bit
+  // persistent: one CTA per SM (its shared memory and all of TMEM), 128-row tiles round-robin
+  const long long nt = (E + ctc::BM - 1) / ctc::BM;
+  const unsigned g = (unsigned)std::min<long long>(nt, tc::num_sms());
+  CUtensorMap mx;
+  if (!tc::make_map(&mx, x, 128, (uint64_t)E, 128, ctc::BM)) return EMP_ERR_CUDA;
+  { Scope sc_("chain_fwd", stream); ctc::k_chain_tc<true><<<g, ctc::THREADS, ctc::smem_bytes(true), stream>>>(E, mx, nullptr, c.bfwd, kc, y0); }
+  if (g_x) {
+    CUtensorMap mg;
+    if (!tc::make_map(&mg, g_y0, 64, (uint64_t)E, 64, ctc::BM)) return EMP_ERR_CUDA;
+    Scope sc_("chain_bwd", stream);
+    ctc::k_chain_tc<false><<<g, ctc::THREADS, ctc::smem_bytes(false), stream>>>(E, mg, g_kc, c.bbwd, g_x, nullptr);
+  }
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
 

@@ -178,8 +178,9 @@ void mp_chain_destroy(void* chain);
 
 /* kc [E][25] = x_flat @ W_eff; y0 [E][64] = x[:,0,:] @ U_0.  If g_x is not
  * NULL also g_x [E][4][32] = g_kc @ W_eff^T (+ g_y0 @ U_0^T into degree 0).
- * x, g_kc, g_y0 row-major; E >= 0.  x, y0, g_kc, g_y0 and g_x 16-byte aligned
- * (EMP_ERR_ARG otherwise: their rows are moved as float4 and by bulk copies). */
+ * Products on the tensor cores in 3xTF32 (FP32 accuracy).  x, g_kc, g_y0
+ * row-major; 0 <= E < 2^31 - 128.  x, y0, g_kc, g_y0 and g_x 16-byte aligned
+ * (EMP_ERR_ARG otherwise: x and g_y0 are read by TMA, g_kc by bulk copies). */
 int mp_radial_chain(const void* chain, int64_t E, const float* x, float* kc, float* y0,
                     const float* g_kc, const float* g_y0, float* g_x, cudaStream_t stream);
 

@@ -221,6 +221,20 @@ def test_radial_chain_ragged_and_empty():
     assert kc.shape == (0, 25)
 
 
+# edges per tile: 128 rows; sizes around one tile and with an uneven number of tiles per SM
+@pytest.mark.parametrize("E", [1, 127, 128, 129, 148 * 128 * 3 + 77])
+def test_radial_chain_tile_edges(E):
+    ci = synth.chain_inputs(E=E, seed=20 + E % 7)
+    ch = emp.Chain(ci.U, ci.M)
+    kc, y0, gx = emp.mp_radial_chain(ch, _cuda(ci.x), _cuda(ci.g_kc), _cuda(ci.g_y0))
+    W_eff = ochain.fold(ci.U, ci.M)
+    rk, ry = ochain.folded_forward(ci.x, W_eff, ci.U[0])
+    rg = ochain.folded_backward(ci.g_kc, ci.g_y0, W_eff, ci.U[0])
+    for got, ref in ((kc, rk), (y0, ry), (gx, rg)):
+        assert np.abs(got.cpu().numpy().reshape(ref.shape) - ref).max() <= 1e-5 * np.abs(ref).max()
+    assert emp.last_device_error() == 0
+
+
 # ------------------------------------------------------------------ full-size workloads
 def _stored_oracle(name):
     path = os.path.join(GOLD, f"{name}_oracle.npz")
