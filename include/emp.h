@@ -179,8 +179,9 @@ void mp_chain_destroy(void* chain);
 /* kc [E][25] = x_flat @ W_eff; y0 [E][64] = x[:,0,:] @ U_0.  If g_x is not
  * NULL also g_x [E][4][32] = g_kc @ W_eff^T (+ g_y0 @ U_0^T into degree 0).
  * Products on the tensor cores in 3xTF32 (FP32 accuracy).  x, g_kc, g_y0
- * row-major; 0 <= E < 2^31 - 128.  x, y0, g_kc, g_y0 and g_x 16-byte aligned
- * (EMP_ERR_ARG otherwise: x and g_y0 are read by TMA, g_kc by bulk copies). */
+ * row-major; 0 <= E < 2^31 - 128.  x, kc, y0, g_kc, g_y0 and g_x 16-byte
+ * aligned (EMP_ERR_ARG otherwise: x and g_y0 are read by TMA, g_kc by bulk
+ * copies, the outputs stored as float4). */
 int mp_radial_chain(const void* chain, int64_t E, const float* x, float* kc, float* y0,
                     const float* g_kc, const float* g_y0, float* g_x, cudaStream_t stream);
 
