@@ -24,6 +24,7 @@ import json
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -85,10 +86,10 @@ class ClockSampler:
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, out_dir: str | None = None):
         self.idx = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        self.path = os.path.join(out_dir or tempfile.gettempdir(), f"clocks_rank{gpu_index}.csv")
 
     def __enter__(self):
         try:
@@ -388,7 +389,7 @@ def run_ours(args):
         emp.profile_enable(False)
         return times, fam
 
-    with ClockSampler(dev) as clk:
+    with ClockSampler(dev, args.clocks_dir) as clk:
         # let the sampler start polling before the timed steps (its start-up stalls the driver)
         for _ in range(2):
             efg.replay()
@@ -515,6 +516,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the other seeded workloads")
+    ap.add_argument("--clocks-dir", default=None, help="where the raw nvidia-smi samples go (default: temp dir)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
