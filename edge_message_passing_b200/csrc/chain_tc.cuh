@@ -284,8 +284,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * ACC_COLS);
       float v[32], w[32];
       if (FWD) {
-        // kc: the four partial column groups; the warp's 32 rows of 25 are 800 contiguous floats
-        // the four partial column groups, two at a time, summed in this lane's staging row
+        // kc: the four partial column groups, two at a time, summed in this lane's staging row
         tmem_ld2(base, base + 96, v, w);
         add32(v, w);
 #pragma unroll
@@ -302,12 +301,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         stg[lane * EPI_PITCH + 24] += v[24];
         __syncwarp();
-        // the 800 floats as 200 float4 (r0 * 25 floats is a multiple of 4: r0 is of 32 rows)
+        // the warp's 32 rows of 25 are 800 contiguous floats, stored as 200 float4
+        // (r0 * 25 is a multiple of 4: r0 is a multiple of 32)
         const long long nflt = (E - r0 < 32 ? E - r0 : 32) * 25;
         float* dst = out0 + (size_t)r0 * 25;
 #pragma unroll 1
-        for (int q = lane; q < 200; q += 32) {
-          const int e0 = 4 * q;
+        for (int p4 = lane; p4 < 200; p4 += 32) {
+          const int e0 = 4 * p4;
           if (e0 + 4 <= nflt) {
             float4 o;
             o.x = stg[((e0 + 0) / 25) * EPI_PITCH + (e0 + 0) % 25];
