@@ -23,6 +23,7 @@ SYMBOLS = (
     "mp_workspace_bytes", "mp_forward", "mp_energy_forces", "mp_so2_mix", "mp_chain_create",
     "mp_chain_destroy", "mp_radial_chain", "emp_status_string", "emp_last_device_error",
     "emp_profile_enable", "emp_profile_read", "emp_profile_names", "emp_launch_count",
+    "emp_set_wait_limit", "emp_wait_selftest",
 )
 
 
@@ -98,6 +99,10 @@ def lib() -> ctypes.CDLL:
         L.emp_profile_names.argtypes = [ctypes.c_char_p, sz]
         L.emp_launch_count.restype = i64
         L.emp_launch_count.argtypes = []
+        L.emp_set_wait_limit.restype = ctypes.c_int
+        L.emp_set_wait_limit.argtypes = [i64]
+        L.emp_wait_selftest.restype = ctypes.c_int
+        L.emp_wait_selftest.argtypes = [vp]
         _lib_handle = L
     return _lib_handle
 
@@ -125,6 +130,17 @@ def _stream():
 def last_device_error() -> int:
     """Read and clear the device error word (0 = none)."""
     return lib().emp_last_device_error()
+
+
+def set_wait_limit(cycles: int = 0) -> None:
+    """Bound (clock64 cycles) of every device-side wait; 0 restores the default (~2 s)."""
+    _check(lib().emp_set_wait_limit(int(cycles)), "emp_set_wait_limit")
+
+
+def wait_selftest() -> int:
+    """One bounded wait that nothing satisfies; returns the device error it records."""
+    _check(lib().emp_wait_selftest(_stream()), "emp_wait_selftest")
+    return last_device_error()
 
 
 def profile_enable(on: bool = True) -> None:

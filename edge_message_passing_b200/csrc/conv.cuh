@@ -875,8 +875,9 @@ __global__ void __launch_bounds__(256, 2)
     bulk_g2s(st + oR, R + (size_t)m.rr * 4 * C, bR, &full[s]);
     bulk_g2s(st + oR + 4 * C, D + (size_t)(e0 + m.el) * NDBLK, NDBLK * 4, &full[s]);
   };
+  int nissued = 0;                     // positions whose copies thread 0 has issued
   if (t == 0)
-    for (int q = 0; q < min(BE_STAGES, np); ++q) issue(q);
+    for (; nissued < min(BE_STAGES, np); ++nissued) issue(nissued);
   T gxs[16];
 #pragma unroll
   for (int k = 0; k < 16; ++k) gxs[k] = vset<T>(0.f);
@@ -884,10 +885,12 @@ __global__ void __launch_bounds__(256, 2)
   T* gHv = reinterpret_cast<T*>(gR_hi);
   T* gLv = reinterpret_cast<T*>(gR_lo);
   T* Pgv = reinterpret_cast<T*>(Pg);
+  int qdone = np;                      // positions waited for by every thread
 #pragma unroll 1
   for (int q = 0; q < np; ++q) {
     const int s = q % BE_STAGES;
-    tc::mbar_wait(&full[s], (uint32_t)((q / BE_STAGES) & 1));   // bounded; a timeout sets the device error
+    // bounded; a timeout sets the device error, and the block leaves the loop (all threads at once)
+    const bool arrived = tc::mbar_wait(&full[s], (uint32_t)((q / BE_STAGES) & 1));
     const float* st = stage0 + s * SF;
     const BeMeta m = meta[q];
     const T* sY = reinterpret_cast<const T*>(st) + t;
@@ -938,8 +941,12 @@ __global__ void __launch_bounds__(256, 2)
       }
       qs = q + 1;
     }
-    __syncthreads();                   // stage s read by every thread: free for reuse
-    if (t == 0 && q + BE_STAGES < np) issue(q + BE_STAGES);
+    // stage s read by every thread: free for reuse (unless a wait ran out: then stop)
+    if (__syncthreads_or(!arrived)) {
+      qdone = q;
+      break;
+    }
+    if (t == 0 && q + BE_STAGES < np) issue(nissued++);
   }
   // torque of every edge of the range: a = -R_e^T (b_x, b_y, 0), g_r += (a x r) / |r|^2
   for (int q = t; q < np; q += CV) {
@@ -962,13 +969,10 @@ __global__ void __launch_bounds__(256, 2)
     g_r[3 * e + 1] += (az * vx - ax * vz) * id2;
     g_r[3 * e + 2] += (ax * vy - ay * vx) * id2;
   }
-  // every copy was waited for above; after a timed-out wait, wait (bounded) once more for the
-  // last copy into each stage so that none is still landing when the block exits
+  // after a wait that ran out, wait (bounded) for the copies still in flight so that none is
+  // landing in shared memory when the block exits
   if (t == 0)
-    for (int s = 0; s < BE_STAGES && s < np; ++s) {
-      const int ql = s + ((np - 1 - s) / BE_STAGES) * BE_STAGES;
-      tc::mbar_wait(&full[s], (uint32_t)((ql / BE_STAGES) & 1));
-    }
+    for (int q = qdone; q < nissued; ++q) tc::mbar_wait(&full[q % BE_STAGES], (uint32_t)((q / BE_STAGES) & 1));
 }
 
 // channels per thread of the backward edge kernel.  One: with the ring's shared memory
@@ -1100,16 +1104,19 @@ __global__ void __launch_bounds__(256)
     bulk_g2s(st + offR, R + (size_t)m.z * 4 * C, bR, &full[s]);
     bulk_g2s(st + offD, D + (size_t)(e0 + p0 + q) * NDBLK, NDBLK * 4, &full[s]);
   };
+  int nissued = 0;                     // positions whose copies thread 0 has issued
   if (t == 0)
-    for (int q = 0; q < min(RS_STAGES, np); ++q) issue(q);
+    for (; nissued < min(RS_STAGES, np); ++nissued) issue(nissued);
   T* XTv = reinterpret_cast<T*>(XT);
   T* XLv = reinterpret_cast<T*>(XTlo);
   T* GHv = reinterpret_cast<T*>(GYhi);
   T* GLv = reinterpret_cast<T*>(GYlo);
+  int qdone = np;                      // positions waited for by every thread
 #pragma unroll 1
   for (int q = 0; q < np; ++q) {
     const int s = q % RS_STAGES;
-    tc::mbar_wait(&full[s], (uint32_t)((q / RS_STAGES) & 1));   // bounded; a timeout sets the device error
+    // bounded; a timeout sets the device error, and the block leaves the loop (all threads at once)
+    const bool arrived = tc::mbar_wait(&full[s], (uint32_t)((q / RS_STAGES) & 1));
     const float* st = stage0 + s * SF;
     const T* sX = reinterpret_cast<const T*>(st) + t;
     const T* sR = reinterpret_cast<const T*>(st + offR) + t;
@@ -1151,14 +1158,16 @@ __global__ void __launch_bounds__(256)
         }
       }
     }
-    __syncthreads();                   // stage s read by every thread: free for reuse
-    if (t == 0 && q + RS_STAGES < np) issue(q + RS_STAGES);
-  }
-  if (t == 0)
-    for (int s = 0; s < RS_STAGES && s < np; ++s) {
-      const int ql = s + ((np - 1 - s) / RS_STAGES) * RS_STAGES;
-      tc::mbar_wait(&full[s], (uint32_t)((ql / RS_STAGES) & 1));
+    // stage s read by every thread: free for reuse (unless a wait ran out: then stop)
+    if (__syncthreads_or(!arrived)) {
+      qdone = q;
+      break;
     }
+    if (t == 0 && q + RS_STAGES < np) issue(nissued++);
+  }
+  // after a wait that ran out, wait (bounded) for the copies still in flight
+  if (t == 0)
+    for (int q = qdone; q < nissued; ++q) tc::mbar_wait(&full[q % RS_STAGES], (uint32_t)((q / RS_STAGES) & 1));
 }
 
 // vector widths (channels per thread) of the staged rotate kernels

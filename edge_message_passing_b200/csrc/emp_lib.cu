@@ -14,6 +14,7 @@
 #include "so2_tc.cuh"
 #include "chain.cuh"
 #include "chain_tc.cuh"
+#include "end_layers.cuh"
 
 using namespace emp;
 
@@ -74,7 +75,7 @@ constexpr int LAYER0_COHORTS = 4;
 
 // ------------------------------------------------------------------ workspace layout
 struct WsLayout {
-  size_t D, dist, R, rbP, gxP, XT2, XTlo2, Y2, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
+  size_t D, dist, R, rbP, nodeZ, nodeX, gxP, XT2, XTlo2, Y2, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
   size_t total;
 };
 
@@ -104,6 +105,8 @@ WsLayout ws_layout(const Model& m, long long E, int N) {
   L.gx0 = take(feat);
   L.gx1 = take(feat);
   L.gS = take(feat);
+  L.nodeZ = take(feat);
+  L.nodeX = take((size_t)N * 4 * C * 4);
   L.e_atom = take((size_t)N * 4);
   const size_t cb = coh * 16 * C * 4;
   L.gxP = take(cb);
@@ -128,9 +131,10 @@ WsLayout ws_layout(const Model& m, long long E, int N) {
 template <typename T>
 T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
 
+// the edge arrays may be null when there are no edges (an empty tensor has no storage)
 bool graph_ok(const emp_graph* g) {
-  return g && g->recv && g->send && g->mirror && g->recv_off && g->vec && g->n_edges >= 0 &&
-         g->n_edges < (1ll << 31);
+  return g && g->recv_off && g->n_edges >= 0 && g->n_edges < (1ll << 31) &&
+         (g->n_edges == 0 || (g->recv && g->send && g->mirror && g->vec));
 }
 
 RadialArgs radial_args(const Model& m, int t) {
@@ -156,6 +160,15 @@ int grid_for(long long n, int per, int cap = 148 * 32) {
 int so2_product(const Model& m, long long M, const So2Part* parts, int nparts, int* counter, cudaStream_t s) {
   Scope sc_("so2_tc", s);
   return so2_tc(M, m.spec.C, parts, nparts, counter, s);
+}
+
+// per-node FP32 product (end_layers.cuh: k_node_gemm)
+void node_gemm(int rows, int K, int Nn, int w, const float* A, long long a_node, int a_comp, const float* B, int ldb,
+               float* out, long long o_node, int o_comp, cudaStream_t s) {
+  if (rows <= 0) return;
+  const dim3 grid((unsigned)((rows + NG_T - 1) / NG_T), (unsigned)((Nn + NG_T - 1) / NG_T));
+  Scope sc_("node_gemm", s);
+  k_node_gemm<<<grid, 256, 0, s>>>(rows, K, Nn, w, A, a_node, a_comp, B, ldb, out, o_node, o_comp);
 }
 
 // tensor maps of a cohort buffer pair for the full cohort size and for the last (short) cohort
@@ -336,8 +349,9 @@ int radial_rows(const Model& m, const emp_graph* g, const int* species, void* ws
 }
 
 // R rows [E][4C] of layer t: hidden layers on SIMT, head R = h2 W3^T on the tensor cores
+// ncols: 4C, or C when only the degree-0 scales are used (the first layer: degree-0 input)
 int radial_forward(const Model& m, const emp_graph* g, int t, const int* species, const float* dist, float* R,
-                   const RadialRows& rr, void* ws, const WsLayout& L, cudaStream_t s) {
+                   const RadialRows& rr, void* ws, const WsLayout& L, cudaStream_t s, int ncols) {
   const long long E = g->n_edges;
   const int C = m.spec.C;
   float* h2hi = at<float>(ws, L.h2hi);
@@ -350,8 +364,8 @@ int radial_forward(const Model& m, const emp_graph* g, int t, const int* species
     MapPair a;
     int st = make_pair(&a, h2hi + r0 * 64, h2lo + r0 * 64, n, 64, 64, tc::BM);
     if (st != EMP_OK) return st;
-    const MapPair& b = m.w3_maps[(size_t)t * m.n_pairs + p];
-    GemmSub sub{&a.hi, &a.lo, &b.hi, &b.lo, 0, 64, 4 * C, 0, R + r0 * 4 * C};
+    const MapPair& b = (ncols == C ? m.w3n_maps : m.w3_maps)[(size_t)t * m.n_pairs + p];
+    GemmSub sub{&a.hi, &a.lo, &b.hi, &b.lo, 0, 64, ncols, 0, R + r0 * 4 * C};
     Scope sc_("radial_head", s);
     st = tc_group(n, 4 * C, &sub, 1, at<int>(ws, L.counter), s);
     if (st != EMP_OK) return st;
@@ -361,8 +375,9 @@ int radial_forward(const Model& m, const emp_graph* g, int t, const int* species
 
 // dE/dd of layer t from dE/dR (rows split hi/lo): dE/dh2 = dE/dR W3 on the tensor cores, then the
 // hidden layers' backward on SIMT; adds (dE/dd) rhat to g_r
+// kcols: 4C, or C when only the degree-0 scales carry a gradient (the first layer)
 int radial_backward(const Model& m, const emp_graph* g, int t, const int* species, const float* dist,
-                    const RadialRows& rr, float* g_r, void* ws, const WsLayout& L, cudaStream_t s) {
+                    const RadialRows& rr, float* g_r, void* ws, const WsLayout& L, cudaStream_t s, int kcols) {
   const long long E = g->n_edges;
   const int C = m.spec.C;
   float* gRhi = at<float>(ws, L.gRhi);
@@ -375,7 +390,7 @@ int radial_backward(const Model& m, const emp_graph* g, int t, const int* specie
     int st = make_pair(&a, gRhi + r0 * 4 * C, gRlo + r0 * 4 * C, n, 4 * C, 4 * C, tc::BM);
     if (st != EMP_OK) return st;
     const MapPair& b = m.w3t_maps[(size_t)t * m.n_pairs + p];
-    GemmSub sub{&a.hi, &a.lo, &b.hi, &b.lo, 0, 4 * C, 64, 0, gh2 + r0 * 64};
+    GemmSub sub{&a.hi, &a.lo, &b.hi, &b.lo, 0, kcols, 64, 0, gh2 + r0 * 64};
     Scope sc_("radial_head_bwd", s);
     st = tc_group(n, 64, &sub, 1, at<int>(ws, L.counter), s);
     if (st != EMP_OK) return st;
@@ -405,6 +420,18 @@ int ensure_attrs() {
   return EMP_OK;
 }
 
+// One bounded wait on an mbarrier that nothing arrives on: it runs out after the limit in
+// force (emp_set_wait_limit), records EMP_ERR_TIMEOUT in the device error word and returns.
+__global__ void k_wait_selftest() {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) tc::mbar_wait(&bar, 0);
+}
+
 int check_device() {
   int dev = 0, major = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return EMP_ERR_UNSUPPORTED;
@@ -423,22 +450,15 @@ int check_device() {
 static __device__ __align__(256) unsigned char g_nl_noalloc_scratch[EMP_NL_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-std::mutex g_noalloc_mu;
-void* g_noalloc_addr[64] = {};
-
-// Device address of the scratch array for the current device.  In host code the
+// Device address of the scratch array on the current device.  In host code the
 // array's name is only a host-side stand-in, so the address is looked up with
-// cudaGetSymbolAddress (once per device, with that device current).
+// cudaGetSymbolAddress, with the device current, on every call: the lookup is
+// cheap once the module is loaded, and an address kept from before a device reset
+// would point into a context that no longer exists.
 int nl_noalloc_scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EMP_ERR_CUDA;
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_nl_noalloc_scratch) != cudaSuccess || !ptr) return EMP_ERR_CUDA;
-    g_noalloc_addr[dev] = ptr;
-  }
-  *out = g_noalloc_addr[dev];
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_nl_noalloc_scratch) != cudaSuccess || !ptr) return EMP_ERR_CUDA;
+  *out = ptr;
   return EMP_OK;
 }
 }  // namespace
@@ -503,6 +523,19 @@ int64_t emp_launch_count(void) {
   return g_prof.launches;
 }
 
+int emp_set_wait_limit(int64_t cycles) {
+  const long long v = cycles > 0 ? (long long)cycles : tc::TIMEOUT_CYCLES;
+  EMP_CUDA_TRY(cudaMemcpyToSymbol(tc::g_wait_cycles, &v, sizeof(v)));
+  return EMP_OK;
+}
+
+int emp_wait_selftest(cudaStream_t stream) {
+  int st = check_device();
+  if (st != EMP_OK) return st;
+  k_wait_selftest<<<1, 32, 0, stream>>>();
+  return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
+}
+
 int emp_last_device_error(void) {
   int h = 0, z = 0;
   if (cudaMemcpyFromSymbol(&h, g_device_error, sizeof(int)) != cudaSuccess) return EMP_ERR_CUDA;
@@ -525,7 +558,7 @@ static int nl_build_impl(const emp_nl_params* p, const double* pos, emp_graph* g
   for (int d = 0; d < 3; ++d)
     if (!(p->box[d] > 0) || !std::isfinite(p->box[d])) return EMP_ERR_ARG;
   if (ws_bytes < nl_workspace_bytes(N)) return EMP_ERR_WORKSPACE;
-  if (p->capacity > 0 && !graph_ok(g)) return EMP_ERR_ARG;
+  if (p->capacity > 0 && !(g->recv && g->send && g->mirror && g->shift && g->vec)) return EMP_ERR_ARG;
   int st = check_device();
   if (st != EMP_OK) return st;
   // cell grid: cells no smaller than rc (1 + 1e-9), at most N cells
@@ -576,6 +609,8 @@ static int nl_build_impl(const emp_nl_params* p, const double* pos, emp_graph* g
   *n_edges = total;
   g->n_edges = total;
   g->n_atoms = N;
+  if (flags[1]) return EMP_ERR_DEVICE;         // a receiver with more than nl::MAX_CAND edges
+  if (flags[2]) return EMP_ERR_UNSUPPORTED;    // an image shift beyond +-nl::MAX_SHIFT box lengths
   if (total > p->capacity) return EMP_ERR_CAPACITY;
   if (total >= (1ll << 31)) return EMP_ERR_CAPACITY;
   { Scope sc_("nl", stream); nl::k_emit<<<N, nl::EMIT_THREADS, 0, stream>>>(pos, N, G, W, g->recv_off, *g); }
@@ -593,8 +628,8 @@ int nl_build(const emp_nl_params* p, const double* pos, emp_graph* g, int64_t* n
 // plug-in inside a host program whose device memory all comes from that
 // program's own pool, or a code path that must not trigger the device-wide
 // synchronisation cudaMalloc/cudaFree can cause.  The scratch is the file-scope
-// array g_nl_noalloc_scratch below; its device address is looked up once per
-// device, on the first call made with that device current.
+// array g_nl_noalloc_scratch above; its device address is looked up on each call,
+// with the caller's device current.
 int nl_build_noalloc(const emp_nl_params* p, const double* pos, emp_graph* g, int64_t* n_edges,
                      cudaStream_t stream) {
   if (!p || !pos || !g || !n_edges) return EMP_ERR_ARG;
@@ -689,10 +724,12 @@ int mp_model_create(const emp_model_spec* spec, const float* weights, size_t n_f
       k_split_tf32<<<64, 256>>>(tmpT, m->w3t_hi + wo, m->w3t_lo + wo, m->w3_stride());
     }
   m->w3_maps.resize(T * m->n_pairs);
+  m->w3n_maps.resize(T * m->n_pairs);
   m->w3t_maps.resize(T * m->n_pairs);
   for (size_t q = 0; q < T * m->n_pairs; ++q) {
     const size_t wo = q * m->w3_stride();
     if (make_pair(&m->w3_maps[q], m->w3_hi + wo, m->w3_lo + wo, 4 * C, 64, 64, tc::b_box_rows(4 * (int)C)) != EMP_OK ||
+        make_pair(&m->w3n_maps[q], m->w3_hi + wo, m->w3_lo + wo, C, 64, 64, tc::b_box_rows((int)C)) != EMP_OK ||
         make_pair(&m->w3t_maps[q], m->w3t_hi + wo, m->w3t_lo + wo, 64, 4 * (int)C, 4 * (int)C, tc::b_box_rows(64)) !=
             EMP_OK)
       return fail(EMP_ERR_CUDA);
@@ -770,7 +807,7 @@ int mp_forward(const void* model, const emp_graph* g, int32_t layer, const int32
   RadialRows rr;
   st = radial_rows(m, g, species, ws, L, rr, stream);
   if (st != EMP_OK) return st;
-  st = radial_forward(m, g, layer, species, dist, R, rr, ws, L, stream);
+  st = radial_forward(m, g, layer, species, dist, R, rr, ws, L, stream, 4 * C);
   if (st != EMP_OK) return st;
   st = layer_forward(m, g, layer, x_in, D, R, rr.inv, 0, agg_out, ws, L, stream);
   if (st != EMP_OK) return st;
@@ -826,90 +863,104 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
   { Scope sc_("embed", stream); k_embed<<<(unsigned)((feat + 255) / 256), 256, 0, stream>>>(N, C, species, m.spec.n_species, m.emb, xs); }
   if (E > 0) {
     { Scope sc_("geometry", stream); k_geometry<<<(unsigned)((E + 127) / 128), 128, 0, stream>>>(E, g->vec, D, dist); }
-    const int ncoh = (int)((E + coh - 1) / coh);
-    int P = 1;
-    while (P < coh) P <<= 1;
-    { Scope sc_("cohort_sort", stream); k_cohort_sort<<<ncoh, 1024, (size_t)P * 8, stream>>>(E, (int)coh, g->send, perm, seg, nseg); }
+    if (T > 2) {      // sender order of the cohorts, for the backward of the layers between the first and the last
+      const int ncoh = (int)((E + coh - 1) / coh);
+      int P = 1;
+      while (P < coh) P <<= 1;
+      { Scope sc_("cohort_sort", stream); k_cohort_sort<<<ncoh, 1024, (size_t)P * 8, stream>>>(E, (int)coh, g->send, perm, seg, nseg); }
+    }
   }
   RadialRows rr;
   if (E > 0) {
     st = radial_rows(m, g, species, ws, L, rr, stream);
     if (st != EMP_OK) return st;
   }
+  // The first layer (its input, the species embedding, is degree 0 only) and the last layer
+  // (read through degree 0 only) sum over each receiver's edges first and mix once per node
+  // (end_layers.cuh); the layers between them run the per-edge products over cohorts.
+  float* nodeZ = at<float>(ws, L.nodeZ);   // Z (first layer forward), H (first layer backward)
+  float* nodeX = at<float>(ws, L.nodeX);   // X (last layer forward), G (last layer backward)
+  const unsigned nb_node = (unsigned)N;
   // ---------------- forward
   for (int t = 0; t < T; ++t) {
     float* R = Rall + (size_t)t * E * 4 * C;
+    float* S = aggs + (size_t)t * feat;
+    const float* W0 = m.so2_fwd + (size_t)t * m.so2_stride();
+    const bool first = t == 0, last = t == T - 1;
     if (E > 0) {
-      st = radial_forward(m, g, t, species, dist, R, rr, ws, L, stream);
+      st = radial_forward(m, g, t, species, dist, R, rr, ws, L, stream, first ? C : 4 * C);
       if (st != EMP_OK) return st;
-      // the first layer's input is the species embedding: degree 0 only
-      st = layer_forward(m, g, t, xs + (size_t)t * feat, D, R, rr.inv, t == 0, aggs + (size_t)t * feat, ws, L, stream);
-      if (st != EMP_OK) return st;
+      if (first) {
+        { Scope sc_("first_fwd", stream); k_first_fwd<<<nb_node, C, 0, stream>>>(C, g->recv_off, g->send, rr.inv, D, R, xs, nodeZ); }
+        // S_i[l, m', c'] = sum_c W0[(l, c'), (0, c)] Z_i[l, m', c], one launch per degree
+        for (int l = 0; l < 4; ++l)
+          node_gemm(N * (2 * l + 1), C, C, 2 * l + 1, nodeZ + l * l * C, 16ll * C, C, W0 + (size_t)l * C * 4 * C,
+                    4 * C, S + l * l * C, 16ll * C, C, stream);
+      } else if (last) {
+        { Scope sc_("last_fwd", stream); k_last_fwd<<<nb_node, C, 0, stream>>>(C, g->recv_off, g->send, rr.inv, D, R, xs + (size_t)t * feat, nodeX); }
+        // S_i[0, c'] = sum_(l, c) W0[(0, c'), (l, c)] X_i[l, c]; the other components are not needed
+        node_gemm(N, 4 * C, C, 1, nodeX, 4ll * C, 0, W0, 4 * C, S, 16ll * C, 0, stream);
+      } else {
+        st = layer_forward(m, g, t, xs + (size_t)t * feat, D, R, rr.inv, 0, S, ws, L, stream);
+        if (st != EMP_OK) return st;
+      }
     }
-    { Scope sc_("update", stream); k_update<<<(unsigned)((N * C + 255) / 256), 256, 0, stream>>>(N, C, inv_avg, m.spec.gated, aggs + (size_t)t * feat,
+    { Scope sc_("update", stream); k_update<<<(unsigned)((N * C + 255) / 256), 256, 0, stream>>>(N, C, inv_avg, m.spec.gated, S,
                                                                    xs + (size_t)t * feat, xs + (size_t)(t + 1) * feat); }
   }
   { Scope sc_("readout", stream); k_readout<<<N, 256, 0, stream>>>(N, C, m.Hro, xs + (size_t)T * feat, m.ro_W, m.ro_w, e_atom, gxa); }
   { Scope sc_("energy_sum", stream); k_energy_sum<<<1, 1024, 0, stream>>>(N, e_atom, energy); }
-  // ---------------- backward, one layer at a time in reverse, one cohort at a time
+  // ---------------- backward, one layer at a time in reverse
   for (int t = T - 1; t >= 0; --t) {
     const float* R = Rall + (size_t)t * E * 4 * C;
     const float* xt = xs + (size_t)t * feat;
+    const float* Wb = m.so2_bwd + (size_t)t * m.so2_stride();
+    const bool first = t == 0, last = t == T - 1;
     { Scope sc_("gate_bwd", stream); k_gate_bwd<<<(unsigned)((N * C + 255) / 256), 256, 0, stream>>>(N, C, inv_avg, m.spec.gated,
                                                                      aggs + (size_t)t * feat, gxa, gS, gxb); }
-    // the first layer (degree-0 input) takes LAYER0_COHORTS cohorts at once, in narrow rows
-    const long long span = t == 0 ? LAYER0_COHORTS * coh : coh;
-    const int xp = t == 0 ? C : 16 * C, gp = t == 0 ? 4 * C : 16 * C;
-    if (t == 0) {
-      st = am_xt.build(C, E, span, XT, XTlo, C, xp);
-      if (st == EMP_OK) st = am_gy.build(C, E, span, GYhi, GYlo, 4 * C, gp);
-      if (st != EMP_OK) return st;
-    }
-    int ci = 0;
-    for (long long e0 = 0; e0 < E; e0 += span, ++ci) {
-      const long long e1 = std::min(E, e0 + span), n = e1 - e0;
-      {
-        const int per = rs_per(n, tc::num_sms(), 3);
-        Scope sc_("bwd_prep", stream);
-        k_rotate_staged<true, RS_V_BWD><<<(unsigned)((n + per - 1) / per), C / RS_V_BWD, rs_smem_bytes(C, true), stream>>>(
-            e0, e1, C, t == 0, per, g->recv, g->send, rr.inv, D, R, xt, gS, XT, XTlo, xp, GYhi, GYlo, gp);
-      }
-      if (t == 0) {
-        // degree-0 input: y needs only the m = 0 block's first C input columns, and only the
-        // degree-0 part of dE/dx~ is used (the radial scale of l = 0)
-        const So2AMaps* ax = am_xt.get(n);
-        const So2AMaps* ag = am_gy.get(n);
-        const MapPair& f0 = m.bmaps_fwd[t].blk[0];
-        const MapPair& b0 = m.b0_bwd_narrow[t];
-        GemmSub subs[2] = {{&ax->hi, &ax->lo, &f0.hi, &f0.lo, 0, C, 4 * C, 0, Y},
-                           {&ag->hi, &ag->lo, &b0.hi, &b0.lo, 0, 4 * C, C, 0, GXT}};
-        Scope sc_("so2_tc", stream);
-        st = tc_group(n, gp, subs, 2, counter, stream);
-      } else {
+    if (E > 0 && first) {
+      // H_i[l, m', c] = sum_c' W0[(l, c'), (0, c)] gS_i[l, m', c']
+      for (int l = 0; l < 4; ++l)
+        node_gemm(N * (2 * l + 1), C, C, 2 * l + 1, gS + l * l * C, 16ll * C, C, Wb + (size_t)l * C, 4 * C,
+                  nodeZ + l * l * C, 16ll * C, C, stream);
+      { Scope sc_("first_bwd", stream); k_first_bwd<<<nb_node, C, 0, stream>>>(C, g->recv_off, g->send, rr.inv, g->vec, D, R, xt, nodeZ, gRhi, gRlo, g_r); }
+    } else if (E > 0 && last) {
+      // the output gradient is degree 0 only: G_i[l, c] = sum_c' W0[(0, c'), (l, c)] gS_i[0, c']
+      node_gemm(N, C, 4 * C, 1, gS, 16ll * C, 0, Wb, 4 * C, nodeX, 4ll * C, 0, stream);
+      { Scope sc_("last_bwd", stream); k_last_bwd<<<nb_node, C, 0, stream>>>(C, g->recv_off, g->send, rr.inv, g->vec, D, R, xt, nodeX, gRhi, gRlo, g_r, gxb); }
+    } else if (E > 0) {
+      int ci = 0;
+      for (long long e0 = 0; e0 < E; e0 += coh, ++ci) {
+        const long long e1 = std::min(E, e0 + coh), n = e1 - e0;
+        {
+          const int per = rs_per(n, tc::num_sms(), 3);
+          Scope sc_("bwd_prep", stream);
+          k_rotate_staged<true, RS_V_BWD><<<(unsigned)((n + per - 1) / per), C / RS_V_BWD, rs_smem_bytes(C, true), stream>>>(
+              e0, e1, C, 0, per, g->recv, g->send, rr.inv, D, R, xt, gS, XT, XTlo, 16 * C, GYhi, GYlo, 16 * C);
+        }
         So2Part parts[2] = {{am_xt.get(n), &m.bmaps_fwd[t], Y}, {am_gy.get(n), &m.bmaps_bwd[t], GXT}};
         st = so2_product(m, n, parts, 2, counter, stream);
-      }
-      if (st != EMP_OK) return st;
-      // per-edge backward; for t > 0 also the sender sums of dE/dx_send into gxb
-      const int per = be_per(n, tc::num_sms());
-      const int nb = (int)((n + per - 1) / per);
-      float* Pg = at<float>(ws, L.gxP);
-      side.wait();      // the previous cohort's combine has read Pg
-      {
-        Scope sc_("bwd_edge", stream);
-        k_bwd_edge<BE_V><<<nb, C / BE_V, be_smem_bytes(C), stream>>>(e0, e1, C, t > 0, t == 0, per, g->send, rr.inv, g->vec, D, R,
-                                                           xt, Y, gS, GXT, gp, gp, g->recv, perm, gRhi, gRlo, g_r, Pg);
-      }
-      if (t > 0)
+        if (st != EMP_OK) return st;
+        // per-edge backward and the sender sums of dE/dx_send into gxb
+        const int per = be_per(n, tc::num_sms());
+        const int nb = (int)((n + per - 1) / per);
+        float* Pg = at<float>(ws, L.gxP);
+        side.wait();      // the previous cohort's combine has read Pg
+        {
+          Scope sc_("bwd_edge", stream);
+          k_bwd_edge<BE_V><<<nb, C / BE_V, be_smem_bytes(C), stream>>>(e0, e1, C, 1, 0, per, g->send, rr.inv, g->vec, D, R,
+                                                             xt, Y, gS, GXT, 16 * C, 16 * C, g->recv, perm, gRhi, gRlo, g_r, Pg);
+        }
         side.run([&](cudaStream_t q) {
           Scope sc_("gx_combine", q);
           k_gx_combine<<<(unsigned)std::min<long long>(n, 2048), C, 0, q>>>(e0, e1, C, ci, per, g->send, perm, seg,
                                                                           nseg, Pg, gxb);
         });
+      }
+      side.wait();        // g_x of this layer complete
     }
-    side.wait();        // g_x of this layer complete
     if (E > 0) {
-      st = radial_backward(m, g, t, species, dist, rr, g_r, ws, L, stream);
+      st = radial_backward(m, g, t, species, dist, rr, g_r, ws, L, stream, first ? C : 4 * C);
       if (st != EMP_OK) return st;
     }
     std::swap(gxa, gxb);

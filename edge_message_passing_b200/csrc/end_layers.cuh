@@ -1,0 +1,401 @@
+// The first and the last interaction layer of the energy + force step, where the
+// SO(2) convolution touches degree 0 on one side only.
+//
+// First layer: its input is the species embedding, degree 0 only (the initial
+// features of the seeded workloads), so the rotated input has the single column
+// x~[l=0, m=0] = R[0] (.) x_send[0] and only the m = 0 mixing block sees it.
+// The message of edge e is then m_e[l, m'] = D^l_e[0, m'] (W0 x~_e)[l], which is
+// linear in x~_e, so the receiver sum can be taken before the mixing:
+//   Z_i[l, m', c] = sum_{e: recv(e) = i} D^l_e[0, m'] R_e[0, c] x_send(e)[0, c]
+//   S_i[l, m', c'] = sum_c W0[(l, c'), (0, c)] Z_i[l, m', c]
+// (one product per node instead of one per edge).  The backward needs, per edge,
+// only the degree-0 radial scale gradient and the edge torque; both follow from
+// the per-node H_i[l, m', c] = sum_c' W0[(l, c'), (0, c)] gS_i[l, m', c'].
+//
+// Last layer: the energy reads the last features through their degree-0
+// channels only (the readout acts on x[l=0], and the gate's degree-0 output
+// SiLU(a0) depends on a0 alone), so only the degree-0 part of the last layer's
+// receiver sums is needed: S_i[0, c'] = sum_e (W0 x~_e)[0, c'] with
+// x~_e[l, 0, c] = R_e[l, c] sum_m' D^l_e[0, m'] x_send(e)[l, m', c] (only the
+// m = 0 block can reach degree 0).  Again the sum over edges comes first:
+//   X_i[l, c] = sum_{e: recv(e) = i} x~_e[l, 0, c],  S_i[0, c'] = sum W0[(0, c'), (l, c)] X_i[l, c].
+// Its output gradient is degree 0 only, so dE/dx~_e = G_recv(e) with the per-node
+// G_i[l, c] = sum_c' W0[(0, c'), (l, c)] gS_i[0, c'] (m = 0 entries; the others vanish),
+// and the y^T J g_y part of the torque vanishes (g_y lives in degree 0, where the
+// generators are zero).
+//
+// These are exact rearrangements of the same sums (the model of the page
+// "first-order SO(2) input-gradient path": radial scales, Wigner-D rotation,
+// per-m mixing, rotation back, normalised receiver sum); they change only the
+// order of floating-point additions.  All sums have a fixed order: receiver i's
+// edges ascending, one block per receiver.
+#pragma once
+#include "emp_common.cuh"
+#include "model.cuh"
+
+namespace emp {
+
+// index, inside the 84 Wigner-D floats of an edge, of D^l[m][n]
+__host__ __device__ constexpr int dix(int l, int m, int n) { return dblk_off(l) + (m + l) * (2 * l + 1) + (n + l); }
+
+// the structural generator pair (a < b) of degree l joining m = a_m and m = b_m
+__host__ __device__ constexpr int jpair_of(int l, int am, int bm, int p = 0) {
+  return p >= NJPAIR ? -1
+       : (jpair_a(p) == lm_index(l, am) && jpair_b(p) == lm_index(l, bm)) ? p
+       : jpair_of(l, am, bm, p + 1);
+}
+
+constexpr int EL_CH = 16;   // edges staged per chunk
+
+// ------------------------------------------------------------------ first layer, forward
+// Z[i][k][c] for the receiver i = blockIdx.x; one thread per channel (blockDim.x = C).
+__global__ void __launch_bounds__(256) k_first_fwd(int C, const int* __restrict__ recv_off,
+                                                   const int* __restrict__ send, const int* __restrict__ rrow,
+                                                   const float* __restrict__ D, const float* __restrict__ R,
+                                                   const float* __restrict__ x, float* __restrict__ Z) {
+  __shared__ float sd[EL_CH][16];      // the m = 0 row of each degree block, per edge
+  __shared__ int ss[EL_CH], sr[EL_CH];
+  const int i = blockIdx.x, c = threadIdx.x;
+  const int e0 = recv_off[i], e1 = recv_off[i + 1];
+  float acc[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+  for (int eb = e0; eb < e1; eb += EL_CH) {
+    const int n = min(EL_CH, e1 - eb);
+    __syncthreads();
+    for (int q = c; q < n * 16; q += blockDim.x) {
+      const int k = q & 15, l = k == 0 ? 0 : k < 4 ? 1 : k < 9 ? 2 : 3;
+      sd[q >> 4][k] = D[(size_t)(eb + (q >> 4)) * NDBLK + dix(l, 0, k - l * l - l)];
+    }
+    for (int q = c; q < n; q += blockDim.x) {
+      ss[q] = send[eb + q];
+      sr[q] = rrow ? rrow[eb + q] : eb + q;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int q = 0; q < n; ++q) {
+      const float v = R[(size_t)sr[q] * 4 * C + c] * x[(size_t)ss[q] * 16 * C + c];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) acc[k] = fmaf(sd[q][k], v, acc[k]);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 16; ++k) Z[((size_t)i * 16 + k) * C + c] = acc[k];
+}
+
+// ------------------------------------------------------------------ last layer, forward
+// X[i][l][c] for the receiver i = blockIdx.x; one thread per channel.
+__global__ void __launch_bounds__(256) k_last_fwd(int C, const int* __restrict__ recv_off,
+                                                  const int* __restrict__ send, const int* __restrict__ rrow,
+                                                  const float* __restrict__ D, const float* __restrict__ R,
+                                                  const float* __restrict__ x, float* __restrict__ X) {
+  __shared__ float sd[EL_CH][16];
+  __shared__ int ss[EL_CH], sr[EL_CH];
+  const int i = blockIdx.x, c = threadIdx.x;
+  const int e0 = recv_off[i], e1 = recv_off[i + 1];
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int eb = e0; eb < e1; eb += EL_CH) {
+    const int n = min(EL_CH, e1 - eb);
+    __syncthreads();
+    for (int q = c; q < n * 16; q += blockDim.x) {
+      const int k = q & 15, l = k == 0 ? 0 : k < 4 ? 1 : k < 9 ? 2 : 3;
+      sd[q >> 4][k] = D[(size_t)(eb + (q >> 4)) * NDBLK + dix(l, 0, k - l * l - l)];
+    }
+    for (int q = c; q < n; q += blockDim.x) {
+      ss[q] = send[eb + q];
+      sr[q] = rrow ? rrow[eb + q] : eb + q;
+    }
+    __syncthreads();
+#pragma unroll 2
+    for (int q = 0; q < n; ++q) {
+      const float* xs = x + (size_t)ss[q] * 16 * C + c;
+      const float* Rr = R + (size_t)sr[q] * 4 * C + c;
+      float xv[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) xv[k] = xs[k * C];
+#pragma unroll
+      for (int l = 0; l < 4; ++l) {
+        float u = 0.f;
+#pragma unroll
+        for (int k = l * l; k < (l + 1) * (l + 1); ++k) u = fmaf(sd[q][k], xv[k], u);
+        acc[l] = fmaf(Rr[l * C], u, acc[l]);
+      }
+    }
+  }
+#pragma unroll
+  for (int l = 0; l < 4; ++l) X[((size_t)i * 4 + l) * C + c] = acc[l];
+}
+
+// ------------------------------------------------------------------ torque of a staged chunk
+// red[q][w][j]: warp w's channel sums of the edge-frame torque components; the sums over the
+// warps (in order), the frame and the cross product with r, added to g_r (one thread per edge).
+__device__ __forceinline__ void finish_torque(int n, int nw, int eb, const float* red, const float* svec,
+                                              float* __restrict__ g_r) {
+  const int q = threadIdx.x;
+  if (q >= n) return;
+  float sx = 0.f, sy = 0.f;
+  for (int w = 0; w < nw; ++w) {
+    sx += red[(q * nw + w) * 2 + 0];
+    sy += red[(q * nw + w) * 2 + 1];
+  }
+  const float vx = svec[3 * q], vy = svec[3 * q + 1], vz = svec[3 * q + 2];
+  const float d2 = vx * vx + vy * vy + vz * vz;
+  const float inv = rsqrtf(d2);
+  float Rf[3][3];
+  edge_frame<float>(vx * inv, vy * inv, vz * inv, Rf);
+  const float ax = -(Rf[0][0] * sx + Rf[1][0] * sy);
+  const float ay = -(Rf[0][1] * sx + Rf[1][1] * sy);
+  const float az = -(Rf[0][2] * sx + Rf[1][2] * sy);
+  const float id2 = 1.f / d2;
+  const size_t e = (size_t)(eb + q);
+  g_r[3 * e + 0] += (ay * vz - az * vy) * id2;
+  g_r[3 * e + 1] += (az * vx - ax * vz) * id2;
+  g_r[3 * e + 2] += (ax * vy - ay * vx) * id2;
+}
+
+// stage the chunk's Wigner-D rows (84 floats per edge), edge vectors, senders and radial rows
+__device__ __forceinline__ void stage_chunk(int eb, int n, const float* __restrict__ D, const float* __restrict__ vec,
+                                            const int* __restrict__ send, const int* __restrict__ rrow, float* sD,
+                                            float* svec, int* ss, int* sr) {
+  const int t = threadIdx.x;
+  for (int q = t; q < n * (NDBLK / 4); q += blockDim.x)
+    reinterpret_cast<float4*>(sD)[q] = reinterpret_cast<const float4*>(D + (size_t)eb * NDBLK)[q];
+  for (int q = t; q < n * 3; q += blockDim.x) svec[q] = vec[(size_t)eb * 3 + q];
+  for (int q = t; q < n; q += blockDim.x) {
+    ss[q] = send[eb + q];
+    sr[q] = rrow ? rrow[eb + q] : eb + q;
+  }
+}
+
+// ------------------------------------------------------------------ first layer, backward
+// Per edge of receiver i = blockIdx.x (one thread per channel): with H_i (per-node, see the
+// top of this file), K[l][m] = sum_m' D^l[m][m'] H_i[l][m'] for m = -1, 0, 1:
+//   dE/dx~[0,0] = sum_l K[l][0];  dE/dR[0] = dE/dx~[0,0] x_send[0]  (split hi/lo, row rr)
+//   torque: the y^T J g_y term with y = W0 x~ (m = 0 only): per degree l, the channel sums
+//   P[l][m] = sum_c x~[0,0,c] K[l][m][c] enter as -P[l][-1] on the pair (-1, 0) and
+//   +P[l][+1] on the pair (0, +1).
+__global__ void __launch_bounds__(256) k_first_bwd(int C, const int* __restrict__ recv_off,
+                                                   const int* __restrict__ send, const int* __restrict__ rrow,
+                                                   const float* __restrict__ vec, const float* __restrict__ D,
+                                                   const float* __restrict__ R, const float* __restrict__ x,
+                                                   const float* __restrict__ H, float* __restrict__ gR_hi,
+                                                   float* __restrict__ gR_lo, float* __restrict__ g_r) {
+  __shared__ __align__(16) float sD[EL_CH * NDBLK];
+  __shared__ float svec[EL_CH * 3];
+  __shared__ int ss[EL_CH], sr[EL_CH];
+  __shared__ float red[EL_CH * 8 * 2];
+  const int i = blockIdx.x, c = threadIdx.x, warp = c >> 5, lane = c & 31, nw = blockDim.x >> 5;
+  const int e0 = recv_off[i], e1 = recv_off[i + 1];
+  float h[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) h[k] = H[((size_t)i * 16 + k) * C + c];
+  constexpr int P1m = jpair_of(1, -1, 0), P1p = jpair_of(1, 0, 1);
+  constexpr int P2m = jpair_of(2, -1, 0), P2p = jpair_of(2, 0, 1);
+  constexpr int P3m = jpair_of(3, -1, 0), P3p = jpair_of(3, 0, 1);
+  static_assert(P1m >= 0 && P1p >= 0 && P2m >= 0 && P2p >= 0 && P3m >= 0 && P3p >= 0, "generator pairs");
+  for (int eb = e0; eb < e1; eb += EL_CH) {
+    const int n = min(EL_CH, e1 - eb);
+    __syncthreads();
+    stage_chunk(eb, n, D, vec, send, rrow, sD, svec, ss, sr);
+    __syncthreads();
+#pragma unroll 1
+    for (int q = 0; q < n; ++q) {
+      const float* Dq = sD + q * NDBLK;
+      const float x0 = x[(size_t)ss[q] * 16 * C + c];
+      const float xt = R[(size_t)sr[q] * 4 * C + c] * x0;
+      float g0 = h[0];
+      float bx = 0.f, by = 0.f;
+#define EMP_FIRST_DEG(L, PM, PP)                                                       \
+      {                                                                                \
+        float km = 0.f, k0 = 0.f, kp = 0.f;                                            \
+        _Pragma("unroll") for (int nn = -L; nn <= L; ++nn) {                           \
+          const float hv = h[L * L + L + nn];                                          \
+          km = fmaf(Dq[dix(L, -1, nn)], hv, km);                                       \
+          k0 = fmaf(Dq[dix(L, 0, nn)], hv, k0);                                        \
+          kp = fmaf(Dq[dix(L, 1, nn)], hv, kp);                                        \
+        }                                                                              \
+        g0 += k0;                                                                      \
+        const float pm = xt * km, pp = xt * kp;                                        \
+        bx = fmaf(c_jx[PP], pp, fmaf(-c_jx[PM], pm, bx));                              \
+        by = fmaf(c_jy[PP], pp, fmaf(-c_jy[PM], pm, by));                              \
+      }
+      EMP_FIRST_DEG(1, P1m, P1p)
+      EMP_FIRST_DEG(2, P2m, P2p)
+      EMP_FIRST_DEG(3, P3m, P3p)
+#undef EMP_FIRST_DEG
+      const float gr = g0 * x0;
+      const float ghi = tf32_rna(gr);
+      gR_hi[(size_t)sr[q] * 4 * C + c] = ghi;
+      gR_lo[(size_t)sr[q] * 4 * C + c] = tf32_rna(gr - ghi);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        bx += __shfl_xor_sync(0xffffffffu, bx, o);
+        by += __shfl_xor_sync(0xffffffffu, by, o);
+      }
+      if (lane == 0) {
+        red[(q * nw + warp) * 2 + 0] = bx;
+        red[(q * nw + warp) * 2 + 1] = by;
+      }
+    }
+    __syncthreads();
+    finish_torque(n, nw, eb, red, svec, g_r);
+  }
+}
+
+// ------------------------------------------------------------------ last layer, backward
+// Per edge e of receiver i = blockIdx.x (one thread per channel), with G_i (per node):
+//   u[l][m] = sum_m' D^l[m][m'] x_send[l][m'] (m = -1, 0, 1);  gu[l] = R[l] G_i[l]
+//   dE/dR[l] = G_i[l] u[l][0]  (split hi/lo, row rr)
+//   torque: the gu^T J u term with gu at m = 0 only: -gu u[l][-1] on the pair (-1, 0),
+//   +gu u[l][+1] on the pair (0, +1)
+// and the sender sums dE/dx_send of the layer, gathered at the receiver: for the edges e'
+// whose sender is i (the mirrors (j, i, -S) of i's own edges (i, j, S)),
+//   dE/dx[i][l][m'] += sum_{e in recv(i)} (-1)^l D^l_e[0][m'] R_e[l] G_send(e)[l]
+// because the m = 0 row of D^l is a multiple of the real spherical harmonics of the edge
+// direction (Y_l(-r) = (-1)^l Y_l(r)) and the radial scale of an edge and its mirror are equal
+// (same length, unordered species pair).  One writer per node: gx[i] += that sum.
+__global__ void __launch_bounds__(256) k_last_bwd(int C, const int* __restrict__ recv_off,
+                                                  const int* __restrict__ send, const int* __restrict__ rrow,
+                                                  const float* __restrict__ vec, const float* __restrict__ D,
+                                                  const float* __restrict__ R, const float* __restrict__ x,
+                                                  const float* __restrict__ G, float* __restrict__ gR_hi,
+                                                  float* __restrict__ gR_lo, float* __restrict__ g_r,
+                                                  float* __restrict__ gx) {
+  __shared__ __align__(16) float sD[EL_CH * NDBLK];
+  __shared__ float svec[EL_CH * 3];
+  __shared__ int ss[EL_CH], sr[EL_CH];
+  __shared__ float red[EL_CH * 8 * 2];
+  const int i = blockIdx.x, c = threadIdx.x, warp = c >> 5, lane = c & 31, nw = blockDim.x >> 5;
+  const int e0 = recv_off[i], e1 = recv_off[i + 1];
+  float gi[4];
+#pragma unroll
+  for (int l = 0; l < 4; ++l) gi[l] = G[((size_t)i * 4 + l) * C + c];
+  float acc[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+  constexpr int P1m = jpair_of(1, -1, 0), P1p = jpair_of(1, 0, 1);
+  constexpr int P2m = jpair_of(2, -1, 0), P2p = jpair_of(2, 0, 1);
+  constexpr int P3m = jpair_of(3, -1, 0), P3p = jpair_of(3, 0, 1);
+  static_assert(P1m >= 0 && P1p >= 0 && P2m >= 0 && P2p >= 0 && P3m >= 0 && P3p >= 0, "generator pairs");
+  for (int eb = e0; eb < e1; eb += EL_CH) {
+    const int n = min(EL_CH, e1 - eb);
+    __syncthreads();
+    stage_chunk(eb, n, D, vec, send, rrow, sD, svec, ss, sr);
+    __syncthreads();
+#pragma unroll 1
+    for (int q = 0; q < n; ++q) {
+      const float* Dq = sD + q * NDBLK;
+      const float* xs = x + (size_t)ss[q] * 16 * C + c;
+      const float* Rr = R + (size_t)sr[q] * 4 * C + c;
+      const float* Gs = G + (size_t)ss[q] * 4 * C + c;
+      float xv[16], rl[4], gs[4];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) xv[k] = xs[k * C];
+#pragma unroll
+      for (int l = 0; l < 4; ++l) {
+        rl[l] = Rr[l * C];
+        gs[l] = Gs[l * C];
+      }
+      float gr[4];
+      float bx = 0.f, by = 0.f;
+      // degree 0: u = x[0], no torque
+      gr[0] = gi[0] * xv[0];
+      acc[0] = fmaf(rl[0], gs[0], acc[0]);
+#define EMP_LAST_DEG(L, PM, PP)                                                        \
+      {                                                                                \
+        float um = 0.f, u0 = 0.f, up = 0.f;                                            \
+        _Pragma("unroll") for (int nn = -L; nn <= L; ++nn) {                           \
+          const float xvv = xv[L * L + L + nn];                                        \
+          um = fmaf(Dq[dix(L, -1, nn)], xvv, um);                                      \
+          u0 = fmaf(Dq[dix(L, 0, nn)], xvv, u0);                                       \
+          up = fmaf(Dq[dix(L, 1, nn)], xvv, up);                                       \
+        }                                                                              \
+        gr[L] = gi[L] * u0;                                                            \
+        const float gu = rl[L] * gi[L];                                                \
+        bx = fmaf(c_jx[PP], gu * up, fmaf(-c_jx[PM], gu * um, bx));                    \
+        by = fmaf(c_jy[PP], gu * up, fmaf(-c_jy[PM], gu * um, by));                    \
+        const float ms = (L & 1 ? -1.f : 1.f) * rl[L] * gs[L];                         \
+        _Pragma("unroll") for (int nn = -L; nn <= L; ++nn)                             \
+          acc[L * L + L + nn] = fmaf(Dq[dix(L, 0, nn)], ms, acc[L * L + L + nn]);      \
+      }
+      EMP_LAST_DEG(1, P1m, P1p)
+      EMP_LAST_DEG(2, P2m, P2p)
+      EMP_LAST_DEG(3, P3m, P3p)
+#undef EMP_LAST_DEG
+      const size_t go = (size_t)sr[q] * 4 * C + c;
+#pragma unroll
+      for (int l = 0; l < 4; ++l) {
+        const float hi = tf32_rna(gr[l]);
+        gR_hi[go + l * C] = hi;
+        gR_lo[go + l * C] = tf32_rna(gr[l] - hi);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        bx += __shfl_xor_sync(0xffffffffu, bx, o);
+        by += __shfl_xor_sync(0xffffffffu, by, o);
+      }
+      if (lane == 0) {
+        red[(q * nw + warp) * 2 + 0] = bx;
+        red[(q * nw + warp) * 2 + 1] = by;
+      }
+    }
+    __syncthreads();
+    finish_torque(n, nw, eb, red, svec, g_r);
+  }
+  float* g = gx + (size_t)i * 16 * C + c;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) g[k * C] += acc[k];
+}
+
+// ------------------------------------------------------------------ per-node products (FP32)
+// out[r][n] = sum_k A(r)[k] B[n * ldb + k], k < K, n < Nn, r < rows, where row r is
+// component r % w of node r / w: A(r) = A + (r / w) a_node + (r % w) a_comp, and likewise
+// out(r) = out + (r / w) o_node + (r % w) o_comp.  64 x 64 output tiles, 256 threads, a 4 x 4
+// register tile each, K in steps of 32 staged in shared memory.  Plain FP32 fused multiply-adds
+// in ascending k.  K must be a multiple of 32.
+constexpr int NG_T = 64, NG_K = 32;
+__global__ void __launch_bounds__(256) k_node_gemm(int rows, int K, int Nn, int w, const float* __restrict__ A,
+                                                   long long a_node, int a_comp, const float* __restrict__ B,
+                                                   int ldb, float* __restrict__ out, long long o_node, int o_comp) {
+  __shared__ __align__(16) float As[NG_K][NG_T + 4];
+  __shared__ __align__(16) float Bs[NG_K][NG_T + 4];
+  const int t = threadIdx.x;
+  const int r0 = blockIdx.x * NG_T, n0 = blockIdx.y * NG_T;
+  const int tr = (t >> 4) * 4, tn = (t & 15) * 4;
+  float acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+  for (int k0 = 0; k0 < K; k0 += NG_K) {
+    __syncthreads();
+    for (int q = t; q < NG_T * NG_K; q += 256) {
+      const int rr = q / NG_K, kk = q % NG_K;
+      const int r = r0 + rr, n = n0 + rr;
+      As[kk][rr] = r < rows ? A[(long long)(r / w) * a_node + (long long)(r % w) * a_comp + k0 + kk] : 0.f;
+      Bs[kk][rr] = n < Nn ? B[(long long)n * ldb + k0 + kk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < NG_K; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(&As[kk][tr]);
+      const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][tn]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(av[p], bv[q], acc[p][q]);
+    }
+  }
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const int r = r0 + tr + p;
+    if (r >= rows) continue;
+    float* o = out + (long long)(r / w) * o_node + (long long)(r % w) * o_comp;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (n0 + tn + q < Nn) o[n0 + tn + q] = acc[p][q];
+  }
+}
+
+}  // namespace emp

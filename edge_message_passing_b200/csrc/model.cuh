@@ -34,6 +34,7 @@ struct Model {
   // radial head W3 [4C][64] of each (layer, pair) split for 3xTF32, and its transpose [64][4C]
   float *w3_hi, *w3_lo, *w3t_hi, *w3t_lo;
   std::vector<MapPair> w3_maps, w3t_maps;      // index t * n_pairs + p
+  std::vector<MapPair> w3n_maps;                // the first C rows of W3 (degree-0 scales only)
   size_t w3_stride() const { return (size_t)4 * spec.C * 64; }
 
   size_t rad_stride() const { return (size_t)H * 8 + (size_t)H * H + (size_t)4 * spec.C * H; }

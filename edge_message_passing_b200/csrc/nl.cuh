@@ -16,6 +16,7 @@ namespace emp {
 namespace nl {
 
 constexpr int MAX_CAND = 4096;       // sort buffer per receiver
+constexpr int MAX_SHIFT = 127;       // |S| per component that the sort key holds (and its mirror -S)
 constexpr int EMIT_THREADS = 512;
 
 struct Grid {
@@ -34,7 +35,7 @@ struct Ws {
   int* cell_cursor;   // [N]
   int* cell_atoms;    // [N]
   int* deg;           // [N]
-  int* flags;         // [4]: nonfinite, ...
+  int* flags;         // [4]: non-finite position, degree above MAX_CAND, shift beyond MAX_SHIFT
   long long* total;   // [1]
 };
 
@@ -139,12 +140,21 @@ __global__ void k_count(const double* __restrict__ pos, int n, Grid G, Ws w) {
   if (warp >= n) return;
   const int i = warp;
   int cnt = 0;
+  bool far = false;
   for_candidates(i, G, w, lane, 32, [&](int j, int Sx, int Sy, int Sz) {
     double rx, ry, rz;
-    if (within(pos, i, j, Sx, Sy, Sz, G, rx, ry, rz)) ++cnt;
+    if (within(pos, i, j, Sx, Sy, Sz, G, rx, ry, rz)) {
+      ++cnt;
+      far |= Sx < -MAX_SHIFT || Sx > MAX_SHIFT || Sy < -MAX_SHIFT || Sy > MAX_SHIFT || Sz < -MAX_SHIFT || Sz > MAX_SHIFT;
+    }
   });
   for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-  if (lane == 0) w.deg[i] = cnt;
+  far = __any_sync(0xffffffffu, far);
+  if (lane == 0) {
+    w.deg[i] = cnt;
+    if (cnt > MAX_CAND) atomicExch(&w.flags[1], 1);   // more edges than the per-receiver sort holds
+    if (far) atomicExch(&w.flags[2], 1);              // an image shift the edge key cannot hold
+  }
 }
 
 __device__ __forceinline__ unsigned long long edge_key(int j, int Sx, int Sy, int Sz) {

@@ -36,7 +36,9 @@ constexpr int BK = 16;                 // fp32 elements per 64-byte swizzled row
 constexpr int THREADS = 192;
 constexpr int MAXSUB = 8;
 constexpr int TMEM_COLS = 512;         // two 128 x 256 fp32 accumulators
-constexpr long long TIMEOUT_CYCLES = 4000000000ll;   // ~2 s at 1.9 GHz
+constexpr long long TIMEOUT_CYCLES = 4000000000ll;   // default bound of every mbarrier wait: ~2 s at 1.9 GHz
+// The bound in force (clock64 cycles); set by emp_set_wait_limit, read by every bounded wait.
+__device__ long long g_wait_cycles = TIMEOUT_CYCLES;
 
 constexpr int A_BYTES = BM * BK * 4;   // 8 KB
 
@@ -87,7 +89,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > TIMEOUT_CYCLES) {
+    if (clock64() - t0 > g_wait_cycles) {
       set_device_error(DEV_ERR_TIMEOUT);
       return false;
     }
@@ -191,7 +193,7 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
   const long long t0 = clock64();
   while (!mbar_try_wait_cluster(bar, parity)) {
-    if (clock64() - t0 > TIMEOUT_CYCLES) {
+    if (clock64() - t0 > g_wait_cycles) {
       set_device_error(DEV_ERR_TIMEOUT);
       return false;
     }

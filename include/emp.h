@@ -77,7 +77,8 @@ typedef struct {
   int32_t* recv_off;   /* [N+1] CSR offsets over receivers */
   int32_t* shift;      /* [capacity][3] image shift S */
   float* vec;          /* [capacity][3] r rounded to float32 */
-  int64_t n_edges;     /* number of valid edges (set by nl_build) */
+  int64_t n_edges;     /* number of valid edges (set by nl_build); with 0 edges the
+                          per-edge pointers may be NULL in the mp_* calls */
   int32_t n_atoms;     /* number of atoms N (set by nl_build) */
 } emp_graph;
 
@@ -89,7 +90,10 @@ size_t nl_workspace_bytes(int32_t n_atoms);
  * returned (two-phase use: call once with capacity 0 to size the buffers).
  * Errors: EMP_ERR_ARG (null pointers, n_atoms < 1, non-positive box or
  * cutoff), EMP_ERR_NONFINITE, EMP_ERR_CAPACITY, EMP_ERR_WORKSPACE,
- * EMP_ERR_DEVICE (more than 4096 candidate neighbours for one receiver). */
+ * EMP_ERR_DEVICE (a receiver with more than 4096 neighbours),
+ * EMP_ERR_UNSUPPORTED (an edge whose image shift has a component beyond
+ * +-127 box lengths, e.g. unwrapped positions that drifted that far apart).
+ * On these two the edge count is still reported and the graph is not written. */
 int nl_build(const emp_nl_params* p, const double* pos, emp_graph* g, int64_t* n_edges,
              void* ws, size_t ws_bytes, cudaStream_t stream);
 
@@ -102,8 +106,9 @@ int nl_build(const emp_nl_params* p, const double* pos, emp_graph* g, int64_t* n
  * every device that loads the library until the process exits).  Nothing is
  * allocated.  The subject pages have no counterpart of this entry point.
  *   - n_atoms above EMP_NL_NOALLOC_MAX_ATOMS: EMP_ERR_WORKSPACE.
- *   - The first call on a device looks up the scratch array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Each call looks up the scratch array's device address on the current
+ *     device (cudaGetSymbolAddress); make the first call on a device before
+ *     any stream capture (it loads the library's module on that device).
  *   - All calls on a device share the scratch; calls whose GPU work overlaps
  *     (unordered streams) race on it.  Each call clears what must start at zero.
  * Other arguments, results and errors as nl_build. */
@@ -203,6 +208,18 @@ int64_t emp_launch_count(void);                        /* kernels launched since
 const char* emp_status_string(int status);
 /* Reads and clears the device error word of the current device (synchronises). */
 int emp_last_device_error(void);
+
+/* ------------------------------------------------------------ bounded waits
+ * Every mbarrier wait of the library's kernels gives up after a bound (clock64
+ * cycles of the waiting SM), records EMP_ERR_TIMEOUT in the device error word,
+ * stops issuing work, waits (bounded) for its own copies in flight and returns.
+ * Sets the bound for the current device; cycles <= 0 restores the default
+ * (4e9 cycles, about 2 s).  Synchronous with respect to the host. */
+int emp_set_wait_limit(int64_t cycles);
+/* Launches one bounded wait on an mbarrier that nothing arrives on: it runs out
+ * after the bound in force, and emp_last_device_error() then reports
+ * EMP_ERR_TIMEOUT.  For checking the failure path without a fault. */
+int emp_wait_selftest(cudaStream_t stream);
 
 #ifdef __cplusplus
 }

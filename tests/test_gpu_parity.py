@@ -155,9 +155,57 @@ def _check_ef(w, cohort=None, virial=True):
     return model, g, (E, F)
 
 
+@pytest.mark.parametrize("n_layers", [2, 3])
 @pytest.mark.parametrize("cohort", [8192, 128])
-def test_energy_forces_small_gated(cohort):
-    _check_ef(synth.small_workload(ncell=1, C=32, n_layers=2, gated=True, sigma=0.1), cohort=cohort)
+def test_energy_forces_small_gated(cohort, n_layers):
+    """Two layers: the first (degree-0 input) and the last (degree-0 output) alone; three: also
+    a layer between them, run over edge cohorts (128 edges: many cohorts and a ragged tail)."""
+    _check_ef(synth.small_workload(ncell=1, C=32, n_layers=n_layers, gated=True, sigma=0.1), cohort=cohort)
+
+
+def test_energy_forces_ungated_three_layers():
+    _check_ef(synth.small_workload(ncell=1, C=32, n_layers=3, gated=False, sigma=0.1), cohort=256)
+
+
+def _cluster_workload(n_layers=3, far=True, seed=9):
+    """A small random cluster in a large periodic box, plus (far=True) one atom out of every
+    other atom's reach: a receiver (and sender) with no edges at all."""
+    rng = np.random.default_rng(seed)
+    w = synth.small_workload(ncell=1, C=32, n_layers=n_layers, gated=True, sigma=0.1)
+    pts = [rng.uniform(0.0, 4.0, 3)]
+    while len(pts) < 10:
+        p = rng.uniform(0.0, 4.0, 3)
+        if min(np.linalg.norm(p - q) for q in pts) > 1.2:
+            pts.append(p)
+    if far:
+        pts.append(np.array([15.0, 15.0, 15.0]))
+    pos = np.array(pts) + 2.0
+    st = synth.Structure(pos=pos, box=np.full(3, 30.0), species=np.zeros(len(pts), dtype=np.int32))
+    return synth.Workload(name="cluster", structure=st, spec=w.spec, weights=w.weights)
+
+
+def test_energy_forces_isolated_atom():
+    w = _cluster_workload()
+    _, g, (E, F) = _check_ef(w, cohort=128)
+    ro = g.recv_off.cpu().numpy()
+    assert ro[-1] - ro[-2] == 0                      # the far atom receives no edge
+    assert np.all(F[-1] == 0.0)
+
+
+def test_energy_forces_no_edges():
+    """E = 0: the energy is the readout of the embeddings, forces and virial vanish."""
+    st = synth.Structure(pos=np.array([[1.0, 1.0, 1.0], [15.0, 15.0, 15.0]]), box=np.full(3, 30.0),
+                         species=np.zeros(2, dtype=np.int32))
+    w0 = synth.small_workload(ncell=1, C=32, n_layers=3, gated=True, sigma=0.1)
+    w = synth.Workload(name="pair", structure=st, spec=w0.spec, weights=w0.weights)
+    g = _graph(st)
+    assert g.n_edges == 0
+    model = emp.Model(w.spec, w.weights)
+    e, f, v, ea = emp.mp_energy_forces(model, g, _cuda(st.species), virial=True, atom_energy=True)
+    ref = omodel.energy_forces(w.spec, w.weights, st.species, np.zeros(0, int), np.zeros(0, int),
+                               np.zeros((0, 3)), 2)
+    assert abs(float(e.cpu()[0]) - ref.energy) <= 1e-5 * abs(ref.energy)
+    assert np.all(f.cpu().numpy() == 0.0) and np.all(v.cpu().numpy() == 0.0)
 
 
 @pytest.mark.parametrize("C", [96, 256])
