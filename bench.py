@@ -4,14 +4,17 @@
 
 Workload: the seeded N=4096 diamond (8x8x8 conventional cells, sigma 0.02 A,
 seed 2), cutoff 6 A (E = 647168 directed edges), C = 128, lmax = 3, three gated
-residual layers, 8192-edge receiver-sorted cohorts.  One step = the whole hot
-path on one frame: neighbour list build + forward (radial, rotate, SO(2)
-mixing, rotate back, receiver sums, gates, readout) + recomputing backward +
-forces.  Metric: edges/s = E / step time (whole job: summed over replicas).
+residual layers, 8192-edge receiver-sorted cohorts.  One step = mp_energy_forces
+on the frame's resident neighbour graph: forward (radial, rotate, SO(2) mixing,
+rotate back, receiver sums, gates, readout) + recomputing backward + forces.  The
+neighbour list build is timed on its own (nl_ms) and is part of the end-to-end
+figure (e2e), not of the step.  Metric: edges/s = E / step time (whole job:
+summed over replicas).
 
-N > 1 (launched with torch.distributed.run, one rank per GPU): every rank runs
-its own replica of the frame (replicas only: weak scaling), timed between
-barriers, max over ranks.
+N > 1 (launched with torch.distributed.run, one rank per GPU; without it, with
+--gpus N > 1, this script launches itself that way): every rank runs its own
+replica of the frame (replicas only: weak scaling), timed between barriers, max
+over ranks.
 
 --impl reference times the float64 oracle (test infrastructure, CPU) on a
 bounded sample of the same workload: the edges of the first receivers.
@@ -204,40 +207,55 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------ per-kernel HBM figures
-# Algorithmic HBM bytes per edge of each SIMT kernel family (layers after the first; the
-# first layer's input is degree 0 only, so it moves the m = 0 columns alone).  Node rows
-# gathered per edge (x of the sender, gS of the receiver; 33.5 MB arrays that stay in L2)
-# are not counted: their minimal HBM traffic is one read per layer.
-def alg_bytes(name: str, C: int, first: bool) -> float:
+# Algorithmic HBM bytes per step of each kernel family, for E edges, N atoms, C channels and
+# T layers.  The first layer (degree-0 input) and the last (read through degree 0 only) run the
+# receiver-centric kernels first_fwd / first_bwd / last_fwd / last_bwd; only the T - 2 layers
+# between them run rotate_in, rotate_back_scatter, bwd_prep and bwd_edge.  Node rows gathered
+# per edge (x of the sender, gS or the per-node products of the receiver; arrays of at most
+# N*16*C floats that stay in L2) are not counted: their minimal traffic is one pass per layer.
+def alg_bytes_step(name: str, C: int, T: int, E: int, N: int) -> float:
     row = 16 * C * 4                      # one [16][C] fp32 row
-    d = 84 * 4                            # Wigner-D blocks
+    d = 84 * 4                            # Wigner-D blocks of an edge
+    d0 = 16 * 4                           # the m = 0 rows of the blocks
+    mid = max(T - 2, 0)                   # layers between the first and the last
+    last = 1 if T >= 2 else 0
     if name == "rotate_in":               # R row in; x~ hi/lo out
-        return (C * 4 + 2 * C * 4 + d) if first else (4 * C * 4 + 2 * row + d)
+        return mid * E * (4 * C * 4 + 2 * row + d)
     if name == "bwd_prep":                # R row in; x~ hi/lo and g_y hi/lo out
-        return (C * 4 + 2 * C * 4 + 2 * 4 * C * 4 + d) if first else (4 * C * 4 + 4 * row + d)
+        return mid * E * (4 * C * 4 + 4 * row + d)
     if name == "bwd_edge":                # y, g_x~, R, D in; dE/dR hi/lo out
-        return (4 * C * 4 + C * 4 + C * 4 + d + 2 * 4 * C * 4) if first else (2 * row + 4 * C * 4 + d + 2 * 4 * C * 4)
+        return mid * E * (2 * row + 4 * C * 4 + d + 2 * 4 * C * 4)
     if name == "rotate_back_scatter":     # y, D in
-        return (4 * C * 4 + d) if first else (row + d)
+        return mid * E * (row + d)
+    if name == "first_fwd":               # R[l=0], m = 0 rows of D in; Z out (per node)
+        return E * (C * 4 + d0) + N * row
+    if name == "first_bwd":               # R[l=0], D, r in; dE/dR[l=0] hi/lo out, g_r read-modify-write
+        return E * (C * 4 + d + 12 + 2 * C * 4 + 24)
+    if name == "last_fwd":                # R, m = 0 rows of D in; X out (per node)
+        return last * (E * (4 * C * 4 + d0) + N * 4 * C * 4)
+    if name == "last_bwd":                # R, D, r in; dE/dR hi/lo out, g_r and g_x read-modify-write
+        return last * (E * (4 * C * 4 + d + 12 + 2 * 4 * C * 4 + 24) + N * 2 * row)
     if name == "radial_h2":               # d in; h2 hi/lo out
-        return 4 + 2 * 64 * 4
-    if name == "radial_head":             # h2 hi/lo in; R out (tensor-core product)
-        return 2 * 64 * 4 + 4 * C * 4
-    if name == "radial_head_bwd":         # dE/dR hi/lo in; dE/dh2 out
-        return 2 * 4 * C * 4 + 64 * 4
+        return T * E * (4 + 2 * 64 * 4)
+    if name == "radial_head":             # h2 hi/lo in; R out (C columns in the first layer, 4C after)
+        return E * (2 * 64 * 4 + C * 4) + (T - 1) * E * (2 * 64 * 4 + 4 * C * 4)
+    if name == "radial_head_bwd":         # dE/dR hi/lo in (C columns in the first layer); dE/dh2 out
+        return E * (2 * C * 4 + 64 * 4) + (T - 1) * E * (2 * 4 * C * 4 + 64 * 4)
     if name == "radial_bwd":              # d, dE/dh2 in; g_r read-modify-write
-        return 4 + 64 * 4 + 2 * 12
+        return T * E * (4 + 64 * 4 + 2 * 12)
     raise KeyError(name)
 
 
-def hbm_fractions(fam, steps: int, E: int, C: int, T: int, hbm_gbs: float):
+HBM_FAMILIES = ("rotate_in", "bwd_prep", "bwd_edge", "rotate_back_scatter", "first_fwd", "first_bwd", "last_fwd",
+                "last_bwd", "radial_h2", "radial_head", "radial_head_bwd", "radial_bwd")
+
+
+def hbm_fractions(fam, steps: int, E: int, N: int, C: int, T: int, hbm_gbs: float):
     out = {}
-    for name in ("rotate_in", "bwd_prep", "bwd_edge", "rotate_back_scatter", "radial_h2", "radial_head",
-                 "radial_head_bwd", "radial_bwd"):
+    for name in HBM_FAMILIES:
         if name not in fam or fam[name][0] <= 0:
             continue
-        per_layer = [alg_bytes(name, C, t == 0) for t in range(T)]
-        bytes_step = E * sum(per_layer)
+        bytes_step = alg_bytes_step(name, C, T, E, N)
         ms = fam[name][0] / steps
         gbs = bytes_step / (ms * 1e-3) / 1e9
         out[name] = {"ms": round(ms, 3), "alg_bytes_per_step": int(bytes_step), "achieved_gbs": round(gbs, 1),
@@ -248,7 +266,7 @@ def hbm_fractions(fam, steps: int, E: int, C: int, T: int, hbm_gbs: float):
 # DRAM bytes per launch of the SO(2) mixing kernel (mean over one N=4096 step's launches), from
 # one ncu capture (see profiles/), valid only for the kernel source and launch structure it was
 # taken on (else the roofline's traffic is null).
-SO2_TRAFFIC = {"source_sha1": "1575825345b35bc4894ab2d415e6cca24264a435", "bytes_per_launch": 346.1e6}
+SO2_TRAFFIC = {"source_sha1": None, "bytes_per_launch": None}
 
 
 def so2_traffic_per_launch():
@@ -400,6 +418,22 @@ def run_ours(args):
         # the same steps again, eagerly, with CUDA events recorded around every library launch
         # (on the launching stream) for the per-kernel times and the roofline
         ptimes, fam = timed_steps(True)
+        # latency distribution of the graph-replayed step: at least 50 reps, L2 flushed between
+        lat = []
+        for _ in range(max(50, args.steps)):
+            flush.fill_(1.0)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            efg.replay()
+            b.record(stream)
+            b.synchronize()
+            lat.append(a.elapsed_time(b))
+        # the tensor pipe's TF32 rate in the products' own form, under the same conditions
+        # (a few warm-up launches, then ~0.5 s back to back: the sustained figure)
+        for _ in range(3):
+            emp.tf32_mma_rate(20000)
+        rates = [emp.tf32_mma_rate(20000) for _ in range(40)]
     # neighbour list alone (cell list + sort + mirror), same frame
     gnl = None                    # own buffers: g0's are captured by the graph
     nl_times = []
@@ -444,38 +478,40 @@ def run_ours(args):
     dom = max(fam.items(), key=lambda kv: kv[1][0])[0] if fam else None
     C = spec.C
     T = spec.n_layers
-    fl_per_edge = 2 * 72 * C * C                      # useful flops of one SO(2) mixing of one edge
     so2_launches = fam.get("so2_tc", (0, 0))[1]
     roof = None
+    tf32_rate = statistics.median(rates)             # TF32 TFLOP/s, every product counted
+    tf32_rate_first = rates[0]
     if so2_launches:
         so2_ms = fam["so2_tc"][0] / so2_launches
-        # per step: every layer mixes every edge three times (forward, backward recompute,
-        # backward transpose), in 2 launches per cohort (forward; grouped backward).  The first
-        # layer's input is the species embedding (degree 0 only): its three products reduce to
-        # the m = 0 block with C inputs (forward, recompute) or C outputs (transpose): 4C^2 each.
-        flops_step = E * 2 * C * C * (3 * 72 * (T - 1) + 3 * 4)
+        # per step: the per-edge products run in the layers between the first and the last (the end
+        # layers mix once per node, end_layers.cuh); each mixes every edge three times (forward,
+        # backward recompute, backward transpose), 2*72*C^2 useful flops each
+        flops_step = E * 2 * C * C * 3 * 72 * max(T - 2, 0)
         achieved = flops_step * len(ptimes) / (fam["so2_tc"][0] * 1e-3) / 1e12
-        # the mixing is timed inside the long step: the sustained BF16 figure is the reference
-        peak = pk["bf16_tflops_sustained"] * TF32_OVER_BF16 / 3.0
-        peak_burst = pk["bf16_tflops"] * TF32_OVER_BF16 / 3.0
+        # the reference: the measured TF32 rate of the same tcgen05 products (operands resident in
+        # shared memory, ~0.5 s back to back right after the step) / 3 for 3xTF32
+        peak = tf32_rate / 3.0
+        bf16_derived = pk["bf16_tflops_sustained"] * TF32_OVER_BF16 / 3.0
         traffic = so2_traffic_per_launch()
         roof = {"bound": "tensor", "kernel": "so2_tc (3xTF32 tcgen05 SO(2) mixing)", "achieved": achieved,
                 "flops_per_step": flops_step,
                 "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                "traffic_unit": "bytes per launch (DRAM read + write, ncu, mean of a forward and a grouped "
-                                "backward cohort launch)" if traffic else None,
+                "traffic_unit": "bytes per launch (DRAM read + write, ncu)" if traffic else None,
                 "launch_ms": so2_ms, "launches_per_step": so2_launches / len(ptimes), "dominant": dom == "so2_tc",
-                "frac_vs_burst": achieved / peak_burst,
-                "peak_note": f"useful FP32 flops of the mixings actually required (2*72*C^2 per edge per "
-                             f"mixing, 3 mixings per layer; 2*4*C^2 in the degree-0-input first layer) over the "
-                             f"summed launch event time (CUDA events on the launching stream), vs sustained "
-                             f"bf16 ({pk_kind}, the kernel runs inside a long step) x {TF32_OVER_BF16:.3f} "
-                             f"(TF32/BF16 nominal) / 3 (3xTF32); median SM clock during the step "
-                             f"{clk.summary().get('sm_mhz')} MHz"}
+                "peak_measured_tf32": tf32_rate, "peak_measured_tf32_first_launch": tf32_rate_first,
+                "peak_bf16_derived": bf16_derived, "frac_vs_bf16_derived": achieved / bf16_derived,
+                "peak_note": f"useful FP32 flops of the per-edge mixings (2*72*C^2 per edge and mixing, three "
+                             f"mixings in each of the {max(T - 2, 0)} layers between the first and the last) over "
+                             f"the summed launch event time (CUDA events on the launching stream), vs the "
+                             f"measured TF32 rate of tcgen05.mma.cta_group::2.kind::tf32 (M=N=256, K=8, "
+                             f"operands in shared memory; median of 40 launches after the step) / 3 (3xTF32); "
+                             f"bf16-derived: {pk_kind} sustained bf16 x {TF32_OVER_BF16:.3f} / 3; median SM clock "
+                             f"during the step {clk.summary().get('sm_mhz')} MHz"}
     elif dom is not None:
         roof = {"bound": "hbm", "kernel": dom, "achieved": None, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": None, "traffic": None}
-    hbm = hbm_fractions(fam, len(ptimes), E, C, T, pk["hbm_gbs"])
+    hbm = hbm_fractions(fam, len(ptimes), E, N, C, T, pk["hbm_gbs"])
     configs = other_configs(emp, torch, stream, flush, pk["hbm_gbs"]) if (ws == 1 and not args.no_configs) else None
     kernel_ms = {k: round(v[0] / len(ptimes), 3) for k, v in sorted(fam.items(), key=lambda kv: -kv[1][0])}
 
@@ -492,6 +528,7 @@ def run_ours(args):
                              "step": "mp_energy_forces on a resident neighbour graph, replayed as one CUDA graph "
                                      "of the library's launches; neighbour list timed separately (nl_ms)"},
                   "nl_ms": sum(nl_times) / len(nl_times),
+                  "p50_ms": statistics.median(lat), "p90_ms": float(np.percentile(lat, 90)), "latency_reps": len(lat),
                   "clocks": clk.summary(), "gpu_launches": launches,
                   "ms_per_step_profiled": sum(ptimes) / len(ptimes),
                   "step_ms": [round(t, 3) for t in times], "step_ms_profiled": [round(t, 3) for t in ptimes],
@@ -518,6 +555,19 @@ def main():
     ap.add_argument("--no-configs", action="store_true", help="skip the other seeded workloads")
     ap.add_argument("--clocks-dir", default=None, help="where the raw nvidia-smi samples go (default: temp dir)")
     args = ap.parse_args()
+    ws = os.environ.get("WORLD_SIZE")
+    if ws is None and args.gpus > 1:
+        # one rank per GPU: launch this script under torch.distributed.run
+        import socket
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+               "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+        return subprocess.call(cmd)
+    if ws is not None and int(ws) != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={ws}", file=sys.stderr)
+        return 2
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

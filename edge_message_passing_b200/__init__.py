@@ -23,7 +23,7 @@ SYMBOLS = (
     "mp_workspace_bytes", "mp_forward", "mp_energy_forces", "mp_so2_mix", "mp_chain_create",
     "mp_chain_destroy", "mp_radial_chain", "emp_status_string", "emp_last_device_error",
     "emp_profile_enable", "emp_profile_read", "emp_profile_names", "emp_launch_count",
-    "emp_set_wait_limit", "emp_wait_selftest",
+    "emp_set_wait_limit", "emp_wait_selftest", "emp_tf32_mma_rate",
 )
 
 
@@ -103,6 +103,8 @@ def lib() -> ctypes.CDLL:
         L.emp_set_wait_limit.argtypes = [i64]
         L.emp_wait_selftest.restype = ctypes.c_int
         L.emp_wait_selftest.argtypes = [vp]
+        L.emp_tf32_mma_rate.restype = ctypes.c_int
+        L.emp_tf32_mma_rate.argtypes = [i32, vp, ctypes.POINTER(ctypes.c_double)]
         _lib_handle = L
     return _lib_handle
 
@@ -141,6 +143,14 @@ def wait_selftest() -> int:
     """One bounded wait that nothing satisfies; returns the device error it records."""
     _check(lib().emp_wait_selftest(_stream()), "emp_wait_selftest")
     return last_device_error()
+
+
+def tf32_mma_rate(iters: int = 20000) -> float:
+    """TF32 TFLOP/s of the tensor cores in the SO(2) products' form (operands resident in
+    shared memory); a 3xTF32 product costs three."""
+    v = ctypes.c_double(0.0)
+    _check(lib().emp_tf32_mma_rate(int(iters), _stream(), ctypes.byref(v)), "emp_tf32_mma_rate")
+    return v.value
 
 
 def profile_enable(on: bool = True) -> None:

@@ -484,14 +484,13 @@ __device__ __forceinline__ void rotate16t_v(const float* __restrict__ D, const T
   }
 }
 
-// One block of C / RB_V threads (RB_V adjacent channels each) per 8-edge chunk.  y rows are
-// y_pitch floats apart (16C; 4C for a degree-0 input, whose y is non-zero only there).
+// One block of C / RB_V threads (RB_V adjacent channels each) per 8-edge chunk; y rows of 16C.
 constexpr int RB_V = 2;
 template <int V>
-__global__ void __launch_bounds__(128) k_rb_chunks(long long e0, long long e1, int C, int scalar_in,
+__global__ void __launch_bounds__(128) k_rb_chunks(long long e0, long long e1, int C,
                                                  const int* __restrict__ recv, const int* __restrict__ recv_off,
                                                  const float* __restrict__ D, const float* __restrict__ Y,
-                                                 int y_pitch, float* __restrict__ S, float* __restrict__ P) {
+                                                 float* __restrict__ S, float* __restrict__ P) {
   typedef typename VecT<V>::type T;
   __shared__ __align__(16) float sD[RB_CHUNK * NDBLK];
   __shared__ int srv[RB_CHUNK];
@@ -515,15 +514,10 @@ __global__ void __launch_bounds__(128) k_rb_chunks(long long e0, long long e1, i
     for (int k = 0; k < 16; ++k) acc[k] = vset<T>(0.f);
 #pragma unroll 1
     for (int k = 0; k < nch; ++k) {
-      const T* y = Yv + (size_t)(c0 + k) * (y_pitch / V) + t;
+      const T* y = Yv + (size_t)(c0 + k) * 16 * CV + t;
       T yv[16];
-      if (scalar_in) {
 #pragma unroll
-        for (int l = 0; l < 4; ++l) yv[l] = y[col_of(l, 0) * CV];
-      } else {
-#pragma unroll
-        for (int q = 0; q < 16; ++q) yv[q] = y[col_of_k(q) * CV];
-      }
+      for (int q = 0; q < 16; ++q) yv[q] = y[col_of_k(q) * CV];
       if (srv[k] != cur) {
         rb_flush(cur, c0, c1, e0, e1, chunk, first, recv_off, CV, t, acc, Sv, Pv);
 #pragma unroll
@@ -531,20 +525,10 @@ __global__ void __launch_bounds__(128) k_rb_chunks(long long e0, long long e1, i
         cur = srv[k];
       }
       const float* Dk = sD + k * NDBLK;
-      if (scalar_in) {
-        // y is non-zero only at m = 0: message[l][n] = D^l[0][n] y[l][0]
+      T m[16];
+      rotate16t_v(Dk, yv, m);
 #pragma unroll
-        for (int l = 0; l < 4; ++l) {
-          const float* row0 = Dk + dblk_off(l) + l * (2 * l + 1);
-#pragma unroll
-          for (int q = 0; q < 2 * l + 1; ++q) acc[l * l + q] = vfma(row0[q], yv[l], acc[l * l + q]);
-        }
-      } else {
-        T m[16];
-        rotate16t_v(Dk, yv, m);
-#pragma unroll
-        for (int q = 0; q < 16; ++q) acc[q] = vadd(acc[q], m[q]);
-      }
+      for (int q = 0; q < 16; ++q) acc[q] = vadd(acc[q], m[q]);
     }
     rb_flush(cur, c0, c1, e0, e1, chunk, first, recv_off, CV, t, acc, Sv, Pv);
   }
@@ -712,28 +696,11 @@ __device__ __forceinline__ void torque_pairs_l(const T* v, const T* w, T& bx, T&
 template <int L, typename T>
 __device__ __forceinline__ void bwd_edge_degree(const float* __restrict__ Dr, const T* __restrict__ xs,
                                                 const T* __restrict__ yrow, const T* __restrict__ gsrow,
-                                                const T* __restrict__ gxtrow, T Rl, int CV, bool need_gx,
-                                                T (&gxs)[16], T& grl, T& bx, T& by, bool scalar_in) {
+                                                const T* __restrict__ gxtrow, T Rl, int CV,
+                                                T (&gxs)[16], T& grl, T& bx, T& by) {
   constexpr int W = 2 * L + 1, O = L * L;
   const float* B = Dr + dblk_off(L);
   T v[W], u[W], gu[W];
-  if (scalar_in && L > 0) {
-    // input of degree 0 only: u, g_x~ and g_R vanish for L > 0 and y is non-zero only at m = 0,
-    // so only the y^T J g_y part of the torque remains (g_y = D gS[recv], edge frame)
-    grl = vset<T>(0.f);
-#pragma unroll
-    for (int n = 0; n < W; ++n) gu[n] = gsrow[(O + n) * CV];
-#pragma unroll
-    for (int m = 0; m < W; ++m) {
-      T a = vset<T>(0.f);
-#pragma unroll
-      for (int n = 0; n < W; ++n) a = vfma(B[m * W + n], gu[n], a);
-      u[m] = a;
-      v[m] = (m == L) ? yrow[col_of_k(O + m) * CV] : vset<T>(0.f);
-    }
-    torque_pairs_l<L>(v, u, bx, by);
-    return;
-  }
 #pragma unroll
   for (int n = 0; n < W; ++n) v[n] = xs[(O + n) * CV];
 #pragma unroll
@@ -766,24 +733,21 @@ __device__ __forceinline__ void bwd_edge_degree(const float* __restrict__ Dr, co
     for (int m = 0; m < W; ++m) v[m] = yrow[col_of_k(O + m) * CV];
     torque_pairs_l<L>(v, u, bx, by);
   }
-  if (need_gx) {
 #pragma unroll
-    for (int m = 0; m < W; ++m) {
-      T a = vset<T>(0.f);
+  for (int m = 0; m < W; ++m) {
+    T a = vset<T>(0.f);
 #pragma unroll
-      for (int n = 0; n < W; ++n) a = vfma(B[n * W + m], gu[n], a);
-      gxs[O + m] = vadd(gxs[O + m], a);
-    }
+    for (int n = 0; n < W; ++n) a = vfma(B[n * W + m], gu[n], a);
+    gxs[O + m] = vadd(gxs[O + m], a);
   }
 }
 
 // Per-edge backward over the cohort, one block of C threads (one per channel) per
-// contiguous range of `per` positions.  With need_gx the positions follow the
-// cohort's sender sort (perm), so each sender's edges are consecutive: the block
-// sums g_xs over each sender run in registers and stores the sum of each run piece
-// (a run, or the part of one that lies in the range) as row Pg[first position of the
-// piece]; k_gx_combine then adds every run's pieces to g_x[sender] in order.  Without
-// need_gx the positions are the cohort's edges in order.
+// contiguous range of `per` positions.  The positions follow the cohort's sender sort
+// (perm), so each sender's edges are consecutive: the block sums g_xs over each sender
+// run in registers and stores the sum of each run piece (a run, or the part of one that
+// lies in the range) as row Pg[first position of the piece]; k_gx_combine then adds every
+// run's pieces to g_x[sender] in order.
 // The rows an edge reads (y, g_x~, gS of the receiver, x of the sender, R and its
 // Wigner-D blocks, all contiguous) are brought into a BE_STAGES-deep shared-memory ring by bulk copies
 // (cp.async.bulk, completing on one mbarrier per stage) issued by thread 0 ahead of
@@ -823,11 +787,11 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
 
 template <int V>
 __global__ void __launch_bounds__(256, 2)
-    k_bwd_edge(long long e0, long long e1, int C, int need_gx, int scalar_in, int per,
+    k_bwd_edge(long long e0, long long e1, int C, int per,
                const int* __restrict__ send, const int* __restrict__ rrow, const float* __restrict__ vec,
                const float* __restrict__ D, const float* __restrict__ R, const float* __restrict__ x,
                const float* __restrict__ Y, const float* __restrict__ gS, const float* __restrict__ GXT,
-               int y_pitch, int gxt_pitch, const int* __restrict__ recv, const int* __restrict__ perm,
+               const int* __restrict__ recv, const int* __restrict__ perm,
                float* __restrict__ gR_hi,
                float* __restrict__ gR_lo, float* __restrict__ g_r, float* __restrict__ Pg) {
   typedef typename VecT<V>::type T;
@@ -851,7 +815,7 @@ __global__ void __launch_bounds__(256, 2)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   for (int q = t; q < np; q += CV) {
-    const int el = need_gx ? perm[e0 + p0 + q] : p0 + q;
+    const int el = perm[e0 + p0 + q];
     const long long e = e0 + el;
     meta[q] = BeMeta{el, rrow ? rrow[e] : (int)e, send[e], recv[e]};
     svec[4 * q + 0] = vec[3 * e];
@@ -860,17 +824,16 @@ __global__ void __launch_bounds__(256, 2)
   }
   __syncthreads();
   // bytes of each section that the edge's arithmetic reads
-  const uint32_t bY = scalar_in ? 16u * C : 64u * C, bG = 64u * C, bX = scalar_in ? 4u * C : 64u * C;
-  const uint32_t bR = scalar_in ? 4u * C : 16u * C;
+  const uint32_t bY = 64u * C, bG = 64u * C, bX = 64u * C, bR = 16u * C;
   auto issue = [&](int q) {
     const int s = q % BE_STAGES;
     float* st = stage0 + s * SF;
     const BeMeta m = meta[q];
     const int oR = BE_STAGE_X ? 64 * C : 48 * C;
     tc::mbar_expect_tx(&full[s], bY + bG + bX + (BE_STAGE_X ? bX : 0u) + bR + NDBLK * 4);
-    bulk_g2s(st, Y + (size_t)m.el * y_pitch, bY, &full[s]);
+    bulk_g2s(st, Y + (size_t)m.el * 16 * C, bY, &full[s]);
     bulk_g2s(st + 16 * C, gS + (size_t)m.i * 16 * C, bG, &full[s]);
-    bulk_g2s(st + 32 * C, GXT + (size_t)m.el * gxt_pitch, bX, &full[s]);
+    bulk_g2s(st + 32 * C, GXT + (size_t)m.el * 16 * C, bX, &full[s]);
     if (BE_STAGE_X) bulk_g2s(st + 48 * C, x + (size_t)m.j * 16 * C, bX, &full[s]);
     bulk_g2s(st + oR, R + (size_t)m.rr * 4 * C, bR, &full[s]);
     bulk_g2s(st + oR + 4 * C, D + (size_t)(e0 + m.el) * NDBLK, NDBLK * 4, &full[s]);
@@ -904,19 +867,19 @@ __global__ void __launch_bounds__(256, 2)
     const size_t go = (size_t)m.rr * 4 * CV + t;
     T bx = vset<T>(0.f), by = vset<T>(0.f), gr, h, l;
     const T zero = vset<T>(0.f);
-    bwd_edge_degree<0>(Dr, sX, sY, sGS, sGX, sR[0], CV, need_gx, gxs, gr, bx, by, scalar_in != 0);
+    bwd_edge_degree<0>(Dr, sX, sY, sGS, sGX, sR[0], CV, gxs, gr, bx, by);
     vsplit(gr, h, l);
     gHv[go] = h;
     gLv[go] = l;
-    bwd_edge_degree<1>(Dr, sX, sY, sGS, sGX, scalar_in ? zero : sR[CV], CV, need_gx, gxs, gr, bx, by, scalar_in != 0);
+    bwd_edge_degree<1>(Dr, sX, sY, sGS, sGX, sR[CV], CV, gxs, gr, bx, by);
     vsplit(gr, h, l);
     gHv[go + CV] = h;
     gLv[go + CV] = l;
-    bwd_edge_degree<2>(Dr, sX, sY, sGS, sGX, scalar_in ? zero : sR[2 * CV], CV, need_gx, gxs, gr, bx, by, scalar_in != 0);
+    bwd_edge_degree<2>(Dr, sX, sY, sGS, sGX, sR[2 * CV], CV, gxs, gr, bx, by);
     vsplit(gr, h, l);
     gHv[go + 2 * CV] = h;
     gLv[go + 2 * CV] = l;
-    bwd_edge_degree<3>(Dr, sX, sY, sGS, sGX, scalar_in ? zero : sR[3 * CV], CV, need_gx, gxs, gr, bx, by, scalar_in != 0);
+    bwd_edge_degree<3>(Dr, sX, sY, sGS, sGX, sR[3 * CV], CV, gxs, gr, bx, by);
     vsplit(gr, h, l);
     gHv[go + 3 * CV] = h;
     gLv[go + 3 * CV] = l;
@@ -931,7 +894,7 @@ __global__ void __launch_bounds__(256, 2)
       red[(q * 2 + 0) * nw + warp] = sx;
       red[(q * 2 + 1) * nw + warp] = sy;
     }
-    if (need_gx && (q == np - 1 || meta[q + 1].j != m.j)) {
+    if (q == np - 1 || meta[q + 1].j != m.j) {
       // end of a sender run piece: its sum becomes row Pg[first position of the piece]
       T* dst = Pgv + (size_t)(p0 + qs) * 16 * CV + t;
 #pragma unroll
@@ -1013,12 +976,9 @@ __global__ void k_gx_combine(long long e0, long long e1, int C, int cohort_idx, 
 // ------------------------------------------------------------------ staged rotate-in / backward prep
 // Rotate-in (BWD = false): XT[e - e0][col(k) C + c] = R_e[l(k)][c] (D_e x_send)[k][c] in
 // the edge frame, m-major columns, split hi/lo for the products.  Backward prep (BWD =
-// true): also GY = D_e gS[recv] (edge-frame output gradient), split.  scalar_in: x has
-// degree 0 only (the first layer's input is the species embedding), so only the (0,0)
-// column of XT is non-zero, and only the m = 0 block of GY (the m = 0 entry of each
-// degree) enters a product.  x~ and g_y rows are xt_pitch / gy_pitch floats apart (16C; for a
-// degree-0 input C and 4C, the only columns that can be non-zero).  One block of C / V threads
-// (V adjacent channels each, vector loads and stores) per contiguous range of `per` edges.  The rows
+// true): also GY = D_e gS[recv] (edge-frame output gradient), split.  x~ and g_y rows are 16C
+// floats.  One block of C / V threads (V adjacent channels each, vector loads and stores) per
+// contiguous range of `per` edges.  The rows
 // an edge reads (x of the sender, gS of the receiver, R and its Wigner-D blocks) are
 // brought into an RS_STAGES-deep shared-memory ring by bulk copies issued by thread 0
 // ahead of use.
@@ -1066,11 +1026,11 @@ __device__ __forceinline__ void rotate_write_degree_v(const float* __restrict__ 
 
 template <bool BWD, int V>
 __global__ void __launch_bounds__(256)
-    k_rotate_staged(long long e0, long long e1, int C, int scalar_in, int per, const int* __restrict__ recv,
+    k_rotate_staged(long long e0, long long e1, int C, int per, const int* __restrict__ recv,
                     const int* __restrict__ send, const int* __restrict__ rrow, const float* __restrict__ D,
                     const float* __restrict__ R, const float* __restrict__ x, const float* __restrict__ gS,
-                    float* __restrict__ XT, float* __restrict__ XTlo, int xt_pitch, float* __restrict__ GYhi,
-                    float* __restrict__ GYlo, int gy_pitch) {
+                    float* __restrict__ XT, float* __restrict__ XTlo, float* __restrict__ GYhi,
+                    float* __restrict__ GYlo) {
   typedef typename VecT<V>::type T;
   extern __shared__ __align__(128) unsigned char rs_smem[];
   const size_t SF = rs_stage_floats(C, BWD);
@@ -1092,7 +1052,7 @@ __global__ void __launch_bounds__(256)
   }
   __syncthreads();
   constexpr bool SG = BWD && RS_STAGE_G;
-  const uint32_t bX = scalar_in ? 4u * C : 64u * C, bG = SG ? 64u * C : 0u, bR = scalar_in ? 4u * C : 16u * C;
+  const uint32_t bX = 64u * C, bG = SG ? 64u * C : 0u, bR = 16u * C;
   const int offG = 16 * C, offR = (SG ? 32 : 16) * C, offD = offR + 4 * C;
   auto issue = [&](int q) {
     const int s = q % RS_STAGES;
@@ -1121,42 +1081,19 @@ __global__ void __launch_bounds__(256)
     const T* sX = reinterpret_cast<const T*>(st) + t;
     const T* sR = reinterpret_cast<const T*>(st + offR) + t;
     const float* Dr = st + offD;
-    const size_t ro = (size_t)(p0 + q) * (xt_pitch / V) + t;
-    const size_t go = (size_t)(p0 + q) * (gy_pitch / V) + t;
-    if (scalar_in) {
-      T h, l;
-      vsplit(vmul(sR[0], sX[0]), h, l);
-      XTv[ro] = h;
-      XLv[ro] = l;
-    } else {
-      rotate_write_degree_v<0>(Dr, sX, CV, sR[0], XTv + ro, XLv + ro);
-      rotate_write_degree_v<1>(Dr, sX, CV, sR[CV], XTv + ro, XLv + ro);
-      rotate_write_degree_v<2>(Dr, sX, CV, sR[2 * CV], XTv + ro, XLv + ro);
-      rotate_write_degree_v<3>(Dr, sX, CV, sR[3 * CV], XTv + ro, XLv + ro);
-    }
+    const size_t ro = (size_t)(p0 + q) * 16 * CV + t;
+    rotate_write_degree_v<0>(Dr, sX, CV, sR[0], XTv + ro, XLv + ro);
+    rotate_write_degree_v<1>(Dr, sX, CV, sR[CV], XTv + ro, XLv + ro);
+    rotate_write_degree_v<2>(Dr, sX, CV, sR[2 * CV], XTv + ro, XLv + ro);
+    rotate_write_degree_v<3>(Dr, sX, CV, sR[3 * CV], XTv + ro, XLv + ro);
     if (BWD) {
       const T* sG = SG ? reinterpret_cast<const T*>(st + offG) + t
                        : reinterpret_cast<const T*>(gS + (size_t)meta[q].y * 16 * C) + t;
       const T one = vset<T>(1.f);
-      if (!scalar_in) {
-        rotate_write_degree_v<0>(Dr, sG, CV, one, GHv + go, GLv + go);
-        rotate_write_degree_v<1>(Dr, sG, CV, one, GHv + go, GLv + go);
-        rotate_write_degree_v<2>(Dr, sG, CV, one, GHv + go, GLv + go);
-        rotate_write_degree_v<3>(Dr, sG, CV, one, GHv + go, GLv + go);
-      } else {
-        // the m = 0 entry of each degree: g_y[l][0] = sum_n D^l[0][n] gS[l][n]
-#pragma unroll
-        for (int l = 0; l < 4; ++l) {
-          const float* row0 = Dr + dblk_off(l) + l * (2 * l + 1);
-          T u = vset<T>(0.f);
-          for (int k = 0; k < 2 * l + 1; ++k) u = vfma(row0[k], sG[(l * l + k) * CV], u);
-          T h, lo;
-          vsplit(u, h, lo);
-          const int col = col_of(l, 0) * CV;
-          GHv[go + col] = h;
-          GLv[go + col] = lo;
-        }
-      }
+      rotate_write_degree_v<0>(Dr, sG, CV, one, GHv + ro, GLv + ro);
+      rotate_write_degree_v<1>(Dr, sG, CV, one, GHv + ro, GLv + ro);
+      rotate_write_degree_v<2>(Dr, sG, CV, one, GHv + ro, GLv + ro);
+      rotate_write_degree_v<3>(Dr, sG, CV, one, GHv + ro, GLv + ro);
     }
     // stage s read by every thread: free for reuse (unless a wait ran out: then stop)
     if (__syncthreads_or(!arrived)) {

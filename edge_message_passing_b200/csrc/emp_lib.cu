@@ -70,9 +70,6 @@ struct Scope {
 
 inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 
-// cohorts the first layer (degree-0 input) takes at once: its rows are a quarter as wide
-constexpr int LAYER0_COHORTS = 4;
-
 // ------------------------------------------------------------------ workspace layout
 struct WsLayout {
   size_t D, dist, R, rbP, nodeZ, nodeX, gxP, XT2, XTlo2, Y2, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
@@ -90,7 +87,7 @@ WsLayout ws_layout(const Model& m, long long E, int N) {
   L.D = take((size_t)E * NDBLK * 4);
   L.dist = take((size_t)E * 4);
   L.R = take(T * (size_t)E * 4 * C * 4);
-  L.rbP = take(((LAYER0_COHORTS * coh + RB_CHUNK - 1) / RB_CHUNK) * 2 * 16 * C * 4);
+  L.rbP = take(((coh + RB_CHUNK - 1) / RB_CHUNK) * 2 * 16 * C * 4);
   L.gRhi = take((size_t)E * 4 * C * 4);
   L.gRlo = take((size_t)E * 4 * C * 4);
   L.h2hi = take((size_t)E * 64 * 4);
@@ -171,21 +168,18 @@ void node_gemm(int rows, int K, int Nn, int w, const float* A, long long a_node,
   k_node_gemm<<<grid, 256, 0, s>>>(rows, K, Nn, w, A, a_node, a_comp, B, ldb, out, o_node, o_comp);
 }
 
-// tensor maps of a cohort buffer pair for the full cohort size and for the last (short) cohort
+// tensor maps of a cohort buffer pair (rows of 16C) for the full cohort size and for the last (short) cohort
 struct CohortMaps {
   So2AMaps full, tail;
   long long coh = 0, tail_rows = 0;
-  // rows of `cols` columns, `ld` floats apart (default: the full 16C-column rows)
-  int build(int C, long long E, long long cohort, const float* hi, const float* lo, int cols = 0, int ld = 0) {
-    if (!cols) cols = 16 * C;
-    if (!ld) ld = 16 * C;
+  int build(int C, long long E, long long cohort, const float* hi, const float* lo) {
     coh = std::min(E, cohort);
     tail_rows = E % cohort;
     if (coh > 0) {
-      int st = make_pair(&full, hi, lo, coh, cols, ld, tc::BM);
+      const int st = make_pair(&full, hi, lo, coh, 16 * C, 16 * C, tc::BM);
       if (st != EMP_OK) return st;
     }
-    if (tail_rows > 0 && tail_rows != coh) return make_pair(&tail, hi, lo, tail_rows, cols, ld, tc::BM);
+    if (tail_rows > 0 && tail_rows != coh) return make_pair(&tail, hi, lo, tail_rows, 16 * C, 16 * C, tc::BM);
     return EMP_OK;
   }
   const So2AMaps* get(long long rows) const { return rows == coh ? &full : &tail; }
@@ -254,11 +248,9 @@ Side side_for(cudaStream_t s) {
   return out;
 }
 
-// forward of layer t over all cohorts: S (raw receiver sums) from x
-// scalar_in: x has only degree-0 components (the first layer's species embedding); then only the
-// m = 0 block with its first C input columns contributes, and y is non-zero only in that block.
+// forward of layer t over all cohorts: S (raw receiver sums) from x (all degrees)
 int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, const float* D, const float* R, const int* rrow,
-                  int scalar_in, float* S, void* ws, const WsLayout& L, cudaStream_t s) {
+                  float* S, void* ws, const WsLayout& L, cudaStream_t s) {
   const int C = m.spec.C;
   const long long E = g->n_edges, coh = m.spec.cohort_edges;
   float* XT[2] = {at<float>(ws, L.XT), at<float>(ws, L.XT2)};
@@ -266,22 +258,18 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
   float* Y[2] = {at<float>(ws, L.Y), at<float>(ws, L.Y2)};
   float* P = at<float>(ws, L.rbP);
   Side side = side_for(s);
-  // A degree-0 input touches only the first C columns of x~ and the first 4C of y: their rows
-  // are stored that narrow, so that a cohort buffer holds LAYER0_COHORTS cohorts, taken at once.
-  const long long span = scalar_in ? LAYER0_COHORTS * coh : coh;
-  const int xp = scalar_in ? C : 16 * C, yp = scalar_in ? 4 * C : 16 * C;
   CohortMaps am[2];
   for (int b = 0; b < 2; ++b) {
-    const int st0 = am[b].build(C, E, span, XT[b], XTlo[b], scalar_in ? C : 0, xp);
+    const int st0 = am[b].build(C, E, coh, XT[b], XTlo[b]);
     if (st0 != EMP_OK) return st0;
   }
   int* counter = at<int>(ws, L.counter);
-  // Full-width cohorts are taken two at a time (a shorter last cohort alone): both are rotated
-  // in, then one grouped launch computes both cohorts' products (twice the tiles, so the CTA
+  // Full cohorts are taken two at a time (a shorter last cohort alone): both are rotated in,
+  // then one grouped launch computes both cohorts' products (twice the tiles, so the CTA
   // pairs stay evenly loaded), then the receiver sums run cohort by cohort, in order.
   for (long long e0 = 0; e0 < E;) {
-    const long long e1 = std::min(E, e0 + span);
-    const bool two = !scalar_in && e1 < E && std::min(E, e1 + span) - e1 == e1 - e0;
+    const long long e1 = std::min(E, e0 + coh);
+    const bool two = e1 < E && std::min(E, e1 + coh) - e1 == e1 - e0;
     const long long ee[3] = {e0, e1, two ? e1 + (e1 - e0) : e1};
     const int nc = two ? 2 : 1;
     const long long M = e1 - e0;
@@ -289,26 +277,16 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
       const int per = rs_per(M, tc::num_sms(), 6);
       Scope sc_("rotate_in", s);
       k_rotate_staged<false, RS_V_FWD><<<(unsigned)((M + per - 1) / per), C / RS_V_FWD, rs_smem_bytes(C, false), s>>>(
-          ee[b], ee[b + 1], C, scalar_in, per, g->recv, g->send, rrow, D, R, x, nullptr, XT[b], XTlo[b], xp,
-          nullptr, nullptr, 16 * C);
+          ee[b], ee[b + 1], C, per, g->recv, g->send, rrow, D, R, x, nullptr, XT[b], XTlo[b], nullptr, nullptr);
     }
-    int st;
-    if (scalar_in) {
-      const MapPair& b0 = m.bmaps_fwd[t].blk[0];
-      const So2AMaps* a = am[0].get(M);
-      GemmSub sub{&a->hi, &a->lo, &b0.hi, &b0.lo, 0, C, 4 * C, 0, Y[0]};
-      Scope sc_("so2_tc", s);
-      st = tc_group(M, yp, &sub, 1, counter, s);
-    } else {
-      So2Part parts[2] = {{am[0].get(M), &m.bmaps_fwd[t], Y[0]}, {am[1].get(M), &m.bmaps_fwd[t], Y[1]}};
-      st = so2_product(m, M, parts, nc, counter, s);
-    }
+    So2Part parts[2] = {{am[0].get(M), &m.bmaps_fwd[t], Y[0]}, {am[1].get(M), &m.bmaps_fwd[t], Y[1]}};
+    const int st = so2_product(m, M, parts, nc, counter, s);
     if (st != EMP_OK) return st;
     for (int b = 0; b < nc; ++b) {
       const long long c0 = ee[b], c1 = ee[b + 1];
       const int nchunks = (int)((c1 - c0 + RB_CHUNK - 1) / RB_CHUNK);
       side.wait();        // the previous cohort's combine: S of its last receiver, and P
-      { Scope sc_("rotate_back_scatter", s); k_rb_chunks<RB_V><<<nchunks, C / RB_V, 0, s>>>(c0, c1, C, scalar_in, g->recv, g->recv_off, D, Y[b], yp, S, P); }
+      { Scope sc_("rotate_back_scatter", s); k_rb_chunks<RB_V><<<nchunks, C / RB_V, 0, s>>>(c0, c1, C, g->recv, g->recv_off, D, Y[b], S, P); }
       side.run([&](cudaStream_t q) {
         Scope sc_("rb_combine", q);
         k_rb_combine<<<dim3((unsigned)std::min<long long>(c1 - c0, 128), 16), C, 0, q>>>(c0, c1, C, g->recv, g->recv_off, P, S);
@@ -521,6 +499,30 @@ int emp_profile_names(char* buf, size_t n) {
 int64_t emp_launch_count(void) {
   std::lock_guard<std::mutex> lk(g_prof.mu);
   return g_prof.launches;
+}
+
+int emp_tf32_mma_rate(int32_t iters, cudaStream_t stream, double* tflops) {
+  if (!tflops || iters < 1) return EMP_ERR_ARG;
+  int st = check_device();
+  if (st != EMP_OK) return st;
+  const int pairs = tc::num_sms() / 2;
+  cudaEvent_t a = nullptr, b = nullptr;
+  EMP_CUDA_TRY(cudaEventCreate(&a));
+  EMP_CUDA_TRY(cudaEventCreate(&b));
+  static unsigned seed = 1;
+  cudaEventRecord(a, stream);
+  { Scope sc_("tf32_rate", stream); tc::k_tf32_rate<<<2 * pairs, 128, tc::RATE_SMEM, stream>>>(iters, seed++); }
+  cudaEventRecord(b, stream);
+  const cudaError_t e1 = cudaEventSynchronize(b);
+  float ms = 0.f;
+  const cudaError_t e2 = cudaEventElapsedTime(&ms, a, b);
+  cudaEventDestroy(a);
+  cudaEventDestroy(b);
+  if (e1 != cudaSuccess || e2 != cudaSuccess || cudaGetLastError() != cudaSuccess) return EMP_ERR_CUDA;
+  // per round: two k-steps of three M = 256, N = 256, K = 8 products per pair
+  const double flops = (double)pairs * iters * 2 * 3 * 2.0 * 256 * 256 * 8;
+  *tflops = flops / (ms * 1e-3) / 1e12;
+  return EMP_OK;
 }
 
 int emp_set_wait_limit(int64_t cycles) {
@@ -736,13 +738,6 @@ int mp_model_create(const emp_model_spec* spec, const float* weights, size_t n_f
   }
   m->bmaps_fwd.resize(T);
   m->bmaps_bwd.resize(T);
-  m->b0_bwd_narrow.resize(T);
-  for (size_t t = 0; t < T; ++t) {
-    const size_t off = t * m->so2_stride();
-    if (make_pair(&m->b0_bwd_narrow[t], m->so2_bwd_hi + off, m->so2_bwd_lo + off, 4 * C, 4 * (int)C, 4 * (int)C,
-                  tc::b_box_rows((int)C)) != EMP_OK)
-      return fail(EMP_ERR_CUDA);
-  }
   for (size_t t = 0; t < T; ++t) {
     const size_t off = t * m->so2_stride();
     if (so2_make_bmaps(&m->bmaps_fwd[t], (int)C, m->so2_fwd_hi + off, m->so2_fwd_lo + off) != EMP_OK ||
@@ -809,7 +804,7 @@ int mp_forward(const void* model, const emp_graph* g, int32_t layer, const int32
   if (st != EMP_OK) return st;
   st = radial_forward(m, g, layer, species, dist, R, rr, ws, L, stream, 4 * C);
   if (st != EMP_OK) return st;
-  st = layer_forward(m, g, layer, x_in, D, R, rr.inv, 0, agg_out, ws, L, stream);
+  st = layer_forward(m, g, layer, x_in, D, R, rr.inv, agg_out, ws, L, stream);
   if (st != EMP_OK) return st;
   const size_t n = (size_t)N * 16 * C;
   { Scope sc_("scale", stream); k_scale<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(n, 1.0f / m.spec.avg_degree, agg_out); }
@@ -901,7 +896,7 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
         // S_i[0, c'] = sum_(l, c) W0[(0, c'), (l, c)] X_i[l, c]; the other components are not needed
         node_gemm(N, 4 * C, C, 1, nodeX, 4ll * C, 0, W0, 4 * C, S, 16ll * C, 0, stream);
       } else {
-        st = layer_forward(m, g, t, xs + (size_t)t * feat, D, R, rr.inv, 0, S, ws, L, stream);
+        st = layer_forward(m, g, t, xs + (size_t)t * feat, D, R, rr.inv, S, ws, L, stream);
         if (st != EMP_OK) return st;
       }
     }
@@ -936,7 +931,7 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
           const int per = rs_per(n, tc::num_sms(), 3);
           Scope sc_("bwd_prep", stream);
           k_rotate_staged<true, RS_V_BWD><<<(unsigned)((n + per - 1) / per), C / RS_V_BWD, rs_smem_bytes(C, true), stream>>>(
-              e0, e1, C, 0, per, g->recv, g->send, rr.inv, D, R, xt, gS, XT, XTlo, 16 * C, GYhi, GYlo, 16 * C);
+              e0, e1, C, per, g->recv, g->send, rr.inv, D, R, xt, gS, XT, XTlo, GYhi, GYlo);
         }
         So2Part parts[2] = {{am_xt.get(n), &m.bmaps_fwd[t], Y}, {am_gy.get(n), &m.bmaps_bwd[t], GXT}};
         st = so2_product(m, n, parts, 2, counter, stream);
@@ -948,8 +943,8 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
         side.wait();      // the previous cohort's combine has read Pg
         {
           Scope sc_("bwd_edge", stream);
-          k_bwd_edge<BE_V><<<nb, C / BE_V, be_smem_bytes(C), stream>>>(e0, e1, C, 1, 0, per, g->send, rr.inv, g->vec, D, R,
-                                                             xt, Y, gS, GXT, 16 * C, 16 * C, g->recv, perm, gRhi, gRlo, g_r, Pg);
+          k_bwd_edge<BE_V><<<nb, C / BE_V, be_smem_bytes(C), stream>>>(e0, e1, C, per, g->send, rr.inv, g->vec, D, R,
+                                                             xt, Y, gS, GXT, g->recv, perm, gRhi, gRlo, g_r, Pg);
         }
         side.run([&](cudaStream_t q) {
           Scope sc_("gx_combine", q);

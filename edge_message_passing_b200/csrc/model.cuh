@@ -30,7 +30,6 @@ struct Model {
   void* base;
   int device;
   std::vector<So2BMaps> bmaps_fwd, bmaps_bwd;   // tensor maps of each layer's stacked blocks
-  std::vector<MapPair> b0_bwd_narrow;           // m = 0 transposed block, tiles of C rows (degree-0 outputs only)
   // radial head W3 [4C][64] of each (layer, pair) split for 3xTF32, and its transpose [64][4C]
   float *w3_hi, *w3_lo, *w3t_hi, *w3t_lo;
   std::vector<MapPair> w3_maps, w3t_maps;      // index t * n_pairs + p

@@ -442,6 +442,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   }
 }
 
+// ------------------------------------------------------------------ tensor-pipe rate
+// The ceiling the SO(2) products are measured against: each CTA pair issues `iters` rounds of
+// the product kernel's k-stage (for each of the two 8-wide k-steps of a 16-column stage, the
+// three 3xTF32 products tcgen05.mma.cta_group::2.kind::tf32 of M = 256, N = 256, K = 8) on
+// operands resident in shared memory, into one TMEM accumulator, then commits once and waits
+// (bounded).  The operands are pseudo-random values of ordinary magnitude so that the pipe
+// switches as it does on real data.
+constexpr int RATE_COLS = 256;
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1) k_tf32_rate(int iters, unsigned seed) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint64_t* done = reinterpret_cast<uint64_t*>(smem + STAGE2);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  const int warp = threadIdx.x >> 5;
+  const uint32_t rank = cluster_rank();
+  float* f = reinterpret_cast<float*>(smem);
+  for (int i = threadIdx.x; i < STAGE2 / 4; i += blockDim.x) {
+    uint32_t h = (uint32_t)i * 2654435761u ^ (seed + 97u * rank + 7919u * blockIdx.x);
+    h ^= h >> 15;
+    h *= 2246822519u;
+    h ^= h >> 13;
+    f[i] = (float)(h & 0xffffu) * (1.0f / 32768.0f) - 1.0f;
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // operands written by threads, read by the MMAs
+  if (threadIdx.x == 0) {
+    mbar_init(done, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"((uint32_t)RATE_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  fence_before();
+  __syncthreads();
+  cluster_sync();
+  fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (rank == 0 && threadIdx.x == 0) {
+    const uint32_t a_hi = smem_u32(smem), a_lo = a_hi + A_BYTES, b_hi = a_hi + 2 * A_BYTES, b_lo = b_hi + B2_BYTES;
+    const uint32_t idesc = idesc_pair(BN);
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+      for (int kk = 0; kk < BK / 8; ++kk) {
+        const uint32_t off = kk * 32;
+        mma_tf32_pair(tmem, sdesc(a_lo + off), sdesc(b_hi + off), idesc, (it | kk) ? 1u : 0u);
+        mma_tf32_pair(tmem, sdesc(a_hi + off), sdesc(b_lo + off), idesc, 1u);
+        mma_tf32_pair(tmem, sdesc(a_hi + off), sdesc(b_hi + off), idesc, 1u);
+      }
+    }
+    mma_commit_pair(done);              // arrives on `done` in both CTAs when every MMA has completed
+  }
+  if (threadIdx.x == 0) mbar_wait(done, 0);
+  fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)RATE_COLS));
+  }
+}
+constexpr int RATE_SMEM = STAGE2 + 1024 + 64;
+
 // ------------------------------------------------------------------ host side
 inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;

@@ -7,27 +7,33 @@ import os
 import bench
 
 
-def test_alg_bytes_per_edge_follow_the_rows_each_kernel_moves():
-    C = 128
-    row, d = 16 * C * 4, 84 * 4
-    # layers after the first: full [16][C] rows
-    assert bench.alg_bytes("rotate_in", C, False) == 4 * C * 4 + 2 * row + d            # R in; x~ hi/lo out
-    assert bench.alg_bytes("bwd_prep", C, False) == 4 * C * 4 + 4 * row + d             # + g_y hi/lo out
-    assert bench.alg_bytes("bwd_edge", C, False) == 2 * row + 4 * C * 4 + d + 8 * C * 4  # y, g_x~, R, D; dE/dR hi/lo
-    assert bench.alg_bytes("rotate_back_scatter", C, False) == row + d
-    # the first layer (degree-0 input) moves only its m = 0 / l = 0 columns
+def test_alg_bytes_follow_the_rows_each_kernel_moves():
+    C, T, E, N = 128, 3, 1000, 10
+    row, d, d0 = 16 * C * 4, 84 * 4, 16 * 4
+    # the per-edge cohort kernels run only in the layers between the first and the last
+    assert bench.alg_bytes_step("rotate_in", C, T, E, N) == E * (4 * C * 4 + 2 * row + d)      # R in; x~ hi/lo out
+    assert bench.alg_bytes_step("bwd_prep", C, T, E, N) == E * (4 * C * 4 + 4 * row + d)       # + g_y hi/lo out
+    assert bench.alg_bytes_step("bwd_edge", C, T, E, N) == E * (2 * row + 4 * C * 4 + d + 8 * C * 4)
+    assert bench.alg_bytes_step("rotate_back_scatter", C, T, E, N) == E * (row + d)
     for k in ("rotate_in", "bwd_prep", "bwd_edge", "rotate_back_scatter"):
-        assert bench.alg_bytes(k, C, True) < bench.alg_bytes(k, C, False)
-    # the radial products do not depend on the layer
-    assert bench.alg_bytes("radial_head", C, True) == bench.alg_bytes("radial_head", C, False) == 2 * 64 * 4 + 4 * C * 4
+        assert bench.alg_bytes_step(k, C, 2, E, N) == 0                                        # no such layer
+        assert bench.alg_bytes_step(k, C, 5, E, N) == 3 * bench.alg_bytes_step(k, C, 3, E, N)
+    # end layers: one pass each; a single-layer model has no last-layer kernels
+    assert bench.alg_bytes_step("first_fwd", C, T, E, N) == E * (C * 4 + d0) + N * row
+    assert bench.alg_bytes_step("last_fwd", C, 1, E, N) == 0
+    assert bench.alg_bytes_step("last_bwd", C, T, E, N) == E * (4 * C * 4 + d + 12 + 8 * C * 4 + 24) + N * 2 * row
+    # the first layer's radial head writes (and its backward reads) the degree-0 columns only
+    assert bench.alg_bytes_step("radial_head", C, 1, E, N) == E * (2 * 64 * 4 + C * 4)
+    assert bench.alg_bytes_step("radial_head", C, T, E, N) == E * (2 * 64 * 4 + C * 4) + 2 * E * (2 * 64 * 4 + 4 * C * 4)
+    assert bench.alg_bytes_step("radial_h2", C, T, E, N) == 3 * E * (4 + 2 * 64 * 4)
 
 
 def test_hbm_fraction_is_bytes_over_time_over_peak():
-    C, T, E, steps = 128, 3, 1000, 4
+    C, T, E, N, steps = 128, 3, 1000, 10, 4
     fam = {"rotate_back_scatter": (steps * 2.0, 0)}          # 2 ms per step
-    out = bench.hbm_fractions(fam, steps, E, C, T, hbm_gbs=1000.0)
+    out = bench.hbm_fractions(fam, steps, E, N, C, T, hbm_gbs=1000.0)
     r = out["rotate_back_scatter"]
-    want = E * (bench.alg_bytes("rotate_back_scatter", C, True) + 2 * bench.alg_bytes("rotate_back_scatter", C, False))
+    want = bench.alg_bytes_step("rotate_back_scatter", C, T, E, N)
     assert r["alg_bytes_per_step"] == want
     assert abs(r["achieved_gbs"] - want / 2e-3 / 1e9) < 0.1
     assert abs(r["frac_of_hbm"] - r["achieved_gbs"] / 1000.0) < 1e-3
