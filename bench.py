@@ -263,23 +263,43 @@ def hbm_fractions(fam, steps: int, E: int, N: int, C: int, T: int, hbm_gbs: floa
     return out
 
 
-# DRAM bytes per launch of the SO(2) mixing kernel (mean over one N=4096 step's launches), from
-# one ncu capture (see profiles/), valid only for the kernel source and launch structure it was
-# taken on (else the roofline's traffic is null).
-SO2_TRAFFIC = {"source_sha1": None, "bytes_per_launch": None}
+# DRAM bytes per launch of the SO(2) mixing kernel (mean over one N=4096 step's 119 launches: 39
+# forward launches of two cohorts, one of a single cohort, 79 backward cohort launches), from ncu
+# captures of the N=512 step's forward pair and backward cohort launches, which have the same
+# shapes (profiles/kernels_n512_step.md).  Valid only for the kernel source and the launch
+# structure it was taken on: so2_tc.cuh and the marked per-edge product launch code of emp_lib.cu
+# must hash to source_sha1, else the roofline's traffic is null.
+SO2_TRAFFIC = {"source_sha1": "86fa8e78eeab526ddde159654fc26bb6a322ea3f", "bytes_per_launch": 389.6e6}
+
+
+def so2_source_hash():
+    import hashlib
+    csrc = os.path.join(ROOT, "edge_message_passing_b200", "csrc")
+    h = hashlib.sha1()
+    so2 = os.path.join(csrc, "so2_tc.cuh")
+    lib = os.path.join(csrc, "emp_lib.cu")
+    if not (os.path.exists(so2) and os.path.exists(lib)):
+        return None
+    h.update(open(so2, "rb").read())
+    text = open(lib).read()
+    begin, end = "// [per-edge product launches: begin]", "// [per-edge product launches: end]"
+    pos = 0
+    while True:
+        a = text.find(begin, pos)
+        if a < 0:
+            break
+        b = text.find(end, a)
+        if b < 0:
+            return None
+        h.update(text[a:b].encode())
+        pos = b + len(end)
+    return h.hexdigest()
 
 
 def so2_traffic_per_launch():
     # the kernel and the launch structure (which cohorts each launch covers) must both be
     # those the counters were taken on
-    import hashlib
-    h = hashlib.sha1()
-    for f in ("so2_tc.cuh", "emp_lib.cu"):
-        src = os.path.join(ROOT, "edge_message_passing_b200", "csrc", f)
-        if not os.path.exists(src):
-            return None
-        h.update(open(src, "rb").read())
-    ok = SO2_TRAFFIC["source_sha1"] and h.hexdigest() == SO2_TRAFFIC["source_sha1"]
+    ok = SO2_TRAFFIC["source_sha1"] and so2_source_hash() == SO2_TRAFFIC["source_sha1"]
     return SO2_TRAFFIC["bytes_per_launch"] if ok else None
 
 

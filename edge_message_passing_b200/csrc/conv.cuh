@@ -68,24 +68,6 @@ __device__ __forceinline__ float hsum(float2 a) { return a.x + a.y; }
 __device__ __forceinline__ float vdot(float a, float b, float c) { return fmaf(a, b, c); }
 __device__ __forceinline__ float2 vdot(float2 a, float2 b, float2 c) { return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y)); }
 
-// ------------------------------------------------------------------ geometry
-// D(R_e) (84 floats) and d = |r_e| from the float32 edge vector.
-__global__ void k_geometry(long long E, const float* __restrict__ vec, float* __restrict__ D, float* __restrict__ dist) {
-  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= E) return;
-  const float vx = vec[3 * e], vy = vec[3 * e + 1], vz = vec[3 * e + 2];
-  const float d = sqrtf(vx * vx + vy * vy + vz * vz);
-  const float inv = 1.0f / d;
-  float R[3][3];
-  edge_frame<float>(vx * inv, vy * inv, vz * inv, R);
-  float Dl[NDBLK];
-  wigner_blocks<float>(R, Dl);
-  float* out = D + (size_t)e * NDBLK;
-#pragma unroll
-  for (int k = 0; k < NDBLK; ++k) out[k] = Dl[k];
-  dist[e] = d;
-}
-
 // ------------------------------------------------------------------ radial part
 // e_n(d) = u(d/rc) sin(n pi d / rc) / d, u(x) = 1 - 28 x^6 + 48 x^7 - 21 x^8 for x < 1,
 // and its derivative in d (one basis function: every (row, n) pair is its own work item).
@@ -590,39 +572,6 @@ __global__ void k_update(int N, int C, float inv_avg, int gated, float* __restri
   } else {
 #pragma unroll
     for (int k = 0; k < 16; ++k) x_next[((size_t)i * 16 + k) * C + c] = a[k];
-  }
-}
-
-// e_i = w_o . SiLU(W_ro h_i[0]); g_h = dE/dh (degree 0 only; other components zero)
-__global__ void k_readout(int N, int C, int Hro, const float* __restrict__ h, const float* __restrict__ ro_W,
-                          const float* __restrict__ ro_w, float* __restrict__ e_atom, float* __restrict__ g_h) {
-  __shared__ float sh[256];
-  __shared__ float gz[256];
-  __shared__ float part[256];
-  const int i = blockIdx.x, t = threadIdx.x;
-  if (t < C) sh[t] = h[(size_t)i * 16 * C + t];
-  __syncthreads();
-  float ep = 0.f;
-  if (t < Hro) {
-    float z = 0.f;
-    for (int c = 0; c < C; ++c) z = fmaf(ro_W[(size_t)t * C + c], sh[c], z);
-    ep = ro_w[t] * silu_f(z);
-    gz[t] = ro_w[t] * dsilu_f(z);
-  }
-  part[t] = ep;
-  __syncthreads();
-  for (int s = 128; s > 0; s >>= 1) {
-    if (t < s) part[t] += part[t + s];
-    __syncthreads();
-  }
-  if (t == 0) e_atom[i] = part[0];
-  if (g_h) {
-    for (int c = t; c < C; c += blockDim.x) {
-      float g = 0.f;
-      for (int k = 0; k < Hro; ++k) g = fmaf(ro_W[(size_t)k * C + c], gz[k], g);
-      g_h[(size_t)i * 16 * C + c] = g;
-      for (int k = 1; k < 16; ++k) g_h[((size_t)i * 16 + k) * C + c] = 0.f;
-    }
   }
 }
 

@@ -72,7 +72,7 @@ inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 
 // ------------------------------------------------------------------ workspace layout
 struct WsLayout {
-  size_t D, dist, R, rbP, nodeZ, nodeX, gxP, XT2, XTlo2, Y2, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
+  size_t D, dist, R, rbP, nodeZ, nodeX, zro, gxP, XT2, XTlo2, Y2, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
   size_t total;
 };
 
@@ -86,7 +86,9 @@ WsLayout ws_layout(const Model& m, long long E, int N) {
   auto take = [&](size_t bytes) { size_t r = o; o = align_up(o + bytes); return r; };
   L.D = take((size_t)E * NDBLK * 4);
   L.dist = take((size_t)E * 4);
-  L.R = take(T * (size_t)E * 4 * C * 4);
+  // radial scales kept for the backward: the first layer's degree-0 columns (rows of C), then
+  // rows of 4C for every later layer (a single layer of mp_forward takes rows of 4C at the start)
+  L.R = take(std::max((size_t)E * C + (T - 1) * (size_t)E * 4 * C, (size_t)E * 4 * C) * 4);
   L.rbP = take(((coh + RB_CHUNK - 1) / RB_CHUNK) * 2 * 16 * C * 4);
   L.gRhi = take((size_t)E * 4 * C * 4);
   L.gRlo = take((size_t)E * 4 * C * 4);
@@ -104,6 +106,7 @@ WsLayout ws_layout(const Model& m, long long E, int N) {
   L.gS = take(feat);
   L.nodeZ = take(feat);
   L.nodeX = take((size_t)N * 4 * C * 4);
+  L.zro = take((size_t)N * std::max(m.Hro, 1) * 4);
   L.e_atom = take((size_t)N * 4);
   const size_t cb = coh * 16 * C * 4;
   L.gxP = take(cb);
@@ -159,14 +162,25 @@ int so2_product(const Model& m, long long M, const So2Part* parts, int nparts, i
   return so2_tc(M, m.spec.C, parts, nparts, counter, s);
 }
 
-// per-node FP32 product (end_layers.cuh: k_node_gemm)
-void node_gemm(int rows, int K, int Nn, int w, const float* A, long long a_node, int a_comp, const float* B, int ldb,
-               float* out, long long o_node, int o_comp, cudaStream_t s) {
-  if (rows <= 0) return;
-  const dim3 grid((unsigned)((rows + NG_T - 1) / NG_T), (unsigned)((Nn + NG_T - 1) / NG_T));
-  Scope sc_("node_gemm", s);
-  k_node_gemm<<<grid, 256, 0, s>>>(rows, K, Nn, w, A, a_node, a_comp, B, ldb, out, o_node, o_comp);
-}
+// per-node FP32 products (end_layers.cuh: k_node_gemm), up to NG_MAX in one launch
+struct NodeProducts {
+  NodeGemm p{};
+  int max_rows = 0;
+  NodeProducts(int K, int Nn) { p.K = K; p.Nn = Nn; }
+  void add(int rows, int w, const float* A, long long a_node, int a_comp, const float* B, int ldb, float* out,
+           long long o_node, int o_comp) {
+    const int z = p.n++;
+    p.rows[z] = rows; p.w[z] = w; p.A[z] = A; p.a_node[z] = a_node; p.a_comp[z] = a_comp;
+    p.B[z] = B; p.ldb[z] = ldb; p.out[z] = out; p.o_node[z] = o_node; p.o_comp[z] = o_comp;
+    max_rows = std::max(max_rows, rows);
+  }
+  void launch(cudaStream_t s, const char* name = "node_gemm") {
+    if (p.n == 0 || max_rows <= 0) return;
+    const dim3 grid((unsigned)((max_rows + NG_T - 1) / NG_T), (unsigned)((p.Nn + NG_T - 1) / NG_T), (unsigned)p.n);
+    Scope sc_(name, s);
+    k_node_gemm<<<grid, 256, 0, s>>>(p);
+  }
+};
 
 // tensor maps of a cohort buffer pair (rows of 16C) for the full cohort size and for the last (short) cohort
 struct CohortMaps {
@@ -248,6 +262,7 @@ Side side_for(cudaStream_t s) {
   return out;
 }
 
+// [per-edge product launches: begin] (bench.py ties the mixing's DRAM traffic figure to this text)
 // forward of layer t over all cohorts: S (raw receiver sums) from x (all degrees)
 int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, const float* D, const float* R, const int* rrow,
                   float* S, void* ws, const WsLayout& L, cudaStream_t s) {
@@ -297,6 +312,7 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
   side.wait();
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
+// [per-edge product launches: end]
 
 // Rows of the radial network: edge order for one radial network, pair-sorted for
 // per-pair networks (stable counting sort; the host reads the pair offsets once).
@@ -327,7 +343,8 @@ int radial_rows(const Model& m, const emp_graph* g, const int* species, void* ws
 }
 
 // R rows [E][4C] of layer t: hidden layers on SIMT, head R = h2 W3^T on the tensor cores
-// ncols: 4C, or C when only the degree-0 scales are used (the first layer: degree-0 input)
+// ncols: 4C, or C when only the degree-0 scales are used (the first layer: degree-0 input);
+// R rows are ncols floats apart
 int radial_forward(const Model& m, const emp_graph* g, int t, const int* species, const float* dist, float* R,
                    const RadialRows& rr, void* ws, const WsLayout& L, cudaStream_t s, int ncols) {
   const long long E = g->n_edges;
@@ -343,9 +360,9 @@ int radial_forward(const Model& m, const emp_graph* g, int t, const int* species
     int st = make_pair(&a, h2hi + r0 * 64, h2lo + r0 * 64, n, 64, 64, tc::BM);
     if (st != EMP_OK) return st;
     const MapPair& b = (ncols == C ? m.w3n_maps : m.w3_maps)[(size_t)t * m.n_pairs + p];
-    GemmSub sub{&a.hi, &a.lo, &b.hi, &b.lo, 0, 64, ncols, 0, R + r0 * 4 * C};
+    GemmSub sub{&a.hi, &a.lo, &b.hi, &b.lo, 0, 64, ncols, 0, R + r0 * ncols};
     Scope sc_("radial_head", s);
-    st = tc_group(n, 4 * C, &sub, 1, at<int>(ws, L.counter), s);
+    st = tc_group(n, ncols, &sub, 1, at<int>(ws, L.counter), s);
     if (st != EMP_OK) return st;
   }
   return EMP_OK;
@@ -664,7 +681,7 @@ int mp_model_create(const emp_model_spec* spec, const float* weights, size_t n_f
   const size_t n_emb = S * C, n_rad = T * m->n_pairs * m->rad_stride(), n_so2 = T * m->so2_stride();
   const size_t n_ro = (size_t)m->Hro * C + m->Hro;
   const size_t n_w3 = T * m->n_pairs * (size_t)4 * C * 64;
-  const size_t total = n_emb + n_rad + 6 * n_so2 + 4 * n_w3 + n_ro + n_floats;   // + raw staging
+  const size_t total = n_emb + n_rad + 6 * n_so2 + 4 * n_w3 + n_ro + (size_t)m->Hro * C + n_floats;   // + raw staging
   float* base = nullptr;
   if (cudaMalloc(&base, total * 4) != cudaSuccess) { delete m; return EMP_ERR_CUDA; }
   m->base = base;
@@ -682,7 +699,8 @@ int mp_model_create(const emp_model_spec* spec, const float* weights, size_t n_f
   m->w3t_lo = m->w3t_hi + n_w3;
   m->ro_W = m->w3t_lo + n_w3;
   m->ro_w = m->ro_W + (size_t)m->Hro * C;
-  float* raw = m->ro_w + m->Hro;
+  m->ro_WT = m->ro_w + m->Hro;
+  float* raw = m->ro_WT + (size_t)m->Hro * C;
   auto fail = [&](int code) { cudaFree(base); delete m; return code; };
   if (cudaMemcpy(raw, weights, n_floats * 4, cudaMemcpyHostToDevice) != cudaSuccess) return fail(EMP_ERR_CUDA);
   // walk the blob in declaration order
@@ -713,6 +731,7 @@ int mp_model_create(const emp_model_spec* spec, const float* weights, size_t n_f
   if (cudaMemcpy(m->ro_W, raw + o, n_ro * 4, cudaMemcpyDeviceToDevice) != cudaSuccess) return fail(EMP_ERR_CUDA);
   o += n_ro;
   if (o != n_floats) return fail(EMP_ERR_ARG);
+  k_transpose<<<(int)((m->Hro * C + 255) / 256), 256>>>(m->ro_W, m->ro_WT, m->Hro, (int)C);
   k_split_tf32<<<256, 256>>>(m->so2_fwd, m->so2_fwd_hi, m->so2_fwd_lo, n_so2);
   k_split_tf32<<<256, 256>>>(m->so2_bwd, m->so2_bwd_hi, m->so2_bwd_lo, n_so2);
   // radial heads: W3 split, and W3^T split (input gradient dE/dh2 = dE/dR W3)
@@ -798,7 +817,7 @@ int mp_forward(const void* model, const emp_graph* g, int32_t layer, const int32
   float* D = at<float>(ws, L.D);
   float* dist = at<float>(ws, L.dist);
   float* R = at<float>(ws, L.R);
-  { Scope sc_("geometry", stream); k_geometry<<<(unsigned)((E + 127) / 128), 128, 0, stream>>>(E, g->vec, D, dist); }
+  { Scope sc_("geometry", stream); k_geometry_staged<<<(unsigned)((E + GEO_EPB - 1) / GEO_EPB), GEO_EPB, 0, stream>>>(E, g->vec, D, dist); }
   RadialRows rr;
   st = radial_rows(m, g, species, ws, L, rr, stream);
   if (st != EMP_OK) return st;
@@ -857,7 +876,7 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
   EMP_CUDA_TRY(cudaMemsetAsync(aggs, 0, (size_t)T * feat * 4, stream));
   { Scope sc_("embed", stream); k_embed<<<(unsigned)((feat + 255) / 256), 256, 0, stream>>>(N, C, species, m.spec.n_species, m.emb, xs); }
   if (E > 0) {
-    { Scope sc_("geometry", stream); k_geometry<<<(unsigned)((E + 127) / 128), 128, 0, stream>>>(E, g->vec, D, dist); }
+    { Scope sc_("geometry", stream); k_geometry_staged<<<(unsigned)((E + GEO_EPB - 1) / GEO_EPB), GEO_EPB, 0, stream>>>(E, g->vec, D, dist); }
     if (T > 2) {      // sender order of the cohorts, for the backward of the layers between the first and the last
       const int ncoh = (int)((E + coh - 1) / coh);
       int P = 1;
@@ -878,7 +897,7 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
   const unsigned nb_node = (unsigned)N;
   // ---------------- forward
   for (int t = 0; t < T; ++t) {
-    float* R = Rall + (size_t)t * E * 4 * C;
+    float* R = Rall + (t == 0 ? 0 : (size_t)E * C + (size_t)(t - 1) * E * 4 * C);
     float* S = aggs + (size_t)t * feat;
     const float* W0 = m.so2_fwd + (size_t)t * m.so2_stride();
     const bool first = t == 0, last = t == T - 1;
@@ -887,14 +906,18 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
       if (st != EMP_OK) return st;
       if (first) {
         { Scope sc_("first_fwd", stream); k_first_fwd<<<nb_node, C, 0, stream>>>(C, g->recv_off, g->send, rr.inv, D, R, xs, nodeZ); }
-        // S_i[l, m', c'] = sum_c W0[(l, c'), (0, c)] Z_i[l, m', c], one launch per degree
+        // S_i[l, m', c'] = sum_c W0[(l, c'), (0, c)] Z_i[l, m', c], one product per degree
+        NodeProducts np(C, C);
         for (int l = 0; l < 4; ++l)
-          node_gemm(N * (2 * l + 1), C, C, 2 * l + 1, nodeZ + l * l * C, 16ll * C, C, W0 + (size_t)l * C * 4 * C,
-                    4 * C, S + l * l * C, 16ll * C, C, stream);
+          np.add(N * (2 * l + 1), 2 * l + 1, nodeZ + l * l * C, 16ll * C, C, W0 + (size_t)l * C * 4 * C, 4 * C,
+                 S + l * l * C, 16ll * C, C);
+        np.launch(stream);
       } else if (last) {
         { Scope sc_("last_fwd", stream); k_last_fwd<<<nb_node, C, 0, stream>>>(C, g->recv_off, g->send, rr.inv, D, R, xs + (size_t)t * feat, nodeX); }
         // S_i[0, c'] = sum_(l, c) W0[(0, c'), (l, c)] X_i[l, c]; the other components are not needed
-        node_gemm(N, 4 * C, C, 1, nodeX, 4ll * C, 0, W0, 4 * C, S, 16ll * C, 0, stream);
+        NodeProducts np(4 * C, C);
+        np.add(N, 1, nodeX, 4ll * C, 0, W0, 4 * C, S, 16ll * C, 0);
+        np.launch(stream);
       } else {
         st = layer_forward(m, g, t, xs + (size_t)t * feat, D, R, rr.inv, S, ws, L, stream);
         if (st != EMP_OK) return st;
@@ -903,11 +926,23 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
     { Scope sc_("update", stream); k_update<<<(unsigned)((N * C + 255) / 256), 256, 0, stream>>>(N, C, inv_avg, m.spec.gated, S,
                                                                    xs + (size_t)t * feat, xs + (size_t)(t + 1) * feat); }
   }
-  { Scope sc_("readout", stream); k_readout<<<N, 256, 0, stream>>>(N, C, m.Hro, xs + (size_t)T * feat, m.ro_W, m.ro_w, e_atom, gxa); }
+  {
+    // e_i = w_o . SiLU(W_ro h_i[0]) and dE/dh_i (degree 0 only): two per-node products around
+    // the activation
+    float* zro = at<float>(ws, L.zro);
+    NodeProducts z(C, m.Hro);
+    z.add(N, 1, xs + (size_t)T * feat, 16ll * C, 0, m.ro_W, C, zro, m.Hro, 0);
+    z.launch(stream, "readout");
+    { Scope sc_("readout", stream); k_readout_act<<<(unsigned)((N * 32 + 255) / 256), 256, 0, stream>>>(N, m.Hro, m.ro_w, zro, e_atom); }
+    EMP_CUDA_TRY(cudaMemsetAsync(gxa, 0, feat * 4, stream));
+    NodeProducts gh(m.Hro, C);
+    gh.add(N, 1, zro, m.Hro, 0, m.ro_WT, m.Hro, gxa, 16ll * C, 0);
+    gh.launch(stream, "readout");
+  }
   { Scope sc_("energy_sum", stream); k_energy_sum<<<1, 1024, 0, stream>>>(N, e_atom, energy); }
   // ---------------- backward, one layer at a time in reverse
   for (int t = T - 1; t >= 0; --t) {
-    const float* R = Rall + (size_t)t * E * 4 * C;
+    const float* R = Rall + (t == 0 ? 0 : (size_t)E * C + (size_t)(t - 1) * E * 4 * C);
     const float* xt = xs + (size_t)t * feat;
     const float* Wb = m.so2_bwd + (size_t)t * m.so2_stride();
     const bool first = t == 0, last = t == T - 1;
@@ -915,15 +950,20 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
                                                                      aggs + (size_t)t * feat, gxa, gS, gxb); }
     if (E > 0 && first) {
       // H_i[l, m', c] = sum_c' W0[(l, c'), (0, c)] gS_i[l, m', c']
+      NodeProducts np(C, C);
       for (int l = 0; l < 4; ++l)
-        node_gemm(N * (2 * l + 1), C, C, 2 * l + 1, gS + l * l * C, 16ll * C, C, Wb + (size_t)l * C, 4 * C,
-                  nodeZ + l * l * C, 16ll * C, C, stream);
+        np.add(N * (2 * l + 1), 2 * l + 1, gS + l * l * C, 16ll * C, C, Wb + (size_t)l * C, 4 * C, nodeZ + l * l * C,
+               16ll * C, C);
+      np.launch(stream);
       { Scope sc_("first_bwd", stream); k_first_bwd<<<nb_node, C, 0, stream>>>(C, g->recv_off, g->send, rr.inv, g->vec, D, R, xt, nodeZ, gRhi, gRlo, g_r); }
     } else if (E > 0 && last) {
       // the output gradient is degree 0 only: G_i[l, c] = sum_c' W0[(0, c'), (l, c)] gS_i[0, c']
-      node_gemm(N, C, 4 * C, 1, gS, 16ll * C, 0, Wb, 4 * C, nodeX, 4ll * C, 0, stream);
+      NodeProducts np(C, 4 * C);
+      np.add(N, 1, gS, 16ll * C, 0, Wb, 4 * C, nodeX, 4ll * C, 0);
+      np.launch(stream);
       { Scope sc_("last_bwd", stream); k_last_bwd<<<nb_node, C, 0, stream>>>(C, g->recv_off, g->send, rr.inv, g->vec, D, R, xt, nodeX, gRhi, gRlo, g_r, gxb); }
     } else if (E > 0) {
+      // [per-edge product launches: begin]
       int ci = 0;
       for (long long e0 = 0; e0 < E; e0 += coh, ++ci) {
         const long long e1 = std::min(E, e0 + coh), n = e1 - e0;
@@ -953,6 +993,7 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
         });
       }
       side.wait();        // g_x of this layer complete
+      // [per-edge product launches: end]
     }
     if (E > 0) {
       st = radial_backward(m, g, t, species, dist, rr, g_r, ws, L, stream, first ? C : 4 * C);

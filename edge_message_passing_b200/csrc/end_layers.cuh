@@ -48,7 +48,8 @@ __host__ __device__ constexpr int jpair_of(int l, int am, int bm, int p = 0) {
 constexpr int EL_CH = 16;   // edges staged per chunk
 
 // ------------------------------------------------------------------ first layer, forward
-// Z[i][k][c] for the receiver i = blockIdx.x; one thread per channel (blockDim.x = C).
+// Z[i][k][c] for the receiver i = blockIdx.x; one thread per channel (blockDim.x = C).  R holds the
+// first layer's degree-0 scales only: rows of C floats.
 __global__ void __launch_bounds__(256) k_first_fwd(int C, const int* __restrict__ recv_off,
                                                    const int* __restrict__ send, const int* __restrict__ rrow,
                                                    const float* __restrict__ D, const float* __restrict__ R,
@@ -74,7 +75,7 @@ __global__ void __launch_bounds__(256) k_first_fwd(int C, const int* __restrict_
     __syncthreads();
 #pragma unroll 4
     for (int q = 0; q < n; ++q) {
-      const float v = R[(size_t)sr[q] * 4 * C + c] * x[(size_t)ss[q] * 16 * C + c];
+      const float v = R[(size_t)sr[q] * C + c] * x[(size_t)ss[q] * 16 * C + c];
 #pragma unroll
       for (int k = 0; k < 16; ++k) acc[k] = fmaf(sd[q][k], v, acc[k]);
     }
@@ -168,7 +169,8 @@ __device__ __forceinline__ void stage_chunk(int eb, int n, const float* __restri
 }
 
 // ------------------------------------------------------------------ first layer, backward
-// Per edge of receiver i = blockIdx.x (one thread per channel): with H_i (per-node, see the
+// Per edge of receiver i = blockIdx.x (one thread per channel; R rows of C floats, the degree-0
+// scales; dE/dR rows of 4C floats, of which the first C are written): with H_i (per-node, see the
 // top of this file), K[l][m] = sum_m' D^l[m][m'] H_i[l][m'] for m = -1, 0, 1:
 //   dE/dx~[0,0] = sum_l K[l][0];  dE/dR[0] = dE/dx~[0,0] x_send[0]  (split hi/lo, row rr)
 //   torque: the y^T J g_y term with y = W0 x~ (m = 0 only): per degree l, the channel sums
@@ -202,7 +204,7 @@ __global__ void __launch_bounds__(256) k_first_bwd(int C, const int* __restrict_
     for (int q = 0; q < n; ++q) {
       const float* Dq = sD + q * NDBLK;
       const float x0 = x[(size_t)ss[q] * 16 * C + c];
-      const float xt = R[(size_t)sr[q] * 4 * C + c] * x0;
+      const float xt = R[(size_t)sr[q] * C + c] * x0;
       float g0 = h[0];
       float bx = 0.f, by = 0.f;
 #define EMP_FIRST_DEG(L, PM, PP)                                                       \
@@ -348,19 +350,34 @@ __global__ void __launch_bounds__(256) k_last_bwd(int C, const int* __restrict__
 }
 
 // ------------------------------------------------------------------ per-node products (FP32)
-// out[r][n] = sum_k A(r)[k] B[n * ldb + k], k < K, n < Nn, r < rows, where row r is
-// component r % w of node r / w: A(r) = A + (r / w) a_node + (r % w) a_comp, and likewise
-// out(r) = out + (r / w) o_node + (r % w) o_comp.  64 x 64 output tiles, 256 threads, a 4 x 4
-// register tile each, K in steps of 32 staged in shared memory.  Plain FP32 fused multiply-adds
-// in ascending k.  K must be a multiple of 32.
-constexpr int NG_T = 64, NG_K = 32;
-__global__ void __launch_bounds__(256) k_node_gemm(int rows, int K, int Nn, int w, const float* __restrict__ A,
-                                                   long long a_node, int a_comp, const float* __restrict__ B,
-                                                   int ldb, float* __restrict__ out, long long o_node, int o_comp) {
+// Up to four products per launch (blockIdx.z): out[r][n] = sum_k A(r)[k] B[n * ldb + k] for
+// k < K, n < Nn, r < rows, where row r is component r % w of node r / w:
+// A(r) = A + (r / w) a_node + (r % w) a_comp, and likewise out(r) = out + (r / w) o_node + (r % w) o_comp.
+// 64 x 64 output tiles, 256 threads, a 4 x 4 register tile each, K in steps of 32 staged in
+// shared memory.  Plain FP32 fused multiply-adds in ascending k.
+constexpr int NG_T = 64, NG_K = 32, NG_MAX = 4;
+struct NodeGemm {
+  int n, K, Nn;
+  int rows[NG_MAX], w[NG_MAX];
+  const float* A[NG_MAX];
+  long long a_node[NG_MAX];
+  int a_comp[NG_MAX];
+  const float* B[NG_MAX];
+  int ldb[NG_MAX];
+  float* out[NG_MAX];
+  long long o_node[NG_MAX];
+  int o_comp[NG_MAX];
+};
+__global__ void __launch_bounds__(256) k_node_gemm(const __grid_constant__ NodeGemm p) {
   __shared__ __align__(16) float As[NG_K][NG_T + 4];
   __shared__ __align__(16) float Bs[NG_K][NG_T + 4];
-  const int t = threadIdx.x;
+  const int z = blockIdx.z;
+  const int rows = p.rows[z], w = p.w[z], K = p.K, Nn = p.Nn;
   const int r0 = blockIdx.x * NG_T, n0 = blockIdx.y * NG_T;
+  if (r0 >= rows) return;
+  const float* __restrict__ A = p.A[z];
+  const float* __restrict__ B = p.B[z];
+  const int t = threadIdx.x;
   const int tr = (t >> 4) * 4, tn = (t & 15) * 4;
   float acc[4][4];
 #pragma unroll
@@ -371,9 +388,9 @@ __global__ void __launch_bounds__(256) k_node_gemm(int rows, int K, int Nn, int 
     __syncthreads();
     for (int q = t; q < NG_T * NG_K; q += 256) {
       const int rr = q / NG_K, kk = q % NG_K;
-      const int r = r0 + rr, n = n0 + rr;
-      As[kk][rr] = r < rows ? A[(long long)(r / w) * a_node + (long long)(r % w) * a_comp + k0 + kk] : 0.f;
-      Bs[kk][rr] = n < Nn ? B[(long long)n * ldb + k0 + kk] : 0.f;
+      const int r = r0 + rr, n = n0 + rr, k = k0 + kk;
+      As[kk][rr] = (r < rows && k < K) ? A[(long long)(r / w) * p.a_node[z] + (long long)(r % w) * p.a_comp[z] + k] : 0.f;
+      Bs[kk][rr] = (n < Nn && k < K) ? B[(long long)n * p.ldb[z] + k] : 0.f;
     }
     __syncthreads();
 #pragma unroll 8
@@ -382,20 +399,69 @@ __global__ void __launch_bounds__(256) k_node_gemm(int rows, int K, int Nn, int 
       const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][tn]);
       const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-      for (int p = 0; p < 4; ++p)
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(av[p], bv[q], acc[p][q]);
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
   }
 #pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    const int r = r0 + tr + p;
+  for (int i = 0; i < 4; ++i) {
+    const int r = r0 + tr + i;
     if (r >= rows) continue;
-    float* o = out + (long long)(r / w) * o_node + (long long)(r % w) * o_comp;
+    float* o = p.out[z] + (long long)(r / w) * p.o_node[z] + (long long)(r % w) * p.o_comp[z];
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (n0 + tn + q < Nn) o[n0 + tn + q] = acc[p][q];
+    for (int j = 0; j < 4; ++j)
+      if (n0 + tn + j < Nn) o[n0 + tn + j] = acc[i][j];
   }
+}
+
+// ------------------------------------------------------------------ readout activation
+// Given z[i][t] = (W_ro h_i[0])_t (a per-node product): e_i = sum_t w_o[t] SiLU(z_it) (one warp per
+// atom, lanes over t in order, then a fixed xor tree) and, in place, z_it <- w_o[t] SiLU'(z_it) =
+// dE/dz (the next per-node product turns it into dE/dh_i[0] = (dE/dz) W_ro).
+__global__ void k_readout_act(int N, int H, const float* __restrict__ w_o, float* __restrict__ z,
+                              float* __restrict__ e_atom) {
+  const int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (i >= N) return;
+  float* zi = z + (size_t)i * H;
+  float e = 0.f;
+  for (int t = lane; t < H; t += 32) {
+    const float v = zi[t], wt = w_o[t];
+    e = fmaf(wt, silu_f(v), e);
+    zi[t] = wt * dsilu_f(v);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+  if (lane == 0) e_atom[i] = e;
+}
+
+// ------------------------------------------------------------------ edge geometry
+// D(R_e) (84 floats) and d = |r_e| from the float32 edge vector; GEO_EPB edges per block of as
+// many threads, the Wigner-D rows staged in shared memory so that the block stores them as
+// contiguous float4 runs.
+constexpr int GEO_EPB = 64;
+__global__ void __launch_bounds__(GEO_EPB) k_geometry_staged(long long E, const float* __restrict__ vec,
+                                                             float* __restrict__ D, float* __restrict__ dist) {
+  __shared__ __align__(16) float sD[GEO_EPB * NDBLK];
+  const long long e0 = (long long)blockIdx.x * GEO_EPB;
+  const long long e = e0 + threadIdx.x;
+  if (e < E) {
+    const float vx = vec[3 * e], vy = vec[3 * e + 1], vz = vec[3 * e + 2];
+    const float d = sqrtf(vx * vx + vy * vy + vz * vz);
+    const float inv = 1.0f / d;
+    float R[3][3];
+    edge_frame<float>(vx * inv, vy * inv, vz * inv, R);
+    float Dl[NDBLK];
+    wigner_blocks<float>(R, Dl);
+#pragma unroll
+    for (int k = 0; k < NDBLK; ++k) sD[threadIdx.x * NDBLK + k] = Dl[k];
+    dist[e] = d;
+  }
+  __syncthreads();
+  const int n = (int)min((long long)GEO_EPB, E - e0);
+  float4* dst = reinterpret_cast<float4*>(D + e0 * NDBLK);
+  const float4* src = reinterpret_cast<const float4*>(sD);
+  for (int q = threadIdx.x; q < n * (NDBLK / 4); q += GEO_EPB) dst[q] = src[q];
 }
 
 }  // namespace emp

@@ -27,6 +27,7 @@ struct Model {
   float* so2_bwd_lo;
   float* ro_W;                  // [Hro][C]
   float* ro_w;                  // [Hro]
+  float* ro_WT;                 // [C][Hro]
   void* base;
   int device;
   std::vector<So2BMaps> bmaps_fwd, bmaps_bwd;   // tensor maps of each layer's stacked blocks

@@ -7,6 +7,8 @@ while the device footprint stays at a few GB):
   so2      one 8192-row cohort of the SO(2) mixing (C = 128), forward map
   so2t     the same, transpose (adjoint) map
   step512  one energy + force step of the N=512 diamond model (C = 128, 3 layers)
+  step4096 one energy + force step of the N=4096 diamond model (the benchmark workload;
+           for one-pass launch lists only: its workspace is several GB)
   chain    the folded radial chain at E = 647170, forward + input gradient
 """
 from __future__ import annotations
@@ -27,7 +29,7 @@ def main() -> int:
     import synth
 
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["so2", "so2t", "step512", "chain"])
+    ap.add_argument("case", choices=["so2", "so2t", "step512", "step4096", "chain"])
     ap.add_argument("--iters", type=int, default=3)
     a = ap.parse_args()
     torch.cuda.set_device(0)
@@ -37,8 +39,8 @@ def main() -> int:
         X = torch.randn((8192, 16 * 128), device="cuda")
         for _ in range(a.iters):
             emp.mp_so2_mix(model, 0, X, transpose=a.case == "so2t")
-    elif a.case == "step512":
-        w = synth.workload("n512_diamond")
+    elif a.case in ("step512", "step4096"):
+        w = synth.workload("n512_diamond" if a.case == "step512" else "n4096_diamond")
         model = emp.Model(w.spec, w.weights)
         g = emp.nl_build(torch.from_numpy(w.structure.pos).cuda(), w.structure.box, w.spec.cutoff)
         sp = torch.from_numpy(w.structure.species).cuda()

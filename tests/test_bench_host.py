@@ -1,7 +1,6 @@
 """Host-side arithmetic of bench.py's measurement: the algorithmic bytes behind the
 per-kernel HBM fractions, the fractions themselves, and the rule that the mixing's
 DRAM traffic is reported only for the sources it was captured on.  No GPU."""
-import hashlib
 import os
 
 import bench
@@ -41,12 +40,21 @@ def test_hbm_fraction_is_bytes_over_time_over_peak():
 
 
 def test_traffic_is_reported_only_for_the_captured_sources(monkeypatch):
-    h = hashlib.sha1()
-    for f in ("so2_tc.cuh", "emp_lib.cu"):
-        h.update(open(os.path.join(bench.ROOT, "edge_message_passing_b200", "csrc", f), "rb").read())
-    monkeypatch.setattr(bench, "SO2_TRAFFIC", {"source_sha1": h.hexdigest(), "bytes_per_launch": 123.0})
+    h = bench.so2_source_hash()
+    assert h is not None
+    monkeypatch.setattr(bench, "SO2_TRAFFIC", {"source_sha1": h, "bytes_per_launch": 123.0})
     assert bench.so2_traffic_per_launch() == 123.0
     monkeypatch.setattr(bench, "SO2_TRAFFIC", {"source_sha1": "0" * 40, "bytes_per_launch": 123.0})
     assert bench.so2_traffic_per_launch() is None
     monkeypatch.setattr(bench, "SO2_TRAFFIC", {"source_sha1": None, "bytes_per_launch": None})
     assert bench.so2_traffic_per_launch() is None
+
+
+def test_traffic_hash_covers_the_kernel_and_the_marked_launch_code():
+    """Edits outside the marked launch code of emp_lib.cu leave the hash alone; edits inside it or
+    in so2_tc.cuh change it."""
+    import hashlib
+    csrc = os.path.join(bench.ROOT, "edge_message_passing_b200", "csrc")
+    text = open(os.path.join(csrc, "emp_lib.cu")).read()
+    assert text.count("// [per-edge product launches: begin]") == 2
+    assert text.count("// [per-edge product launches: end]") == 2
