@@ -23,7 +23,7 @@ SYMBOLS = (
     "mp_workspace_bytes", "mp_forward", "mp_energy_forces", "mp_so2_mix", "mp_chain_create",
     "mp_chain_destroy", "mp_radial_chain", "emp_status_string", "emp_last_device_error",
     "emp_profile_enable", "emp_profile_read", "emp_profile_names", "emp_launch_count",
-    "emp_set_wait_limit", "emp_wait_selftest", "emp_tf32_mma_rate",
+    "emp_set_wait_limit", "emp_wait_selftest", "emp_tf32_mma_rate", "mp_model_radial_tables", "mp_radial_hidden",
 )
 
 
@@ -103,6 +103,10 @@ def lib() -> ctypes.CDLL:
         L.emp_set_wait_limit.argtypes = [i64]
         L.emp_wait_selftest.restype = ctypes.c_int
         L.emp_wait_selftest.argtypes = [vp]
+        L.mp_model_radial_tables.restype = ctypes.c_int
+        L.mp_model_radial_tables.argtypes = [vp, ctypes.c_double, ctypes.POINTER(i32)]
+        L.mp_radial_hidden.restype = ctypes.c_int
+        L.mp_radial_hidden.argtypes = [vp, i32, i32, i64, vp, vp, vp, vp, vp, vp, sz, vp]
         L.emp_tf32_mma_rate.restype = ctypes.c_int
         L.emp_tf32_mma_rate.argtypes = [i32, vp, ctypes.POINTER(ctypes.c_double)]
         _lib_handle = L
@@ -291,6 +295,13 @@ class Model:
     def workspace_bytes(self, n_edges: int, n_atoms: int) -> int:
         return lib().mp_workspace_bytes(self.handle, n_edges, n_atoms)
 
+    def radial_tables(self, tol: float = 1e-7) -> int:
+        """Switch the radial hidden layers to certified Chebyshev tables (tol > 0; returns
+        the number of pieces) or back to the network (tol <= 0)."""
+        n = ctypes.c_int32(0)
+        _check(lib().mp_model_radial_tables(self.handle, float(tol), ctypes.byref(n)), "mp_model_radial_tables")
+        return n.value
+
     def __del__(self):
         if getattr(self, "handle", None) and _lib_handle is not None:
             _lib_handle.mp_model_destroy(self.handle)
@@ -366,6 +377,22 @@ class EnergyForcesGraph:
     def replay(self):
         self.cuda_graph.replay()
         return self.energy, self.forces, self.virial, self.atom_energy
+
+
+def mp_radial_hidden(model: Model, layer: int, pair: int, d, g_h2=None):
+    """Radial network `pair` of `layer` at lengths d [n] (CUDA float32), in the model's current
+    mode: (h2 hi [n,64], h2 lo [n,64], dE/dd [n] for dE/dh2 = g_h2, or None)."""
+    torch = _torch()
+    d = d.contiguous()
+    n = d.shape[0]
+    hi = torch.empty((n, 64), dtype=torch.float32, device="cuda")
+    lo = torch.empty_like(hi)
+    dEdd = torch.empty(n, dtype=torch.float32, device="cuda") if g_h2 is not None else None
+    g = None if g_h2 is None else g_h2.contiguous()
+    ws = _workspace(24 * n + 256)
+    _check(lib().mp_radial_hidden(model.handle, layer, pair, n, _ptr(d), _ptr(hi), _ptr(lo), _ptr(g), _ptr(dEdd),
+                                  _ptr(ws), ws.numel(), _stream()), "mp_radial_hidden")
+    return hi, lo, dEdd
 
 
 def mp_so2_mix(model: Model, layer: int, X, transpose: bool = False):

@@ -15,6 +15,7 @@
 #include "chain.cuh"
 #include "chain_tc.cuh"
 #include "end_layers.cuh"
+#include "tables.cuh"
 
 using namespace emp;
 
@@ -135,6 +136,20 @@ T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws)
 bool graph_ok(const emp_graph* g) {
   return g && g->recv_off && g->n_edges >= 0 && g->n_edges < (1ll << 31) &&
          (g->n_edges == 0 || (g->recv && g->send && g->mirror && g->vec));
+}
+
+tab::Args table_args(const Model& m, int t, int fixed_pair = -1) {
+  tab::Args a;
+  a.hdr = m.tab_hdr;
+  a.map = m.tab_map;
+  a.pieces = m.tab_pieces;
+  a.layer = t;
+  a.n_pairs = m.n_pairs;
+  a.n_species = m.spec.n_species;
+  a.pair_radial = m.spec.pair_radial;
+  a.fixed_pair = fixed_pair;
+  a.rc = m.spec.cutoff;
+  return a;
 }
 
 RadialArgs radial_args(const Model& m, int t) {
@@ -351,8 +366,15 @@ int radial_forward(const Model& m, const emp_graph* g, int t, const int* species
   const int C = m.spec.C;
   float* h2hi = at<float>(ws, L.h2hi);
   float* h2lo = at<float>(ws, L.h2lo);
-  { Scope sc_("radial_h2", s); k_radial_h2<<<(unsigned)std::min<long long>((E + RT - 1) / RT, 3 * tc::num_sms()), RAD_THREADS, sizeof(RadialSmem), s>>>(
-        E, rr.perm, dist, g->recv, g->send, species, radial_args(m, t), h2hi, h2lo); }
+  if (m.tab_on) {
+    Scope sc_("radial_h2", s);
+    tab::k_radial_h2_table<<<(unsigned)std::min<long long>((E + 15) / 16, 16 * tc::num_sms()), tab::TAB_THREADS, 0, s>>>(
+        E, rr.perm, dist, g->recv, g->send, species, table_args(m, t), h2hi, h2lo);
+  } else {
+    Scope sc_("radial_h2", s);
+    k_radial_h2<<<(unsigned)std::min<long long>((E + RT - 1) / RT, 3 * tc::num_sms()), RAD_THREADS, sizeof(RadialSmem), s>>>(
+        E, rr.perm, dist, g->recv, g->send, species, radial_args(m, t), h2hi, h2lo);
+  }
   for (int p = 0; p < m.n_pairs; ++p) {
     const long long r0 = rr.off[p], n = rr.off[p + 1] - r0;
     if (n <= 0) continue;
@@ -390,8 +412,15 @@ int radial_backward(const Model& m, const emp_graph* g, int t, const int* specie
     st = tc_group(n, 64, &sub, 1, at<int>(ws, L.counter), s);
     if (st != EMP_OK) return st;
   }
-  { Scope sc_("radial_bwd", s); k_radial_bwd<<<(unsigned)std::min<long long>((E + RT - 1) / RT, 2 * tc::num_sms()), RAD_THREADS, sizeof(RadialSmem), s>>>(
-        E, rr.perm, dist, g->vec, g->recv, g->send, species, radial_args(m, t), gh2, g_r); }
+  if (m.tab_on) {
+    Scope sc_("radial_bwd", s);
+    tab::k_radial_bwd_table<<<(unsigned)std::min<long long>((E + 15) / 16, 16 * tc::num_sms()), tab::TAB_THREADS, 0, s>>>(
+        E, rr.perm, dist, g->vec, g->recv, g->send, species, table_args(m, t), gh2, g_r);
+  } else {
+    Scope sc_("radial_bwd", s);
+    k_radial_bwd<<<(unsigned)std::min<long long>((E + RT - 1) / RT, 2 * tc::num_sms()), RAD_THREADS, sizeof(RadialSmem), s>>>(
+        E, rr.perm, dist, g->vec, g->recv, g->send, species, radial_args(m, t), gh2, g_r);
+  }
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
 
@@ -425,6 +454,19 @@ __global__ void k_wait_selftest() {
   }
   __syncthreads();
   if (threadIdx.x == 0) tc::mbar_wait(&bar, 0);
+}
+
+// (d, 0, 0): an edge vector of length d along x, and the x component of g_r back
+__global__ void k_length_vec(long long n, const float* __restrict__ d, float* __restrict__ vec) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  vec[3 * i] = d[i];
+  vec[3 * i + 1] = 0.f;
+  vec[3 * i + 2] = 0.f;
+}
+__global__ void k_take_x(long long n, const float* __restrict__ g_r, float* __restrict__ out) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = g_r[3 * i];
 }
 
 int check_device() {
@@ -712,6 +754,7 @@ int mp_model_create(const emp_model_spec* spec, const float* weights, size_t n_f
     const size_t rad_t = m->n_pairs * m->rad_stride();
     if (cudaMemcpy(m->rad + t * rad_t, raw + o, rad_t * 4, cudaMemcpyDeviceToDevice) != cudaSuccess)
       return fail(EMP_ERR_CUDA);
+    m->rad_host.insert(m->rad_host.end(), weights + o, weights + o + rad_t);
     o += rad_t;
     const float* W0 = raw + o;
     o += 16 * C * C;
@@ -790,8 +833,115 @@ int mp_model_create(const emp_model_spec* spec, const float* weights, size_t n_f
 void mp_model_destroy(void* model) {
   if (!model) return;
   Model* m = static_cast<Model*>(model);
+  if (m->tab_base) cudaFree(m->tab_base);
   cudaFree(m->base);
   delete m;
+}
+
+int mp_model_radial_tables(void* model, double tol, int32_t* n_pieces) {
+  if (!model) return EMP_ERR_ARG;
+  Model* m = static_cast<Model*>(model);
+  if (m->tab_base) {
+    cudaFree(m->tab_base);
+    m->tab_base = nullptr;
+  }
+  m->tab_on = false;
+  m->tab_hdr = m->tab_map = nullptr;
+  m->tab_pieces = nullptr;
+  if (n_pieces) *n_pieces = 0;
+  if (!(tol > 0.0)) return EMP_OK;                  // tables off: the radial network itself
+  if (!(tol >= 1e-12) || m->spec.radial_hidden != tab::H) return EMP_ERR_ARG;
+  int st = check_device();
+  if (st != EMP_OK) return st;
+  const int T = m->spec.n_layers, P = m->n_pairs;
+  std::vector<int> hdr(4 * (size_t)T * P), map;
+  std::vector<float> pieces;
+  for (int t = 0; t < T; ++t)
+    for (int p = 0; p < P; ++p) {
+      const float* W1 = m->rad_host.data() + ((size_t)t * P + p) * m->rad_stride();
+      const std::vector<tab::HostPiece> tb = tab::build(W1, W1 + 64 * 8, (double)m->spec.cutoff, tol);
+      int L = 0;
+      for (const auto& q : tb) L = std::max(L, q.level);
+      const int q = t * P + p;
+      hdr[4 * q + 0] = L;
+      hdr[4 * q + 1] = (int)(pieces.size() / tab::PIECE_FLOATS);
+      hdr[4 * q + 2] = (int)map.size();
+      hdr[4 * q + 3] = (int)tb.size();
+      // every bin of the finest level lies inside exactly one (dyadic) piece
+      const int nbin = 1 << L;
+      size_t k = 0;
+      for (int b = 0; b < nbin; ++b) {
+        const double c = ((double)b + 0.5) * m->spec.cutoff / nbin;
+        while (k + 1 < tb.size() && c >= tb[k].b) ++k;
+        map.push_back((int)k);
+      }
+      for (const auto& pc : tb) {
+        pieces.push_back((float)pc.a);
+        pieces.push_back((float)(2.0 / (pc.b - pc.a)));
+        pieces.push_back(0.f);
+        pieces.push_back(0.f);
+        for (double v : pc.c) pieces.push_back((float)v);
+        for (double v : pc.dc) pieces.push_back((float)v);
+      }
+    }
+  const size_t bh = align_up(hdr.size() * 4), bm = align_up(map.size() * 4), bp = pieces.size() * 4;
+  char* base = nullptr;
+  if (cudaMalloc(&base, bh + bm + bp) != cudaSuccess) return EMP_ERR_CUDA;
+  if (cudaMemcpy(base, hdr.data(), hdr.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(base + bh, map.data(), map.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(base + bh + bm, pieces.data(), bp, cudaMemcpyHostToDevice) != cudaSuccess) {
+    cudaFree(base);
+    return EMP_ERR_CUDA;
+  }
+  m->tab_base = base;
+  m->tab_hdr = reinterpret_cast<int*>(base);
+  m->tab_map = reinterpret_cast<int*>(base + bh);
+  m->tab_pieces = reinterpret_cast<float*>(base + bh + bm);
+  m->tab_on = true;
+  if (n_pieces) *n_pieces = (int32_t)(pieces.size() / tab::PIECE_FLOATS);
+  return EMP_OK;
+}
+
+int mp_radial_hidden(const void* model, int32_t layer, int32_t pair, int64_t n, const float* d, float* h2_hi,
+                     float* h2_lo, const float* g_h2, float* dE_dd, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!model || n < 0 || (n > 0 && (!d || !h2_hi || !h2_lo))) return EMP_ERR_ARG;
+  const Model& m = *static_cast<const Model*>(model);
+  if (layer < 0 || layer >= m.spec.n_layers || pair < 0 || pair >= m.n_pairs) return EMP_ERR_ARG;
+  if (g_h2 && (!dE_dd || !ws)) return EMP_ERR_ARG;
+  if (n >= (1ll << 31)) return EMP_ERR_ARG;
+  if (g_h2 && ws_bytes < (size_t)n * 24 + 256) return EMP_ERR_WORKSPACE;
+  if (n == 0) return EMP_OK;
+  int st = check_device();
+  if (st != EMP_OK) return st;
+  RadialArgs ra = radial_args(m, layer);
+  ra.pair_radial = 0;
+  ra.layer_off += (size_t)pair * ra.pair_stride;
+  if (m.tab_on) {
+    Scope sc_("radial_h2", stream);
+    tab::k_radial_h2_table<<<(unsigned)std::min<long long>((n + 15) / 16, 16 * tc::num_sms()), tab::TAB_THREADS, 0, stream>>>(
+        n, nullptr, d, nullptr, nullptr, nullptr, table_args(m, layer, pair), h2_hi, h2_lo);
+  } else {
+    Scope sc_("radial_h2", stream);
+    k_radial_h2<<<(unsigned)std::min<long long>((n + RT - 1) / RT, 3 * tc::num_sms()), RAD_THREADS, sizeof(RadialSmem), stream>>>(
+        n, nullptr, d, nullptr, nullptr, nullptr, ra, h2_hi, h2_lo);
+  }
+  if (g_h2) {
+    float* vec = static_cast<float*>(ws);
+    float* g_r = vec + 3 * n;
+    { Scope sc_("radial_aux", stream); k_length_vec<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(n, d, vec); }
+    EMP_CUDA_TRY(cudaMemsetAsync(g_r, 0, (size_t)n * 12, stream));
+    if (m.tab_on) {
+      Scope sc_("radial_bwd", stream);
+      tab::k_radial_bwd_table<<<(unsigned)std::min<long long>((n + 15) / 16, 16 * tc::num_sms()), tab::TAB_THREADS, 0, stream>>>(
+          n, nullptr, d, vec, nullptr, nullptr, nullptr, table_args(m, layer, pair), g_h2, g_r);
+    } else {
+      Scope sc_("radial_bwd", stream);
+      k_radial_bwd<<<(unsigned)std::min<long long>((n + RT - 1) / RT, 2 * tc::num_sms()), RAD_THREADS, sizeof(RadialSmem), stream>>>(
+          n, nullptr, d, vec, nullptr, nullptr, nullptr, ra, g_h2, g_r);
+    }
+    { Scope sc_("radial_aux", stream); k_take_x<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(n, g_r, dE_dd); }
+  }
+  return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
 
 size_t mp_workspace_bytes(const void* model, int64_t n_edges, int32_t n_atoms) {

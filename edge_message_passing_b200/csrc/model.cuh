@@ -36,6 +36,14 @@ struct Model {
   std::vector<MapPair> w3_maps, w3t_maps;      // index t * n_pairs + p
   std::vector<MapPair> w3n_maps;                // the first C rows of W3 (degree-0 scales only)
   size_t w3_stride() const { return (size_t)4 * spec.C * 64; }
+  // host copy of the radial weights (W1, W2, W3 per layer and pair), for building radial tables
+  std::vector<float> rad_host;
+  // certified radial tables (tables.cuh), when enabled: one device allocation
+  void* tab_base = nullptr;
+  int* tab_hdr = nullptr;
+  int* tab_map = nullptr;
+  float* tab_pieces = nullptr;
+  bool tab_on = false;
 
   size_t rad_stride() const { return (size_t)H * 8 + (size_t)H * H + (size_t)4 * spec.C * H; }
   const float* W1(int t, int p) const { return rad + ((size_t)t * n_pairs + p) * rad_stride(); }

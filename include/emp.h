@@ -148,6 +148,27 @@ int mp_model_create(const emp_model_spec* spec, const float* weights /*(host)*/,
                     void** model);
 void mp_model_destroy(void* model);
 
+/* Certified radial tables (opt-in approximation; page FastMACE, "Rewrite screens:
+ * adopted and rejected", OPT6-T04 / OPT6-T05 radial tables).  With tol > 0, builds for
+ * every layer and radial network, in double precision on the host, a piecewise Chebyshev
+ * table of degree 10 of the network's hidden output h2(d) (64 values) on dyadic pieces of
+ * [0, cutoff], bisected until every value and length derivative is within tol of its local
+ * scale (its largest magnitude on the piece, at least 1e-3 of its largest magnitude on
+ * [0, cutoff]); from then on mp_forward and mp_energy_forces evaluate h2 and its length
+ * derivative from the tables (float32, on the device) instead of the network's hidden
+ * layers; the head W3 stays a product.  tol <= 0 frees the tables and goes back to the
+ * network.  The model owns the tables.  n_pieces (host, out, may be NULL): pieces over all
+ * tables.  Synchronous.  Errors: EMP_ERR_ARG (no model, 0 < tol < 1e-12), EMP_ERR_CUDA. */
+int mp_model_radial_tables(void* model, double tol, int32_t* n_pieces);
+
+/* The radial network p of `layer` on its own, in the model's current mode (network or
+ * tables): for n lengths d [n], h2 [n][64] as its 3xTF32 split (h2_hi + h2_lo, the head's
+ * operand), and, if g_h2 [n][64] is not NULL, dE_dd [n] = sum_j g_h2[j] dh2_j/dd.
+ * Workspace >= 24 n + 256 bytes when g_h2 is given.  For inspecting the radial part
+ * (e.g. the certificate of the tables); the energy and force calls do not need it. */
+int mp_radial_hidden(const void* model, int32_t layer, int32_t pair, int64_t n, const float* d, float* h2_hi,
+                     float* h2_lo, const float* g_h2, float* dE_dd, void* ws, size_t ws_bytes, cudaStream_t stream);
+
 /* Workspace bytes mp_forward / mp_energy_forces need. */
 size_t mp_workspace_bytes(const void* model, int64_t n_edges, int32_t n_atoms);
 
