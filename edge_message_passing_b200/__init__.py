@@ -24,6 +24,7 @@ SYMBOLS = (
     "mp_chain_destroy", "mp_radial_chain", "emp_status_string", "emp_last_device_error",
     "emp_profile_enable", "emp_profile_read", "emp_profile_names", "emp_launch_count",
     "emp_set_wait_limit", "emp_wait_selftest", "emp_tf32_mma_rate", "mp_model_radial_tables", "mp_radial_hidden",
+    "mp_weight_grad_workspace_bytes", "mp_energy_weight_grad",
 )
 
 
@@ -103,6 +104,10 @@ def lib() -> ctypes.CDLL:
         L.emp_set_wait_limit.argtypes = [i64]
         L.emp_wait_selftest.restype = ctypes.c_int
         L.emp_wait_selftest.argtypes = [vp]
+        L.mp_weight_grad_workspace_bytes.restype = sz
+        L.mp_weight_grad_workspace_bytes.argtypes = [vp, i64, i32]
+        L.mp_energy_weight_grad.restype = ctypes.c_int
+        L.mp_energy_weight_grad.argtypes = [vp, ctypes.POINTER(GraphC), vp, vp, vp, vp, vp, sz, vp]
         L.mp_model_radial_tables.restype = ctypes.c_int
         L.mp_model_radial_tables.argtypes = [vp, ctypes.c_double, ctypes.POINTER(i32)]
         L.mp_radial_hidden.restype = ctypes.c_int
@@ -284,6 +289,7 @@ class Model:
         sc = spec_c(spec)
         blob = np.concatenate([np.ascontiguousarray(weights[k], dtype=np.float32).ravel()
                                for k in weight_order(spec)])
+        self.shapes = [(k, tuple(np.shape(weights[k]))) for k in weight_order(spec)]
         n = lib().mp_weight_count(ctypes.byref(sc))
         if n != blob.size:
             raise EmpError(f"weight blob has {blob.size} floats, the library expects {n}")
@@ -333,6 +339,28 @@ def mp_energy_forces(model: Model, graph: Graph, species, virial: bool = False, 
     _check(lib().mp_energy_forces(model.handle, ctypes.byref(gc), _ptr(species), _ptr(energy), _ptr(forces),
                                   _ptr(vir), _ptr(ea), _ptr(ws), ws.numel(), _stream()), "mp_energy_forces")
     return energy, forces, vir, ea
+
+
+def mp_energy_weight_grad(model: Model, graph: Graph, species):
+    """(energy [1] float64, forces [N,3], {weight name: dE/dW} as CUDA float32 tensors shaped like
+    the weights) -- the weight gradient of the energy (the training path)."""
+    torch = _torch()
+    N = graph.n_atoms
+    energy = torch.empty(1, dtype=torch.float64, device="cuda")
+    forces = torch.empty((N, 3), dtype=torch.float32, device="cuda")
+    sc = spec_c(model.spec)
+    n = lib().mp_weight_count(ctypes.byref(sc))
+    grad = torch.empty(n, dtype=torch.float32, device="cuda")
+    ws = _workspace(lib().mp_weight_grad_workspace_bytes(model.handle, graph.n_edges, N))
+    gc = graph.c()
+    _check(lib().mp_energy_weight_grad(model.handle, ctypes.byref(gc), _ptr(species), _ptr(energy), _ptr(forces),
+                                       _ptr(grad), _ptr(ws), ws.numel(), _stream()), "mp_energy_weight_grad")
+    out, o = {}, 0
+    for name, shape in model.shapes:
+        k = int(np.prod(shape))
+        out[name] = grad[o:o + k].view(*shape)
+        o += k
+    return energy, forces, out
 
 
 class EnergyForcesGraph:

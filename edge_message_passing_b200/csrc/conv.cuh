@@ -247,13 +247,17 @@ __global__ void __launch_bounds__(RAD_THREADS) k_radial_h2(long long E, const in
   }
 }
 
-// dE/dd from dE/dh2 (rows gh2 [E][64], the tensor-core product dE/dR W3); adds (dE/dd) rhat to g_r
+// dE/dd from dE/dh2 (rows gh2 [E][64], the tensor-core product dE/dR W3); adds (dE/dd) rhat to g_r.
+// With rows_out (weight gradients), also each row's basis e [8], h1 [64], dE/dz1 [64] and
+// dE/dz2 [64] into rows_out[row][200], for the sums dE/dW2 = sum dE/dz2 (x) h1 and
+// dE/dW1 = sum dE/dz1 (x) e.
+constexpr int RAD_ROW_FLOATS = 8 + 3 * 64;
 __global__ void __launch_bounds__(RAD_THREADS) k_radial_bwd(long long E, const int* __restrict__ perm,
                                                            const float* __restrict__ dist,
                                                            const float* __restrict__ vec, const int* __restrict__ recv,
                                                            const int* __restrict__ send, const int* __restrict__ species,
                                                            RadialArgs a, const float* __restrict__ gh2,
-                                                           float* __restrict__ g_r) {
+                                                           float* __restrict__ g_r, float* __restrict__ rows_out) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   RadialSmem& s = *reinterpret_cast<RadialSmem*>(smem_raw);
   const int t = threadIdx.x;
@@ -304,6 +308,23 @@ __global__ void __launch_bounds__(RAD_THREADS) k_radial_bwd(long long E, const i
       for (int q = 0; q < 4; ++q)
 #pragma unroll
         for (int b = 0; b < 4; ++b) gh[q][b] = fmaf(gv[q], wv[b], gh[q][b]);
+    }
+    if (rows_out) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const long long r = r0g + r0 + q;
+        if (s.pair[r0 + q] != p) continue;
+        float* ro = rows_out + (size_t)r * RAD_ROW_FLOATS;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          ro[8 + j0 + b] = s.h1T[j0 + b][r0 + q];
+          ro[72 + j0 + b] = gh[q][b] * dsilu_fast(z1[q][b]);
+          ro[136 + j0 + b] = s.gT[j0 + b][r0 + q];
+        }
+        if (j0 == 0)
+#pragma unroll
+          for (int n = 0; n < 8; ++n) ro[n] = s.e[r0 + q][n];
+      }
     }
     // dE/dd[r] = sum_j dE/dz1[r][j] sum_n W1[j][n] de_n[r]: this thread's 4 units, then
     // summed over the 16 threads of the half-warp that share the rows

@@ -73,11 +73,15 @@ inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 
 // ------------------------------------------------------------------ workspace layout
 struct WsLayout {
-  size_t D, dist, R, rbP, nodeZ, nodeX, zro, gxP, XT2, XTlo2, Y2, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
+  size_t D, dist, R, rbP, nodeZ, nodeX, zro, dB, tnp, silu, radrows, gxP, XT2, XTlo2, Y2, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
   size_t total;
 };
 
-WsLayout ws_layout(const Model& m, long long E, int N) {
+// partial sums of the weight-gradient reductions (k_tn): room for the largest splits used
+constexpr int TN_SPLITS = 64;
+inline size_t tn_part_floats(int C) { return std::max((size_t)2 * 36 * C * C, (size_t)TN_SPLITS * 4 * C * 64); }
+
+WsLayout ws_layout(const Model& m, long long E, int N, bool grad = false) {
   WsLayout L{};
   const size_t C = m.spec.C, T = m.spec.n_layers;
   const size_t coh = std::min<long long>(m.spec.cohort_edges, std::max<long long>(E, 1));
@@ -125,6 +129,12 @@ WsLayout ws_layout(const Model& m, long long E, int N) {
   L.nseg = take(ncoh * 4 + 4);
   L.vir = take(VIR_BLOCKS * 9 * 8);
   L.counter = take(64);
+  if (grad) {               // weight gradients: stacked SO(2) block sums, reduction partials, SiLU of the
+    L.dB = take((size_t)WLAYER_CC * C * C * 4);          // readout, per-row radial values
+    L.tnp = take(tn_part_floats((int)C) * 4);
+    L.silu = take((size_t)N * std::max(m.Hro, 1) * 4);
+    L.radrows = take((size_t)E * RAD_ROW_FLOATS * 4);
+  }
   L.total = o;
   return L;
 }
@@ -196,6 +206,47 @@ struct NodeProducts {
     k_node_gemm<<<grid, 256, 0, s>>>(p);
   }
 };
+
+// weight-gradient reduction over rows (end_layers.cuh: k_tn, k_tn_reduce): out (+)= sum_r A(r) (x) B(r)
+void tn_sum(int Na, int Nb, int rows, int w, const float* A, const float* A2, long long a_node, int a_comp,
+            const float* B, const float* B2, long long b_node, int b_comp, float* out, int ldo, bool accumulate,
+            float* part, size_t part_floats, cudaStream_t s) {
+  int splits = 0, rps = NG_K;
+  if (rows > 0) {
+    splits = std::min(TN_SPLITS, std::max(1, (rows + 4095) / 4096));
+    while (splits > 1 && (size_t)splits * Na * Nb > part_floats) --splits;
+    rps = (rows + splits - 1) / splits;
+    rps = (rps + NG_K - 1) / NG_K * NG_K;
+    splits = (rows + rps - 1) / rps;
+    TnArgs a{rows, w, Na, Nb, rps, A, A2, a_node, a_comp, B, B2, b_node, b_comp, part};
+    Scope sc_("weight_grad", s);
+    k_tn<<<dim3((unsigned)((Na + NG_T - 1) / NG_T), (unsigned)((Nb + NG_T - 1) / NG_T), (unsigned)splits), 256, 0, s>>>(a);
+  }
+  Scope sc_("weight_grad", s);
+  k_tn_reduce<<<(unsigned)((Na * Nb + 255) / 256), 256, 0, s>>>(splits, Na, Nb, part, out, ldo, accumulate ? 1 : 0);
+}
+
+// float offsets of each weight in the blob order (include/emp.h: mp_weight_count)
+struct BlobOffsets {
+  std::vector<size_t> rad, so2;     // rad[t * n_pairs + p] (W1, then W2, then W3), so2[t] (W0, Wr1, Wi1, ...)
+  size_t ro_W = 0, ro_w = 0;
+};
+BlobOffsets blob_offsets(const Model& m) {
+  BlobOffsets b;
+  const size_t C = m.spec.C;
+  size_t o = (size_t)m.spec.n_species * C;
+  for (int t = 0; t < m.spec.n_layers; ++t) {
+    for (int p = 0; p < m.n_pairs; ++p) {
+      b.rad.push_back(o);
+      o += m.rad_stride();
+    }
+    b.so2.push_back(o);
+    o += (size_t)(16 + 2 * (9 + 4 + 1)) * C * C;
+  }
+  b.ro_W = o;
+  b.ro_w = o + (size_t)m.Hro * C;
+  return b;
+}
 
 // tensor maps of a cohort buffer pair (rows of 16C) for the full cohort size and for the last (short) cohort
 struct CohortMaps {
@@ -360,13 +411,16 @@ int radial_rows(const Model& m, const emp_graph* g, const int* species, void* ws
 // R rows [E][4C] of layer t: hidden layers on SIMT, head R = h2 W3^T on the tensor cores
 // ncols: 4C, or C when only the degree-0 scales are used (the first layer: degree-0 input);
 // R rows are ncols floats apart
+// use_tables: the radial hidden layers from the certified tables (when the model has them);
+// h2_only: stop after the hidden layers (h2 hi/lo in the workspace), no head product
 int radial_forward(const Model& m, const emp_graph* g, int t, const int* species, const float* dist, float* R,
-                   const RadialRows& rr, void* ws, const WsLayout& L, cudaStream_t s, int ncols) {
+                   const RadialRows& rr, void* ws, const WsLayout& L, cudaStream_t s, int ncols, bool use_tables = true,
+                   bool h2_only = false) {
   const long long E = g->n_edges;
   const int C = m.spec.C;
   float* h2hi = at<float>(ws, L.h2hi);
   float* h2lo = at<float>(ws, L.h2lo);
-  if (m.tab_on) {
+  if (m.tab_on && use_tables) {
     Scope sc_("radial_h2", s);
     tab::k_radial_h2_table<<<(unsigned)std::min<long long>((E + 15) / 16, 16 * tc::num_sms()), tab::TAB_THREADS, 0, s>>>(
         E, rr.perm, dist, g->recv, g->send, species, table_args(m, t), h2hi, h2lo);
@@ -375,6 +429,7 @@ int radial_forward(const Model& m, const emp_graph* g, int t, const int* species
     k_radial_h2<<<(unsigned)std::min<long long>((E + RT - 1) / RT, 3 * tc::num_sms()), RAD_THREADS, sizeof(RadialSmem), s>>>(
         E, rr.perm, dist, g->recv, g->send, species, radial_args(m, t), h2hi, h2lo);
   }
+  if (h2_only) return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
   for (int p = 0; p < m.n_pairs; ++p) {
     const long long r0 = rr.off[p], n = rr.off[p + 1] - r0;
     if (n <= 0) continue;
@@ -393,8 +448,10 @@ int radial_forward(const Model& m, const emp_graph* g, int t, const int* species
 // dE/dd of layer t from dE/dR (rows split hi/lo): dE/dh2 = dE/dR W3 on the tensor cores, then the
 // hidden layers' backward on SIMT; adds (dE/dd) rhat to g_r
 // kcols: 4C, or C when only the degree-0 scales carry a gradient (the first layer)
+// rows_out (weight gradients; network only): each row's e, h1, dE/dz1, dE/dz2 (k_radial_bwd)
 int radial_backward(const Model& m, const emp_graph* g, int t, const int* species, const float* dist,
-                    const RadialRows& rr, float* g_r, void* ws, const WsLayout& L, cudaStream_t s, int kcols) {
+                    const RadialRows& rr, float* g_r, void* ws, const WsLayout& L, cudaStream_t s, int kcols,
+                    bool use_tables = true, float* rows_out = nullptr) {
   const long long E = g->n_edges;
   const int C = m.spec.C;
   float* gRhi = at<float>(ws, L.gRhi);
@@ -412,14 +469,14 @@ int radial_backward(const Model& m, const emp_graph* g, int t, const int* specie
     st = tc_group(n, 64, &sub, 1, at<int>(ws, L.counter), s);
     if (st != EMP_OK) return st;
   }
-  if (m.tab_on) {
+  if (m.tab_on && use_tables) {
     Scope sc_("radial_bwd", s);
     tab::k_radial_bwd_table<<<(unsigned)std::min<long long>((E + 15) / 16, 16 * tc::num_sms()), tab::TAB_THREADS, 0, s>>>(
         E, rr.perm, dist, g->vec, g->recv, g->send, species, table_args(m, t), gh2, g_r);
   } else {
     Scope sc_("radial_bwd", s);
     k_radial_bwd<<<(unsigned)std::min<long long>((E + RT - 1) / RT, 2 * tc::num_sms()), RAD_THREADS, sizeof(RadialSmem), s>>>(
-        E, rr.perm, dist, g->vec, g->recv, g->send, species, radial_args(m, t), gh2, g_r);
+        E, rr.perm, dist, g->vec, g->recv, g->send, species, radial_args(m, t), gh2, g_r, rows_out);
   }
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
@@ -937,7 +994,7 @@ int mp_radial_hidden(const void* model, int32_t layer, int32_t pair, int64_t n, 
     } else {
       Scope sc_("radial_bwd", stream);
       k_radial_bwd<<<(unsigned)std::min<long long>((n + RT - 1) / RT, 2 * tc::num_sms()), RAD_THREADS, sizeof(RadialSmem), stream>>>(
-          n, nullptr, d, vec, nullptr, nullptr, nullptr, ra, g_h2, g_r);
+          n, nullptr, d, vec, nullptr, nullptr, nullptr, ra, g_h2, g_r, nullptr);
     }
     { Scope sc_("radial_aux", stream); k_take_x<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(n, g_r, dE_dd); }
   }
@@ -980,14 +1037,16 @@ int mp_forward(const void* model, const emp_graph* g, int32_t layer, const int32
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
 
-int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* species, double* energy, float* forces,
-                     float* virial, float* atom_energy, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  if (!model || !graph_ok(g) || !energy || !forces || !ws || g->n_atoms < 1) return EMP_ERR_ARG;
-  const Model& m = *static_cast<const Model*>(model);
+// Energy and forces (mp_energy_forces); with grad (mp_energy_weight_grad) also dE/dW in the blob order.
+static int energy_forces_impl(const Model& m, const emp_graph* g, const int32_t* species, double* energy, float* forces,
+                              float* virial, float* atom_energy, float* grad, void* ws, size_t ws_bytes,
+                              cudaStream_t stream) {
   if ((m.spec.pair_radial || m.spec.n_species > 1) && !species) return EMP_ERR_ARG;
   const long long E = g->n_edges, coh = m.spec.cohort_edges;
   const int N = g->n_atoms, C = m.spec.C, T = m.spec.n_layers;
-  const WsLayout L = ws_layout(m, E, N);
+  const bool wgrad = grad != nullptr;
+  const bool tables = !wgrad;           // weight gradients need the radial network itself
+  const WsLayout L = ws_layout(m, E, N, wgrad);
   if (ws_bytes < L.total) return EMP_ERR_WORKSPACE;
   int st = check_device();
   if (st != EMP_OK) return st;
@@ -1044,6 +1103,10 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
   // (end_layers.cuh); the layers between them run the per-edge products over cohorts.
   float* nodeZ = at<float>(ws, L.nodeZ);   // Z (first layer forward), H (first layer backward)
   float* nodeX = at<float>(ws, L.nodeX);   // X (last layer forward), G (last layer backward)
+  const BlobOffsets bo = blob_offsets(m);
+  float* dB = wgrad ? at<float>(ws, L.dB) : nullptr;       // dE/d(stacked SO(2) blocks) of one layer
+  float* tnp = wgrad ? at<float>(ws, L.tnp) : nullptr;
+  float* radrows = wgrad ? at<float>(ws, L.radrows) : nullptr;
   const unsigned nb_node = (unsigned)N;
   // ---------------- forward
   for (int t = 0; t < T; ++t) {
@@ -1052,7 +1115,7 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
     const float* W0 = m.so2_fwd + (size_t)t * m.so2_stride();
     const bool first = t == 0, last = t == T - 1;
     if (E > 0) {
-      st = radial_forward(m, g, t, species, dist, R, rr, ws, L, stream, first ? C : 4 * C);
+      st = radial_forward(m, g, t, species, dist, R, rr, ws, L, stream, first ? C : 4 * C, tables);
       if (st != EMP_OK) return st;
       if (first) {
         { Scope sc_("first_fwd", stream); k_first_fwd<<<nb_node, C, 0, stream>>>(C, g->recv_off, g->send, rr.inv, D, R, xs, nodeZ); }
@@ -1083,7 +1146,15 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
     NodeProducts z(C, m.Hro);
     z.add(N, 1, xs + (size_t)T * feat, 16ll * C, 0, m.ro_W, C, zro, m.Hro, 0);
     z.launch(stream, "readout");
-    { Scope sc_("readout", stream); k_readout_act<<<(unsigned)((N * 32 + 255) / 256), 256, 0, stream>>>(N, m.Hro, m.ro_w, zro, e_atom); }
+    float* silu = wgrad ? at<float>(ws, L.silu) : nullptr;
+    { Scope sc_("readout", stream); k_readout_act<<<(unsigned)((N * 32 + 255) / 256), 256, 0, stream>>>(N, m.Hro, m.ro_w, zro, e_atom, silu); }
+    if (wgrad) {
+      // dE/dw_o = sum_i SiLU(z_i); dE/dW_ro = sum_i (dE/dz_i) (x) h_i[0]
+      EMP_CUDA_TRY(cudaMemsetAsync(grad, 0, weight_count(m.spec) * 4, stream));
+      { Scope sc_("weight_grad", stream); k_colsum<<<(unsigned)((m.Hro + 127) / 128), 128, 0, stream>>>(N, m.Hro, silu, m.Hro, grad + bo.ro_w); }
+      tn_sum(m.Hro, C, N, 1, zro, nullptr, m.Hro, 0, xs + (size_t)T * feat, nullptr, 16ll * C, 0, grad + bo.ro_W, C, false,
+             tnp, tn_part_floats(C), stream);
+    }
     EMP_CUDA_TRY(cudaMemsetAsync(gxa, 0, feat * 4, stream));
     NodeProducts gh(m.Hro, C);
     gh.add(N, 1, zro, m.Hro, 0, m.ro_WT, m.Hro, gxa, 16ll * C, 0);
@@ -1098,6 +1169,19 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
     const bool first = t == 0, last = t == T - 1;
     { Scope sc_("gate_bwd", stream); k_gate_bwd<<<(unsigned)((N * C + 255) / 256), 256, 0, stream>>>(N, C, inv_avg, m.spec.gated,
                                                                      aggs + (size_t)t * feat, gxa, gS, gxb); }
+    if (wgrad) {
+      EMP_CUDA_TRY(cudaMemsetAsync(dB, 0, (size_t)WLAYER_CC * C * C * 4, stream));
+      if (E > 0 && first) {
+        // dW0[(l, c'), (0, c)] = sum over (i, m') of gS_i[l, m', c'] Z_i[l, m', c]  (Z: the forward's sums)
+        for (int l = 0; l < 4; ++l)
+          tn_sum(C, C, N * (2 * l + 1), 2 * l + 1, gS + l * l * C, nullptr, 16ll * C, C, nodeZ + l * l * C, nullptr,
+                 16ll * C, C, dB + (size_t)l * C * 4 * C, 4 * C, false, tnp, tn_part_floats(C), stream);
+      } else if (E > 0 && last) {
+        // dW0[(0, c'), (l, c)] = sum_i gS_i[0, c'] X_i[l, c]
+        tn_sum(C, 4 * C, N, 1, gS, nullptr, 16ll * C, 0, nodeX, nullptr, 4ll * C, 0, dB, 4 * C, false, tnp,
+               tn_part_floats(C), stream);
+      }
+    }
     if (E > 0 && first) {
       // H_i[l, m', c] = sum_c' W0[(l, c'), (0, c)] gS_i[l, m', c']
       NodeProducts np(C, C);
@@ -1105,7 +1189,8 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
         np.add(N * (2 * l + 1), 2 * l + 1, gS + l * l * C, 16ll * C, C, Wb + (size_t)l * C, 4 * C, nodeZ + l * l * C,
                16ll * C, C);
       np.launch(stream);
-      { Scope sc_("first_bwd", stream); k_first_bwd<<<nb_node, C, 0, stream>>>(C, g->recv_off, g->send, rr.inv, g->vec, D, R, xt, nodeZ, gRhi, gRlo, g_r); }
+      // with weight gradients also dE/dx_0 (degree 0 of the senders) for dE/demb
+      { Scope sc_("first_bwd", stream); k_first_bwd<<<nb_node, C, 0, stream>>>(C, g->recv_off, g->send, rr.inv, g->vec, D, R, xt, nodeZ, gRhi, gRlo, g_r, wgrad ? gxb : nullptr); }
     } else if (E > 0 && last) {
       // the output gradient is degree 0 only: G_i[l, c] = sum_c' W0[(0, c'), (l, c)] gS_i[0, c']
       NodeProducts np(C, 4 * C);
@@ -1126,6 +1211,12 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
         So2Part parts[2] = {{am_xt.get(n), &m.bmaps_fwd[t], Y}, {am_gy.get(n), &m.bmaps_bwd[t], GXT}};
         st = so2_product(m, n, parts, 2, counter, stream);
         if (st != EMP_OK) return st;
+        if (wgrad)   // dB_b += sum over the cohort's edges of g_y (x) x~ per block (both as their hi + lo)
+          for (int b = 0; b < 4; ++b) {
+            const int K = blk_width(b) * C, o = blk_off(b) * C;
+            tn_sum(K, K, (int)n, 1, GYhi + o, GYlo + o, 16ll * C, 0, XT + o, XTlo + o, 16ll * C, 0,
+                   dB + (size_t)wblk_off(b) * C * C, K, true, tnp, tn_part_floats(C), stream);
+          }
         // per-edge backward and the sender sums of dE/dx_send into gxb
         const int per = be_per(n, tc::num_sms());
         const int nb = (int)((n + per - 1) / per);
@@ -1145,11 +1236,43 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
       side.wait();        // g_x of this layer complete
       // [per-edge product launches: end]
     }
+    if (wgrad) {
+      Scope sc_("weight_grad", stream);
+      k_unstack_so2<<<256, 256, 0, stream>>>(C, dB, grad + bo.so2[t]);
+    }
     if (E > 0) {
-      st = radial_backward(m, g, t, species, dist, rr, g_r, ws, L, stream, first ? C : 4 * C);
+      if (wgrad) {
+        // dW3 = sum over a network's rows of dE/dR (x) h2 (h2 of this layer recomputed)
+        st = radial_forward(m, g, t, species, dist, nullptr, rr, ws, L, stream, first ? C : 4 * C, false, true);
+        if (st != EMP_OK) return st;
+        const float* h2hi = at<float>(ws, L.h2hi);
+        const float* h2lo = at<float>(ws, L.h2lo);
+        for (int p = 0; p < m.n_pairs; ++p) {
+          const int r0 = rr.off[p], n = rr.off[p + 1] - r0;
+          tn_sum(first ? C : 4 * C, 64, n, 1, gRhi + (size_t)r0 * 4 * C, gRlo + (size_t)r0 * 4 * C, 4ll * C, 0,
+                 h2hi + (size_t)r0 * 64, h2lo + (size_t)r0 * 64, 64, 0, grad + bo.rad[(size_t)t * m.n_pairs + p] + 64 * 8 + 64 * 64,
+                 64, false, tnp, tn_part_floats(C), stream);
+        }
+      }
+      st = radial_backward(m, g, t, species, dist, rr, g_r, ws, L, stream, first ? C : 4 * C, tables, radrows);
       if (st != EMP_OK) return st;
+      if (wgrad)
+        for (int p = 0; p < m.n_pairs; ++p) {
+          // dW2 = sum dE/dz2 (x) h1, dW1 = sum dE/dz1 (x) e over the network's rows
+          const int r0 = rr.off[p], n = rr.off[p + 1] - r0;
+          const float* rows = radrows + (size_t)r0 * RAD_ROW_FLOATS;
+          float* gw = grad + bo.rad[(size_t)t * m.n_pairs + p];
+          tn_sum(64, 64, n, 1, rows + 136, nullptr, RAD_ROW_FLOATS, 0, rows + 8, nullptr, RAD_ROW_FLOATS, 0, gw + 64 * 8, 64,
+                 false, tnp, tn_part_floats(C), stream);
+          tn_sum(64, 8, n, 1, rows + 72, nullptr, RAD_ROW_FLOATS, 0, rows, nullptr, RAD_ROW_FLOATS, 0, gw, 8, false, tnp,
+                 tn_part_floats(C), stream);
+        }
     }
     std::swap(gxa, gxb);
+  }
+  if (wgrad) {
+    Scope sc_("weight_grad", stream);
+    k_species_sum<<<(unsigned)((m.spec.n_species * C + 127) / 128), 128, 0, stream>>>(N, C, m.spec.n_species, species, gxa, grad);
   }
   { Scope sc_("forces", stream); k_forces<<<(N + 127) / 128, 128, 0, stream>>>(N, g->recv_off, g->mirror, g_r, forces); }
   if (virial) {
@@ -1158,6 +1281,25 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
     { Scope sc_("virial", stream); k_virial_final<<<1, 32, 0, stream>>>(VIR_BLOCKS, part, virial); }
   }
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
+}
+
+int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* species, double* energy, float* forces,
+                     float* virial, float* atom_energy, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!model || !graph_ok(g) || !energy || !forces || !ws || g->n_atoms < 1) return EMP_ERR_ARG;
+  return energy_forces_impl(*static_cast<const Model*>(model), g, species, energy, forces, virial, atom_energy, nullptr, ws,
+                            ws_bytes, stream);
+}
+
+size_t mp_weight_grad_workspace_bytes(const void* model, int64_t n_edges, int32_t n_atoms) {
+  if (!model || n_edges < 0 || n_atoms < 1) return 0;
+  return ws_layout(*static_cast<const Model*>(model), n_edges, n_atoms, true).total;
+}
+
+int mp_energy_weight_grad(const void* model, const emp_graph* g, const int32_t* species, double* energy, float* forces,
+                          float* grad, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!model || !graph_ok(g) || !energy || !forces || !grad || !ws || g->n_atoms < 1) return EMP_ERR_ARG;
+  return energy_forces_impl(*static_cast<const Model*>(model), g, species, energy, forces, nullptr, nullptr, grad, ws,
+                            ws_bytes, stream);
 }
 
 // One SO(2) mixing of a batch of edge-frame rows (the per-m block products

@@ -176,12 +176,16 @@ __device__ __forceinline__ void stage_chunk(int eb, int n, const float* __restri
 //   torque: the y^T J g_y term with y = W0 x~ (m = 0 only): per degree l, the channel sums
 //   P[l][m] = sum_c x~[0,0,c] K[l][m][c] enter as -P[l][-1] on the pair (-1, 0) and
 //   +P[l][+1] on the pair (0, +1).
+// With gx (weight gradients: dE/demb needs dE/dx_0), also the layer's gradient with respect to
+// the degree-0 input of the senders, gathered at the receiver through the mirror edges as in
+// the last layer: gx[i][0] += sum_{e in recv(i)} R_e[0] sum_l (-1)^l sum_m' D^l_e[0][m'] H_send(e)[l][m'].
 __global__ void __launch_bounds__(256) k_first_bwd(int C, const int* __restrict__ recv_off,
                                                    const int* __restrict__ send, const int* __restrict__ rrow,
                                                    const float* __restrict__ vec, const float* __restrict__ D,
                                                    const float* __restrict__ R, const float* __restrict__ x,
                                                    const float* __restrict__ H, float* __restrict__ gR_hi,
-                                                   float* __restrict__ gR_lo, float* __restrict__ g_r) {
+                                                   float* __restrict__ gR_lo, float* __restrict__ g_r,
+                                                   float* __restrict__ gx) {
   __shared__ __align__(16) float sD[EL_CH * NDBLK];
   __shared__ float svec[EL_CH * 3];
   __shared__ int ss[EL_CH], sr[EL_CH];
@@ -195,6 +199,7 @@ __global__ void __launch_bounds__(256) k_first_bwd(int C, const int* __restrict_
   constexpr int P2m = jpair_of(2, -1, 0), P2p = jpair_of(2, 0, 1);
   constexpr int P3m = jpair_of(3, -1, 0), P3p = jpair_of(3, 0, 1);
   static_assert(P1m >= 0 && P1p >= 0 && P2m >= 0 && P2p >= 0 && P3m >= 0 && P3p >= 0, "generator pairs");
+  float gsend = 0.f;
   for (int eb = e0; eb < e1; eb += EL_CH) {
     const int n = min(EL_CH, e1 - eb);
     __syncthreads();
@@ -204,7 +209,20 @@ __global__ void __launch_bounds__(256) k_first_bwd(int C, const int* __restrict_
     for (int q = 0; q < n; ++q) {
       const float* Dq = sD + q * NDBLK;
       const float x0 = x[(size_t)ss[q] * 16 * C + c];
-      const float xt = R[(size_t)sr[q] * C + c] * x0;
+      const float r0 = R[(size_t)sr[q] * C + c];
+      const float xt = r0 * x0;
+      if (gx) {
+        const float* hs = H + (size_t)ss[q] * 16 * C + c;
+        float v = hs[0];
+#pragma unroll
+        for (int l = 1; l <= 3; ++l) {
+          float u = 0.f;
+#pragma unroll
+          for (int nn = -l; nn <= l; ++nn) u = fmaf(Dq[dix(l, 0, nn)], hs[(l * l + l + nn) * C], u);
+          v = (l & 1) ? v - u : v + u;
+        }
+        gsend = fmaf(r0, v, gsend);
+      }
       float g0 = h[0];
       float bx = 0.f, by = 0.f;
 #define EMP_FIRST_DEG(L, PM, PP)                                                       \
@@ -242,6 +260,7 @@ __global__ void __launch_bounds__(256) k_first_bwd(int C, const int* __restrict_
     __syncthreads();
     finish_torque(n, nw, eb, red, svec, g_r);
   }
+  if (gx) gx[(size_t)i * 16 * C + c] += gsend;
 }
 
 // ------------------------------------------------------------------ last layer, backward
@@ -419,16 +438,18 @@ __global__ void __launch_bounds__(256) k_node_gemm(const __grid_constant__ NodeG
 // Given z[i][t] = (W_ro h_i[0])_t (a per-node product): e_i = sum_t w_o[t] SiLU(z_it) (one warp per
 // atom, lanes over t in order, then a fixed xor tree) and, in place, z_it <- w_o[t] SiLU'(z_it) =
 // dE/dz (the next per-node product turns it into dE/dh_i[0] = (dE/dz) W_ro).
+// With silu_out (weight gradients), also SiLU(z_it) there (dE/dw_o = sum_i SiLU(z_i)).
 __global__ void k_readout_act(int N, int H, const float* __restrict__ w_o, float* __restrict__ z,
-                              float* __restrict__ e_atom) {
+                              float* __restrict__ e_atom, float* __restrict__ silu_out) {
   const int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (i >= N) return;
   float* zi = z + (size_t)i * H;
   float e = 0.f;
   for (int t = lane; t < H; t += 32) {
-    const float v = zi[t], wt = w_o[t];
-    e = fmaf(wt, silu_f(v), e);
+    const float v = zi[t], wt = w_o[t], sv = silu_f(v);
+    e = fmaf(wt, sv, e);
     zi[t] = wt * dsilu_f(v);
+    if (silu_out) silu_out[(size_t)i * H + t] = sv;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
@@ -462,6 +483,135 @@ __global__ void __launch_bounds__(GEO_EPB) k_geometry_staged(long long E, const 
   float4* dst = reinterpret_cast<float4*>(D + e0 * NDBLK);
   const float4* src = reinterpret_cast<const float4*>(sD);
   for (int q = threadIdx.x; q < n * (NDBLK / 4); q += GEO_EPB) dst[q] = src[q];
+}
+
+// ------------------------------------------------------------------ weight gradients
+// Sums over rows of outer products (the reduction of a weight gradient over edges or nodes):
+// part[z][a][b] = sum over rows r of split z of A(r)[a] B(r)[b], a < Na, b < Nb, with
+// A(r) = A + (r / w) a_node + (r % w) a_comp (and A2 at the same offset added when not null:
+// the two halves of a 3xTF32 split give back the value), likewise B(r).  64 x 64 output tiles
+// (blockIdx.x over a, blockIdx.y over b), rows in steps of 32 staged in shared memory, splits of
+// rows_per_split rows over blockIdx.z; k_tn_reduce adds the splits in order.  FP32, every sum in
+// a fixed order.
+struct TnArgs {
+  int rows, w, Na, Nb, rows_per_split;
+  const float* A;
+  const float* A2;
+  long long a_node;
+  int a_comp;
+  const float* B;
+  const float* B2;
+  long long b_node;
+  int b_comp;
+  float* part;
+};
+__global__ void __launch_bounds__(256) k_tn(const __grid_constant__ TnArgs p) {
+  __shared__ __align__(16) float As[NG_K][NG_T + 4];
+  __shared__ __align__(16) float Bs[NG_K][NG_T + 4];
+  const int a0 = blockIdx.x * NG_T, b0 = blockIdx.y * NG_T;
+  const int r_begin = blockIdx.z * p.rows_per_split, r_end = min(p.rows, r_begin + p.rows_per_split);
+  const int t = threadIdx.x;
+  const int ta = (t >> 4) * 4, tb = (t & 15) * 4;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  for (int rb = r_begin; rb < r_end; rb += NG_K) {
+    __syncthreads();
+    for (int q = t; q < NG_K * NG_T; q += 256) {
+      const int rr = q / NG_T, cc = q % NG_T;
+      const int r = rb + rr;
+      float av = 0.f, bv = 0.f;
+      if (r < r_end) {
+        const long long ao = (long long)(r / p.w) * p.a_node + (long long)(r % p.w) * p.a_comp;
+        const long long bo = (long long)(r / p.w) * p.b_node + (long long)(r % p.w) * p.b_comp;
+        if (a0 + cc < p.Na) av = p.A[ao + a0 + cc] + (p.A2 ? p.A2[ao + a0 + cc] : 0.f);
+        if (b0 + cc < p.Nb) bv = p.B[bo + b0 + cc] + (p.B2 ? p.B2[bo + b0 + cc] : 0.f);
+      }
+      As[rr][cc] = av;
+      Bs[rr][cc] = bv;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < NG_K; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(&As[kk][ta]);
+      const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][tb]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+  }
+  float* out = p.part + (size_t)blockIdx.z * p.Na * p.Nb;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (a0 + ta + i >= p.Na) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (b0 + tb + j < p.Nb) out[(size_t)(a0 + ta + i) * p.Nb + b0 + tb + j] = acc[i][j];
+  }
+}
+
+// out[a * ldo + b] = (accumulate ? out : 0) + sum over z in order of part[z][a][b]
+__global__ void k_tn_reduce(int splits, int Na, int Nb, const float* __restrict__ part, float* __restrict__ out,
+                            int ldo, int accumulate) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= Na * Nb) return;
+  const int a = idx / Nb, b = idx % Nb;
+  float s = accumulate ? out[(size_t)a * ldo + b] : 0.f;
+  for (int z = 0; z < splits; ++z) s += part[(size_t)z * Na * Nb + idx];
+  out[(size_t)a * ldo + b] = s;
+}
+
+// From the gradient dB of a layer's stacked blocks (72 C^2 floats, [n][k] per block, as the
+// forward stacks them) to the weights in the blob's order: W0 [4C][4C], then for m = 1, 2, 3
+// Wr_m, Wi_m [(4-m)C][(4-m)C].  With block b = [[Wr, -Wi], [Wi, Wr]] (rows +, -; columns +, -):
+// dWr = dB[+][+] + dB[-][-], dWi = dB[-][+] - dB[+][-].
+__global__ void k_unstack_so2(int C, const float* __restrict__ dB, float* __restrict__ out) {
+  const size_t total = (size_t)(16 + 2 * (9 + 4 + 1)) * C * C;   // W0 and the three (Wr, Wi) pairs
+  for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += (size_t)gridDim.x * blockDim.x) {
+    if (idx < (size_t)16 * C * C) {
+      out[idx] = dB[idx];
+      continue;
+    }
+    size_t o = (size_t)16 * C * C;
+    for (int m = 1; m <= 3; ++m) {
+      const size_t h = (size_t)(4 - m) * C, hh = h * h;
+      if (idx < o + 2 * hh) {
+        const size_t q = idx - o;
+        const bool imag = q >= hh;
+        const size_t i = (q % hh) / h, j = q % h;
+        const float* B = dB + (size_t)wblk_off(m) * C * C;
+        const size_t K = 2 * h;
+        out[idx] = imag ? B[(h + i) * K + j] - B[i * K + h + j] : B[i * K + j] + B[(h + i) * K + h + j];
+        break;
+      }
+      o += 2 * hh;
+    }
+  }
+}
+
+// out[c] = sum_i v[i][c] (i ascending), c < n, rows of ld floats
+__global__ void k_colsum(int N, int n, const float* __restrict__ v, int ld, float* __restrict__ out) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= n) return;
+  float s = 0.f;
+  for (int i = 0; i < N; ++i) s += v[(size_t)i * ld + c];
+  out[c] = s;
+}
+
+// dE/demb[s][c] = sum over atoms i of species s (ascending) of g[i][0][c]
+__global__ void k_species_sum(int N, int C, int S, const int* __restrict__ species, const float* __restrict__ g,
+                              float* __restrict__ demb) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= S * C) return;
+  const int s = idx / C, c = idx % C;
+  float acc = 0.f;
+  for (int i = 0; i < N; ++i)
+    if ((species ? species[i] : 0) == s) acc += g[(size_t)i * 16 * C + c];
+  demb[idx] = acc;
 }
 
 }  // namespace emp

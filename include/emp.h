@@ -184,6 +184,19 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
                      double* energy, float* forces, float* virial, float* atom_energy,
                      void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* Weight gradients of the energy (the training path, which the page "first-order SO(2)
+ * input-gradient path" leaves on its old code path: "Implementation and scope"): energy,
+ * forces, and grad [mp_weight_count] = dE/dW for every weight, in the blob order of
+ * mp_weight_count (embedding, per layer the radial networks and the SO(2) blocks W0, Wr_m,
+ * Wi_m, then the readout).  Sums over edges and nodes run in FP32 in a fixed order, so the
+ * result is reproducible.  The radial hidden layers are the network's even when the model
+ * has radial tables (their weights get gradients).  Gradients of force terms (mixed second
+ * derivatives) are not computed.  Workspace: mp_weight_grad_workspace_bytes (larger than
+ * mp_workspace_bytes: per-row radial values, block sums and reduction partials). */
+size_t mp_weight_grad_workspace_bytes(const void* model, int64_t n_edges, int32_t n_atoms);
+int mp_energy_weight_grad(const void* model, const emp_graph* g, const int32_t* species, double* energy,
+                          float* forces, float* grad, void* ws, size_t ws_bytes, cudaStream_t stream);
+
 /* The per-m SO(2) channel mixing of a batch of edge-frame rows on its own
  * (page "first-order SO(2) input-gradient path": the mixing GEMMs, strict
  * FP32 -- here 3xTF32 on the tensor cores).  X, Y [M][16C] in the m-major
