@@ -24,8 +24,12 @@ SYMBOLS = (
     "mp_chain_destroy", "mp_radial_chain", "emp_status_string", "emp_last_device_error",
     "emp_profile_enable", "emp_profile_read", "emp_profile_names", "emp_launch_count",
     "emp_set_wait_limit", "emp_wait_selftest", "emp_tf32_mma_rate", "mp_model_radial_tables", "mp_radial_hidden",
-    "mp_weight_grad_workspace_bytes", "mp_energy_weight_grad",
+    "mp_weight_grad_workspace_bytes", "mp_energy_weight_grad", "nl_refresh",
+    "mp_sharded_workspace_bytes", "mp_energy_forces_sharded",
 )
+
+# int (*)(float* buf, size_t n, cudaStream_t stream, void* ctx): the sum over ranks, in place
+ALLREDUCE_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p)
 
 
 class EmpError(RuntimeError):
@@ -68,6 +72,14 @@ def lib() -> ctypes.CDLL:
         L.nl_build.argtypes = [ctypes.POINTER(NlParams), vp, ctypes.POINTER(GraphC), ctypes.POINTER(i64), vp, sz, vp]
         L.nl_build_noalloc.restype = ctypes.c_int
         L.nl_build_noalloc.argtypes = [ctypes.POINTER(NlParams), vp, ctypes.POINTER(GraphC), ctypes.POINTER(i64), vp]
+        L.mp_sharded_workspace_bytes.restype = sz
+        L.mp_sharded_workspace_bytes.argtypes = [vp, i64, i64, i32]
+        L.mp_energy_forces_sharded.restype = ctypes.c_int
+        L.mp_energy_forces_sharded.argtypes = [vp, ctypes.POINTER(GraphC), i32, i32, i32, vp, vp, vp, vp, vp,
+                                               ALLREDUCE_FN, vp, vp, sz, vp]
+        L.nl_refresh.restype = ctypes.c_int
+        L.nl_refresh.argtypes = [ctypes.POINTER(NlParams), vp, vp, ctypes.c_double, ctypes.POINTER(GraphC),
+                                 ctypes.POINTER(i32), vp, sz, vp]
         L.mp_weight_count.restype = sz
         L.mp_weight_count.argtypes = [ctypes.POINTER(SpecC)]
         L.mp_model_create.restype = ctypes.c_int
@@ -259,6 +271,37 @@ def nl_build(pos, box: Sequence[float], cutoff: float, capacity: Optional[int] =
     raise EmpError("nl_build: capacity retry failed")
 
 
+def nl_refresh(graph: Graph, pos, pos_ref, box: Sequence[float], skin: float) -> bool:
+    """Edge vectors of `graph` (built with cutoff + skin at pos_ref) at positions pos; True when
+    some atom moved more than skin / 2 from pos_ref (the graph must then be built again)."""
+    torch = _torch()
+    pos = pos.contiguous()
+    ws = _workspace(256)
+    p = NlParams(graph.n_atoms, (ctypes.c_double * 3)(*[float(b) for b in box]), 0.0, graph.n_edges)
+    gc = graph.c()
+    flag = ctypes.c_int32(0)
+    _check(lib().nl_refresh(ctypes.byref(p), _ptr(pos), _ptr(pos_ref), float(skin), ctypes.byref(gc),
+                            ctypes.byref(flag), _ptr(ws), ws.numel(), _stream()), "nl_refresh")
+    return bool(flag.value)
+
+
+class NeighbourCache:
+    """Neighbour list for an MD loop: built with cutoff + skin and reused, with its edge vectors
+    refreshed at every call, until some atom has moved more than skin / 2 since the build."""
+
+    def __init__(self, box: Sequence[float], cutoff: float, skin: float):
+        self.box, self.cutoff, self.skin = list(box), float(cutoff), float(skin)
+        self.graph, self.pos_ref, self.builds = None, None, 0
+
+    def update(self, pos) -> Graph:
+        if self.graph is not None and not nl_refresh(self.graph, pos, self.pos_ref, self.box, self.skin):
+            return self.graph
+        self.graph = nl_build(pos, self.box, self.cutoff + self.skin, reuse=self.graph)
+        self.pos_ref = pos.clone()
+        self.builds += 1
+        return self.graph
+
+
 # ------------------------------------------------------------------ model
 def weight_order(spec) -> list:
     """Weight names in the blob order documented in include/emp.h."""
@@ -361,6 +404,56 @@ def mp_energy_weight_grad(model: Model, graph: Graph, species):
         out[name] = grad[o:o + k].view(*shape)
         o += k
     return energy, forces, out
+
+
+def receiver_ranges(recv_off, world: int):
+    """Contiguous receiver ranges [(a, b)] for `world` ranks, cut where the running edge count
+    crosses r E / world (balanced by edges, each atom in exactly one range)."""
+    ro = np.asarray(recv_off, dtype=np.int64)
+    N, E = ro.shape[0] - 1, int(ro[-1])
+    cuts = [0] + [int(np.searchsorted(ro, r * E / world, side="left")) for r in range(1, world)] + [N]
+    cuts = np.minimum(np.maximum.accumulate(np.asarray(cuts)), N)
+    return [(int(cuts[r]), int(cuts[r + 1])) for r in range(world)]
+
+
+def mp_energy_forces_sharded(model: Model, graph: Graph, species, rank: int, world: int, group=None,
+                             virial: bool = False):
+    """This rank's part of the energy + force step over receiver ranges (one process per GPU,
+    torch.distributed initialised): returns the whole (energy, forces, virial or None) on every
+    rank.  The sums over ranks go through torch.distributed.all_reduce (NCCL on the GPU; with the
+    gloo backend through host copies)."""
+    import torch.distributed as dist
+    torch = _torch()
+    N = graph.n_atoms
+    a, b = receiver_ranges(graph.recv_off.cpu().numpy(), world)[rank]
+    ro = graph.recv_off.cpu().numpy()
+    El = int(ro[b] - ro[a])
+    ws = _workspace(lib().mp_sharded_workspace_bytes(model.handle, El, graph.n_edges, N))
+    gloo = dist.get_backend(group) == "gloo"
+    base = ws.data_ptr()
+
+    def allreduce(buf, n, stream, ctx):
+        try:
+            t = ws[buf - base: buf - base + 4 * n].view(torch.float32)
+            if gloo:
+                h = t.cpu()
+                dist.all_reduce(h, group=group)
+                t.copy_(h)
+            else:
+                dist.all_reduce(t, group=group)
+            return 0
+        except Exception:                     # no exception crosses the C ABI: report a failure
+            return 1
+
+    fn = ALLREDUCE_FN(allreduce)
+    energy = torch.empty(1, dtype=torch.float64, device="cuda")
+    forces = torch.empty((N, 3), dtype=torch.float32, device="cuda")
+    vir = torch.empty((3, 3), dtype=torch.float32, device="cuda") if virial else None
+    gc = graph.c()
+    _check(lib().mp_energy_forces_sharded(model.handle, ctypes.byref(gc), a, b, rank, _ptr(species), _ptr(energy),
+                                          _ptr(forces), _ptr(vir), None, fn, None, _ptr(ws), ws.numel(), _stream()),
+           "mp_energy_forces_sharded")
+    return energy, forces, vir
 
 
 class EnergyForcesGraph:

@@ -526,6 +526,14 @@ __global__ void k_take_x(long long n, const float* __restrict__ g_r, float* __re
   if (i < n) out[i] = g_r[3 * i];
 }
 
+// recv_off of a rank's local view: its edges [eb, eb + El) re-based to 0, every other receiver's range empty
+__global__ void k_local_offsets(int N, const int* __restrict__ recv_off, int eb, int El, int* __restrict__ out) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i > N) return;
+  const int v = recv_off[i] - eb;
+  out[i] = v < 0 ? 0 : v > El ? El : v;
+}
+
 int check_device() {
   int dev = 0, major = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return EMP_ERR_UNSUPPORTED;
@@ -757,6 +765,32 @@ int nl_build_noalloc(const emp_nl_params* p, const double* pos, emp_graph* g, in
   const int st = nl_noalloc_scratch_address(&scratch);
   if (st != EMP_OK) return st;
   return nl_build_impl(p, pos, g, n_edges, scratch, sizeof(g_nl_noalloc_scratch), stream);
+}
+
+int nl_refresh(const emp_nl_params* p, const double* pos, const double* pos_ref, double skin, emp_graph* g,
+               int32_t* rebuild, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!p || !pos || !pos_ref || !g || !rebuild || !ws || !(skin >= 0.0) || !graph_ok(g)) return EMP_ERR_ARG;
+  if (p->n_atoms < 1 || g->n_atoms != p->n_atoms || g->n_edges > 0 && !g->shift) return EMP_ERR_ARG;
+  for (int d = 0; d < 3; ++d)
+    if (!(p->box[d] > 0) || !std::isfinite(p->box[d])) return EMP_ERR_ARG;
+  if (ws_bytes < 64) return EMP_ERR_WORKSPACE;
+  int st = check_device();
+  if (st != EMP_OK) return st;
+  double* L = static_cast<double*>(ws);
+  double* disp2 = L + 4;
+  EMP_CUDA_TRY(cudaMemcpyAsync(L, p->box, 3 * sizeof(double), cudaMemcpyHostToDevice, stream));
+  if (g->n_edges > 0) {
+    Scope sc_("nl", stream);
+    nl::k_refresh<<<(unsigned)((g->n_edges + 255) / 256), 256, 0, stream>>>(g->n_edges, pos, L, *g);
+  }
+  { Scope sc_("nl", stream); nl::k_max_disp2<<<1, 256, 0, stream>>>(p->n_atoms, pos, pos_ref, disp2); }
+  double h = 0.0;
+  EMP_CUDA_TRY(cudaMemcpyAsync(&h, disp2, sizeof(double), cudaMemcpyDeviceToHost, stream));
+  EMP_CUDA_TRY(cudaStreamSynchronize(stream));
+  if (!std::isfinite(h)) return EMP_ERR_NONFINITE;
+  // a pair within rc now was within rc + skin at pos_ref while no atom moved more than skin / 2
+  *rebuild = 4.0 * h > skin * skin ? 1 : 0;
+  return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------ model
@@ -1037,20 +1071,38 @@ int mp_forward(const void* model, const emp_graph* g, int32_t layer, const int32
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
 
-// Energy and forces (mp_energy_forces); with grad (mp_energy_weight_grad) also dE/dW in the blob order.
+// Receiver-range sharding: this rank takes the edges of receivers [a, b); `g` is then the rank's
+// local view (its edges, recv_off re-based, empty ranges outside [a, b)), `global` the whole graph.
+struct Shard {
+  const emp_graph* global = nullptr;
+  long long e_begin = 0;
+  int rank = 0;
+  emp_allreduce_fn allreduce = nullptr;
+  void* ctx = nullptr;
+};
+
+// Energy and forces (mp_energy_forces); with grad (mp_energy_weight_grad) also dE/dW in the blob order;
+// with sh (mp_energy_forces_sharded) the part of the step of one rank.
 static int energy_forces_impl(const Model& m, const emp_graph* g, const int32_t* species, double* energy, float* forces,
                               float* virial, float* atom_energy, float* grad, void* ws, size_t ws_bytes,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, const Shard* sh = nullptr) {
   if ((m.spec.pair_radial || m.spec.n_species > 1) && !species) return EMP_ERR_ARG;
   const long long E = g->n_edges, coh = m.spec.cohort_edges;
   const int N = g->n_atoms, C = m.spec.C, T = m.spec.n_layers;
   const bool wgrad = grad != nullptr;
   const bool tables = !wgrad;           // weight gradients need the radial network itself
   const WsLayout L = ws_layout(m, E, N, wgrad);
-  if (ws_bytes < L.total) return EMP_ERR_WORKSPACE;
+  const long long E_all = sh ? sh->global->n_edges : E;
+  const size_t shard_extra = sh ? align_up((size_t)E_all * 12 + 4) : 0;   // the whole graph's g_r
+  if (ws_bytes < L.total + shard_extra) return EMP_ERR_WORKSPACE;
   int st = check_device();
   if (st != EMP_OK) return st;
   const size_t feat = (size_t)N * 16 * C;
+  // the caller's sum over the ranks, in place, ordered on the stream
+  auto allreduce = [&](float* buf, size_t n) -> int {
+    if (!sh) return EMP_OK;
+    return sh->allreduce(buf, n, stream, sh->ctx) == 0 ? EMP_OK : EMP_ERR_CUDA;
+  };
   float* D = at<float>(ws, L.D);
   float* dist = at<float>(ws, L.dist);
   float* Rall = at<float>(ws, L.R);
@@ -1136,6 +1188,9 @@ static int energy_forces_impl(const Model& m, const emp_graph* g, const int32_t*
         if (st != EMP_OK) return st;
       }
     }
+    // sharded: every receiver's sums come from the one rank that owns it; the sum over ranks gathers them
+    st = allreduce(S, feat);
+    if (st != EMP_OK) return st;
     { Scope sc_("update", stream); k_update<<<(unsigned)((N * C + 255) / 256), 256, 0, stream>>>(N, C, inv_avg, m.spec.gated, S,
                                                                    xs + (size_t)t * feat, xs + (size_t)(t + 1) * feat); }
   }
@@ -1169,6 +1224,8 @@ static int energy_forces_impl(const Model& m, const emp_graph* g, const int32_t*
     const bool first = t == 0, last = t == T - 1;
     { Scope sc_("gate_bwd", stream); k_gate_bwd<<<(unsigned)((N * C + 255) / 256), 256, 0, stream>>>(N, C, inv_avg, m.spec.gated,
                                                                      aggs + (size_t)t * feat, gxa, gS, gxb); }
+    // sharded: the residual part of dE/dx_t enters the sum over ranks once (rank 0)
+    if (sh && sh->rank != 0 && t > 0) EMP_CUDA_TRY(cudaMemsetAsync(gxb, 0, feat * 4, stream));
     if (wgrad) {
       EMP_CUDA_TRY(cudaMemsetAsync(dB, 0, (size_t)WLAYER_CC * C * C * 4, stream));
       if (E > 0 && first) {
@@ -1268,16 +1325,31 @@ static int energy_forces_impl(const Model& m, const emp_graph* g, const int32_t*
                  tn_part_floats(C), stream);
         }
     }
+    if (t > 0) {     // sharded: the senders' gradients from every rank's edges
+      st = allreduce(gxb, feat);
+      if (st != EMP_OK) return st;
+    }
     std::swap(gxa, gxb);
   }
   if (wgrad) {
     Scope sc_("weight_grad", stream);
     k_species_sum<<<(unsigned)((m.spec.n_species * C + 127) / 128), 128, 0, stream>>>(N, C, m.spec.n_species, species, gxa, grad);
   }
-  { Scope sc_("forces", stream); k_forces<<<(N + 127) / 128, 128, 0, stream>>>(N, g->recv_off, g->mirror, g_r, forces); }
+  const emp_graph* gf = g;                  // the graph the forces and the virial are summed over
+  float* gr_all = g_r;
+  if (sh) {
+    // the edge gradients of every rank, placed at their edges of the whole graph and summed over ranks
+    gf = sh->global;
+    gr_all = reinterpret_cast<float*>(static_cast<char*>(ws) + L.total);
+    EMP_CUDA_TRY(cudaMemsetAsync(gr_all, 0, (size_t)E_all * 12, stream));
+    if (E > 0) EMP_CUDA_TRY(cudaMemcpyAsync(gr_all + 3 * sh->e_begin, g_r, (size_t)E * 12, cudaMemcpyDeviceToDevice, stream));
+    st = allreduce(gr_all, (size_t)E_all * 3);
+    if (st != EMP_OK) return st;
+  }
+  { Scope sc_("forces", stream); k_forces<<<(N + 127) / 128, 128, 0, stream>>>(N, gf->recv_off, gf->mirror, gr_all, forces); }
   if (virial) {
     double* part = at<double>(ws, L.vir);
-    { Scope sc_("virial", stream); k_virial_partial<<<VIR_BLOCKS, 256, 0, stream>>>(E, g->vec, g_r, part); }
+    { Scope sc_("virial", stream); k_virial_partial<<<VIR_BLOCKS, 256, 0, stream>>>(gf->n_edges, gf->vec, gr_all, part); }
     { Scope sc_("virial", stream); k_virial_final<<<1, 32, 0, stream>>>(VIR_BLOCKS, part, virial); }
   }
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
@@ -1288,6 +1360,50 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
   if (!model || !graph_ok(g) || !energy || !forces || !ws || g->n_atoms < 1) return EMP_ERR_ARG;
   return energy_forces_impl(*static_cast<const Model*>(model), g, species, energy, forces, virial, atom_energy, nullptr, ws,
                             ws_bytes, stream);
+}
+
+size_t mp_sharded_workspace_bytes(const void* model, int64_t n_edges_local, int64_t n_edges, int32_t n_atoms) {
+  if (!model || n_edges_local < 0 || n_edges < n_edges_local || n_atoms < 1) return 0;
+  return ws_layout(*static_cast<const Model*>(model), n_edges_local, n_atoms).total + align_up((size_t)n_edges * 12 + 4) +
+         align_up((size_t)(n_atoms + 1) * 4);
+}
+
+int mp_energy_forces_sharded(const void* model, const emp_graph* g, int32_t atom_begin, int32_t atom_end, int32_t rank,
+                             const int32_t* species, double* energy, float* forces, float* virial, float* atom_energy,
+                             emp_allreduce_fn allreduce, void* ctx, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!model || !graph_ok(g) || !energy || !forces || !ws || !allreduce || g->n_atoms < 1) return EMP_ERR_ARG;
+  if (atom_begin < 0 || atom_end < atom_begin || atom_end > g->n_atoms || rank < 0) return EMP_ERR_ARG;
+  const Model& m = *static_cast<const Model*>(model);
+  const int N = g->n_atoms;
+  int st = check_device();
+  if (st != EMP_OK) return st;
+  // this rank's edges: those of receivers [atom_begin, atom_end) (read back: the local view needs them)
+  int off[2] = {0, 0};
+  EMP_CUDA_TRY(cudaMemcpyAsync(&off[0], g->recv_off + atom_begin, 4, cudaMemcpyDeviceToHost, stream));
+  EMP_CUDA_TRY(cudaMemcpyAsync(&off[1], g->recv_off + atom_end, 4, cudaMemcpyDeviceToHost, stream));
+  EMP_CUDA_TRY(cudaStreamSynchronize(stream));
+  const long long eb = off[0], El = (long long)off[1] - off[0];
+  if (El < 0) return EMP_ERR_ARG;
+  const size_t need = mp_sharded_workspace_bytes(model, El, g->n_edges, N);
+  if (ws_bytes < need) return EMP_ERR_WORKSPACE;
+  const size_t ro_at = need - align_up((size_t)(N + 1) * 4);
+  int* recv_off_local = reinterpret_cast<int*>(static_cast<char*>(ws) + ro_at);
+  { Scope sc_("shard", stream); k_local_offsets<<<(unsigned)((N + 1 + 255) / 256), 256, 0, stream>>>(N, g->recv_off, (int)eb, (int)El, recv_off_local); }
+  emp_graph gl = *g;
+  gl.recv = g->recv + eb;
+  gl.send = g->send + eb;
+  gl.mirror = nullptr;           // global edge indices: only the whole graph's forces use them
+  gl.shift = g->shift ? g->shift + 3 * eb : nullptr;
+  gl.vec = g->vec + 3 * eb;
+  gl.recv_off = recv_off_local;
+  gl.n_edges = El;
+  Shard sh;
+  sh.global = g;
+  sh.e_begin = eb;
+  sh.rank = rank;
+  sh.allreduce = allreduce;
+  sh.ctx = ctx;
+  return energy_forces_impl(m, &gl, species, energy, forces, virial, atom_energy, nullptr, ws, ws_bytes, stream, &sh);
 }
 
 size_t mp_weight_grad_workspace_bytes(const void* model, int64_t n_edges, int32_t n_atoms) {

@@ -246,5 +246,40 @@ __global__ void k_mirror(long long E, int n, emp_graph g) {
   g.mirror[e] = found < 0 ? (int)e : found;
 }
 
+// ------------------------------------------------------------------ skin reuse
+// Edge vectors of an existing graph at new positions (same (i, j, S) topology, the same
+// operations as the build: r = (x_j - x_i) + S L per component in double, rounded to float)
+__global__ void k_refresh(long long E, const double* __restrict__ pos, const double* __restrict__ L, emp_graph g) {
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= E) return;
+  const int i = g.recv[e], j = g.send[e];
+#pragma unroll
+  for (int d = 0; d < 3; ++d) {
+    const double r = __dadd_rn(__dsub_rn(pos[3 * j + d], pos[3 * i + d]), __dmul_rn((double)g.shift[3 * e + d], L[d]));
+    g.vec[3 * e + d] = __double2float_rn(r);
+  }
+}
+
+// largest squared displacement |x_i - x_ref_i|^2 over the atoms (one block; fixed tree)
+__global__ void k_max_disp2(int n, const double* __restrict__ pos, const double* __restrict__ ref, double* __restrict__ out) {
+  __shared__ double m[256];
+  double v = 0.0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    double s = 0.0;
+    for (int d = 0; d < 3; ++d) {
+      const double q = pos[3 * i + d] - ref[3 * i + d];
+      s += q * q;
+    }
+    v = fmax(v, s);
+  }
+  m[threadIdx.x] = v;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) m[threadIdx.x] = fmax(m[threadIdx.x], m[threadIdx.x + w]);
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *out = m[0];
+}
+
 }  // namespace nl
 }  // namespace emp

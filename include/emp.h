@@ -117,6 +117,18 @@ int nl_build(const emp_nl_params* p, const double* pos, emp_graph* g, int64_t* n
 int nl_build_noalloc(const emp_nl_params* p, const double* pos, emp_graph* g, int64_t* n_edges,
                      cudaStream_t stream);
 
+/* Neighbour-list reuse in an MD loop (skin).  A graph built by nl_build with cutoff
+ * rc + skin at positions pos_ref stays valid for a model of cutoff rc while no atom has
+ * moved more than skin / 2: the edges longer than rc contribute exactly zero (the radial
+ * envelope and its derivative vanish there and every layer is bias-free).  nl_refresh
+ * writes the edge vectors of g at the new positions pos (same edges and shifts, the same
+ * double-precision operations as nl_build, rounded to float) and sets rebuild (host, out)
+ * to 1 when some atom is more than skin / 2 from its pos_ref position (then call nl_build
+ * again), else 0.  p: the box and n_atoms of the build.  Workspace >= 64 bytes.
+ * Synchronises (reads the displacement back).  Errors: EMP_ERR_ARG, EMP_ERR_NONFINITE. */
+int nl_refresh(const emp_nl_params* p, const double* pos, const double* pos_ref, double skin, emp_graph* g,
+               int32_t* rebuild, void* ws, size_t ws_bytes, cudaStream_t stream);
+
 /* ------------------------------------------------------------ the model
  * Hyper-parameters of the interatomic potential (configs of the seeded
  * workloads; model of the page "first-order SO(2) input-gradient path":
@@ -183,6 +195,28 @@ int mp_forward(const void* model, const emp_graph* g, int32_t layer, const int32
 int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* species,
                      double* energy, float* forces, float* virial, float* atom_energy,
                      void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------ multi-GPU: receiver ranges
+ * Sum of a float buffer over all ranks, in place, ordered on `stream` (e.g. an NCCL
+ * all-reduce); returns 0 on success.  Provided by the caller. */
+typedef int (*emp_allreduce_fn)(float* buf, size_t n, cudaStream_t stream, void* ctx);
+
+/* One rank's part of the energy + force step when the receivers are split into contiguous
+ * ranges over ranks (one process per GPU): this rank computes the edges of receivers
+ * [atom_begin, atom_end) of the whole graph g (every rank holds g and all node features).
+ * After each layer's receiver sums, the sums are added over the ranks (allreduce; each
+ * receiver's row comes from exactly one rank, so the sum is exact); in the backward, each
+ * layer's gradient with respect to the layer's input is added over the ranks (the
+ * residual part counted on rank 0 only), and at the end the per-edge gradients, so that
+ * every rank returns the whole energy, forces, virial and atom energies.  The ranges must
+ * cover the atoms, each once, over the ranks; any split is valid (balanced by edge count
+ * for speed).  Workspace: mp_sharded_workspace_bytes(model, local edges, all edges, N).
+ * Reads the range's edge offsets back to the host (synchronises once).  Not for CUDA-graph
+ * capture unless allreduce is capturable. */
+size_t mp_sharded_workspace_bytes(const void* model, int64_t n_edges_local, int64_t n_edges, int32_t n_atoms);
+int mp_energy_forces_sharded(const void* model, const emp_graph* g, int32_t atom_begin, int32_t atom_end, int32_t rank,
+                             const int32_t* species, double* energy, float* forces, float* virial, float* atom_energy,
+                             emp_allreduce_fn allreduce, void* ctx, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Weight gradients of the energy (the training path, which the page "first-order SO(2)
  * input-gradient path" leaves on its old code path: "Implementation and scope"): energy,
