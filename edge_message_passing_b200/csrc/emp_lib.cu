@@ -79,7 +79,7 @@ struct WsLayout {
 
 // partial sums of the weight-gradient reductions (k_tn): room for the largest splits used
 constexpr int TN_SPLITS = 64;
-inline size_t tn_part_floats(int C) { return std::max((size_t)2 * 36 * C * C, (size_t)TN_SPLITS * 4 * C * 64); }
+inline size_t tn_part_floats(int C) { return std::max((size_t)16 * 36 * C * C, (size_t)TN_SPLITS * 4 * C * 64); }
 
 WsLayout ws_layout(const Model& m, long long E, int N, bool grad = false) {
   WsLayout L{};
@@ -213,14 +213,17 @@ void tn_sum(int Na, int Nb, int rows, int w, const float* A, const float* A2, lo
             float* part, size_t part_floats, cudaStream_t s) {
   int splits = 0, rps = NG_K;
   if (rows > 0) {
-    splits = std::min(TN_SPLITS, std::max(1, (rows + 4095) / 4096));
+    // enough blocks for two per SM, each split at least 256 rows, within the partials' room
+    const int tiles = ((Na + TN_T - 1) / TN_T) * ((Nb + TN_T - 1) / TN_T);
+    splits = std::min(TN_SPLITS, std::max(1, (2 * tc::num_sms() + tiles - 1) / tiles));
+    splits = std::min(splits, std::max(1, rows / 256));
     while (splits > 1 && (size_t)splits * Na * Nb > part_floats) --splits;
     rps = (rows + splits - 1) / splits;
-    rps = (rps + NG_K - 1) / NG_K * NG_K;
+    rps = (rps + TN_K - 1) / TN_K * TN_K;
     splits = (rows + rps - 1) / rps;
     TnArgs a{rows, w, Na, Nb, rps, A, A2, a_node, a_comp, B, B2, b_node, b_comp, part};
     Scope sc_("weight_grad", s);
-    k_tn<<<dim3((unsigned)((Na + NG_T - 1) / NG_T), (unsigned)((Nb + NG_T - 1) / NG_T), (unsigned)splits), 256, 0, s>>>(a);
+    k_tn<<<dim3((unsigned)((Na + TN_T - 1) / TN_T), (unsigned)((Nb + TN_T - 1) / TN_T), (unsigned)splits), 256, 0, s>>>(a);
   }
   Scope sc_("weight_grad", s);
   k_tn_reduce<<<(unsigned)((Na * Nb + 255) / 256), 256, 0, s>>>(splits, Na, Nb, part, out, ldo, accumulate ? 1 : 0);

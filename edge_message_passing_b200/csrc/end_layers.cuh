@@ -489,10 +489,10 @@ __global__ void __launch_bounds__(GEO_EPB) k_geometry_staged(long long E, const 
 // Sums over rows of outer products (the reduction of a weight gradient over edges or nodes):
 // part[z][a][b] = sum over rows r of split z of A(r)[a] B(r)[b], a < Na, b < Nb, with
 // A(r) = A + (r / w) a_node + (r % w) a_comp (and A2 at the same offset added when not null:
-// the two halves of a 3xTF32 split give back the value), likewise B(r).  64 x 64 output tiles
-// (blockIdx.x over a, blockIdx.y over b), rows in steps of 32 staged in shared memory, splits of
-// rows_per_split rows over blockIdx.z; k_tn_reduce adds the splits in order.  FP32, every sum in
-// a fixed order.
+// the two halves of a 3xTF32 split give back the value), likewise B(r).  128 x 128 output tiles
+// (blockIdx.x over a, blockIdx.y over b; an 8 x 8 register tile per thread), rows in steps of 16
+// staged in shared memory, splits of rows_per_split rows over blockIdx.z; k_tn_reduce adds the
+// splits in order.  FP32, every sum in a fixed order.
 struct TnArgs {
   int rows, w, Na, Nb, rows_per_split;
   const float* A;
@@ -505,22 +505,25 @@ struct TnArgs {
   int b_comp;
   float* part;
 };
+constexpr int TN_T = 128, TN_K = 16;       // output tile edge, rows per staged step
 __global__ void __launch_bounds__(256) k_tn(const __grid_constant__ TnArgs p) {
-  __shared__ __align__(16) float As[NG_K][NG_T + 4];
-  __shared__ __align__(16) float Bs[NG_K][NG_T + 4];
-  const int a0 = blockIdx.x * NG_T, b0 = blockIdx.y * NG_T;
+  __shared__ __align__(16) float As[TN_K][TN_T + 4];
+  __shared__ __align__(16) float Bs[TN_K][TN_T + 4];
+  const int a0 = blockIdx.x * TN_T, b0 = blockIdx.y * TN_T;
   const int r_begin = blockIdx.z * p.rows_per_split, r_end = min(p.rows, r_begin + p.rows_per_split);
   const int t = threadIdx.x;
-  const int ta = (t >> 4) * 4, tb = (t & 15) * 4;
-  float acc[4][4];
+  // thread (ty, tx) owns a 8 x 8 register tile: rows a0 + 4 ty + {0..3, 64..67}, columns b0 + 4 tx + {0..3, 64..67}
+  const int ty = t >> 4, tx = t & 15;
+  float acc[8][8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-  for (int rb = r_begin; rb < r_end; rb += NG_K) {
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  for (int rb = r_begin; rb < r_end; rb += TN_K) {
     __syncthreads();
-    for (int q = t; q < NG_K * NG_T; q += 256) {
-      const int rr = q / NG_T, cc = q % NG_T;
+#pragma unroll
+    for (int q = t; q < TN_K * TN_T; q += 256) {
+      const int rr = q / TN_T, cc = q % TN_T;
       const int r = rb + rr;
       float av = 0.f, bv = 0.f;
       if (r < r_end) {
@@ -533,24 +536,30 @@ __global__ void __launch_bounds__(256) k_tn(const __grid_constant__ TnArgs p) {
       Bs[rr][cc] = bv;
     }
     __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < NG_K; ++kk) {
-      const float4 a = *reinterpret_cast<const float4*>(&As[kk][ta]);
-      const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][tb]);
-      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll 4
+    for (int kk = 0; kk < TN_K; ++kk) {
+      const float4 a_lo = *reinterpret_cast<const float4*>(&As[kk][4 * ty]);
+      const float4 a_hi = *reinterpret_cast<const float4*>(&As[kk][64 + 4 * ty]);
+      const float4 b_lo = *reinterpret_cast<const float4*>(&Bs[kk][4 * tx]);
+      const float4 b_hi = *reinterpret_cast<const float4*>(&Bs[kk][64 + 4 * tx]);
+      const float av[8] = {a_lo.x, a_lo.y, a_lo.z, a_lo.w, a_hi.x, a_hi.y, a_hi.z, a_hi.w};
+      const float bv[8] = {b_lo.x, b_lo.y, b_lo.z, b_lo.w, b_hi.x, b_hi.y, b_hi.z, b_hi.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
   }
   float* out = p.part + (size_t)blockIdx.z * p.Na * p.Nb;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    if (a0 + ta + i >= p.Na) continue;
+  for (int i = 0; i < 8; ++i) {
+    const int a = a0 + (i < 4 ? 4 * ty + i : 64 + 4 * ty + i - 4);
+    if (a >= p.Na) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (b0 + tb + j < p.Nb) out[(size_t)(a0 + ta + i) * p.Nb + b0 + tb + j] = acc[i][j];
+    for (int j = 0; j < 8; ++j) {
+      const int b = b0 + (j < 4 ? 4 * tx + j : 64 + 4 * tx + j - 4);
+      if (b < p.Nb) out[(size_t)a * p.Nb + b] = acc[i][j];
+    }
   }
 }
 
