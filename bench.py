@@ -333,13 +333,9 @@ def other_configs(emp, torch, stream, flush, hbm_gbs: float, steps: int = 10):
         pos = torch.from_numpy(st.pos).cuda()
         sp = torch.from_numpy(st.species).cuda()
         g = emp.nl_build(pos, st.box, spec.cutoff)
-        if spec.pair_radial:
-            fn = lambda: emp.mp_energy_forces(model, g, sp)           # eager: one pair-offset read-back per call
-            how = "eager call"
-        else:
-            efg = emp.EnergyForcesGraph(model, g, sp)
-            fn = efg.replay
-            how = "CUDA-graph replay"
+        efg = emp.EnergyForcesGraph(model, g, sp)
+        fn = efg.replay
+        how = "CUDA-graph replay"
         ms = timed(fn)
         N = st.pos.shape[0]
         out[name] = {"n_atoms": N, "n_edges": g.n_edges, "C": spec.C, "layers": spec.n_layers,

@@ -466,9 +466,6 @@ class EnergyForcesGraph:
 
     def __init__(self, model: Model, graph: Graph, species, virial: bool = False, atom_energy: bool = False):
         torch = _torch()
-        if getattr(model.spec, "pair_radial", False):
-            # per-pair radial networks read the pair offsets back to the host once per call
-            raise EmpError("EnergyForcesGraph: models with per-pair radial networks cannot be captured")
         N = graph.n_atoms
         self.model, self.graph, self.species = model, graph, species
         self.energy = torch.empty(1, dtype=torch.float64, device="cuda")

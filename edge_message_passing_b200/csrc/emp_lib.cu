@@ -384,15 +384,18 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
 // [per-edge product launches: end]
 
 // Rows of the radial network: edge order for one radial network, pair-sorted for
-// per-pair networks (stable counting sort; the host reads the pair offsets once).
+// per-pair networks (stable counting sort on the device; the pair offsets stay there, and the
+// radial products take their row ranges from them).  host_offsets: also read the offsets back
+// (the weight-gradient sums need them on the host; this synchronises).
 struct RadialRows {
   const int* perm = nullptr;   // row -> edge (null: identity)
   const int* inv = nullptr;    // edge -> row
-  std::vector<int> off;        // [n_pairs + 1] first row of each pair
+  const int* off_dev = nullptr;// [n_pairs + 1] first row of each pair (device; null for one network)
+  std::vector<int> off;        // the same on the host, when asked for (one network: {0, E})
 };
 
 int radial_rows(const Model& m, const emp_graph* g, const int* species, void* ws, const WsLayout& L,
-                RadialRows& rr, cudaStream_t s) {
+                RadialRows& rr, cudaStream_t s, bool host_offsets = false) {
   const long long E = g->n_edges;
   rr.off.assign(m.n_pairs + 1, 0);
   if (!m.spec.pair_radial) {
@@ -404,10 +407,13 @@ int radial_rows(const Model& m, const emp_graph* g, const int* species, void* ws
   int* off = at<int>(ws, L.poff);
   { Scope sc_("pair_sort", s); k_pair_sort<<<1, PS_THREADS, (size_t)m.n_pairs * PS_THREADS * 4, s>>>(
         E, m.spec.n_species, m.n_pairs, g->recv, g->send, species, perm, inv, off); }
-  EMP_CUDA_TRY(cudaMemcpyAsync(rr.off.data(), off, (m.n_pairs + 1) * sizeof(int), cudaMemcpyDeviceToHost, s));
-  EMP_CUDA_TRY(cudaStreamSynchronize(s));
+  if (host_offsets) {
+    EMP_CUDA_TRY(cudaMemcpyAsync(rr.off.data(), off, (m.n_pairs + 1) * sizeof(int), cudaMemcpyDeviceToHost, s));
+    EMP_CUDA_TRY(cudaStreamSynchronize(s));
+  }
   rr.perm = perm;
   rr.inv = inv;
+  rr.off_dev = off;
   return EMP_OK;
 }
 
@@ -433,19 +439,17 @@ int radial_forward(const Model& m, const emp_graph* g, int t, const int* species
         E, rr.perm, dist, g->recv, g->send, species, radial_args(m, t), h2hi, h2lo);
   }
   if (h2_only) return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
+  // one launch: a sub-problem per radial network over its (device) row range
+  MapPair a;
+  int st = make_pair(&a, h2hi, h2lo, E, 64, 64, tc::BM);
+  if (st != EMP_OK) return st;
+  GemmSub subs[tc::MAXSUB];
   for (int p = 0; p < m.n_pairs; ++p) {
-    const long long r0 = rr.off[p], n = rr.off[p + 1] - r0;
-    if (n <= 0) continue;
-    MapPair a;
-    int st = make_pair(&a, h2hi + r0 * 64, h2lo + r0 * 64, n, 64, 64, tc::BM);
-    if (st != EMP_OK) return st;
     const MapPair& b = (ncols == C ? m.w3n_maps : m.w3_maps)[(size_t)t * m.n_pairs + p];
-    GemmSub sub{&a.hi, &a.lo, &b.hi, &b.lo, 0, 64, ncols, 0, R + r0 * ncols};
-    Scope sc_("radial_head", s);
-    st = tc_group(n, ncols, &sub, 1, at<int>(ws, L.counter), s);
-    if (st != EMP_OK) return st;
+    subs[p] = GemmSub{&a.hi, &a.lo, &b.hi, &b.lo, 0, 64, ncols, 0, R};
   }
-  return EMP_OK;
+  Scope sc_("radial_head", s);
+  return tc_group(E, ncols, subs, m.n_pairs, at<int>(ws, L.counter), s, rr.off_dev);
 }
 
 // dE/dd of layer t from dE/dR (rows split hi/lo): dE/dh2 = dE/dR W3 on the tensor cores, then the
@@ -460,16 +464,17 @@ int radial_backward(const Model& m, const emp_graph* g, int t, const int* specie
   float* gRhi = at<float>(ws, L.gRhi);
   float* gRlo = at<float>(ws, L.gRlo);
   float* gh2 = at<float>(ws, L.gh2);
-  for (int p = 0; p < m.n_pairs; ++p) {
-    const long long r0 = rr.off[p], n = rr.off[p + 1] - r0;
-    if (n <= 0) continue;
+  {
     MapPair a;
-    int st = make_pair(&a, gRhi + r0 * 4 * C, gRlo + r0 * 4 * C, n, 4 * C, 4 * C, tc::BM);
+    int st = make_pair(&a, gRhi, gRlo, E, 4 * C, 4 * C, tc::BM);
     if (st != EMP_OK) return st;
-    const MapPair& b = m.w3t_maps[(size_t)t * m.n_pairs + p];
-    GemmSub sub{&a.hi, &a.lo, &b.hi, &b.lo, 0, kcols, 64, 0, gh2 + r0 * 64};
+    GemmSub subs[tc::MAXSUB];
+    for (int p = 0; p < m.n_pairs; ++p) {
+      const MapPair& b = m.w3t_maps[(size_t)t * m.n_pairs + p];
+      subs[p] = GemmSub{&a.hi, &a.lo, &b.hi, &b.lo, 0, kcols, 64, 0, gh2};
+    }
     Scope sc_("radial_head_bwd", s);
-    st = tc_group(n, 64, &sub, 1, at<int>(ws, L.counter), s);
+    st = tc_group(E, 64, subs, m.n_pairs, at<int>(ws, L.counter), s, rr.off_dev);
     if (st != EMP_OK) return st;
   }
   if (m.tab_on && use_tables) {
@@ -1150,7 +1155,7 @@ static int energy_forces_impl(const Model& m, const emp_graph* g, const int32_t*
   }
   RadialRows rr;
   if (E > 0) {
-    st = radial_rows(m, g, species, ws, L, rr, stream);
+    st = radial_rows(m, g, species, ws, L, rr, stream, wgrad);
     if (st != EMP_OK) return st;
   }
   // The first layer (its input, the species embedding, is degree 0 only) and the last layer

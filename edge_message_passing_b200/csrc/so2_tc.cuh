@@ -56,6 +56,9 @@ struct Group {
   int ldc;              // row pitch (elements) of the outputs
   float* out[MAXSUB];
   int* counter;         // dynamic tile counter (zeroed by the host before the launch)
+  // null, or device row ranges: sub-problem s covers rows [row_off[s], row_off[s + 1]) of its A
+  // operand and output (M and mtiles are then upper bounds; tiles past a range are skipped)
+  const int* row_off;
 };
 
 struct Maps {
@@ -238,6 +241,23 @@ __device__ __forceinline__ TileInfo tile_info2(const Group& g, int t) {
   return ti;
 }
 
+__device__ __forceinline__ int row_base(const Group& g, int sub) { return g.row_off ? g.row_off[sub] : 0; }
+__device__ __forceinline__ int row_end(const Group& g, int sub) { return g.row_off ? g.row_off[sub + 1] : g.M; }
+
+// next tile index for the pair: with device row ranges, a tile past its sub-problem's rows is
+// dead, and so is every later tile of that sub-problem (m-tiles in order), so the counter jumps
+// to the next sub-problem
+__device__ __forceinline__ int next_tile(const Group& g, int total) {
+  int t = atomicAdd(g.counter, 1);
+  while (g.row_off && t < total) {
+    const TileInfo ti = tile_info2(g, t);
+    if (ti.m0 < row_end(g, ti.sub) - row_base(g, ti.sub)) break;
+    atomicMax(g.counter, g.first[ti.sub + 1]);
+    t = atomicAdd(g.counter, 1);
+  }
+  return t;
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     k_so2_tc2(const __grid_constant__ Group g, const __grid_constant__ Maps maps, int total_tiles) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -303,7 +323,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int t;
       if (leader) {
         if (j >= TQ && !mbar_wait_cluster(&tq_empty[slot], ((j / TQ) - 1) & 1)) { *vabort = 1; t = total_tiles; }
-        else t = *vabort ? total_tiles : atomicAdd(g.counter, 1);
+        else t = *vabort ? total_tiles : next_tile(g, total_tiles);
         tq[slot] = t;
         remote_store(map_to_rank(smem_u32(&tq[slot]), 1), t);
         mbar_arrive(&tq_full[slot]);
@@ -325,8 +345,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         unsigned char* st = smem + s * STAGE2;
         if (leader) mbar_expect_tx(&full[s], 2 * (2 * A_BYTES + 2 * bh * BK * 4));
         const uint32_t fb = full_l + (uint32_t)(s * 8);
-        tma_load_pair(st, &maps.a_hi[a], fb, g.acol[ti.sub] + kc * BK, ti.m0 + (int)rank * BM);
-        tma_load_pair(st + A_BYTES, &maps.a_lo[a], fb, g.acol[ti.sub] + kc * BK, ti.m0 + (int)rank * BM);
+        const int arow = row_base(g, ti.sub) + ti.m0 + (int)rank * BM;
+        tma_load_pair(st, &maps.a_hi[a], fb, g.acol[ti.sub] + kc * BK, arow);
+        tma_load_pair(st + A_BYTES, &maps.a_lo[a], fb, g.acol[ti.sub] + kc * BK, arow);
         tma_load_pair(st + 2 * A_BYTES, &maps.b_hi[b], fb, kc * BK, ti.n0 + (int)rank * bh);
         tma_load_pair(st + 2 * A_BYTES + B2_BYTES, &maps.b_lo[b], fb, kc * BK, ti.n0 + (int)rank * bh);
         *issued = it + 1;
@@ -393,7 +414,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       fence_after();
       // 32 x 32 chunks: TMEM -> registers (a row per thread) -> this warp's staging tile ->
       // rows stored 8 threads x 16 bytes at a time, so every store writes whole 128-byte segments
-      const int mw = ti.m0 + (int)rank * BM + q * 32;
+      const int mw = row_base(g, ti.sub) + ti.m0 + (int)rank * BM + q * 32;
+      const int mend = row_end(g, ti.sub);
       const int N = g.N[ti.sub], bn = g.bn[ti.sub];
       float* obase = g.out[ti.sub] + (size_t)g.ccol[ti.sub] + ti.n0;
       float* stg = epi + q * 32 * EPI_PITCH;
@@ -412,7 +434,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const int rr = k * 4 + (lane >> 3), c4 = (lane & 7) * 4;
             const int m = mw + rr;
             const float4 w = *reinterpret_cast<const float4*>(stg + rr * EPI_PITCH + c4);
-            if (m < g.M) *reinterpret_cast<float4*>(obase + (size_t)m * g.ldc + cc + c4) = w;
+            if (m < mend) *reinterpret_cast<float4*>(obase + (size_t)m * g.ldc + cc + c4) = w;
           }
           __syncwarp();
         }
@@ -562,20 +584,25 @@ struct GemmSub {
 };
 
 // Launch a group of products sharing the row count M (at most two distinct A operands).
-// Sub-problems are reordered by decreasing K; counter: one device int, zeroed here.
-inline int tc_group(long long M, int ldc, const GemmSub* subs, int nsub, int* counter, cudaStream_t s) {
+// Sub-problems are reordered by decreasing K; counter: one device int, zeroed here.  With
+// row_off (device, nsub + 1 entries in the subs' given order), sub-problem s covers rows
+// [row_off[s], row_off[s + 1]) only, M being an upper bound of every range.
+inline int tc_group(long long M, int ldc, const GemmSub* subs, int nsub, int* counter, cudaStream_t s,
+                    const int* row_off = nullptr) {
   if (M <= 0) return EMP_OK;
   if (nsub < 1 || nsub > tc::MAXSUB || M >= (1ll << 31)) return EMP_ERR_ARG;
   tc::Group g{};
   tc::Maps maps;
   g.M = (int)M;
+  g.row_off = row_off;
   g.ldc = ldc;
   g.nsub = nsub;
   g.mtiles = (int)((M + 2 * tc::BM - 1) / (2 * tc::BM));
   g.counter = counter;
   int ord[tc::MAXSUB];
   for (int i = 0; i < nsub; ++i) ord[i] = i;
-  std::stable_sort(ord, ord + nsub, [&](int a, int b) { return subs[a].K > subs[b].K; });
+  if (!row_off)        // with device row ranges the subs keep their order (row_off is indexed by it)
+    std::stable_sort(ord, ord + nsub, [&](int a, int b) { return subs[a].K > subs[b].K; });
   const CUtensorMap* a_seen[2] = {nullptr, nullptr};
   int na = 0;
   long long first = 0;

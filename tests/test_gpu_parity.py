@@ -311,6 +311,26 @@ def test_energy_forces_full_size_against_stored_oracle(name):
     assert emp.last_device_error() == 0
 
 
+def test_graph_replay_matches_eager_ternary_per_pair_networks():
+    """Per-pair radial networks are captured too (their row ranges stay on the device)."""
+    ref = _stored_oracle("ternary_n2000")
+    w = synth.workload("ternary_n2000")
+    st = w.structure
+    g = _graph(st, w.spec.cutoff)
+    sp = _cuda(st.species)
+    model = emp.Model(w.spec, w.weights)
+    e, f, _, _ = emp.mp_energy_forces(model, g, sp)
+    e, f = e.clone(), f.clone()
+    efg = emp.EnergyForcesGraph(model, g, sp)
+    for _ in range(2):
+        e2, f2, _, _ = efg.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(e, e2) and torch.equal(f, f2)
+    assert abs(float(e2.cpu()[0]) - float(ref["energy"])) <= 1e-5 * abs(float(ref["energy"]))
+    assert np.abs(f2.cpu().numpy() - ref["forces"]).max() <= 1e-4 * np.abs(ref["forces"]).max()
+    assert emp.last_device_error() == 0
+
+
 def test_graph_replay_matches_eager_n4096():
     """The launch configuration bench.py times: the step captured once as a CUDA graph and
     replayed gives the eager call's results bit for bit (and so the stored oracle's)."""
