@@ -73,7 +73,7 @@ inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 
 // ------------------------------------------------------------------ workspace layout
 struct WsLayout {
-  size_t D, dist, R, rbP, nodeZ, nodeX, zro, dB, tnp, silu, radrows, gxP, XT2, XTlo2, Y2, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
+  size_t gxP2, D, dist, R, rbP, nodeZ, nodeX, zro, dB, tnp, silu, radrows, gxP, XT2, XTlo2, Y2, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
   size_t total;
 };
 
@@ -115,6 +115,7 @@ WsLayout ws_layout(const Model& m, long long E, int N, bool grad = false) {
   L.e_atom = take((size_t)N * 4);
   const size_t cb = coh * 16 * C * 4;
   L.gxP = take(cb);
+  L.gxP2 = take(cb);        // run pieces of every other cohort (the backward's sender sums)
   L.XT2 = take(cb);
   L.XTlo2 = take(cb);
   L.Y2 = take(cb);
@@ -282,8 +283,9 @@ void split(const float* a, float* hi, float* lo, size_t n, cudaStream_t s) {
 // orders their combines but adds no other dependency.
 struct Side {
   cudaStream_t aux = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr, join2 = nullptr;
   bool pending = false;       // a combine was issued on aux and not yet joined
+  int issued = 0;             // combines issued through this Side
   cudaStream_t s = nullptr;
   // run the launch f on aux after everything issued on s so far
   template <typename F>
@@ -292,13 +294,18 @@ struct Side {
     cudaEventRecord(fork, s);
     cudaStreamWaitEvent(aux, fork, 0);
     f(aux);
-    cudaEventRecord(join, aux);
+    cudaEventRecord(issued & 1 ? join2 : join, aux);
+    ++issued;
     pending = true;
   }
   // make s wait for the last combine
   void wait() {
-    if (aux && pending) cudaStreamWaitEvent(s, join, 0);
+    if (aux && pending) cudaStreamWaitEvent(s, (issued - 1) & 1 ? join2 : join, 0);
     pending = false;
+  }
+  // make s wait for the combine before the last (for buffers used every other combine)
+  void wait_second_last() {
+    if (aux && issued >= 2) cudaStreamWaitEvent(s, issued & 1 ? join2 : join, 0);
   }
 };
 thread_local Side g_side[64];
@@ -314,20 +321,23 @@ Side side_for(cudaStream_t s) {
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return out;
     cudaStream_t a = nullptr;
-    cudaEvent_t f = nullptr, j = nullptr;
+    cudaEvent_t f = nullptr, j = nullptr, j2 = nullptr;
     if (cudaStreamCreateWithFlags(&a, cudaStreamNonBlocking) != cudaSuccess) { cudaGetLastError(); return out; }
     if (cudaEventCreateWithFlags(&f, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&j, cudaEventDisableTiming) != cudaSuccess) {
+        cudaEventCreateWithFlags(&j, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&j2, cudaEventDisableTiming) != cudaSuccess) {
       cudaGetLastError();
       return out;
     }
     d.aux = a;
     d.fork = f;
     d.join = j;
+    d.join2 = j2;
   }
   out.aux = d.aux;
   out.fork = d.fork;
   out.join = d.join;
+  out.join2 = d.join2;
   return out;
 }
 
@@ -1285,8 +1295,10 @@ static int energy_forces_impl(const Model& m, const emp_graph* g, const int32_t*
         // per-edge backward and the sender sums of dE/dx_send into gxb
         const int per = be_per(n, tc::num_sms());
         const int nb = (int)((n + per - 1) / per);
-        float* Pg = at<float>(ws, L.gxP);
-        side.wait();      // the previous cohort's combine has read Pg
+        // run pieces in two buffers, cohort by cohort in turn: the combine of the cohort before
+        // last has read this one (the last combine may still run beside this kernel)
+        float* Pg = at<float>(ws, ci & 1 ? L.gxP2 : L.gxP);
+        side.wait_second_last();
         {
           Scope sc_("bwd_edge", stream);
           k_bwd_edge<BE_V><<<nb, C / BE_V, be_smem_bytes(C), stream>>>(e0, e1, C, per, g->send, rr.inv, g->vec, D, R,
