@@ -269,7 +269,7 @@ def hbm_fractions(fam, steps: int, E: int, N: int, C: int, T: int, hbm_gbs: floa
 # shapes (profiles/kernels_n512_step.md).  Valid only for the kernel source and the launch
 # structure it was taken on: so2_tc.cuh and the marked per-edge product launch code of emp_lib.cu
 # must hash to source_sha1, else the roofline's traffic is null.
-SO2_TRAFFIC = {"source_sha1": "86fa8e78eeab526ddde159654fc26bb6a322ea3f", "bytes_per_launch": 389.6e6}
+SO2_TRAFFIC = {"source_sha1": "ce709d4c4d2e8ac7b7432db596fca495fb14a9a7", "bytes_per_launch": 388.6e6}
 
 
 def so2_source_hash():
@@ -353,12 +353,48 @@ def other_configs(emp, torch, stream, flush, hbm_gbs: float, steps: int = 10):
     g = emp.nl_build(pos, st.box, spec.cutoff)
     efg = emp.EnergyForcesGraph(model, g, sp)
     ms = timed(efg.replay)
-    out[WORKLOAD + "_radial_tables"] = {"n_atoms": st.pos.shape[0], "n_edges": g.n_edges, "ms_per_step": round(ms, 4),
-                                        "edges_per_s": g.n_edges / (ms * 1e-3), "table_pieces": n_pieces,
-                                        "timed": "CUDA-graph replay",
-                                        "note": "opt-in certified Chebyshev tables (degree 10, tol 1e-7) for the radial "
-                                                "hidden layers; an approximation, not the headline"}
-    del efg, model, g
+    # the table kernels alone (event-timed in one eager call) against their HBM bytes
+    emp.profile_enable(True)
+    emp.mp_energy_forces(model, g, sp)
+    torch.cuda.synchronize()
+    fam = {n: emp.profile_read(n) for n in ("radial_h2", "radial_bwd")}
+    emp.profile_enable(False)
+    E, T = g.n_edges, spec.n_layers
+    tab_bytes = {"radial_h2": T * E * (4 + 2 * 64 * 4), "radial_bwd": T * E * (4 + 64 * 4 + 12 + 2 * 12)}
+    out[WORKLOAD + "_radial_tables"] = {
+        "n_atoms": st.pos.shape[0], "n_edges": g.n_edges, "ms_per_step": round(ms, 4),
+        "edges_per_s": g.n_edges / (ms * 1e-3), "table_pieces": n_pieces, "timed": "CUDA-graph replay",
+        "table_kernels": {k: {"ms": round(v[0], 4), "alg_bytes": tab_bytes[k],
+                              "frac_of_hbm": round(tab_bytes[k] / (v[0] * 1e-3) / 1e9 / hbm_gbs, 3)}
+                          for k, v in fam.items()},
+        "note": "opt-in certified Chebyshev tables (degree 10, tol 1e-7) for the radial hidden layers; an "
+                "approximation, not the headline"}
+    del efg
+    # the weight gradient of the energy (the training path), eager, on the same frame
+    model.radial_tables(0.0)
+    for _ in range(2):
+        emp.mp_energy_weight_grad(model, g, sp)
+    torch.cuda.synchronize()
+    emp.profile_enable(True)
+    ms_g = timed(lambda: emp.mp_energy_weight_grad(model, g, sp))
+    red_ms = emp.profile_read("weight_grad")[0] / (steps + 3)
+    emp.profile_enable(False)
+    C = spec.C
+    # FLOPs of the sums over edges and nodes: the middle layers' SO(2) blocks, the radial W3 (C or 4C
+    # rows), W2, W1 of every layer, and the end layers' per-node W0 sums
+    flops = (2.0 * E * 72 * C * C * max(T - 2, 0)
+             + 2.0 * E * 64 * (C + 4 * C * (T - 1)) + 2.0 * T * E * (64 * 64 + 64 * 8)
+             + 2.0 * st.pos.shape[0] * (16 * C * C + 4 * C * C))
+    clk = _sm_clock_mhz(torch)
+    fp32_peak = 148 * 128 * 2 * clk * 1e6 / 1e12 if clk else None          # FMA lanes x 2 flops x SM clock
+    out[WORKLOAD + "_weight_grad"] = {
+        "ms_per_call": round(ms_g, 3), "edges_per_s": E / (ms_g * 1e-3), "timed": "eager call",
+        "reductions": {"ms": round(red_ms, 3), "flops": flops, "achieved_tflops": round(flops / (red_ms * 1e-3) / 1e12, 2),
+                       "bound": "alu", "peak_tflops": round(fp32_peak, 1) if fp32_peak else None,
+                       "frac": round(flops / (red_ms * 1e-3) / 1e12 / fp32_peak, 3) if fp32_peak else None,
+                       "peak_note": "FP32 FMA: 148 SMs x 128 lanes x 2 flops x the SM clock read at the start"},
+        "note": "energy, forces and dE/dW of every weight in one call"}
+    del model, g
     ci = synth.chain_inputs()
     ch = emp.Chain(ci.U, ci.M)
     x, gk, gy = (torch.from_numpy(t).cuda() for t in (ci.x, ci.g_kc, ci.g_y0))
@@ -371,6 +407,16 @@ def other_configs(emp, torch, stream, flush, hbm_gbs: float, steps: int = 10):
                            "frac_of_hbm": round(gbs / hbm_gbs, 3),
                            "note": "forward (x -> kc, y0) + input gradient (g_kc, g_y0 -> g_x) per call"}
     return out
+
+
+def _sm_clock_mhz(torch):
+    """Current SM clock of GPU 0 (nvidia-smi), or None."""
+    try:
+        outp = subprocess.run(["nvidia-smi", "--query-gpu=clocks.sm", "--format=csv,noheader,nounits", "-i",
+                               str(torch.cuda.current_device())], capture_output=True, text=True, timeout=20).stdout
+        return float(outp.strip().splitlines()[0])
+    except Exception:
+        return None
 
 
 # ------------------------------------------------------------------ our arm
