@@ -235,6 +235,8 @@ def alg_bytes_step(name: str, C: int, T: int, E: int, N: int) -> float:
         return last * (E * (4 * C * 4 + d0) + N * 4 * C * 4)
     if name == "last_bwd":                # R, D, r in; dE/dR hi/lo out, g_r and g_x read-modify-write
         return last * (E * (4 * C * 4 + d + 12 + 2 * 4 * C * 4 + 24) + N * 2 * row)
+    if name == "radial_fwd":              # d in; R out (C columns in the first layer, 4C after): the fused network
+        return E * (4 + C * 4) + (T - 1) * E * (4 + 4 * C * 4)
     if name == "radial_h2":               # d in; h2 hi/lo out
         return T * E * (4 + 2 * 64 * 4)
     if name == "radial_head":             # h2 hi/lo in; R out (C columns in the first layer, 4C after)
@@ -247,7 +249,7 @@ def alg_bytes_step(name: str, C: int, T: int, E: int, N: int) -> float:
 
 
 HBM_FAMILIES = ("rotate_in", "bwd_prep", "bwd_edge", "rotate_back_scatter", "first_fwd", "first_bwd", "last_fwd",
-                "last_bwd", "radial_h2", "radial_head", "radial_head_bwd", "radial_bwd")
+                "last_bwd", "radial_fwd", "radial_h2", "radial_head", "radial_head_bwd", "radial_bwd")
 
 
 def hbm_fractions(fam, steps: int, E: int, N: int, C: int, T: int, hbm_gbs: float):

@@ -16,6 +16,7 @@
 #include "chain_tc.cuh"
 #include "end_layers.cuh"
 #include "tables.cuh"
+#include "radial_tc.cuh"
 
 using namespace emp;
 
@@ -439,6 +440,15 @@ int radial_forward(const Model& m, const emp_graph* g, int t, const int* species
   const int C = m.spec.C;
   float* h2hi = at<float>(ws, L.h2hi);
   float* h2lo = at<float>(ws, L.h2lo);
+  if (!(m.tab_on && use_tables) && !h2_only) {
+    // the network itself: basis, hidden layers and head in one kernel (h2 stays on chip)
+    const MapPair* bm[tc::MAXSUB];
+    for (int p = 0; p < m.n_pairs; ++p) bm[p] = &(ncols == C ? m.w3n_maps : m.w3_maps)[(size_t)t * m.n_pairs + p];
+    const RadialArgs ra = radial_args(m, t);
+    Scope sc_("radial_fwd", s);
+    return rtc::radial_fwd(E, ncols, rr.off_dev, m.n_pairs, rr.perm, dist, ra.rad, ra.layer_off, ra.pair_stride, ra.rc,
+                           bm, R, at<int>(ws, L.counter), s);
+  }
   if (m.tab_on && use_tables) {
     Scope sc_("radial_h2", s);
     tab::k_radial_h2_table<<<(unsigned)std::min<long long>((E + 15) / 16, 16 * tc::num_sms()), tab::TAB_THREADS, 0, s>>>(
@@ -514,6 +524,8 @@ int ensure_attrs() {
   EMP_CUDA_TRY(cudaFuncSetAttribute(ctc::k_chain_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, ctc::smem_bytes(true)));
   EMP_CUDA_TRY(cudaFuncSetAttribute(ctc::k_chain_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, ctc::smem_bytes(false)));
   int st = so2_tc_init();
+  if (st != EMP_OK) return st;
+  st = rtc::init();
   if (st != EMP_OK) return st;
   g_attrs_set = true;
   return EMP_OK;

@@ -1,0 +1,513 @@
+// The radial network of a layer in one kernel (page "deepmd-kit PR #6108": edge
+// length -> radial basis -> radial network -> per-(l, channel) scales; the model's
+// network is 8 Bessel functions with the polynomial envelope, 8 -> 64 -> 64 with
+// SiLU, then the head 64 -> 4C):
+//   R[row] = W3 SiLU(W2 SiLU(W1 e(d_row)))
+// for the rows of one or several radial networks (species pairs), each over its own
+// device row range of the pair-sorted row list.
+//
+// Persistent kernel on CTA pairs (clusters of 2, cta_group::2); a tile is 256 rows
+// (128 per CTA) of one network.  In each CTA:
+//  - eight hidden warps evaluate the basis and the two hidden layers on SIMT (8 x 4
+//    register tiles, the same FP32 operation order as the standalone hidden-layer
+//    kernel) and write h2 split into TF32 hi and lo straight into the shared-memory
+//    A operand of the head, in the 64-byte-swizzled K-major layout the MMA
+//    descriptors read (two A buffers: the next tile's h2 is written while the head of
+//    the current one runs);
+//  - the leader's hidden warps take tiles from the counter and publish them to every
+//    role of both CTAs (so the next tile's hidden layers never wait for the head);
+//  - warp 0 streams the head weights W3 (hi, lo; this CTA's half of a 256-row tile per
+//    k-block) into a 3-stage TMA ring;
+//  - the leader's warp 1 issues the 3xTF32 head products into one of two TMEM
+//    accumulators per n-tile;
+//  - four epilogue warps store the R rows: TMEM -> registers -> a 128-byte-swizzled
+//    staging tile per warp -> one TMA bulk store per 32 x 32 block (plain masked stores
+//    for a block whose rows run past the network's range).
+// h2 never reaches global memory.  Every wait is bounded: on timeout the CTA records
+// a device error, stops, waits (bounded) for its own copies and MMAs and frees TMEM.
+#pragma once
+#include "so2_tc.cuh"
+#include "conv.cuh"
+
+namespace emp {
+namespace rtc {
+
+constexpr int BM = 128;                          // rows per CTA (256 per pair)
+constexpr int HID_WARPS = 8;
+constexpr int HID_THREADS = 32 * HID_WARPS;
+constexpr int HID_W0 = 6;                        // first hidden warp
+constexpr int THREADS = 32 * (HID_W0 + HID_WARPS);
+constexpr int KB = 4;                            // 16-wide k-blocks of h2 (K = 64)
+constexpr int AK_BYTES = BM * 64;                // one k-block of hi (or lo): 128 rows x 64 bytes
+constexpr int ABUF_BYTES = 2 * KB * AK_BYTES;    // hi k-blocks, then lo k-blocks: 64 KB
+constexpr int BST = 3;                           // W3 ring stages
+constexpr int BHALF = 128 * 64;                  // hi (or lo) half of a stage: up to 128 rows x 64 bytes
+constexpr int BSTAGE_BYTES = 2 * BHALF;
+constexpr int H1P = BM + 4;                      // pitch of the transposed hidden tile h1T[64][H1P]
+constexpr int W2P = 68;                          // pitch of W2T[64][W2P]
+constexpr int ACC_COLS = 256;                    // one accumulator
+constexpr int EPI_TILE = 32 * 128;                // one epilogue warp's 32 x 32 fp32 staging tile (128-byte swizzle)
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + 2 * ABUF_BYTES;
+constexpr int OFF_EPI = OFF_B + BST * BSTAGE_BYTES;
+constexpr int OFF_W2T = OFF_EPI + 4 * EPI_TILE;
+constexpr int OFF_W1 = OFF_W2T + 64 * W2P * 4;
+constexpr int OFF_E = OFF_W1 + 64 * 8 * 4;
+constexpr int OFF_D = OFF_E + BM * 8 * 4;
+constexpr int OFF_BAR = OFF_D + BM * 4;
+constexpr int BAR_BYTES = 512;
+constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;
+static_assert(SMEM <= 232448, "shared memory per CTA");
+static_assert(64 * H1P * 4 <= ABUF_BYTES, "h1T fits in an A buffer");
+static_assert(OFF_EPI % 1024 == 0, "swizzled staging tiles");
+
+struct Args {
+  int nsub;              // radial networks, each over rows [row_off[s], row_off[s + 1])
+  int mtiles;            // 256-row tiles per network (an upper bound when row_off is set)
+  int M;                 // rows (upper bound of every range)
+  int ncols, bn, ntiles; // output columns, MMA N, n-tiles per row tile
+  const int* row_off;    // device [nsub + 1], or null (one network over [0, M))
+  int* counter;          // tile counter (zeroed by the host)
+  float* out;            // R [M][ncols]
+  const int* perm;       // row -> edge, or null (identity)
+  const float* dist;     // edge lengths by edge
+  const float* rad;      // radial weights: per network W1 [64][8], W2 [64][64], ...
+  size_t layer_off, pair_stride;
+  float rc;
+};
+struct Maps {
+  CUtensorMap b_hi[tc::MAXSUB], b_lo[tc::MAXSUB];   // W3 rows [ncols][64], boxes of bn / 2 rows
+  CUtensorMap out;                                  // R [M][ncols], 32 x 32 boxes, 128-byte swizzle (stores)
+};
+
+__device__ __forceinline__ int row_base(const Args& a, int s) { return a.row_off ? a.row_off[s] : 0; }
+__device__ __forceinline__ int row_end(const Args& a, int s) { return a.row_off ? a.row_off[s + 1] : a.M; }
+
+// next row tile; tiles past a network's range are skipped along with the rest of that network
+__device__ __forceinline__ int next_tile(const Args& a, int total) {
+  int t = atomicAdd(a.counter, 1);
+  while (a.row_off && t < total) {
+    const int s = t / a.mtiles;
+    if ((t % a.mtiles) * 2 * BM < row_end(a, s) - row_base(a, s)) break;
+    atomicMax(a.counter, (s + 1) * a.mtiles);
+    t = atomicAdd(a.counter, 1);
+  }
+  return t;
+}
+
+__device__ __forceinline__ void hid_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_store(const CUtensorMap* map, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// the bulk stores this thread issued have read their shared-memory source
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// byte offset of element (row r, k) (k < 16) in a k-block of 64-byte rows, 64-byte swizzle
+__device__ __forceinline__ uint32_t swz(int r, int k) {
+  return (uint32_t)(r * 64 + ((((k >> 2) ^ (r >> 1)) & 3) << 4) + (k & 3) * 4);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    k_radial_fwd_tc(const __grid_constant__ Args g, const __grid_constant__ Maps maps, int total_tiles) {
+  using namespace tc;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);    // [BST] (the leader's are used)
+  uint64_t* empty = full + BST;                                    // [BST]
+  uint64_t* acc_full = empty + BST;                                // [2]
+  uint64_t* acc_empty = acc_full + 2;                              // [2] (the leader's are used)
+  uint64_t* a_full = acc_empty + 2;                                // [2] (the leader's are used)
+  uint64_t* a_empty = a_full + 2;                                  // [2]
+  uint64_t* drain = a_empty + 2;
+  uint64_t* tq_full = drain + 1;                                   // [TQ]
+  uint64_t* tq_empty = tq_full + TQ;                               // [TQ] (the leader's are used)
+  int* tq = reinterpret_cast<int*>(tq_empty + TQ);                 // [TQ]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tq + TQ);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int* issued = abort_flag + 1;
+  int* consumed = issued + 1;
+  int* hid_tile = consumed + 1;                                    // tile index broadcast to the hidden warps
+  float* epi = reinterpret_cast<float*>(smem + OFF_EPI);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < BST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 8);        // 4 epilogue warps in each CTA
+      mbar_init(&a_full[b], 2);           // the hidden warps of each CTA, once
+      mbar_init(&a_empty[b], 1);
+    }
+    mbar_init(drain, 1);
+    for (int j = 0; j < TQ; ++j) {
+      mbar_init(&tq_full[j], 1);
+      mbar_init(&tq_empty[j], 12);        // leader: producer, MMA, 4 epilogue; peer: producer, 4 epilogue, hidden
+    }
+    *abort_flag = 0;
+    *issued = 0;
+    *consumed = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"((uint32_t)TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  fence_before();
+  __syncthreads();
+  cluster_sync();
+  fence_after();
+  const uint32_t tmem = *tmem_slot;
+  volatile int* vabort = abort_flag;
+  const uint32_t full_l = map_to_rank(smem_u32(full), 0);
+  const uint32_t acc_empty_l = map_to_rank(smem_u32(acc_empty), 0);
+  const uint32_t a_full_l = map_to_rank(smem_u32(a_full), 0);
+  const uint32_t tq_empty_l = map_to_rank(smem_u32(tq_empty), 0);
+  const int bh = g.bn / 2;                 // this CTA's W3 rows per n-tile
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------------- W3 producer (both CTAs)
+    int it = 0;
+    for (int j = 0;; ++j) {
+      const int slot = j % TQ;
+      if (!mbar_wait_cluster(&tq_full[slot], (j / TQ) & 1)) { *vabort = 1; break; }
+      const int t = tq[slot];
+      if (leader) mbar_arrive(&tq_empty[slot]);
+      else remote_arrive(tq_empty_l + (uint32_t)(slot * 8));
+      if (t >= total_tiles) break;
+      const int sub = t / g.mtiles;
+      bool stop = false;
+      for (int n = 0; n < g.ntiles && !stop; ++n)
+        for (int kc = 0; kc < KB; ++kc, ++it) {
+          const int s = it % BST;
+          if (it >= BST && !mbar_wait(&empty[s], ((it / BST) - 1) & 1)) { *vabort = 1; stop = true; break; }
+          if (*vabort) { stop = true; break; }   // the scheduler then publishes the end to every role
+          unsigned char* st = smem + OFF_B + s * BSTAGE_BYTES;
+          if (leader) mbar_expect_tx(&full[s], 2 * 2 * bh * 64);
+          const uint32_t fb = full_l + (uint32_t)(s * 8);
+          tma_load_pair(st, &maps.b_hi[sub], fb, kc * BK, n * g.bn + (int)rank * bh);
+          tma_load_pair(st + BHALF, &maps.b_lo[sub], fb, kc * BK, n * g.bn + (int)rank * bh);
+          *issued = it + 1;
+        }
+    }
+  } else if (warp == 1 && lane == 0 && leader) {
+    // ---------------------------------------------------------------- head MMA issuer (leader only)
+    int it = 0, i = 0;
+    bool ok = true;
+    const uint32_t idesc = idesc_pair(g.bn);
+    for (int j = 0; ok; ++j) {
+      const int slot = j % TQ;
+      if (!mbar_wait(&tq_full[slot], (j / TQ) & 1)) { ok = false; break; }
+      const int t = tq[slot];
+      mbar_arrive(&tq_empty[slot]);
+      if (t >= total_tiles) break;
+      const int ab = j & 1;
+      if (!mbar_wait_cluster(&a_full[ab], (j >> 1) & 1)) { ok = false; break; }
+      fence_after();
+      const uint32_t a_base = smem_u32(smem + OFF_A + ab * ABUF_BYTES);
+      for (int n = 0; n < g.ntiles; ++n, ++i) {
+        const int buf = i & 1;
+        if (i >= 2 && !mbar_wait_cluster(&acc_empty[buf], ((i >> 1) - 1) & 1)) { ok = false; break; }
+        fence_after();
+        const uint32_t d = tmem + (uint32_t)(buf * ACC_COLS);
+        for (int kc = 0; kc < KB; ++kc, ++it) {
+          const int s = it % BST;
+          if (!mbar_wait(&full[s], (it / BST) & 1)) { ok = false; break; }
+          *consumed = it + 1;
+          fence_after();
+          const uint32_t a_hi = a_base + kc * AK_BYTES;
+          const uint32_t a_lo = a_hi + KB * AK_BYTES;
+          const uint32_t b_hi = smem_u32(smem + OFF_B + s * BSTAGE_BYTES);
+          const uint32_t b_lo = b_hi + BHALF;
+#pragma unroll
+          for (int kk = 0; kk < BK / 8; ++kk) {
+            const uint32_t off = kk * 32;
+            mma_tf32_pair(d, sdesc(a_lo + off), sdesc(b_hi + off), idesc, (kc | kk) ? 1u : 0u);
+            mma_tf32_pair(d, sdesc(a_hi + off), sdesc(b_lo + off), idesc, 1u);
+            mma_tf32_pair(d, sdesc(a_hi + off), sdesc(b_hi + off), idesc, 1u);
+          }
+          mma_commit_pair(&empty[s]);
+        }
+        if (!ok) break;
+        mma_commit_pair(&acc_full[buf]);
+      }
+      if (!ok) break;
+      mma_commit_pair(&a_empty[ab]);     // both CTAs may overwrite this h2 buffer once these MMAs are done
+    }
+    if (!ok) *vabort = 1;
+    mma_commit_pair(drain);
+    mbar_wait(drain, 0);
+  } else if (warp >= 2 && warp < HID_W0) {
+    // ---------------------------------------------------------------- epilogue (both CTAs: own 128 rows)
+    const int q = warp & 3;
+    int i = 0;
+    for (int j = 0;; ++j) {
+      const int slot = j % TQ;
+      if (!mbar_wait_cluster(&tq_full[slot], (j / TQ) & 1)) { *vabort = 1; break; }
+      const int t = tq[slot];
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(&tq_empty[slot]);
+        else remote_arrive(tq_empty_l + (uint32_t)(slot * 8));
+      }
+      if (t >= total_tiles) break;
+      const int sub = t / g.mtiles;
+      const int mw = row_base(g, sub) + (t % g.mtiles) * 2 * BM + (int)rank * BM + q * 32;
+      const int mend = row_end(g, sub);
+      bool ok = true;
+      for (int n = 0; n < g.ntiles; ++n, ++i) {
+        const int buf = i & 1;
+        if (!mbar_wait(&acc_full[buf], (i >> 1) & 1)) { ok = false; break; }
+        fence_after();
+        float* obase = g.out + (size_t)n * g.bn;
+        unsigned char* stg = smem + OFF_EPI + q * EPI_TILE;
+        const bool whole = mw + 32 <= mend;        // else the rows past the range are masked
+#pragma unroll 1
+        for (int cc = 0; cc < g.bn; cc += 32) {
+          float v[32];
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * ACC_COLS + cc), v);
+          if (lane == 0) bulk_wait_read();         // this warp's previous store has left the staging tile
+          __syncwarp();
+          // row `lane` as eight 16-byte chunks, chunk c at position c ^ (row & 7)
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<float4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+          if (whole) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // staged by threads, read by the copy engine
+            __syncwarp();
+            if (lane == 0) tma_store(&maps.out, stg, n * g.bn + cc, mw);
+          } else {
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int rr = k * 4 + (lane >> 3), c = lane & 7;
+              const int m = mw + rr;
+              const float4 w = *reinterpret_cast<const float4*>(stg + rr * 128 + ((c ^ (rr & 7)) << 4));
+              if (m < mend) *reinterpret_cast<float4*>(obase + (size_t)m * g.ncols + cc + 4 * c) = w;
+            }
+            __syncwarp();
+          }
+        }
+        fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (leader) mbar_arrive(&acc_empty[buf]);
+          else remote_arrive(acc_empty_l + (uint32_t)(buf * 8));
+        }
+      }
+      if (!ok) { *vabort = 1; break; }
+    }
+    if (lane == 0) bulk_wait_all();
+  } else if (warp >= HID_W0) {
+    // ---------------------------------------------------------------- hidden layers -> h2 hi/lo in the A buffer
+    const int h = threadIdx.x - 32 * HID_W0;
+    const int r0 = (h >> 4) * 8, j0 = (h & 15) * 4;
+    float* W2T = reinterpret_cast<float*>(smem + OFF_W2T);     // [i][o] = W2[o][i]
+    float* W1T = reinterpret_cast<float*>(smem + OFF_W1);      // [n][j] = W1[j][n]
+    float* sE = reinterpret_cast<float*>(smem + OFF_E);        // [r][n]
+    float* sD = reinterpret_cast<float*>(smem + OFF_D);
+    int staged = -1;
+    for (int j = 0;; ++j) {
+      const int slot = j % TQ;
+      const int ab = j & 1;
+      if (h == 0) {
+        int t;
+        if (leader) {
+          // the scheduler: the next tile for the pair, published to every role of both CTAs
+          if (j >= TQ && !mbar_wait_cluster(&tq_empty[slot], ((j / TQ) - 1) & 1)) { *vabort = 1; t = total_tiles; }
+          else t = *vabort ? total_tiles : next_tile(g, total_tiles);
+          tq[slot] = t;
+          remote_store(map_to_rank(smem_u32(&tq[slot]), 1), t);
+          mbar_arrive(&tq_full[slot]);
+          remote_arrive(map_to_rank(smem_u32(&tq_full[slot]), 1));
+        } else if (mbar_wait_cluster(&tq_full[slot], (j / TQ) & 1)) {
+          t = tq[slot];
+          remote_arrive(tq_empty_l + (uint32_t)(slot * 8));
+        } else {
+          t = -1;
+        }
+        if (t >= 0 && t < total_tiles && j >= 2 && !mbar_wait(&a_empty[ab], ((j >> 1) - 1) & 1)) t = -1;
+        if (t < 0) { *vabort = 1; t = total_tiles; }
+        *hid_tile = t;
+      }
+      hid_sync();
+      const int t = *hid_tile;
+      if (t >= total_tiles) break;
+      const int sub = t / g.mtiles;
+      const int base = row_base(g, sub) + (t % g.mtiles) * 2 * BM + (int)rank * BM;
+      const int rend = row_end(g, sub);
+      if (h < BM) {
+        const int r = base + h;
+        float d = 1.f;
+        if (r < rend) d = g.dist[g.perm ? g.perm[r] : r];
+        sD[h] = d;
+      }
+      if (sub != staged) {
+        const float* w1 = g.rad + g.layer_off + (size_t)sub * g.pair_stride;
+        const float* w2 = w1 + 64 * 8;
+        for (int idx = h; idx < 64 * 8; idx += HID_THREADS) W1T[(idx & 7) * 64 + (idx >> 3)] = __ldg(&w1[idx]);
+        for (int idx = h; idx < 64 * 64; idx += HID_THREADS) W2T[(idx & 63) * W2P + (idx >> 6)] = __ldg(&w2[idx]);
+        staged = sub;
+      }
+      hid_sync();
+      for (int idx = h; idx < BM * 8; idx += HID_THREADS) {
+        float ev, dv;
+        bessel_n(sD[idx >> 3], g.rc, idx & 7, ev, dv);
+        sE[idx] = ev;
+      }
+      hid_sync();
+      // layer 1: z1[r][j] = sum_n W1[j][n] e[r][n], h1 = SiLU(z1) stored transposed in the A buffer
+      float* h1T = reinterpret_cast<float*>(smem + OFF_A + ab * ABUF_BYTES);
+      float z[8][4];
+      float w1v[8][4];
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+        const float4 w = *reinterpret_cast<const float4*>(W1T + n * 64 + j0);
+        w1v[n][0] = w.x; w1v[n][1] = w.y; w1v[n][2] = w.z; w1v[n][3] = w.w;
+      }
+#pragma unroll
+      for (int a = 0; a < 8; ++a) {
+        const float4 ea = *reinterpret_cast<const float4*>(sE + (r0 + a) * 8);
+        const float4 eb = *reinterpret_cast<const float4*>(sE + (r0 + a) * 8 + 4);
+        const float ev[8] = {ea.x, ea.y, ea.z, ea.w, eb.x, eb.y, eb.z, eb.w};
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          float acc = 0.f;
+#pragma unroll
+          for (int n = 0; n < 8; ++n) acc = fmaf(w1v[n][b], ev[n], acc);
+          z[a][b] = acc;
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        float* dst = h1T + (j0 + b) * H1P + r0;
+        *reinterpret_cast<float4*>(dst) =
+            make_float4(silu_fast(z[0][b]), silu_fast(z[1][b]), silu_fast(z[2][b]), silu_fast(z[3][b]));
+        *reinterpret_cast<float4*>(dst + 4) =
+            make_float4(silu_fast(z[4][b]), silu_fast(z[5][b]), silu_fast(z[6][b]), silu_fast(z[7][b]));
+      }
+      hid_sync();
+      // layer 2: z2[r][o] = sum_i W2[o][i] h1[r][i]
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) z[a][b] = 0.f;
+#pragma unroll 4
+      for (int i2 = 0; i2 < 64; ++i2) {
+        const float4 ha = *reinterpret_cast<const float4*>(h1T + i2 * H1P + r0);
+        const float4 hb = *reinterpret_cast<const float4*>(h1T + i2 * H1P + r0 + 4);
+        const float4 w = *reinterpret_cast<const float4*>(W2T + i2 * W2P + j0);
+        const float hv[8] = {ha.x, ha.y, ha.z, ha.w, hb.x, hb.y, hb.z, hb.w}, wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int a = 0; a < 8; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) z[a][b] = fmaf(hv[a], wv[b], z[a][b]);
+      }
+      hid_sync();                          // every read of h1T is done before h2 overwrites the buffer
+      unsigned char* abuf = smem + OFF_A + ab * ABUF_BYTES + (j0 >> 4) * AK_BYTES;
+#pragma unroll
+      for (int a = 0; a < 8; ++a) {
+        float hi[4], lo[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const float v = silu_fast(z[a][b]);
+          hi[b] = tf32_rna(v);
+          lo[b] = tf32_rna(v - hi[b]);
+        }
+        const uint32_t o = swz(r0 + a, j0 & 15);
+        *reinterpret_cast<float4*>(abuf + o) = make_float4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<float4*>(abuf + KB * AK_BYTES + o) = make_float4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // h2 written by threads, read by the MMAs
+      hid_sync();
+      if (h == 0) {
+        if (leader) mbar_arrive(&a_full[ab]);
+        else remote_arrive(a_full_l + (uint32_t)(ab * 8));
+      }
+    }
+  }
+  fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (threadIdx.x == 0 && leader && *vabort) {
+    // let W3 loads of either CTA still in flight land (they complete on the leader's barriers)
+    const int peer_issued = remote_load(map_to_rank(smem_u32(issued), 1));
+    const int last = max(*issued, peer_issued);
+    for (int it = *consumed; it < last; ++it) mbar_wait(&full[it % BST], (it / BST) & 1);
+  }
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)TMEM_COLS));
+  }
+}
+
+inline int init() {
+  if (cudaFuncSetAttribute(k_radial_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
+    return EMP_ERR_CUDA;
+  return EMP_OK;
+}
+
+// R rows [M][ncols] of nsub radial networks over their row ranges (row_off, device; or one network
+// over [0, M) when null); b_maps[s]: network s's W3 (hi, lo) maps with boxes of tile_n(ncols) / 2 rows.
+inline int radial_fwd(long long M, int ncols, const int* row_off, int nsub, const int* perm, const float* dist,
+                      const float* rad, size_t layer_off, size_t pair_stride, float rc, const MapPair* const* b_maps,
+                      float* out, int* counter, cudaStream_t s) {
+  if (M <= 0) return EMP_OK;
+  if (nsub < 1 || nsub > tc::MAXSUB || M >= (1ll << 31) || ncols < 32 || ncols % 32 != 0) return EMP_ERR_ARG;
+  Args g{};
+  Maps maps;
+  g.nsub = nsub;
+  g.M = (int)M;
+  g.mtiles = (int)((M + 2 * BM - 1) / (2 * BM));
+  g.ncols = ncols;
+  g.bn = tc::tile_n(ncols);
+  if (g.bn / 2 > 128 || ncols % g.bn != 0) return EMP_ERR_ARG;
+  g.ntiles = ncols / g.bn;
+  g.row_off = row_off;
+  g.counter = counter;
+  g.out = out;
+  g.perm = perm;
+  g.dist = dist;
+  g.rad = rad;
+  g.layer_off = layer_off;
+  g.pair_stride = pair_stride;
+  g.rc = rc;
+  for (int q = 0; q < nsub; ++q) {
+    maps.b_hi[q] = b_maps[q]->hi;
+    maps.b_lo[q] = b_maps[q]->lo;
+  }
+  {
+    auto fn = tc::encode_fn();
+    if (!fn) return EMP_ERR_UNSUPPORTED;
+    cuuint64_t dims[2] = {(cuuint64_t)ncols, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)ncols * 4};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(&maps.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, out, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return EMP_ERR_CUDA;
+  }
+  const long long total = (long long)nsub * g.mtiles;
+  if (total >= (1ll << 31)) return EMP_ERR_UNSUPPORTED;
+  if (cudaMemsetAsync(counter, 0, sizeof(int), s) != cudaSuccess) return EMP_ERR_CUDA;
+  const int pairs = (int)std::min<long long>(total, tc::num_sms() / 2);
+  k_radial_fwd_tc<<<2 * pairs, THREADS, SMEM, s>>>(g, maps, (int)total);
+  return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
+}
+
+}  // namespace rtc
+}  // namespace emp
