@@ -247,7 +247,8 @@ __global__ void __launch_bounds__(RAD_THREADS) k_radial_h2(long long E, const in
   }
 }
 
-// dE/dd from dE/dh2 (rows gh2 [E][64], the tensor-core product dE/dR W3); adds (dE/dd) rhat to g_r.
+// dE/dd from dE/dh2 (rows gh2 [E][64], the tensor-core product dE/dR W3); adds (dE/dd) rhat to g_r
+// (when g_r is not null).
 // With rows_out (weight gradients), also each row's basis e [8], h1 [64], dE/dz1 [64] and
 // dE/dz2 [64] into rows_out[row][200], for the sums dE/dW2 = sum dE/dz2 (x) h1 and
 // dE/dW1 = sum dE/dz1 (x) e.
@@ -345,7 +346,7 @@ __global__ void __launch_bounds__(RAD_THREADS) k_radial_bwd(long long E, const i
     for (int q = 0; q < 4; ++q)
 #pragma unroll
       for (int off = 8; off >= 1; off >>= 1) part[q] += __shfl_xor_sync(0xffffffffu, part[q], off);
-    if ((t & 15) == 0) {
+    if ((t & 15) == 0 && g_r) {
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         if (s.pair[r0 + q] != p) continue;

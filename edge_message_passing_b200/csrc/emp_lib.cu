@@ -472,10 +472,12 @@ int radial_forward(const Model& m, const emp_graph* g, int t, const int* species
   return tc_group(E, ncols, subs, m.n_pairs, at<int>(ws, L.counter), s, rr.off_dev);
 }
 
-// dE/dd of layer t from dE/dR (rows split hi/lo): dE/dh2 = dE/dR W3 on the tensor cores, then the
-// hidden layers' backward on SIMT; adds (dE/dd) rhat to g_r
+// dE/dd of layer t from dE/dR (rows split hi/lo), added as (dE/dd) rhat to g_r: with the network, one
+// kernel (head transpose, recomputed hidden layers and their backward; radial_tc.cuh); with the
+// tables, dE/dh2 = dE/dR W3 on the tensor cores, then the tables' derivative
 // kcols: 4C, or C when only the degree-0 scales carry a gradient (the first layer)
-// rows_out (weight gradients; network only): each row's e, h1, dE/dz1, dE/dz2 (k_radial_bwd)
+// rows_out (weight gradients; network only): also each row's e, h1, dE/dz1, dE/dz2 (dE/dh2 on the
+// tensor cores, then k_radial_bwd without the g_r update)
 int radial_backward(const Model& m, const emp_graph* g, int t, const int* species, const float* dist,
                     const RadialRows& rr, float* g_r, void* ws, const WsLayout& L, cudaStream_t s, int kcols,
                     bool use_tables = true, float* rows_out = nullptr) {
@@ -484,6 +486,22 @@ int radial_backward(const Model& m, const emp_graph* g, int t, const int* specie
   float* gRhi = at<float>(ws, L.gRhi);
   float* gRlo = at<float>(ws, L.gRlo);
   float* gh2 = at<float>(ws, L.gh2);
+  if (!(m.tab_on && use_tables)) {
+    // the network itself: head transpose, recomputed hidden layers and their backward in one kernel
+    MapPair a;
+    int st = make_pair(&a, gRhi, gRlo, E, 4 * C, 4 * C, tc::BM);
+    if (st != EMP_OK) return st;
+    const MapPair* bm[tc::MAXSUB];
+    for (int p = 0; p < m.n_pairs; ++p) bm[p] = &m.w3t_maps[(size_t)t * m.n_pairs + p];
+    const RadialArgs ra = radial_args(m, t);
+    {
+      Scope sc_("radial_bwd", s);
+      st = rtc::radial_bwd(E, kcols, rr.off_dev, m.n_pairs, rr.perm, dist, g->vec, g_r, ra.rad, ra.layer_off,
+                           ra.pair_stride, ra.rc, a, bm, at<int>(ws, L.counter), s);
+    }
+    if (st != EMP_OK || !rows_out) return st;
+    g_r = nullptr;          // weight gradients: the per-row values below, g_r already done
+  }
   {
     MapPair a;
     int st = make_pair(&a, gRhi, gRlo, E, 4 * C, 4 * C, tc::BM);
@@ -502,7 +520,7 @@ int radial_backward(const Model& m, const emp_graph* g, int t, const int* specie
     tab::k_radial_bwd_table<<<(unsigned)std::min<long long>((E + 15) / 16, 16 * tc::num_sms()), tab::TAB_THREADS, 0, s>>>(
         E, rr.perm, dist, g->vec, g->recv, g->send, species, table_args(m, t), gh2, g_r);
   } else {
-    Scope sc_("radial_bwd", s);
+    Scope sc_("radial_rows", s);
     k_radial_bwd<<<(unsigned)std::min<long long>((E + RT - 1) / RT, 2 * tc::num_sms()), RAD_THREADS, sizeof(RadialSmem), s>>>(
         E, rr.perm, dist, g->vec, g->recv, g->send, species, radial_args(m, t), gh2, g_r, rows_out);
   }
