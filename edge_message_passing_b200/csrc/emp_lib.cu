@@ -98,9 +98,11 @@ WsLayout ws_layout(const Model& m, long long E, int N, bool grad = false) {
   L.rbP = take(((coh + RB_CHUNK - 1) / RB_CHUNK) * 2 * 16 * C * 4);
   L.gRhi = take((size_t)E * 4 * C * 4);
   L.gRlo = take((size_t)E * 4 * C * 4);
-  L.h2hi = take((size_t)E * 64 * 4);
-  L.h2lo = take((size_t)E * 64 * 4);
-  L.gh2 = take((size_t)E * 64 * 4);
+  if (grad || m.tab_on) {   // per-row radial hidden values: only the tables' path and the weight gradients
+    L.h2hi = take((size_t)E * 64 * 4);
+    L.h2lo = take((size_t)E * 64 * 4);
+    L.gh2 = take((size_t)E * 64 * 4);
+  }
   L.pperm = take((size_t)E * 4);
   L.pinv = take((size_t)E * 4);
   L.poff = take(64 * 4);
@@ -117,15 +119,17 @@ WsLayout ws_layout(const Model& m, long long E, int N, bool grad = false) {
   const size_t cb = coh * 16 * C * 4;
   L.gxP = take(cb);
   L.gxP2 = take(cb);        // run pieces of every other cohort (the backward's sender sums)
-  L.XT2 = take(cb);
-  L.XTlo2 = take(cb);
-  L.Y2 = take(cb);
-  L.XT = take(cb);
-  L.Y = take(cb);
-  L.GXT = take(cb);
-  L.XTlo = take(cb);
-  L.GYhi = take(cb);
-  L.GYlo = take(cb);
+  // the per-edge product operands and results hold two cohorts (one product launch per pair of
+  // cohorts); the second cohort's rows start one cohort in (XT2, XTlo2, Y2)
+  L.XT = take(2 * cb);
+  L.XT2 = L.XT + cb;
+  L.XTlo = take(2 * cb);
+  L.XTlo2 = L.XTlo + cb;
+  L.Y = take(2 * cb);
+  L.Y2 = L.Y + cb;
+  L.GXT = take(2 * cb);
+  L.GYhi = take(2 * cb);
+  L.GYlo = take(2 * cb);
   L.perm = take((size_t)E * 4);
   L.seg = take((size_t)E * 4);
   L.nseg = take(ncoh * 4 + 4);
@@ -443,7 +447,7 @@ int radial_forward(const Model& m, const emp_graph* g, int t, const int* species
   if (!(m.tab_on && use_tables) && !h2_only) {
     // the network itself: basis, hidden layers and head in one kernel (h2 stays on chip)
     const MapPair* bm[tc::MAXSUB];
-    for (int p = 0; p < m.n_pairs; ++p) bm[p] = &(ncols == C ? m.w3n_maps : m.w3_maps)[(size_t)t * m.n_pairs + p];
+    for (int p = 0; p < m.n_pairs; ++p) bm[p] = &(ncols == C ? m.w3fn_maps : m.w3f_maps)[(size_t)t * m.n_pairs + p];
     const RadialArgs ra = radial_args(m, t);
     Scope sc_("radial_fwd", s);
     return rtc::radial_fwd(E, ncols, rr.off_dev, m.n_pairs, rr.perm, dist, ra.rad, ra.layer_off, ra.pair_stride, ra.rc,
@@ -928,11 +932,15 @@ int mp_model_create(const emp_model_spec* spec, const float* weights, size_t n_f
     }
   m->w3_maps.resize(T * m->n_pairs);
   m->w3n_maps.resize(T * m->n_pairs);
+  m->w3f_maps.resize(T * m->n_pairs);
+  m->w3fn_maps.resize(T * m->n_pairs);
   m->w3t_maps.resize(T * m->n_pairs);
   for (size_t q = 0; q < T * m->n_pairs; ++q) {
     const size_t wo = q * m->w3_stride();
     if (make_pair(&m->w3_maps[q], m->w3_hi + wo, m->w3_lo + wo, 4 * C, 64, 64, tc::b_box_rows(4 * (int)C)) != EMP_OK ||
         make_pair(&m->w3n_maps[q], m->w3_hi + wo, m->w3_lo + wo, C, 64, 64, tc::b_box_rows((int)C)) != EMP_OK ||
+        make_pair(&m->w3f_maps[q], m->w3_hi + wo, m->w3_lo + wo, 4 * C, 64, 64, rtc::fwd_bn(4 * (int)C) / 2) != EMP_OK ||
+        make_pair(&m->w3fn_maps[q], m->w3_hi + wo, m->w3_lo + wo, C, 64, 64, rtc::fwd_bn((int)C) / 2) != EMP_OK ||
         make_pair(&m->w3t_maps[q], m->w3t_hi + wo, m->w3t_lo + wo, 64, 4 * (int)C, 4 * (int)C, tc::b_box_rows(64)) !=
             EMP_OK)
       return fail(EMP_ERR_CUDA);
@@ -1175,10 +1183,10 @@ static int energy_forces_impl(const Model& m, const emp_graph* g, const int32_t*
   const float inv_avg = 1.0f / m.spec.avg_degree;
   int* counter = at<int>(ws, L.counter);
   Side side = side_for(stream);
-  CohortMaps am_xt, am_gy;
-  st = am_xt.build(C, E, coh, XT, XTlo);
+  CohortMaps am_xt, am_gy;                 // pairs of cohorts (the backward's product launches)
+  st = am_xt.build(C, E, 2 * coh, XT, XTlo);
   if (st != EMP_OK) return st;
-  st = am_gy.build(C, E, coh, GYhi, GYlo);
+  st = am_gy.build(C, E, 2 * coh, GYhi, GYlo);
   if (st != EMP_OK) return st;
 
   EMP_CUDA_TRY(cudaMemsetAsync(g_r, 0, (size_t)E * 12 + 4, stream));
@@ -1304,41 +1312,48 @@ static int energy_forces_impl(const Model& m, const emp_graph* g, const int32_t*
       { Scope sc_("last_bwd", stream); k_last_bwd<<<nb_node, C, 0, stream>>>(C, g->recv_off, g->send, rr.inv, g->vec, D, R, xt, nodeX, gRhi, gRlo, g_r, gxb); }
     } else if (E > 0) {
       // [per-edge product launches: begin]
+      // Cohorts are taken two at a time: one backward prep and one grouped product launch (the
+      // recomputed forward blocks and the transposed blocks) over both, then the per-edge backward
+      // and the sender sums cohort by cohort, in order.
       int ci = 0;
-      for (long long e0 = 0; e0 < E; e0 += coh, ++ci) {
-        const long long e1 = std::min(E, e0 + coh), n = e1 - e0;
+      for (long long g0 = 0; g0 < E; g0 += 2 * coh) {
+        const long long g1 = std::min(E, g0 + 2 * coh), M = g1 - g0;
         {
-          const int per = rs_per(n, tc::num_sms(), 3);
+          const int per = rs_per(M, tc::num_sms(), 3);
           Scope sc_("bwd_prep", stream);
-          k_rotate_staged<true, RS_V_BWD><<<(unsigned)((n + per - 1) / per), C / RS_V_BWD, rs_smem_bytes(C, true), stream>>>(
-              e0, e1, C, per, g->recv, g->send, rr.inv, D, R, xt, gS, XT, XTlo, GYhi, GYlo);
+          k_rotate_staged<true, RS_V_BWD><<<(unsigned)((M + per - 1) / per), C / RS_V_BWD, rs_smem_bytes(C, true), stream>>>(
+              g0, g1, C, per, g->recv, g->send, rr.inv, D, R, xt, gS, XT, XTlo, GYhi, GYlo);
         }
-        So2Part parts[2] = {{am_xt.get(n), &m.bmaps_fwd[t], Y}, {am_gy.get(n), &m.bmaps_bwd[t], GXT}};
-        st = so2_product(m, n, parts, 2, counter, stream);
+        So2Part parts[2] = {{am_xt.get(M), &m.bmaps_fwd[t], Y}, {am_gy.get(M), &m.bmaps_bwd[t], GXT}};
+        st = so2_product(m, M, parts, 2, counter, stream);
         if (st != EMP_OK) return st;
-        if (wgrad)   // dB_b += sum over the cohort's edges of g_y (x) x~ per block (both as their hi + lo)
+        if (wgrad)   // dB_b += sum over the cohorts' edges of g_y (x) x~ per block (both as their hi + lo)
           for (int b = 0; b < 4; ++b) {
             const int K = blk_width(b) * C, o = blk_off(b) * C;
-            tn_sum(K, K, (int)n, 1, GYhi + o, GYlo + o, 16ll * C, 0, XT + o, XTlo + o, 16ll * C, 0,
+            tn_sum(K, K, (int)M, 1, GYhi + o, GYlo + o, 16ll * C, 0, XT + o, XTlo + o, 16ll * C, 0,
                    dB + (size_t)wblk_off(b) * C * C, K, true, tnp, tn_part_floats(C), stream);
           }
-        // per-edge backward and the sender sums of dE/dx_send into gxb
-        const int per = be_per(n, tc::num_sms());
-        const int nb = (int)((n + per - 1) / per);
-        // run pieces in two buffers, cohort by cohort in turn: the combine of the cohort before
-        // last has read this one (the last combine may still run beside this kernel)
-        float* Pg = at<float>(ws, ci & 1 ? L.gxP2 : L.gxP);
-        side.wait_second_last();
-        {
-          Scope sc_("bwd_edge", stream);
-          k_bwd_edge<BE_V><<<nb, C / BE_V, be_smem_bytes(C), stream>>>(e0, e1, C, per, g->send, rr.inv, g->vec, D, R,
-                                                             xt, Y, gS, GXT, g->recv, perm, gRhi, gRlo, g_r, Pg);
+        for (long long e0 = g0; e0 < g1; e0 += coh, ++ci) {
+          const long long e1 = std::min(g1, e0 + coh), n = e1 - e0;
+          const size_t ro = (size_t)(e0 - g0) * 16 * C;     // the cohort's rows in the pair's buffers
+          // per-edge backward and the sender sums of dE/dx_send into gxb
+          const int per = be_per(n, tc::num_sms());
+          const int nb = (int)((n + per - 1) / per);
+          // run pieces in two buffers, cohort by cohort in turn: the combine of the cohort before
+          // last has read this one (the last combine may still run beside this kernel)
+          float* Pg = at<float>(ws, ci & 1 ? L.gxP2 : L.gxP);
+          side.wait_second_last();
+          {
+            Scope sc_("bwd_edge", stream);
+            k_bwd_edge<BE_V><<<nb, C / BE_V, be_smem_bytes(C), stream>>>(e0, e1, C, per, g->send, rr.inv, g->vec, D, R,
+                                                               xt, Y + ro, gS, GXT + ro, g->recv, perm, gRhi, gRlo, g_r, Pg);
+          }
+          side.run([&](cudaStream_t q) {
+            Scope sc_("gx_combine", q);
+            k_gx_combine<<<(unsigned)std::min<long long>(n, 2048), C, 0, q>>>(e0, e1, C, ci, per, g->send, perm, seg,
+                                                                            nseg, Pg, gxb);
+          });
         }
-        side.run([&](cudaStream_t q) {
-          Scope sc_("gx_combine", q);
-          k_gx_combine<<<(unsigned)std::min<long long>(n, 2048), C, 0, q>>>(e0, e1, C, ci, per, g->send, perm, seg,
-                                                                          nseg, Pg, gxb);
-        });
       }
       side.wait();        // g_x of this layer complete
       // [per-edge product launches: end]

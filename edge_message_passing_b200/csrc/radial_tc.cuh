@@ -40,26 +40,32 @@ constexpr int THREADS = 32 * (HID_W0 + HID_WARPS);
 constexpr int KB = 4;                            // 16-wide k-blocks of h2 (K = 64)
 constexpr int AK_BYTES = BM * 64;                // one k-block of hi (or lo): 128 rows x 64 bytes
 constexpr int ABUF_BYTES = 2 * KB * AK_BYTES;    // hi k-blocks, then lo k-blocks: 64 KB
-constexpr int BST = 3;                           // W3 ring stages
-constexpr int BHALF = 128 * 64;                  // hi (or lo) half of a stage: up to 128 rows x 64 bytes
+constexpr int BST = 4;                           // W3 ring stages
+constexpr int BHALF = 64 * 64;                   // hi (or lo) half of a stage: up to 64 rows x 64 bytes
 constexpr int BSTAGE_BYTES = 2 * BHALF;
-constexpr int H1P = BM + 4;                      // pitch of the transposed hidden tile h1T[64][H1P]
-constexpr int W2P = 68;                          // pitch of W2T[64][W2P]
-constexpr int ACC_COLS = 256;                    // one accumulator
-constexpr int EPI_TILE = 32 * 128;                // one epilogue warp's 32 x 32 fp32 staging tile (128-byte swizzle)
-constexpr int OFF_A = 0;
+constexpr int NACC = 3;                          // head accumulators (ring of n-tiles)
+constexpr int ACC_COLS = 128;                    // one head accumulator (MMA N <= 128)
+constexpr int ZCOL = NACC * ACC_COLS;            // z2, 64 columns
+constexpr int TMEM_FWD = 512;
+constexpr int EPI_TILE = 32 * 128;               // a 32 x 32 fp32 staging tile (128-byte swizzle)
+constexpr int OFF_A = 0;                         // two A buffers: h1, then h2 (hi k-blocks, then lo)
 constexpr int OFF_B = OFF_A + 2 * ABUF_BYTES;
-constexpr int OFF_EPI = OFF_B + BST * BSTAGE_BYTES;
-constexpr int OFF_W2T = OFF_EPI + 4 * EPI_TILE;
-constexpr int OFF_W1 = OFF_W2T + 64 * W2P * 4;
+constexpr int OFF_EPI = OFF_B + BST * BSTAGE_BYTES;   // two staging tiles per epilogue warp
+constexpr int OFF_W2 = OFF_EPI + 8 * EPI_TILE;   // W2 (B of z2): this CTA's 32 rows, hi then lo
+constexpr int OFF_W1 = OFF_W2 + 2 * KB * 32 * 64;
 constexpr int OFF_E = OFF_W1 + 64 * 8 * 4;
 constexpr int OFF_D = OFF_E + BM * 8 * 4;
 constexpr int OFF_BAR = OFF_D + BM * 4;
 constexpr int BAR_BYTES = 512;
 constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;
 static_assert(SMEM <= 232448, "shared memory per CTA");
-static_assert(64 * H1P * 4 <= ABUF_BYTES, "h1T fits in an A buffer");
-static_assert(OFF_EPI % 1024 == 0, "swizzled staging tiles");
+static_assert(OFF_EPI % 1024 == 0 && OFF_W2 % 1024 == 0 && OFF_B % 1024 == 0, "operand and staging alignment");
+static_assert(ZCOL + 64 <= TMEM_FWD, "tensor memory columns");
+
+// MMA N of the head for ncols output columns: ncols up to 128, else the widest of 128, 96, 64, 32 dividing it
+__host__ __device__ constexpr int fwd_bn(int n) {
+  return n <= 128 ? n : n % 128 == 0 ? 128 : n % 96 == 0 ? 96 : n % 64 == 0 ? 64 : 32;
+}
 
 struct Args {
   int nsub;              // radial networks, each over rows [row_off[s], row_off[s + 1])
@@ -103,13 +109,100 @@ __device__ __forceinline__ void tma_store(const CUtensorMap* map, const void* sr
                : "memory");
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
-// the bulk stores this thread issued have read their shared-memory source
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// all bulk stores this thread issued (all but the last) have read their shared-memory source
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // byte offset of element (row r, k) (k < 16) in a k-block of 64-byte rows, 64-byte swizzle
 __device__ __forceinline__ uint32_t swz(int r, int k) {
   return (uint32_t)(r * 64 + ((((k >> 2) ^ (r >> 1)) & 3) << 4) + (k & 3) * 4);
+}
+
+// the 3xTF32 products of a 64-deep contraction (4 k-blocks of A and B) into TMEM column block d
+__device__ __forceinline__ void mma_k64(uint32_t d, uint32_t a_hi, uint32_t a_lo, uint32_t b_hi, uint32_t b_lo,
+                                        uint32_t b_kstride, uint32_t idesc) {
+#pragma unroll
+  for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+    for (int kk = 0; kk < tc::BK / 8; ++kk) {
+      const uint32_t ao = kb * AK_BYTES + kk * 32, bo = kb * b_kstride + kk * 32;
+      tc::mma_tf32_pair(d, tc::sdesc(a_lo + ao), tc::sdesc(b_hi + bo), idesc, (kb | kk) ? 1u : 0u);
+      tc::mma_tf32_pair(d, tc::sdesc(a_hi + ao), tc::sdesc(b_lo + bo), idesc, 1u);
+      tc::mma_tf32_pair(d, tc::sdesc(a_hi + ao), tc::sdesc(b_hi + bo), idesc, 1u);
+    }
+}
+
+// W2 of network `sub` for the hidden products, split and swizzled as this CTA's 32 rows of a
+// 64-row K-major B operand: rows n of W2 (W2 itself, z2 = h1 W2^T) or of W2^T (the backward's
+// dE/dh1 = dE/dz2 W2), hi k-blocks at dst, lo k-blocks at dst + 4 * 2048
+__device__ __forceinline__ void stage_w2(unsigned char* dst, const float* w2, uint32_t rank, bool transposed, int h) {
+  for (int idx = h; idx < 32 * 64; idx += HID_THREADS) {
+    const int nl = idx >> 6, k = idx & 63, n = (int)rank * 32 + nl;
+    const float a = __ldg(&w2[transposed ? k * 64 + n : n * 64 + k]);
+    const uint32_t o = (uint32_t)((k >> 4) * 2048) + swz(nl, k & 15);
+    const float ah = tf32_rna(a);
+    *reinterpret_cast<float*>(dst + o) = ah;
+    *reinterpret_cast<float*>(dst + KB * 2048 + o) = tf32_rna(a - ah);
+  }
+}
+
+// layer 1 of a 128-row tile (rows r0..r0+7, units j0..j0+3 of thread h): h1 = SiLU(W1 e) split into
+// hi/lo and written as the A operand of z2 (abuf: hi k-blocks, then lo k-blocks)
+__device__ __forceinline__ void layer1_to_a(const float* W1T, const float* sE, unsigned char* abuf, int r0, int j0) {
+  float w1v[8][4];
+#pragma unroll
+  for (int n = 0; n < 8; ++n) {
+    const float4 w = *reinterpret_cast<const float4*>(W1T + n * 64 + j0);
+    w1v[n][0] = w.x; w1v[n][1] = w.y; w1v[n][2] = w.z; w1v[n][3] = w.w;
+  }
+  unsigned char* ab = abuf + (j0 >> 4) * AK_BYTES;
+#pragma unroll
+  for (int a = 0; a < 8; ++a) {
+    const float4 ea = *reinterpret_cast<const float4*>(sE + (r0 + a) * 8);
+    const float4 eb = *reinterpret_cast<const float4*>(sE + (r0 + a) * 8 + 4);
+    const float ev[8] = {ea.x, ea.y, ea.z, ea.w, eb.x, eb.y, eb.z, eb.w};
+    float hi[4], lo[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      float acc = 0.f;
+#pragma unroll
+      for (int n = 0; n < 8; ++n) acc = fmaf(w1v[n][b], ev[n], acc);
+      const float v = silu_fast(acc);
+      hi[b] = tf32_rna(v);
+      lo[b] = tf32_rna(v - hi[b]);
+    }
+    const uint32_t o = swz(r0 + a, j0 & 15);
+    *reinterpret_cast<float4*>(ab + o) = make_float4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<float4*>(ab + KB * AK_BYTES + o) = make_float4(lo[0], lo[1], lo[2], lo[3]);
+  }
+}
+
+__device__ __forceinline__ int next_tile_of(const Args& a, int total) { return next_tile(a, total); }
+
+// The leader's hidden thread h == 0 as the tile scheduler: keeps the published tiles one ahead of
+// its own loop (so that the other roles start the next tile early) and returns tile j.
+template <class A>
+__device__ __forceinline__ int publish_ahead(int j, int& published, bool& ended, uint64_t* tq_full, uint64_t* tq_empty,
+                                             int* tq, volatile int* vabort, int total, const A& args) {
+  using namespace tc;
+  while (published <= j + 1 && !ended) {
+    const int ps = published % TQ;
+    int tn;
+    if (published >= TQ && !mbar_wait_cluster(&tq_empty[ps], ((published / TQ) - 1) & 1)) {
+      *vabort = 1;
+      tn = total;
+    } else {
+      tn = *vabort ? total : next_tile_of(args, total);
+    }
+    tq[ps] = tn;
+    remote_store(map_to_rank(smem_u32(&tq[ps]), 1), tn);
+    mbar_arrive(&tq_full[ps]);
+    remote_arrive(map_to_rank(smem_u32(&tq_full[ps]), 1));
+    ended = tn >= total;
+    ++published;
+  }
+  return tq[j % TQ];
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
@@ -119,20 +212,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);    // [BST] (the leader's are used)
   uint64_t* empty = full + BST;                                    // [BST]
-  uint64_t* acc_full = empty + BST;                                // [2]
-  uint64_t* acc_empty = acc_full + 2;                              // [2] (the leader's are used)
-  uint64_t* a_full = acc_empty + 2;                                // [2] (the leader's are used)
+  uint64_t* acc_full = empty + BST;                                // [NACC]
+  uint64_t* acc_empty = acc_full + NACC;                           // [NACC] (the leader's are used)
+  uint64_t* a_full = acc_empty + NACC;                             // [2] (the leader's are used)
   uint64_t* a_empty = a_full + 2;                                  // [2]
-  uint64_t* drain = a_empty + 2;
-  uint64_t* tq_full = drain + 1;                                   // [TQ]
+  uint64_t* a1_full = a_empty + 2;                                 // (the leader's is used)
+  uint64_t* z2_full = a1_full + 1;
+  uint64_t* drain = z2_full + 1;
+  uint64_t* drain2 = drain + 1;
+  uint64_t* tq_full = drain2 + 1;                                  // [TQ]
   uint64_t* tq_empty = tq_full + TQ;                               // [TQ] (the leader's are used)
   int* tq = reinterpret_cast<int*>(tq_empty + TQ);                 // [TQ]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tq + TQ);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* issued = abort_flag + 1;
   int* consumed = issued + 1;
-  int* hid_tile = consumed + 1;                                    // tile index broadcast to the hidden warps
-  float* epi = reinterpret_cast<float*>(smem + OFF_EPI);
+  int* hid_word = consumed + 1;                                    // broadcast to the hidden warps
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
@@ -143,13 +238,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NACC; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 8);        // 4 epilogue warps in each CTA
+    }
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&a_full[b], 2);           // the hidden warps of each CTA, once
       mbar_init(&a_empty[b], 1);
     }
+    mbar_init(a1_full, 2);
+    mbar_init(z2_full, 1);
     mbar_init(drain, 1);
+    mbar_init(drain2, 1);
     for (int j = 0; j < TQ; ++j) {
       mbar_init(&tq_full[j], 1);
       mbar_init(&tq_empty[j], 12);        // leader: producer, MMA, 4 epilogue; peer: producer, 4 epilogue, hidden
@@ -161,7 +261,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"((uint32_t)TMEM_COLS));
+                 "r"((uint32_t)TMEM_FWD));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
   }
   fence_before();
@@ -173,6 +273,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const uint32_t full_l = map_to_rank(smem_u32(full), 0);
   const uint32_t acc_empty_l = map_to_rank(smem_u32(acc_empty), 0);
   const uint32_t a_full_l = map_to_rank(smem_u32(a_full), 0);
+  const uint32_t a1_full_l = map_to_rank(smem_u32(a1_full), 0);
   const uint32_t tq_empty_l = map_to_rank(smem_u32(tq_empty), 0);
   const int bh = g.bn / 2;                 // this CTA's W3 rows per n-tile
 
@@ -217,8 +318,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       fence_after();
       const uint32_t a_base = smem_u32(smem + OFF_A + ab * ABUF_BYTES);
       for (int n = 0; n < g.ntiles; ++n, ++i) {
-        const int buf = i & 1;
-        if (i >= 2 && !mbar_wait_cluster(&acc_empty[buf], ((i >> 1) - 1) & 1)) { ok = false; break; }
+        const int buf = i % NACC;
+        if (i >= NACC && !mbar_wait_cluster(&acc_empty[buf], ((i / NACC) - 1) & 1)) { ok = false; break; }
         fence_after();
         const uint32_t d = tmem + (uint32_t)(buf * ACC_COLS);
         for (int kc = 0; kc < KB; ++kc, ++it) {
@@ -243,7 +344,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         mma_commit_pair(&acc_full[buf]);
       }
       if (!ok) break;
-      mma_commit_pair(&a_empty[ab]);     // both CTAs may overwrite this h2 buffer once these MMAs are done
+      mma_commit_pair(&a_empty[ab]);     // both CTAs may overwrite this A buffer once these MMAs are done
     }
     if (!ok) *vabort = 1;
     mma_commit_pair(drain);
@@ -251,7 +352,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   } else if (warp >= 2 && warp < HID_W0) {
     // ---------------------------------------------------------------- epilogue (both CTAs: own 128 rows)
     const int q = warp & 3;
-    int i = 0;
+    int i = 0, chunk = 0;
     for (int j = 0;; ++j) {
       const int slot = j % TQ;
       if (!mbar_wait_cluster(&tq_full[slot], (j / TQ) & 1)) { *vabort = 1; break; }
@@ -265,19 +366,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const int sub = t / g.mtiles;
       const int mw = row_base(g, sub) + (t % g.mtiles) * 2 * BM + (int)rank * BM + q * 32;
       const int mend = row_end(g, sub);
+      const bool whole = mw + 32 <= mend;          // else the rows past the range are masked
       bool ok = true;
       for (int n = 0; n < g.ntiles; ++n, ++i) {
-        const int buf = i & 1;
-        if (!mbar_wait(&acc_full[buf], (i >> 1) & 1)) { ok = false; break; }
+        const int buf = i % NACC;
+        if (!mbar_wait(&acc_full[buf], (i / NACC) & 1)) { ok = false; break; }
         fence_after();
         float* obase = g.out + (size_t)n * g.bn;
-        unsigned char* stg = smem + OFF_EPI + q * EPI_TILE;
-        const bool whole = mw + 32 <= mend;        // else the rows past the range are masked
 #pragma unroll 1
-        for (int cc = 0; cc < g.bn; cc += 32) {
+        for (int cc = 0; cc < g.bn; cc += 32, ++chunk) {
           float v[32];
           tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * ACC_COLS + cc), v);
-          if (lane == 0) bulk_wait_read();         // this warp's previous store has left the staging tile
+          unsigned char* stg = smem + OFF_EPI + (q * 2 + (chunk & 1)) * EPI_TILE;
+          // the store that last used this staging tile has read it (a tile whose rows are masked
+          // issues no store, so after one every earlier store is waited for)
+          if (lane == 0) {
+            if (whole) bulk_wait_read1();
+            else bulk_wait_read0();
+          }
           __syncwarp();
           // row `lane` as eight 16-byte chunks, chunk c at position c ^ (row & 7)
 #pragma unroll
@@ -295,7 +401,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               const int rr = k * 4 + (lane >> 3), c = lane & 7;
               const int m = mw + rr;
               const float4 w = *reinterpret_cast<const float4*>(stg + rr * 128 + ((c ^ (rr & 7)) << 4));
-              if (m < mend) *reinterpret_cast<float4*>(obase + (size_t)m * g.ncols + cc + 4 * c) = w;
+              if (m < mend && cc + 4 * c < g.bn) *reinterpret_cast<float4*>(obase + (size_t)m * g.ncols + cc + 4 * c) = w;
             }
             __syncwarp();
           }
@@ -313,25 +419,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   } else if (warp >= HID_W0) {
     // ---------------------------------------------------------------- hidden layers -> h2 hi/lo in the A buffer
     const int h = threadIdx.x - 32 * HID_W0;
-    const int r0 = (h >> 4) * 8, j0 = (h & 15) * 4;
-    float* W2T = reinterpret_cast<float*>(smem + OFF_W2T);     // [i][o] = W2[o][i]
-    float* W1T = reinterpret_cast<float*>(smem + OFF_W1);      // [n][j] = W1[j][n]
-    float* sE = reinterpret_cast<float*>(smem + OFF_E);        // [r][n]
+    const int r0 = (h >> 4) * 8, j0 = (h & 15) * 4;     // layer-1 register tile
+    const int qz = warp & 3, half = (warp - HID_W0) >> 2;
+    const int row = qz * 32 + lane, u0 = half * 32;     // z2 read-back: a row, 32 units
+    float* W1T = reinterpret_cast<float*>(smem + OFF_W1);     // [n][j] = W1[j][n]
+    float* sE = reinterpret_cast<float*>(smem + OFF_E);       // [r][n]
     float* sD = reinterpret_cast<float*>(smem + OFF_D);
-    int staged = -1;
+    unsigned char* w2s = smem + OFF_W2;
+    int staged = -1, published = 0;
+    bool ended = false, issued_any = false;
     for (int j = 0;; ++j) {
       const int slot = j % TQ;
       const int ab = j & 1;
+      unsigned char* abuf = smem + OFF_A + ab * ABUF_BYTES;
       if (h == 0) {
         int t;
         if (leader) {
-          // the scheduler: the next tile for the pair, published to every role of both CTAs
-          if (j >= TQ && !mbar_wait_cluster(&tq_empty[slot], ((j / TQ) - 1) & 1)) { *vabort = 1; t = total_tiles; }
-          else t = *vabort ? total_tiles : next_tile(g, total_tiles);
-          tq[slot] = t;
-          remote_store(map_to_rank(smem_u32(&tq[slot]), 1), t);
-          mbar_arrive(&tq_full[slot]);
-          remote_arrive(map_to_rank(smem_u32(&tq_full[slot]), 1));
+          t = publish_ahead(j, published, ended, tq_full, tq_empty, tq, vabort, total_tiles, g);
         } else if (mbar_wait_cluster(&tq_full[slot], (j / TQ) & 1)) {
           t = tq[slot];
           remote_arrive(tq_empty_l + (uint32_t)(slot * 8));
@@ -340,10 +444,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         if (t >= 0 && t < total_tiles && j >= 2 && !mbar_wait(&a_empty[ab], ((j >> 1) - 1) & 1)) t = -1;
         if (t < 0) { *vabort = 1; t = total_tiles; }
-        *hid_tile = t;
+        *hid_word = t;
       }
       hid_sync();
-      const int t = *hid_tile;
+      const int t = *hid_word;
       if (t >= total_tiles) break;
       const int sub = t / g.mtiles;
       const int base = row_base(g, sub) + (t % g.mtiles) * 2 * BM + (int)rank * BM;
@@ -356,9 +460,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       }
       if (sub != staged) {
         const float* w1 = g.rad + g.layer_off + (size_t)sub * g.pair_stride;
-        const float* w2 = w1 + 64 * 8;
         for (int idx = h; idx < 64 * 8; idx += HID_THREADS) W1T[(idx & 7) * 64 + (idx >> 3)] = __ldg(&w1[idx]);
-        for (int idx = h; idx < 64 * 64; idx += HID_THREADS) W2T[(idx & 63) * W2P + (idx >> 6)] = __ldg(&w2[idx]);
+        stage_w2(w2s, w1 + 64 * 8, rank, false, h);
         staged = sub;
       }
       hid_sync();
@@ -368,74 +471,62 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         sE[idx] = ev;
       }
       hid_sync();
-      // layer 1: z1[r][j] = sum_n W1[j][n] e[r][n], h1 = SiLU(z1) stored transposed in the A buffer
-      float* h1T = reinterpret_cast<float*>(smem + OFF_A + ab * ABUF_BYTES);
-      float z[8][4];
-      float w1v[8][4];
-#pragma unroll
-      for (int n = 0; n < 8; ++n) {
-        const float4 w = *reinterpret_cast<const float4*>(W1T + n * 64 + j0);
-        w1v[n][0] = w.x; w1v[n][1] = w.y; w1v[n][2] = w.z; w1v[n][3] = w.w;
-      }
-#pragma unroll
-      for (int a = 0; a < 8; ++a) {
-        const float4 ea = *reinterpret_cast<const float4*>(sE + (r0 + a) * 8);
-        const float4 eb = *reinterpret_cast<const float4*>(sE + (r0 + a) * 8 + 4);
-        const float ev[8] = {ea.x, ea.y, ea.z, ea.w, eb.x, eb.y, eb.z, eb.w};
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          float acc = 0.f;
-#pragma unroll
-          for (int n = 0; n < 8; ++n) acc = fmaf(w1v[n][b], ev[n], acc);
-          z[a][b] = acc;
+      layer1_to_a(W1T, sE, abuf, r0, j0);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // h1 and W2 written by threads, read by the MMAs
+      hid_sync();
+      if (h == 0) {
+        if (leader) {
+          mbar_arrive(a1_full);
+          // z2 = h1 W2^T once both CTAs' h1 rows are in place
+          if (mbar_wait_cluster(a1_full, j & 1)) {
+            fence_after();
+            const uint32_t au = smem_u32(abuf);
+            mma_k64(tmem + ZCOL, au, au + KB * AK_BYTES, smem_u32(w2s), smem_u32(w2s + KB * 2048), 2048, idesc_pair(64));
+            mma_commit_pair(z2_full);
+            issued_any = true;
+          } else {
+            *vabort = 1;
+          }
+        } else {
+          remote_arrive(a1_full_l);
         }
-      }
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        float* dst = h1T + (j0 + b) * H1P + r0;
-        *reinterpret_cast<float4*>(dst) =
-            make_float4(silu_fast(z[0][b]), silu_fast(z[1][b]), silu_fast(z[2][b]), silu_fast(z[3][b]));
-        *reinterpret_cast<float4*>(dst + 4) =
-            make_float4(silu_fast(z[4][b]), silu_fast(z[5][b]), silu_fast(z[6][b]), silu_fast(z[7][b]));
+        const bool ok = !*vabort && mbar_wait(z2_full, j & 1);
+        if (!ok) *vabort = 1;
+        *hid_word = ok ? 1 : 0;
       }
       hid_sync();
-      // layer 2: z2[r][o] = sum_i W2[o][i] h1[r][i]
+      if (!*hid_word) break;
+      fence_after();
+      // h2 = SiLU(z2): a row and 32 units per thread, over h1 in the A buffer (z2 has read it)
+      {
+        float z2[32];
+        tmem_ld32(tmem + ((uint32_t)(qz * 32) << 16) + (uint32_t)(ZCOL + u0), z2);
 #pragma unroll
-      for (int a = 0; a < 8; ++a)
+        for (int c = 0; c < 8; ++c) {
+          float hi[4], lo[4];
 #pragma unroll
-        for (int b = 0; b < 4; ++b) z[a][b] = 0.f;
-#pragma unroll 4
-      for (int i2 = 0; i2 < 64; ++i2) {
-        const float4 ha = *reinterpret_cast<const float4*>(h1T + i2 * H1P + r0);
-        const float4 hb = *reinterpret_cast<const float4*>(h1T + i2 * H1P + r0 + 4);
-        const float4 w = *reinterpret_cast<const float4*>(W2T + i2 * W2P + j0);
-        const float hv[8] = {ha.x, ha.y, ha.z, ha.w, hb.x, hb.y, hb.z, hb.w}, wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int a = 0; a < 8; ++a)
-#pragma unroll
-          for (int b = 0; b < 4; ++b) z[a][b] = fmaf(hv[a], wv[b], z[a][b]);
-      }
-      hid_sync();                          // every read of h1T is done before h2 overwrites the buffer
-      unsigned char* abuf = smem + OFF_A + ab * ABUF_BYTES + (j0 >> 4) * AK_BYTES;
-#pragma unroll
-      for (int a = 0; a < 8; ++a) {
-        float hi[4], lo[4];
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const float v = silu_fast(z[a][b]);
-          hi[b] = tf32_rna(v);
-          lo[b] = tf32_rna(v - hi[b]);
+          for (int b = 0; b < 4; ++b) {
+            const float v = silu_fast(z2[4 * c + b]);
+            hi[b] = tf32_rna(v);
+            lo[b] = tf32_rna(v - hi[b]);
+          }
+          const int k = u0 + 4 * c;
+          const uint32_t o = (uint32_t)((k >> 4) * AK_BYTES) + swz(row, k & 15);
+          *reinterpret_cast<float4*>(abuf + o) = make_float4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<float4*>(abuf + KB * AK_BYTES + o) = make_float4(lo[0], lo[1], lo[2], lo[3]);
         }
-        const uint32_t o = swz(r0 + a, j0 & 15);
-        *reinterpret_cast<float4*>(abuf + o) = make_float4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<float4*>(abuf + KB * AK_BYTES + o) = make_float4(lo[0], lo[1], lo[2], lo[3]);
       }
+      fence_before();
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // h2 written by threads, read by the MMAs
       hid_sync();
       if (h == 0) {
         if (leader) mbar_arrive(&a_full[ab]);
         else remote_arrive(a_full_l + (uint32_t)(ab * 8));
       }
+    }
+    if (h == 0 && leader && issued_any) {
+      mma_commit_pair(drain2);           // every product this thread issued has completed
+      mbar_wait(drain2, 0);
     }
   }
   fence_before();
@@ -451,12 +542,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   cluster_sync();
   if (warp == 1) {
     fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)TMEM_COLS));
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)TMEM_FWD));
   }
 }
 
 // R rows [M][ncols] of nsub radial networks over their row ranges (row_off, device; or one network
-// over [0, M) when null); b_maps[s]: network s's W3 (hi, lo) maps with boxes of tile_n(ncols) / 2 rows.
+// over [0, M) when null); b_maps[s]: network s's W3 (hi, lo) maps with boxes of fwd_bn(ncols) / 2 rows.
 inline int radial_fwd(long long M, int ncols, const int* row_off, int nsub, const int* perm, const float* dist,
                       const float* rad, size_t layer_off, size_t pair_stride, float rc, const MapPair* const* b_maps,
                       float* out, int* counter, cudaStream_t s) {
@@ -468,8 +559,7 @@ inline int radial_fwd(long long M, int ncols, const int* row_off, int nsub, cons
   g.M = (int)M;
   g.mtiles = (int)((M + 2 * BM - 1) / (2 * BM));
   g.ncols = ncols;
-  g.bn = tc::tile_n(ncols);
-  if (g.bn / 2 > 128 || ncols % g.bn != 0) return EMP_ERR_ARG;
+  g.bn = fwd_bn(ncols);
   g.ntiles = ncols / g.bn;
   g.row_off = row_off;
   g.counter = counter;
@@ -502,7 +592,6 @@ inline int radial_fwd(long long M, int ncols, const int* row_off, int nsub, cons
   k_radial_fwd_tc<<<2 * pairs, THREADS, SMEM, s>>>(g, maps, (int)total);
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
-
 
 // ------------------------------------------------------------------ backward
 // dE/dd of every row from dE/dR (rows split hi/lo), adding (dE/dd) rhat to g_r:
@@ -576,19 +665,7 @@ __device__ __forceinline__ int next_tile_b(const BwdArgs& a, int total) {
   return t;
 }
 
-// the 3xTF32 products of a 64-deep contraction (4 k-blocks) into TMEM column block d
-__device__ __forceinline__ void mma_k64(uint32_t d, uint32_t a_hi, uint32_t a_lo, uint32_t b_hi, uint32_t b_lo,
-                                        uint32_t b_kstride, uint32_t idesc) {
-#pragma unroll
-  for (int kb = 0; kb < KB; ++kb)
-#pragma unroll
-    for (int kk = 0; kk < tc::BK / 8; ++kk) {
-      const uint32_t ao = kb * AK_BYTES + kk * 32, bo = kb * b_kstride + kk * 32;
-      tc::mma_tf32_pair(d, tc::sdesc(a_lo + ao), tc::sdesc(b_hi + bo), idesc, (kb | kk) ? 1u : 0u);
-      tc::mma_tf32_pair(d, tc::sdesc(a_hi + ao), tc::sdesc(b_lo + bo), idesc, 1u);
-      tc::mma_tf32_pair(d, tc::sdesc(a_hi + ao), tc::sdesc(b_hi + bo), idesc, 1u);
-    }
-}
+__device__ __forceinline__ int next_tile_of(const BwdArgs& a, int total) { return next_tile_b(a, total); }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
     k_radial_bwd_tc(const __grid_constant__ BwdArgs g, const __grid_constant__ BwdMaps maps, int total_tiles) {
@@ -739,18 +816,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
     const uint32_t hbuf_u = smem_u32(hbuf);
     int staged = -1;
     bool issued_any = false;                            // the leader's h == 0 issued MMAs (drained at exit)
+    int published = 0;                                  // the leader's h == 0: tiles published so far
+    bool ended = false;
     for (int j = 0;; ++j) {
       const int slot = j % TQ;
       const int gb = j & 1;
       if (h == 0) {
         int t;
         if (leader) {
-          if (j >= TQ && !mbar_wait_cluster(&tq_empty[slot], ((j / TQ) - 1) & 1)) { *vabort = 1; t = total_tiles; }
-          else t = *vabort ? total_tiles : next_tile_b(g, total_tiles);
-          tq[slot] = t;
-          remote_store(map_to_rank(smem_u32(&tq[slot]), 1), t);
-          mbar_arrive(&tq_full[slot]);
-          remote_arrive(map_to_rank(smem_u32(&tq_full[slot]), 1));
+          // the scheduler, one tile ahead: the head of tile j + 1 streams while these warps finish tile j
+          t = publish_ahead(j, published, ended, tq_full, tq_empty, tq, vabort, total_tiles, g);
         } else if (mbar_wait_cluster(&tq_full[slot], (j / TQ) & 1)) {
           t = tq[slot];
           remote_arrive(tq_empty_l + (uint32_t)(slot * 8));
@@ -780,19 +855,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
       if (sub != staged) {
         // W1 transposed; this CTA's 32 rows of W2 (B of z2) and of W2^T (B of dE/dh1), split and swizzled
         const float* w1 = g.rad + g.layer_off + (size_t)sub * g.pair_stride;
-        const float* w2 = w1 + 64 * 8;
         for (int idx = h; idx < 64 * 8; idx += HID_THREADS) W1T[(idx & 7) * 64 + (idx >> 3)] = __ldg(&w1[idx]);
-        for (int idx = h; idx < 32 * 64; idx += HID_THREADS) {
-          const int nl = idx >> 6, k = idx & 63, n = (int)rank * 32 + nl;
-          const uint32_t o = (uint32_t)((k >> 4) * B_BK) + swz(nl, k & 15);
-          const float a = __ldg(&w2[n * 64 + k]);          // W2[o = n][i = k]
-          const float b = __ldg(&w2[k * 64 + n]);          // W2^T[n][k] = W2[k][n]
-          const float ah = tf32_rna(a), bh = tf32_rna(b);
-          *reinterpret_cast<float*>(smem + B_OFF_W2 + o) = ah;
-          *reinterpret_cast<float*>(smem + B_OFF_W2 + 4 * B_BK + o) = tf32_rna(a - ah);
-          *reinterpret_cast<float*>(smem + B_OFF_W2T + o) = bh;
-          *reinterpret_cast<float*>(smem + B_OFF_W2T + 4 * B_BK + o) = tf32_rna(b - bh);
-        }
+        stage_w2(smem + B_OFF_W2, w1 + 64 * 8, rank, false, h);
+        stage_w2(smem + B_OFF_W2T, w1 + 64 * 8, rank, true, h);
         staged = sub;
       }
       hid_sync();
@@ -804,34 +869,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
       }
       hid_sync();
       // ---- z1, h1 = SiLU(z1) as the A operand of z2
-      {
-        float w1v[8][4];
-#pragma unroll
-        for (int n = 0; n < 8; ++n) {
-          const float4 w = *reinterpret_cast<const float4*>(W1T + n * 64 + j0);
-          w1v[n][0] = w.x; w1v[n][1] = w.y; w1v[n][2] = w.z; w1v[n][3] = w.w;
-        }
-        unsigned char* ab = hbuf + (j0 >> 4) * AK_BYTES;
-#pragma unroll
-        for (int a = 0; a < 8; ++a) {
-          const float4 ea = *reinterpret_cast<const float4*>(sE + (r0 + a) * 8);
-          const float4 eb = *reinterpret_cast<const float4*>(sE + (r0 + a) * 8 + 4);
-          const float ev[8] = {ea.x, ea.y, ea.z, ea.w, eb.x, eb.y, eb.z, eb.w};
-          float hi[4], lo[4];
-#pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            float acc = 0.f;
-#pragma unroll
-            for (int n = 0; n < 8; ++n) acc = fmaf(w1v[n][b], ev[n], acc);
-            const float v = silu_fast(acc);
-            hi[b] = tf32_rna(v);
-            lo[b] = tf32_rna(v - hi[b]);
-          }
-          const uint32_t o = swz(r0 + a, j0 & 15);
-          *reinterpret_cast<float4*>(ab + o) = make_float4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<float4*>(ab + KB * AK_BYTES + o) = make_float4(lo[0], lo[1], lo[2], lo[3]);
-        }
-      }
+      layer1_to_a(W1T, sE, hbuf, r0, j0);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // h1 and W2 written by threads, read by the MMAs
       hid_sync();
       if (h == 0) {

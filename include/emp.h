@@ -181,7 +181,10 @@ int mp_model_radial_tables(void* model, double tol, int32_t* n_pieces);
 int mp_radial_hidden(const void* model, int32_t layer, int32_t pair, int64_t n, const float* d, float* h2_hi,
                      float* h2_lo, const float* g_h2, float* dE_dd, void* ws, size_t ws_bytes, cudaStream_t stream);
 
-/* Workspace bytes mp_forward / mp_energy_forces need. */
+/* Workspace bytes mp_forward / mp_energy_forces need.  The size depends on the model's radial
+ * mode: with radial tables (mp_model_radial_tables) the per-row hidden values take 768 bytes per
+ * edge more, so query it after the tables are built (a workspace sized before them is rejected
+ * with EMP_ERR_WORKSPACE). */
 size_t mp_workspace_bytes(const void* model, int64_t n_edges, int32_t n_atoms);
 
 /* One interaction layer (forward only): agg_out[i] = (1/avg_degree) * sum over
