@@ -7,23 +7,26 @@
 // device row range of the pair-sorted row list.
 //
 // Persistent kernel on CTA pairs (clusters of 2, cta_group::2); a tile is 256 rows
-// (128 per CTA) of one network.  In each CTA:
-//  - eight hidden warps evaluate the basis and the two hidden layers on SIMT (8 x 4
-//    register tiles, the same FP32 operation order as the standalone hidden-layer
-//    kernel) and write h2 split into TF32 hi and lo straight into the shared-memory
-//    A operand of the head, in the 64-byte-swizzled K-major layout the MMA
-//    descriptors read (two A buffers: the next tile's h2 is written while the head of
-//    the current one runs);
-//  - the leader's hidden warps take tiles from the counter and publish them to every
-//    role of both CTAs (so the next tile's hidden layers never wait for the head);
-//  - warp 0 streams the head weights W3 (hi, lo; this CTA's half of a 256-row tile per
-//    k-block) into a 3-stage TMA ring;
-//  - the leader's warp 1 issues the 3xTF32 head products into one of two TMEM
-//    accumulators per n-tile;
-//  - four epilogue warps store the R rows: TMEM -> registers -> a 128-byte-swizzled
+// (128 per CTA) of one network; every product is 3xTF32 (a = hi + lo, hi = RN_tf32(a),
+// lo = RN_tf32(a - hi); lo.hi + hi.lo + hi.hi accumulated in FP32 in tensor memory).
+// In each CTA:
+//  - eight hidden warps evaluate the basis and z1 = W1 e on SIMT (8 x 4 register tiles)
+//    and write h1 = SiLU(z1), split, into the shared-memory A operand (64-byte-swizzled
+//    K-major, the layout the MMA descriptors read); the leader's hidden thread issues
+//    z2 = h1 W2^T (N = 64, W2 split into shared memory when the network changes); the
+//    hidden warps read z2 back from tensor memory (a row and 32 units per thread) and
+//    write h2 = SiLU(z2), split, over h1: the A operand of the head.  Two A buffers, so
+//    the next tile's hidden layers run while the head of this one does;
+//  - the leader's hidden thread also takes the tiles from the counter and publishes
+//    them, one tile ahead, to every role of both CTAs;
+//  - warp 0 streams the head weights W3 (hi, lo; this CTA's half of each n-tile's rows
+//    per k-block) into a TMA ring deep enough to cover the L2 latency;
+//  - the leader's warp 1 issues the head products R = h2 W3^T in n-tiles of up to 128
+//    columns into a ring of three TMEM accumulators;
+//  - eight epilogue warps (two per TMEM lane quarter) store the R rows: TMEM -> registers -> a 128-byte-swizzled
 //    staging tile per warp -> one TMA bulk store per 32 x 32 block (plain masked stores
 //    for a block whose rows run past the network's range).
-// h2 never reaches global memory.  Every wait is bounded: on timeout the CTA records
+// h1 and h2 never reach global memory.  Every wait is bounded: on timeout the CTA records
 // a device error, stops, waits (bounded) for its own copies and MMAs and frees TMEM.
 #pragma once
 #include "so2_tc.cuh"
@@ -35,7 +38,8 @@ namespace rtc {
 constexpr int BM = 128;                          // rows per CTA (256 per pair)
 constexpr int HID_WARPS = 8;
 constexpr int HID_THREADS = 32 * HID_WARPS;
-constexpr int HID_W0 = 6;                        // first hidden warp
+constexpr int EPI_WARPS = 8;                     // two per TMEM lane quarter, alternate 32-column chunks
+constexpr int HID_W0 = 2 + EPI_WARPS;            // first hidden warp
 constexpr int THREADS = 32 * (HID_W0 + HID_WARPS);
 constexpr int KB = 4;                            // 16-wide k-blocks of h2 (K = 64)
 constexpr int AK_BYTES = BM * 64;                // one k-block of hi (or lo): 128 rows x 64 bytes
@@ -50,8 +54,8 @@ constexpr int TMEM_FWD = 512;
 constexpr int EPI_TILE = 32 * 128;               // a 32 x 32 fp32 staging tile (128-byte swizzle)
 constexpr int OFF_A = 0;                         // two A buffers: h1, then h2 (hi k-blocks, then lo)
 constexpr int OFF_B = OFF_A + 2 * ABUF_BYTES;
-constexpr int OFF_EPI = OFF_B + BST * BSTAGE_BYTES;   // two staging tiles per epilogue warp
-constexpr int OFF_W2 = OFF_EPI + 8 * EPI_TILE;   // W2 (B of z2): this CTA's 32 rows, hi then lo
+constexpr int OFF_EPI = OFF_B + BST * BSTAGE_BYTES;   // a staging tile per epilogue warp
+constexpr int OFF_W2 = OFF_EPI + EPI_WARPS * EPI_TILE;   // W2 (B of z2): this CTA's 32 rows, hi then lo
 constexpr int OFF_W1 = OFF_W2 + 2 * KB * 32 * 64;
 constexpr int OFF_E = OFF_W1 + 64 * 8 * 4;
 constexpr int OFF_D = OFF_E + BM * 8 * 4;
@@ -109,9 +113,8 @@ __device__ __forceinline__ void tma_store(const CUtensorMap* map, const void* sr
                : "memory");
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
-// all bulk stores this thread issued (all but the last) have read their shared-memory source
+// the bulk stores this thread issued have read their shared-memory source
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // byte offset of element (row r, k) (k < 16) in a k-block of 64-byte rows, 64-byte swizzle
@@ -240,7 +243,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
     for (int b = 0; b < NACC; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 8);        // 4 epilogue warps in each CTA
+      mbar_init(&acc_empty[b], 2 * EPI_WARPS);   // the epilogue warps of both CTAs
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&a_full[b], 2);           // the hidden warps of each CTA, once
@@ -252,7 +255,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     mbar_init(drain2, 1);
     for (int j = 0; j < TQ; ++j) {
       mbar_init(&tq_full[j], 1);
-      mbar_init(&tq_empty[j], 12);        // leader: producer, MMA, 4 epilogue; peer: producer, 4 epilogue, hidden
+      mbar_init(&tq_empty[j], 2 * (2 + EPI_WARPS));   // leader: producer, MMA, epilogue; peer: producer, epilogue, hidden
     }
     *abort_flag = 0;
     *issued = 0;
@@ -351,8 +354,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     mbar_wait(drain, 0);
   } else if (warp >= 2 && warp < HID_W0) {
     // ---------------------------------------------------------------- epilogue (both CTAs: own 128 rows)
-    const int q = warp & 3;
-    int i = 0, chunk = 0;
+    const int q = warp & 3, ehalf = (warp - 2) >> 2;    // lane quarter; which 32-column chunks
+    int i = 0;
     for (int j = 0;; ++j) {
       const int slot = j % TQ;
       if (!mbar_wait_cluster(&tq_full[slot], (j / TQ) & 1)) { *vabort = 1; break; }
@@ -374,16 +377,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         fence_after();
         float* obase = g.out + (size_t)n * g.bn;
 #pragma unroll 1
-        for (int cc = 0; cc < g.bn; cc += 32, ++chunk) {
+        for (int cc = 32 * ehalf; cc < g.bn; cc += 64) {
           float v[32];
           tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * ACC_COLS + cc), v);
-          unsigned char* stg = smem + OFF_EPI + (q * 2 + (chunk & 1)) * EPI_TILE;
-          // the store that last used this staging tile has read it (a tile whose rows are masked
-          // issues no store, so after one every earlier store is waited for)
-          if (lane == 0) {
-            if (whole) bulk_wait_read1();
-            else bulk_wait_read0();
-          }
+          unsigned char* stg = smem + OFF_EPI + (warp - 2) * EPI_TILE;
+          if (lane == 0) bulk_wait_read0();        // this warp's previous store has read the staging tile
           __syncwarp();
           // row `lane` as eight 16-byte chunks, chunk c at position c ^ (row & 7)
 #pragma unroll
