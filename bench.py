@@ -243,8 +243,9 @@ def alg_bytes_step(name: str, C: int, T: int, E: int, N: int) -> float:
         return E * (2 * 64 * 4 + C * 4) + (T - 1) * E * (2 * 64 * 4 + 4 * C * 4)
     if name == "radial_head_bwd":         # dE/dR hi/lo in (C columns in the first layer); dE/dh2 out
         return E * (2 * C * 4 + 64 * 4) + (T - 1) * E * (2 * 4 * C * 4 + 64 * 4)
-    if name == "radial_bwd":              # d, dE/dh2 in; g_r read-modify-write
-        return T * E * (4 + 64 * 4 + 2 * 12)
+    if name == "radial_bwd":              # the fused network backward: dE/dR hi/lo (C columns in the first
+        # layer, 4C after), d and the edge vector in; g_r read-modify-write
+        return E * (2 * C * 4 + 4 + 12 + 2 * 12) + (T - 1) * E * (2 * 4 * C * 4 + 4 + 12 + 2 * 12)
     raise KeyError(name)
 
 
@@ -265,13 +266,14 @@ def hbm_fractions(fam, steps: int, E: int, N: int, C: int, T: int, hbm_gbs: floa
     return out
 
 
-# DRAM bytes per launch of the SO(2) mixing kernel (mean over one N=4096 step's 119 launches: 39
-# forward launches of two cohorts, one of a single cohort, 79 backward cohort launches), from ncu
-# captures of the N=512 step's forward pair and backward cohort launches, which have the same
-# shapes (profiles/kernels_n512_step.md).  Valid only for the kernel source and the launch
-# structure it was taken on: so2_tc.cuh and the marked per-edge product launch code of emp_lib.cu
-# must hash to source_sha1, else the roofline's traffic is null.
-SO2_TRAFFIC = {"source_sha1": "ce709d4c4d2e8ac7b7432db596fca495fb14a9a7", "bytes_per_launch": 388.6e6}
+# DRAM bytes per launch of the SO(2) mixing kernel (mean over one N=4096 step's 80 launches: 39
+# forward launches of two cohorts and one of a single cohort, 39 backward launches of two cohorts and
+# one of a single cohort), from ncu captures of the N=512 step's forward and backward two-cohort
+# launches, which have the same shapes (profiles/kernels_n512_step.md; a single-cohort launch counted
+# at half).  Valid only for the kernel source and the launch structure it was taken on: so2_tc.cuh
+# and the marked per-edge product launch code of emp_lib.cu must hash to source_sha1, else the
+# roofline's traffic is null.
+SO2_TRAFFIC = {"source_sha1": "22d06415696fc248214d106eafa843314dbe6826", "bytes_per_launch": 585.4e6}
 
 
 def so2_source_hash():

@@ -25,6 +25,9 @@ def test_alg_bytes_follow_the_rows_each_kernel_moves():
     assert bench.alg_bytes_step("radial_head", C, 1, E, N) == E * (2 * 64 * 4 + C * 4)
     assert bench.alg_bytes_step("radial_head", C, T, E, N) == E * (2 * 64 * 4 + C * 4) + 2 * E * (2 * 64 * 4 + 4 * C * 4)
     assert bench.alg_bytes_step("radial_h2", C, T, E, N) == 3 * E * (4 + 2 * 64 * 4)
+    # the fused network kernels: d in, R out (forward); dE/dR hi/lo, d, r in, g_r updated (backward)
+    assert bench.alg_bytes_step("radial_fwd", C, T, E, N) == E * (4 + C * 4) + 2 * E * (4 + 4 * C * 4)
+    assert bench.alg_bytes_step("radial_bwd", C, T, E, N) == E * (2 * C * 4 + 40) + 2 * E * (2 * 4 * C * 4 + 40)
 
 
 def test_hbm_fraction_is_bytes_over_time_over_peak():
