@@ -23,7 +23,7 @@ SYMBOLS = (
     "mp_workspace_bytes", "mp_forward", "mp_energy_forces", "mp_so2_mix", "mp_chain_create",
     "mp_chain_destroy", "mp_radial_chain", "emp_status_string", "emp_last_device_error",
     "emp_profile_enable", "emp_profile_read", "emp_profile_names", "emp_launch_count",
-    "emp_set_wait_limit", "emp_wait_selftest", "emp_tf32_mma_rate", "mp_model_radial_tables", "mp_radial_hidden",
+    "emp_set_wait_limit", "emp_wait_selftest", "emp_tf32_split_selftest", "emp_tf32_mma_rate", "mp_model_radial_tables", "mp_radial_hidden",
     "mp_weight_grad_workspace_bytes", "mp_energy_weight_grad", "nl_refresh",
     "mp_sharded_workspace_bytes", "mp_energy_forces_sharded",
 )
@@ -116,6 +116,8 @@ def lib() -> ctypes.CDLL:
         L.emp_set_wait_limit.argtypes = [i64]
         L.emp_wait_selftest.restype = ctypes.c_int
         L.emp_wait_selftest.argtypes = [vp]
+        L.emp_tf32_split_selftest.restype = ctypes.c_int
+        L.emp_tf32_split_selftest.argtypes = [ctypes.POINTER(ctypes.c_uint64)]
         L.mp_weight_grad_workspace_bytes.restype = sz
         L.mp_weight_grad_workspace_bytes.argtypes = [vp, i64, i32]
         L.mp_energy_weight_grad.restype = ctypes.c_int
@@ -164,6 +166,14 @@ def wait_selftest() -> int:
     """One bounded wait that nothing satisfies; returns the device error it records."""
     _check(lib().emp_wait_selftest(_stream()), "emp_wait_selftest")
     return last_device_error()
+
+
+def tf32_split_selftest() -> int:
+    """Patterns (of all non-NaN 32-bit ones) where the library's TF32 rounding differs from
+    cvt.rna.tf32.f32 (0 expected)."""
+    n = ctypes.c_uint64(0)
+    _check(lib().emp_tf32_split_selftest(ctypes.byref(n)), "emp_tf32_split_selftest")
+    return int(n.value)
 
 
 def tf32_mma_rate(iters: int = 20000) -> float:

@@ -553,6 +553,19 @@ int ensure_attrs() {
   return EMP_OK;
 }
 
+// tf32_rna against the conversion instruction over every 32-bit pattern (NaNs skipped): the count of
+// patterns where they differ
+__global__ void k_tf32_selftest(unsigned long long* mismatches) {
+  unsigned long long bad = 0;
+  for (uint64_t b = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; b < (1ull << 32);
+       b += (uint64_t)gridDim.x * blockDim.x) {
+    const float a = __uint_as_float((uint32_t)b);
+    if (a != a) continue;
+    if (__float_as_uint(tf32_rna(a)) != __float_as_uint(tf32_rna_cvt(a))) ++bad;
+  }
+  if (bad) atomicAdd(mismatches, bad);
+}
+
 // One bounded wait on an mbarrier that nothing arrives on: it runs out after the limit in
 // force (emp_set_wait_limit), records EMP_ERR_TIMEOUT in the device error word and returns.
 __global__ void k_wait_selftest() {
@@ -712,6 +725,22 @@ int emp_wait_selftest(cudaStream_t stream) {
   if (st != EMP_OK) return st;
   k_wait_selftest<<<1, 32, 0, stream>>>();
   return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
+}
+
+int emp_tf32_split_selftest(uint64_t* mismatches) {
+  if (!mismatches) return EMP_ERR_ARG;
+  int st = check_device();
+  if (st != EMP_OK) return st;
+  unsigned long long* d = nullptr;
+  EMP_CUDA_TRY(cudaMalloc(&d, sizeof(unsigned long long)));
+  cudaMemset(d, 0, sizeof(unsigned long long));
+  k_tf32_selftest<<<148 * 8, 256>>>(d);
+  unsigned long long h = 0;
+  const cudaError_t e = cudaMemcpy(&h, d, sizeof(h), cudaMemcpyDeviceToHost);
+  cudaFree(d);
+  if (e != cudaSuccess) return EMP_ERR_CUDA;
+  *mismatches = h;
+  return EMP_OK;
 }
 
 int emp_last_device_error(void) {

@@ -150,8 +150,18 @@ __global__ void k_transpose(const float* __restrict__ src, float* __restrict__ d
   dst[(size_t)c * rows + r] = src[idx];
 }
 
-// 3xTF32 split: hi = round-to-nearest TF32 of a, lo = TF32(a - hi)
+// 3xTF32 split: hi = TF32(a), lo = TF32(a - hi), TF32 being round to nearest, ties away from zero,
+// at the 10th explicit mantissa bit.  Done on the bits: add half of the 13 dropped bits' range to
+// the magnitude and clear them (a carry out of the mantissa steps the exponent, which is the
+// correct rounding up to the next binade; subnormals, zeros and infinities come out right too).
+// Two full-rate integer operations, where the conversion instruction issues at a lower rate; the
+// kernels that split whole tiles run it millions of times per launch.  emp_tf32_split_selftest
+// checks it against cvt.rna.tf32.f32 on every non-NaN 32-bit pattern.
 __device__ __forceinline__ float tf32_rna(float a) {
+  return __uint_as_float((__float_as_uint(a) + 0x1000u) & 0xFFFFE000u);
+}
+// the same rounding by the conversion instruction (the self-test's reference)
+__device__ __forceinline__ float tf32_rna_cvt(float a) {
   uint32_t r;
   asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(a));
   return __uint_as_float(r);

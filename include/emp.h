@@ -299,6 +299,12 @@ int emp_set_wait_limit(int64_t cycles);
  * after the bound in force, and emp_last_device_error() then reports
  * EMP_ERR_TIMEOUT.  For checking the failure path without a fault. */
 int emp_wait_selftest(cudaStream_t stream);
+/* The library rounds to TF32 (the 3xTF32 split: round to nearest, ties away from zero, at the
+ * 10th mantissa bit) with integer operations on the bits.  This runs that rounding and the
+ * conversion instruction cvt.rna.tf32.f32 on every 32-bit pattern that is not a NaN and stores
+ * in *mismatches how many differ (0 expected).  Allocates 8 bytes of device memory; synchronous.
+ * Errors: EMP_ERR_ARG (null), EMP_ERR_UNSUPPORTED (not sm_100), EMP_ERR_CUDA. */
+int emp_tf32_split_selftest(uint64_t* mismatches);
 
 #ifdef __cplusplus
 }

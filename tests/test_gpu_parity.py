@@ -371,3 +371,9 @@ def test_single_layer_n4096_sampled_receivers():
         ref = omodel.single_layer(w.spec, w.weights, 1, x, ref_g.recv[sl], ref_g.send[sl], ref_g.r[sl], st.species,
                                   st.pos.shape[0])[i]
         assert np.abs(agg[i] - ref).max() <= 2e-5 * np.abs(ref).max()
+
+
+def test_tf32_rounding_matches_the_conversion_instruction():
+    """The 3xTF32 split rounds on the bits (integer add and mask); over every non-NaN 32-bit
+    pattern it must give what cvt.rna.tf32.f32 gives."""
+    assert emp.tf32_split_selftest() == 0
