@@ -265,10 +265,10 @@ struct CohortMaps {
     coh = std::min(E, cohort);
     tail_rows = E % cohort;
     if (coh > 0) {
-      const int st = make_pair(&full, hi, lo, coh, 16 * C, 16 * C, tc::BM);
+      const int st = make_pair128(&full, hi, lo, coh, 16 * C, 16 * C, tc::BM);
       if (st != EMP_OK) return st;
     }
-    if (tail_rows > 0 && tail_rows != coh) return make_pair(&tail, hi, lo, tail_rows, 16 * C, 16 * C, tc::BM);
+    if (tail_rows > 0 && tail_rows != coh) return make_pair128(&tail, hi, lo, tail_rows, 16 * C, 16 * C, tc::BM);
     return EMP_OK;
   }
   const So2AMaps* get(long long rows) const { return rows == coh ? &full : &tail; }
@@ -465,7 +465,7 @@ int radial_forward(const Model& m, const emp_graph* g, int t, const int* species
   if (h2_only) return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
   // one launch: a sub-problem per radial network over its (device) row range
   MapPair a;
-  int st = make_pair(&a, h2hi, h2lo, E, 64, 64, tc::BM);
+  int st = make_pair128(&a, h2hi, h2lo, E, 64, 64, tc::BM);
   if (st != EMP_OK) return st;
   GemmSub subs[tc::MAXSUB];
   for (int p = 0; p < m.n_pairs; ++p) {
@@ -508,11 +508,11 @@ int radial_backward(const Model& m, const emp_graph* g, int t, const int* specie
   }
   {
     MapPair a;
-    int st = make_pair(&a, gRhi, gRlo, E, 4 * C, 4 * C, tc::BM);
+    int st = make_pair128(&a, gRhi, gRlo, E, 4 * C, 4 * C, tc::BM);
     if (st != EMP_OK) return st;
     GemmSub subs[tc::MAXSUB];
     for (int p = 0; p < m.n_pairs; ++p) {
-      const MapPair& b = m.w3t_maps[(size_t)t * m.n_pairs + p];
+      const MapPair& b = m.w3t128_maps[(size_t)t * m.n_pairs + p];
       subs[p] = GemmSub{&a.hi, &a.lo, &b.hi, &b.lo, 0, kcols, 64, 0, gh2};
     }
     Scope sc_("radial_head_bwd", s);
@@ -694,6 +694,8 @@ int emp_tf32_mma_rate(int32_t iters, cudaStream_t stream, double* tflops) {
   if (!tflops || iters < 1) return EMP_ERR_ARG;
   int st = check_device();
   if (st != EMP_OK) return st;
+  st = ensure_attrs();
+  if (st != EMP_OK) return st;
   const int pairs = tc::num_sms() / 2;
   cudaEvent_t a = nullptr, b = nullptr;
   EMP_CUDA_TRY(cudaEventCreate(&a));
@@ -708,8 +710,8 @@ int emp_tf32_mma_rate(int32_t iters, cudaStream_t stream, double* tflops) {
   cudaEventDestroy(a);
   cudaEventDestroy(b);
   if (e1 != cudaSuccess || e2 != cudaSuccess || cudaGetLastError() != cudaSuccess) return EMP_ERR_CUDA;
-  // per round: two k-steps of three M = 256, N = 256, K = 8 products per pair
-  const double flops = (double)pairs * iters * 2 * 3 * 2.0 * 256 * 256 * 8;
+  // per round: the k-steps of one 32-wide stage (four), each three M = 256, N = 256, K = 8 products per pair
+  const double flops = (double)pairs * iters * (tc::BK2 / 8) * 3 * 2.0 * 256 * 256 * 8;
   *tflops = flops / (ms * 1e-3) / 1e12;
   return EMP_OK;
 }
@@ -964,10 +966,13 @@ int mp_model_create(const emp_model_spec* spec, const float* weights, size_t n_f
   m->w3f_maps.resize(T * m->n_pairs);
   m->w3fn_maps.resize(T * m->n_pairs);
   m->w3t_maps.resize(T * m->n_pairs);
+  m->w3t128_maps.resize(T * m->n_pairs);
   for (size_t q = 0; q < T * m->n_pairs; ++q) {
     const size_t wo = q * m->w3_stride();
-    if (make_pair(&m->w3_maps[q], m->w3_hi + wo, m->w3_lo + wo, 4 * C, 64, 64, tc::b_box_rows(4 * (int)C)) != EMP_OK ||
-        make_pair(&m->w3n_maps[q], m->w3_hi + wo, m->w3_lo + wo, C, 64, 64, tc::b_box_rows((int)C)) != EMP_OK ||
+    if (make_pair128(&m->w3_maps[q], m->w3_hi + wo, m->w3_lo + wo, 4 * C, 64, 64, tc::b_box_rows(4 * (int)C)) != EMP_OK ||
+        make_pair128(&m->w3n_maps[q], m->w3_hi + wo, m->w3_lo + wo, C, 64, 64, tc::b_box_rows((int)C)) != EMP_OK ||
+        make_pair128(&m->w3t128_maps[q], m->w3t_hi + wo, m->w3t_lo + wo, 64, 4 * (int)C, 4 * (int)C, tc::b_box_rows(64)) !=
+            EMP_OK ||
         make_pair(&m->w3f_maps[q], m->w3_hi + wo, m->w3_lo + wo, 4 * C, 64, 64, rtc::fwd_bn(4 * (int)C) / 2) != EMP_OK ||
         make_pair(&m->w3fn_maps[q], m->w3_hi + wo, m->w3_lo + wo, C, 64, 64, rtc::fwd_bn((int)C) / 2) != EMP_OK ||
         make_pair(&m->w3t_maps[q], m->w3t_hi + wo, m->w3t_lo + wo, 64, 4 * (int)C, 4 * (int)C, tc::b_box_rows(64)) !=

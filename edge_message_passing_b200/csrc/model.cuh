@@ -36,6 +36,7 @@ struct Model {
   std::vector<MapPair> w3_maps, w3t_maps;      // index t * n_pairs + p
   std::vector<MapPair> w3n_maps;                // the first C rows of W3 (degree-0 scales only)
   std::vector<MapPair> w3f_maps, w3fn_maps;     // the same for the fused radial kernel (its MMA N)
+  std::vector<MapPair> w3t128_maps;             // W3^T for the grouped products (w3t_maps: the fused backward's)
   size_t w3_stride() const { return (size_t)4 * spec.C * 64; }
   // host copy of the radial weights (W1, W2, W3 per layer and pair), for building radial tables
   std::vector<float> rad_host;

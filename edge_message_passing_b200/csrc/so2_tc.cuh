@@ -32,7 +32,8 @@ namespace tc {
 
 constexpr int BM = 128;
 constexpr int BN = 256;
-constexpr int BK = 16;                 // fp32 elements per 64-byte swizzled row
+constexpr int BK = 16;                 // fp32 elements per 64-byte swizzled row (the radial kernels' operands)
+constexpr int BK2 = 32;                // fp32 elements per 128-byte swizzled row (the grouped products' operands)
 constexpr int THREADS = 192;
 constexpr int MAXSUB = 8;
 constexpr int TMEM_COLS = 512;         // two 128 x 256 fp32 accumulators
@@ -40,7 +41,7 @@ constexpr long long TIMEOUT_CYCLES = 4000000000ll;   // default bound of every m
 // The bound in force (clock64 cycles); set by emp_set_wait_limit, read by every bounded wait.
 __device__ long long g_wait_cycles = TIMEOUT_CYCLES;
 
-constexpr int A_BYTES = BM * BK * 4;   // 8 KB
+constexpr int A_BYTES = BM * BK2 * 4;  // 16 KB: 128 rows of one 32-wide k-block
 
 struct Group {
   int M, nsub, mtiles;
@@ -112,6 +113,11 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr) {
   return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(512 >> 4) << 32) |
          ((uint64_t)1 << 46) | ((uint64_t)4 << 61);
 }
+// the same for 128-byte rows: 128-byte swizzle, 8-row groups 1024 B apart
+__device__ __forceinline__ uint64_t sdesc128(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
 
 __device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -154,9 +160,9 @@ __host__ __device__ constexpr int b_box_rows(int n) { return tile_n(n) / 2; }
 // on the leader's full barrier; the MMA completion is multicast to both CTAs' stage
 // and accumulator barriers; the leader takes tiles from the counter and publishes
 // each index to both CTAs (distributed shared memory + remote mbarrier arrive).
-constexpr int ST2 = 6;
-constexpr int B2_BYTES = (BN / 2) * BK * 4;            // 8 KB: half of a 256-row B tile
-constexpr int STAGE2 = 2 * A_BYTES + 2 * B2_BYTES;     // 32 KB per CTA
+constexpr int ST2 = 3;
+constexpr int B2_BYTES = (BN / 2) * BK2 * 4;           // 16 KB: half of a 256-row B tile
+constexpr int STAGE2 = 2 * A_BYTES + 2 * B2_BYTES;     // 64 KB per CTA
 constexpr int EPI_PITCH = 36;                          // floats per staged row (16-byte aligned, conflict-free)
 constexpr int EPI_BYTES = 4 * 32 * EPI_PITCH * 4;      // one 32 x 32 staging tile per epilogue warp
 constexpr int SMEM2 = ST2 * STAGE2 + 1024 + 512 + EPI_BYTES;
@@ -336,20 +342,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       if (t >= total_tiles) break;
       const TileInfo ti = tile_info2(g, t);
       const int a = g.a_idx[ti.sub], b = g.b_idx[ti.sub];
-      const int nk = g.K[ti.sub] / BK;
+      const int nk = g.K[ti.sub] / BK2;
       const int bh = g.bn[ti.sub] / 2;                       // this CTA's B rows
       for (int kc = 0; kc < nk; ++kc, ++it) {
         const int s = it % ST2;
         if (it >= ST2 && !mbar_wait(&empty[s], ((it / ST2) - 1) & 1)) { *vabort = 1; break; }
         if (*vabort) break;
         unsigned char* st = smem + s * STAGE2;
-        if (leader) mbar_expect_tx(&full[s], 2 * (2 * A_BYTES + 2 * bh * BK * 4));
+        if (leader) mbar_expect_tx(&full[s], 2 * (2 * A_BYTES + 2 * bh * BK2 * 4));
         const uint32_t fb = full_l + (uint32_t)(s * 8);
         const int arow = row_base(g, ti.sub) + ti.m0 + (int)rank * BM;
-        tma_load_pair(st, &maps.a_hi[a], fb, g.acol[ti.sub] + kc * BK, arow);
-        tma_load_pair(st + A_BYTES, &maps.a_lo[a], fb, g.acol[ti.sub] + kc * BK, arow);
-        tma_load_pair(st + 2 * A_BYTES, &maps.b_hi[b], fb, kc * BK, ti.n0 + (int)rank * bh);
-        tma_load_pair(st + 2 * A_BYTES + B2_BYTES, &maps.b_lo[b], fb, kc * BK, ti.n0 + (int)rank * bh);
+        tma_load_pair(st, &maps.a_hi[a], fb, g.acol[ti.sub] + kc * BK2, arow);
+        tma_load_pair(st + A_BYTES, &maps.a_lo[a], fb, g.acol[ti.sub] + kc * BK2, arow);
+        tma_load_pair(st + 2 * A_BYTES, &maps.b_hi[b], fb, kc * BK2, ti.n0 + (int)rank * bh);
+        tma_load_pair(st + 2 * A_BYTES + B2_BYTES, &maps.b_lo[b], fb, kc * BK2, ti.n0 + (int)rank * bh);
         *issued = it + 1;
       }
     }
@@ -364,7 +370,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       mbar_arrive(&tq_empty[slot]);
       if (t >= total_tiles) break;
       const TileInfo ti = tile_info2(g, t);
-      const int nk = g.K[ti.sub] / BK;
+      const int nk = g.K[ti.sub] / BK2;
       const int buf = i & 1;
       if (i >= 2 && !mbar_wait_cluster(&acc_empty[buf], ((i >> 1) - 1) & 1)) { ok = false; break; }
       fence_after();
@@ -380,11 +386,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const uint32_t b_hi = a_hi + 2 * A_BYTES;
         const uint32_t b_lo = b_hi + B2_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < BK / 8; ++kk) {
+        for (int kk = 0; kk < BK2 / 8; ++kk) {
           const uint32_t off = kk * 32;
-          mma_tf32_pair(d, sdesc(a_lo + off), sdesc(b_hi + off), idesc, (kc | kk) ? 1u : 0u);
-          mma_tf32_pair(d, sdesc(a_hi + off), sdesc(b_lo + off), idesc, 1u);
-          mma_tf32_pair(d, sdesc(a_hi + off), sdesc(b_hi + off), idesc, 1u);
+          mma_tf32_pair(d, sdesc128(a_lo + off), sdesc128(b_hi + off), idesc, (kc | kk) ? 1u : 0u);
+          mma_tf32_pair(d, sdesc128(a_hi + off), sdesc128(b_lo + off), idesc, 1u);
+          mma_tf32_pair(d, sdesc128(a_hi + off), sdesc128(b_hi + off), idesc, 1u);
         }
         mma_commit_pair(&empty[s]);
       }
@@ -466,7 +472,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
 // ------------------------------------------------------------------ tensor-pipe rate
 // The ceiling the SO(2) products are measured against: each CTA pair issues `iters` rounds of
-// the product kernel's k-stage (for each of the two 8-wide k-steps of a 16-column stage, the
+// the product kernel's k-stage (for each of the four 8-wide k-steps of a 32-column stage, the
 // three 3xTF32 products tcgen05.mma.cta_group::2.kind::tf32 of M = 256, N = 256, K = 8) on
 // operands resident in shared memory, into one TMEM accumulator, then commits once and waits
 // (bounded).  The operands are pseudo-random values of ordinary magnitude so that the pipe
@@ -507,11 +513,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1) k_tf32_rate(
     const uint32_t idesc = idesc_pair(BN);
     for (int it = 0; it < iters; ++it) {
 #pragma unroll
-      for (int kk = 0; kk < BK / 8; ++kk) {
+      for (int kk = 0; kk < BK2 / 8; ++kk) {
         const uint32_t off = kk * 32;
-        mma_tf32_pair(tmem, sdesc(a_lo + off), sdesc(b_hi + off), idesc, (it | kk) ? 1u : 0u);
-        mma_tf32_pair(tmem, sdesc(a_hi + off), sdesc(b_lo + off), idesc, 1u);
-        mma_tf32_pair(tmem, sdesc(a_hi + off), sdesc(b_hi + off), idesc, 1u);
+        mma_tf32_pair(tmem, sdesc128(a_lo + off), sdesc128(b_hi + off), idesc, (it | kk) ? 1u : 0u);
+        mma_tf32_pair(tmem, sdesc128(a_hi + off), sdesc128(b_lo + off), idesc, 1u);
+        mma_tf32_pair(tmem, sdesc128(a_hi + off), sdesc128(b_hi + off), idesc, 1u);
       }
     }
     mma_commit_pair(done);              // arrives on `done` in both CTAs when every MMA has completed
@@ -540,17 +546,19 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// box_cols 16 with the 64-byte swizzle (the radial kernels' operands) or 32 with the 128-byte
+// swizzle (the grouped products' operands)
 inline bool make_map(CUtensorMap* m, const float* base, uint64_t cols, uint64_t rows, uint64_t row_pitch_elems,
-                     uint32_t box_rows) {
+                     uint32_t box_rows, uint32_t box_cols = BK) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {row_pitch_elems * 4};
-  cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            CU_TENSOR_MAP_INTERLEAVE_NONE, box_cols == BK2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 inline int num_sms() {
@@ -568,7 +576,8 @@ inline int num_sms() {
 
 inline int so2_tc_init() {
   if (!tc::encode_fn()) return EMP_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(tc::k_so2_tc2, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM2) != cudaSuccess)
+  if (cudaFuncSetAttribute(tc::k_so2_tc2, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM2) != cudaSuccess ||
+      cudaFuncSetAttribute(tc::k_tf32_rate, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::RATE_SMEM) != cudaSuccess)
     return EMP_ERR_CUDA;
   return EMP_OK;
 }
@@ -608,7 +617,7 @@ inline int tc_group(long long M, int ldc, const GemmSub* subs, int nsub, int* co
   long long first = 0;
   for (int q = 0; q < nsub; ++q) {
     const GemmSub& u = subs[ord[q]];
-    if (u.K % tc::BK != 0 || u.N < 32 || u.N % 32 != 0) return EMP_ERR_ARG;
+    if (u.K % tc::BK2 != 0 || u.N < 32 || u.N % 32 != 0) return EMP_ERR_ARG;
     int a = 0;
     while (a < na && a_seen[a] != u.a_hi) ++a;
     if (a == na) {
@@ -641,14 +650,19 @@ inline int tc_group(long long M, int ldc, const GemmSub* subs, int nsub, int* co
 }
 
 // Tensor maps (hi, lo) of a row-major fp32 matrix [rows][cols] with row pitch ld,
-// tiles of box_rows rows (BM for A operands, min(N, 256) for B operands).
+// tiles of box_rows rows (BM for A operands, min(N, 256) / 2 for B operands): make_pair for the
+// radial kernels (16-column boxes), make_pair128 for the grouped products (32-column boxes).
 struct MapPair {
   CUtensorMap hi, lo;
 };
-inline int make_pair(MapPair* m, const float* hi, const float* lo, long long rows, int cols, int ld, int box_rows) {
-  if (!tc::make_map(&m->hi, hi, cols, rows, ld, box_rows)) return EMP_ERR_CUDA;
-  if (!tc::make_map(&m->lo, lo, cols, rows, ld, box_rows)) return EMP_ERR_CUDA;
+inline int make_pair(MapPair* m, const float* hi, const float* lo, long long rows, int cols, int ld, int box_rows,
+                     int box_cols = tc::BK) {
+  if (!tc::make_map(&m->hi, hi, cols, rows, ld, box_rows, box_cols)) return EMP_ERR_CUDA;
+  if (!tc::make_map(&m->lo, lo, cols, rows, ld, box_rows, box_cols)) return EMP_ERR_CUDA;
   return EMP_OK;
+}
+inline int make_pair128(MapPair* m, const float* hi, const float* lo, long long rows, int cols, int ld, int box_rows) {
+  return make_pair(m, hi, lo, rows, cols, ld, box_rows, tc::BK2);
 }
 
 // Tensor maps of one operand set of the SO(2) mixing: A (hi, lo) rows [M][16C] and a
@@ -663,14 +677,14 @@ inline int so2_make_bmaps(So2BMaps* m, int C, const float* b_hi, const float* b_
   for (int b = 0; b < 4; ++b) {
     const int K = blk_width(b) * C;
     const size_t off = (size_t)wblk_off(b) * C * C;
-    int st = make_pair(&m->blk[b], b_hi + off, b_lo + off, K, K, K, tc::b_box_rows(K));
+    int st = make_pair128(&m->blk[b], b_hi + off, b_lo + off, K, K, K, tc::b_box_rows(K));
     if (st != EMP_OK) return st;
   }
   return EMP_OK;
 }
 
 inline int so2_make_amaps(So2AMaps* m, int C, long long M, const float* a_hi, const float* a_lo) {
-  return make_pair(m, a_hi, a_lo, M, 16 * C, 16 * C, tc::BM);
+  return make_pair128(m, a_hi, a_lo, M, 16 * C, 16 * C, tc::BM);
 }
 
 struct So2Part {

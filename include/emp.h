@@ -283,7 +283,7 @@ int emp_last_device_error(void);
 /* ------------------------------------------------------------ tensor-pipe rate
  * Measures the TF32 rate of the tensor cores in the form the SO(2) products use
  * (tcgen05.mma.cta_group::2.kind::tf32, M = 256, N = 256, K = 8, operands resident in
- * shared memory): one CTA pair per two SMs issues `iters` rounds of six products, timed
+ * shared memory): one CTA pair per two SMs issues `iters` rounds of twelve products, timed
  * with CUDA events on `stream` (synchronises).  tflops (host, out): TF32 flops per
  * second / 1e12, counting every product; a 3xTF32 product does three of them. */
 int emp_tf32_mma_rate(int32_t iters, cudaStream_t stream, double* tflops);
