@@ -44,7 +44,7 @@ constexpr int THREADS = 32 * (HID_W0 + HID_WARPS);
 constexpr int KB = 4;                            // 16-wide k-blocks of h2 (K = 64)
 constexpr int AK_BYTES = BM * 64;                // one k-block of hi (or lo): 128 rows x 64 bytes
 constexpr int ABUF_BYTES = 2 * KB * AK_BYTES;    // hi k-blocks, then lo k-blocks: 64 KB
-constexpr int BST = 4;                           // W3 ring stages
+constexpr int BST = 5;                           // W3 ring stages
 constexpr int BHALF = 64 * 64;                   // hi (or lo) half of a stage: up to 64 rows x 64 bytes
 constexpr int BSTAGE_BYTES = 2 * BHALF;
 constexpr int NACC = 3;                          // head accumulators (ring of n-tiles)
