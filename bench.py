@@ -382,18 +382,27 @@ def other_configs(emp, torch, stream, flush, hbm_gbs: float, steps: int = 10):
     emp.profile_enable(True)
     ms_g = timed(lambda: emp.mp_energy_weight_grad(model, g, sp))
     red_ms = emp.profile_read("weight_grad")[0] / (steps + 3)
+    blk_ms = emp.profile_read("wgrad_blocks")[0] / (steps + 3)
     emp.profile_enable(False)
     C = spec.C
-    # FLOPs of the sums over edges and nodes: the middle layers' SO(2) blocks, the radial W3 (C or 4C
-    # rows), W2, W1 of every layer, and the end layers' per-node W0 sums
-    flops = (2.0 * E * 72 * C * C * max(T - 2, 0)
-             + 2.0 * E * 64 * (C + 4 * C * (T - 1)) + 2.0 * T * E * (64 * 64 + 64 * 8)
+    # FLOPs of the sums over edges and nodes: the middle layers' SO(2) blocks (3xTF32 products on the
+    # tensor cores, with the transposes that make the edge index their K), and on SIMT the radial W3
+    # (C or 4C rows), W2, W1 of every layer and the end layers' per-node W0 sums
+    blk_flops = 2.0 * E * 72 * C * C * max(T - 2, 0)
+    flops = (2.0 * E * 64 * (C + 4 * C * (T - 1)) + 2.0 * T * E * (64 * 64 + 64 * 8)
              + 2.0 * st.pos.shape[0] * (16 * C * C + 4 * C * C))
     clk = _sm_clock_mhz(torch)
     fp32_peak = 148 * 128 * 2 * clk * 1e6 / 1e12 if clk else None          # FMA lanes x 2 flops x SM clock
+    rates = sorted(emp.tf32_mma_rate(20000) for _ in range(5))
+    tf32_peak = rates[len(rates) // 2] / 3.0                                # 3xTF32: three products each
     out[WORKLOAD + "_weight_grad"] = {
         "ms_per_call": round(ms_g, 3), "edges_per_s": E / (ms_g * 1e-3), "timed": "eager call",
-        "reductions": {"ms": round(red_ms, 3), "flops": flops, "achieved_tflops": round(flops / (red_ms * 1e-3) / 1e12, 2),
+        "so2_block_sums": {"ms": round(blk_ms, 3), "flops": blk_flops,
+                           "achieved_tflops": round(blk_flops / (blk_ms * 1e-3) / 1e12, 2) if blk_ms > 0 else None,
+                           "bound": "tensor", "peak_tflops": round(tf32_peak, 1) if tf32_peak else None,
+                           "frac": round(blk_flops / (blk_ms * 1e-3) / 1e12 / tf32_peak, 3) if tf32_peak and blk_ms > 0 else None,
+                           "peak_note": "the measured 3xTF32 rate of the products (as for the mixing); the time includes the transposes"},
+        "other_sums": {"ms": round(red_ms, 3), "flops": flops, "achieved_tflops": round(flops / (red_ms * 1e-3) / 1e12, 2),
                        "bound": "alu", "peak_tflops": round(fp32_peak, 1) if fp32_peak else None,
                        "frac": round(flops / (red_ms * 1e-3) / 1e12 / fp32_peak, 3) if fp32_peak else None,
                        "peak_note": "FP32 FMA: 148 SMs x 128 lanes x 2 flops x the SM clock read at the start"},

@@ -74,12 +74,12 @@ inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 
 // ------------------------------------------------------------------ workspace layout
 struct WsLayout {
-  size_t gxP2, D, dist, R, rbP, nodeZ, nodeX, zro, dB, tnp, silu, radrows, gxP, XT2, XTlo2, Y2, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
+  size_t gxP2, D, dist, R, rbP, nodeZ, nodeX, zro, dB, tnp, silu, radrows, trT, trTmp, trPad, gxP, XT2, XTlo2, Y2, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
   size_t total;
 };
 
 // partial sums of the weight-gradient reductions (k_tn): room for the largest splits used
-constexpr int TN_SPLITS = 64;
+constexpr int TN_SPLITS = 296;     // row splits of a reduction: up to two blocks per SM when it has few output tiles
 inline size_t tn_part_floats(int C) { return std::max((size_t)16 * 36 * C * C, (size_t)TN_SPLITS * 4 * C * 64); }
 
 WsLayout ws_layout(const Model& m, long long E, int N, bool grad = false) {
@@ -140,6 +140,11 @@ WsLayout ws_layout(const Model& m, long long E, int N, bool grad = false) {
     L.tnp = take(tn_part_floats((int)C) * 4);
     L.silu = take((size_t)N * std::max(m.Hro, 1) * 4);
     L.radrows = take((size_t)E * RAD_ROW_FLOATS * 4);
+    // the SO(2) block sums on the tensor cores: a cohort pair's g_y and x~ (hi, lo) transposed to
+    // [16C][rows padded to 32], and one block's product before it is added to dB
+    L.trPad = (2 * coh + 31) / 32 * 32;
+    L.trT = take(4 * (size_t)16 * C * L.trPad * 4);
+    L.trTmp = take((size_t)tc::MAXSUB * 6 * C * 6 * C * 4);
   }
   L.total = o;
   return L;
@@ -233,6 +238,69 @@ void tn_sum(int Na, int Nb, int rows, int w, const float* A, const float* A2, lo
   }
   Scope sc_("weight_grad", s);
   k_tn_reduce<<<(unsigned)((Na * Nb + 255) / 256), 256, 0, s>>>(splits, Na, Nb, part, out, ldo, accumulate ? 1 : 0);
+}
+
+// dst[c][r] = src[r][c] for r < rows (dst rows ld_dst floats apart), 0 for rows <= r < ld_dst:
+// 32 x 32 tiles through shared memory
+__global__ void k_transpose_pad(const float* __restrict__ src, int rows, int cols, long long ld_src,
+                                float* __restrict__ dst, int ld_dst) {
+  __shared__ float tile[32][33];
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int k = threadIdx.y; k < 32; k += blockDim.y) {
+    const int r = r0 + k, c = c0 + threadIdx.x;
+    tile[k][threadIdx.x] = (r < rows && c < cols) ? src[(size_t)r * ld_src + c] : 0.f;
+  }
+  __syncthreads();
+  for (int k = threadIdx.y; k < 32; k += blockDim.y) {
+    const int c = c0 + k, r = r0 + threadIdx.x;
+    if (c < cols && r < ld_dst) dst[(size_t)c * ld_dst + r] = tile[threadIdx.x][k];
+  }
+}
+
+// dB_b += sum over the rows of a cohort pair of g_y (x) x~ for the four SO(2) blocks, as 3xTF32
+// products on the tensor cores: the hi and lo rows transposed (the row index becomes K, padded with
+// zero rows to a multiple of 32).  Per block the rows are cut into up to eight K-chunks, one
+// product each (a sub-problem of one launch: eight times the output tiles, and each accumulator
+// sums at most a few thousand rows in tensor memory); the chunks' products are then added to dB
+// in FP32, in chunk order.
+int so2_block_sums(int C, long long M, const float* GYhi, const float* GYlo, const float* XThi, const float* XTlo,
+                   float* dB, void* ws, const WsLayout& L, int* counter, cudaStream_t s) {
+  const int pad = (int)((M + 31) / 32 * 32);
+  if (pad > (int)L.trPad) return EMP_ERR_ARG;
+  float* T = at<float>(ws, L.trT);
+  const size_t plane = (size_t)16 * C * L.trPad;
+  const float* src[4] = {GYhi, GYlo, XThi, XTlo};
+  {
+    Scope sc_("wgrad_blocks", s);
+    const dim3 grid((unsigned)((16 * C + 31) / 32), (unsigned)(pad / 32));
+    for (int q = 0; q < 4; ++q)
+      k_transpose_pad<<<grid, dim3(32, 8), 0, s>>>(src[q], (int)M, 16 * C, 16ll * C, T + q * plane, (int)L.trPad);
+  }
+  const int csz = ((pad + tc::MAXSUB - 1) / tc::MAXSUB + 31) / 32 * 32;   // rows per K-chunk
+  const int nch = (pad + csz - 1) / csz;
+  float* tmp = at<float>(ws, L.trTmp);
+  for (int b = 0; b < 4; ++b) {
+    const int K = blk_width(b) * C, o = blk_off(b) * C;
+    MapPair a, bm[tc::MAXSUB];
+    int st = make_pair128(&a, T + (size_t)o * L.trPad, T + plane + (size_t)o * L.trPad, K, pad, (int)L.trPad, tc::BM);
+    if (st != EMP_OK) return st;
+    GemmSub subs[tc::MAXSUB];
+    for (int c = 0; c < nch; ++c) {
+      const int k0 = c * csz, kn = std::min(csz, pad - k0);
+      st = make_pair128(&bm[c], T + 2 * plane + (size_t)o * L.trPad + k0, T + 3 * plane + (size_t)o * L.trPad + k0, K,
+                        kn, (int)L.trPad, tc::b_box_rows(K));
+      if (st != EMP_OK) return st;
+      subs[c] = GemmSub{&a.hi, &a.lo, &bm[c].hi, &bm[c].lo, k0, kn, K, 0, tmp + (size_t)c * K * K};
+    }
+    {
+      Scope sc_("wgrad_blocks", s);
+      st = tc_group(K, K, subs, nch, counter, s);
+    }
+    if (st != EMP_OK) return st;
+    Scope sc_("wgrad_blocks", s);
+    k_tn_reduce<<<(unsigned)((K * K + 255) / 256), 256, 0, s>>>(nch, K, K, tmp, dB + (size_t)wblk_off(b) * C * C, K, 1);
+  }
+  return cudaGetLastError() == cudaSuccess ? EMP_OK : EMP_ERR_CUDA;
 }
 
 // float offsets of each weight in the blob order (include/emp.h: mp_weight_count)
@@ -1361,12 +1429,10 @@ static int energy_forces_impl(const Model& m, const emp_graph* g, const int32_t*
         So2Part parts[2] = {{am_xt.get(M), &m.bmaps_fwd[t], Y}, {am_gy.get(M), &m.bmaps_bwd[t], GXT}};
         st = so2_product(m, M, parts, 2, counter, stream);
         if (st != EMP_OK) return st;
-        if (wgrad)   // dB_b += sum over the cohorts' edges of g_y (x) x~ per block (both as their hi + lo)
-          for (int b = 0; b < 4; ++b) {
-            const int K = blk_width(b) * C, o = blk_off(b) * C;
-            tn_sum(K, K, (int)M, 1, GYhi + o, GYlo + o, 16ll * C, 0, XT + o, XTlo + o, 16ll * C, 0,
-                   dB + (size_t)wblk_off(b) * C * C, K, true, tnp, tn_part_floats(C), stream);
-          }
+        if (wgrad) {   // dB_b += sum over the cohorts' edges of g_y (x) x~ per block (both as their hi + lo)
+          st = so2_block_sums(C, M, GYhi, GYlo, XT, XTlo, dB, ws, L, counter, stream);
+          if (st != EMP_OK) return st;
+        }
         for (long long e0 = g0; e0 < g1; e0 += coh, ++ci) {
           const long long e1 = std::min(g1, e0 + coh), n = e1 - e0;
           const size_t ro = (size_t)(e0 - g0) * 16 * C;     // the cohort's rows in the pair's buffers

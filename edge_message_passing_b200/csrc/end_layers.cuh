@@ -505,7 +505,8 @@ struct TnArgs {
   int b_comp;
   float* part;
 };
-constexpr int TN_T = 128, TN_K = 16;       // output tile edge, rows per staged step
+constexpr int TN_T = 128, TN_K = 32;       // output tile edge, rows per staged step
+constexpr int TN_PER = TN_K * TN_T / 256;  // staged elements of each operand per thread and step
 __global__ void __launch_bounds__(256) k_tn(const __grid_constant__ TnArgs p) {
   __shared__ __align__(16) float As[TN_K][TN_T + 4];
   __shared__ __align__(16) float Bs[TN_K][TN_T + 4];
@@ -519,24 +520,37 @@ __global__ void __launch_bounds__(256) k_tn(const __grid_constant__ TnArgs p) {
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-  for (int rb = r_begin; rb < r_end; rb += TN_K) {
-    __syncthreads();
+  // thread t stages column t % 128 of rows t / 128 + 2 i of a step; the next step's values are
+  // loaded into registers while this step is computed
+  const int cc = t & (TN_T - 1), r_lane = t >> 7;
+  float pa[TN_PER], pb[TN_PER];
+  auto load = [&](int rb) {
 #pragma unroll
-    for (int q = t; q < TN_K * TN_T; q += 256) {
-      const int rr = q / TN_T, cc = q % TN_T;
-      const int r = rb + rr;
+    for (int i = 0; i < TN_PER; ++i) {
+      const int r = rb + r_lane + 2 * i;
       float av = 0.f, bv = 0.f;
       if (r < r_end) {
-        const long long ao = (long long)(r / p.w) * p.a_node + (long long)(r % p.w) * p.a_comp;
-        const long long bo = (long long)(r / p.w) * p.b_node + (long long)(r % p.w) * p.b_comp;
+        const int rn = p.w == 1 ? r : r / p.w, rc = p.w == 1 ? 0 : r % p.w;
+        const long long ao = (long long)rn * p.a_node + (long long)rc * p.a_comp;
+        const long long bo = (long long)rn * p.b_node + (long long)rc * p.b_comp;
         if (a0 + cc < p.Na) av = p.A[ao + a0 + cc] + (p.A2 ? p.A2[ao + a0 + cc] : 0.f);
         if (b0 + cc < p.Nb) bv = p.B[bo + b0 + cc] + (p.B2 ? p.B2[bo + b0 + cc] : 0.f);
       }
-      As[rr][cc] = av;
-      Bs[rr][cc] = bv;
+      pa[i] = av;
+      pb[i] = bv;
+    }
+  };
+  if (r_begin < r_end) load(r_begin);
+  for (int rb = r_begin; rb < r_end; rb += TN_K) {
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < TN_PER; ++i) {
+      As[r_lane + 2 * i][cc] = pa[i];
+      Bs[r_lane + 2 * i][cc] = pb[i];
     }
     __syncthreads();
-#pragma unroll 4
+    if (rb + TN_K < r_end) load(rb + TN_K);
+#pragma unroll 8
     for (int kk = 0; kk < TN_K; ++kk) {
       const float4 a_lo = *reinterpret_cast<const float4*>(&As[kk][4 * ty]);
       const float4 a_hi = *reinterpret_cast<const float4*>(&As[kk][64 + 4 * ty]);
