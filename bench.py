@@ -6,7 +6,7 @@ Workload: the seeded N=4096 diamond (8x8x8 conventional cells, sigma 0.02 A,
 seed 2), cutoff 6 A (E = 647168 directed edges), C = 128, lmax = 3, three gated
 residual layers, 8192-edge receiver-sorted cohorts.  One step = mp_energy_forces
 on the frame's resident neighbour graph: forward (radial, rotate, SO(2) mixing,
-rotate back, receiver sums, gates, readout) + recomputing backward + forces.  The
+rotate back, receiver sums, gates, readout) + backward + forces.  The
 neighbour list build is timed on its own (nl_ms) and is part of the end-to-end
 figure (e2e), not of the step.  Metric: edges/s = E / step time (whole job:
 summed over replicas).
@@ -221,8 +221,8 @@ def alg_bytes_step(name: str, C: int, T: int, E: int, N: int) -> float:
     last = 1 if T >= 2 else 0
     if name == "rotate_in":               # R row in; x~ hi/lo out
         return mid * E * (4 * C * 4 + 2 * row + d)
-    if name == "bwd_prep":                # R row in; x~ hi/lo and g_y hi/lo out
-        return mid * E * (4 * C * 4 + 4 * row + d)
+    if name == "bwd_prep":                # D in; g_y hi/lo out (y is kept from the forward: no x~)
+        return mid * E * (2 * row + d)
     if name == "bwd_edge":                # y, g_x~, R, D in; dE/dR hi/lo out
         return mid * E * (2 * row + 4 * C * 4 + d + 2 * 4 * C * 4)
     if name == "rotate_back_scatter":     # y, D in
@@ -577,9 +577,9 @@ def run_ours(args):
     if so2_launches:
         so2_ms = fam["so2_tc"][0] / so2_launches
         # per step: the per-edge products run in the layers between the first and the last (the end
-        # layers mix once per node, end_layers.cuh); each mixes every edge three times (forward,
-        # backward recompute, backward transpose), 2*72*C^2 useful flops each
-        flops_step = E * 2 * C * C * 3 * 72 * max(T - 2, 0)
+        # layers mix once per node, end_layers.cuh); each mixes every edge twice (forward, backward
+        # transpose: the backward reads y kept from the forward), 2*72*C^2 useful flops each
+        flops_step = E * 2 * C * C * 2 * 72 * max(T - 2, 0)
         achieved = flops_step * len(ptimes) / (fam["so2_tc"][0] * 1e-3) / 1e12
         # the reference: the measured TF32 rate of the same tcgen05 products (operands resident in
         # shared memory, ~0.5 s back to back right after the step) / 3 for 3xTF32
@@ -593,7 +593,7 @@ def run_ours(args):
                 "launch_ms": so2_ms, "launches_per_step": so2_launches / len(ptimes), "dominant": dom == "so2_tc",
                 "peak_measured_tf32": tf32_rate, "peak_measured_tf32_first_launch": tf32_rate_first,
                 "peak_bf16_derived": bf16_derived, "frac_vs_bf16_derived": achieved / bf16_derived,
-                "peak_note": f"useful FP32 flops of the per-edge mixings (2*72*C^2 per edge and mixing, three "
+                "peak_note": f"useful FP32 flops of the per-edge mixings (2*72*C^2 per edge and mixing, two "
                              f"mixings in each of the {max(T - 2, 0)} layers between the first and the last) over "
                              f"the summed launch event time (CUDA events on the launching stream), vs the "
                              f"measured TF32 rate of tcgen05.mma.cta_group::2.kind::tf32 (M=N=256, K=8, "

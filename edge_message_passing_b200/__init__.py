@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libemp.so")
 # exported symbols (kept in step with include/emp.h)
 SYMBOLS = (
     "nl_workspace_bytes", "nl_build", "nl_build_noalloc", "mp_weight_count", "mp_model_create", "mp_model_destroy",
-    "mp_workspace_bytes", "mp_forward", "mp_energy_forces", "mp_so2_mix", "mp_chain_create",
+    "mp_workspace_bytes", "mp_workspace_bytes_min", "mp_forward", "mp_energy_forces", "mp_so2_mix", "mp_chain_create",
     "mp_chain_destroy", "mp_radial_chain", "emp_status_string", "emp_last_device_error",
     "emp_profile_enable", "emp_profile_read", "emp_profile_names", "emp_launch_count",
     "emp_set_wait_limit", "emp_wait_selftest", "emp_tf32_split_selftest", "emp_tf32_mma_rate", "mp_model_radial_tables", "mp_radial_hidden",
@@ -88,6 +88,8 @@ def lib() -> ctypes.CDLL:
         L.mp_model_destroy.argtypes = [vp]
         L.mp_workspace_bytes.restype = sz
         L.mp_workspace_bytes.argtypes = [vp, i64, i32]
+        L.mp_workspace_bytes_min.restype = sz
+        L.mp_workspace_bytes_min.argtypes = [vp, i64, i32]
         L.mp_forward.restype = ctypes.c_int
         L.mp_forward.argtypes = [vp, ctypes.POINTER(GraphC), i32, vp, vp, vp, vp, sz, vp]
         L.mp_energy_forces.restype = ctypes.c_int
@@ -354,6 +356,9 @@ class Model:
     def workspace_bytes(self, n_edges: int, n_atoms: int) -> int:
         return lib().mp_workspace_bytes(self.handle, n_edges, n_atoms)
 
+    def workspace_bytes_min(self, n_edges: int, n_atoms: int) -> int:
+        return lib().mp_workspace_bytes_min(self.handle, n_edges, n_atoms)
+
     def radial_tables(self, tol: float = 1e-7) -> int:
         """Switch the radial hidden layers to certified Chebyshev tables (tol > 0; returns
         the number of pieces) or back to the network (tol <= 0)."""
@@ -372,25 +377,29 @@ def mp_forward(model: Model, graph: Graph, layer: int, species, x):
     torch = _torch()
     x = x.contiguous()
     agg = torch.empty_like(x)
-    ws = _workspace(model.workspace_bytes(graph.n_edges, graph.n_atoms))
+    ws = _workspace(model.workspace_bytes_min(graph.n_edges, graph.n_atoms))
     gc = graph.c()
     _check(lib().mp_forward(model.handle, ctypes.byref(gc), layer, _ptr(species), _ptr(x), _ptr(agg), _ptr(ws),
                             ws.numel(), _stream()), "mp_forward")
     return agg
 
 
-def mp_energy_forces(model: Model, graph: Graph, species, virial: bool = False, atom_energy: bool = False):
-    """(energy [1] float64, forces [N,3], virial [3,3] or None, atom energies [N] or None)."""
+def mp_energy_forces(model: Model, graph: Graph, species, virial: bool = False, atom_energy: bool = False,
+                     compact: bool = False):
+    """(energy [1] float64, forces [N,3], virial [3,3] or None, atom energies [N] or None).
+    compact: run in the smallest workspace (the backward recomputes the per-edge mixing outputs
+    instead of keeping them from the forward); the results are the same bits."""
     torch = _torch()
     N = graph.n_atoms
     energy = torch.empty(1, dtype=torch.float64, device="cuda")
     forces = torch.empty((N, 3), dtype=torch.float32, device="cuda")
     vir = torch.empty((3, 3), dtype=torch.float32, device="cuda") if virial else None
     ea = torch.empty(N, dtype=torch.float32, device="cuda") if atom_energy else None
-    ws = _workspace(model.workspace_bytes(graph.n_edges, N))
+    nbytes = (model.workspace_bytes_min if compact else model.workspace_bytes)(graph.n_edges, N)
+    ws = _workspace(nbytes)
     gc = graph.c()
     _check(lib().mp_energy_forces(model.handle, ctypes.byref(gc), _ptr(species), _ptr(energy), _ptr(forces),
-                                  _ptr(vir), _ptr(ea), _ptr(ws), ws.numel(), _stream()), "mp_energy_forces")
+                                  _ptr(vir), _ptr(ea), _ptr(ws), nbytes, _stream()), "mp_energy_forces")
     return energy, forces, vir, ea
 
 

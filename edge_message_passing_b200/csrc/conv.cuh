@@ -1,4 +1,4 @@
-// Per-edge kernels of the SO(2) message-passing layer and its recomputing
+// Per-edge kernels of the SO(2) message-passing layer and its cohort-wise
 // backward (page "first-order SO(2) input-gradient path": the reverse mixing
 // chain is finished one receiver-sorted 8192-edge cohort at a time; page
 // "deepmd-kit PR #6108": radial basis -> radial network; the model's steps are
@@ -642,7 +642,7 @@ __global__ void k_gate_bwd(int N, int C, float inv_avg, int gated, const float* 
   }
 }
 
-// per edge, from y (recomputed), g_y and g_x~ = W^T g_y:
+// per edge, from y (kept from the forward, or recomputed), g_y and g_x~ = W^T g_y:
 //   gR[e][l][c] = sum_m g_x~ u;  g_u = R (.) g_x~;  g_xs = D^T g_u (-> GXS, [16][C] rows)
 //   b_j = sum_c (y^T J_j g_y + g_u^T J_j u), j = x, y (edge frame); a = -R_e^T (b_x, b_y, 0);
 //   g_r[e] += (a x r) / |r|^2  (direction part of dE/dr; the radial part is added by k_radial_bwd)
@@ -947,7 +947,9 @@ __global__ void k_gx_combine(long long e0, long long e1, int C, int cohort_idx, 
 // ------------------------------------------------------------------ staged rotate-in / backward prep
 // Rotate-in (BWD = false): XT[e - e0][col(k) C + c] = R_e[l(k)][c] (D_e x_send)[k][c] in
 // the edge frame, m-major columns, split hi/lo for the products.  Backward prep (BWD =
-// true): also GY = D_e gS[recv] (edge-frame output gradient), split.  x~ and g_y rows are 16C
+// true): also GY = D_e gS[recv] (edge-frame output gradient), split.  Rotate-in with R null
+// rotates the rows unscaled: called with the receivers as `send` and gS as `x`, it writes g_y
+// alone (the backward prep when y is kept from the forward).  x~ and g_y rows are 16C
 // floats.  One block of C / V threads (V adjacent channels each, vector loads and stores) per
 // contiguous range of `per` edges.  The rows
 // an edge reads (x of the sender, gS of the receiver, R and its Wigner-D blocks) are
@@ -1023,7 +1025,8 @@ __global__ void __launch_bounds__(256)
   }
   __syncthreads();
   constexpr bool SG = BWD && RS_STAGE_G;
-  const uint32_t bX = 64u * C, bG = SG ? 64u * C : 0u, bR = 16u * C;
+  const bool hasR = R != nullptr;      // forward form without R: the rows are rotated unscaled
+  const uint32_t bX = 64u * C, bG = SG ? 64u * C : 0u, bR = hasR ? 16u * C : 0u;
   const int offG = 16 * C, offR = (SG ? 32 : 16) * C, offD = offR + 4 * C;
   auto issue = [&](int q) {
     const int s = q % RS_STAGES;
@@ -1032,7 +1035,7 @@ __global__ void __launch_bounds__(256)
     tc::mbar_expect_tx(&full[s], bX + bG + bR + NDBLK * 4);
     bulk_g2s(st, x + (size_t)m.x * 16 * C, bX, &full[s]);
     if (SG) bulk_g2s(st + offG, gS + (size_t)m.y * 16 * C, bG, &full[s]);
-    bulk_g2s(st + offR, R + (size_t)m.z * 4 * C, bR, &full[s]);
+    if (hasR) bulk_g2s(st + offR, R + (size_t)m.z * 4 * C, bR, &full[s]);
     bulk_g2s(st + offD, D + (size_t)(e0 + p0 + q) * NDBLK, NDBLK * 4, &full[s]);
   };
   int nissued = 0;                     // positions whose copies thread 0 has issued
@@ -1053,14 +1056,14 @@ __global__ void __launch_bounds__(256)
     const T* sR = reinterpret_cast<const T*>(st + offR) + t;
     const float* Dr = st + offD;
     const size_t ro = (size_t)(p0 + q) * 16 * CV + t;
-    rotate_write_degree_v<0>(Dr, sX, CV, sR[0], XTv + ro, XLv + ro);
-    rotate_write_degree_v<1>(Dr, sX, CV, sR[CV], XTv + ro, XLv + ro);
-    rotate_write_degree_v<2>(Dr, sX, CV, sR[2 * CV], XTv + ro, XLv + ro);
-    rotate_write_degree_v<3>(Dr, sX, CV, sR[3 * CV], XTv + ro, XLv + ro);
+    const T one = vset<T>(1.f);
+    rotate_write_degree_v<0>(Dr, sX, CV, hasR ? sR[0] : one, XTv + ro, XLv + ro);
+    rotate_write_degree_v<1>(Dr, sX, CV, hasR ? sR[CV] : one, XTv + ro, XLv + ro);
+    rotate_write_degree_v<2>(Dr, sX, CV, hasR ? sR[2 * CV] : one, XTv + ro, XLv + ro);
+    rotate_write_degree_v<3>(Dr, sX, CV, hasR ? sR[3 * CV] : one, XTv + ro, XLv + ro);
     if (BWD) {
       const T* sG = SG ? reinterpret_cast<const T*>(st + offG) + t
                        : reinterpret_cast<const T*>(gS + (size_t)meta[q].y * 16 * C) + t;
-      const T one = vset<T>(1.f);
       rotate_write_degree_v<0>(Dr, sG, CV, one, GHv + ro, GLv + ro);
       rotate_write_degree_v<1>(Dr, sG, CV, one, GHv + ro, GLv + ro);
       rotate_write_degree_v<2>(Dr, sG, CV, one, GHv + ro, GLv + ro);

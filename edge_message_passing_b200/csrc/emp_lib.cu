@@ -75,6 +75,8 @@ inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 // ------------------------------------------------------------------ workspace layout
 struct WsLayout {
   size_t gxP2, D, dist, R, rbP, nodeZ, nodeX, zro, dB, tnp, silu, radrows, trT, trTmp, trPad, gxP, XT2, XTlo2, Y2, gRhi, gRlo, h2hi, h2lo, gh2, pperm, pinv, poff, g_r, xs, aggs, gx0, gx1, gS, e_atom, XT, Y, GXT, XTlo, GYhi, GYlo, perm, seg, nseg, vir, counter;
+  size_t Ykeep = 0;          // y of every per-edge layer, kept from the forward (keep_y)
+  bool keep_y = false;
   size_t total;
 };
 
@@ -82,8 +84,12 @@ struct WsLayout {
 constexpr int TN_SPLITS = 296;     // row splits of a reduction: up to two blocks per SM when it has few output tiles
 inline size_t tn_part_floats(int C) { return std::max((size_t)16 * 36 * C * C, (size_t)TN_SPLITS * 4 * C * 64); }
 
-WsLayout ws_layout(const Model& m, long long E, int N, bool grad = false) {
+// keep_y: the layers between the first and the last keep their per-edge mixing outputs y
+// [E][16C] from the forward for the backward (one product fewer per cohort there, and no x~ in
+// the backward prep); without it the backward recomputes y from x~ cohort by cohort.
+WsLayout ws_layout(const Model& m, long long E, int N, bool grad = false, bool keep_y = false) {
   WsLayout L{};
+  L.keep_y = keep_y;
   const size_t C = m.spec.C, T = m.spec.n_layers;
   const size_t coh = std::min<long long>(m.spec.cohort_edges, std::max<long long>(E, 1));
   const size_t ncoh = E > 0 ? (E + m.spec.cohort_edges - 1) / m.spec.cohort_edges : 0;
@@ -125,8 +131,10 @@ WsLayout ws_layout(const Model& m, long long E, int N, bool grad = false) {
   L.XT2 = L.XT + cb;
   L.XTlo = take(2 * cb);
   L.XTlo2 = L.XTlo + cb;
-  L.Y = take(2 * cb);
-  L.Y2 = L.Y + cb;
+  if (!keep_y) {
+    L.Y = take(2 * cb);
+    L.Y2 = L.Y + cb;
+  }
   L.GXT = take(2 * cb);
   L.GYhi = take(2 * cb);
   L.GYlo = take(2 * cb);
@@ -146,8 +154,17 @@ WsLayout ws_layout(const Model& m, long long E, int N, bool grad = false) {
     L.trT = take(4 * (size_t)16 * C * L.trPad * 4);
     L.trTmp = take((size_t)tc::MAXSUB * 6 * C * 6 * C * 4);
   }
+  if (keep_y && T > 2) L.Ykeep = take((T - 2) * (size_t)E * 16 * C * 4);
   L.total = o;
   return L;
+}
+
+// The layout an energy call runs with: y kept from the forward when the workspace (less `extra`
+// bytes the call places after the layout) holds it, else recomputed in the backward.
+WsLayout call_layout(const Model& m, long long E, int N, bool grad, size_t ws_bytes, size_t extra) {
+  WsLayout L = ws_layout(m, E, N, grad, true);
+  if (ws_bytes >= L.total + extra) return L;
+  return ws_layout(m, E, N, grad, false);
 }
 
 template <typename T>
@@ -192,7 +209,7 @@ int grid_for(long long n, int per, int cap = 148 * 32) {
 }
 
 // SO(2) block products of a cohort on the tensor cores (3xTF32, operands pre-split):
-// one operand set (forward) or two sharing the rows (backward: recompute + transpose)
+// one operand set (forward; backward transpose) or two sharing the rows (backward: recompute + transpose)
 int so2_product(const Model& m, long long M, const So2Part* parts, int nparts, int* counter, cudaStream_t s) {
   Scope sc_("so2_tc", s);
   return so2_tc(M, m.spec.C, parts, nparts, counter, s);
@@ -416,8 +433,10 @@ Side side_for(cudaStream_t s) {
 
 // [per-edge product launches: begin] (bench.py ties the mixing's DRAM traffic figure to this text)
 // forward of layer t over all cohorts: S (raw receiver sums) from x (all degrees)
+// Ykeep: where y of all E edges goes (rows in edge order, kept for the backward), or null (the
+// cohort buffers)
 int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, const float* D, const float* R, const int* rrow,
-                  float* S, void* ws, const WsLayout& L, cudaStream_t s) {
+                  float* S, void* ws, const WsLayout& L, cudaStream_t s, float* Ykeep = nullptr) {
   const int C = m.spec.C;
   const long long E = g->n_edges, coh = m.spec.cohort_edges;
   float* XT[2] = {at<float>(ws, L.XT), at<float>(ws, L.XT2)};
@@ -440,6 +459,8 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
     const long long ee[3] = {e0, e1, two ? e1 + (e1 - e0) : e1};
     const int nc = two ? 2 : 1;
     const long long M = e1 - e0;
+    if (Ykeep)
+      for (int b = 0; b < nc; ++b) Y[b] = Ykeep + (size_t)ee[b] * 16 * C;
     for (int b = 0; b < nc; ++b) {
       const int per = rs_per(M, tc::num_sms(), 6);
       Scope sc_("rotate_in", s);
@@ -1195,6 +1216,11 @@ int mp_radial_hidden(const void* model, int32_t layer, int32_t pair, int64_t n, 
 
 size_t mp_workspace_bytes(const void* model, int64_t n_edges, int32_t n_atoms) {
   if (!model || n_edges < 0 || n_atoms < 1) return 0;
+  return ws_layout(*static_cast<const Model*>(model), n_edges, n_atoms, false, true).total;
+}
+
+size_t mp_workspace_bytes_min(const void* model, int64_t n_edges, int32_t n_atoms) {
+  if (!model || n_edges < 0 || n_atoms < 1) return 0;
   return ws_layout(*static_cast<const Model*>(model), n_edges, n_atoms).total;
 }
 
@@ -1249,9 +1275,10 @@ static int energy_forces_impl(const Model& m, const emp_graph* g, const int32_t*
   const int N = g->n_atoms, C = m.spec.C, T = m.spec.n_layers;
   const bool wgrad = grad != nullptr;
   const bool tables = !wgrad;           // weight gradients need the radial network itself
-  const WsLayout L = ws_layout(m, E, N, wgrad);
   const long long E_all = sh ? sh->global->n_edges : E;
-  const size_t shard_extra = sh ? align_up((size_t)E_all * 12 + 4) : 0;   // the whole graph's g_r
+  // sharded: the whole graph's g_r, then the rank's receiver offsets, after the layout
+  const size_t shard_extra = sh ? align_up((size_t)E_all * 12 + 4) + align_up((size_t)(N + 1) * 4) : 0;
+  const WsLayout L = call_layout(m, E, N, wgrad, ws_bytes, shard_extra);
   if (ws_bytes < L.total + shard_extra) return EMP_ERR_WORKSPACE;
   int st = check_device();
   if (st != EMP_OK) return st;
@@ -1275,7 +1302,7 @@ static int energy_forces_impl(const Model& m, const emp_graph* g, const int32_t*
   float* e_atom = atom_energy ? atom_energy : at<float>(ws, L.e_atom);
   float* XT = at<float>(ws, L.XT);
   float* XTlo = at<float>(ws, L.XTlo);
-  float* Y = at<float>(ws, L.Y);
+  float* Y = L.keep_y ? nullptr : at<float>(ws, L.Y);
   float* GYhi = at<float>(ws, L.GYhi);
   float* GYlo = at<float>(ws, L.GYlo);
   float* GXT = at<float>(ws, L.GXT);
@@ -1342,7 +1369,8 @@ static int energy_forces_impl(const Model& m, const emp_graph* g, const int32_t*
         np.add(N, 1, nodeX, 4ll * C, 0, W0, 4 * C, S, 16ll * C, 0);
         np.launch(stream);
       } else {
-        st = layer_forward(m, g, t, xs + (size_t)t * feat, D, R, rr.inv, S, ws, L, stream);
+        st = layer_forward(m, g, t, xs + (size_t)t * feat, D, R, rr.inv, S, ws, L, stream,
+                           L.keep_y ? at<float>(ws, L.Ykeep) + (size_t)(t - 1) * E * 16 * C : nullptr);
         if (st != EMP_OK) return st;
       }
     }
@@ -1415,20 +1443,29 @@ static int energy_forces_impl(const Model& m, const emp_graph* g, const int32_t*
     } else if (E > 0) {
       // [per-edge product launches: begin]
       // Cohorts are taken two at a time: one backward prep and one grouped product launch (the
-      // recomputed forward blocks and the transposed blocks) over both, then the per-edge backward
-      // and the sender sums cohort by cohort, in order.
+      // transposed blocks, and the recomputed forward blocks unless y was kept) over both, then
+      // the per-edge backward and the sender sums cohort by cohort, in order.
+      const float* Ykept = L.keep_y ? at<float>(ws, L.Ykeep) + (size_t)(t - 1) * E * 16 * C : nullptr;
       int ci = 0;
       for (long long g0 = 0; g0 < E; g0 += 2 * coh) {
         const long long g1 = std::min(E, g0 + 2 * coh), M = g1 - g0;
-        {
+        if (Ykept && !wgrad) {
+          // g_y alone: the receivers' gS rows rotated into the edge frame
+          const int per = rs_per(M, tc::num_sms(), 6);
+          Scope sc_("bwd_prep", stream);
+          k_rotate_staged<false, RS_V_FWD><<<(unsigned)((M + per - 1) / per), C / RS_V_FWD, rs_smem_bytes(C, false), stream>>>(
+              g0, g1, C, per, nullptr, g->recv, nullptr, D, nullptr, gS, nullptr, GYhi, GYlo, nullptr, nullptr);
+        } else {
           const int per = rs_per(M, tc::num_sms(), 3);
           Scope sc_("bwd_prep", stream);
           k_rotate_staged<true, RS_V_BWD><<<(unsigned)((M + per - 1) / per), C / RS_V_BWD, rs_smem_bytes(C, true), stream>>>(
               g0, g1, C, per, g->recv, g->send, rr.inv, D, R, xt, gS, XT, XTlo, GYhi, GYlo);
         }
-        So2Part parts[2] = {{am_xt.get(M), &m.bmaps_fwd[t], Y}, {am_gy.get(M), &m.bmaps_bwd[t], GXT}};
-        st = so2_product(m, M, parts, 2, counter, stream);
+        const So2Part xt_part{am_xt.get(M), &m.bmaps_fwd[t], Y}, gy_part{am_gy.get(M), &m.bmaps_bwd[t], GXT};
+        So2Part parts[2] = {xt_part, gy_part};
+        st = Ykept ? so2_product(m, M, &gy_part, 1, counter, stream) : so2_product(m, M, parts, 2, counter, stream);
         if (st != EMP_OK) return st;
+        const float* Yg = Ykept ? Ykept + (size_t)g0 * 16 * C : Y;   // the pair's y rows
         if (wgrad) {   // dB_b += sum over the cohorts' edges of g_y (x) x~ per block (both as their hi + lo)
           st = so2_block_sums(C, M, GYhi, GYlo, XT, XTlo, dB, ws, L, counter, stream);
           if (st != EMP_OK) return st;
@@ -1446,7 +1483,7 @@ static int energy_forces_impl(const Model& m, const emp_graph* g, const int32_t*
           {
             Scope sc_("bwd_edge", stream);
             k_bwd_edge<BE_V><<<nb, C / BE_V, be_smem_bytes(C), stream>>>(e0, e1, C, per, g->send, rr.inv, g->vec, D, R,
-                                                               xt, Y + ro, gS, GXT + ro, g->recv, perm, gRhi, gRlo, g_r, Pg);
+                                                               xt, Yg + ro, gS, GXT + ro, g->recv, perm, gRhi, gRlo, g_r, Pg);
           }
           side.run([&](cudaStream_t q) {
             Scope sc_("gx_combine", q);
@@ -1529,8 +1566,8 @@ int mp_energy_forces(const void* model, const emp_graph* g, const int32_t* speci
 
 size_t mp_sharded_workspace_bytes(const void* model, int64_t n_edges_local, int64_t n_edges, int32_t n_atoms) {
   if (!model || n_edges_local < 0 || n_edges < n_edges_local || n_atoms < 1) return 0;
-  return ws_layout(*static_cast<const Model*>(model), n_edges_local, n_atoms).total + align_up((size_t)n_edges * 12 + 4) +
-         align_up((size_t)(n_atoms + 1) * 4);
+  return ws_layout(*static_cast<const Model*>(model), n_edges_local, n_atoms, false, true).total +
+         align_up((size_t)n_edges * 12 + 4) + align_up((size_t)(n_atoms + 1) * 4);
 }
 
 int mp_energy_forces_sharded(const void* model, const emp_graph* g, int32_t atom_begin, int32_t atom_end, int32_t rank,
@@ -1549,7 +1586,9 @@ int mp_energy_forces_sharded(const void* model, const emp_graph* g, int32_t atom
   EMP_CUDA_TRY(cudaStreamSynchronize(stream));
   const long long eb = off[0], El = (long long)off[1] - off[0];
   if (El < 0) return EMP_ERR_ARG;
-  const size_t need = mp_sharded_workspace_bytes(model, El, g->n_edges, N);
+  // the layout energy_forces_impl takes (y kept if the workspace holds it), then the extras
+  const size_t extra = align_up((size_t)g->n_edges * 12 + 4) + align_up((size_t)(N + 1) * 4);
+  const size_t need = call_layout(m, El, N, false, ws_bytes, extra).total + extra;
   if (ws_bytes < need) return EMP_ERR_WORKSPACE;
   const size_t ro_at = need - align_up((size_t)(N + 1) * 4);
   int* recv_off_local = reinterpret_cast<int*>(static_cast<char*>(ws) + ro_at);
@@ -1573,7 +1612,7 @@ int mp_energy_forces_sharded(const void* model, const emp_graph* g, int32_t atom
 
 size_t mp_weight_grad_workspace_bytes(const void* model, int64_t n_edges, int32_t n_atoms) {
   if (!model || n_edges < 0 || n_atoms < 1) return 0;
-  return ws_layout(*static_cast<const Model*>(model), n_edges, n_atoms, true).total;
+  return ws_layout(*static_cast<const Model*>(model), n_edges, n_atoms, true, true).total;
 }
 
 int mp_energy_weight_grad(const void* model, const emp_graph* g, const int32_t* species, double* energy, float* forces,

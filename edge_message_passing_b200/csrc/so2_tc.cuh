@@ -8,13 +8,15 @@
 // A launch is a group of sub-problems that share the row count M (one cohort):
 //   out_s[:, col_s : col_s + K_s] = A_{a(s)}[:, col_s : col_s + K_s] @ B_s^T,
 // B_s a (K_s x K_s) matrix stored [n][k] (K-major).  The forward of a layer is
-// the 4 m-blocks of the cohort; the backward groups the 4 recomputed forward
-// blocks with the 4 transposed blocks (8 sub-problems, two A operands).
+// the 4 m-blocks of the cohort, the backward the 4 transposed blocks; when the
+// backward recomputes y (smallest workspace) it groups the 4 forward blocks with
+// the 4 transposed blocks (8 sub-problems, two A operands).
 //
 // Persistent kernel on CTA pairs (clusters of 2, cta_group::2): each pair computes
 // 256 x 256 output tiles taken from a shared atomic counter (tiles ordered by
-// decreasing K).  In each CTA warp 0 issues TMA loads (64-byte swizzle, 16 fp32 of
-// K per row) of its 128 A rows and its half of the B rows into a 6-stage ring; the
+// decreasing K).  In each CTA warp 0 issues TMA loads (128-byte swizzle, 32 fp32 of
+// K per row) of its 128 A rows and its half of the B rows, hi and lo, into a 3-stage
+// ring of 64 KB stages; the
 // even CTA's warp 1 issues tcgen05.mma (one thread) into one of two TMEM
 // accumulators (2 x 256 columns) in both CTAs; warps 2..5 of each CTA drain its
 // other accumulator with tcgen05.ld and store FP32 rows, so the epilogue of a tile

@@ -181,11 +181,17 @@ int mp_model_radial_tables(void* model, double tol, int32_t* n_pieces);
 int mp_radial_hidden(const void* model, int32_t layer, int32_t pair, int64_t n, const float* d, float* h2_hi,
                      float* h2_lo, const float* g_h2, float* dE_dd, void* ws, size_t ws_bytes, cudaStream_t stream);
 
-/* Workspace bytes mp_forward / mp_energy_forces need.  The size depends on the model's radial
- * mode: with radial tables (mp_model_radial_tables) the per-row hidden values take 768 bytes per
- * edge more, so query it after the tables are built (a workspace sized before them is rejected
- * with EMP_ERR_WORKSPACE). */
+/* Workspace bytes for mp_energy_forces at full speed: the layers between the first and the last
+ * keep their per-edge mixing outputs y (n_edges x 16C floats each) from the forward for the
+ * backward.  mp_workspace_bytes_min is the least mp_forward and mp_energy_forces accept: there
+ * the backward recomputes y cohort by cohort (one more SO(2) product per edge and layer).
+ * Any size from the minimum up runs; the path is chosen by the size passed, and both give the
+ * same bits.  The sizes depend on the model's radial mode: with radial tables
+ * (mp_model_radial_tables) the per-row hidden values take 768 bytes per edge more, so query
+ * them after the tables are built (a workspace sized before them may be rejected with
+ * EMP_ERR_WORKSPACE). */
 size_t mp_workspace_bytes(const void* model, int64_t n_edges, int32_t n_atoms);
+size_t mp_workspace_bytes_min(const void* model, int64_t n_edges, int32_t n_atoms);
 
 /* One interaction layer (forward only): agg_out[i] = (1/avg_degree) * sum over
  * edges e with recv(e) = i of D(R_e)^T SO2_layer(R_e(d) (.) D(R_e) x_in[send(e)]).
@@ -213,7 +219,9 @@ typedef int (*emp_allreduce_fn)(float* buf, size_t n, cudaStream_t stream, void*
  * residual part counted on rank 0 only), and at the end the per-edge gradients, so that
  * every rank returns the whole energy, forces, virial and atom energies.  The ranges must
  * cover the atoms, each once, over the ranks; any split is valid (balanced by edge count
- * for speed).  Workspace: mp_sharded_workspace_bytes(model, local edges, all edges, N).
+ * for speed).  Workspace: mp_sharded_workspace_bytes(model, local edges, all edges, N) (y kept,
+ * as for mp_workspace_bytes; down to (layers - 2) x local edges x 16C x 4 bytes less runs with y
+ * recomputed).
  * Reads the range's edge offsets back to the host (synchronises once).  Not for CUDA-graph
  * capture unless allreduce is capturable. */
 size_t mp_sharded_workspace_bytes(const void* model, int64_t n_edges_local, int64_t n_edges, int32_t n_atoms);
@@ -229,7 +237,8 @@ int mp_energy_forces_sharded(const void* model, const emp_graph* g, int32_t atom
  * result is reproducible.  The radial hidden layers are the network's even when the model
  * has radial tables (their weights get gradients).  Gradients of force terms (mixed second
  * derivatives) are not computed.  Workspace: mp_weight_grad_workspace_bytes (larger than
- * mp_workspace_bytes: per-row radial values, block sums and reduction partials). */
+ * mp_workspace_bytes: per-row radial values, block sums and reduction partials; like it, with y
+ * kept, and down to (layers - 2) x edges x 16C x 4 bytes less with y recomputed). */
 size_t mp_weight_grad_workspace_bytes(const void* model, int64_t n_edges, int32_t n_atoms);
 int mp_energy_weight_grad(const void* model, const emp_graph* g, const int32_t* species, double* energy,
                           float* forces, float* grad, void* ws, size_t ws_bytes, cudaStream_t stream);

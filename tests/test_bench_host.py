@@ -11,7 +11,7 @@ def test_alg_bytes_follow_the_rows_each_kernel_moves():
     row, d, d0 = 16 * C * 4, 84 * 4, 16 * 4
     # the per-edge cohort kernels run only in the layers between the first and the last
     assert bench.alg_bytes_step("rotate_in", C, T, E, N) == E * (4 * C * 4 + 2 * row + d)      # R in; x~ hi/lo out
-    assert bench.alg_bytes_step("bwd_prep", C, T, E, N) == E * (4 * C * 4 + 4 * row + d)       # + g_y hi/lo out
+    assert bench.alg_bytes_step("bwd_prep", C, T, E, N) == E * (2 * row + d)                   # D in; g_y hi/lo out
     assert bench.alg_bytes_step("bwd_edge", C, T, E, N) == E * (2 * row + 4 * C * 4 + d + 8 * C * 4)
     assert bench.alg_bytes_step("rotate_back_scatter", C, T, E, N) == E * (row + d)
     for k in ("rotate_in", "bwd_prep", "bwd_edge", "rotate_back_scatter"):

@@ -50,7 +50,7 @@ def test_workspace_too_small_is_rejected():
     w, g, model = _small_model()
     L = emp.lib()
     gc = g.c()
-    need = model.workspace_bytes(g.n_edges, g.n_atoms)
+    need = model.workspace_bytes_min(g.n_edges, g.n_atoms)     # the least any call runs in
     ws = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
     N, C = g.n_atoms, w.spec.C
     sp = torch.from_numpy(w.structure.species).cuda()

@@ -224,6 +224,24 @@ def test_energy_forces_n64():
     _check_ef(synth.workload("n64_diamond"))
 
 
+@pytest.mark.parametrize("n_layers", [3, 4])
+def test_kept_and_recomputed_mixing_outputs_agree_bit_for_bit(n_layers):
+    """In the workspace of mp_workspace_bytes the per-edge layers keep their mixing outputs y
+    from the forward; in that of mp_workspace_bytes_min the backward recomputes them: the same
+    products, so the same bits (128-edge cohorts: many cohort pairs and a ragged tail)."""
+    w = synth.small_workload(ncell=1, C=32, n_layers=n_layers, gated=True, sigma=0.1)
+    spec = synth.ModelSpec(**{**w.spec.__dict__, "cohort_edges": 128})
+    g = _graph(w.structure, spec.cutoff)
+    sp = _cuda(w.structure.species)
+    model = emp.Model(spec, w.weights)
+    assert model.workspace_bytes_min(g.n_edges, g.n_atoms) < model.workspace_bytes(g.n_edges, g.n_atoms)
+    a = [t.clone() for t in emp.mp_energy_forces(model, g, sp, virial=True, atom_energy=True)]
+    b = emp.mp_energy_forces(model, g, sp, virial=True, atom_energy=True, compact=True)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+    assert emp.last_device_error() == 0
+
+
 def test_results_are_deterministic_and_inputs_untouched():
     w = synth.small_workload(ncell=1, C=32, n_layers=2, gated=True, sigma=0.1)
     st = w.structure
@@ -342,6 +360,8 @@ def test_graph_replay_matches_eager_n4096():
     model = emp.Model(w.spec, w.weights)
     e, f, _, _ = emp.mp_energy_forces(model, g, sp)
     e, f = e.clone(), f.clone()
+    ec, fc, _, _ = emp.mp_energy_forces(model, g, sp, compact=True)    # y recomputed in the backward
+    assert torch.equal(e, ec) and torch.equal(f, fc)
     efg = emp.EnergyForcesGraph(model, g, sp)
     assert efg.launches > 0
     for _ in range(2):
