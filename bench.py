@@ -374,8 +374,17 @@ def other_configs(emp, torch, stream, flush, hbm_gbs: float, steps: int = 10):
         "note": "opt-in certified Chebyshev tables (degree 10, tol 1e-7) for the radial hidden layers; an "
                 "approximation, not the headline"}
     del efg
-    # the weight gradient of the energy (the training path), eager, on the same frame
     model.radial_tables(0.0)
+    # the same frame in the smallest workspace: the backward recomputes y cohort by cohort and no
+    # [E, 16C] tensor is kept (the same bits as the headline step)
+    efg = emp.EnergyForcesGraph(model, g, sp, compact=True)
+    ms_c = timed(efg.replay)
+    out[WORKLOAD + "_recompute_y"] = {
+        "n_atoms": st.pos.shape[0], "n_edges": g.n_edges, "ms_per_step": round(ms_c, 4),
+        "edges_per_s": g.n_edges / (ms_c * 1e-3), "workspace_bytes": int(efg.ws.numel()),
+        "timed": "CUDA-graph replay"}
+    del efg
+    # the weight gradient of the energy (the training path), eager, on the same frame
     for _ in range(2):
         emp.mp_energy_weight_grad(model, g, sp)
     torch.cuda.synchronize()
@@ -618,7 +627,10 @@ def run_ours(args):
                              "parallelism": "replicas" if ws > 1 else "single",
                              "l2": "flushed between timed steps (256 MB write outside the timed events)",
                              "step": "mp_energy_forces on a resident neighbour graph, replayed as one CUDA graph "
-                                     "of the library's launches; neighbour list timed separately (nl_ms)"},
+                                     "of the library's launches; neighbour list timed separately (nl_ms)",
+                             "workspace_bytes": int(efg.ws.numel()),
+                             "backward": "y of the middle layer kept from the forward (mp_workspace_bytes); the "
+                                         "recomputing form is timed in configs." + WORKLOAD + "_recompute_y"},
                   "nl_ms": sum(nl_times) / len(nl_times),
                   "p50_ms": statistics.median(lat), "p90_ms": float(np.percentile(lat, 90)), "latency_reps": len(lat),
                   "clocks": clk.summary(), "gpu_launches": launches,

@@ -481,9 +481,11 @@ class EnergyForcesGraph:
     pointers captured here: the outputs (energy, forces, virial, atom_energy) are
     this object's tensors, overwritten by every replay, and graph, species and the
     workspace are kept alive by the object.  The positions must not change between
-    replays without a new capture (the graph's edge vectors are inputs)."""
+    replays without a new capture (the graph's edge vectors are inputs).  compact: the smallest
+    workspace (the backward recomputes the per-edge mixing outputs; the same bits)."""
 
-    def __init__(self, model: Model, graph: Graph, species, virial: bool = False, atom_energy: bool = False):
+    def __init__(self, model: Model, graph: Graph, species, virial: bool = False, atom_energy: bool = False,
+                 compact: bool = False):
         torch = _torch()
         N = graph.n_atoms
         self.model, self.graph, self.species = model, graph, species
@@ -491,7 +493,8 @@ class EnergyForcesGraph:
         self.forces = torch.empty((N, 3), dtype=torch.float32, device="cuda")
         self.virial = torch.empty((3, 3), dtype=torch.float32, device="cuda") if virial else None
         self.atom_energy = torch.empty(N, dtype=torch.float32, device="cuda") if atom_energy else None
-        self.ws = torch.empty(max(model.workspace_bytes(graph.n_edges, N), 256), dtype=torch.uint8, device="cuda")
+        nbytes = (model.workspace_bytes_min if compact else model.workspace_bytes)(graph.n_edges, N)
+        self.ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device="cuda")
         self._gc = graph.c()
         side = torch.cuda.Stream()
         side.wait_stream(torch.cuda.current_stream())
