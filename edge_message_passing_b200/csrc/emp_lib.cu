@@ -101,7 +101,7 @@ WsLayout ws_layout(const Model& m, long long E, int N, bool grad = false, bool k
   // radial scales kept for the backward: the first layer's degree-0 columns (rows of C), then
   // rows of 4C for every later layer (a single layer of mp_forward takes rows of 4C at the start)
   L.R = take(std::max((size_t)E * C + (T - 1) * (size_t)E * 4 * C, (size_t)E * 4 * C) * 4);
-  L.rbP = take(((coh + RB_CHUNK - 1) / RB_CHUNK) * 2 * 16 * C * 4);
+  L.rbP = take(((2 * coh + RB_CHUNK - 1) / RB_CHUNK) * 2 * 16 * C * 4);   // chunk partials of two cohorts
   L.gRhi = take((size_t)E * 4 * C * 4);
   L.gRlo = take((size_t)E * 4 * C * 4);
   if (grad || m.tab_on) {   // per-row radial hidden values: only the tables' path and the weight gradients
@@ -470,11 +470,14 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
     So2Part parts[2] = {{am[0].get(M), &m.bmaps_fwd[t], Y[0]}, {am[1].get(M), &m.bmaps_fwd[t], Y[1]}};
     const int st = so2_product(m, M, parts, nc, counter, s);
     if (st != EMP_OK) return st;
-    for (int b = 0; b < nc; ++b) {
-      const long long c0 = ee[b], c1 = ee[b + 1];
+    {
+      // the receiver sums of the group's cohorts in one launch: their y rows are contiguous (a
+      // pair is two full cohorts), and chunk partials fold in chunk order across the cohort
+      // boundary as they would cohort by cohort
+      const long long c0 = ee[0], c1 = ee[nc];
       const int nchunks = (int)((c1 - c0 + RB_CHUNK - 1) / RB_CHUNK);
-      side.wait();        // the previous cohort's combine: S of its last receiver, and P
-      { Scope sc_("rotate_back_scatter", s); k_rb_chunks<RB_V><<<nchunks, C / RB_V, 0, s>>>(c0, c1, C, g->recv, g->recv_off, D, Y[b], S, P); }
+      side.wait();        // the previous group's combine: S of its last receiver, and P
+      { Scope sc_("rotate_back_scatter", s); k_rb_chunks<RB_V><<<nchunks, C / RB_V, 0, s>>>(c0, c1, C, g->recv, g->recv_off, D, Y[0], S, P); }
       side.run([&](cudaStream_t q) {
         Scope sc_("rb_combine", q);
         k_rb_combine<<<dim3((unsigned)std::min<long long>(c1 - c0, 128), 16), C, 0, q>>>(c0, c1, C, g->recv, g->recv_off, P, S);
