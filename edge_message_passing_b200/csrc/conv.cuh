@@ -516,23 +516,12 @@ __global__ void __launch_bounds__(128) k_rb_chunks(long long e0, long long e1, i
     T acc[16];
 #pragma unroll
     for (int k = 0; k < 16; ++k) acc[k] = vset<T>(0.f);
-    // each edge's y row is loaded one edge ahead, so that two rows' loads are in flight
-    T yn[16];
-    {
-      const T* y = Yv + (size_t)c0 * 16 * CV + t;
-#pragma unroll
-      for (int q = 0; q < 16; ++q) yn[q] = y[col_of_k(q) * CV];
-    }
 #pragma unroll 1
     for (int k = 0; k < nch; ++k) {
+      const T* y = Yv + (size_t)(c0 + k) * 16 * CV + t;
       T yv[16];
 #pragma unroll
-      for (int q = 0; q < 16; ++q) yv[q] = yn[q];
-      if (k + 1 < nch) {
-        const T* y = Yv + (size_t)(c0 + k + 1) * 16 * CV + t;
-#pragma unroll
-        for (int q = 0; q < 16; ++q) yn[q] = y[col_of_k(q) * CV];
-      }
+      for (int q = 0; q < 16; ++q) yv[q] = y[col_of_k(q) * CV];
       if (srv[k] != cur) {
         rb_flush(cur, c0, c1, e0, e1, chunk, first, recv_off, CV, t, acc, Sv, Pv);
 #pragma unroll

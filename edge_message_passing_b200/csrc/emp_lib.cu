@@ -450,9 +450,9 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
     if (st0 != EMP_OK) return st0;
   }
   int* counter = at<int>(ws, L.counter);
-  // Full cohorts are taken two at a time (a shorter last cohort alone): both are rotated in,
-  // then one grouped launch computes both cohorts' products (twice the tiles, so the CTA
-  // pairs stay evenly loaded), then the receiver sums run cohort by cohort, in order.
+  // Full cohorts are taken two at a time (a shorter last cohort alone): both are rotated in
+  // by one launch, one grouped launch computes both cohorts' products (twice the tiles, so the
+  // CTA pairs stay evenly loaded), and one launch takes the receiver sums of both.
   for (long long e0 = 0; e0 < E;) {
     const long long e1 = std::min(E, e0 + coh);
     const bool two = e1 < E && std::min(E, e1 + coh) - e1 == e1 - e0;
@@ -461,11 +461,14 @@ int layer_forward(const Model& m, const emp_graph* g, int t, const float* x, con
     const long long M = e1 - e0;
     if (Ykeep)
       for (int b = 0; b < nc; ++b) Y[b] = Ykeep + (size_t)ee[b] * 16 * C;
-    for (int b = 0; b < nc; ++b) {
-      const int per = rs_per(M, tc::num_sms(), 6);
+    {
+      // rotate-in of the group's cohorts in one launch: the second cohort's x~ rows follow the
+      // first's (a pair is two full cohorts, and its buffers are contiguous)
+      const long long Mt = ee[nc] - ee[0];
+      const int per = rs_per(Mt, tc::num_sms(), 6);
       Scope sc_("rotate_in", s);
-      k_rotate_staged<false, RS_V_FWD><<<(unsigned)((M + per - 1) / per), C / RS_V_FWD, rs_smem_bytes(C, false), s>>>(
-          ee[b], ee[b + 1], C, per, g->recv, g->send, rrow, D, R, x, nullptr, XT[b], XTlo[b], nullptr, nullptr);
+      k_rotate_staged<false, RS_V_FWD><<<(unsigned)((Mt + per - 1) / per), C / RS_V_FWD, rs_smem_bytes(C, false), s>>>(
+          ee[0], ee[nc], C, per, g->recv, g->send, rrow, D, R, x, nullptr, XT[0], XTlo[0], nullptr, nullptr);
     }
     So2Part parts[2] = {{am[0].get(M), &m.bmaps_fwd[t], Y[0]}, {am[1].get(M), &m.bmaps_fwd[t], Y[1]}};
     const int st = so2_product(m, M, parts, nc, counter, s);
