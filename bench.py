@@ -273,7 +273,7 @@ def hbm_fractions(fam, steps: int, E: int, N: int, C: int, T: int, hbm_gbs: floa
 # at half).  Valid only for the kernel source and the launch structure it was taken on: so2_tc.cuh
 # and the marked per-edge product launch code of emp_lib.cu must hash to source_sha1, else the
 # roofline's traffic is null.
-SO2_TRAFFIC = {"source_sha1": "eada48ee78f825d300341851164605c88ce9adbd", "bytes_per_launch": 377.6e6}
+SO2_TRAFFIC = {"source_sha1": "ddac4e4305648c3a9083e13e1778cad9ba2252c5", "bytes_per_launch": 379.0e6}
 
 
 def so2_source_hash():
