@@ -59,4 +59,7 @@ def test_null_arguments_are_rejected_on_the_host():
     assert L.mp_radial_chain(None, 0, None, None, None, None, None, None, None) == -1
     assert L.mp_so2_mix(None, 0, 0, 0, None, None, None, 0, None) == -1
     assert L.mp_workspace_bytes(None, 10, 10) == 0
+    assert L.mp_workspace_bytes_min(None, 10, 10) == 0
+    assert L.mp_sharded_workspace_bytes(None, 10, 10, 10) == 0
+    assert L.mp_weight_grad_workspace_bytes(None, 10, 10) == 0
     assert L.nl_workspace_bytes(100) > 0
