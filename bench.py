@@ -249,6 +249,14 @@ def alg_bytes_step(name: str, C: int, T: int, E: int, N: int) -> float:
     raise KeyError(name)
 
 
+def mixing_flops_step(C: int, T: int, E: int) -> float:
+    """Useful FP32 flops of the per-edge SO(2) mixings in one energy + force step: they run in the
+    T - 2 layers between the first and the last (the end layers mix once per node); each mixes
+    every edge twice, forward and backward transpose (the backward reads y kept from the forward),
+    2 * 72 * C^2 flops each (the four m-blocks: 16 + 36 + 16 + 4 = 72 C^2 multiply-adds)."""
+    return float(E) * 2 * C * C * 2 * 72 * max(T - 2, 0)
+
+
 HBM_FAMILIES = ("rotate_in", "bwd_prep", "bwd_edge", "rotate_back_scatter", "first_fwd", "first_bwd", "last_fwd",
                 "last_bwd", "radial_fwd", "radial_h2", "radial_head", "radial_head_bwd", "radial_bwd")
 
@@ -585,10 +593,7 @@ def run_ours(args):
     tf32_rate_first = rates[0]
     if so2_launches:
         so2_ms = fam["so2_tc"][0] / so2_launches
-        # per step: the per-edge products run in the layers between the first and the last (the end
-        # layers mix once per node, end_layers.cuh); each mixes every edge twice (forward, backward
-        # transpose: the backward reads y kept from the forward), 2*72*C^2 useful flops each
-        flops_step = E * 2 * C * C * 2 * 72 * max(T - 2, 0)
+        flops_step = mixing_flops_step(C, T, E)
         achieved = flops_step * len(ptimes) / (fam["so2_tc"][0] * 1e-3) / 1e12
         # the reference: the measured TF32 rate of the same tcgen05 products (operands resident in
         # shared memory, ~0.5 s back to back right after the step) / 3 for 3xTF32

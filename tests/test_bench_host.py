@@ -61,3 +61,13 @@ def test_traffic_hash_covers_the_kernel_and_the_marked_launch_code():
     text = open(os.path.join(csrc, "emp_lib.cu")).read()
     assert text.count("// [per-edge product launches: begin]") == 2
     assert text.count("// [per-edge product launches: end]") == 2
+
+
+def test_mixing_flops_count_two_mixings_per_middle_layer():
+    # 72 C^2 multiply-adds per edge and mixing (m-blocks of widths 4, 6, 4, 2 channel blocks:
+    # 16 + 36 + 16 + 4), forward and backward transpose, middle layers only
+    assert sum(w * w for w in (4, 6, 4, 2)) == 72
+    C, E = 128, 1000
+    assert bench.mixing_flops_step(C, 3, E) == E * 2 * 72 * C * C * 2
+    assert bench.mixing_flops_step(C, 2, E) == 0
+    assert bench.mixing_flops_step(C, 5, E) == 3 * bench.mixing_flops_step(C, 3, E)
